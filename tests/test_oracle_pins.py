@@ -1,0 +1,424 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself:
+brute force on tiny inputs, closed forms, invariants of softmax attention and of
+the rotary embedding, a library routine on a special case, and the prompt-length
+worked values of the pages.  CPU only.
+
+Pages cited: "ARK-ASR-3B -- INT8 ONNX" model card (sections Shapes, Inference),
+SGLang-Omni cookbook "ARK-ASR-3B" (introduction, Audio Handling, dtype).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gqa_attention_static_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16_bits(x: torch.Tensor) -> np.ndarray:
+    return x.to(torch.bfloat16).contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def rand_bits(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return bf16_bits(torch.randn(shape, generator=g) * scale)
+
+
+# ------------------------------------------------------------------ bf16 ----
+
+def _all_bf16_finite_sorted():
+    pats = np.arange(0, 0x10000, dtype=np.uint32).astype(np.uint16)
+    vals = oracle.bf16_array_to_f64(pats)
+    fin = np.isfinite(vals)
+    pats, vals = pats[fin], vals[fin]
+    # one entry per value (+0/-0 collapse); keep +0
+    order = np.lexsort((pats, vals))
+    vals, pats = vals[order], pats[order]
+    keep = np.concatenate([[True], vals[1:] != vals[:-1]])
+    return vals[keep], pats[keep]
+
+
+def brute_nearest_bf16(x: float, vals, pats) -> int:
+    """Nearest bf16 by exhaustive search over all finite bf16 values; ties go
+    to the one with an even last mantissa bit."""
+    i = np.searchsorted(vals, x)
+    cands = [k for k in (i - 1, i) if 0 <= k < len(vals)]
+    best = min(cands, key=lambda k: (abs(vals[k] - x), int(pats[k]) & 1))
+    return int(pats[best])
+
+
+def test_bf16_widening_known_patterns(oracle_lib):
+    assert oracle.bf16_to_f64(np.array([0x3F80], np.uint16))[0] == 1.0
+    assert oracle.bf16_to_f64(np.array([0xC000], np.uint16))[0] == -2.0
+    assert oracle.bf16_to_f64(np.array([0x0001], np.uint16))[0] == 2.0 ** -133
+    assert oracle.bf16_to_f64(np.array([0x7F7F], np.uint16))[0] == (2 - 2 ** -7) * 2.0 ** 127
+    assert math.isinf(oracle.bf16_to_f64(np.array([0x7F80], np.uint16))[0])
+
+
+def test_bf16_rounding_matches_exhaustive_search(oracle_lib):
+    vals, pats = _all_bf16_finite_sorted()
+    rng = np.random.default_rng(0)
+    xs = list(rng.standard_normal(3000) * np.exp(rng.uniform(-20, 20, 3000)))
+    # exact midpoints between neighbours (the tie cases), and near-boundaries
+    for k in rng.integers(1, len(vals) - 2, 500):
+        mid = (vals[k] + vals[k + 1]) / 2.0
+        xs += [mid, np.nextafter(mid, np.inf), np.nextafter(mid, -np.inf)]
+    xs += [2.0 ** -133, 2.0 ** -134, 3 * 2.0 ** -135, 2.0 ** -126 * 1.00390625, 1e-300,
+           (2 - 2 ** -7) * 2.0 ** 127, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -1.0 - 2 ** -8]
+    got = oracle.f64_to_bf16(np.array(xs))
+    for x, g in zip(xs, got):
+        want = brute_nearest_bf16(float(x), vals, pats)
+        # signed zero: brute force returns +0 for tiny negatives; compare values
+        if oracle.bf16_array_to_f64(np.array([want], np.uint16))[0] == 0.0:
+            assert oracle.bf16_array_to_f64(np.array([g], np.uint16))[0] == 0.0
+        else:
+            assert int(g) == want, (x, hex(int(g)), hex(want))
+
+
+def test_bf16_overflow_and_specials(oracle_lib):
+    top = (2 - 2 ** -7) * 2.0 ** 127
+    half_ulp = 2.0 ** (127 - 8)
+    assert int(oracle.f64_to_bf16(np.array([top + half_ulp]))[0]) == 0x7F80  # tie rounds up to inf
+    assert int(oracle.f64_to_bf16(np.array([top + half_ulp * 0.99]))[0]) == 0x7F7F
+    assert int(oracle.f64_to_bf16(np.array([-np.inf]))[0]) == 0xFF80
+    assert int(oracle.f64_to_bf16(np.array([np.nan]))[0]) & 0x7F80 == 0x7F80
+
+
+# ------------------------------------------------------------------ RoPE ----
+
+def test_rope_rotation_preserves_norm(oracle_lib):
+    """A rotation of each (i, i+64) pair preserves the row norm exactly in
+    real arithmetic: a wrong sign or a wrong partner breaks it."""
+    rng = np.random.default_rng(1)
+    for _ in range(20):
+        x = rng.standard_normal(128)
+        ang = rng.uniform(-50, 50, 64)
+        y = oracle.rope_rotate(x, np.cos(ang), np.sin(ang))
+        assert abs(np.linalg.norm(y) - np.linalg.norm(x)) < 1e-12 * np.linalg.norm(x)
+
+
+def test_rope_pairs_rotate_as_complex_numbers(oracle_lib):
+    """Rotate-half RoPE read as complex multiplication:
+    (x_i + i x_{i+64}) * (c_i + i s_i) = y_i + i y_{i+64}."""
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal(128)
+    ang = rng.uniform(-5, 5, 64)
+    y = oracle.rope_rotate(x, np.cos(ang), np.sin(ang))
+    for i in range(64):
+        z = complex(x[i], x[i + 64]) * complex(math.cos(ang[i]), math.sin(ang[i]))
+        assert abs(z.real - y[i]) < 1e-13 and abs(z.imag - y[i + 64]) < 1e-13
+
+
+def test_rope_table_frequencies_closed_form(oracle_lib):
+    """With theta = 1e6 and head dim 128 the pair frequencies form a geometric
+    sequence from 1 (pair 0) to 1e6^-0.5 = 1e-3 (pair 32).  Read the angles back
+    from the fp32 table at position 1 and check them against that closed form."""
+    c, s = oracle.rope_table(4, 128, 1e6)
+    ang = np.arctan2(s[1].astype(np.float64), c[1].astype(np.float64))
+    expect = np.array([1e-3 ** (i / 32.0) for i in range(64)])
+    assert abs(ang[0] - 1.0) < 1e-6
+    assert abs(ang[32] - 1e-3) < 1e-9
+    np.testing.assert_allclose(ang, expect, rtol=2e-6, atol=1e-12)
+    # position 0 is the identity: cos = 1, sin = 0 exactly
+    assert np.all(c[0] == 1.0) and np.all(s[0] == 0.0)
+    # fp32 rounding of the true cos/sin (one rounding, so within half an fp32 ulp)
+    p = 3
+    true_c = np.cos(p * expect)
+    assert np.all(np.abs(c[p] - true_c) <= np.spacing(np.abs(c[p]).astype(np.float32)).astype(np.float64))
+
+
+def test_rope_relative_position(oracle_lib):
+    """<R_p q, R_r k> depends only on p - r (fp32 table, so to 1e-5)."""
+    T = 300
+    c, s = oracle.rope_table(T, 128, 1e6)
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal(128)
+    k = rng.standard_normal(128)
+
+    def rot(x, p):
+        return oracle.rope_rotate(x, c[p].astype(np.float64), s[p].astype(np.float64))
+
+    for p, r, dlt in [(10, 3, 100), (0, 0, 250), (57, 200, 41), (5, 9, 7)]:
+        a = float(np.dot(rot(q, p), rot(k, r)))
+        b = float(np.dot(rot(q, p + dlt), rot(k, r + dlt)))
+        assert abs(a - b) < 1e-4 * np.linalg.norm(q) * np.linalg.norm(k), (p, r, dlt, a, b)
+
+
+def test_append_rope_position0_identity_and_bit_copies(oracle_lib):
+    """At position 0 the rotation is the identity (bit-exact after rounding);
+    V rows are copied bit for bit; rows outside [pos0, pos0+n_new) keep their
+    bits; padded rows t >= n_new are not written."""
+    B, S, T = 2, 3, 8
+    q = rand_bits((B, S, 16, 128), 10)
+    kn = rand_bits((B, S, 2, 128), 11)
+    vn = rand_bits((B, S, 2, 128), 12)
+    ck = rand_bits((B, T, 2, 128), 13)
+    cv = rand_bits((B, T, 2, 128), 14)
+    pos0 = np.array([0, 4], np.int32)
+    n_new = np.array([3, 2], np.int32)
+    q2, ck2, cv2, skipped = oracle.append_rope(q, kn, vn, ck, cv, pos0, n_new)
+    assert skipped == 0
+    assert np.array_equal(q2[0, 0], q[0, 0]) and np.array_equal(ck2[0, 0], kn[0, 0])
+    for b in range(B):
+        for t in range(n_new[b]):
+            assert np.array_equal(cv2[b, pos0[b] + t], vn[b, t])
+        written = set(range(pos0[b], pos0[b] + n_new[b]))
+        for j in range(T):
+            if j not in written:
+                assert np.array_equal(ck2[b, j], ck[b, j]) and np.array_equal(cv2[b, j], cv[b, j])
+    assert np.array_equal(q2[1, 2], q[1, 2])  # t = 2 >= n_new[1]: untouched
+
+
+def test_append_rope_unit_vector_gives_table_entries(oracle_lib):
+    """x = e_i (1 at pair index i) rotates to (cos, sin) of that pair's angle:
+    out[i] = bf16(c_i), out[i+64] = bf16(s_i) -- the sign convention of the
+    rotation (positive angle turns x_i towards x_{i+64})."""
+    T = 100
+    c, s = oracle.rope_table(T, 128, 1e6)
+    for p, i in [(1, 0), (37, 5), (99, 63), (50, 32)]:
+        q = np.zeros((1, 1, 16, 128), np.uint16)
+        q[0, 0, 0, i] = 0x3F80  # 1.0
+        kn = np.zeros((1, 1, 2, 128), np.uint16)
+        vn = np.zeros((1, 1, 2, 128), np.uint16)
+        ck = np.zeros((1, T, 2, 128), np.uint16)
+        q2, _, _, _ = oracle.append_rope(q, kn, vn, ck, ck.copy(), np.array([p], np.int32),
+                                         np.array([1], np.int32))
+        got_c = oracle.bf16_array_to_f64(q2[0, 0, 0, i:i + 1])[0]
+        got_s = oracle.bf16_array_to_f64(q2[0, 0, 0, i + 64:i + 65])[0]
+        assert got_c == float(torch.tensor(float(c[p, i])).to(torch.bfloat16))
+        assert got_s == float(torch.tensor(float(s[p, i])).to(torch.bfloat16))
+
+
+def test_append_rope_skips_rows_past_T(oracle_lib):
+    q = rand_bits((1, 3, 16, 128), 20)
+    kn = rand_bits((1, 3, 2, 128), 21)
+    ck = rand_bits((1, 8, 2, 128), 22)
+    q2, ck2, _, skipped = oracle.append_rope(q, kn, kn, ck, ck, np.array([6], np.int32),
+                                             np.array([3], np.int32))
+    assert skipped == 1
+    assert np.array_equal(q2[0, 2], q[0, 2])
+
+
+# ------------------------------------------------------------- attention ----
+
+def brute_attention_py(q, k, v, vis, scale):
+    """Independent pure-Python softmax attention (lists, math.exp with the
+    largest score subtracted), one query row over rows j < vis."""
+    qf = [float(x) for x in q]
+    scores = []
+    for j in range(vis):
+        scores.append(scale * sum(a * float(b) for a, b in zip(qf, k[j])))
+    mx = max(scores)
+    ws = [math.exp(x - mx) for x in scores]
+    tot = math.fsum(ws)
+    out = [math.fsum(w * float(v[j][d]) for j, w in enumerate(ws)) / tot for d in range(len(qf))]
+    return out, mx + math.log(tot)
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,T", [(4, 2, 4, 8), (2, 1, 8, 5), (8, 2, 4, 7)])
+def test_attention_brute_force_tiny(oracle_lib, Hq, Hkv, D, T):
+    B, S = 2, 3
+    q = rand_bits((B, S, Hq, D), 30)
+    ck = rand_bits((B, T, Hkv, D), 31)
+    cv = rand_bits((B, T, Hkv, D), 32)
+    first_vis = np.array([2, T - S + 1], np.int32)
+    n_rows = np.array([S, S], np.int32)
+    scale = 1.0 / math.sqrt(D)
+    o, lse = oracle.attention(q, ck, cv, first_vis, n_rows, scale)
+    qf = oracle.bf16_array_to_f64(q)
+    kf = oracle.bf16_array_to_f64(ck)
+    vf = oracle.bf16_array_to_f64(cv)
+    G = Hq // Hkv
+    for b in range(B):
+        for t in range(S):
+            for h in range(Hq):
+                g = h // G
+                vis = first_vis[b] + t
+                ref_o, ref_l = brute_attention_py(qf[b, t, h], kf[b, :, g], vf[b, :, g], vis, scale)
+                np.testing.assert_allclose(o[b, t, h], ref_o, rtol=0, atol=1e-12)
+                assert abs(lse[b, h, t] - ref_l) < 1e-12
+
+
+def test_attention_matches_torch_sdpa_fp64(oracle_lib):
+    """Cross-check against torch's SDPA in float64 on CPU, with each KV head
+    repeated for its 8 query heads and an explicit causal/length mask."""
+    B, S, T, Hq, Hkv, D = 2, 5, 40, 16, 2, 128
+    q = rand_bits((B, S, Hq, D), 40)
+    ck = rand_bits((B, T, Hkv, D), 41)
+    cv = rand_bits((B, T, Hkv, D), 42)
+    pos0 = np.array([7, 30], np.int32)
+    n_new = np.array([5, 3], np.int32)
+    scale = 1.0 / math.sqrt(D)
+    o, lse = oracle.prefill(q, ck, cv, pos0, n_new, scale)
+    qt = torch.from_numpy(oracle.bf16_array_to_f64(q)).permute(0, 2, 1, 3)        # B,Hq,S,D
+    kt = torch.from_numpy(oracle.bf16_array_to_f64(ck)).permute(0, 2, 1, 3)       # B,Hkv,T,D
+    vt = torch.from_numpy(oracle.bf16_array_to_f64(cv)).permute(0, 2, 1, 3)
+    kt = kt.repeat_interleave(Hq // Hkv, dim=1)
+    vt = vt.repeat_interleave(Hq // Hkv, dim=1)
+    j = torch.arange(T).view(1, 1, 1, T)
+    t = torch.arange(S).view(1, 1, S, 1)
+    mask = j <= (torch.from_numpy(pos0).view(B, 1, 1, 1) + t)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale)
+    ref = ref.permute(0, 2, 1, 3).numpy()
+    for b in range(B):
+        np.testing.assert_allclose(o[b, :n_new[b]], ref[b, :n_new[b]], rtol=0, atol=1e-12)
+
+
+def test_single_valid_position_returns_its_v_row(oracle_lib):
+    B, T = 3, 16
+    q = rand_bits((B, 1, 16, 128), 50)
+    ck = rand_bits((B, T, 2, 128), 51)
+    cv = rand_bits((B, T, 2, 128), 52)
+    o, lse = oracle.decode(q, ck, cv, np.ones(B, np.int32), 1.0 / math.sqrt(128))
+    vf = oracle.bf16_array_to_f64(cv)
+    qf = oracle.bf16_array_to_f64(q)
+    kf = oracle.bf16_array_to_f64(ck)
+    for b in range(B):
+        for h in range(16):
+            assert np.array_equal(o[b, 0, h], vf[b, 0, h // 8])
+            s0 = float(np.dot(qf[b, 0, h], kf[b, 0, h // 8])) / math.sqrt(128)
+            assert abs(lse[b, h] - s0) < 1e-12
+
+
+def test_equal_scores_give_mean_of_v(oracle_lib):
+    """q = 0 makes every score 0: o is the mean of the visible V rows and
+    lse = ln(n)."""
+    B, T = 2, 33
+    q = np.zeros((B, 1, 16, 128), np.uint16)
+    ck = rand_bits((B, T, 2, 128), 60)
+    cv = rand_bits((B, T, 2, 128), 61)
+    kv = np.array([33, 17], np.int32)
+    o, lse = oracle.decode(q, ck, cv, kv, 1.0 / math.sqrt(128))
+    vf = oracle.bf16_array_to_f64(cv)
+    for b in range(B):
+        for h in range(16):
+            np.testing.assert_allclose(o[b, 0, h], vf[b, :kv[b], h // 8].mean(axis=0), atol=1e-14)
+            assert abs(lse[b, h] - math.log(kv[b])) < 1e-14
+    # all K rows equal: same result for any q
+    ck2 = np.repeat(ck[:, :1], T, axis=1)
+    q2 = rand_bits((B, 1, 16, 128), 62)
+    o2, _ = oracle.decode(q2, ck2, cv, kv, 1.0 / math.sqrt(128))
+    for b in range(B):
+        np.testing.assert_allclose(o2[b, 0, 0], vf[b, :kv[b], 0].mean(axis=0), atol=1e-13)
+
+
+def test_gqa_equals_mha_with_repeated_kv(oracle_lib):
+    B, S, T = 2, 4, 24
+    q = rand_bits((B, S, 16, 128), 70)
+    ck = rand_bits((B, T, 2, 128), 71)
+    cv = rand_bits((B, T, 2, 128), 72)
+    pos0 = np.array([3, 19], np.int32)
+    n_new = np.array([4, 2], np.int32)
+    sc = 1.0 / math.sqrt(128)
+    o1, l1 = oracle.prefill(q, ck, cv, pos0, n_new, sc)
+    ckr = np.repeat(ck, 8, axis=2)
+    cvr = np.repeat(cv, 8, axis=2)
+    o2, l2 = oracle.prefill(q, ckr, cvr, pos0, n_new, sc)
+    np.testing.assert_array_equal(np.nan_to_num(o1, nan=7.0), np.nan_to_num(o2, nan=7.0))
+    np.testing.assert_array_equal(np.nan_to_num(l1, nan=7.0), np.nan_to_num(l2, nan=7.0))
+
+
+def test_garbage_past_valid_length_changes_nothing(oracle_lib):
+    B, T = 4, 64
+    kv = torch.tensor([1, 20, 63, 64], dtype=torch.int32)
+    b1 = W.make_batch(80, B=B, S=1, T=T, pos0=kv, n_new=torch.zeros(B, dtype=torch.int32),
+                      garbage="none")
+    b2 = W.make_batch(80, B=B, S=1, T=T, pos0=kv, n_new=torch.zeros(B, dtype=torch.int32),
+                      garbage="nan")
+    sc = 1.0 / math.sqrt(128)
+    q = bf16_bits(b1.q[0])
+    o1, l1 = oracle.decode(q, bf16_bits(b1.cache_k[0]), bf16_bits(b1.cache_v[0]), kv.numpy(), sc)
+    o2, l2 = oracle.decode(q, bf16_bits(b2.cache_k[0]), bf16_bits(b2.cache_v[0]), kv.numpy(), sc)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    assert np.isfinite(o2).all()
+
+
+def test_static_masked_equals_length_aware(oracle_lib):
+    """Attending over all T rows with rows past the valid length masked
+    ("ARK-ASR-3B -- INT8 ONNX", section Shapes) gives the valid-prefix result
+    when the garbage is finite."""
+    B, T = 3, 48
+    kv = torch.tensor([5, 30, 48], dtype=torch.int32)
+    b = W.make_batch(90, B=B, S=1, T=T, pos0=kv, n_new=torch.zeros(B, dtype=torch.int32),
+                     garbage="big")
+    sc = 1.0 / math.sqrt(128)
+    q, ck, cv = bf16_bits(b.q[0]), bf16_bits(b.cache_k[0]), bf16_bits(b.cache_v[0])
+    o1, l1 = oracle.decode(q, ck, cv, kv.numpy(), sc)
+    o2, l2 = oracle.decode(q, ck, cv, kv.numpy(), sc, static_mode=True)
+    np.testing.assert_allclose(o1, o2, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, atol=1e-12)
+
+
+def test_split_and_combine_equals_unsplit(oracle_lib):
+    """Attention over [0, n) equals the log-sum-exp merge of attention over
+    any partition of [0, n) into chunks (empty chunks included)."""
+    T = 100
+    qrow = rand_bits((128,), 100)
+    k = rand_bits((T, 128), 101, scale=3.0)
+    v = rand_bits((T, 128), 102)
+    sc = 1.0 / math.sqrt(128)
+    o_ref, l_ref = oracle.attend_one(qrow, k, v, 0, T, sc)
+    for cuts in ([0, 64, 100], [0, 1, 2, 50, 99, 100], [0, 16, 16, 80, 100], [0, 100]):
+        parts = [oracle.attend_one(qrow, k, v, a, b_, sc) for a, b_ in zip(cuts[:-1], cuts[1:])]
+        o, l = oracle.combine(np.stack([p[0] for p in parts]), np.array([p[1] for p in parts]))
+        np.testing.assert_allclose(o, o_ref, atol=1e-12)
+        assert abs(l - l_ref) < 1e-12
+
+
+def test_combine_closed_forms(oracle_lib):
+    a = np.arange(8, dtype=np.float64)
+    o, l = oracle.combine(np.stack([a, a + 2]), np.array([1.5, 1.5]))
+    np.testing.assert_allclose(o, a + 1)
+    assert abs(l - (1.5 + math.log(2))) < 1e-15
+    o, l = oracle.combine(np.stack([a, np.full(8, np.nan)]), np.array([0.25, -np.inf]))
+    np.testing.assert_array_equal(o, a)
+    assert l == 0.25
+    o, l = oracle.combine(np.stack([a, a]), np.array([-np.inf, -np.inf]))
+    assert np.all(o == 0) and l == -np.inf
+
+
+def test_prefill_row_equals_decode_at_that_length(oracle_lib):
+    """Causal consistency: prefill row t of a request equals a decode at
+    kv_len = pos0 + t + 1 over the same cache."""
+    B, S, T = 2, 6, 32
+    q = rand_bits((B, S, 16, 128), 110)
+    ck = rand_bits((B, T, 2, 128), 111)
+    cv = rand_bits((B, T, 2, 128), 112)
+    pos0 = np.array([0, 20], np.int32)
+    n_new = np.array([6, 4], np.int32)
+    sc = 1.0 / math.sqrt(128)
+    o, lse = oracle.prefill(q, ck, cv, pos0, n_new, sc)
+    for b in range(B):
+        for t in range(n_new[b]):
+            od, ld = oracle.decode(q[b:b + 1, t:t + 1], ck[b:b + 1], cv[b:b + 1],
+                                   np.array([pos0[b] + t + 1], np.int32), sc)
+            np.testing.assert_array_equal(o[b, t], od[0, 0])
+            assert lse[b, :, t].tolist() == ld[0].tolist()
+
+
+def test_empty_visible_range(oracle_lib):
+    q = rand_bits((1, 1, 16, 128), 120)
+    ck = rand_bits((1, 8, 2, 128), 121)
+    o, lse = oracle.decode(q, ck, ck, np.array([0], np.int32), 0.1)
+    assert np.all(o == 0) and np.all(lse == -np.inf)
+
+
+# -------------------------------------------------------- prompt lengths ----
+
+def test_audio_slots_golden():
+    rows = []
+    with open(os.path.join(GOLDEN, "audio_slots.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                rows.append([int(x) for x in line.split()])
+    assert rows
+    for samples, mel, slots in rows:
+        assert W.audio_slots(samples) == slots
+        assert mel == samples // 160
+        assert max(W.audio_slots_from_mel(mel), 1) == slots
+    assert W.sweep_prompt_len() == 50
+    assert W.audio_slots(30 * 16000) + 12 == 387
