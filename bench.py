@@ -1,0 +1,407 @@
+"""Benchmark of the decode hot path: GQA attention over the static KV cache.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config ragged|single|long2048|long1024|prefill] [--mode aware|masked]
+
+A step is one pass of the whole decode path over one batch: for each of the
+36 layers, RoPE on the new q/k rows with the delta write into that layer's
+static cache, then split-KV decode attention (with its log-sum-exp merge).
+The default workload is the ragged decode batch: 32 requests, T = 512,
+valid lengths uniform in [40, 511] before the append (41..512 rows read),
+K/V with 1% x8 row outliers, 36 independent layers (604 MB of caches, larger
+than the 126 MB L2, so every step streams from HBM).
+
+Timing: W untimed warm-up steps, then exactly K steps replayed from one CUDA
+graph, bracketed by a barrier and a device synchronisation, timed with CUDA
+events on the launching stream; max over ranks.  Rank 0 prints one JSON line.
+Multi-GPU runs are independent replicas (weak scaling, no collective on the
+data path).
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload (the oracle is the only reference implementation there is).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn KV GB/s & tokens·layers/s (1×B200); % of HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+N_LAYERS = 36
+
+# Per-launch DRAM traffic of the decode kernel from an ncu capture, keyed by the
+# sha256 of the kernel source it was taken on; reported as null once the source
+# has changed.
+DECODE_TRAFFIC = {}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="ragged", choices=["ragged", "single", "long2048", "long1024"])
+    ap.add_argument("--mode", default="aware", choices=["aware", "masked"])
+    ap.add_argument("--max-splits", type=int, default=8)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def make_workload(name: str, layers: int, device: str):
+    from gqa_attention_static_b200 import workloads as W
+    if name == "ragged":
+        b = W.cfg_ragged_decode(layers=layers, device=device)
+        desc = "ragged decode B=32 T=512 kv_len U[41,512] 1% x8 K/V row outliers, 36 layers"
+    elif name == "single":
+        b = W.cfg_single_decode(layers=layers, device=device)
+        desc = "single decode B=1 T=512 kv_len 65, 36 layers"
+    elif name == "long2048":
+        b = W.cfg_long_decode(layers=layers, T=2048, device=device)
+        desc = "long decode B=32 T=2048 kv_len U[1501,2048], 36 layers"
+    else:
+        b = W.cfg_long_decode(layers=layers, T=1024, device=device)
+        desc = "long decode B=32 T=1024 full (kv_len 1024), 36 layers"
+    return b, desc
+
+
+def algorithmic_bytes(kv_len, B: int) -> int:
+    """Decode attention per layer: K+V rows read (1024 B per position for the
+    2 KV heads) + q read (4096 B) + o written (4096 B), per request."""
+    return int(sum(int(x) for x in kv_len) * 1024 + B * 8192)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def src_hash(rel: str) -> str:
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+class OracleRunner:
+    """The fp64 oracle (as it stands) on this host's cores: whole decode
+    layer-steps (RoPE + delta write + attention) over a bounded sample of the
+    workload's layers.  OpenMP threads = all host cores."""
+
+    def __init__(self, workload: str, mode: str, layers: int = 4):
+        import numpy as np
+        import torch
+        cores = os.cpu_count() or 1
+        os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+        import oracle
+        oracle.build()
+        self.oracle = oracle
+        self.cores = oracle.num_threads()
+        batch, self.desc = make_workload(workload, layers, "cpu")
+
+        def bits(x):
+            return x.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+        self.inputs = [(bits(batch.q[l]), bits(batch.k_new[l]), bits(batch.v_new[l]),
+                        bits(batch.cache_k[l]), bits(batch.cache_v[l])) for l in range(layers)]
+        self.pos0 = batch.pos0.numpy()
+        self.n_new = batch.n_new.numpy()
+        self.kv = batch.kv_len.numpy()
+        self.B = batch.B
+        self.static = (mode == "masked")
+        self.bytes_per_layer = algorithmic_bytes(self.kv, self.B)
+        self.i = 0
+
+    def layer_step(self):
+        q, kn, vn, ck, cv = self.inputs[self.i % len(self.inputs)]
+        self.i += 1
+        qr, ck2, cv2, _ = self.oracle.append_rope(q, kn, vn, ck, cv, self.pos0, self.n_new)
+        self.oracle.decode(qr, ck2, cv2, self.kv, 1.0 / math.sqrt(128), static_mode=self.static)
+
+    def timed(self, seconds: float = 0.0, min_layers: int = 1):
+        n = 0
+        t0 = time.perf_counter()
+        while True:
+            self.layer_step()
+            n += 1
+            el = time.perf_counter() - t0
+            if n >= min_layers and el >= seconds:
+                return n, el
+
+
+def cpu_baseline(workload: str, seconds: float, mode: str):
+    r = OracleRunner(workload, mode)
+    r.timed(0.0, 1)   # warm
+    n, el = r.timed(seconds, 1)
+    return {"value": r.bytes_per_layer * n / el / 1e9, "unit": "GB/s", "cores": r.cores, "kind": "oracle",
+            "sample": f"{n} layer-steps (4 distinct layers of: {r.desc}) in {el:.1f} s; fp64; OpenMP over "
+                      f"(request, head); GB/s by the same algorithmic-byte count as the GPU line",
+            "tokens_layers_per_s": r.B * n / el}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    r = OracleRunner(args.config, args.mode)
+    for _ in range(max(1, args.warmup)):
+        r.layer_step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r.layer_step()          # one step = one layer of the workload (bounded sample)
+    el = time.perf_counter() - t0
+    v = r.bytes_per_layer * args.steps / el / 1e9
+    sample = (f"each step = RoPE + delta write + decode attention of ONE of the 36 layers of: {r.desc} "
+              f"(4 distinct layers cycled); fp64 oracle; GB/s by the GPU line's algorithmic-byte count")
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": r.desc, "mode": args.mode},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": r.cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = f"cuda:{local}"
+
+    from gqa_attention_static_b200 import ops
+    from gqa_attention_static_b200.step import DecodeStep
+
+    ops.load()
+    mode = ops.ARK_MASKED_STATIC if args.mode == "masked" else ops.ARK_LENGTH_AWARE
+    batch, desc = make_workload(args.config, N_LAYERS, "cpu")
+    B, T = batch.B, batch.T
+    L = batch.layers
+
+    # device buffers: one packed input buffer (q | k_new | v_new) and one packed output (o | lse)
+    qsz = B * 16 * 128
+    ksz = B * 2 * 128
+    in_elems = L * (qsz + 2 * ksz)
+    d_in = torch.empty(in_elems, dtype=torch.bfloat16, device=dev)
+    qv = d_in[:L * qsz].view(L, B, 1, 16, 128)
+    kv_ = d_in[L * qsz:L * (qsz + ksz)].view(L, B, 1, 2, 128)
+    vv = d_in[L * (qsz + ksz):].view(L, B, 1, 2, 128)
+    for l in range(L):
+        qv[l].copy_(batch.q[l])
+        kv_[l].copy_(batch.k_new[l])
+        vv[l].copy_(batch.v_new[l])
+    ck = [x.to(dev) for x in batch.cache_k]
+    cv = [x.to(dev) for x in batch.cache_v]
+    pos0 = batch.pos0.to(dev)
+    n_new = batch.n_new.to(dev)
+    kv_len = batch.kv_len.to(dev)
+    step = DecodeStep([qv[l] for l in range(L)], [kv_[l] for l in range(L)], [vv[l] for l in range(L)],
+                      ck, cv, pos0, n_new, kv_len, max_splits=args.max_splits, mode=mode)
+    # outputs packed for the device->host read of the e2e leg
+    osz = B * 16 * 128
+    d_out_o = torch.empty(L * osz, dtype=torch.bfloat16, device=dev)
+    d_out_lse = torch.empty(L * B * 16, dtype=torch.float32, device=dev)
+    step.o = [d_out_o[l * osz:(l + 1) * osz].view(B, 1, 16, 128) for l in range(L)]
+    step.lse = [d_out_lse[l * B * 16:(l + 1) * B * 16].view(B, 16) for l in range(L)]
+
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step.run(s)                 # eager run before capture (loads kernels, sets attributes)
+    torch.cuda.synchronize()
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=s):
+        step.run(s)
+    g_attn = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_attn, stream=s):
+        step.attention_only(s)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed(fn, K):
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            e0.record(s)
+            for _ in range(K):
+                fn()
+            e1.record(s)
+        barrier()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    for _ in range(max(3, args.warmup)):
+        g_step.replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ms_total = timed(g_step.replay, args.steps)
+    # the dominant kernel alone, same stream, right after the timed region
+    ms_attn = timed(g_attn.replay, args.steps)
+    clk = clocks.stop()
+    ms_step = ms_total / args.steps
+    if int(step.status.item()) != 0:
+        print(f"device status word set: {int(step.status.item())}", file=sys.stderr)
+
+    kvl = batch.kv_len.tolist()
+    bytes_layer = algorithmic_bytes(kvl, B)
+    step_bytes = bytes_layer * L
+    value = step_bytes * world / (ms_step * 1e-3) / 1e9
+    tl = B * L * world / (ms_step * 1e-3)
+    per_launch_ms = ms_attn / args.steps / L         # one decode call (kernel + merge) per layer
+    peak, peak_kind = measured_peaks()
+    achieved = bytes_layer / (per_launch_ms * 1e-3) / 1e9
+    h = src_hash("gqa_attention_static_b200/csrc/decode.cu")
+    traffic = DECODE_TRAFFIC.get(h)
+
+    e2e = None
+    if not args.no_e2e:
+        h_in = torch.empty(in_elems, dtype=torch.bfloat16, pin_memory=True)
+        h_in.copy_(d_in.cpu())
+        h_o = torch.empty(L * osz, dtype=torch.bfloat16, pin_memory=True)
+        h_lse = torch.empty(L * B * 16, dtype=torch.float32, pin_memory=True)
+
+        def e2e_step():
+            d_in.copy_(h_in, non_blocking=True)
+            g_step.replay()
+            h_o.copy_(d_out_o, non_blocking=True)
+            h_lse.copy_(d_out_lse, non_blocking=True)
+
+        K2 = max(10, args.steps // 2)
+        with torch.cuda.stream(s):
+            for _ in range(3):
+                e2e_step()
+            ms_e2e = timed(e2e_step, K2) / K2
+        e2e = {"value": step_bytes * world / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": in_elems * 2, "d2h_bytes_per_step": L * osz * 2 + L * B * 16 * 4,
+               "ms_per_step": ms_e2e}
+
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(args.config, args.cpu_seconds, args.mode)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": desc, "batch": B, "max_total_len": T, "layers": L,
+                       "mode": "masked-static" if args.mode == "masked" else "length-aware",
+                       "max_splits": args.max_splits, "nsplit": step.nsplit,
+                       "l2": "inputs larger than L2 (%.0f MB of caches streamed per step)" %
+                             (2 * L * B * T * 2 * 128 * 2 / 1e6),
+                       "parallelism": f"replicas x{world}", "path": "per-layer calls in one CUDA graph"},
+            "tokens_layers_per_s": tl,
+            "roofline": {"kernel": "ark_attn_decode (decode_split_kernel + combine_kernel)", "bound": "hbm",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "peak_kind": peak_kind, "traffic": traffic,
+                         "launch_ms": per_launch_ms, "algorithmic_bytes_per_launch": bytes_layer},
+            "cpu_baseline": cb,
+            "e2e": e2e,
+            "gpu_launches": step.launches_per_step() * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        del g_step, g_attn
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

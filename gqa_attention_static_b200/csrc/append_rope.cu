@@ -1,0 +1,167 @@
+// append_rope.cu -- RoPE on the new query/key rows and the delta write into
+// the static cache.
+//
+// "ARK-ASR-3B -- INT8 ONNX" model card, section Shapes: the decoder returns
+// key_delta_i / value_delta_i rows for the positions written by this call, and
+// the host copies them into cache_{key,value}_i at cache_position.  Here that
+// copy is a device-side scatter fused with the rotary embedding of the new
+// rows (Qwen2 rotate-half form: SGLang-Omni cookbook "ARK-ASR-3B",
+// introduction).
+//
+// Rounding: table entries are fp32, inputs bf16, so every product is exact in
+// double; each output x[i]*c - x[i+64]*s (or x[i+64]*c + x[i]*s) is one double
+// subtraction/addition rounded once to bf16 with cvt.rn.bf16.f64.  The result
+// is therefore bit-reproducible.
+//
+// Work: one CTA per (t, b, layer) row; 128 threads cover (Hq + Hkv) heads x 16
+// groups of 4 rotary pairs, plus Hkv x 16 16-byte pieces of the V copy.  The op
+// moves ~10 KB per row and is latency-bound; it exists so the caller never
+// crosses to the host between the projection and the attention.
+#include "common.cuh"
+
+namespace ark {
+
+struct AppendLayer {
+    uint16_t* q;
+    const uint16_t* k_new;
+    const uint16_t* v_new;
+    uint16_t* cache_k;
+    uint16_t* cache_v;
+};
+
+struct AppendParams {
+    const int32_t* pos0;
+    const int32_t* n_new;
+    const float2* table;  // [T][64] {cos, sin}
+    uint32_t* status;
+    int B, S, T, Hq, Hkv;
+    AppendLayer layer[ARK_MAX_LAYERS];
+};
+
+__global__ void __launch_bounds__(128) append_rope_kernel(const __grid_constant__ AppendParams p) {
+    const int t = blockIdx.x;
+    const int b = blockIdx.y;
+    const AppendLayer& L = p.layer[blockIdx.z];
+
+    int nn = __ldg(p.n_new + b);
+    if (nn < 0 || nn > p.S) {
+        if (threadIdx.x == 0 && t == 0 && blockIdx.z == 0) report(p.status, ARK_DEV_BAD_KVLEN);
+        nn = nn < 0 ? 0 : p.S;
+    }
+    if (t >= nn) return;
+    const int pos = __ldg(p.pos0 + b) + t;
+    if (pos < 0 || pos >= p.T) {
+        if (threadIdx.x == 0 && blockIdx.z == 0) report(p.status, ARK_DEV_BAD_POS);
+        return;
+    }
+
+    const int nrot = (p.Hq + p.Hkv) * 16;    // items of 4 rotary pairs
+    const int ncopy = p.Hkv * 16;            // 16-byte pieces of V rows
+    const float4* trow = reinterpret_cast<const float4*>(p.table + static_cast<size_t>(pos) * 64);
+
+    for (int it = threadIdx.x; it < nrot + ncopy; it += blockDim.x) {
+        if (it < nrot) {
+            const int head = it >> 4;
+            const int pg = it & 15;           // pairs 4pg .. 4pg+3
+            const uint16_t* src;
+            uint16_t* dst;
+            if (head < p.Hq) {
+                uint16_t* row = L.q + ((static_cast<size_t>(b) * p.S + t) * p.Hq + head) * kHeadDim;
+                src = row;
+                dst = row;
+            } else {
+                const int g = head - p.Hq;
+                src = L.k_new + ((static_cast<size_t>(b) * p.S + t) * p.Hkv + g) * kHeadDim;
+                dst = L.cache_k + ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + g) * kHeadDim;
+            }
+            const uint2 lo = *reinterpret_cast<const uint2*>(src + 4 * pg);
+            const uint2 hi = *reinterpret_cast<const uint2*>(src + 64 + 4 * pg);
+            const float4 cs01 = __ldg(trow + 2 * pg);      // c0 s0 c1 s1
+            const float4 cs23 = __ldg(trow + 2 * pg + 1);  // c2 s2 c3 s3
+            const uint16_t xl[4] = {static_cast<uint16_t>(lo.x & 0xffff), static_cast<uint16_t>(lo.x >> 16),
+                                    static_cast<uint16_t>(lo.y & 0xffff), static_cast<uint16_t>(lo.y >> 16)};
+            const uint16_t xh[4] = {static_cast<uint16_t>(hi.x & 0xffff), static_cast<uint16_t>(hi.x >> 16),
+                                    static_cast<uint16_t>(hi.y & 0xffff), static_cast<uint16_t>(hi.y >> 16)};
+            const float cc[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
+            const float ss[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
+            uint16_t yl[4], yh[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const double a = bf16_bits_to_f64(xl[i]);
+                const double h = bf16_bits_to_f64(xh[i]);
+                const double c = static_cast<double>(cc[i]);
+                const double s = static_cast<double>(ss[i]);
+                // both products are exact in double, so contraction cannot change the result
+                yl[i] = f64_to_bf16_rn(a * c - h * s);
+                yh[i] = f64_to_bf16_rn(h * c + a * s);
+            }
+            uint2 ol, oh;
+            ol.x = static_cast<uint32_t>(yl[0]) | (static_cast<uint32_t>(yl[1]) << 16);
+            ol.y = static_cast<uint32_t>(yl[2]) | (static_cast<uint32_t>(yl[3]) << 16);
+            oh.x = static_cast<uint32_t>(yh[0]) | (static_cast<uint32_t>(yh[1]) << 16);
+            oh.y = static_cast<uint32_t>(yh[2]) | (static_cast<uint32_t>(yh[3]) << 16);
+            *reinterpret_cast<uint2*>(dst + 4 * pg) = ol;
+            *reinterpret_cast<uint2*>(dst + 64 + 4 * pg) = oh;
+        } else {
+            const int c = it - nrot;
+            const int g = c >> 4;
+            const int piece = c & 15;
+            const uint4* src = reinterpret_cast<const uint4*>(
+                L.v_new + ((static_cast<size_t>(b) * p.S + t) * p.Hkv + g) * kHeadDim);
+            uint4* dst = reinterpret_cast<uint4*>(
+                L.cache_v + ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + g) * kHeadDim);
+            dst[piece] = src[piece];
+        }
+    }
+}
+
+}  // namespace ark
+
+using namespace ark;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ark_status check_common(int B, int S, int T, int Hq, int Hkv, int D) {
+    if (B <= 0 || S <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0) return ARK_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return ARK_ERR_INVALID_ARG;
+    if (T > ARK_MAX_T) return ARK_ERR_UNSUPPORTED;
+    if (D != kHeadDim || Hq / Hkv != kGroup) return ARK_ERR_UNSUPPORTED;
+    if (B > 65535 || S > 2147483647 / 2) return ARK_ERR_UNSUPPORTED;
+    return ARK_OK;
+}
+
+ark_status launch_append(AppendParams& prm, int L, cudaStream_t stream) {
+    dim3 grid(prm.S, prm.B, L);
+    append_rope_kernel<<<grid, 128, 0, stream>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" ark_status ark_attn_append_rope(void* q, const void* k_new, const void* v_new,
+                                           void* cache_k, void* cache_v,
+                                           const int32_t* pos0, const int32_t* n_new,
+                                           int B, int S, int T, int Hq, int Hkv, int D,
+                                           const float* d_table, uint32_t* d_status,
+                                           cudaStream_t stream) {
+    if (!q || !k_new || !v_new || !cache_k || !cache_v || !pos0 || !n_new || !d_table)
+        return ARK_ERR_INVALID_ARG;
+    ark_status st = check_common(B, S, T, Hq, Hkv, D);
+    if (st != ARK_OK) return st;
+    if (S > 65535) return ARK_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(cache_k) ||
+        !aligned16(cache_v) || !aligned16(d_table))
+        return ARK_ERR_INVALID_ARG;
+    AppendParams prm{};
+    prm.pos0 = pos0;
+    prm.n_new = n_new;
+    prm.table = reinterpret_cast<const float2*>(d_table);
+    prm.status = d_status;
+    prm.B = B; prm.S = S; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
+    prm.layer[0] = AppendLayer{static_cast<uint16_t*>(q), static_cast<const uint16_t*>(k_new),
+                               static_cast<const uint16_t*>(v_new), static_cast<uint16_t*>(cache_k),
+                               static_cast<uint16_t*>(cache_v)};
+    return launch_append(prm, 1, stream);
+}

@@ -1,0 +1,222 @@
+"""Thin ctypes binding of libarkattn (``include/arkattn.h``).
+
+Each ``ark_attn_*`` function here has the name and the meaning of the C entry
+point it forwards to; it only derives sizes from tensor shapes, checks dtype /
+device / contiguity, and passes ``data_ptr()`` and the current CUDA stream.
+All compute happens in the library's CUDA kernels.  There is no fallback: if
+``libarkattn.so`` is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libarkattn.so")
+
+ARK_OK = 0
+ARK_ERR_INVALID_ARG = 1
+ARK_ERR_UNSUPPORTED = 2
+ARK_ERR_WORKSPACE = 3
+ARK_ERR_CUDA = 4
+ARK_ERR_TIMEOUT = 5
+
+ARK_LENGTH_AWARE = 0
+ARK_MASKED_STATIC = 1
+
+ARK_DEV_BAD_POS = 1
+ARK_DEV_BAD_KVLEN = 2
+ARK_DEV_TIMEOUT = 4
+
+ARK_MAX_LAYERS = 64
+
+# every symbol include/arkattn.h declares
+EXPORTS = (
+    "ark_attn_status_string",
+    "ark_attn_rope_table_bytes",
+    "ark_attn_rope_table_init",
+    "ark_attn_append_rope",
+    "ark_attn_decode_workspace_size",
+    "ark_attn_decode",
+    "ark_attn_combine",
+)
+
+
+class ArkError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libarkattn.so (built in-tree by ``gqa_attention_static_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libarkattn.so is not built ({LIB_PATH}); run "
+                           "`python -m gqa_attention_static_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.ark_attn_status_string.argtypes = [I]
+    lib.ark_attn_status_string.restype = ctypes.c_char_p
+    lib.ark_attn_rope_table_bytes.argtypes = [I, I]
+    lib.ark_attn_rope_table_bytes.restype = Z
+    lib.ark_attn_rope_table_init.argtypes = [P, I, I, ctypes.c_double, P]
+    lib.ark_attn_rope_table_init.restype = I
+    lib.ark_attn_append_rope.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P]
+    lib.ark_attn_append_rope.restype = I
+    lib.ark_attn_decode_workspace_size.argtypes = [I, I, I, I, I]
+    lib.ark_attn_decode_workspace_size.restype = Z
+    lib.ark_attn_decode.argtypes = [P, P, P, P, I, I, I, I, I, ctypes.c_float, I, I, P, Z, P, P, P, P]
+    lib.ark_attn_decode.restype = I
+    lib.ark_attn_combine.argtypes = [P, P, I, I, I, I, P, P, P]
+    lib.ark_attn_combine.restype = I
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load().ark_attn_status_string(int(code)).decode()
+
+
+def _raise(code: int, what: str) -> None:
+    if code != ARK_OK:
+        raise ArkError(code, what)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: Optional[int] = None) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+
+
+# ------------------------------------------------------------------ RoPE ----
+
+def ark_attn_rope_table_bytes(T: int, D: int = 128) -> int:
+    return int(load().ark_attn_rope_table_bytes(T, D))
+
+
+def ark_attn_rope_table_init(table: torch.Tensor, T: int, D: int = 128, rope_theta: float = 1e6,
+                             stream=None) -> None:
+    _need(table, "table", torch.float32)
+    if table.numel() * 4 < ark_attn_rope_table_bytes(T, D):
+        raise ValueError("table too small")
+    _raise(load().ark_attn_rope_table_init(_ptr(table), T, D, float(rope_theta), _stream(stream)),
+           "ark_attn_rope_table_init")
+
+
+def rope_table(T: int, D: int = 128, rope_theta: float = 1e6, device="cuda") -> torch.Tensor:
+    """Allocate and fill a rotary table [T, D/2, 2] (fp32 cos, sin)."""
+    t = torch.empty((T, D // 2, 2), dtype=torch.float32, device=device)
+    ark_attn_rope_table_init(t, T, D, rope_theta)
+    return t
+
+
+# --------------------------------------------------------- RoPE + append ----
+
+def ark_attn_append_rope(q, k_new, v_new, cache_k, cache_v, pos0, n_new, table,
+                         status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """q [B,S,Hq,D] (rotated in place), k_new/v_new [B,S,Hkv,D] -> rows
+    pos0[b] + t of cache_k/cache_v [B,T,Hkv,D]."""
+    for name, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("cache_k", cache_k),
+                    ("cache_v", cache_v)):
+        _need(t, name, torch.bfloat16, 4)
+    _need(pos0, "pos0", torch.int32, 1)
+    _need(n_new, "n_new", torch.int32, 1)
+    _need(table, "table", torch.float32)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    B, S, Hq, D = q.shape
+    T, Hkv = cache_k.shape[1], cache_k.shape[2]
+    if tuple(k_new.shape) != (B, S, Hkv, D) or tuple(v_new.shape) != (B, S, Hkv, D):
+        raise ValueError("k_new/v_new shape")
+    if tuple(cache_v.shape) != tuple(cache_k.shape) or cache_k.shape[0] != B or cache_k.shape[3] != D:
+        raise ValueError("cache shape")
+    if table.numel() < T * (D // 2) * 2:
+        raise ValueError("rotary table has fewer than T rows")
+    _raise(load().ark_attn_append_rope(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(cache_k), _ptr(cache_v),
+                                       _ptr(pos0), _ptr(n_new), B, S, T, Hq, Hkv, D, _ptr(table),
+                                       _ptr(status), _stream(stream)),
+           "ark_attn_append_rope")
+
+
+# ---------------------------------------------------------------- decode ----
+
+def ark_attn_decode_workspace_size(B: int, Hq: int, D: int, T: int, max_splits: int) -> int:
+    return int(load().ark_attn_decode_workspace_size(B, Hq, D, T, max_splits))
+
+
+def ark_attn_decode(q, cache_k, cache_v, kv_len, o, lse, scale: float, mode: int = ARK_LENGTH_AWARE,
+                    max_splits: int = 8, workspace: Optional[torch.Tensor] = None,
+                    status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """q [B,1,Hq,D] -> o [B,1,Hq,D] bf16, lse [B,Hq] fp32 over kv_len[b] rows."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(cache_k, "cache_k", torch.bfloat16, 4)
+    _need(cache_v, "cache_v", torch.bfloat16, 4)
+    _need(kv_len, "kv_len", torch.int32, 1)
+    _need(o, "o", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32)
+    B, S, Hq, D = q.shape
+    if S != 1:
+        raise ValueError("decode takes one query row per request")
+    T, Hkv = cache_k.shape[1], cache_k.shape[2]
+    if tuple(o.shape) != tuple(q.shape) or lse.numel() != B * Hq:
+        raise ValueError("o/lse shape")
+    ws_bytes = 0
+    if workspace is not None:
+        _need(workspace, "workspace", workspace.dtype)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    if status is not None:
+        _need(status, "status", torch.int32)
+    _raise(load().ark_attn_decode(_ptr(q), _ptr(cache_k), _ptr(cache_v), _ptr(kv_len), B, T, Hq, Hkv, D,
+                                  float(scale), int(mode), int(max_splits), _ptr(workspace), ws_bytes,
+                                  _ptr(o), _ptr(lse), _ptr(status), _stream(stream)),
+           "ark_attn_decode")
+
+
+def decode_workspace(B: int, Hq: int, D: int, T: int, max_splits: int, device="cuda"):
+    n = ark_attn_decode_workspace_size(B, Hq, D, T, max_splits)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device) if n else None
+
+
+# --------------------------------------------------------------- combine ----
+
+def ark_attn_combine(o_part, lse_part, o, lse, stream=None) -> None:
+    """o_part [B,Hq,nsplit,D] fp32, lse_part [B,Hq,nsplit] fp32 -> o [B,Hq,D]
+    bf16 (any shape with that many elements), lse [B,Hq] fp32."""
+    _need(o_part, "o_part", torch.float32, 4)
+    _need(lse_part, "lse_part", torch.float32, 3)
+    _need(o, "o", torch.bfloat16)
+    _need(lse, "lse", torch.float32)
+    B, Hq, nsplit, D = o_part.shape
+    if tuple(lse_part.shape) != (B, Hq, nsplit) or o.numel() != B * Hq * D or lse.numel() != B * Hq:
+        raise ValueError("combine shapes")
+    _raise(load().ark_attn_combine(_ptr(o_part), _ptr(lse_part), B, Hq, nsplit, D, _ptr(o), _ptr(lse),
+                                   _stream(stream)),
+           "ark_attn_combine")

@@ -1,0 +1,78 @@
+"""Host-side plumbing for one decode step over L independent layers.
+
+A decode step is, per layer: RoPE on the new q/k rows and the delta write into
+that layer's static cache (``ark_attn_append_rope``), then split-KV decode
+attention over the valid rows (``ark_attn_decode``, which runs the
+log-sum-exp merge when it splits).  All launches go to one CUDA stream; the
+step can be captured in a CUDA graph.  This module only owns buffers and
+orders calls -- every step of the computation is a libarkattn kernel.
+"""
+from __future__ import annotations
+
+import math
+from typing import List, Optional
+
+import torch
+
+from . import ops
+
+
+class DecodeStep:
+    """Decode step of ``layers`` layers over a batch of B requests.
+
+    Buffers (per layer lists, all on ``device``):
+      q [B,1,Hq,D] (rotated in place), k_new/v_new [B,1,Hkv,D],
+      cache_k/cache_v [B,T,Hkv,D], o [B,1,Hq,D], lse [B,Hq];
+    shared: pos0, n_new, kv_len int32[B], rotary table, workspace, status.
+    """
+
+    def __init__(self, q: List[torch.Tensor], k_new: List[torch.Tensor], v_new: List[torch.Tensor],
+                 cache_k: List[torch.Tensor], cache_v: List[torch.Tensor], pos0: torch.Tensor,
+                 n_new: torch.Tensor, kv_len: torch.Tensor, max_splits: int = 8,
+                 mode: int = ops.ARK_LENGTH_AWARE, rope_theta: float = 1e6,
+                 scale: Optional[float] = None):
+        self.q, self.k_new, self.v_new = q, k_new, v_new
+        self.cache_k, self.cache_v = cache_k, cache_v
+        self.pos0, self.n_new, self.kv_len = pos0, n_new, kv_len
+        self.layers = len(q)
+        self.B, _, self.Hq, self.D = q[0].shape
+        self.T = cache_k[0].shape[1]
+        self.Hkv = cache_k[0].shape[2]
+        dev = q[0].device
+        self.max_splits = max_splits
+        self.mode = mode
+        self.scale = scale if scale is not None else 1.0 / math.sqrt(self.D)
+        self.table = ops.rope_table(self.T, self.D, rope_theta, device=dev)
+        self.workspace = ops.decode_workspace(self.B, self.Hq, self.D, self.T, max_splits, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.o = [torch.empty_like(x) for x in q]
+        self.lse = [torch.empty(self.B, self.Hq, dtype=torch.float32, device=dev) for _ in q]
+
+    @property
+    def nsplit(self) -> int:
+        ws = ops.ark_attn_decode_workspace_size(self.B, self.Hq, self.D, self.T, self.max_splits)
+        if ws == 0:
+            return 1
+        per = -(-self.T // self.max_splits)
+        chunk = max(64, -(-per // 16) * 16)
+        return -(-self.T // chunk)
+
+    def launches_per_step(self) -> int:
+        return self.layers * (2 + (1 if self.nsplit > 1 else 0))
+
+    def run(self, stream=None) -> None:
+        for l in range(self.layers):
+            ops.ark_attn_append_rope(self.q[l], self.k_new[l], self.v_new[l], self.cache_k[l],
+                                     self.cache_v[l], self.pos0, self.n_new, self.table, self.status,
+                                     stream)
+            ops.ark_attn_decode(self.q[l], self.cache_k[l], self.cache_v[l], self.kv_len, self.o[l],
+                                self.lse[l], self.scale, self.mode, self.max_splits, self.workspace,
+                                self.status, stream)
+
+    def attention_only(self, stream=None) -> None:
+        """The decode attention of every layer without the append (for timing
+        the dominant kernel alone)."""
+        for l in range(self.layers):
+            ops.ark_attn_decode(self.q[l], self.cache_k[l], self.cache_v[l], self.kv_len, self.o[l],
+                                self.lse[l], self.scale, self.mode, self.max_splits, self.workspace,
+                                self.status, stream)

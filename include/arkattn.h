@@ -1,0 +1,171 @@
+/*
+ * arkattn.h -- C ABI of libarkattn: grouped-query attention over a static,
+ * sequence-major KV cache, hand-written for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the attention step of the ARK-ASR-3B decoder as the
+ * "ARK-ASR-3B -- INT8 ONNX" model card describes it in its section Shapes:
+ * 16 query heads share 2 KV heads (8 query heads per KV head), head dim 128,
+ * and each layer keeps a static cache cache_{key,value}_i of shape
+ * [1, max_total_len, 2, 128], sequence-major; each call produces
+ * key_delta/value_delta rows for the positions it writes, and those rows go
+ * into the cache at cache_position.  Here the batch dimension is B, so one
+ * layer's cache is [B, T, Hkv, D] with T = max_total_len.  The decoder is a
+ * Qwen2 language model (SGLang-Omni cookbook "ARK-ASR-3B", introduction), so
+ * RoPE (rotate-half form) is applied to the new query and key rows.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers to contiguous, row-major memory
+ *     in the layouts stated per call; bf16 tensors are `void*`.  Every tensor
+ *     pointer must be 16-byte aligned.
+ *   - The caller owns and allocates every buffer (tensors, workspace, RoPE
+ *     table, status word).  The library allocates no device memory and keeps
+ *     no per-call state.
+ *   - Calls are asynchronous on `stream` and enqueue kernels only (except
+ *     ark_attn_rope_table_init, which copies from the host and synchronises).
+ *   - Arguments the host can see are checked before anything is launched; a
+ *     failed check returns an error and launches nothing.
+ *   - Values that live on the device (cache positions, lengths) cannot be
+ *     checked by the host without a synchronisation.  Kernels check them,
+ *     skip or clamp what is out of range and OR a bit into the caller's
+ *     status word `*d_status` (device memory, uint32).  The caller reads the
+ *     word after synchronising.  `d_status` may be NULL to skip reporting.
+ *   - Only D = 128 and Hq/Hkv = 8 are instantiated (ARK_ERR_UNSUPPORTED
+ *     otherwise); T <= ARK_MAX_T.
+ *   - A launch failure returns ARK_ERR_CUDA; the CUDA error is left to the
+ *     caller (cudaGetLastError).
+ */
+#ifndef ARKATTN_H_
+#define ARKATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define ARK_API __attribute__((visibility("default")))
+#else
+#define ARK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ark_status {
+    ARK_OK = 0,
+    ARK_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, misalignment, Hq % Hkv != 0 */
+    ARK_ERR_UNSUPPORTED = 2,   /* a shape this build does not instantiate (D != 128, Hq/Hkv != 8) */
+    ARK_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the *_workspace_size answer */
+    ARK_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+    ARK_ERR_TIMEOUT = 5        /* reserved: a bounded device wait gave up (see ARK_DEV_TIMEOUT) */
+} ark_status;
+
+/* Decode modes.  Both give the same result (to fp32 rounding order).
+ * LENGTH_AWARE reads only the kv_len[b] valid rows of each request.
+ * MASKED_STATIC reads all T rows and gives the rows at or past kv_len[b] a
+ * score of -inf, which is what a static cache graph does: the ONNX model card
+ * ("ARK-ASR-3B -- INT8 ONNX", section Shapes) states that the decoder attends
+ * over ALL max_total_len positions on every token however few are valid.
+ * Precondition of MASKED_STATIC: the rows past kv_len hold finite values
+ * (a masked row contributes 0 x its V row, which is NaN for a non-finite row). */
+typedef enum ark_decode_mode {
+    ARK_LENGTH_AWARE = 0,
+    ARK_MASKED_STATIC = 1
+} ark_decode_mode;
+
+/* Bits OR-ed into the device status word. */
+#define ARK_DEV_BAD_POS   1u  /* cache_position + t outside [0, T): that row was skipped */
+#define ARK_DEV_BAD_KVLEN 2u  /* kv_len or n_new outside its range: clamped (kv_len 0 gives o = 0, lse = -inf) */
+#define ARK_DEV_TIMEOUT   4u  /* a bounded wait on an asynchronous copy gave up; outputs of that block not written */
+
+#define ARK_MAX_T 65536
+#define ARK_MAX_LAYERS 64
+
+/* Human-readable name of a status code (static string, never NULL). */
+ARK_API const char* ark_attn_status_string(ark_status s);
+
+/* ------------------------------------------------------------------ RoPE ----
+ * Rotary table for positions 0..T-1: for pair i < D/2, inv_freq_i =
+ * rope_theta^(-2i/D), angle = p * inv_freq_i computed in double, and the
+ * table holds (float)cos(angle), (float)sin(angle).  The pages name the
+ * decoder as Qwen2 (SGLang-Omni cookbook "ARK-ASR-3B", introduction) and give
+ * no formula; this is the Qwen2 convention, with theta 1e6 for ARK-ASR-3B's
+ * decoder as configured by the caller.
+ * d_table: device, ark_attn_rope_table_bytes(T, D) bytes, layout [T][D/2] of
+ *   float2 {cos, sin}.  Caller-owned.  Computed on the host, copied with
+ *   cudaMemcpyAsync on `stream`, and the call synchronises `stream` before it
+ *   returns (set-up only; not for stream capture).
+ */
+ARK_API size_t ark_attn_rope_table_bytes(int T, int D);
+ARK_API ark_status ark_attn_rope_table_init(float* d_table, int T, int D, double rope_theta,
+                                    cudaStream_t stream);
+
+/* ---------------------------------------------------------- RoPE + write ----
+ * For each request b < B and new row t < n_new[b] (t < S), at the absolute
+ * position p = pos0[b] + t (pos0 is cache_position: the number of valid
+ * cache rows before this call):
+ *   q[b,t,h,:]       <- RoPE_p(q[b,t,h,:])     for h < Hq   (in place)
+ *   cache_k[b,p,g,:] <- RoPE_p(k_new[b,t,g,:]) for g < Hkv  (the key delta)
+ *   cache_v[b,p,g,:] <- v_new[b,t,g,:]                      (the value delta, bit copy)
+ * ("ARK-ASR-3B -- INT8 ONNX", section Shapes: the delta rows land in the
+ * cache at cache_position.)  RoPE_p pairs element i with i + D/2:
+ *   x'[i] = x[i] c - x[i+D/2] s,  x'[i+D/2] = x[i+D/2] c + x[i] s,
+ * c, s the fp32 table entries of (p, i); each output is formed in double and
+ * rounded once to bf16 (nearest-even), so the result is bit-reproducible.
+ * Layouts: q [B,S,Hq,D] bf16; k_new, v_new [B,S,Hkv,D] bf16; cache_k, cache_v
+ * [B,T,Hkv,D] bf16; pos0, n_new int32[B] (device); d_table from
+ * ark_attn_rope_table_init with at least T rows.
+ * Rows t >= n_new[b] are not touched.  A row with p outside [0, T) is skipped
+ * entirely (q not rotated, nothing written) and sets ARK_DEV_BAD_POS.
+ */
+ARK_API ark_status ark_attn_append_rope(void* q, const void* k_new, const void* v_new,
+                                void* cache_k, void* cache_v,
+                                const int32_t* pos0, const int32_t* n_new,
+                                int B, int S, int T, int Hq, int Hkv, int D,
+                                const float* d_table, uint32_t* d_status, cudaStream_t stream);
+
+/* ---------------------------------------------------------------- decode ----
+ * One query row per request (the new token, already rotated) attends to the
+ * kv_len[b] valid cache rows of its KV head g = h / (Hq/Hkv):
+ *   s_j = scale * <q[b,0,h,:], cache_k[b,j,g,:]>,  j < kv_len[b]
+ *   o[b,0,h,:] = sum_j softmax(s)_j cache_v[b,j,g,:],   lse[b,h] = ln sum_j exp(s_j)
+ * All 8 query heads of a KV group are served from one read of each K/V row.
+ * The key range is split into chunks of equal length processed in parallel;
+ * with more than one chunk the partial results go to `workspace` and a
+ * log-sum-exp merge (the kernel behind ark_attn_combine) writes o and lse.
+ * Layouts: q [B,1,Hq,D] bf16; cache_k, cache_v [B,T,Hkv,D] bf16; kv_len
+ * int32[B] (device; the new row is already appended, so the query attends to
+ * itself); o [B,1,Hq,D] bf16; lse [B,Hq] fp32 (natural log).
+ * kv_len outside [0, T] is clamped and sets ARK_DEV_BAD_KVLEN; kv_len = 0
+ * gives o = 0, lse = -inf.
+ * max_splits >= 1 bounds the number of chunks; workspace may be NULL when
+ * ark_attn_decode_workspace_size(...) returns 0.  Accumulation is fp32 from
+ * bf16 operands on the tensor cores; P is rounded to bf16 before P.V.
+ */
+ARK_API size_t ark_attn_decode_workspace_size(int B, int Hq, int D, int T, int max_splits);
+ARK_API ark_status ark_attn_decode(const void* q, const void* cache_k, const void* cache_v,
+                           const int32_t* kv_len, int B, int T, int Hq, int Hkv, int D,
+                           float scale, ark_decode_mode mode, int max_splits,
+                           void* workspace, size_t workspace_bytes,
+                           void* o, float* lse, uint32_t* d_status, cudaStream_t stream);
+
+/* --------------------------------------------------------------- combine ----
+ * Log-sum-exp merge of nsplit partial results of the same query over
+ * disjoint key ranges.  For each (b, h):
+ *   M = max_c lse_part[b,h,c],  w_c = exp(lse_part[b,h,c] - M)
+ *   o[b,h,:] = sum_c w_c o_part[b,h,c,:] / sum_c w_c,   lse[b,h] = M + ln sum_c w_c
+ * A part with lse_part = -inf (no keys) has weight 0 and its o_part row is not
+ * read; all parts empty gives o = 0, lse = -inf.  (The pages have no split;
+ * this is the exact identity that lets a softmax be computed in pieces.)
+ * Layouts: o_part [B,Hq,nsplit,D] fp32 (each part normalised by its own sum),
+ * lse_part [B,Hq,nsplit] fp32; o [B,Hq,D] bf16 (the same memory as
+ * [B,1,Hq,D]); lse [B,Hq] fp32.
+ */
+ARK_API ark_status ark_attn_combine(const float* o_part, const float* lse_part, int B, int Hq,
+                            int nsplit, int D, void* o, float* lse, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ARKATTN_H_ */

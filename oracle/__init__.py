@@ -62,6 +62,8 @@ def _load():
         lib.ora_attention.restype = None
         lib.ora_combine.argtypes = [P, P, I, I, P, P]
         lib.ora_combine.restype = None
+        lib.ora_num_threads.argtypes = []
+        lib.ora_num_threads.restype = I
         _lib = lib
     return _lib
 
@@ -73,6 +75,11 @@ def _ptr(a: np.ndarray) -> int:
 def _c(a, dtype) -> np.ndarray:
     a = np.ascontiguousarray(a, dtype=dtype)
     return a
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle's attention loop uses."""
+    return int(_load().ora_num_threads())
 
 
 # ------------------------------------------------------------------ bf16 ----
