@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--config", default="ragged", choices=["ragged", "single", "long2048", "long1024"])
     ap.add_argument("--mode", default="aware", choices=["aware", "masked"])
     ap.add_argument("--max-splits", type=int, default=8)
+    ap.add_argument("--per-layer", action="store_true",
+                    help="issue the single-layer calls layer by layer instead of the layer-batched calls")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -281,7 +283,8 @@ def main():
     n_new = batch.n_new.to(dev)
     kv_len = batch.kv_len.to(dev)
     step = DecodeStep([qv[l] for l in range(L)], [kv_[l] for l in range(L)], [vv[l] for l in range(L)],
-                      ck, cv, pos0, n_new, kv_len, max_splits=args.max_splits, mode=mode)
+                      ck, cv, pos0, n_new, kv_len, max_splits=args.max_splits, mode=mode,
+                      batched=not args.per_layer)
     # outputs packed for the device->host read of the e2e leg
     osz = B * 16 * 128
     d_out_o = torch.empty(L * osz, dtype=torch.bfloat16, device=dev)
@@ -297,9 +300,18 @@ def main():
     g_step = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_step, stream=s):
         step.run(s)
-    g_attn = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_attn, stream=s):
-        step.attention_only(s)
+    # The same steps with event-record nodes around each kernel group, to read
+    # per-launch kernel durations from inside the timed stream.
+    U = 8 if step.batched else 2
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(U)]
+    g_inst = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_inst, stream=s):
+        for u in range(U):
+            ev[u][0].record(s)
+            step.append(s)
+            ev[u][1].record(s)
+            step.attention(s)
+            ev[u][2].record(s)
     torch.cuda.synchronize()
 
     def barrier():
@@ -332,21 +344,26 @@ def main():
     clocks.start()
     time.sleep(0.3)
     ms_total = timed(g_step.replay, args.steps)
-    # the dominant kernel alone, same stream, right after the timed region
-    ms_attn = timed(g_attn.replay, args.steps)
+    # kernel durations: the instrumented graph, replayed right after, same stream
+    reps = max(1, args.steps // U)
+    timed(g_inst.replay, reps)
     clk = clocks.stop()
     ms_step = ms_total / args.steps
     if int(step.status.item()) != 0:
         print(f"device status word set: {int(step.status.item())}", file=sys.stderr)
+    attn_ms = [ev[u][1].elapsed_time(ev[u][2]) for u in range(U)]
+    app_ms = [ev[u][0].elapsed_time(ev[u][1]) for u in range(U)]
+    calls_per_group = 1 if step.batched else L          # decode launches per attention group
+    per_launch_ms = sum(attn_ms) / len(attn_ms) / calls_per_group
 
     kvl = batch.kv_len.tolist()
     bytes_layer = algorithmic_bytes(kvl, B)
     step_bytes = bytes_layer * L
     value = step_bytes * world / (ms_step * 1e-3) / 1e9
     tl = B * L * world / (ms_step * 1e-3)
-    per_launch_ms = ms_attn / args.steps / L         # one decode call (kernel + merge) per layer
+    bytes_launch = bytes_layer * (L if step.batched else 1)
     peak, peak_kind = measured_peaks()
-    achieved = bytes_layer / (per_launch_ms * 1e-3) / 1e9
+    achieved = bytes_launch / (per_launch_ms * 1e-3) / 1e9
     h = src_hash("gqa_attention_static_b200/csrc/decode.cu")
     traffic = DECODE_TRAFFIC.get(h)
 
@@ -386,12 +403,16 @@ def main():
                        "max_splits": args.max_splits, "nsplit": step.nsplit,
                        "l2": "inputs larger than L2 (%.0f MB of caches streamed per step)" %
                              (2 * L * B * T * 2 * 128 * 2 / 1e6),
-                       "parallelism": f"replicas x{world}", "path": "per-layer calls in one CUDA graph"},
+                       "parallelism": f"replicas x{world}",
+                       "path": ("per-layer calls" if args.per_layer else "layer-batched calls") +
+                               " replayed from one CUDA graph"},
             "tokens_layers_per_s": tl,
-            "roofline": {"kernel": "ark_attn_decode (decode_split_kernel + combine_kernel)", "bound": "hbm",
-                         "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                         "peak_kind": peak_kind, "traffic": traffic,
-                         "launch_ms": per_launch_ms, "algorithmic_bytes_per_launch": bytes_layer},
+            "roofline": {"kernel": "decode_kernel (ark_attn_decode%s, merge fused)" %
+                                   ("" if args.per_layer else "_layers"),
+                         "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
+                         "launch_ms": per_launch_ms, "algorithmic_bytes_per_launch": bytes_launch,
+                         "append_ms_per_step": sum(app_ms) / len(app_ms)},
             "cpu_baseline": cb,
             "e2e": e2e,
             "gpu_launches": step.launches_per_step() * args.steps,
@@ -399,7 +420,7 @@ def main():
         }
         print(json.dumps(line), flush=True)
     if world > 1:
-        del g_step, g_attn
+        del g_step, g_inst
         dist.destroy_process_group()
 
 

@@ -165,3 +165,35 @@ extern "C" ark_status ark_attn_append_rope(void* q, const void* k_new, const voi
                                static_cast<uint16_t*>(cache_v)};
     return launch_append(prm, 1, stream);
 }
+
+extern "C" ark_status ark_attn_append_rope_layers(int L, void* const* q, const void* const* k_new,
+                                                  const void* const* v_new, void* const* cache_k,
+                                                  void* const* cache_v, const int32_t* pos0,
+                                                  const int32_t* n_new, int B, int S, int T, int Hq, int Hkv,
+                                                  int D, const float* d_table, uint32_t* d_status,
+                                                  cudaStream_t stream) {
+    if (!q || !k_new || !v_new || !cache_k || !cache_v || !pos0 || !n_new || !d_table)
+        return ARK_ERR_INVALID_ARG;
+    if (L <= 0) return ARK_ERR_INVALID_ARG;
+    if (L > ARK_MAX_LAYERS) return ARK_ERR_UNSUPPORTED;
+    ark_status st = check_common(B, S, T, Hq, Hkv, D);
+    if (st != ARK_OK) return st;
+    if (S > 65535) return ARK_ERR_UNSUPPORTED;
+    if (!aligned16(d_table)) return ARK_ERR_INVALID_ARG;
+    AppendParams prm{};
+    prm.pos0 = pos0;
+    prm.n_new = n_new;
+    prm.table = reinterpret_cast<const float2*>(d_table);
+    prm.status = d_status;
+    prm.B = B; prm.S = S; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
+    for (int l = 0; l < L; ++l) {
+        if (!q[l] || !k_new[l] || !v_new[l] || !cache_k[l] || !cache_v[l]) return ARK_ERR_INVALID_ARG;
+        if (!aligned16(q[l]) || !aligned16(k_new[l]) || !aligned16(v_new[l]) || !aligned16(cache_k[l]) ||
+            !aligned16(cache_v[l]))
+            return ARK_ERR_INVALID_ARG;
+        prm.layer[l] = AppendLayer{static_cast<uint16_t*>(q[l]), static_cast<const uint16_t*>(k_new[l]),
+                                   static_cast<const uint16_t*>(v_new[l]), static_cast<uint16_t*>(cache_k[l]),
+                                   static_cast<uint16_t*>(cache_v[l])};
+    }
+    return launch_append(prm, L, stream);
+}

@@ -1,5 +1,6 @@
-// decode.cu -- split-KV single-token GQA decode over a ragged batch, and the
-// log-sum-exp merge of its partial results.
+// decode.cu -- split-KV single-token GQA decode over a ragged batch, for one
+// layer or many independent layers in one launch, with a fused log-sum-exp
+// merge of the split partials; and the standalone merge kernel.
 //
 // The attention is the decoder's, over the static cache of the "ARK-ASR-3B --
 // INT8 ONNX" model card (section Shapes): 16 query heads, 2 KV heads, head dim
@@ -10,21 +11,27 @@
 // the invalid ones -inf) so the two can be timed side by side.
 //
 // Design (B200):
-//   - One CTA per (split, KV head g, request b, layer).  The 8 query heads of
-//     group g are served from a single read of each K/V row.
-//   - Each of the 4 warps owns a private 2-stage ring of 16-row K/V tiles in
-//     shared memory, filled by the TMA engine with 1-D bulk copies (one 256 B
-//     row per copy, completion counted on an mbarrier).  Rows are padded to
-//     272 B so that ldmatrix reads are bank-conflict free.
+//   - Work item = (layer, request b, KV head g, chunk of C rows).  Items are
+//     enumerated compactly on the device from kv_len (a prefix sum over the
+//     batch in shared memory), so no block is spent on rows past a request's
+//     length.  A persistent grid (a few CTAs per SM) walks the items; each
+//     WARP owns an item from start to end.  The 8 query heads of group g are
+//     served from a single read of each K/V row.
+//   - Each warp streams its item's 16-row K/V tiles through a private 2-stage
+//     ring in shared memory, filled by the TMA engine with 1-D bulk copies
+//     (one 256 B row per copy, completion counted on an mbarrier).  Rows are
+//     padded to 272 B so ldmatrix reads are bank-conflict free.
 //   - Scores are computed transposed, S^T[16 pos x 8 heads] = K_tile * Q^T,
 //     with m16n8k16 bf16 tensor-core MMAs: positions fill M = 16 and the 8
 //     heads of the group fill N = 8 exactly, so no MMA lane is wasted.  P^T is
 //     moved from the accumulator layout to the B-operand layout with two
 //     movmatrix transposes, and O^T[dims x heads] += V^T * P^T uses
-//     ldmatrix.trans on the same V tile.
-//   - fp32 online softmax in the log2 domain; per-head max across the 16
-//     positions by warp shuffles.  The four warps merge in shared memory;
-//     with one split the CTA writes o/lse directly, otherwise fp32 partials.
+//     ldmatrix.trans on the same V tile.  fp32 online softmax in the log2
+//     domain; per-head maxima across positions by warp shuffles.
+//   - An item that covers its whole sequence writes o/lse directly.  Split
+//     items write a normalised fp32 partial and bump a per-(layer, b, g)
+//     counter; the warp that arrives last merges the partials (they are still
+//     in L2) and resets the counter to zero.  No warp ever waits for another.
 //
 // Why tensor cores: per (position, KV head) the kernel reads 512 B and does
 // 2 x 8 x 128 multiply-adds, 4 FMA per byte.  At B200 HBM rates that needs
@@ -39,29 +46,27 @@ constexpr int kRowPitch = 272;                      // bytes per smem row (256 +
 constexpr int kTileRows = 16;
 constexpr int kTileBytes = kTileRows * kRowPitch;   // one 16-row K or V tile
 constexpr int kStageBytes = 2 * kTileBytes;         // K tile + V tile
-constexpr int kRingBytes = kWarps * kStages * kStageBytes;
-constexpr int kMergeBytes = kWarps * kGroup * kHeadDim * 4 + kWarps * kGroup * 2 * 4;
-static_assert(kMergeBytes <= kRingBytes, "merge area aliases the rings");
-constexpr int kDecodeSmem = kRingBytes + kWarps * kStages * 8 + 16;
-
-struct DecodeLayer {
-    const uint16_t* q;
-    const uint16_t* k;
-    const uint16_t* v;
-    uint16_t* o;
-    float* lse;
-    float* o_part;
-    float* lse_part;
-};
+constexpr int kWarpRing = kStages * kStageBytes;
+constexpr int kRingBytes = kWarps * kWarpRing;
+constexpr int kBarBytes = kWarps * kStages * 8;
+constexpr int kMaxBatch = 4096;
+static_assert(kGroup * kHeadDim * 4 <= kWarpRing, "per-warp output staging fits in the ring");
 
 struct DecodeParams {
     const int32_t* kv_len;
     uint32_t* status;
-    int B, T, Hq, Hkv;
-    int nsplit, chunk;
+    float* o_part;       // [L][B][Hq][nsplit][D]   (null when nsplit == 1)
+    float* lse_part;     // [L][B][Hq][nsplit]
+    int* counters;       // [L][B][Hkv]
+    int L, B, T, Hq, Hkv;
+    int chunk, nsplit;
     int masked;
     float scale_log2;
-    DecodeLayer layer[ARK_MAX_LAYERS];
+    const uint16_t* q[ARK_MAX_LAYERS];
+    const uint16_t* k[ARK_MAX_LAYERS];
+    const uint16_t* v[ARK_MAX_LAYERS];
+    uint16_t* o[ARK_MAX_LAYERS];
+    float* lse[ARK_MAX_LAYERS];
 };
 
 struct CombineLayer {
@@ -76,9 +81,9 @@ struct CombineParams {
     CombineLayer layer[ARK_MAX_LAYERS];
 };
 
-// Issue the bulk copies of one 16-row tile (rows r0 .. r0+nrows-1 of KV head
-// g of request b) into a stage; V rows past nrows are zeroed so that their
-// zero softmax weight cannot meet a NaN.
+// Issue the bulk copies of one 16-row tile (rows r0 .. r0+nrows-1) into a
+// stage; V rows past nrows are zeroed so that their zero softmax weight never
+// meets a NaN.
 __device__ __forceinline__ void issue_tile(uint8_t* stage, uint64_t* bar, const uint16_t* kbase,
                                            const uint16_t* vbase, int row_stride, int r0, int nrows,
                                            int lane) {
@@ -101,51 +106,40 @@ __device__ __forceinline__ void issue_tile(uint8_t* stage, uint64_t* bar, const 
     }
 }
 
-__global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(const __grid_constant__ DecodeParams p) {
+__device__ __forceinline__ int clamp_len(int x, int T) { return x < 0 ? 0 : (x > T ? T : x); }
+
+__global__ void __launch_bounds__(kWarps * 32) decode_kernel(const __grid_constant__ DecodeParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const int split = blockIdx.x;
-    const int g = blockIdx.y;
-    const int b = blockIdx.z % p.B;
-    const int l = blockIdx.z / p.B;
-    const DecodeLayer& L = p.layer[l];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int gid = lane >> 2;
     const int tig = lane & 3;
-
-    int kvl = __ldg(p.kv_len + b);
-    if (kvl < 0 || kvl > p.T) {
-        if (threadIdx.x == 0 && split == 0 && g == 0 && l == 0) report(p.status, ARK_DEV_BAD_KVLEN);
-        kvl = kvl < 0 ? 0 : p.T;
-    }
-    const int hi = p.masked ? p.T : kvl;          // rows read
-    const int j_begin = split * p.chunk;
-    const int j_end = min(j_begin + p.chunk, hi);
-    const int lim = min(kvl, j_end);                // rows scored
-    const int head0 = g * kGroup;
-
-    if (j_begin >= j_end) {
-        // no rows in this chunk: an empty partial (or, unsplit, o = 0 / lse = -inf)
-        if (threadIdx.x < kGroup) {
-            const int h = head0 + threadIdx.x;
-            if (p.nsplit == 1) {
-                L.lse[static_cast<size_t>(b) * p.Hq + h] = -INFINITY;
-            } else {
-                L.lse_part[(static_cast<size_t>(b) * p.Hq + h) * p.nsplit + split] = -INFINITY;
-            }
-        }
-        if (p.nsplit == 1) {
-            // o = 0 for the 8 heads: 8 x 128 bf16 = 128 x 16 B
-            uint4* o4 = reinterpret_cast<uint4*>(L.o + (static_cast<size_t>(b) * p.Hq + head0) * kHeadDim);
-            o4[threadIdx.x] = make_uint4(0, 0, 0, 0);
-        }
-        return;
-    }
-
-    uint8_t* ring = smem + warp * (kStages * kStageBytes);
+    uint8_t* ring = smem + warp * kWarpRing;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRingBytes) + warp * kStages;
-    int& s_failed = *reinterpret_cast<int*>(smem + kRingBytes + kWarps * kStages * 8);
-    if (threadIdx.x == 0) s_failed = 0;
+    int* s_pref = reinterpret_cast<int*>(smem + kRingBytes + kBarBytes);   // [B + 1]
+
+    // ---- per CTA: prefix over the batch of the number of items per request
+    if (warp == 0) {
+        if (lane == 0) s_pref[0] = 0;
+        int run = 0;
+        for (int base = 0; base < p.B; base += 32) {
+            const int b = base + lane;
+            int n = 0;
+            if (b < p.B) {
+                const int raw = __ldg(p.kv_len + b);
+                if ((raw < 0 || raw > p.T) && blockIdx.x == 0) report(p.status, ARK_DEV_BAD_KVLEN);
+                const int hi = p.masked ? p.T : clamp_len(raw, p.T);
+                n = max(1, (hi + p.chunk - 1) / p.chunk) * p.Hkv;
+            }
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, n, off);
+                if (lane >= off) n += y;
+            }
+            if (b < p.B) s_pref[b + 1] = run + n;
+            run += __shfl_sync(0xffffffffu, n, 31);
+        }
+    }
     if (lane == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
@@ -153,41 +147,9 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(const __grid_
     fence_proxy_async_smem();
     __syncthreads();
 
+    const int per_layer = s_pref[p.B];
+    const int total = per_layer * p.L;
     const int row_stride = p.Hkv * kHeadDim;
-    const uint16_t* kbase = L.k + static_cast<size_t>(b) * p.T * row_stride + g * kHeadDim;
-    const uint16_t* vbase = L.v + static_cast<size_t>(b) * p.T * row_stride + g * kHeadDim;
-
-    const int ntiles = (j_end - j_begin + kTileRows - 1) / kTileRows;
-    const int my_tiles = ntiles > warp ? (ntiles - warp + kWarps - 1) / kWarps : 0;
-
-    // prologue: fill the ring
-    for (int s = 0; s < kStages && s < my_tiles; ++s) {
-        const int r0 = j_begin + (warp + s * kWarps) * kTileRows;
-        issue_tile(ring + s * kStageBytes, &bars[s], kbase, vbase, row_stride, r0,
-                   min(kTileRows, j_end - r0), lane);
-    }
-
-    // Q of the 8 heads as B fragments: b0 = Q[head gid][16kk + 2tig .. +1], b1 = same + 8
-    uint32_t qf[8][2];
-    {
-        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-            L.q + (static_cast<size_t>(b) * p.Hq + head0 + gid) * kHeadDim);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            qf[kk][0] = __ldg(qrow + kk * 8 + tig);
-            qf[kk][1] = __ldg(qrow + kk * 8 + 4 + tig);
-        }
-    }
-
-    float acc[8][4];
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[mt][i] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY;   // running max of heads 2tig, 2tig+1 (log2 domain)
-    float l0 = 0.f, l1 = 0.f;               // this lane's share of the running sums
-
-    // ldmatrix lane roles
     const int lr = lane & 7;
     const int lm = lane >> 3;
     const uint32_t ring_u32 = smem_u32(ring);
@@ -195,168 +157,244 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(const __grid_
     const uint32_t k_off = (lr + 8 * (lm & 1)) * kRowPitch + 16 * (lm >> 1);
     // V (A operand of V^T, transposed load): matrix lm -> rows 8*(lm>>1), cols 8*(lm&1)
     const uint32_t v_off = kTileBytes + (lr + 8 * (lm >> 1)) * kRowPitch + 16 * (lm & 1);
+    uint32_t tile_seq = 0;    // tiles this warp has consumed so far (drives stage and parity)
 
-    bool failed = false;
-    int failed_at = 0;
-    for (int it = 0; it < my_tiles; ++it) {
-        const int s = it % kStages;
-        const uint32_t parity = (it / kStages) & 1;
-        if (!mbar_wait(&bars[s], parity)) {
-            failed = true;
-            failed_at = it;
-            break;
+    for (int item = blockIdx.x * kWarps + warp; item < total; item += gridDim.x * kWarps) {
+        // ---- decode the item
+        const int l = item / per_layer;
+        const int r = item - l * per_layer;
+        int lo = 0, hi_b = p.B - 1;           // largest b with s_pref[b] <= r
+        while (lo < hi_b) {
+            const int mid = (lo + hi_b + 1) >> 1;
+            if (s_pref[mid] <= r) lo = mid; else hi_b = mid - 1;
         }
-        __syncwarp();   // zero rows written by other lanes are visible from here on
-        const int r0 = j_begin + (warp + it * kWarps) * kTileRows;
-        const uint32_t st = ring_u32 + s * kStageBytes;
+        const int b = lo;
+        const int nch = (s_pref[b + 1] - s_pref[b]) / p.Hkv;
+        const int off = r - s_pref[b];
+        const int g = off / nch;
+        const int c = off - g * nch;
+        const int kvl = clamp_len(__ldg(p.kv_len + b), p.T);
+        const int hi = p.masked ? p.T : kvl;
+        const int j_begin = c * p.chunk;
+        const int j_end = min(j_begin + p.chunk, hi);
+        const int lim = min(kvl, j_end);
+        const int head0 = g * kGroup;
+        const int ntiles = j_end > j_begin ? (j_end - j_begin + kTileRows - 1) / kTileRows : 0;
 
-        float sc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(st + k_off + kk * 32, a0, a1, a2, a3);
-            mma_bf16_16816(sc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-        }
-        const bool v0 = (r0 + gid) < lim;
-        const bool v1 = (r0 + gid + 8) < lim;
-        sc[0] = v0 ? sc[0] * p.scale_log2 : -INFINITY;
-        sc[1] = v0 ? sc[1] * p.scale_log2 : -INFINITY;
-        sc[2] = v1 ? sc[2] * p.scale_log2 : -INFINITY;
-        sc[3] = v1 ? sc[3] * p.scale_log2 : -INFINITY;
+        const uint16_t* kbase = p.k[l] + static_cast<size_t>(b) * p.T * row_stride + g * kHeadDim;
+        const uint16_t* vbase = p.v[l] + static_cast<size_t>(b) * p.T * row_stride + g * kHeadDim;
 
-        float t0 = fmaxf(sc[0], sc[2]);
-        float t1 = fmaxf(sc[1], sc[3]);
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-            t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, off));
-            t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, off));
+        for (int s = 0; s < kStages && s < ntiles; ++s) {
+            const int r0 = j_begin + s * kTileRows;
+            issue_tile(ring + ((tile_seq + s) % kStages) * kStageBytes, &bars[(tile_seq + s) % kStages],
+                       kbase, vbase, row_stride, r0, min(kTileRows, j_end - r0), lane);
         }
-        const float n0 = fmaxf(m0, t0);
-        const float n1 = fmaxf(m1, t1);
-        const float u0 = (n0 == -INFINITY) ? 0.f : n0;
-        const float u1 = (n1 == -INFINITY) ? 0.f : n1;
-        const float alpha0 = fast_exp2(m0 - u0);
-        const float alpha1 = fast_exp2(m1 - u1);
-        m0 = n0;
-        m1 = n1;
 
-        const __nv_bfloat162 p01 = __floats2bfloat162_rn(fast_exp2(sc[0] - u0), fast_exp2(sc[1] - u1));
-        const __nv_bfloat162 p23 = __floats2bfloat162_rn(fast_exp2(sc[2] - u0), fast_exp2(sc[3] - u1));
-        // the sums use the same bf16-rounded weights that multiply V
-        l0 = l0 * alpha0 + __low2float(p01) + __low2float(p23);
-        l1 = l1 * alpha1 + __high2float(p01) + __high2float(p23);
+        // Q of the 8 heads as B fragments: b0 = Q[head gid][16kk + 2tig .. +1], b1 = same + 8
+        uint32_t qf[8][2];
+        {
+            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+                p.q[l] + (static_cast<size_t>(b) * p.Hq + head0 + gid) * kHeadDim);
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-            acc[mt][0] *= alpha0;
-            acc[mt][1] *= alpha1;
-            acc[mt][2] *= alpha0;
-            acc[mt][3] *= alpha1;
+            for (int kk = 0; kk < 8; ++kk) {
+                qf[kk][0] = __ldg(qrow + kk * 8 + tig);
+                qf[kk][1] = __ldg(qrow + kk * 8 + 4 + tig);
+            }
         }
-        const uint32_t pb0 = movmatrix_t(*reinterpret_cast<const uint32_t*>(&p01));
-        const uint32_t pb1 = movmatrix_t(*reinterpret_cast<const uint32_t*>(&p23));
+
+        float acc[8][4];
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(st + v_off + mt * 32, a0, a1, a2, a3);
-            mma_bf16_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[mt][i] = 0.f;
+        float m0 = -INFINITY, m1 = -INFINITY;   // running max of heads 2tig, 2tig+1 (log2 domain)
+        // this lane's share of the running sums: e* of the fp32 weights (for
+        // lse), r* of the bf16-rounded weights that multiply V (to normalise
+        // o, so that o stays an exact convex combination of V rows)
+        float e0 = 0.f, e1 = 0.f, r0s = 0.f, r1s = 0.f;
+        bool failed = false;
+
+        int issued = ntiles;      // tiles whose copies were issued (all, unless a wait gives up)
+        for (int t = 0; t < ntiles; ++t) {
+            const uint32_t seq = tile_seq + t;
+            const int s = seq % kStages;
+            if (!mbar_wait(&bars[s], (seq / kStages) & 1)) {
+                // give up on this item; drain what else is in flight (bounded)
+                issued = min(ntiles, t + kStages);
+                for (int t2 = t + 1; t2 < issued; ++t2) {
+                    const uint32_t q2 = tile_seq + t2;
+                    (void)mbar_wait(&bars[q2 % kStages], (q2 / kStages) & 1);
+                }
+                failed = true;
+                break;
+            }
+            __syncwarp();   // zero rows written by other lanes are visible from here on
+            const int r0 = j_begin + t * kTileRows;
+            const uint32_t st = ring_u32 + s * kStageBytes;
+
+            float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(st + k_off + kk * 32, a0, a1, a2, a3);
+                mma_bf16_16816(sc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+            }
+            const bool v0 = (r0 + gid) < lim;
+            const bool v1 = (r0 + gid + 8) < lim;
+            sc[0] = v0 ? sc[0] * p.scale_log2 : -INFINITY;
+            sc[1] = v0 ? sc[1] * p.scale_log2 : -INFINITY;
+            sc[2] = v1 ? sc[2] * p.scale_log2 : -INFINITY;
+            sc[3] = v1 ? sc[3] * p.scale_log2 : -INFINITY;
+
+            float t0 = fmaxf(sc[0], sc[2]);
+            float t1 = fmaxf(sc[1], sc[3]);
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, o));
+                t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, o));
+            }
+            const float n0 = fmaxf(m0, t0);
+            const float n1 = fmaxf(m1, t1);
+            const float u0 = (n0 == -INFINITY) ? 0.f : n0;
+            const float u1 = (n1 == -INFINITY) ? 0.f : n1;
+            const float alpha0 = fast_exp2(m0 - u0);
+            const float alpha1 = fast_exp2(m1 - u1);
+            m0 = n0;
+            m1 = n1;
+
+            const float p0 = fast_exp2(sc[0] - u0), p1 = fast_exp2(sc[1] - u1);
+            const float p2 = fast_exp2(sc[2] - u0), p3 = fast_exp2(sc[3] - u1);
+            const __nv_bfloat162 p01 = __floats2bfloat162_rn(p0, p1);
+            const __nv_bfloat162 p23 = __floats2bfloat162_rn(p2, p3);
+            e0 = e0 * alpha0 + (p0 + p2);
+            e1 = e1 * alpha1 + (p1 + p3);
+            r0s = r0s * alpha0 + (__low2float(p01) + __low2float(p23));
+            r1s = r1s * alpha1 + (__high2float(p01) + __high2float(p23));
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                acc[mt][0] *= alpha0;
+                acc[mt][1] *= alpha1;
+                acc[mt][2] *= alpha0;
+                acc[mt][3] *= alpha1;
+            }
+            const uint32_t pb0 = movmatrix_t(*reinterpret_cast<const uint32_t*>(&p01));
+            const uint32_t pb1 = movmatrix_t(*reinterpret_cast<const uint32_t*>(&p23));
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(st + v_off + mt * 32, a0, a1, a2, a3);
+                mma_bf16_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
+            }
+            __syncwarp();
+            if (t + kStages < ntiles) {
+                const int rn = j_begin + (t + kStages) * kTileRows;
+                issue_tile(ring + s * kStageBytes, &bars[s], kbase, vbase, row_stride, rn,
+                           min(kTileRows, j_end - rn), lane);
+            }
+        }
+        tile_seq += issued;
+        if (failed) {
+            if (lane == 0) report(p.status, ARK_DEV_TIMEOUT);
+            m0 = m1 = -INFINITY;   // publish an empty result so that counters stay consistent
+        }
+
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            e0 += __shfl_xor_sync(0xffffffffu, e0, o);
+            e1 += __shfl_xor_sync(0xffffffffu, e1, o);
+            r0s += __shfl_xor_sync(0xffffffffu, r0s, o);
+            r1s += __shfl_xor_sync(0xffffffffu, r1s, o);
+        }
+        const bool empty0 = (m0 == -INFINITY), empty1 = (m1 == -INFINITY);
+        const float inv0 = empty0 ? 0.f : 1.f / r0s;
+        const float inv1 = empty1 ? 0.f : 1.f / r1s;
+        const float lse0 = empty0 ? -INFINITY : (m0 + __log2f(e0)) * kLn2;
+        const float lse1 = empty1 ? -INFINITY : (m1 + __log2f(e1)) * kLn2;
+
+        // stage the normalised output [8 heads][128 dims] fp32 in this warp's ring
+        float* stg = reinterpret_cast<float*>(ring);
+        {
+            const int h0 = 2 * tig, h1 = 2 * tig + 1;
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                const int d = 16 * mt + gid;
+                stg[h0 * kHeadDim + d] = acc[mt][0] * inv0;
+                stg[h1 * kHeadDim + d] = acc[mt][1] * inv1;
+                stg[h0 * kHeadDim + d + 8] = acc[mt][2] * inv0;
+                stg[h1 * kHeadDim + d + 8] = acc[mt][3] * inv1;
+            }
         }
         __syncwarp();
-        if (it + kStages < my_tiles) {
-            const int rn = j_begin + (warp + (it + kStages) * kWarps) * kTileRows;
-            issue_tile(ring + s * kStageBytes, &bars[s], kbase, vbase, row_stride, rn,
-                       min(kTileRows, j_end - rn), lane);
-        }
-    }
-    if (failed) {
-        // Drain this warp's other copies in flight, with the same bound: tiles
-        // 0 .. issued-1 were issued; wait for the last one of each stage.
-        const int issued = min(my_tiles, failed_at + kStages);
-        for (int s = 0; s < kStages; ++s) {
-            int last = -1;
-            for (int i = s; i < issued; i += kStages) last = i;
-            if (last >= 0) (void)mbar_wait(&bars[s], static_cast<uint32_t>((last / kStages) & 1));
-        }
-        if (lane == 0) {
-            s_failed = 1;
-            report(p.status, ARK_DEV_TIMEOUT);
-        }
-    }
-
-    // full per-head sums of this warp
+        const size_t bh0 = static_cast<size_t>(b) * p.Hq + head0;    // row of head 0 of the group
+        if (nch == 1) {
+            // whole sequence in this item: write o (bf16) and lse
+            uint16_t* og = p.o[l] + bh0 * kHeadDim;
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-    }
-
-    __syncthreads();   // rings are free: reuse them as the merge area
-    float* o_s = reinterpret_cast<float*>(smem);                       // [warp][head][dim]
-    float* ml_s = o_s + kWarps * kGroup * kHeadDim;                    // [warp][head][2]
-    {
-        float* ow = o_s + warp * kGroup * kHeadDim;
-        const int h0 = 2 * tig, h1 = 2 * tig + 1;
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-            const int d = 16 * mt + gid;
-            ow[h0 * kHeadDim + d] = acc[mt][0];
-            ow[h1 * kHeadDim + d] = acc[mt][1];
-            ow[h0 * kHeadDim + d + 8] = acc[mt][2];
-            ow[h1 * kHeadDim + d + 8] = acc[mt][3];
-        }
-        if (gid == 0) {
-            float* mw = ml_s + warp * kGroup * 2;
-            mw[h0 * 2] = m0;  mw[h0 * 2 + 1] = l0;
-            mw[h1 * 2] = m1;  mw[h1 * 2 + 1] = l1;
-        }
-    }
-    __syncthreads();
-    if (s_failed) return;
-
-    {
-        const int h = threadIdx.x >> 4;          // 0..7
-        const int d0 = (threadIdx.x & 15) * 8;   // 8 dims per thread
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, ml_s[(w * kGroup + h) * 2]);
-        float e[kWarps];
-        float lsum = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const float mw = ml_s[(w * kGroup + h) * 2];
-            e[w] = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-            lsum += e[w] * ml_s[(w * kGroup + h) * 2 + 1];
-        }
-        float o[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            if (e[w] == 0.f) continue;
-            const float4* src = reinterpret_cast<const float4*>(o_s + (w * kGroup + h) * kHeadDim + d0);
-            const float4 x0 = src[0], x1 = src[1];
-            o[0] += e[w] * x0.x; o[1] += e[w] * x0.y; o[2] += e[w] * x0.z; o[3] += e[w] * x0.w;
-            o[4] += e[w] * x1.x; o[5] += e[w] * x1.y; o[6] += e[w] * x1.z; o[7] += e[w] * x1.w;
-        }
-        const bool empty = (M == -INFINITY);
-        const float inv = empty ? 0.f : 1.f / lsum;
-        const float lse = empty ? -INFINITY : (M + __log2f(lsum)) * kLn2;
-        const size_t bh = static_cast<size_t>(b) * p.Hq + head0 + h;
-        if (p.nsplit == 1) {
-            uint4 packed;
-            packed.x = pack_bf16x2(o[0] * inv, o[1] * inv);
-            packed.y = pack_bf16x2(o[2] * inv, o[3] * inv);
-            packed.z = pack_bf16x2(o[4] * inv, o[5] * inv);
-            packed.w = pack_bf16x2(o[6] * inv, o[7] * inv);
-            *reinterpret_cast<uint4*>(L.o + bh * kHeadDim + d0) = packed;
-            if ((threadIdx.x & 15) == 0) L.lse[bh] = lse;
-        } else {
-            if (!empty) {
-                float4* dst = reinterpret_cast<float4*>(L.o_part + (bh * p.nsplit + split) * kHeadDim + d0);
-                dst[0] = make_float4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
-                dst[1] = make_float4(o[4] * inv, o[5] * inv, o[6] * inv, o[7] * inv);
+            for (int i = 0; i < 4; ++i) {          // 8 heads x 128 dims = 4 x 32 lanes x 8 values
+                const int e = (i * 32 + lane) * 8;
+                const float4 x0 = *reinterpret_cast<const float4*>(stg + e);
+                const float4 x1 = *reinterpret_cast<const float4*>(stg + e + 4);
+                uint4 pk;
+                pk.x = pack_bf16x2(x0.x, x0.y);
+                pk.y = pack_bf16x2(x0.z, x0.w);
+                pk.z = pack_bf16x2(x1.x, x1.y);
+                pk.w = pack_bf16x2(x1.z, x1.w);
+                *reinterpret_cast<uint4*>(og + e) = pk;
             }
-            if ((threadIdx.x & 15) == 0) L.lse_part[bh * p.nsplit + split] = lse;
+            if (gid == 0) {
+                p.lse[l][bh0 + 2 * tig] = lse0;
+                p.lse[l][bh0 + 2 * tig + 1] = lse1;
+            }
+        } else {
+            const size_t lb = static_cast<size_t>(l) * p.B * p.Hq + bh0;   // (layer, b, head0) row
+            // partial: o_part[(lb + h) * nsplit + c][:], lse_part[(lb + h) * nsplit + c]
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) {
+                const float4 x = *reinterpret_cast<const float4*>(stg + h * kHeadDim + lane * 4);
+                *reinterpret_cast<float4*>(p.o_part + ((lb + h) * p.nsplit + c) * kHeadDim + lane * 4) = x;
+            }
+            if (gid == 0) {
+                p.lse_part[(lb + 2 * tig) * p.nsplit + c] = lse0;
+                p.lse_part[(lb + 2 * tig + 1) * p.nsplit + c] = lse1;
+            }
+            __threadfence();
+            __syncwarp();
+            int last = 0;
+            int* cnt = p.counters + (static_cast<size_t>(l) * p.B + b) * p.Hkv + g;
+            if (lane == 0) last = (atomicAdd(cnt, 1) == nch - 1);
+            last = __shfl_sync(0xffffffffu, last, 0);
+            if (last) {
+                __threadfence();
+                // merge the nch partials of the 8 heads; lane owns dims 4*lane .. 4*lane+3
+                for (int h = 0; h < kGroup; ++h) {
+                    const float* lp = p.lse_part + (lb + h) * p.nsplit;
+                    float M = -INFINITY;
+                    for (int cc = 0; cc < nch; ++cc) M = fmaxf(M, __ldcg(lp + cc));
+                    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+                    float wsum = 0.f;
+                    if (M != -INFINITY) {
+                        for (int cc = 0; cc < nch; ++cc) {
+                            const float lc = __ldcg(lp + cc);
+                            if (lc == -INFINITY) continue;
+                            const float w = fast_exp2((lc - M) * kLog2e);
+                            wsum += w;
+                            const float4 x = __ldcg(reinterpret_cast<const float4*>(
+                                p.o_part + ((lb + h) * p.nsplit + cc) * kHeadDim) + lane);
+                            a.x += w * x.x; a.y += w * x.y; a.z += w * x.z; a.w += w * x.w;
+                        }
+                    }
+                    const bool emp = (M == -INFINITY);
+                    const float iw = emp ? 0.f : 1.f / wsum;
+                    uint2 pk;
+                    pk.x = pack_bf16x2(a.x * iw, a.y * iw);
+                    pk.y = pack_bf16x2(a.z * iw, a.w * iw);
+                    reinterpret_cast<uint2*>(p.o[l] + (bh0 + h) * kHeadDim)[lane] = pk;
+                    if (lane == 0) p.lse[l][bh0 + h] = emp ? -INFINITY : M + __log2f(wsum) * kLn2;
+                }
+                if (lane == 0) atomicExch(cnt, 0);
+            }
         }
+        __syncwarp();   // the staging area is the ring of the next item
     }
 }
 
@@ -415,12 +453,19 @@ int decode_nsplit(int T, int max_splits) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-size_t part_o_bytes(int B, int Hq, int D, int nsplit) {
-    return align256(static_cast<size_t>(B) * Hq * nsplit * D * sizeof(float));
-}
+struct WsLayout {
+    size_t o_part, lse_part, counters, total;
+};
 
-size_t part_lse_bytes(int B, int Hq, int nsplit) {
-    return align256(static_cast<size_t>(B) * Hq * nsplit * sizeof(float));
+WsLayout ws_layout(int L, int B, int Hq, int Hkv, int D, int nsplit) {
+    WsLayout w{};
+    if (nsplit <= 1) return w;
+    const size_t rows = static_cast<size_t>(L) * B * Hq * nsplit;
+    w.o_part = 0;
+    w.lse_part = align256(rows * D * sizeof(float));
+    w.counters = w.lse_part + align256(rows * sizeof(float));
+    w.total = w.counters + align256(static_cast<size_t>(L) * B * Hkv * sizeof(int));
+    return w;
 }
 
 ark_status check_decode_shape(int B, int T, int Hq, int Hkv, int D) {
@@ -428,29 +473,89 @@ ark_status check_decode_shape(int B, int T, int Hq, int Hkv, int D) {
     if (Hq % Hkv != 0) return ARK_ERR_INVALID_ARG;
     if (T > ARK_MAX_T) return ARK_ERR_UNSUPPORTED;
     if (D != kHeadDim || Hq / Hkv != kGroup) return ARK_ERR_UNSUPPORTED;
-    if (static_cast<long long>(B) * ARK_MAX_LAYERS > 2147483647LL) return ARK_ERR_UNSUPPORTED;
+    if (B > kMaxBatch) return ARK_ERR_UNSUPPORTED;
     return ARK_OK;
 }
 
-bool g_decode_attr_set = false;
+size_t decode_smem(int B) { return kRingBytes + kBarBytes + align256((B + 1) * sizeof(int)); }
 
-ark_status ensure_decode_attr() {
-    if (!g_decode_attr_set) {
-        if (cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kDecodeSmem) != cudaSuccess)
+// SM count and resident CTAs per SM, queried once per device.
+struct DeviceInfo {
+    int sms = 0, ctas_per_sm = 0;
+};
+DeviceInfo g_dev[64];
+
+ark_status device_info(DeviceInfo& out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARK_ERR_CUDA;
+    DeviceInfo& d = g_dev[dev];
+    if (d.sms == 0) {
+        if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(decode_smem(kMaxBatch))) != cudaSuccess)
             return ARK_ERR_CUDA;
-        g_decode_attr_set = true;
+        int sms = 0, per = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ARK_ERR_CUDA;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_kernel, kWarps * 32, decode_smem(64)) !=
+            cudaSuccess)
+            return ARK_ERR_CUDA;
+        d.ctas_per_sm = per > 0 ? per : 1;
+        d.sms = sms;
     }
+    out = d;
+    return ARK_OK;
+}
+
+ark_status launch_decode(DecodeParams& prm, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    const WsLayout w = ws_layout(prm.L, prm.B, prm.Hq, prm.Hkv, kHeadDim, prm.nsplit);
+    if (w.total > 0) {
+        if (!workspace || ws_bytes < w.total || !aligned16(workspace)) return ARK_ERR_WORKSPACE;
+        uint8_t* base = static_cast<uint8_t*>(workspace);
+        prm.o_part = reinterpret_cast<float*>(base + w.o_part);
+        prm.lse_part = reinterpret_cast<float*>(base + w.lse_part);
+        prm.counters = reinterpret_cast<int*>(base + w.counters);
+    }
+    DeviceInfo d;
+    ark_status st = device_info(d);
+    if (st != ARK_OK) return st;
+    const long long max_items = static_cast<long long>(prm.L) * prm.B * prm.Hkv * prm.nsplit;
+    long long grid = static_cast<long long>(d.sms) * d.ctas_per_sm;
+    const long long need = (max_items + kWarps - 1) / kWarps;
+    if (need < grid) grid = need;
+    if (grid < 1) grid = 1;
+    decode_kernel<<<static_cast<unsigned>(grid), kWarps * 32, decode_smem(prm.B), stream>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
+}
+
+ark_status fill_common(DecodeParams& prm, const int32_t* kv_len, int L, int B, int T, int Hq, int Hkv, int D,
+                       float scale, ark_decode_mode mode, int max_splits, uint32_t* d_status) {
+    if (!kv_len) return ARK_ERR_INVALID_ARG;
+    ark_status st = check_decode_shape(B, T, Hq, Hkv, D);
+    if (st != ARK_OK) return st;
+    if (L <= 0) return ARK_ERR_INVALID_ARG;
+    if (L > ARK_MAX_LAYERS) return ARK_ERR_UNSUPPORTED;
+    if (max_splits <= 0 || !(scale > 0.f) || (mode != ARK_LENGTH_AWARE && mode != ARK_MASKED_STATIC))
+        return ARK_ERR_INVALID_ARG;
+    const long long items = static_cast<long long>(L) * B * Hkv * decode_nsplit(T, max_splits);
+    if (items > 2147483647LL / 2) return ARK_ERR_UNSUPPORTED;
+    prm.kv_len = kv_len;
+    prm.status = d_status;
+    prm.L = L; prm.B = B; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
+    prm.chunk = decode_chunk(T, max_splits);
+    prm.nsplit = decode_nsplit(T, max_splits);
+    prm.masked = (mode == ARK_MASKED_STATIC) ? 1 : 0;
+    prm.scale_log2 = scale * kLog2e;
     return ARK_OK;
 }
 
 }  // namespace
 
+extern "C" size_t ark_attn_decode_layers_workspace_size(int L, int B, int Hq, int D, int T, int max_splits) {
+    if (L <= 0 || B <= 0 || Hq <= 0 || D <= 0 || T <= 0 || max_splits <= 0 || Hq % kGroup) return 0;
+    return ws_layout(L, B, Hq, Hq / kGroup, D, decode_nsplit(T, max_splits)).total;
+}
+
 extern "C" size_t ark_attn_decode_workspace_size(int B, int Hq, int D, int T, int max_splits) {
-    if (B <= 0 || Hq <= 0 || D <= 0 || T <= 0 || max_splits <= 0) return 0;
-    const int nsplit = decode_nsplit(T, max_splits);
-    if (nsplit <= 1) return 0;
-    return part_o_bytes(B, Hq, D, nsplit) + part_lse_bytes(B, Hq, nsplit);
+    return ark_attn_decode_layers_workspace_size(1, B, Hq, D, T, max_splits);
 }
 
 extern "C" ark_status ark_attn_decode(const void* q, const void* cache_k, const void* cache_v,
@@ -458,49 +563,43 @@ extern "C" ark_status ark_attn_decode(const void* q, const void* cache_k, const 
                                       float scale, ark_decode_mode mode, int max_splits,
                                       void* workspace, size_t workspace_bytes,
                                       void* o, float* lse, uint32_t* d_status, cudaStream_t stream) {
-    if (!q || !cache_k || !cache_v || !kv_len || !o || !lse) return ARK_ERR_INVALID_ARG;
-    ark_status st = check_decode_shape(B, T, Hq, Hkv, D);
+    if (!q || !cache_k || !cache_v || !o || !lse) return ARK_ERR_INVALID_ARG;
+    DecodeParams prm{};
+    ark_status st = fill_common(prm, kv_len, 1, B, T, Hq, Hkv, D, scale, mode, max_splits, d_status);
     if (st != ARK_OK) return st;
-    if (max_splits <= 0 || !(scale > 0.f) || (mode != ARK_LENGTH_AWARE && mode != ARK_MASKED_STATIC))
-        return ARK_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(cache_k) || !aligned16(cache_v) || !aligned16(o) ||
         (reinterpret_cast<uintptr_t>(lse) & 3u))
         return ARK_ERR_INVALID_ARG;
-    const int chunk = decode_chunk(T, max_splits);
-    const int nsplit = (T + chunk - 1) / chunk;
-    const size_t need = ark_attn_decode_workspace_size(B, Hq, D, T, max_splits);
-    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return ARK_ERR_WORKSPACE;
-    if ((st = ensure_decode_attr()) != ARK_OK) return st;
+    prm.q[0] = static_cast<const uint16_t*>(q);
+    prm.k[0] = static_cast<const uint16_t*>(cache_k);
+    prm.v[0] = static_cast<const uint16_t*>(cache_v);
+    prm.o[0] = static_cast<uint16_t*>(o);
+    prm.lse[0] = lse;
+    return launch_decode(prm, workspace, workspace_bytes, stream);
+}
 
+extern "C" ark_status ark_attn_decode_layers(int L, const void* const* q, const void* const* cache_k,
+                                             const void* const* cache_v, const int32_t* kv_len, int B, int T,
+                                             int Hq, int Hkv, int D, float scale, ark_decode_mode mode,
+                                             int max_splits, void* workspace, size_t workspace_bytes,
+                                             void* const* o, float* const* lse, uint32_t* d_status,
+                                             cudaStream_t stream) {
+    if (!q || !cache_k || !cache_v || !o || !lse) return ARK_ERR_INVALID_ARG;
     DecodeParams prm{};
-    prm.kv_len = kv_len;
-    prm.status = d_status;
-    prm.B = B; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
-    prm.nsplit = nsplit;
-    prm.chunk = chunk;
-    prm.masked = (mode == ARK_MASKED_STATIC) ? 1 : 0;
-    prm.scale_log2 = scale * kLog2e;
-    float* o_part = nullptr;
-    float* lse_part = nullptr;
-    if (nsplit > 1) {
-        o_part = static_cast<float*>(workspace);
-        lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + part_o_bytes(B, Hq, D, nsplit));
+    ark_status st = fill_common(prm, kv_len, L, B, T, Hq, Hkv, D, scale, mode, max_splits, d_status);
+    if (st != ARK_OK) return st;
+    for (int l = 0; l < L; ++l) {
+        if (!q[l] || !cache_k[l] || !cache_v[l] || !o[l] || !lse[l]) return ARK_ERR_INVALID_ARG;
+        if (!aligned16(q[l]) || !aligned16(cache_k[l]) || !aligned16(cache_v[l]) || !aligned16(o[l]) ||
+            (reinterpret_cast<uintptr_t>(lse[l]) & 3u))
+            return ARK_ERR_INVALID_ARG;
+        prm.q[l] = static_cast<const uint16_t*>(q[l]);
+        prm.k[l] = static_cast<const uint16_t*>(cache_k[l]);
+        prm.v[l] = static_cast<const uint16_t*>(cache_v[l]);
+        prm.o[l] = static_cast<uint16_t*>(o[l]);
+        prm.lse[l] = lse[l];
     }
-    prm.layer[0] = DecodeLayer{static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(cache_k),
-                               static_cast<const uint16_t*>(cache_v), static_cast<uint16_t*>(o), lse,
-                               o_part, lse_part};
-    dim3 grid(nsplit, Hkv, B);
-    decode_split_kernel<<<grid, kWarps * 32, kDecodeSmem, stream>>>(prm);
-    if (cudaGetLastError() != cudaSuccess) return ARK_ERR_CUDA;
-    if (nsplit > 1) {
-        CombineParams cp{};
-        cp.B = B; cp.Hq = Hq; cp.nsplit = nsplit;
-        cp.layer[0] = CombineLayer{o_part, lse_part, static_cast<uint16_t*>(o), lse};
-        dim3 cgrid((B * Hq + 3) / 4, 1);
-        combine_kernel<<<cgrid, 128, 0, stream>>>(cp);
-        if (cudaGetLastError() != cudaSuccess) return ARK_ERR_CUDA;
-    }
-    return ARK_OK;
+    return launch_decode(prm, workspace, workspace_bytes, stream);
 }
 
 extern "C" ark_status ark_attn_combine(const float* o_part, const float* lse_part, int B, int Hq,

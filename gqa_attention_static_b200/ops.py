@@ -42,6 +42,9 @@ EXPORTS = (
     "ark_attn_decode_workspace_size",
     "ark_attn_decode",
     "ark_attn_combine",
+    "ark_attn_append_rope_layers",
+    "ark_attn_decode_layers_workspace_size",
+    "ark_attn_decode_layers",
 )
 
 
@@ -78,6 +81,14 @@ def load() -> ctypes.CDLL:
     lib.ark_attn_decode.restype = I
     lib.ark_attn_combine.argtypes = [P, P, I, I, I, I, P, P, P]
     lib.ark_attn_combine.restype = I
+    PP = ctypes.POINTER(ctypes.c_void_p)
+    lib.ark_attn_append_rope_layers.argtypes = [I, PP, PP, PP, PP, PP, P, P, I, I, I, I, I, I, P, P, P]
+    lib.ark_attn_append_rope_layers.restype = I
+    lib.ark_attn_decode_layers_workspace_size.argtypes = [I, I, I, I, I, I]
+    lib.ark_attn_decode_layers_workspace_size.restype = Z
+    lib.ark_attn_decode_layers.argtypes = [I, PP, PP, PP, P, I, I, I, I, I, ctypes.c_float, I, I, P, Z,
+                                           PP, PP, P, P]
+    lib.ark_attn_decode_layers.restype = I
     _lib = lib
     return lib
 
@@ -200,9 +211,11 @@ def ark_attn_decode(q, cache_k, cache_v, kv_len, o, lse, scale: float, mode: int
            "ark_attn_decode")
 
 
-def decode_workspace(B: int, Hq: int, D: int, T: int, max_splits: int, device="cuda"):
-    n = ark_attn_decode_workspace_size(B, Hq, D, T, max_splits)
-    return torch.empty(max(n, 16), dtype=torch.uint8, device=device) if n else None
+def decode_workspace(B: int, Hq: int, D: int, T: int, max_splits: int, device="cuda", layers: int = 1):
+    """Zero-filled decode workspace (its counters must start at zero), or None
+    when the call needs none."""
+    n = ark_attn_decode_layers_workspace_size(layers, B, Hq, D, T, max_splits)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device) if n else None
 
 
 # --------------------------------------------------------------- combine ----
@@ -220,3 +233,83 @@ def ark_attn_combine(o_part, lse_part, o, lse, stream=None) -> None:
     _raise(load().ark_attn_combine(_ptr(o_part), _ptr(lse_part), B, Hq, nsplit, D, _ptr(o), _ptr(lse),
                                    _stream(stream)),
            "ark_attn_combine")
+
+
+# ------------------------------------------------- layer-batched variants ----
+
+def _ptr_array(ts: Sequence[torch.Tensor]):
+    arr = (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+    return arr
+
+
+def ark_attn_append_rope_layers(q: Sequence[torch.Tensor], k_new, v_new, cache_k, cache_v, pos0, n_new, table,
+                                status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """ark_attn_append_rope over L independent layers in one launch (lists of
+    per-layer tensors, same shapes as the single-layer call)."""
+    L = len(q)
+    if not (len(k_new) == len(v_new) == len(cache_k) == len(cache_v) == L) or L == 0:
+        raise ValueError("per-layer lists must have the same non-zero length")
+    for i in range(L):
+        for name, t in (("q", q[i]), ("k_new", k_new[i]), ("v_new", v_new[i]), ("cache_k", cache_k[i]),
+                        ("cache_v", cache_v[i])):
+            _need(t, name, torch.bfloat16, 4)
+        if q[i].shape != q[0].shape or cache_k[i].shape != cache_k[0].shape or \
+                k_new[i].shape != k_new[0].shape or v_new[i].shape != k_new[0].shape or \
+                cache_v[i].shape != cache_k[0].shape:
+            raise ValueError("all layers must have the same shapes")
+    _need(pos0, "pos0", torch.int32, 1)
+    _need(n_new, "n_new", torch.int32, 1)
+    _need(table, "table", torch.float32)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    B, S, Hq, D = q[0].shape
+    T, Hkv = cache_k[0].shape[1], cache_k[0].shape[2]
+    if tuple(k_new[0].shape) != (B, S, Hkv, D) or cache_k[0].shape[0] != B:
+        raise ValueError("shapes")
+    if table.numel() < T * (D // 2) * 2:
+        raise ValueError("rotary table has fewer than T rows")
+    _raise(load().ark_attn_append_rope_layers(L, _ptr_array(q), _ptr_array(k_new), _ptr_array(v_new),
+                                              _ptr_array(cache_k), _ptr_array(cache_v), _ptr(pos0),
+                                              _ptr(n_new), B, S, T, Hq, Hkv, D, _ptr(table), _ptr(status),
+                                              _stream(stream)),
+           "ark_attn_append_rope_layers")
+
+
+def ark_attn_decode_layers_workspace_size(L: int, B: int, Hq: int, D: int, T: int, max_splits: int) -> int:
+    return int(load().ark_attn_decode_layers_workspace_size(L, B, Hq, D, T, max_splits))
+
+
+def ark_attn_decode_layers(q: Sequence[torch.Tensor], cache_k, cache_v, kv_len, o, lse, scale: float,
+                           mode: int = ARK_LENGTH_AWARE, max_splits: int = 8,
+                           workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                           stream=None) -> None:
+    """ark_attn_decode over L independent layers in one launch."""
+    L = len(q)
+    if not (len(cache_k) == len(cache_v) == len(o) == len(lse) == L) or L == 0:
+        raise ValueError("per-layer lists must have the same non-zero length")
+    for i in range(L):
+        _need(q[i], "q", torch.bfloat16, 4)
+        _need(cache_k[i], "cache_k", torch.bfloat16, 4)
+        _need(cache_v[i], "cache_v", torch.bfloat16, 4)
+        _need(o[i], "o", torch.bfloat16, 4)
+        _need(lse[i], "lse", torch.float32)
+        if q[i].shape != q[0].shape or cache_k[i].shape != cache_k[0].shape or \
+                cache_v[i].shape != cache_k[0].shape or o[i].shape != q[0].shape or \
+                lse[i].numel() != q[0].shape[0] * q[0].shape[2]:
+            raise ValueError("all layers must have the same shapes")
+    _need(kv_len, "kv_len", torch.int32, 1)
+    B, S, Hq, D = q[0].shape
+    if S != 1:
+        raise ValueError("decode takes one query row per request")
+    T, Hkv = cache_k[0].shape[1], cache_k[0].shape[2]
+    ws_bytes = 0
+    if workspace is not None:
+        _need(workspace, "workspace", workspace.dtype)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    if status is not None:
+        _need(status, "status", torch.int32)
+    _raise(load().ark_attn_decode_layers(L, _ptr_array(q), _ptr_array(cache_k), _ptr_array(cache_v), _ptr(kv_len),
+                                         B, T, Hq, Hkv, D, float(scale), int(mode), int(max_splits),
+                                         _ptr(workspace), ws_bytes, _ptr_array(o), _ptr_array(lse), _ptr(status),
+                                         _stream(stream)),
+           "ark_attn_decode_layers")

@@ -1,11 +1,15 @@
 """Host-side plumbing for one decode step over L independent layers.
 
 A decode step is, per layer: RoPE on the new q/k rows and the delta write into
-that layer's static cache (``ark_attn_append_rope``), then split-KV decode
-attention over the valid rows (``ark_attn_decode``, which runs the
-log-sum-exp merge when it splits).  All launches go to one CUDA stream; the
-step can be captured in a CUDA graph.  This module only owns buffers and
-orders calls -- every step of the computation is a libarkattn kernel.
+that layer's static cache, then split-KV decode attention over the valid rows
+with its log-sum-exp merge.  ``batched=True`` issues both for all layers at
+once (``ark_attn_append_rope_layers`` + ``ark_attn_decode_layers``: two
+launches per step); ``batched=False`` issues the single-layer calls layer by
+layer (``ark_attn_append_rope`` + ``ark_attn_decode``: two launches per
+layer), the way a decoder that runs its layers one after another would.  All
+launches go to one CUDA stream; the step can be captured in a CUDA graph.
+This module only owns buffers and orders calls -- every step of the
+computation is a libarkattn kernel.
 """
 from __future__ import annotations
 
@@ -30,7 +34,7 @@ class DecodeStep:
                  cache_k: List[torch.Tensor], cache_v: List[torch.Tensor], pos0: torch.Tensor,
                  n_new: torch.Tensor, kv_len: torch.Tensor, max_splits: int = 8,
                  mode: int = ops.ARK_LENGTH_AWARE, rope_theta: float = 1e6,
-                 scale: Optional[float] = None):
+                 scale: Optional[float] = None, batched: bool = True):
         self.q, self.k_new, self.v_new = q, k_new, v_new
         self.cache_k, self.cache_v = cache_k, cache_v
         self.pos0, self.n_new, self.kv_len = pos0, n_new, kv_len
@@ -41,38 +45,50 @@ class DecodeStep:
         dev = q[0].device
         self.max_splits = max_splits
         self.mode = mode
+        self.batched = batched
         self.scale = scale if scale is not None else 1.0 / math.sqrt(self.D)
         self.table = ops.rope_table(self.T, self.D, rope_theta, device=dev)
-        self.workspace = ops.decode_workspace(self.B, self.Hq, self.D, self.T, max_splits, device=dev)
+        self.workspace = ops.decode_workspace(self.B, self.Hq, self.D, self.T, max_splits, device=dev,
+                                              layers=self.layers if batched else 1)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.o = [torch.empty_like(x) for x in q]
         self.lse = [torch.empty(self.B, self.Hq, dtype=torch.float32, device=dev) for _ in q]
 
     @property
     def nsplit(self) -> int:
-        ws = ops.ark_attn_decode_workspace_size(self.B, self.Hq, self.D, self.T, self.max_splits)
-        if ws == 0:
-            return 1
         per = -(-self.T // self.max_splits)
         chunk = max(64, -(-per // 16) * 16)
         return -(-self.T // chunk)
 
     def launches_per_step(self) -> int:
-        return self.layers * (2 + (1 if self.nsplit > 1 else 0))
+        return 2 if self.batched else 2 * self.layers
+
+    def append(self, stream=None) -> None:
+        if self.batched:
+            ops.ark_attn_append_rope_layers(self.q, self.k_new, self.v_new, self.cache_k, self.cache_v,
+                                            self.pos0, self.n_new, self.table, self.status, stream)
+        else:
+            for l in range(self.layers):
+                ops.ark_attn_append_rope(self.q[l], self.k_new[l], self.v_new[l], self.cache_k[l],
+                                         self.cache_v[l], self.pos0, self.n_new, self.table, self.status,
+                                         stream)
+
+    def attention(self, stream=None) -> None:
+        if self.batched:
+            ops.ark_attn_decode_layers(self.q, self.cache_k, self.cache_v, self.kv_len, self.o, self.lse,
+                                       self.scale, self.mode, self.max_splits, self.workspace, self.status,
+                                       stream)
+        else:
+            for l in range(self.layers):
+                ops.ark_attn_decode(self.q[l], self.cache_k[l], self.cache_v[l], self.kv_len, self.o[l],
+                                    self.lse[l], self.scale, self.mode, self.max_splits, self.workspace,
+                                    self.status, stream)
 
     def run(self, stream=None) -> None:
-        for l in range(self.layers):
-            ops.ark_attn_append_rope(self.q[l], self.k_new[l], self.v_new[l], self.cache_k[l],
-                                     self.cache_v[l], self.pos0, self.n_new, self.table, self.status,
-                                     stream)
-            ops.ark_attn_decode(self.q[l], self.cache_k[l], self.cache_v[l], self.kv_len, self.o[l],
-                                self.lse[l], self.scale, self.mode, self.max_splits, self.workspace,
-                                self.status, stream)
+        self.append(stream)
+        self.attention(stream)
 
     def attention_only(self, stream=None) -> None:
         """The decode attention of every layer without the append (for timing
         the dominant kernel alone)."""
-        for l in range(self.layers):
-            ops.ark_attn_decode(self.q[l], self.cache_k[l], self.cache_v[l], self.kv_len, self.o[l],
-                                self.lse[l], self.scale, self.mode, self.max_splits, self.workspace,
-                                self.status, stream)
+        self.attention(stream)

@@ -30,7 +30,7 @@
  *     status word `*d_status` (device memory, uint32).  The caller reads the
  *     word after synchronising.  `d_status` may be NULL to skip reporting.
  *   - Only D = 128 and Hq/Hkv = 8 are instantiated (ARK_ERR_UNSUPPORTED
- *     otherwise); T <= ARK_MAX_T.
+ *     otherwise); T <= ARK_MAX_T; decode takes B <= 4096.
  *   - A launch failure returns ARK_ERR_CUDA; the CUDA error is left to the
  *     caller (cudaGetLastError).
  */
@@ -129,25 +129,59 @@ ARK_API ark_status ark_attn_append_rope(void* q, const void* k_new, const void* 
  * kv_len[b] valid cache rows of its KV head g = h / (Hq/Hkv):
  *   s_j = scale * <q[b,0,h,:], cache_k[b,j,g,:]>,  j < kv_len[b]
  *   o[b,0,h,:] = sum_j softmax(s)_j cache_v[b,j,g,:],   lse[b,h] = ln sum_j exp(s_j)
- * All 8 query heads of a KV group are served from one read of each K/V row.
- * The key range is split into chunks of equal length processed in parallel;
- * with more than one chunk the partial results go to `workspace` and a
- * log-sum-exp merge (the kernel behind ark_attn_combine) writes o and lse.
+ * ("ARK-ASR-3B -- INT8 ONNX", section Shapes: 16 heads share 2 KV heads over
+ * the static cache.)  All 8 query heads of a KV group are served from one read
+ * of each K/V row.  Each request's rows are cut into chunks of C rows
+ * (C = max(64, T / max_splits rounded up to 16)); chunks run in parallel and,
+ * when a request has more than one, their fp32 partial results go to
+ * `workspace` and are merged by log-sum-exp inside the same launch (the last
+ * chunk to finish merges).
  * Layouts: q [B,1,Hq,D] bf16; cache_k, cache_v [B,T,Hkv,D] bf16; kv_len
  * int32[B] (device; the new row is already appended, so the query attends to
  * itself); o [B,1,Hq,D] bf16; lse [B,Hq] fp32 (natural log).
  * kv_len outside [0, T] is clamped and sets ARK_DEV_BAD_KVLEN; kv_len = 0
  * gives o = 0, lse = -inf.
- * max_splits >= 1 bounds the number of chunks; workspace may be NULL when
- * ark_attn_decode_workspace_size(...) returns 0.  Accumulation is fp32 from
- * bf16 operands on the tensor cores; P is rounded to bf16 before P.V.
+ * Workspace: ark_attn_decode_workspace_size(...) bytes (0 when T fits one
+ * chunk; then `workspace` may be NULL), 16-byte aligned, caller-owned.  It
+ * holds the partials and one counter per (request, KV head); the counters
+ * MUST be zero before the first call (zero-fill the whole workspace once after
+ * allocating it); every call leaves them at zero again.  Calls that run
+ * concurrently must not share a workspace.
+ * Numerics: bf16 operands on the tensor cores with fp32 accumulation; the
+ * softmax weights are rounded to bf16 before they multiply V, o is normalised
+ * by the sum of those rounded weights and lse uses the fp32 weights.
  */
 ARK_API size_t ark_attn_decode_workspace_size(int B, int Hq, int D, int T, int max_splits);
 ARK_API ark_status ark_attn_decode(const void* q, const void* cache_k, const void* cache_v,
-                           const int32_t* kv_len, int B, int T, int Hq, int Hkv, int D,
-                           float scale, ark_decode_mode mode, int max_splits,
-                           void* workspace, size_t workspace_bytes,
-                           void* o, float* lse, uint32_t* d_status, cudaStream_t stream);
+                                   const int32_t* kv_len, int B, int T, int Hq, int Hkv, int D,
+                                   float scale, ark_decode_mode mode, int max_splits,
+                                   void* workspace, size_t workspace_bytes,
+                                   void* o, float* lse, uint32_t* d_status, cudaStream_t stream);
+
+/* -------------------------------------------------- layer-batched variants ----
+ * The same operations over L <= ARK_MAX_LAYERS independent layers in ONE
+ * launch.  Every pointer argument that is per layer is a HOST array of L
+ * device pointers (read during the call; the array itself may be freed when
+ * the call returns).  All layers share B, S, T, the positions/lengths and the
+ * rotary table.  Each layer's tensors follow the single-layer layouts above.
+ * The decode workspace is ark_attn_decode_layers_workspace_size(L, ...) bytes
+ * with the same zero-before-first-use rule.  Meant for callers that hold
+ * several independent caches (the ARK-ASR-3B decoder has 36 layers), and for
+ * measuring the kernels without per-launch overhead.
+ */
+ARK_API ark_status ark_attn_append_rope_layers(int L, void* const* q, const void* const* k_new,
+                                               const void* const* v_new, void* const* cache_k,
+                                               void* const* cache_v, const int32_t* pos0,
+                                               const int32_t* n_new, int B, int S, int T, int Hq,
+                                               int Hkv, int D, const float* d_table,
+                                               uint32_t* d_status, cudaStream_t stream);
+ARK_API size_t ark_attn_decode_layers_workspace_size(int L, int B, int Hq, int D, int T, int max_splits);
+ARK_API ark_status ark_attn_decode_layers(int L, const void* const* q, const void* const* cache_k,
+                                          const void* const* cache_v, const int32_t* kv_len, int B,
+                                          int T, int Hq, int Hkv, int D, float scale,
+                                          ark_decode_mode mode, int max_splits, void* workspace,
+                                          size_t workspace_bytes, void* const* o, float* const* lse,
+                                          uint32_t* d_status, cudaStream_t stream);
 
 /* --------------------------------------------------------------- combine ----
  * Log-sum-exp merge of nsplit partial results of the same query over

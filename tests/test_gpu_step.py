@@ -20,7 +20,7 @@ SCALE = 1.0 / math.sqrt(128)
 BENCH_MAX_SPLITS = 8
 
 
-def run_step(batch, mode=ops.ARK_LENGTH_AWARE, max_splits=BENCH_MAX_SPLITS):
+def run_step(batch, mode=ops.ARK_LENGTH_AWARE, max_splits=BENCH_MAX_SPLITS, batched=True):
     dev = "cuda"
     q = [x.to(dev).clone() for x in batch.q]
     kn = [x.to(dev) for x in batch.k_new]
@@ -28,7 +28,7 @@ def run_step(batch, mode=ops.ARK_LENGTH_AWARE, max_splits=BENCH_MAX_SPLITS):
     ck = [x.to(dev).clone() for x in batch.cache_k]
     cv = [x.to(dev).clone() for x in batch.cache_v]
     step = DecodeStep(q, kn, vn, ck, cv, batch.pos0.to(dev), batch.n_new.to(dev), batch.kv_len.to(dev),
-                      max_splits=max_splits, mode=mode)
+                      max_splits=max_splits, mode=mode, batched=batched)
     step.run()
     torch.cuda.synchronize()
     return step
@@ -55,19 +55,38 @@ def compare(step, batch, layers):
         check_lse(f64(step.lse[l]), lse_ref, f"lse layer {l}")
 
 
-def test_step_single_decode_36_layers(oracle_lib):
+@pytest.mark.parametrize("batched", [True, False])
+def test_step_single_decode_36_layers(oracle_lib, batched):
     """Batch 1, 36 layers, 64 valid rows + the new row at position 64."""
     batch = W.cfg_single_decode()
-    step = run_step(batch)
+    step = run_step(batch, batched=batched)
     compare(step, batch, range(36))
 
 
-def test_step_ragged_batch_full_size(oracle_lib):
+@pytest.mark.parametrize("batched", [True, False])
+def test_step_ragged_batch_full_size(oracle_lib, batched):
     """Ragged batch of 32, 36 layers, T = 512: the benchmark's workload at its
-    full size, every output compared."""
+    full size and launch configuration, every output compared."""
     batch = W.cfg_ragged_decode()
-    step = run_step(batch)
+    step = run_step(batch, batched=batched)
     compare(step, batch, range(36))
+
+
+def test_step_repeated_calls_reuse_workspace(oracle_lib):
+    """The merge counters return to zero after every call: the same workspace
+    serves consecutive steps (here: the same step three times, with q restored)."""
+    batch = W.cfg_ragged_decode(layers=3, seed=21)
+    step = run_step(batch)
+    o1 = [x.clone() for x in step.o]
+    for _ in range(2):
+        for l in range(3):
+            step.q[l].copy_(batch.q[l].cuda())
+        step.run()
+    torch.cuda.synchronize()
+    for l in range(3):
+        assert torch.equal(step.o[l], o1[l])
+    ws = step.workspace
+    assert ws is not None
 
 
 def test_step_ragged_batch_masked_static(oracle_lib):
@@ -78,10 +97,11 @@ def test_step_ragged_batch_masked_static(oracle_lib):
 
 @pytest.mark.parametrize("T", [2048, 1024])
 @pytest.mark.parametrize("mode", [ops.ARK_LENGTH_AWARE, ops.ARK_MASKED_STATIC])
-def test_step_long_cache(oracle_lib, T, mode):
+@pytest.mark.parametrize("max_splits", [8, 32])
+def test_step_long_cache(oracle_lib, T, mode, max_splits):
     """T = 2048 with 1501..2048 rows read, and T = 1024 full (1024 rows)."""
     batch = W.cfg_long_decode(layers=2, T=T)
-    step = run_step(batch, mode=mode)
+    step = run_step(batch, mode=mode, max_splits=max_splits)
     compare(step, batch, range(2))
 
 
