@@ -400,7 +400,7 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": desc, "batch": B, "max_total_len": T, "layers": L,
                        "mode": "masked-static" if args.mode == "masked" else "length-aware",
-                       "max_splits": args.max_splits, "nsplit": step.nsplit,
+                       "max_splits": args.max_splits, "min_tiles_per_warp": step.min_tiles,
                        "l2": "inputs larger than L2 (%.0f MB of caches streamed per step)" %
                              (2 * L * B * T * 2 * 128 * 2 / 1e6),
                        "parallelism": f"replicas x{world}",

@@ -11,16 +11,21 @@
 // the invalid ones -inf) so the two can be timed side by side.
 //
 // Design (B200):
-//   - Work item = (layer, request b, KV head g, chunk of C rows).  Items are
-//     enumerated compactly on the device from kv_len (a prefix sum over the
-//     batch in shared memory), so no block is spent on rows past a request's
-//     length.  A persistent grid (a few CTAs per SM) walks the items; each
-//     WARP owns an item from start to end.  The 8 query heads of group g are
-//     served from a single read of each K/V row.
-//   - Each warp streams its item's 16-row K/V tiles through a private 2-stage
-//     ring in shared memory, filled by the TMA engine with 1-D bulk copies
-//     (one 256 B row per copy, completion counted on an mbarrier).  Rows are
-//     padded to 272 B so ldmatrix reads are bank-conflict free.
+//   - The work is a list of 16-row K/V tiles: segment (layer l, request b, KV
+//     head g) holds ceil(rows/16) tiles, where rows = kv_len[b] (length-aware)
+//     or T (masked).  The list is enumerated on the device from kv_len with a
+//     prefix sum over the batch in shared memory, so nothing is spent on rows
+//     past a request's length.
+//   - A persistent grid (a few CTAs per SM) splits the list into one
+//     contiguous range of tiles per WARP, equal to within one tile, so every
+//     warp streams the same number of bytes whatever the length mix.  A range
+//     may start or end inside a segment; that is the split-KV cut.
+//   - Each warp streams its range through a private 2-stage ring in shared
+//     memory, filled by the TMA engine with 1-D bulk copies (one 256 B row
+//     per copy, completion counted on an mbarrier), and keeps streaming
+//     across segment boundaries.  Rows are padded to 272 B so ldmatrix reads
+//     are bank-conflict free.  The 8 query heads of group g are served from a
+//     single read of each K/V row.
 //   - Scores are computed transposed, S^T[16 pos x 8 heads] = K_tile * Q^T,
 //     with m16n8k16 bf16 tensor-core MMAs: positions fill M = 16 and the 8
 //     heads of the group fill N = 8 exactly, so no MMA lane is wasted.  P^T is
@@ -28,10 +33,11 @@
 //     movmatrix transposes, and O^T[dims x heads] += V^T * P^T uses
 //     ldmatrix.trans on the same V tile.  fp32 online softmax in the log2
 //     domain; per-head maxima across positions by warp shuffles.
-//   - An item that covers its whole sequence writes o/lse directly.  Split
-//     items write a normalised fp32 partial and bump a per-(layer, b, g)
-//     counter; the warp that arrives last merges the partials (they are still
-//     in L2) and resets the counter to zero.  No warp ever waits for another.
+//   - A warp that covers a whole segment writes o/lse directly.  A cut
+//     segment's pieces write normalised fp32 partials (at most two per warp)
+//     and bump a per-segment counter; the warp that arrives last merges the
+//     pieces by log-sum-exp (they are still in L2) and resets the counter to
+//     zero.  No warp ever waits for another.
 //
 // Why tensor cores: per (position, KV head) the kernel reads 512 B and does
 // 2 x 8 x 128 multiply-adds, 4 FMA per byte.  At B200 HBM rates that needs
@@ -50,16 +56,16 @@ constexpr int kWarpRing = kStages * kStageBytes;
 constexpr int kRingBytes = kWarps * kWarpRing;
 constexpr int kBarBytes = kWarps * kStages * 8;
 constexpr int kMaxBatch = 4096;
-static_assert(kGroup * kHeadDim * 4 <= kWarpRing, "per-warp output staging fits in the ring");
+constexpr int kMaxWarps = 2048;                     // upper bound on warps per launch (sizes the partials)
 
 struct DecodeParams {
     const int32_t* kv_len;
     uint32_t* status;
-    float* o_part;       // [L][B][Hq][nsplit][D]   (null when nsplit == 1)
-    float* lse_part;     // [L][B][Hq][nsplit]
+    float* part_o;       // [kMaxWarps][2][8][D]  two partial slots per warp
+    float* part_lse;     // [kMaxWarps][2][8]
     int* counters;       // [L][B][Hkv]
     int L, B, T, Hq, Hkv;
-    int chunk, nsplit;
+    int min_tiles;       // fewest tiles one warp takes (bounds the pieces per segment)
     int masked;
     float scale_log2;
     const uint16_t* q[ARK_MAX_LAYERS];
@@ -83,7 +89,8 @@ struct CombineParams {
 
 // Issue the bulk copies of one 16-row tile (rows r0 .. r0+nrows-1) into a
 // stage; V rows past nrows are zeroed so that their zero softmax weight never
-// meets a NaN.
+// meets a NaN.  nrows may be 0 (an empty request): the phase then completes
+// on the arrival alone.
 __device__ __forceinline__ void issue_tile(uint8_t* stage, uint64_t* bar, const uint16_t* kbase,
                                            const uint16_t* vbase, int row_stride, int r0, int nrows,
                                            int lane) {
@@ -108,7 +115,36 @@ __device__ __forceinline__ void issue_tile(uint8_t* stage, uint64_t* bar, const 
 
 __device__ __forceinline__ int clamp_len(int x, int T) { return x < 0 ? 0 : (x > T ? T : x); }
 
-__global__ void __launch_bounds__(kWarps * 32) decode_kernel(const __grid_constant__ DecodeParams p) {
+// One segment = (layer, request, KV head): its tiles are s0 .. s0+n-1 of the
+// global tile list.
+struct Seg {
+    long long s0;
+    int l, b, g, n, kvl, hi;
+};
+
+// Segment of global tile t, and t's index j inside it.
+__device__ __forceinline__ Seg locate(long long t, const int* s_pref, int per_layer, const DecodeParams& p,
+                                      int& j) {
+    Seg s;
+    s.l = static_cast<int>(t / per_layer);
+    const int r = static_cast<int>(t - static_cast<long long>(s.l) * per_layer);
+    int lo = 0, hi = p.B - 1;                // largest b with s_pref[b] <= r
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_pref[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    s.b = lo;
+    s.n = (s_pref[lo + 1] - s_pref[lo]) / p.Hkv;
+    const int off = r - s_pref[lo];
+    s.g = off / s.n;
+    j = off - s.g * s.n;
+    s.s0 = t - j;
+    s.kvl = clamp_len(__ldg(p.kv_len + s.b), p.T);
+    s.hi = p.masked ? p.T : s.kvl;
+    return s;
+}
+
+__global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_constant__ DecodeParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -118,7 +154,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const __grid_consta
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRingBytes) + warp * kStages;
     int* s_pref = reinterpret_cast<int*>(smem + kRingBytes + kBarBytes);   // [B + 1]
 
-    // ---- per CTA: prefix over the batch of the number of items per request
+    // ---- per CTA: prefix over the batch of the tiles per request (all KV heads)
     if (warp == 0) {
         if (lane == 0) s_pref[0] = 0;
         int run = 0;
@@ -129,7 +165,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const __grid_consta
                 const int raw = __ldg(p.kv_len + b);
                 if ((raw < 0 || raw > p.T) && blockIdx.x == 0) report(p.status, ARK_DEV_BAD_KVLEN);
                 const int hi = p.masked ? p.T : clamp_len(raw, p.T);
-                n = max(1, (hi + p.chunk - 1) / p.chunk) * p.Hkv;
+                n = max(1, (hi + kTileRows - 1) / kTileRows) * p.Hkv;
             }
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -145,10 +181,18 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const __grid_consta
         fence_mbar_init();
     }
     fence_proxy_async_smem();
-    __syncthreads();
+    __syncthreads();   // the last block-wide barrier: warps run independently from here
 
     const int per_layer = s_pref[p.B];
-    const int total = per_layer * p.L;
+    const long long N = static_cast<long long>(per_layer) * p.L;
+    long long W = N / p.min_tiles;
+    if (W < 1) W = 1;
+    if (W > static_cast<long long>(gridDim.x) * kWarps) W = static_cast<long long>(gridDim.x) * kWarps;
+    const int w = blockIdx.x * kWarps + warp;
+    if (w >= W) return;
+    const long long T0 = static_cast<long long>(w) * N / W;
+    const long long T1 = static_cast<long long>(w + 1) * N / W;
+
     const int row_stride = p.Hkv * kHeadDim;
     const int lr = lane & 7;
     const int lm = lane >> 3;
@@ -157,81 +201,64 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const __grid_consta
     const uint32_t k_off = (lr + 8 * (lm & 1)) * kRowPitch + 16 * (lm >> 1);
     // V (A operand of V^T, transposed load): matrix lm -> rows 8*(lm>>1), cols 8*(lm&1)
     const uint32_t v_off = kTileBytes + (lr + 8 * (lm >> 1)) * kRowPitch + 16 * (lm & 1);
-    uint32_t tile_seq = 0;    // tiles this warp has consumed so far (drives stage and parity)
 
-    for (int item = blockIdx.x * kWarps + warp; item < total; item += gridDim.x * kWarps) {
-        // ---- decode the item
-        const int l = item / per_layer;
-        const int r = item - l * per_layer;
-        int lo = 0, hi_b = p.B - 1;           // largest b with s_pref[b] <= r
-        while (lo < hi_b) {
-            const int mid = (lo + hi_b + 1) >> 1;
-            if (s_pref[mid] <= r) lo = mid; else hi_b = mid - 1;
-        }
-        const int b = lo;
-        const int nch = (s_pref[b + 1] - s_pref[b]) / p.Hkv;
-        const int off = r - s_pref[b];
-        const int g = off / nch;
-        const int c = off - g * nch;
-        const int kvl = clamp_len(__ldg(p.kv_len + b), p.T);
-        const int hi = p.masked ? p.T : kvl;
-        const int j_begin = c * p.chunk;
-        const int j_end = min(j_begin + p.chunk, hi);
-        const int lim = min(kvl, j_end);
-        const int head0 = g * kGroup;
-        const int ntiles = j_end > j_begin ? (j_end - j_begin + kTileRows - 1) / kTileRows : 0;
+    // ---- producer cursor: next tile to issue
+    long long tp = T0;
+    int pj;
+    Seg ps = locate(T0, s_pref, per_layer, p, pj);
+    uint32_t pseq = 0;
+    auto issue_next = [&]() {
+        const int r0 = pj * kTileRows;
+        const int nrows = max(0, min(kTileRows, ps.hi - r0));
+        const uint16_t* kb = p.k[ps.l] + static_cast<size_t>(ps.b) * p.T * row_stride + ps.g * kHeadDim;
+        const uint16_t* vb = p.v[ps.l] + static_cast<size_t>(ps.b) * p.T * row_stride + ps.g * kHeadDim;
+        const int st = pseq % kStages;
+        issue_tile(ring + st * kStageBytes, &bars[st], kb, vb, row_stride, r0, nrows, lane);
+        ++pseq;
+        ++tp;
+        if (++pj == ps.n && tp < T1) ps = locate(tp, s_pref, per_layer, p, pj);
+    };
+    for (int s = 0; s < kStages && tp < T1; ++s) issue_next();
 
-        const uint16_t* kbase = p.k[l] + static_cast<size_t>(b) * p.T * row_stride + g * kHeadDim;
-        const uint16_t* vbase = p.v[l] + static_cast<size_t>(b) * p.T * row_stride + g * kHeadDim;
-
-        for (int s = 0; s < kStages && s < ntiles; ++s) {
-            const int r0 = j_begin + s * kTileRows;
-            issue_tile(ring + ((tile_seq + s) % kStages) * kStageBytes, &bars[(tile_seq + s) % kStages],
-                       kbase, vbase, row_stride, r0, min(kTileRows, j_end - r0), lane);
-        }
-
+    // ---- consumer cursor
+    int cj;
+    Seg cs = locate(T0, s_pref, per_layer, p, cj);
+    uint32_t qf[8][2];
+    float acc[8][4];
+    float m0, m1, e0, e1, r0s, r1s;
+    auto begin_segment = [&]() {
         // Q of the 8 heads as B fragments: b0 = Q[head gid][16kk + 2tig .. +1], b1 = same + 8
-        uint32_t qf[8][2];
-        {
-            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-                p.q[l] + (static_cast<size_t>(b) * p.Hq + head0 + gid) * kHeadDim);
+        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+            p.q[cs.l] + (static_cast<size_t>(cs.b) * p.Hq + cs.g * kGroup + gid) * kHeadDim);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                qf[kk][0] = __ldg(qrow + kk * 8 + tig);
-                qf[kk][1] = __ldg(qrow + kk * 8 + 4 + tig);
-            }
+        for (int kk = 0; kk < 8; ++kk) {
+            qf[kk][0] = __ldg(qrow + kk * 8 + tig);
+            qf[kk][1] = __ldg(qrow + kk * 8 + 4 + tig);
         }
-
-        float acc[8][4];
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[mt][i] = 0.f;
-        float m0 = -INFINITY, m1 = -INFINITY;   // running max of heads 2tig, 2tig+1 (log2 domain)
+        m0 = m1 = -INFINITY;   // running max of heads 2tig, 2tig+1 (log2 domain)
         // this lane's share of the running sums: e* of the fp32 weights (for
         // lse), r* of the bf16-rounded weights that multiply V (to normalise
         // o, so that o stays an exact convex combination of V rows)
-        float e0 = 0.f, e1 = 0.f, r0s = 0.f, r1s = 0.f;
-        bool failed = false;
+        e0 = e1 = r0s = r1s = 0.f;
+    };
+    begin_segment();
 
-        int issued = ntiles;      // tiles whose copies were issued (all, unless a wait gives up)
-        for (int t = 0; t < ntiles; ++t) {
-            const uint32_t seq = tile_seq + t;
-            const int s = seq % kStages;
-            if (!mbar_wait(&bars[s], (seq / kStages) & 1)) {
-                // give up on this item; drain what else is in flight (bounded)
-                issued = min(ntiles, t + kStages);
-                for (int t2 = t + 1; t2 < issued; ++t2) {
-                    const uint32_t q2 = tile_seq + t2;
-                    (void)mbar_wait(&bars[q2 % kStages], (q2 / kStages) & 1);
-                }
-                failed = true;
-                break;
-            }
-            __syncwarp();   // zero rows written by other lanes are visible from here on
-            const int r0 = j_begin + t * kTileRows;
+    bool failed = false;
+    for (long long t = T0; t < T1; ++t) {
+        const uint32_t seq = static_cast<uint32_t>(t - T0);
+        const int s = seq % kStages;
+        if (!failed && !mbar_wait(&bars[s], (seq / kStages) & 1)) {
+            failed = true;
+            if (lane == 0) report(p.status, ARK_DEV_TIMEOUT);
+        }
+        __syncwarp();   // zero rows written by other lanes are visible from here on
+        if (!failed) {
+            const int r0 = cj * kTileRows;
             const uint32_t st = ring_u32 + s * kStageBytes;
-
             float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
@@ -239,8 +266,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const __grid_consta
                 ldsm_x4(st + k_off + kk * 32, a0, a1, a2, a3);
                 mma_bf16_16816(sc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
             }
-            const bool v0 = (r0 + gid) < lim;
-            const bool v1 = (r0 + gid + 8) < lim;
+            const bool v0 = (r0 + gid) < cs.kvl;
+            const bool v1 = (r0 + gid + 8) < cs.kvl;
             sc[0] = v0 ? sc[0] * p.scale_log2 : -INFINITY;
             sc[1] = v0 ? sc[1] * p.scale_log2 : -INFINITY;
             sc[2] = v1 ? sc[2] * p.scale_log2 : -INFINITY;
@@ -286,18 +313,13 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const __grid_consta
                 mma_bf16_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
             }
             __syncwarp();
-            if (t + kStages < ntiles) {
-                const int rn = j_begin + (t + kStages) * kTileRows;
-                issue_tile(ring + s * kStageBytes, &bars[s], kbase, vbase, row_stride, rn,
-                           min(kTileRows, j_end - rn), lane);
-            }
-        }
-        tile_seq += issued;
-        if (failed) {
-            if (lane == 0) report(p.status, ARK_DEV_TIMEOUT);
-            m0 = m1 = -INFINITY;   // publish an empty result so that counters stay consistent
+            if (tp < T1) issue_next();     // refill the stage just consumed
         }
 
+        if (++cj < cs.n && t + 1 < T1) continue;
+
+        // ---- the consumer leaves segment cs: publish its result
+        if (failed) m0 = m1 = -INFINITY;   // an empty result keeps the merge counters consistent
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
             e0 += __shfl_xor_sync(0xffffffffu, e0, o);
@@ -310,77 +332,70 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const __grid_consta
         const float inv1 = empty1 ? 0.f : 1.f / r1s;
         const float lse0 = empty0 ? -INFINITY : (m0 + __log2f(e0)) * kLn2;
         const float lse1 = empty1 ? -INFINITY : (m1 + __log2f(e1)) * kLn2;
-
-        // stage the normalised output [8 heads][128 dims] fp32 in this warp's ring
-        float* stg = reinterpret_cast<float*>(ring);
-        {
-            const int h0 = 2 * tig, h1 = 2 * tig + 1;
+        const int h0 = 2 * tig, h1 = 2 * tig + 1;
+        const size_t bh0 = static_cast<size_t>(cs.b) * p.Hq + cs.g * kGroup;   // row of the group's head 0
+        const bool whole = (cs.s0 >= T0) && (cs.s0 + cs.n <= T1);
+        if (whole) {
+            uint16_t* og = p.o[cs.l] + bh0 * kHeadDim;
+            __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(og);
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 const int d = 16 * mt + gid;
-                stg[h0 * kHeadDim + d] = acc[mt][0] * inv0;
-                stg[h1 * kHeadDim + d] = acc[mt][1] * inv1;
-                stg[h0 * kHeadDim + d + 8] = acc[mt][2] * inv0;
-                stg[h1 * kHeadDim + d + 8] = acc[mt][3] * inv1;
-            }
-        }
-        __syncwarp();
-        const size_t bh0 = static_cast<size_t>(b) * p.Hq + head0;    // row of head 0 of the group
-        if (nch == 1) {
-            // whole sequence in this item: write o (bf16) and lse
-            uint16_t* og = p.o[l] + bh0 * kHeadDim;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {          // 8 heads x 128 dims = 4 x 32 lanes x 8 values
-                const int e = (i * 32 + lane) * 8;
-                const float4 x0 = *reinterpret_cast<const float4*>(stg + e);
-                const float4 x1 = *reinterpret_cast<const float4*>(stg + e + 4);
-                uint4 pk;
-                pk.x = pack_bf16x2(x0.x, x0.y);
-                pk.y = pack_bf16x2(x0.z, x0.w);
-                pk.z = pack_bf16x2(x1.x, x1.y);
-                pk.w = pack_bf16x2(x1.z, x1.w);
-                *reinterpret_cast<uint4*>(og + e) = pk;
+                ob[h0 * kHeadDim + d] = __float2bfloat16_rn(acc[mt][0] * inv0);
+                ob[h1 * kHeadDim + d] = __float2bfloat16_rn(acc[mt][1] * inv1);
+                ob[h0 * kHeadDim + d + 8] = __float2bfloat16_rn(acc[mt][2] * inv0);
+                ob[h1 * kHeadDim + d + 8] = __float2bfloat16_rn(acc[mt][3] * inv1);
             }
             if (gid == 0) {
-                p.lse[l][bh0 + 2 * tig] = lse0;
-                p.lse[l][bh0 + 2 * tig + 1] = lse1;
+                p.lse[cs.l][bh0 + h0] = lse0;
+                p.lse[cs.l][bh0 + h1] = lse1;
             }
         } else {
-            const size_t lb = static_cast<size_t>(l) * p.B * p.Hq + bh0;   // (layer, b, head0) row
-            // partial: o_part[(lb + h) * nsplit + c][:], lse_part[(lb + h) * nsplit + c]
+            const int slot = (cs.s0 < T0) ? 0 : 1;
+            float* po = p.part_o + (static_cast<size_t>(w) * 2 + slot) * kGroup * kHeadDim;
 #pragma unroll
-            for (int h = 0; h < kGroup; ++h) {
-                const float4 x = *reinterpret_cast<const float4*>(stg + h * kHeadDim + lane * 4);
-                *reinterpret_cast<float4*>(p.o_part + ((lb + h) * p.nsplit + c) * kHeadDim + lane * 4) = x;
+            for (int mt = 0; mt < 8; ++mt) {
+                const int d = 16 * mt + gid;
+                po[h0 * kHeadDim + d] = acc[mt][0] * inv0;
+                po[h1 * kHeadDim + d] = acc[mt][1] * inv1;
+                po[h0 * kHeadDim + d + 8] = acc[mt][2] * inv0;
+                po[h1 * kHeadDim + d + 8] = acc[mt][3] * inv1;
             }
             if (gid == 0) {
-                p.lse_part[(lb + 2 * tig) * p.nsplit + c] = lse0;
-                p.lse_part[(lb + 2 * tig + 1) * p.nsplit + c] = lse1;
+                p.part_lse[(static_cast<size_t>(w) * 2 + slot) * kGroup + h0] = lse0;
+                p.part_lse[(static_cast<size_t>(w) * 2 + slot) * kGroup + h1] = lse1;
             }
+            // warps whose ranges meet this segment: wa .. wb
+            const long long last_tile = cs.s0 + cs.n - 1;
+            const int wa = static_cast<int>(((cs.s0 + 1) * W - 1) / N);
+            const int wb = static_cast<int>(((last_tile + 1) * W - 1) / N);
             __threadfence();
             __syncwarp();
             int last = 0;
-            int* cnt = p.counters + (static_cast<size_t>(l) * p.B + b) * p.Hkv + g;
-            if (lane == 0) last = (atomicAdd(cnt, 1) == nch - 1);
+            int* cnt = p.counters + (static_cast<size_t>(cs.l) * p.B + cs.b) * p.Hkv + cs.g;
+            if (lane == 0) last = (atomicAdd(cnt, 1) == wb - wa);
             last = __shfl_sync(0xffffffffu, last, 0);
             if (last) {
                 __threadfence();
-                // merge the nch partials of the 8 heads; lane owns dims 4*lane .. 4*lane+3
+                // merge the pieces of the 8 heads; lane owns dims 4*lane .. 4*lane+3
                 for (int h = 0; h < kGroup; ++h) {
-                    const float* lp = p.lse_part + (lb + h) * p.nsplit;
                     float M = -INFINITY;
-                    for (int cc = 0; cc < nch; ++cc) M = fmaxf(M, __ldcg(lp + cc));
+                    for (int wi = wa; wi <= wb; ++wi) {
+                        const int sl = (cs.s0 < static_cast<long long>(wi) * N / W) ? 0 : 1;
+                        M = fmaxf(M, __ldcg(p.part_lse + (static_cast<size_t>(wi) * 2 + sl) * kGroup + h));
+                    }
                     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
                     float wsum = 0.f;
                     if (M != -INFINITY) {
-                        for (int cc = 0; cc < nch; ++cc) {
-                            const float lc = __ldcg(lp + cc);
+                        for (int wi = wa; wi <= wb; ++wi) {
+                            const int sl = (cs.s0 < static_cast<long long>(wi) * N / W) ? 0 : 1;
+                            const size_t row = (static_cast<size_t>(wi) * 2 + sl) * kGroup + h;
+                            const float lc = __ldcg(p.part_lse + row);
                             if (lc == -INFINITY) continue;
-                            const float w = fast_exp2((lc - M) * kLog2e);
-                            wsum += w;
-                            const float4 x = __ldcg(reinterpret_cast<const float4*>(
-                                p.o_part + ((lb + h) * p.nsplit + cc) * kHeadDim) + lane);
-                            a.x += w * x.x; a.y += w * x.y; a.z += w * x.z; a.w += w * x.w;
+                            const float wgt = fast_exp2((lc - M) * kLog2e);
+                            wsum += wgt;
+                            const float4 x = __ldcg(reinterpret_cast<const float4*>(p.part_o + row * kHeadDim) + lane);
+                            a.x += wgt * x.x; a.y += wgt * x.y; a.z += wgt * x.z; a.w += wgt * x.w;
                         }
                     }
                     const bool emp = (M == -INFINITY);
@@ -388,13 +403,22 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const __grid_consta
                     uint2 pk;
                     pk.x = pack_bf16x2(a.x * iw, a.y * iw);
                     pk.y = pack_bf16x2(a.z * iw, a.w * iw);
-                    reinterpret_cast<uint2*>(p.o[l] + (bh0 + h) * kHeadDim)[lane] = pk;
-                    if (lane == 0) p.lse[l][bh0 + h] = emp ? -INFINITY : M + __log2f(wsum) * kLn2;
+                    reinterpret_cast<uint2*>(p.o[cs.l] + (bh0 + h) * kHeadDim)[lane] = pk;
+                    if (lane == 0) p.lse[cs.l][bh0 + h] = emp ? -INFINITY : M + __log2f(wsum) * kLn2;
                 }
                 if (lane == 0) atomicExch(cnt, 0);
             }
         }
-        __syncwarp();   // the staging area is the ring of the next item
+        if (t + 1 < T1) {
+            cs = locate(t + 1, s_pref, per_layer, p, cj);
+            begin_segment();
+        }
+    }
+    // Never leave with copies in flight: a timed-out warp stops consuming, so
+    // wait (bounded) for the tiles it issued but did not consume.
+    if (failed) {
+        for (uint32_t q2 = pseq > kStages ? pseq - kStages : 0; q2 < pseq; ++q2)
+            (void)mbar_wait(&bars[q2 % kStages], (q2 / kStages) & 1);
     }
 }
 
@@ -439,31 +463,25 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int decode_chunk(int T, int max_splits) {
-    const int per = (T + max_splits - 1) / max_splits;
-    int chunk = ((per + kTileRows - 1) / kTileRows) * kTileRows;
-    if (chunk < 64) chunk = 64;
-    return chunk;
-}
-
-int decode_nsplit(int T, int max_splits) {
-    const int chunk = decode_chunk(T, max_splits);
-    return (T + chunk - 1) / chunk;
+// Fewest 16-row tiles one warp takes: a (request, KV head) of up to
+// ceil(T/16) tiles is then cut into at most max_splits + 1 pieces.
+int decode_min_tiles(int T, int max_splits) {
+    const int tiles = (T + kTileRows - 1) / kTileRows;
+    int m = (tiles + max_splits - 1) / max_splits;
+    return m < 1 ? 1 : m;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct WsLayout {
-    size_t o_part, lse_part, counters, total;
+    size_t part_o, part_lse, counters, total;
 };
 
-WsLayout ws_layout(int L, int B, int Hq, int Hkv, int D, int nsplit) {
+WsLayout ws_layout(int L, int B, int Hkv) {
     WsLayout w{};
-    if (nsplit <= 1) return w;
-    const size_t rows = static_cast<size_t>(L) * B * Hq * nsplit;
-    w.o_part = 0;
-    w.lse_part = align256(rows * D * sizeof(float));
-    w.counters = w.lse_part + align256(rows * sizeof(float));
+    w.part_o = 0;
+    w.part_lse = align256(static_cast<size_t>(kMaxWarps) * 2 * kGroup * kHeadDim * sizeof(float));
+    w.counters = w.part_lse + align256(static_cast<size_t>(kMaxWarps) * 2 * kGroup * sizeof(float));
     w.total = w.counters + align256(static_cast<size_t>(L) * B * Hkv * sizeof(int));
     return w;
 }
@@ -506,21 +524,22 @@ ark_status device_info(DeviceInfo& out) {
 }
 
 ark_status launch_decode(DecodeParams& prm, void* workspace, size_t ws_bytes, cudaStream_t stream) {
-    const WsLayout w = ws_layout(prm.L, prm.B, prm.Hq, prm.Hkv, kHeadDim, prm.nsplit);
-    if (w.total > 0) {
-        if (!workspace || ws_bytes < w.total || !aligned16(workspace)) return ARK_ERR_WORKSPACE;
-        uint8_t* base = static_cast<uint8_t*>(workspace);
-        prm.o_part = reinterpret_cast<float*>(base + w.o_part);
-        prm.lse_part = reinterpret_cast<float*>(base + w.lse_part);
-        prm.counters = reinterpret_cast<int*>(base + w.counters);
-    }
+    const WsLayout w = ws_layout(prm.L, prm.B, prm.Hkv);
+    if (!workspace || ws_bytes < w.total || !aligned16(workspace)) return ARK_ERR_WORKSPACE;
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    prm.part_o = reinterpret_cast<float*>(base + w.part_o);
+    prm.part_lse = reinterpret_cast<float*>(base + w.part_lse);
+    prm.counters = reinterpret_cast<int*>(base + w.counters);
     DeviceInfo d;
     ark_status st = device_info(d);
     if (st != ARK_OK) return st;
-    const long long max_items = static_cast<long long>(prm.L) * prm.B * prm.Hkv * prm.nsplit;
+    // tiles in the largest case the device lengths can produce
+    const long long max_tiles =
+        static_cast<long long>(prm.L) * prm.B * prm.Hkv * ((prm.T + kTileRows - 1) / kTileRows);
     long long grid = static_cast<long long>(d.sms) * d.ctas_per_sm;
-    const long long need = (max_items + kWarps - 1) / kWarps;
+    const long long need = (max_tiles / prm.min_tiles + kWarps - 1) / kWarps;
     if (need < grid) grid = need;
+    if (grid > kMaxWarps / kWarps) grid = kMaxWarps / kWarps;
     if (grid < 1) grid = 1;
     decode_kernel<<<static_cast<unsigned>(grid), kWarps * 32, decode_smem(prm.B), stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
@@ -535,13 +554,10 @@ ark_status fill_common(DecodeParams& prm, const int32_t* kv_len, int L, int B, i
     if (L > ARK_MAX_LAYERS) return ARK_ERR_UNSUPPORTED;
     if (max_splits <= 0 || !(scale > 0.f) || (mode != ARK_LENGTH_AWARE && mode != ARK_MASKED_STATIC))
         return ARK_ERR_INVALID_ARG;
-    const long long items = static_cast<long long>(L) * B * Hkv * decode_nsplit(T, max_splits);
-    if (items > 2147483647LL / 2) return ARK_ERR_UNSUPPORTED;
     prm.kv_len = kv_len;
     prm.status = d_status;
     prm.L = L; prm.B = B; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
-    prm.chunk = decode_chunk(T, max_splits);
-    prm.nsplit = decode_nsplit(T, max_splits);
+    prm.min_tiles = decode_min_tiles(T, max_splits);
     prm.masked = (mode == ARK_MASKED_STATIC) ? 1 : 0;
     prm.scale_log2 = scale * kLog2e;
     return ARK_OK;
@@ -551,7 +567,7 @@ ark_status fill_common(DecodeParams& prm, const int32_t* kv_len, int L, int B, i
 
 extern "C" size_t ark_attn_decode_layers_workspace_size(int L, int B, int Hq, int D, int T, int max_splits) {
     if (L <= 0 || B <= 0 || Hq <= 0 || D <= 0 || T <= 0 || max_splits <= 0 || Hq % kGroup) return 0;
-    return ws_layout(L, B, Hq, Hq / kGroup, D, decode_nsplit(T, max_splits)).total;
+    return ws_layout(L, B, Hq / kGroup).total;
 }
 
 extern "C" size_t ark_attn_decode_workspace_size(int B, int Hq, int D, int T, int max_splits) {

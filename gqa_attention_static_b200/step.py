@@ -55,10 +55,10 @@ class DecodeStep:
         self.lse = [torch.empty(self.B, self.Hq, dtype=torch.float32, device=dev) for _ in q]
 
     @property
-    def nsplit(self) -> int:
-        per = -(-self.T // self.max_splits)
-        chunk = max(64, -(-per // 16) * 16)
-        return -(-self.T // chunk)
+    def min_tiles(self) -> int:
+        """Fewest 16-row tiles one warp takes (the library's split bound)."""
+        tiles = -(-self.T // 16)
+        return max(1, -(-tiles // self.max_splits))
 
     def launches_per_step(self) -> int:
         return 2 if self.batched else 2 * self.layers

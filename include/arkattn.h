@@ -131,22 +131,24 @@ ARK_API ark_status ark_attn_append_rope(void* q, const void* k_new, const void* 
  *   o[b,0,h,:] = sum_j softmax(s)_j cache_v[b,j,g,:],   lse[b,h] = ln sum_j exp(s_j)
  * ("ARK-ASR-3B -- INT8 ONNX", section Shapes: 16 heads share 2 KV heads over
  * the static cache.)  All 8 query heads of a KV group are served from one read
- * of each K/V row.  Each request's rows are cut into chunks of C rows
- * (C = max(64, T / max_splits rounded up to 16)); chunks run in parallel and,
- * when a request has more than one, their fp32 partial results go to
- * `workspace` and are merged by log-sum-exp inside the same launch (the last
- * chunk to finish merges).
+ * of each K/V row.  The rows of all (request, KV head) pairs form one list of
+ * 16-row tiles that the GPU's warps split into equal contiguous ranges, so a
+ * request's rows may be cut into pieces processed in parallel; every warp
+ * takes at least ceil(ceil(T/16) / max_splits) tiles, so one (request, KV
+ * head) is cut into at most max_splits + 1 pieces.  Cut pieces leave fp32
+ * partial results in `workspace` and are merged by log-sum-exp inside the
+ * same launch (the last piece to finish merges).
  * Layouts: q [B,1,Hq,D] bf16; cache_k, cache_v [B,T,Hkv,D] bf16; kv_len
  * int32[B] (device; the new row is already appended, so the query attends to
  * itself); o [B,1,Hq,D] bf16; lse [B,Hq] fp32 (natural log).
  * kv_len outside [0, T] is clamped and sets ARK_DEV_BAD_KVLEN; kv_len = 0
  * gives o = 0, lse = -inf.
- * Workspace: ark_attn_decode_workspace_size(...) bytes (0 when T fits one
- * chunk; then `workspace` may be NULL), 16-byte aligned, caller-owned.  It
- * holds the partials and one counter per (request, KV head); the counters
- * MUST be zero before the first call (zero-fill the whole workspace once after
- * allocating it); every call leaves them at zero again.  Calls that run
- * concurrently must not share a workspace.
+ * Workspace: ark_attn_decode_workspace_size(...) bytes (about 16 MB: two
+ * partial slots for each of up to 2048 warps, plus one counter per (request,
+ * KV head)), 16-byte aligned, caller-owned, required.  The counters MUST be
+ * zero before the first call (zero-fill the whole workspace once after
+ * allocating it); every call leaves them at zero again.  Calls that can run
+ * at the same time must not share a workspace.
  * Numerics: bf16 operands on the tensor cores with fp32 accumulation; the
  * softmax weights are rounded to bf16 before they multiply V, o is normalised
  * by the sum of those rounded weights and lse uses the fp32 weights.

@@ -100,11 +100,14 @@ def test_decode_arg_checks(lib):
 
 def test_decode_workspace_size(lib):
     ws = lib.ark_attn_decode_workspace_size
-    assert ws(32, 16, 128, 512, 1) == 0           # one split: no partials
-    assert ws(32, 16, 128, 64, 8) == 0            # T = 64 fits one 64-row chunk
-    n = ws(32, 16, 128, 512, 8)                   # 8 chunks of 64 rows
-    assert n >= 32 * 16 * 8 * 128 * 4 + 32 * 16 * 8 * 4
+    wsl = lib.ark_attn_decode_layers_workspace_size
+    n = ws(32, 16, 128, 512, 8)
+    # two partial slots [8 heads x 128] fp32 for each of up to 2048 warps + counters
+    assert n >= 2048 * 2 * 8 * 128 * 4 + 2048 * 2 * 8 * 4 + 32 * 2 * 4
+    assert n == ws(32, 16, 128, 2048, 1)          # independent of T and the split bound
+    assert wsl(36, 32, 16, 128, 512, 8) >= n + 35 * 32 * 2 * 4
     assert ws(0, 16, 128, 512, 8) == 0
+    assert wsl(0, 32, 16, 128, 512, 8) == 0
 
 
 def test_combine_arg_checks(lib):

@@ -92,6 +92,20 @@ def test_decode_long_cache(oracle_lib, T):
             check_lse(f64(lse), lse_ref)
 
 
+@pytest.mark.parametrize("max_splits", [64, 128])
+def test_decode_many_pieces_per_request(oracle_lib, max_splits):
+    """One long request cut into up to 129 pieces (every warp takes one or two
+    tiles), next to short ones: the in-launch merge over many partials."""
+    T = 2048
+    kv = torch.tensor([2048, 5, 1000, 17], dtype=torch.int32)
+    B = kv.numel()
+    batch = W.make_batch(250 + max_splits, B=B, S=1, T=T, pos0=kv, n_new=[0] * B, garbage="nan")
+    o, lse = gpu_decode(batch.q[0], batch.cache_k[0], batch.cache_v[0], kv, max_splits=max_splits)
+    o_ref, lse_ref = oracle_decode(batch.q[0], batch.cache_k[0], batch.cache_v[0], kv)
+    check_o(f64(o), o_ref)
+    check_lse(f64(lse), lse_ref)
+
+
 def test_decode_single_valid_row_is_exact(oracle_lib):
     """kv_len = 1: the output is that V row, exactly, after bf16 rounding."""
     B, T = 8, 64
