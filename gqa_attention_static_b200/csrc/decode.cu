@@ -116,32 +116,134 @@ __device__ __forceinline__ void issue_tile(uint8_t* stage, uint64_t* bar, const 
 __device__ __forceinline__ int clamp_len(int x, int T) { return x < 0 ? 0 : (x > T ? T : x); }
 
 // One segment = (layer, request, KV head): its tiles are s0 .. s0+n-1 of the
-// global tile list.
+// global tile list.  Tile indices fit in 32 bits (the host checks the size).
 struct Seg {
-    long long s0;
-    int l, b, g, n, kvl, hi;
+    int s0, l, b, g, n, kvl, hi;
 };
 
-// Segment of global tile t, and t's index j inside it.
-__device__ __forceinline__ Seg locate(long long t, const int* s_pref, int per_layer, const DecodeParams& p,
-                                      int& j) {
+__device__ __forceinline__ void seg_fill(Seg& s, const int* s_pref, const DecodeParams& p) {
+    s.n = (s_pref[s.b + 1] - s_pref[s.b]) / p.Hkv;
+    s.kvl = clamp_len(__ldg(p.kv_len + s.b), p.T);
+    s.hi = p.masked ? p.T : s.kvl;
+}
+
+// Segment of global tile t, and t's index j inside it (binary search over
+// the batch prefix; used once per warp).
+__device__ __forceinline__ Seg locate(int t, const int* s_pref, int per_layer, const DecodeParams& p, int& j) {
     Seg s;
-    s.l = static_cast<int>(t / per_layer);
-    const int r = static_cast<int>(t - static_cast<long long>(s.l) * per_layer);
+    s.l = t / per_layer;
+    const int r = t - s.l * per_layer;
     int lo = 0, hi = p.B - 1;                // largest b with s_pref[b] <= r
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (s_pref[mid] <= r) lo = mid; else hi = mid - 1;
     }
     s.b = lo;
-    s.n = (s_pref[lo + 1] - s_pref[lo]) / p.Hkv;
+    seg_fill(s, s_pref, p);
     const int off = r - s_pref[lo];
     s.g = off / s.n;
     j = off - s.g * s.n;
     s.s0 = t - j;
-    s.kvl = clamp_len(__ldg(p.kv_len + s.b), p.T);
-    s.hi = p.masked ? p.T : s.kvl;
     return s;
+}
+
+// The segment after s in list order: next KV head, then next request, then
+// next layer.
+__device__ __forceinline__ void seg_next(Seg& s, const int* s_pref, const DecodeParams& p) {
+    s.s0 += s.n;
+    if (++s.g == p.Hkv) {
+        s.g = 0;
+        if (++s.b == p.B) {
+            s.b = 0;
+            ++s.l;
+        }
+        seg_fill(s, s_pref, p);
+    }
+}
+
+// Log-sum-exp merge of the pieces of one cut segment, run by the warp that
+// finished last.  Pieces come from warps wa..wb; warp wi keeps a piece of this
+// segment in slot 0 if the segment began before its range (T0(wi) > s0), in
+// slot 1 otherwise.  Lane i first reads the 8 heads' lse of piece wa + i
+// (32 pieces at a time), the warp reduces max and sum per head with
+// shuffles, then every lane accumulates dims 4*lane .. 4*lane+3 of all 8
+// heads, two pieces per iteration so that 16 loads are in flight.
+__device__ __noinline__ void merge_pieces(const DecodeParams& p, const Seg& cs, int wa, int wb, int W, int N,
+                                          int lane, size_t bh0) {
+    const int count = wb - wa + 1;
+    float M[kGroup], S[kGroup];
+#pragma unroll
+    for (int h = 0; h < kGroup; ++h) { M[h] = -INFINITY; S[h] = 0.f; }
+    auto slot_row = [&](int wi) -> size_t {   // first row of piece wi's 8 heads
+        const int sl = (static_cast<long long>(wi) * N >= static_cast<long long>(cs.s0 + 1) * W) ? 0 : 1;
+        return (static_cast<size_t>(wi) * 2 + sl) * kGroup;
+    };
+    for (int base = 0; base < count; base += 32) {
+        float l8[kGroup];
+        const int i = base + lane;
+        if (i < count) {
+            const float4* src = reinterpret_cast<const float4*>(p.part_lse + slot_row(wa + i));
+            const float4 x0 = __ldcg(src), x1 = __ldcg(src + 1);
+            l8[0] = x0.x; l8[1] = x0.y; l8[2] = x0.z; l8[3] = x0.w;
+            l8[4] = x1.x; l8[5] = x1.y; l8[6] = x1.z; l8[7] = x1.w;
+        } else {
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) l8[h] = -INFINITY;
+        }
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) {
+            float m = l8[h];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            const float nm = fmaxf(M[h], m);
+            float e = (l8[h] == -INFINITY) ? 0.f : fast_exp2((l8[h] - nm) * kLog2e);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+            S[h] = (M[h] == -INFINITY ? 0.f : S[h] * fast_exp2((M[h] - nm) * kLog2e)) + e;
+            M[h] = nm;
+        }
+    }
+    float4 a[kGroup];
+#pragma unroll
+    for (int h = 0; h < kGroup; ++h) a[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < count; i += 2) {
+        float4 x[2][kGroup];
+        float l2[2][kGroup];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const bool ok = (i + u) < count;
+            const size_t row = slot_row(wa + min(i + u, count - 1));
+            const float4* lsrc = reinterpret_cast<const float4*>(p.part_lse + row);
+            const float4 y0 = __ldcg(lsrc), y1 = __ldcg(lsrc + 1);
+            l2[u][0] = y0.x; l2[u][1] = y0.y; l2[u][2] = y0.z; l2[u][3] = y0.w;
+            l2[u][4] = y1.x; l2[u][5] = y1.y; l2[u][6] = y1.z; l2[u][7] = y1.w;
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) {
+                x[u][h] = __ldcg(reinterpret_cast<const float4*>(p.part_o + (row + h) * kHeadDim) + lane);
+                if (!ok) l2[u][h] = -INFINITY;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) {
+                if (l2[u][h] == -INFINITY || M[h] == -INFINITY) continue;   // empty piece: never read its o
+                const float wgt = fast_exp2((l2[u][h] - M[h]) * kLog2e);
+                a[h].x += wgt * x[u][h].x; a[h].y += wgt * x[u][h].y;
+                a[h].z += wgt * x[u][h].z; a[h].w += wgt * x[u][h].w;
+            }
+    }
+    const int l = cs.l;
+#pragma unroll
+    for (int h = 0; h < kGroup; ++h) {
+        const bool emp = (M[h] == -INFINITY);
+        const float iw = emp ? 0.f : 1.f / S[h];
+        uint2 pk;
+        pk.x = pack_bf16x2(a[h].x * iw, a[h].y * iw);
+        pk.y = pack_bf16x2(a[h].z * iw, a[h].w * iw);
+        reinterpret_cast<uint2*>(p.o[l] + (bh0 + h) * kHeadDim)[lane] = pk;
+        if (lane == 0) p.lse[l][bh0 + h] = emp ? -INFINITY : M[h] + __logf(S[h]);
+    }
 }
 
 __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_constant__ DecodeParams p) {
@@ -184,14 +286,15 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     __syncthreads();   // the last block-wide barrier: warps run independently from here
 
     const int per_layer = s_pref[p.B];
-    const long long N = static_cast<long long>(per_layer) * p.L;
-    long long W = N / p.min_tiles;
+    const int N = per_layer * p.L;
+    int W = N / p.min_tiles;
     if (W < 1) W = 1;
-    if (W > static_cast<long long>(gridDim.x) * kWarps) W = static_cast<long long>(gridDim.x) * kWarps;
+    if (W > static_cast<int>(gridDim.x) * kWarps) W = static_cast<int>(gridDim.x) * kWarps;
     const int w = blockIdx.x * kWarps + warp;
     if (w >= W) return;
-    const long long T0 = static_cast<long long>(w) * N / W;
-    const long long T1 = static_cast<long long>(w + 1) * N / W;
+    // warp w takes tiles [T0, T1); tile t belongs to warp floor(((t+1) W - 1) / N)
+    const int T0 = static_cast<int>(static_cast<long long>(w) * N / W);
+    const int T1 = static_cast<int>(static_cast<long long>(w + 1) * N / W);
 
     const int row_stride = p.Hkv * kHeadDim;
     const int lr = lane & 7;
@@ -203,20 +306,25 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     const uint32_t v_off = kTileBytes + (lr + 8 * (lm >> 1)) * kRowPitch + 16 * (lm & 1);
 
     // ---- producer cursor: next tile to issue
-    long long tp = T0;
+    int tp = T0;
     int pj;
     Seg ps = locate(T0, s_pref, per_layer, p, pj);
+    const uint16_t* pkb = p.k[ps.l] + static_cast<size_t>(ps.b) * p.T * row_stride + ps.g * kHeadDim;
+    const uint16_t* pvb = p.v[ps.l] + static_cast<size_t>(ps.b) * p.T * row_stride + ps.g * kHeadDim;
     uint32_t pseq = 0;
     auto issue_next = [&]() {
         const int r0 = pj * kTileRows;
         const int nrows = max(0, min(kTileRows, ps.hi - r0));
-        const uint16_t* kb = p.k[ps.l] + static_cast<size_t>(ps.b) * p.T * row_stride + ps.g * kHeadDim;
-        const uint16_t* vb = p.v[ps.l] + static_cast<size_t>(ps.b) * p.T * row_stride + ps.g * kHeadDim;
         const int st = pseq % kStages;
-        issue_tile(ring + st * kStageBytes, &bars[st], kb, vb, row_stride, r0, nrows, lane);
+        issue_tile(ring + st * kStageBytes, &bars[st], pkb, pvb, row_stride, r0, nrows, lane);
         ++pseq;
         ++tp;
-        if (++pj == ps.n && tp < T1) ps = locate(tp, s_pref, per_layer, p, pj);
+        if (++pj == ps.n && tp < T1) {
+            seg_next(ps, s_pref, p);
+            pj = 0;
+            pkb = p.k[ps.l] + static_cast<size_t>(ps.b) * p.T * row_stride + ps.g * kHeadDim;
+            pvb = p.v[ps.l] + static_cast<size_t>(ps.b) * p.T * row_stride + ps.g * kHeadDim;
+        }
     };
     for (int s = 0; s < kStages && tp < T1; ++s) issue_next();
 
@@ -248,7 +356,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     begin_segment();
 
     bool failed = false;
-    for (long long t = T0; t < T1; ++t) {
+    for (int t = T0; t < T1; ++t) {
         const uint32_t seq = static_cast<uint32_t>(t - T0);
         const int s = seq % kStages;
         if (!failed && !mbar_wait(&bars[s], (seq / kStages) & 1)) {
@@ -259,13 +367,19 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
         if (!failed) {
             const int r0 = cj * kTileRows;
             const uint32_t st = ring_u32 + s * kStageBytes;
+            // two independent accumulation chains over the head dim, summed at the end
             float sc[4] = {0.f, 0.f, 0.f, 0.f};
+            float sd[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                uint32_t a0, a1, a2, a3;
+            for (int kk = 0; kk < 8; kk += 2) {
+                uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
                 ldsm_x4(st + k_off + kk * 32, a0, a1, a2, a3);
+                ldsm_x4(st + k_off + (kk + 1) * 32, b0, b1, b2, b3);
                 mma_bf16_16816(sc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+                mma_bf16_16816(sd, b0, b1, b2, b3, qf[kk + 1][0], qf[kk + 1][1]);
             }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sc[i] += sd[i];
             const bool v0 = (r0 + gid) < cs.kvl;
             const bool v1 = (r0 + gid + 8) < cs.kvl;
             sc[0] = v0 ? sc[0] * p.scale_log2 : -INFINITY;
@@ -284,8 +398,10 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
             const float n1 = fmaxf(m1, t1);
             const float u0 = (n0 == -INFINITY) ? 0.f : n0;
             const float u1 = (n1 == -INFINITY) ? 0.f : n1;
-            const float alpha0 = fast_exp2(m0 - u0);
-            const float alpha1 = fast_exp2(m1 - u1);
+            // the running max rarely moves once a few tiles are in: skip the rescale then
+            const bool moved = __any_sync(0xffffffffu, (n0 != m0) || (n1 != m1));
+            const float alpha0 = moved ? fast_exp2(m0 - u0) : 1.f;
+            const float alpha1 = moved ? fast_exp2(m1 - u1) : 1.f;
             m0 = n0;
             m1 = n1;
 
@@ -297,12 +413,14 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
             e1 = e1 * alpha1 + (p1 + p3);
             r0s = r0s * alpha0 + (__low2float(p01) + __low2float(p23));
             r1s = r1s * alpha1 + (__high2float(p01) + __high2float(p23));
+            if (moved) {
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                acc[mt][0] *= alpha0;
-                acc[mt][1] *= alpha1;
-                acc[mt][2] *= alpha0;
-                acc[mt][3] *= alpha1;
+                for (int mt = 0; mt < 8; ++mt) {
+                    acc[mt][0] *= alpha0;
+                    acc[mt][1] *= alpha1;
+                    acc[mt][2] *= alpha0;
+                    acc[mt][3] *= alpha1;
+                }
             }
             const uint32_t pb0 = movmatrix_t(*reinterpret_cast<const uint32_t*>(&p01));
             const uint32_t pb1 = movmatrix_t(*reinterpret_cast<const uint32_t*>(&p23));
@@ -366,9 +484,8 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
                 p.part_lse[(static_cast<size_t>(w) * 2 + slot) * kGroup + h1] = lse1;
             }
             // warps whose ranges meet this segment: wa .. wb
-            const long long last_tile = cs.s0 + cs.n - 1;
-            const int wa = static_cast<int>(((cs.s0 + 1) * W - 1) / N);
-            const int wb = static_cast<int>(((last_tile + 1) * W - 1) / N);
+            const int wa = static_cast<int>((static_cast<long long>(cs.s0 + 1) * W - 1) / N);
+            const int wb = static_cast<int>((static_cast<long long>(cs.s0 + cs.n) * W - 1) / N);
             __threadfence();
             __syncwarp();
             int last = 0;
@@ -377,40 +494,13 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
             last = __shfl_sync(0xffffffffu, last, 0);
             if (last) {
                 __threadfence();
-                // merge the pieces of the 8 heads; lane owns dims 4*lane .. 4*lane+3
-                for (int h = 0; h < kGroup; ++h) {
-                    float M = -INFINITY;
-                    for (int wi = wa; wi <= wb; ++wi) {
-                        const int sl = (cs.s0 < static_cast<long long>(wi) * N / W) ? 0 : 1;
-                        M = fmaxf(M, __ldcg(p.part_lse + (static_cast<size_t>(wi) * 2 + sl) * kGroup + h));
-                    }
-                    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-                    float wsum = 0.f;
-                    if (M != -INFINITY) {
-                        for (int wi = wa; wi <= wb; ++wi) {
-                            const int sl = (cs.s0 < static_cast<long long>(wi) * N / W) ? 0 : 1;
-                            const size_t row = (static_cast<size_t>(wi) * 2 + sl) * kGroup + h;
-                            const float lc = __ldcg(p.part_lse + row);
-                            if (lc == -INFINITY) continue;
-                            const float wgt = fast_exp2((lc - M) * kLog2e);
-                            wsum += wgt;
-                            const float4 x = __ldcg(reinterpret_cast<const float4*>(p.part_o + row * kHeadDim) + lane);
-                            a.x += wgt * x.x; a.y += wgt * x.y; a.z += wgt * x.z; a.w += wgt * x.w;
-                        }
-                    }
-                    const bool emp = (M == -INFINITY);
-                    const float iw = emp ? 0.f : 1.f / wsum;
-                    uint2 pk;
-                    pk.x = pack_bf16x2(a.x * iw, a.y * iw);
-                    pk.y = pack_bf16x2(a.z * iw, a.w * iw);
-                    reinterpret_cast<uint2*>(p.o[cs.l] + (bh0 + h) * kHeadDim)[lane] = pk;
-                    if (lane == 0) p.lse[cs.l][bh0 + h] = emp ? -INFINITY : M + __log2f(wsum) * kLn2;
-                }
+                merge_pieces(p, cs, wa, wb, W, N, lane, bh0);
                 if (lane == 0) atomicExch(cnt, 0);
             }
         }
         if (t + 1 < T1) {
-            cs = locate(t + 1, s_pref, per_layer, p, cj);
+            seg_next(cs, s_pref, p);
+            cj = 0;
             begin_segment();
         }
     }
@@ -554,6 +644,8 @@ ark_status fill_common(DecodeParams& prm, const int32_t* kv_len, int L, int B, i
     if (L > ARK_MAX_LAYERS) return ARK_ERR_UNSUPPORTED;
     if (max_splits <= 0 || !(scale > 0.f) || (mode != ARK_LENGTH_AWARE && mode != ARK_MASKED_STATIC))
         return ARK_ERR_INVALID_ARG;
+    const long long max_tiles = static_cast<long long>(L) * B * Hkv * ((T + kTileRows - 1) / kTileRows);
+    if (max_tiles >= (1LL << 30)) return ARK_ERR_UNSUPPORTED;
     prm.kv_len = kv_len;
     prm.status = d_status;
     prm.L = L; prm.B = B; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
