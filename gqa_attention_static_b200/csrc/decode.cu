@@ -21,11 +21,13 @@
 //     warp streams the same number of bytes whatever the length mix.  A range
 //     may start or end inside a segment; that is the split-KV cut.
 //   - Each warp streams its range through a private 2-stage ring in shared
-//     memory, filled by the TMA engine with 1-D bulk copies (one 256 B row
-//     per copy, completion counted on an mbarrier), and keeps streaming
-//     across segment boundaries.  Rows are padded to 272 B so ldmatrix reads
-//     are bank-conflict free.  The 8 query heads of group g are served from a
-//     single read of each K/V row.
+//     memory.  One lane issues four TMA tensor loads per tile (K and V, two
+//     64-element halves each, 128-byte swizzle so that ldmatrix reads are
+//     bank-conflict free); completion is counted on an mbarrier.  The warp
+//     keeps streaming across segment boundaries, and the next segment's 8
+//     query rows (2 KB) arrive by a bulk copy while the current one runs.
+//     The 8 query heads of group g are served from a single read of each K/V
+//     row.
 //   - Scores are computed transposed, S^T[16 pos x 8 heads] = K_tile * Q^T,
 //     with m16n8k16 bf16 tensor-core MMAs: positions fill M = 16 and the 8
 //     heads of the group fill N = 8 exactly, so no MMA lane is wasted.  P^T is
@@ -43,22 +45,25 @@
 // 2 x 8 x 128 multiply-adds, 4 FMA per byte.  At B200 HBM rates that needs
 // most of the fp32 FMA pipe; on the tensor pipe it is a few percent.
 #include "common.cuh"
+#include "tma_host.h"
 
 namespace ark {
 
 constexpr int kWarps = 4;
 constexpr int kStages = 2;
-constexpr int kRowPitch = 272;                      // bytes per smem row (256 + 16 pad)
 constexpr int kTileRows = 16;
-constexpr int kTileBytes = kTileRows * kRowPitch;   // one 16-row K or V tile
-constexpr int kStageBytes = 2 * kTileBytes;         // K tile + V tile
+constexpr int kHalfBytes = kTileRows * 128;          // 16 rows x 64 elements, 128B-swizzled
+constexpr int kTileBytes = 2 * kHalfBytes;           // one 16-row K or V tile (4 KB)
+constexpr int kStageBytes = 2 * kTileBytes;          // K tile + V tile (8 KB)
 constexpr int kWarpRing = kStages * kStageBytes;
 constexpr int kRingBytes = kWarps * kWarpRing;
-constexpr int kBarBytes = kWarps * kStages * 8;
+constexpr int kQSlotBytes = kGroup * kHeadDim * 2;   // the 8 query rows of one group
+constexpr int kQBytes = kWarps * kQSlotBytes;
+constexpr int kBarBytes = kWarps * (kStages + 1) * 8;
 constexpr int kMaxBatch = 4096;
-constexpr int kMaxWarps = 2048;                     // upper bound on warps per launch (sizes the partials)
+constexpr int kMaxWarps = 2048;                      // upper bound on warps per launch (sizes the partials)
 
-struct DecodeParams {
+struct DecodeCore {
     const int32_t* kv_len;
     uint32_t* status;
     float* part_o;       // [kMaxWarps][2][8][D]  two partial slots per warp
@@ -68,11 +73,16 @@ struct DecodeParams {
     int min_tiles;       // fewest tiles one warp takes (bounds the pieces per segment)
     int masked;
     float scale_log2;
-    const uint16_t* q[ARK_MAX_LAYERS];
-    const uint16_t* k[ARK_MAX_LAYERS];
-    const uint16_t* v[ARK_MAX_LAYERS];
-    uint16_t* o[ARK_MAX_LAYERS];
-    float* lse[ARK_MAX_LAYERS];
+};
+
+template <int MaxL>
+struct DecodeParamsT {
+    CUtensorMap kmap[MaxL];   // per layer: cache_k as (128 dims, Hkv, B*T rows), box (64, 1, 16)
+    CUtensorMap vmap[MaxL];
+    DecodeCore c;
+    const uint16_t* q[MaxL];
+    uint16_t* o[MaxL];
+    float* lse[MaxL];
 };
 
 struct CombineLayer {
@@ -87,32 +97,6 @@ struct CombineParams {
     CombineLayer layer[ARK_MAX_LAYERS];
 };
 
-// Issue the bulk copies of one 16-row tile (rows r0 .. r0+nrows-1) into a
-// stage; V rows past nrows are zeroed so that their zero softmax weight never
-// meets a NaN.  nrows may be 0 (an empty request): the phase then completes
-// on the arrival alone.
-__device__ __forceinline__ void issue_tile(uint8_t* stage, uint64_t* bar, const uint16_t* kbase,
-                                           const uint16_t* vbase, int row_stride, int r0, int nrows,
-                                           int lane) {
-    if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nrows) * 2u * 256u);
-    __syncwarp();
-    fence_proxy_async_smem();
-    if (lane < kTileRows) {
-        if (lane < nrows)
-            bulk_g2s(stage + lane * kRowPitch, kbase + static_cast<size_t>(r0 + lane) * row_stride, 256, bar);
-    } else {
-        const int r = lane - kTileRows;
-        if (r < nrows) {
-            bulk_g2s(stage + kTileBytes + r * kRowPitch, vbase + static_cast<size_t>(r0 + r) * row_stride,
-                     256, bar);
-        } else {
-            uint4* z = reinterpret_cast<uint4*>(stage + kTileBytes + r * kRowPitch);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) z[i] = make_uint4(0, 0, 0, 0);
-        }
-    }
-}
-
 __device__ __forceinline__ int clamp_len(int x, int T) { return x < 0 ? 0 : (x > T ? T : x); }
 
 // One segment = (layer, request, KV head): its tiles are s0 .. s0+n-1 of the
@@ -121,25 +105,25 @@ struct Seg {
     int s0, l, b, g, n, kvl, hi;
 };
 
-__device__ __forceinline__ void seg_fill(Seg& s, const int* s_pref, const DecodeParams& p) {
-    s.n = (s_pref[s.b + 1] - s_pref[s.b]) / p.Hkv;
-    s.kvl = clamp_len(__ldg(p.kv_len + s.b), p.T);
-    s.hi = p.masked ? p.T : s.kvl;
+__device__ __forceinline__ void seg_fill(Seg& s, const int* s_pref, const DecodeCore& c) {
+    s.n = (s_pref[s.b + 1] - s_pref[s.b]) / c.Hkv;
+    s.kvl = clamp_len(__ldg(c.kv_len + s.b), c.T);
+    s.hi = c.masked ? c.T : s.kvl;
 }
 
 // Segment of global tile t, and t's index j inside it (binary search over
 // the batch prefix; used once per warp).
-__device__ __forceinline__ Seg locate(int t, const int* s_pref, int per_layer, const DecodeParams& p, int& j) {
+__device__ __forceinline__ Seg locate(int t, const int* s_pref, int per_layer, const DecodeCore& c, int& j) {
     Seg s;
     s.l = t / per_layer;
     const int r = t - s.l * per_layer;
-    int lo = 0, hi = p.B - 1;                // largest b with s_pref[b] <= r
+    int lo = 0, hi = c.B - 1;                // largest b with s_pref[b] <= r
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (s_pref[mid] <= r) lo = mid; else hi = mid - 1;
     }
     s.b = lo;
-    seg_fill(s, s_pref, p);
+    seg_fill(s, s_pref, c);
     const int off = r - s_pref[lo];
     s.g = off / s.n;
     j = off - s.g * s.n;
@@ -149,15 +133,15 @@ __device__ __forceinline__ Seg locate(int t, const int* s_pref, int per_layer, c
 
 // The segment after s in list order: next KV head, then next request, then
 // next layer.
-__device__ __forceinline__ void seg_next(Seg& s, const int* s_pref, const DecodeParams& p) {
+__device__ __forceinline__ void seg_next(Seg& s, const int* s_pref, const DecodeCore& c) {
     s.s0 += s.n;
-    if (++s.g == p.Hkv) {
+    if (++s.g == c.Hkv) {
         s.g = 0;
-        if (++s.b == p.B) {
+        if (++s.b == c.B) {
             s.b = 0;
             ++s.l;
         }
-        seg_fill(s, s_pref, p);
+        seg_fill(s, s_pref, c);
     }
 }
 
@@ -168,8 +152,8 @@ __device__ __forceinline__ void seg_next(Seg& s, const int* s_pref, const Decode
 // (32 pieces at a time), the warp reduces max and sum per head with
 // shuffles, then every lane accumulates dims 4*lane .. 4*lane+3 of all 8
 // heads, two pieces per iteration so that 16 loads are in flight.
-__device__ __noinline__ void merge_pieces(const DecodeParams& p, const Seg& cs, int wa, int wb, int W, int N,
-                                          int lane, size_t bh0) {
+__device__ __forceinline__ void merge_pieces(const DecodeCore& c, uint16_t* o, float* lse_out, const Seg& cs, int wa,
+                                          int wb, int W, int N, int lane, size_t bh0) {
     const int count = wb - wa + 1;
     float M[kGroup], S[kGroup];
 #pragma unroll
@@ -182,7 +166,7 @@ __device__ __noinline__ void merge_pieces(const DecodeParams& p, const Seg& cs, 
         float l8[kGroup];
         const int i = base + lane;
         if (i < count) {
-            const float4* src = reinterpret_cast<const float4*>(p.part_lse + slot_row(wa + i));
+            const float4* src = reinterpret_cast<const float4*>(c.part_lse + slot_row(wa + i));
             const float4 x0 = __ldcg(src), x1 = __ldcg(src + 1);
             l8[0] = x0.x; l8[1] = x0.y; l8[2] = x0.z; l8[3] = x0.w;
             l8[4] = x1.x; l8[5] = x1.y; l8[6] = x1.z; l8[7] = x1.w;
@@ -194,11 +178,11 @@ __device__ __noinline__ void merge_pieces(const DecodeParams& p, const Seg& cs, 
         for (int h = 0; h < kGroup; ++h) {
             float m = l8[h];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
             const float nm = fmaxf(M[h], m);
             float e = (l8[h] == -INFINITY) ? 0.f : fast_exp2((l8[h] - nm) * kLog2e);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+            for (int off = 16; off > 0; off >>= 1) e += __shfl_xor_sync(0xffffffffu, e, off);
             S[h] = (M[h] == -INFINITY ? 0.f : S[h] * fast_exp2((M[h] - nm) * kLog2e)) + e;
             M[h] = nm;
         }
@@ -213,13 +197,13 @@ __device__ __noinline__ void merge_pieces(const DecodeParams& p, const Seg& cs, 
         for (int u = 0; u < 2; ++u) {
             const bool ok = (i + u) < count;
             const size_t row = slot_row(wa + min(i + u, count - 1));
-            const float4* lsrc = reinterpret_cast<const float4*>(p.part_lse + row);
+            const float4* lsrc = reinterpret_cast<const float4*>(c.part_lse + row);
             const float4 y0 = __ldcg(lsrc), y1 = __ldcg(lsrc + 1);
             l2[u][0] = y0.x; l2[u][1] = y0.y; l2[u][2] = y0.z; l2[u][3] = y0.w;
             l2[u][4] = y1.x; l2[u][5] = y1.y; l2[u][6] = y1.z; l2[u][7] = y1.w;
 #pragma unroll
             for (int h = 0; h < kGroup; ++h) {
-                x[u][h] = __ldcg(reinterpret_cast<const float4*>(p.part_o + (row + h) * kHeadDim) + lane);
+                x[u][h] = __ldcg(reinterpret_cast<const float4*>(c.part_o + (row + h) * kHeadDim) + lane);
                 if (!ok) l2[u][h] = -INFINITY;
             }
         }
@@ -233,7 +217,6 @@ __device__ __noinline__ void merge_pieces(const DecodeParams& p, const Seg& cs, 
                 a[h].z += wgt * x[u][h].z; a[h].w += wgt * x[u][h].w;
             }
     }
-    const int l = cs.l;
 #pragma unroll
     for (int h = 0; h < kGroup; ++h) {
         const bool emp = (M[h] == -INFINITY);
@@ -241,53 +224,62 @@ __device__ __noinline__ void merge_pieces(const DecodeParams& p, const Seg& cs, 
         uint2 pk;
         pk.x = pack_bf16x2(a[h].x * iw, a[h].y * iw);
         pk.y = pack_bf16x2(a[h].z * iw, a[h].w * iw);
-        reinterpret_cast<uint2*>(p.o[l] + (bh0 + h) * kHeadDim)[lane] = pk;
-        if (lane == 0) p.lse[l][bh0 + h] = emp ? -INFINITY : M[h] + __logf(S[h]);
+        reinterpret_cast<uint2*>(o + (bh0 + h) * kHeadDim)[lane] = pk;
+        if (lane == 0) lse_out[bh0 + h] = emp ? -INFINITY : M[h] + __logf(S[h]);
     }
 }
 
-__global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_constant__ DecodeParams p) {
-    extern __shared__ __align__(128) uint8_t smem[];
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
+}
+
+template <int MaxL>
+__global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_constant__ DecodeParamsT<MaxL> p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    const DecodeCore& c = p.c;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int gid = lane >> 2;
     const int tig = lane & 3;
     uint8_t* ring = smem + warp * kWarpRing;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRingBytes) + warp * kStages;
-    int* s_pref = reinterpret_cast<int*>(smem + kRingBytes + kBarBytes);   // [B + 1]
+    uint8_t* qslot = smem + kRingBytes + warp * kQSlotBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRingBytes + kQBytes) + warp * (kStages + 1);
+    uint64_t* qbar = bars + kStages;
+    int* s_pref = reinterpret_cast<int*>(smem + kRingBytes + kQBytes + kBarBytes);   // [B + 1]
 
     // ---- per CTA: prefix over the batch of the tiles per request (all KV heads)
     if (warp == 0) {
         if (lane == 0) s_pref[0] = 0;
         int run = 0;
-        for (int base = 0; base < p.B; base += 32) {
+        for (int base = 0; base < c.B; base += 32) {
             const int b = base + lane;
             int n = 0;
-            if (b < p.B) {
-                const int raw = __ldg(p.kv_len + b);
-                if ((raw < 0 || raw > p.T) && blockIdx.x == 0) report(p.status, ARK_DEV_BAD_KVLEN);
-                const int hi = p.masked ? p.T : clamp_len(raw, p.T);
-                n = max(1, (hi + kTileRows - 1) / kTileRows) * p.Hkv;
+            if (b < c.B) {
+                const int raw = __ldg(c.kv_len + b);
+                if ((raw < 0 || raw > c.T) && blockIdx.x == 0) report(c.status, ARK_DEV_BAD_KVLEN);
+                const int hi = c.masked ? c.T : clamp_len(raw, c.T);
+                n = max(1, (hi + kTileRows - 1) / kTileRows) * c.Hkv;
             }
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, n, off);
                 if (lane >= off) n += y;
             }
-            if (b < p.B) s_pref[b + 1] = run + n;
+            if (b < c.B) s_pref[b + 1] = run + n;
             run += __shfl_sync(0xffffffffu, n, 31);
         }
     }
     if (lane == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+        for (int s = 0; s <= kStages; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
     }
     fence_proxy_async_smem();
     __syncthreads();   // the last block-wide barrier: warps run independently from here
 
-    const int per_layer = s_pref[p.B];
-    const int N = per_layer * p.L;
-    int W = N / p.min_tiles;
+    const int per_layer = s_pref[c.B];
+    const int N = per_layer * c.L;
+    int W = N / c.min_tiles;
     if (W < 1) W = 1;
     if (W > static_cast<int>(gridDim.x) * kWarps) W = static_cast<int>(gridDim.x) * kWarps;
     const int w = blockIdx.x * kWarps + warp;
@@ -296,53 +288,75 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     const int T0 = static_cast<int>(static_cast<long long>(w) * N / W);
     const int T1 = static_cast<int>(static_cast<long long>(w + 1) * N / W);
 
-    const int row_stride = p.Hkv * kHeadDim;
     const int lr = lane & 7;
     const int lm = lane >> 3;
     const uint32_t ring_u32 = smem_u32(ring);
-    // K (A operand, non-transposed): matrix lm -> rows 8*(lm&1), cols 8*(lm>>1)
-    const uint32_t k_off = (lr + 8 * (lm & 1)) * kRowPitch + 16 * (lm >> 1);
-    // V (A operand of V^T, transposed load): matrix lm -> rows 8*(lm>>1), cols 8*(lm&1)
-    const uint32_t v_off = kTileBytes + (lr + 8 * (lm >> 1)) * kRowPitch + 16 * (lm & 1);
+    // swizzled ldmatrix addressing: a 16-byte chunk k of row r sits at chunk k ^ (r & 7)
+    const uint32_t k_row = (lr + 8 * (lm & 1)) * 128;          // K: matrix lm -> rows 8*(lm&1)
+    const uint32_t k_x = (lm >> 1) ^ lr;                       //    and the column chunk lm>>1
+    const uint32_t v_row = kTileBytes + (lr + 8 * (lm >> 1)) * 128;   // V^T: rows 8*(lm>>1)
+    const uint32_t v_x = (lm & 1) ^ lr;                        //      column chunk lm&1
 
     // ---- producer cursor: next tile to issue
     int tp = T0;
     int pj;
-    Seg ps = locate(T0, s_pref, per_layer, p, pj);
-    const uint16_t* pkb = p.k[ps.l] + static_cast<size_t>(ps.b) * p.T * row_stride + ps.g * kHeadDim;
-    const uint16_t* pvb = p.v[ps.l] + static_cast<size_t>(ps.b) * p.T * row_stride + ps.g * kHeadDim;
+    Seg ps = locate(T0, s_pref, per_layer, c, pj);
     uint32_t pseq = 0;
     auto issue_next = [&]() {
-        const int r0 = pj * kTileRows;
-        const int nrows = max(0, min(kTileRows, ps.hi - r0));
         const int st = pseq % kStages;
-        issue_tile(ring + st * kStageBytes, &bars[st], pkb, pvb, row_stride, r0, nrows, lane);
+        if (lane == 0) {
+            uint8_t* dst = ring + st * kStageBytes;
+            const int row = ps.b * c.T + pj * kTileRows;
+            mbar_arrive_expect_tx(&bars[st], kStageBytes);
+            tma_load_3d(dst, &p.kmap[ps.l], 0, ps.g, row, &bars[st]);
+            tma_load_3d(dst + kHalfBytes, &p.kmap[ps.l], 64, ps.g, row, &bars[st]);
+            tma_load_3d(dst + kTileBytes, &p.vmap[ps.l], 0, ps.g, row, &bars[st]);
+            tma_load_3d(dst + kTileBytes + kHalfBytes, &p.vmap[ps.l], 64, ps.g, row, &bars[st]);
+        }
         ++pseq;
         ++tp;
         if (++pj == ps.n && tp < T1) {
-            seg_next(ps, s_pref, p);
+            seg_next(ps, s_pref, c);
             pj = 0;
-            pkb = p.k[ps.l] + static_cast<size_t>(ps.b) * p.T * row_stride + ps.g * kHeadDim;
-            pvb = p.v[ps.l] + static_cast<size_t>(ps.b) * p.T * row_stride + ps.g * kHeadDim;
         }
     };
     for (int s = 0; s < kStages && tp < T1; ++s) issue_next();
 
+    // ---- query rows of a segment: one 2 KB bulk copy into this warp's slot
+    auto issue_q = [&](const Seg& s) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(qbar, kQSlotBytes);
+            bulk_g2s(qslot, p.q[s.l] + (static_cast<size_t>(s.b) * c.Hq + s.g * kGroup) * kHeadDim, kQSlotBytes,
+                     qbar);
+        }
+    };
+
     // ---- consumer cursor
     int cj;
-    Seg cs = locate(T0, s_pref, per_layer, p, cj);
+    Seg cs = locate(T0, s_pref, per_layer, c, cj);
+    issue_q(cs);
+    uint32_t qseq = 0;       // query copies consumed
+    uint32_t qissued = 1;    // query copies issued
+    bool q_next = false;     // the next segment's query rows are still to be fetched
+    bool failed = false;
     uint32_t qf[8][2];
     float acc[8][4];
     float m0, m1, e0, e1, r0s, r1s;
     auto begin_segment = [&]() {
-        // Q of the 8 heads as B fragments: b0 = Q[head gid][16kk + 2tig .. +1], b1 = same + 8
-        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-            p.q[cs.l] + (static_cast<size_t>(cs.b) * p.Hq + cs.g * kGroup + gid) * kHeadDim);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            qf[kk][0] = __ldg(qrow + kk * 8 + tig);
-            qf[kk][1] = __ldg(qrow + kk * 8 + 4 + tig);
+        if (!failed && !mbar_wait(qbar, qseq & 1)) {
+            failed = true;
+            if (lane == 0) report(c.status, ARK_DEV_TIMEOUT);
         }
+        ++qseq;
+        // B fragments of Q [8 heads][128 dims]: block (heads 0-7, dims 8k..8k+7) -> b0/b1 of k-step k/2
+        const uint32_t qa = smem_u32(qslot) + lr * 256 + lm * 16;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            ldsm_x4(qa + i * 64, qf[2 * i][0], qf[2 * i][1], qf[2 * i + 1][0], qf[2 * i + 1][1]);
+        __syncwarp();
+        // fetch the next segment's rows into the slot once the fragments above
+        // have been consumed by the first tile's MMAs
+        q_next = (cs.s0 + cs.n < T1);
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
@@ -355,26 +369,39 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     };
     begin_segment();
 
-    bool failed = false;
     for (int t = T0; t < T1; ++t) {
         const uint32_t seq = static_cast<uint32_t>(t - T0);
         const int s = seq % kStages;
         if (!failed && !mbar_wait(&bars[s], (seq / kStages) & 1)) {
             failed = true;
-            if (lane == 0) report(p.status, ARK_DEV_TIMEOUT);
+            if (lane == 0) report(c.status, ARK_DEV_TIMEOUT);
         }
-        __syncwarp();   // zero rows written by other lanes are visible from here on
         if (!failed) {
             const int r0 = cj * kTileRows;
             const uint32_t st = ring_u32 + s * kStageBytes;
+            const int live = cs.hi - r0;   // rows of this tile that belong to the request's read range
+            if (live < kTileRows) {
+                // the box also brought rows past the range (next request, or garbage):
+                // zero their V rows so that their zero weights never meet a NaN
+                uint8_t* vt = ring + s * kStageBytes + kTileBytes;
+                const int z0 = max(live, 0);
+                for (int i = lane; i < (kTileRows - z0) * 16; i += 32) {
+                    const int r = z0 + (i >> 4), part = i & 15;
+                    *reinterpret_cast<uint4*>(vt + (part >> 3) * kHalfBytes + r * 128 + (part & 7) * 16) =
+                        make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
             // two independent accumulation chains over the head dim, summed at the end
             float sc[4] = {0.f, 0.f, 0.f, 0.f};
             float sd[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int kk = 0; kk < 8; kk += 2) {
                 uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-                ldsm_x4(st + k_off + kk * 32, a0, a1, a2, a3);
-                ldsm_x4(st + k_off + (kk + 1) * 32, b0, b1, b2, b3);
+                ldsm_x4(st + (kk >> 2) * kHalfBytes + k_row + (((2 * (kk & 3)) ^ k_x) << 4), a0, a1, a2, a3);
+                ldsm_x4(st + ((kk + 1) >> 2) * kHalfBytes + k_row + (((2 * ((kk + 1) & 3)) ^ k_x) << 4),
+                        b0, b1, b2, b3);
                 mma_bf16_16816(sc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
                 mma_bf16_16816(sd, b0, b1, b2, b3, qf[kk + 1][0], qf[kk + 1][1]);
             }
@@ -382,10 +409,10 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
             for (int i = 0; i < 4; ++i) sc[i] += sd[i];
             const bool v0 = (r0 + gid) < cs.kvl;
             const bool v1 = (r0 + gid + 8) < cs.kvl;
-            sc[0] = v0 ? sc[0] * p.scale_log2 : -INFINITY;
-            sc[1] = v0 ? sc[1] * p.scale_log2 : -INFINITY;
-            sc[2] = v1 ? sc[2] * p.scale_log2 : -INFINITY;
-            sc[3] = v1 ? sc[3] * p.scale_log2 : -INFINITY;
+            sc[0] = v0 ? sc[0] * c.scale_log2 : -INFINITY;
+            sc[1] = v0 ? sc[1] * c.scale_log2 : -INFINITY;
+            sc[2] = v1 ? sc[2] * c.scale_log2 : -INFINITY;
+            sc[3] = v1 ? sc[3] * c.scale_log2 : -INFINITY;
 
             float t0 = fmaxf(sc[0], sc[2]);
             float t1 = fmaxf(sc[1], sc[3]);
@@ -427,11 +454,18 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 uint32_t a0, a1, a2, a3;
-                ldsm_x4_t(st + v_off + mt * 32, a0, a1, a2, a3);
+                ldsm_x4_t(st + v_row + (mt >> 2) * kHalfBytes + (((2 * (mt & 3)) ^ v_x) << 4), a0, a1, a2, a3);
                 mma_bf16_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
             }
             __syncwarp();
             if (tp < T1) issue_next();     // refill the stage just consumed
+            if (q_next) {
+                Seg nx = cs;
+                seg_next(nx, s_pref, c);
+                issue_q(nx);
+                ++qissued;
+                q_next = false;
+            }
         }
 
         if (++cj < cs.n && t + 1 < T1) continue;
@@ -451,11 +485,10 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
         const float lse0 = empty0 ? -INFINITY : (m0 + __log2f(e0)) * kLn2;
         const float lse1 = empty1 ? -INFINITY : (m1 + __log2f(e1)) * kLn2;
         const int h0 = 2 * tig, h1 = 2 * tig + 1;
-        const size_t bh0 = static_cast<size_t>(cs.b) * p.Hq + cs.g * kGroup;   // row of the group's head 0
+        const size_t bh0 = static_cast<size_t>(cs.b) * c.Hq + cs.g * kGroup;   // row of the group's head 0
         const bool whole = (cs.s0 >= T0) && (cs.s0 + cs.n <= T1);
         if (whole) {
-            uint16_t* og = p.o[cs.l] + bh0 * kHeadDim;
-            __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(og);
+            __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(p.o[cs.l] + bh0 * kHeadDim);
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 const int d = 16 * mt + gid;
@@ -470,7 +503,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
             }
         } else {
             const int slot = (cs.s0 < T0) ? 0 : 1;
-            float* po = p.part_o + (static_cast<size_t>(w) * 2 + slot) * kGroup * kHeadDim;
+            float* po = c.part_o + (static_cast<size_t>(w) * 2 + slot) * kGroup * kHeadDim;
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 const int d = 16 * mt + gid;
@@ -480,8 +513,8 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
                 po[h1 * kHeadDim + d + 8] = acc[mt][3] * inv1;
             }
             if (gid == 0) {
-                p.part_lse[(static_cast<size_t>(w) * 2 + slot) * kGroup + h0] = lse0;
-                p.part_lse[(static_cast<size_t>(w) * 2 + slot) * kGroup + h1] = lse1;
+                c.part_lse[(static_cast<size_t>(w) * 2 + slot) * kGroup + h0] = lse0;
+                c.part_lse[(static_cast<size_t>(w) * 2 + slot) * kGroup + h1] = lse1;
             }
             // warps whose ranges meet this segment: wa .. wb
             const int wa = static_cast<int>((static_cast<long long>(cs.s0 + 1) * W - 1) / N);
@@ -489,26 +522,27 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
             __threadfence();
             __syncwarp();
             int last = 0;
-            int* cnt = p.counters + (static_cast<size_t>(cs.l) * p.B + cs.b) * p.Hkv + cs.g;
+            int* cnt = c.counters + (static_cast<size_t>(cs.l) * c.B + cs.b) * c.Hkv + cs.g;
             if (lane == 0) last = (atomicAdd(cnt, 1) == wb - wa);
             last = __shfl_sync(0xffffffffu, last, 0);
             if (last) {
                 __threadfence();
-                merge_pieces(p, cs, wa, wb, W, N, lane, bh0);
+                merge_pieces(c, p.o[cs.l], p.lse[cs.l], cs, wa, wb, W, N, lane, bh0);
                 if (lane == 0) atomicExch(cnt, 0);
             }
         }
         if (t + 1 < T1) {
-            seg_next(cs, s_pref, p);
+            seg_next(cs, s_pref, c);
             cj = 0;
             begin_segment();
         }
     }
     // Never leave with copies in flight: a timed-out warp stops consuming, so
-    // wait (bounded) for the tiles it issued but did not consume.
+    // wait (bounded) for the tiles and query rows it issued but did not consume.
     if (failed) {
         for (uint32_t q2 = pseq > kStages ? pseq - kStages : 0; q2 < pseq; ++q2)
             (void)mbar_wait(&bars[q2 % kStages], (q2 / kStages) & 1);
+        if (qissued > qseq) (void)mbar_wait(qbar, qseq & 1);
     }
 }
 
@@ -585,26 +619,27 @@ ark_status check_decode_shape(int B, int T, int Hq, int Hkv, int D) {
     return ARK_OK;
 }
 
-size_t decode_smem(int B) { return kRingBytes + kBarBytes + align256((B + 1) * sizeof(int)); }
+size_t decode_smem(int B) { return 1024 + kRingBytes + kQBytes + kBarBytes + align256((B + 1) * sizeof(int)); }
 
-// SM count and resident CTAs per SM, queried once per device.
+// SM count and resident CTAs per SM, queried once per device and kernel.
 struct DeviceInfo {
     int sms = 0, ctas_per_sm = 0;
 };
-DeviceInfo g_dev[64];
 
+template <int MaxL>
 ark_status device_info(DeviceInfo& out) {
+    static DeviceInfo table[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARK_ERR_CUDA;
-    DeviceInfo& d = g_dev[dev];
+    DeviceInfo& d = table[dev];
     if (d.sms == 0) {
-        if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(decode_kernel<MaxL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(decode_smem(kMaxBatch))) != cudaSuccess)
             return ARK_ERR_CUDA;
         int sms = 0, per = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ARK_ERR_CUDA;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_kernel, kWarps * 32, decode_smem(64)) !=
-            cudaSuccess)
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_kernel<MaxL>, kWarps * 32,
+                                                          decode_smem(64)) != cudaSuccess)
             return ARK_ERR_CUDA;
         d.ctas_per_sm = per > 0 ? per : 1;
         d.sms = sms;
@@ -613,29 +648,36 @@ ark_status device_info(DeviceInfo& out) {
     return ARK_OK;
 }
 
-ark_status launch_decode(DecodeParams& prm, void* workspace, size_t ws_bytes, cudaStream_t stream) {
-    const WsLayout w = ws_layout(prm.L, prm.B, prm.Hkv);
+template <int MaxL>
+ark_status launch_decode(DecodeParamsT<MaxL>& prm, const void* const* k, const void* const* v, void* workspace,
+                         size_t ws_bytes, int max_warps, cudaStream_t stream) {
+    DecodeCore& c = prm.c;
+    const WsLayout w = ws_layout(c.L, c.B, c.Hkv);
     if (!workspace || ws_bytes < w.total || !aligned16(workspace)) return ARK_ERR_WORKSPACE;
     uint8_t* base = static_cast<uint8_t*>(workspace);
-    prm.part_o = reinterpret_cast<float*>(base + w.part_o);
-    prm.part_lse = reinterpret_cast<float*>(base + w.part_lse);
-    prm.counters = reinterpret_cast<int*>(base + w.counters);
+    c.part_o = reinterpret_cast<float*>(base + w.part_o);
+    c.part_lse = reinterpret_cast<float*>(base + w.part_lse);
+    c.counters = reinterpret_cast<int*>(base + w.counters);
+    for (int l = 0; l < c.L; ++l) {
+        if (!kv_tensor_map(&prm.kmap[l], k[l], static_cast<long long>(c.B) * c.T, c.Hkv, 64, kTileRows) ||
+            !kv_tensor_map(&prm.vmap[l], v[l], static_cast<long long>(c.B) * c.T, c.Hkv, 64, kTileRows))
+            return ARK_ERR_CUDA;
+    }
     DeviceInfo d;
-    ark_status st = device_info(d);
+    ark_status st = device_info<MaxL>(d);
     if (st != ARK_OK) return st;
     // tiles in the largest case the device lengths can produce
-    const long long max_tiles =
-        static_cast<long long>(prm.L) * prm.B * prm.Hkv * ((prm.T + kTileRows - 1) / kTileRows);
+    const long long max_tiles = static_cast<long long>(c.L) * c.B * c.Hkv * ((c.T + kTileRows - 1) / kTileRows);
     long long grid = static_cast<long long>(d.sms) * d.ctas_per_sm;
-    const long long need = (max_tiles / prm.min_tiles + kWarps - 1) / kWarps;
+    const long long need = (max_tiles / c.min_tiles + kWarps - 1) / kWarps;
     if (need < grid) grid = need;
-    if (grid > kMaxWarps / kWarps) grid = kMaxWarps / kWarps;
+    if (grid > max_warps / kWarps) grid = max_warps / kWarps;
     if (grid < 1) grid = 1;
-    decode_kernel<<<static_cast<unsigned>(grid), kWarps * 32, decode_smem(prm.B), stream>>>(prm);
+    decode_kernel<MaxL><<<static_cast<unsigned>(grid), kWarps * 32, decode_smem(c.B), stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
 }
 
-ark_status fill_common(DecodeParams& prm, const int32_t* kv_len, int L, int B, int T, int Hq, int Hkv, int D,
+ark_status fill_common(DecodeCore& c, const int32_t* kv_len, int L, int B, int T, int Hq, int Hkv, int D,
                        float scale, ark_decode_mode mode, int max_splits, uint32_t* d_status) {
     if (!kv_len) return ARK_ERR_INVALID_ARG;
     ark_status st = check_decode_shape(B, T, Hq, Hkv, D);
@@ -646,12 +688,12 @@ ark_status fill_common(DecodeParams& prm, const int32_t* kv_len, int L, int B, i
         return ARK_ERR_INVALID_ARG;
     const long long max_tiles = static_cast<long long>(L) * B * Hkv * ((T + kTileRows - 1) / kTileRows);
     if (max_tiles >= (1LL << 30)) return ARK_ERR_UNSUPPORTED;
-    prm.kv_len = kv_len;
-    prm.status = d_status;
-    prm.L = L; prm.B = B; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
-    prm.min_tiles = decode_min_tiles(T, max_splits);
-    prm.masked = (mode == ARK_MASKED_STATIC) ? 1 : 0;
-    prm.scale_log2 = scale * kLog2e;
+    c.kv_len = kv_len;
+    c.status = d_status;
+    c.L = L; c.B = B; c.T = T; c.Hq = Hq; c.Hkv = Hkv;
+    c.min_tiles = decode_min_tiles(T, max_splits);
+    c.masked = (mode == ARK_MASKED_STATIC) ? 1 : 0;
+    c.scale_log2 = scale * kLog2e;
     return ARK_OK;
 }
 
@@ -672,18 +714,16 @@ extern "C" ark_status ark_attn_decode(const void* q, const void* cache_k, const 
                                       void* workspace, size_t workspace_bytes,
                                       void* o, float* lse, uint32_t* d_status, cudaStream_t stream) {
     if (!q || !cache_k || !cache_v || !o || !lse) return ARK_ERR_INVALID_ARG;
-    DecodeParams prm{};
-    ark_status st = fill_common(prm, kv_len, 1, B, T, Hq, Hkv, D, scale, mode, max_splits, d_status);
+    DecodeParamsT<1> prm{};
+    ark_status st = fill_common(prm.c, kv_len, 1, B, T, Hq, Hkv, D, scale, mode, max_splits, d_status);
     if (st != ARK_OK) return st;
     if (!aligned16(q) || !aligned16(cache_k) || !aligned16(cache_v) || !aligned16(o) ||
         (reinterpret_cast<uintptr_t>(lse) & 3u))
         return ARK_ERR_INVALID_ARG;
     prm.q[0] = static_cast<const uint16_t*>(q);
-    prm.k[0] = static_cast<const uint16_t*>(cache_k);
-    prm.v[0] = static_cast<const uint16_t*>(cache_v);
     prm.o[0] = static_cast<uint16_t*>(o);
     prm.lse[0] = lse;
-    return launch_decode(prm, workspace, workspace_bytes, stream);
+    return launch_decode<1>(prm, &cache_k, &cache_v, workspace, workspace_bytes, kMaxWarps, stream);
 }
 
 extern "C" ark_status ark_attn_decode_layers(int L, const void* const* q, const void* const* cache_k,
@@ -693,8 +733,9 @@ extern "C" ark_status ark_attn_decode_layers(int L, const void* const* q, const 
                                              void* const* o, float* const* lse, uint32_t* d_status,
                                              cudaStream_t stream) {
     if (!q || !cache_k || !cache_v || !o || !lse) return ARK_ERR_INVALID_ARG;
-    DecodeParams prm{};
-    ark_status st = fill_common(prm, kv_len, L, B, T, Hq, Hkv, D, scale, mode, max_splits, d_status);
+    static thread_local DecodeParamsT<ARK_MAX_LAYERS> prm;
+    prm = DecodeParamsT<ARK_MAX_LAYERS>{};
+    ark_status st = fill_common(prm.c, kv_len, L, B, T, Hq, Hkv, D, scale, mode, max_splits, d_status);
     if (st != ARK_OK) return st;
     for (int l = 0; l < L; ++l) {
         if (!q[l] || !cache_k[l] || !cache_v[l] || !o[l] || !lse[l]) return ARK_ERR_INVALID_ARG;
@@ -702,12 +743,10 @@ extern "C" ark_status ark_attn_decode_layers(int L, const void* const* q, const 
             (reinterpret_cast<uintptr_t>(lse[l]) & 3u))
             return ARK_ERR_INVALID_ARG;
         prm.q[l] = static_cast<const uint16_t*>(q[l]);
-        prm.k[l] = static_cast<const uint16_t*>(cache_k[l]);
-        prm.v[l] = static_cast<const uint16_t*>(cache_v[l]);
         prm.o[l] = static_cast<uint16_t*>(o[l]);
         prm.lse[l] = lse[l];
     }
-    return launch_decode(prm, workspace, workspace_bytes, stream);
+    return launch_decode<ARK_MAX_LAYERS>(prm, cache_k, cache_v, workspace, workspace_bytes, kMaxWarps, stream);
 }
 
 extern "C" ark_status ark_attn_combine(const float* o_part, const float* lse_part, int B, int Hq,

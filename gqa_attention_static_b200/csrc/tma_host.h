@@ -1,0 +1,20 @@
+// tma_host.h -- host-side encoding of TMA tensor maps over the KV cache, with
+// a small cache so that repeated calls on the same buffers do not re-encode.
+#pragma once
+
+#include <cuda.h>
+#include <cstdint>
+
+namespace ark {
+
+// 3-D tiled map over a cache [B, T, Hkv, 128] bf16 viewed as
+// (dim 0: 128 head-dim elements, dim 1: Hkv heads, dim 2: B*T rows), box
+// (box_inner elements, 1 head, box_rows rows), 128-byte swizzle, zero fill
+// out of bounds.  Returns false if the driver rejects it.
+bool kv_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv, int box_inner, int box_rows);
+
+// 2-D tiled map over a row-major [rows, 128] bf16 matrix (row pitch 256 B),
+// box (box_inner elements, box_rows rows), 128-byte swizzle.
+bool rows_tensor_map(CUtensorMap* out, const void* base, long long rows, int box_inner, int box_rows);
+
+}  // namespace ark
