@@ -339,8 +339,6 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     uint32_t qissued = 1;    // query copies issued
     bool q_next = false;     // the next segment's query rows are still to be fetched
     bool failed = false;
-    Seg cut[2];              // segments this warp holds a piece of (slot 0: began before T0, slot 1: ends after T1)
-    int has_cut = 0;
     uint32_t qf[8][2];
     float acc[8][4];
     float m0, m1, e0, e1, r0s, r1s;
@@ -518,36 +516,25 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
                 c.part_lse[(static_cast<size_t>(w) * 2 + slot) * kGroup + h0] = lse0;
                 c.part_lse[(static_cast<size_t>(w) * 2 + slot) * kGroup + h1] = lse1;
             }
-            cut[slot] = cs;         // published after the loop, behind one fence
-            has_cut |= 1 << slot;
+            // warps whose ranges meet this segment: wa .. wb
+            const int wa = static_cast<int>((static_cast<long long>(cs.s0 + 1) * W - 1) / N);
+            const int wb = static_cast<int>((static_cast<long long>(cs.s0 + cs.n) * W - 1) / N);
+            __threadfence();
+            __syncwarp();
+            int last = 0;
+            int* cnt = c.counters + (static_cast<size_t>(cs.l) * c.B + cs.b) * c.Hkv + cs.g;
+            if (lane == 0) last = (atomicAdd(cnt, 1) == wb - wa);
+            last = __shfl_sync(0xffffffffu, last, 0);
+            if (last) {
+                __threadfence();
+                merge_pieces(c, p.o[cs.l], p.lse[cs.l], cs, wa, wb, W, N, lane, bh0);
+                if (lane == 0) atomicExch(cnt, 0);
+            }
         }
         if (t + 1 < T1) {
             seg_next(cs, s_pref, c);
             cj = 0;
             begin_segment();
-        }
-    }
-    // ---- publish the (at most two) cut segments: one fence for both, then the
-    // per-segment counters; the warp that completes a segment merges it.
-    if (has_cut) {
-        __threadfence();
-        __syncwarp();
-        for (int sl = 0; sl < 2; ++sl) {
-            if (!(has_cut & (1 << sl))) continue;
-            const Seg& sg = cut[sl];
-            // warps whose ranges meet this segment: wa .. wb
-            const int wa = static_cast<int>((static_cast<long long>(sg.s0 + 1) * W - 1) / N);
-            const int wb = static_cast<int>((static_cast<long long>(sg.s0 + sg.n) * W - 1) / N);
-            int last = 0;
-            int* cnt = c.counters + (static_cast<size_t>(sg.l) * c.B + sg.b) * c.Hkv + sg.g;
-            if (lane == 0) last = (atomicAdd(cnt, 1) == wb - wa);
-            last = __shfl_sync(0xffffffffu, last, 0);
-            if (last) {
-                __threadfence();
-                const size_t bh0 = static_cast<size_t>(sg.b) * c.Hq + sg.g * kGroup;
-                merge_pieces(c, p.o[sg.l], p.lse[sg.l], sg, wa, wb, W, N, lane, bh0);
-                if (lane == 0) atomicExch(cnt, 0);
-            }
         }
     }
     // Never leave with copies in flight: a timed-out warp stops consuming, so
