@@ -17,10 +17,12 @@ constexpr int kGroup = 8;                 // query heads per KV head
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// Upper bound on polls of one mbarrier phase before a wait gives up.  Each
-// poll is a try_wait with the hardware's own suspend window, so this is far
-// beyond any legitimate copy latency.
-constexpr uint32_t kMaxPolls = 1u << 22;
+// A wait on an mbarrier phase gives up after this many nanoseconds of the
+// GPU's global timer (or after kMaxPolls polls, whichever comes first); far
+// beyond any legitimate copy latency, short enough that a lost copy returns
+// an error instead of holding the GPU.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr uint32_t kMaxPolls = 1u << 26;
 
 __device__ __forceinline__ void report(uint32_t* status, uint32_t bit) {
     if (status) atomicOr(status, bit);
@@ -65,11 +67,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 // Bounded wait for the phase with the given parity to complete.  Returns
-// false if it did not complete within kMaxPolls polls.
+// false if it did not complete within kWaitLimitNs (or kMaxPolls polls).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kMaxPolls; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1; i < kMaxPolls; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
     return false;
 }
 
