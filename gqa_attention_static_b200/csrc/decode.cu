@@ -44,6 +44,8 @@
 // Why tensor cores: per (position, KV head) the kernel reads 512 B and does
 // 2 x 8 x 128 multiply-adds, 4 FMA per byte.  At B200 HBM rates that needs
 // most of the fp32 FMA pipe; on the tensor pipe it is a few percent.
+#include <mutex>
+
 #include "common.cuh"
 #include "tma_host.h"
 
@@ -649,15 +651,9 @@ ark_status device_info(DeviceInfo& out) {
 }
 
 template <int MaxL>
-ark_status launch_decode(DecodeParamsT<MaxL>& prm, const void* const* k, const void* const* v, void* workspace,
-                         size_t ws_bytes, int max_warps, cudaStream_t stream) {
+ark_status launch_decode_core(DecodeParamsT<MaxL>& prm, const void* const* k, const void* const* v, int max_warps,
+                              cudaStream_t stream) {
     DecodeCore& c = prm.c;
-    const WsLayout w = ws_layout(c.L, c.B, c.Hkv);
-    if (!workspace || ws_bytes < w.total || !aligned16(workspace)) return ARK_ERR_WORKSPACE;
-    uint8_t* base = static_cast<uint8_t*>(workspace);
-    c.part_o = reinterpret_cast<float*>(base + w.part_o);
-    c.part_lse = reinterpret_cast<float*>(base + w.part_lse);
-    c.counters = reinterpret_cast<int*>(base + w.counters);
     for (int l = 0; l < c.L; ++l) {
         if (!kv_tensor_map(&prm.kmap[l], k[l], static_cast<long long>(c.B) * c.T, c.Hkv, 64, kTileRows) ||
             !kv_tensor_map(&prm.vmap[l], v[l], static_cast<long long>(c.B) * c.T, c.Hkv, 64, kTileRows))
@@ -675,6 +671,19 @@ ark_status launch_decode(DecodeParamsT<MaxL>& prm, const void* const* k, const v
     if (grid < 1) grid = 1;
     decode_kernel<MaxL><<<static_cast<unsigned>(grid), kWarps * 32, decode_smem(c.B), stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
+}
+
+template <int MaxL>
+ark_status launch_decode(DecodeParamsT<MaxL>& prm, const void* const* k, const void* const* v, void* workspace,
+                         size_t ws_bytes, int max_warps, cudaStream_t stream) {
+    DecodeCore& c = prm.c;
+    const WsLayout w = ws_layout(c.L, c.B, c.Hkv);
+    if (!workspace || ws_bytes < w.total || !aligned16(workspace)) return ARK_ERR_WORKSPACE;
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    c.part_o = reinterpret_cast<float*>(base + w.part_o);
+    c.part_lse = reinterpret_cast<float*>(base + w.part_lse);
+    c.counters = reinterpret_cast<int*>(base + w.counters);
+    return launch_decode_core<MaxL>(prm, k, v, max_warps, stream);
 }
 
 ark_status fill_common(DecodeCore& c, const int32_t* kv_len, int L, int B, int T, int Hq, int Hkv, int D,
@@ -764,4 +773,74 @@ extern "C" ark_status ark_attn_combine(const float* o_part, const float* lse_par
     dim3 cgrid((B * Hq + 3) / 4, 1);
     combine_kernel<<<cgrid, 128, 0, stream>>>(cp);
     return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
+}
+
+// ------------------------------------------------ decode without allocation ----
+// Scratch of ark_attn_decode_noalloc: partial results for up to
+// kNoAllocWarps warps and merge counters for up to kNoAllocMaxSegments
+// (request, KV head) pairs, in one file-scope device array that every GPU
+// loading this library holds until the process exits.  Host code must not pass
+// the array's name to a kernel (on the host it is a stand-in, not a device
+// address); each device's address is looked up once with
+// cudaGetSymbolAddress, with that device current.
+namespace {
+
+constexpr int kNoAllocWarps = 512;
+constexpr int kNoAllocMaxSegments = 4096;
+constexpr size_t kNoAllocPartO = static_cast<size_t>(kNoAllocWarps) * 2 * kGroup * kHeadDim * sizeof(float);
+constexpr size_t kNoAllocPartLse = static_cast<size_t>(kNoAllocWarps) * 2 * kGroup * sizeof(float);
+constexpr size_t kNoAllocCounters = static_cast<size_t>(kNoAllocMaxSegments) * sizeof(int);
+constexpr size_t kNoAllocBytes = kNoAllocPartO + kNoAllocPartLse + kNoAllocCounters;   // about 4.1 MB
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocBytes];
+
+namespace {
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64];
+
+ark_status scratch_address(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARK_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) return ARK_ERR_CUDA;
+        g_scratch_addr[dev] = ptr;
+    }
+    *out = g_scratch_addr[dev];
+    return ARK_OK;
+}
+
+}  // namespace
+
+extern "C" size_t ark_attn_decode_noalloc_scratch_bytes(void) { return kNoAllocBytes; }
+
+extern "C" ark_status ark_attn_decode_noalloc(const void* q, const void* cache_k, const void* cache_v,
+                                              const int32_t* kv_len, int B, int T, int Hq, int Hkv, int D,
+                                              float scale, ark_decode_mode mode, int max_splits, void* o,
+                                              float* lse, uint32_t* d_status, cudaStream_t stream) {
+    if (!q || !cache_k || !cache_v || !o || !lse) return ARK_ERR_INVALID_ARG;
+    DecodeParamsT<1> prm{};
+    ark_status st = fill_common(prm.c, kv_len, 1, B, T, Hq, Hkv, D, scale, mode, max_splits, d_status);
+    if (st != ARK_OK) return st;
+    if (static_cast<long long>(B) * Hkv > kNoAllocMaxSegments) return ARK_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(cache_k) || !aligned16(cache_v) || !aligned16(o) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return ARK_ERR_INVALID_ARG;
+    void* base = nullptr;
+    if ((st = scratch_address(&base)) != ARK_OK) return st;
+    uint8_t* b8 = static_cast<uint8_t*>(base);
+    prm.c.part_o = reinterpret_cast<float*>(b8);
+    prm.c.part_lse = reinterpret_cast<float*>(b8 + kNoAllocPartO);
+    prm.c.counters = reinterpret_cast<int*>(b8 + kNoAllocPartO + kNoAllocPartLse);
+    // the counters must start at zero; the array keeps whatever the last call left
+    if (cudaMemsetAsync(prm.c.counters, 0, static_cast<size_t>(B) * Hkv * sizeof(int), stream) != cudaSuccess)
+        return ARK_ERR_CUDA;
+    prm.q[0] = static_cast<const uint16_t*>(q);
+    prm.o[0] = static_cast<uint16_t*>(o);
+    prm.lse[0] = lse;
+    return launch_decode_core<1>(prm, &cache_k, &cache_v, kNoAllocWarps, stream);
 }

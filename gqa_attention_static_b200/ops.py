@@ -45,6 +45,8 @@ EXPORTS = (
     "ark_attn_append_rope_layers",
     "ark_attn_decode_layers_workspace_size",
     "ark_attn_decode_layers",
+    "ark_attn_decode_noalloc_scratch_bytes",
+    "ark_attn_decode_noalloc",
 )
 
 
@@ -89,6 +91,10 @@ def load() -> ctypes.CDLL:
     lib.ark_attn_decode_layers.argtypes = [I, PP, PP, PP, P, I, I, I, I, I, ctypes.c_float, I, I, P, Z,
                                            PP, PP, P, P]
     lib.ark_attn_decode_layers.restype = I
+    lib.ark_attn_decode_noalloc_scratch_bytes.argtypes = []
+    lib.ark_attn_decode_noalloc_scratch_bytes.restype = Z
+    lib.ark_attn_decode_noalloc.argtypes = [P, P, P, P, I, I, I, I, I, ctypes.c_float, I, I, P, P, P, P]
+    lib.ark_attn_decode_noalloc.restype = I
     _lib = lib
     return lib
 
@@ -313,3 +319,29 @@ def ark_attn_decode_layers(q: Sequence[torch.Tensor], cache_k, cache_v, kv_len, 
                                          _ptr(workspace), ws_bytes, _ptr_array(o), _ptr_array(lse), _ptr(status),
                                          _stream(stream)),
            "ark_attn_decode_layers")
+
+
+# ------------------------------------------------ decode, no allocation ----
+
+def ark_attn_decode_noalloc(q, cache_k, cache_v, kv_len, o, lse, scale: float, mode: int = ARK_LENGTH_AWARE,
+                            max_splits: int = 8, status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """ark_attn_decode without a workspace: the library's own fixed scratch is
+    used (see include/arkattn.h for its limits and the one-stream rule)."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(cache_k, "cache_k", torch.bfloat16, 4)
+    _need(cache_v, "cache_v", torch.bfloat16, 4)
+    _need(kv_len, "kv_len", torch.int32, 1)
+    _need(o, "o", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32)
+    B, S, Hq, D = q.shape
+    if S != 1:
+        raise ValueError("decode takes one query row per request")
+    T, Hkv = cache_k.shape[1], cache_k.shape[2]
+    if tuple(o.shape) != tuple(q.shape) or lse.numel() != B * Hq:
+        raise ValueError("o/lse shape")
+    if status is not None:
+        _need(status, "status", torch.int32)
+    _raise(load().ark_attn_decode_noalloc(_ptr(q), _ptr(cache_k), _ptr(cache_v), _ptr(kv_len), B, T, Hq, Hkv, D,
+                                          float(scale), int(mode), int(max_splits), _ptr(o), _ptr(lse), _ptr(status),
+                                          _stream(stream)),
+           "ark_attn_decode_noalloc")

@@ -200,6 +200,33 @@ ARK_API ark_status ark_attn_decode_layers(int L, const void* const* q, const voi
 ARK_API ark_status ark_attn_combine(const float* o_part, const float* lse_part, int B, int Hq,
                             int nsplit, int D, void* o, float* lse, cudaStream_t stream);
 
+/* ------------------------------------------------- decode, no allocation ----
+ * The pages have no counterpart of this entry point; it exists for callers
+ * that cannot call cudaMalloc (or any allocating routine) at the point where
+ * they decode: code that runs while a CUDA graph is being captured, engines
+ * that reserve all device memory up front and hand out none afterwards, and
+ * plugins whose host framework owns the allocator.  Such a caller still
+ * passes its inputs and outputs, but no workspace.
+ * Same operation, arguments, layouts and results as ark_attn_decode, without
+ * the workspace arguments.  The scratch (partial results and merge counters)
+ * is a fixed array inside the library, ark_attn_decode_noalloc_scratch_bytes()
+ * bytes (about 4.1 MB) on every GPU that loads the library, kept until the
+ * process exits.  It limits a call to B * Hkv <= 4096 (request, KV head)
+ * pairs (ARK_ERR_UNSUPPORTED beyond) and to at most 512 warps, so very large
+ * batches run slower than with ark_attn_decode.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call clears the counters it needs with cudaMemsetAsync on `stream`
+ * and allocates nothing.  All calls share the one array, so calls that can
+ * overlap on the GPU (different streams, or graphs replayed concurrently)
+ * race: serialise them.
+ */
+ARK_API size_t ark_attn_decode_noalloc_scratch_bytes(void);
+ARK_API ark_status ark_attn_decode_noalloc(const void* q, const void* cache_k, const void* cache_v,
+                                           const int32_t* kv_len, int B, int T, int Hq, int Hkv, int D,
+                                           float scale, ark_decode_mode mode, int max_splits, void* o,
+                                           float* lse, uint32_t* d_status, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
