@@ -1,0 +1,416 @@
+// prefill.cu -- causal GQA prefill of the prompt on the 5th-generation tensor
+// cores (tcgen05, accumulators in tensor memory, operands staged by TMA).
+//
+// The ONNX model card ("ARK-ASR-3B -- INT8 ONNX", sections Shapes and
+// Inference) runs the whole audio+text prompt through the decoder in one call
+// ("Prefill, then decode"); each call's key/value rows are written into the
+// static cache at cache_position.  Here the rows are already appended (by
+// ark_attn_append_rope) and query row t of request b, at absolute position
+// p = pos0[b] + t, attends to the cache rows j <= p of its KV head.
+//
+// Tiling (B200):
+//   - One CTA per (16 query positions, KV head g, request b).  Its 128 MMA
+//     rows are the 16 positions x the 8 query heads of group g, so every K/V
+//     block is read once for all 8 heads (GQA packing).  The Q tile arrives
+//     by two 4-D TMA boxes (64 head-dim elements each, 128-byte swizzle),
+//     already in the K-major layout tcgen05 reads.
+//   - KV blocks of 128 keys stream through a 2-stage ring (TMA, 3-D boxes
+//     over the cache).  S = Q K^T for a block is 8 MMAs of 128x128x16 into a
+//     TMEM buffer (two buffers, so QK of block j+1 overlaps the softmax of
+//     block j); O += P V is 8 MMAs with V as an MN-major operand (no
+//     transpose), accumulated in TMEM.
+//   - Warp roles: warp 0 issues TMA (and owns the TMEM allocation), warp 1
+//     issues MMAs from one thread, warps 2..5 run the softmax: thread r owns
+//     TMEM lane r, i.e. one query row, so row max and row sum need no
+//     shuffles.  P (bf16) goes to shared memory in the swizzled K-major
+//     layout and feeds the PV MMA.
+//   - Softmax in the log2 domain with a lazily moved reference max: O is
+//     rescaled (read, scale, write back in TMEM) only when a row's block max
+//     exceeds its reference by more than 2^8, which for real data is almost
+//     never after the first block.  Rows past n_new[b] are computed on
+//     whatever the padded q holds and never written.
+//   - Only the last block needs the causal mask; V rows past the causal range
+//     of the tile are zeroed in shared memory before their (zero-weight) use,
+//     so garbage past the valid rows cannot turn into NaN.
+//
+// Roofline: per request of L prompt rows and per layer, 4096 * L * (L + 1)
+// FLOPs (the causal half of QK^T and PV for 16 heads) against 9216 * L bytes
+// (q read, o written, K/V rows read once per tile from L2); at the prompt
+// lengths of the coalesced-prefill workload (<= 387) that is HBM- and
+// latency-bound rather than tensor-bound.
+#include "common.cuh"
+#include "tma_host.h"
+
+namespace ark {
+namespace pf {
+
+constexpr int kRows = 128;               // MMA M: 16 positions x 8 heads
+constexpr int kPos = 16;                 // query positions per tile
+constexpr int kBN = 128;                 // keys per KV block
+constexpr int kHalf = kRows * 128;       // one 64-element half of a 128-row tile (16 KB)
+constexpr int kTile = 2 * kHalf;         // a 128 x 128 bf16 tile (32 KB)
+constexpr int kThreads = 192;            // warp 0: TMA, warp 1: MMA, warps 2..5: softmax
+
+// shared memory map (offsets from a 1024-aligned base)
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kTile;     // 2 stages
+constexpr int kOffV = kOffK + 2 * kTile; // 2 stages
+constexpr int kOffP = kOffV + 2 * kTile;
+constexpr int kOffBar = kOffP + kTile;
+constexpr int kNumBars = 10;
+constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
+constexpr int kOffFlag = kOffTmemPtr + 8;
+constexpr int kSmemBytes = 1024 + kOffFlag + 16;
+
+// bar indices
+constexpr int kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarSFull = 5, kBarPFull = 7, kBarPvDone = 8;
+
+// TMEM columns
+constexpr uint32_t kColS = 0;            // two S buffers: 0..127, 128..255
+constexpr uint32_t kColO = 256;          // O: 256..383
+constexpr uint32_t kTmemCols = 512;
+
+// instruction descriptors (kind::f16): D fp32, A/B bf16, M = 128, N = 128
+constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescQK = kIdescBase;               // A = Q (K-major), B = K (K-major)
+constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);  // A = P (K-major), B = V (MN-major)
+
+constexpr float kLazyRescale = 8.0f;     // log2 units: rescale O only past a factor 2^8
+
+struct Params {
+    CUtensorMap qmap;    // q as (128, 8, Hq/8, B*S), box (64, 8, 1, 16)
+    CUtensorMap kmap;    // cache_k as (128, Hkv, B*T), box (64, 1, 128)
+    CUtensorMap vmap;
+    uint16_t* o;         // [B, S, Hq, 128]
+    float* lse;          // [B, Hq, S]
+    const int32_t* pos0;
+    const int32_t* n_new;
+    uint32_t* status;
+    int B, S, T, Hq, Hkv;
+    float scale_log2;
+};
+
+}  // namespace pf
+
+__global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_constant__ pf::Params p) {
+    using namespace pf;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int qt = blockIdx.x;
+    const int g = blockIdx.y;
+    const int b = blockIdx.z;
+
+    // ---- lengths (device values: checked here)
+    int nn = __ldg(p.n_new + b);
+    int p0 = __ldg(p.pos0 + b);
+    if (nn < 0 || nn > p.S || p0 < 0 || p0 + (nn < 0 ? 0 : (nn > p.S ? p.S : nn)) > p.T) {
+        if (threadIdx.x == 0 && qt == 0 && g == 0) report(p.status, ARK_DEV_BAD_POS);
+        nn = nn < 0 ? 0 : (nn > p.S ? p.S : nn);
+        if (p0 < 0) p0 = 0;
+        if (p0 > p.T) p0 = p.T;
+        if (p0 + nn > p.T) nn = p.T - p0;
+    }
+    const int t0 = qt * kPos;
+    if (t0 >= nn) return;                                   // whole CTA: no live row
+    const int kv_end = p0 + min(t0 + kPos, nn);             // keys visible to the tile's last row
+    const int nblk = (kv_end + kBN - 1) / kBN;
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
+    int* failed_flag = reinterpret_cast<int*>(smem + kOffFlag);
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[kBarQ], 1);
+        mbar_init(&bars[kBarKvFull], 1);
+        mbar_init(&bars[kBarKvFull + 1], 1);
+        mbar_init(&bars[kBarKvEmpty], 1);
+        mbar_init(&bars[kBarKvEmpty + 1], 1);
+        mbar_init(&bars[kBarSFull], 1);
+        mbar_init(&bars[kBarSFull + 1], 1);
+        mbar_init(&bars[kBarPFull], 128);
+        mbar_init(&bars[kBarPvDone], 1);
+        *failed_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_ptr, kTmemCols);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_ptr;
+    const uint32_t sbase = smem_u32(smem);
+
+    if (warp == 0) {
+        // ================================================= TMA producer
+        if (lane == 0) {
+            bool ok = true;
+            mbar_arrive_expect_tx(&bars[kBarQ], kTile);
+            const int qrow = b * p.S + t0;
+            tma_load_4d(smem + kOffQ, &p.qmap, 0, 0, g, qrow, &bars[kBarQ]);
+            tma_load_4d(smem + kOffQ + kHalf, &p.qmap, 64, 0, g, qrow, &bars[kBarQ]);
+            for (int j = 0; j < nblk && ok; ++j) {
+                const int st = j & 1;
+                if (j >= 2 && !mbar_wait(&bars[kBarKvEmpty + st], ((j >> 1) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                uint64_t* full = &bars[kBarKvFull + st];
+                mbar_arrive_expect_tx(full, 2 * kTile);
+                const int row = b * p.T + j * kBN;
+                uint8_t* kd = smem + kOffK + st * kTile;
+                uint8_t* vd = smem + kOffV + st * kTile;
+                tma_load_3d(kd, &p.kmap, 0, g, row, full);
+                tma_load_3d(kd + kHalf, &p.kmap, 64, g, row, full);
+                tma_load_3d(vd, &p.vmap, 0, g, row, full);
+                tma_load_3d(vd + kHalf, &p.vmap, 64, g, row, full);
+            }
+            if (!ok) {
+                atomicExch(failed_flag, 1);
+                report(p.status, ARK_DEV_TIMEOUT);
+            }
+        }
+    } else if (warp == 1) {
+        // ================================================= MMA issuer
+        bool ok = mbar_wait(&bars[kBarQ], 0);
+        auto wait_kv = [&](int j) {
+            // K/V block j landed; zero the V rows past the tile's causal range
+            if (!mbar_wait(&bars[kBarKvFull + (j & 1)], (j >> 1) & 1)) return false;
+            const int live = kv_end - j * kBN;
+            if (live < kBN) {
+                uint8_t* vt = smem + kOffV + (j & 1) * kTile;
+                for (int i = lane; i < (kBN - live) * 16; i += 32) {
+                    const int r = live + (i >> 4), part = i & 15;
+                    *reinterpret_cast<uint4*>(vt + (part >> 3) * kHalf + r * 128 + (part & 7) * 16) =
+                        make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            return true;
+        };
+        auto issue_qk = [&](int j) {
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t d = tmem + kColS + (j & 1) * kBN;
+                const uint32_t kb = sbase + kOffK + (j & 1) * kTile;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+                    umma_f16(d, umma_desc_sw128(sbase + kOffQ + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024),
+                             kIdescQK, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&bars[kBarSFull + (j & 1)]);
+            }
+            __syncwarp();
+        };
+        auto issue_pv = [&](int j) {
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t vb = sbase + kOffV + (j & 1) * kTile;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t aoff = (kk >> 2) * kHalf + (kk & 3) * 32;
+                    umma_f16(tmem + kColO, umma_desc_sw128(sbase + kOffP + aoff, 16, 1024),
+                             umma_desc_sw128(vb + kk * 16 * 128, kHalf, 1024), kIdescPV,
+                             (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&bars[kBarKvEmpty + (j & 1)]);
+                umma_commit(&bars[kBarPvDone]);
+            }
+            __syncwarp();
+        };
+        if (ok) ok = wait_kv(0);
+        if (ok) issue_qk(0);
+        for (int j = 0; j < nblk && ok; ++j) {
+            if (j + 1 < nblk) {
+                // S buffer (j+1)&1 was last read by the softmax of block j-1 (waited below at j-1)
+                if (!(ok = wait_kv(j + 1))) break;
+                issue_qk(j + 1);
+            }
+            if (!(ok = mbar_wait(&bars[kBarPFull], j & 1))) break;
+            issue_pv(j);
+        }
+        if (!ok && lane == 0) {
+            atomicExch(failed_flag, 1);
+            report(p.status, ARK_DEV_TIMEOUT);
+        }
+    } else {
+        // ================================================= softmax + epilogue
+        const int quad = warp & 3;                      // TMEM lanes 32*quad .. +31
+        const int r = quad * 32 + lane;                 // this thread's row of the tile
+        const int tr = t0 + (r >> 3);                   // its query position (within the call)
+        const int hh = r & 7;
+        const int prow = p0 + tr;                       // its absolute position
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+        float m_ref = -INFINITY, e_sum = 0.f, r_sum = 0.f;
+        bool ok = true;
+        uint8_t* prow_smem = smem + kOffP + r * 128;
+        for (int j = 0; j < nblk && ok; ++j) {
+            if (!(ok = mbar_wait(&bars[kBarSFull + (j & 1)], (j >> 1) & 1))) break;
+            tc_fence_after();
+            const uint32_t scol = lane_base + kColS + (j & 1) * kBN;
+            const int kbase = j * kBN;
+            const int nvalid = min(kBN, prow - kbase + 1);   // keys kbase .. prow of this block
+            // pass 1: block max of the visible scores
+            float bm = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                tmem_ld32(scol + c * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (c * 32 + i < nvalid) bm = fmaxf(bm, __uint_as_float(v[i]));
+            }
+            bm *= p.scale_log2;
+            float alpha = 1.f;
+            bool rescale = false;
+            if (m_ref == -INFINITY) {
+                m_ref = bm;
+            } else if (bm > m_ref + kLazyRescale) {
+                alpha = fast_exp2(m_ref - bm);
+                m_ref = bm;
+                rescale = true;
+            }
+            const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+            // the P buffer and O are free once PV of block j-1 has completed
+            if (j >= 1 && !(ok = mbar_wait(&bars[kBarPvDone], (j - 1) & 1))) break;
+            tc_fence_after();
+            if (rescale) {
+                e_sum *= alpha;
+                r_sum *= alpha;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_base + kColO + c * 32, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+                    tmem_st32(lane_base + kColO + c * 32, v);
+                }
+                tmem_wait_st();
+            }
+            // pass 2: P = exp2(s * scale_log2 - m_ref) as bf16 into the swizzled K-major P tile
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                tmem_ld32(scol + c * 32, v);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const float s0 = (c * 32 + i < nvalid) ? fast_exp2(__uint_as_float(v[i]) * p.scale_log2 - mu) : 0.f;
+                    const float s1 =
+                        (c * 32 + i + 1 < nvalid) ? fast_exp2(__uint_as_float(v[i + 1]) * p.scale_log2 - mu) : 0.f;
+                    const __nv_bfloat162 pb = __floats2bfloat162_rn(s0, s1);
+                    e_sum += s0 + s1;
+                    r_sum += __low2float(pb) + __high2float(pb);
+                    pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&pb);
+                }
+                // keys c*32 .. c*32+31: half c/2, 16-byte chunks 4*(c&1) .. +3
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int chunk = 4 * (c & 1) + q;
+                    *reinterpret_cast<uint4*>(prow_smem + (c >> 1) * kHalf + ((chunk ^ (r & 7)) << 4)) =
+                        make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                }
+            }
+            fence_proxy_async_smem();      // P is read by the tensor core (async proxy)
+            tc_fence_before();
+            mbar_arrive(&bars[kBarPFull]);
+        }
+        if (ok) ok = mbar_wait(&bars[kBarPvDone], (nblk - 1) & 1);
+        tc_fence_after();
+        if (!ok) {
+            atomicExch(failed_flag, 1);
+            if (lane == 0) report(p.status, ARK_DEV_TIMEOUT);
+        } else if (tr < nn) {
+            // epilogue: o row = O / sum of the bf16 weights; lse from the fp32 weights
+            const float inv = 1.f / r_sum;
+            const int h = g * kGroup + hh;
+            uint16_t* orow = p.o + ((static_cast<size_t>(b) * p.S + tr) * p.Hq + h) * kHeadDim;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                tmem_ld32(lane_base + kColO + c * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint4 w;
+                    w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv);
+                    w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv);
+                    w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv);
+                    w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv);
+                    reinterpret_cast<uint4*>(orow + c * 32)[q] = w;
+                }
+            }
+            p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + tr] = (m_ref + __log2f(e_sum)) * kLn2;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        if (*failed_flag) {
+            // do not release shared or tensor memory under copies or MMAs still in flight
+            for (int s = 0; s < 2; ++s) (void)mbar_wait(&bars[kBarKvFull + s], 0);
+            (void)mbar_wait(&bars[kBarPvDone], (nblk - 1) & 1);
+        }
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace ark
+
+using namespace ark;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool g_prefill_attr[64];
+
+}  // namespace
+
+extern "C" ark_status ark_attn_prefill(const void* q, const void* cache_k, const void* cache_v,
+                                       const int32_t* pos0, const int32_t* n_new, int B, int S, int T, int Hq,
+                                       int Hkv, int D, float scale, void* o, float* lse, uint32_t* d_status,
+                                       cudaStream_t stream) {
+    if (!q || !cache_k || !cache_v || !pos0 || !n_new || !o || !lse) return ARK_ERR_INVALID_ARG;
+    if (B <= 0 || S <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || !(scale > 0.f)) return ARK_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return ARK_ERR_INVALID_ARG;
+    if (D != kHeadDim || Hq / Hkv != kGroup) return ARK_ERR_UNSUPPORTED;
+    if (T > ARK_MAX_T || B > 65535 || Hkv > 65535) return ARK_ERR_UNSUPPORTED;
+    if (static_cast<long long>(B) * S >= (1LL << 31) || static_cast<long long>(B) * T >= (1LL << 31))
+        return ARK_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(cache_k) || !aligned16(cache_v) || !aligned16(o) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return ARK_ERR_INVALID_ARG;
+    pf::Params prm{};
+    if (!q_group_tensor_map(&prm.qmap, q, static_cast<long long>(B) * S, Hq, 64, pf::kPos) ||
+        !kv_tensor_map(&prm.kmap, cache_k, static_cast<long long>(B) * T, Hkv, 64, pf::kBN) ||
+        !kv_tensor_map(&prm.vmap, cache_v, static_cast<long long>(B) * T, Hkv, 64, pf::kBN))
+        return ARK_ERR_CUDA;
+    prm.o = static_cast<uint16_t*>(o);
+    prm.lse = lse;
+    prm.pos0 = pos0;
+    prm.n_new = n_new;
+    prm.status = d_status;
+    prm.B = B; prm.S = S; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
+    prm.scale_log2 = scale * kLog2e;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARK_ERR_CUDA;
+    if (!g_prefill_attr[dev]) {
+        if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::kSmemBytes) !=
+            cudaSuccess)
+            return ARK_ERR_CUDA;
+        g_prefill_attr[dev] = true;
+    }
+    dim3 grid((S + pf::kPos - 1) / pf::kPos, Hkv, B);
+    prefill_kernel<<<grid, pf::kThreads, pf::kSmemBytes, stream>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
+}

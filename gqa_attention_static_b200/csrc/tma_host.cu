@@ -64,7 +64,7 @@ bool cached_encode(const Key& key, CUtensorMap* out, cuuint32_t rank, const cuui
     }
     EncodeFn fn = encode_fn();
     if (!fn) return false;
-    const cuuint32_t es[3] = {1, 1, 1};
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
     CUtensorMap m;
     if (fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, reinterpret_cast<void*>(key.base), dims, strides, box, es,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -85,6 +85,14 @@ bool kv_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv, 
     const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(Hkv) * 256};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 1, static_cast<cuuint32_t>(box_rows)};
     return cached_encode(key, out, 3, dims, strides, box);
+}
+
+bool q_group_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hq, int box_inner, int box_rows) {
+    const Key key{reinterpret_cast<uintptr_t>(base), rows, 2, Hq, box_inner, box_rows};
+    const cuuint64_t dims[4] = {128, 8, static_cast<cuuint64_t>(Hq / 8), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[3] = {256, 2048, static_cast<cuuint64_t>(Hq) * 256};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(box_inner), 8, 1, static_cast<cuuint32_t>(box_rows)};
+    return cached_encode(key, out, 4, dims, strides, box);
 }
 
 bool rows_tensor_map(CUtensorMap* out, const void* base, long long rows, int box_inner, int box_rows) {

@@ -17,4 +17,10 @@ bool kv_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv, 
 // box (box_inner elements, box_rows rows), 128-byte swizzle.
 bool rows_tensor_map(CUtensorMap* out, const void* base, long long rows, int box_inner, int box_rows);
 
+// 4-D tiled map over q [B, S, Hq, 128] bf16 viewed as (dim 0: 128 head-dim
+// elements, dim 1: 8 heads of a group, dim 2: Hq/8 groups, dim 3: B*S rows),
+// box (box_inner, 8, 1, box_rows), 128-byte swizzle: one box lands as
+// box_rows x 8 rows of box_inner elements, ordered (position, head).
+bool q_group_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hq, int box_inner, int box_rows);
+
 }  // namespace ark

@@ -42,6 +42,7 @@ EXPORTS = (
     "ark_attn_decode_workspace_size",
     "ark_attn_decode",
     "ark_attn_combine",
+    "ark_attn_prefill",
     "ark_attn_append_rope_layers",
     "ark_attn_decode_layers_workspace_size",
     "ark_attn_decode_layers",
@@ -83,6 +84,8 @@ def load() -> ctypes.CDLL:
     lib.ark_attn_decode.restype = I
     lib.ark_attn_combine.argtypes = [P, P, I, I, I, I, P, P, P]
     lib.ark_attn_combine.restype = I
+    lib.ark_attn_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, I, ctypes.c_float, P, P, P, P]
+    lib.ark_attn_prefill.restype = I
     PP = ctypes.POINTER(ctypes.c_void_p)
     lib.ark_attn_append_rope_layers.argtypes = [I, PP, PP, PP, PP, PP, P, P, I, I, I, I, I, I, P, P, P]
     lib.ark_attn_append_rope_layers.restype = I
@@ -239,6 +242,32 @@ def ark_attn_combine(o_part, lse_part, o, lse, stream=None) -> None:
     _raise(load().ark_attn_combine(_ptr(o_part), _ptr(lse_part), B, Hq, nsplit, D, _ptr(o), _ptr(lse),
                                    _stream(stream)),
            "ark_attn_combine")
+
+
+# --------------------------------------------------------------- prefill ----
+
+def ark_attn_prefill(q, cache_k, cache_v, pos0, n_new, o, lse, scale: float,
+                     status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Causal prefill: q [B,S,Hq,D] (rotated) over the cache -> o [B,S,Hq,D]
+    bf16 (rows t >= n_new[b] untouched), lse [B,Hq,S] fp32."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(cache_k, "cache_k", torch.bfloat16, 4)
+    _need(cache_v, "cache_v", torch.bfloat16, 4)
+    _need(pos0, "pos0", torch.int32, 1)
+    _need(n_new, "n_new", torch.int32, 1)
+    _need(o, "o", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    B, S, Hq, D = q.shape
+    T, Hkv = cache_k.shape[1], cache_k.shape[2]
+    if tuple(o.shape) != tuple(q.shape) or lse.numel() != B * Hq * S:
+        raise ValueError("o/lse shape")
+    if tuple(cache_v.shape) != tuple(cache_k.shape) or cache_k.shape[0] != B:
+        raise ValueError("cache shape")
+    _raise(load().ark_attn_prefill(_ptr(q), _ptr(cache_k), _ptr(cache_v), _ptr(pos0), _ptr(n_new), B, S, T, Hq,
+                                   Hkv, D, float(scale), _ptr(o), _ptr(lse), _ptr(status), _stream(stream)),
+           "ark_attn_prefill")
 
 
 # ------------------------------------------------- layer-batched variants ----

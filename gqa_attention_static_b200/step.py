@@ -92,3 +92,45 @@ class DecodeStep:
         """The decode attention of every layer without the append (for timing
         the dominant kernel alone)."""
         self.attention(stream)
+
+
+class PrefillStep:
+    """Prefill of one prompt batch over L independent layers: RoPE + delta
+    write of the prompt rows for all layers (one launch), then the causal
+    tcgen05 prefill of each layer (one launch per layer).
+
+    Buffers (per layer lists): q [B,S,Hq,D] (rotated in place), k_new/v_new
+    [B,S,Hkv,D], cache_k/cache_v [B,T,Hkv,D]; outputs o [B,S,Hq,D] bf16 and
+    lse [B,Hq,S] fp32 (rows t >= n_new[b] are not written).
+    """
+
+    def __init__(self, q, k_new, v_new, cache_k, cache_v, pos0, n_new, rope_theta: float = 1e6,
+                 scale: Optional[float] = None):
+        self.q, self.k_new, self.v_new = q, k_new, v_new
+        self.cache_k, self.cache_v = cache_k, cache_v
+        self.pos0, self.n_new = pos0, n_new
+        self.layers = len(q)
+        self.B, self.S, self.Hq, self.D = q[0].shape
+        self.T = cache_k[0].shape[1]
+        dev = q[0].device
+        self.scale = scale if scale is not None else 1.0 / math.sqrt(self.D)
+        self.table = ops.rope_table(self.T, self.D, rope_theta, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.o = [torch.empty_like(x) for x in q]
+        self.lse = [torch.empty(self.B, self.Hq, self.S, dtype=torch.float32, device=dev) for _ in q]
+
+    def launches_per_step(self) -> int:
+        return 1 + self.layers
+
+    def append(self, stream=None) -> None:
+        ops.ark_attn_append_rope_layers(self.q, self.k_new, self.v_new, self.cache_k, self.cache_v, self.pos0,
+                                        self.n_new, self.table, self.status, stream)
+
+    def attention(self, stream=None) -> None:
+        for l in range(self.layers):
+            ops.ark_attn_prefill(self.q[l], self.cache_k[l], self.cache_v[l], self.pos0, self.n_new, self.o[l],
+                                 self.lse[l], self.scale, self.status, stream)
+
+    def run(self, stream=None) -> None:
+        self.append(stream)
+        self.attention(stream)

@@ -160,6 +160,27 @@ ARK_API ark_status ark_attn_decode(const void* q, const void* cache_k, const voi
                                    void* workspace, size_t workspace_bytes,
                                    void* o, float* lse, uint32_t* d_status, cudaStream_t stream);
 
+/* --------------------------------------------------------------- prefill ----
+ * Causal prefill of a prompt ("ARK-ASR-3B -- INT8 ONNX", section Inference:
+ * the audio+text prompt is prefilled, then decoded; section Shapes: the
+ * call's rows are written into the static cache at cache_position).  Call it
+ * after ark_attn_append_rope has rotated q and written this call's K/V rows.
+ * For request b and new row t < n_new[b], at position p = pos0[b] + t, and
+ * each query head h (KV head g = h / (Hq/Hkv)):
+ *   o[b,t,h,:] = sum_{j <= p} softmax_j(scale * <q[b,t,h,:], cache_k[b,j,g,:]>) cache_v[b,j,g,:]
+ *   lse[b,h,t] = ln sum_{j <= p} exp(scale * <q[b,t,h,:], cache_k[b,j,g,:]>)
+ * Layouts: q [B,S,Hq,D] bf16 (rotated); cache_k, cache_v [B,T,Hkv,D] bf16;
+ * pos0, n_new int32[B] (device); o [B,S,Hq,D] bf16; lse [B,Hq,S] fp32.
+ * Rows t >= n_new[b] of o and lse are not written.  n_new outside [0, S] or
+ * pos0 + n_new > T is clamped and sets ARK_DEV_BAD_POS.  The 5th-generation
+ * tensor cores (tcgen05) compute Q K^T and P V with fp32 accumulation in
+ * tensor memory; the softmax weights are rounded to bf16 before P V.
+ */
+ARK_API ark_status ark_attn_prefill(const void* q, const void* cache_k, const void* cache_v,
+                                    const int32_t* pos0, const int32_t* n_new, int B, int S, int T,
+                                    int Hq, int Hkv, int D, float scale, void* o, float* lse,
+                                    uint32_t* d_status, cudaStream_t stream);
+
 /* -------------------------------------------------- layer-batched variants ----
  * The same operations over L <= ARK_MAX_LAYERS independent layers in ONE
  * launch.  Every pointer argument that is per layer is a HOST array of L

@@ -1,0 +1,130 @@
+"""Causal prefill on the tcgen05 tensor cores against the fp64 oracle.
+
+The prompt's rows are appended (RoPE + delta write) and then prefilled, on the
+GPU through the C ABI and in the oracle from the same inputs
+("ARK-ASR-3B -- INT8 ONNX", sections Inference and Shapes: prefill of the
+audio+text prompt, rows written at cache_position)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gqa_attention_static_b200 import ops
+from gqa_attention_static_b200 import workloads as W
+from tests.helpers import bits, check_lse, check_o, f64
+
+pytestmark = pytest.mark.gpu
+
+SCALE = 1.0 / math.sqrt(128)
+SENTINEL = 0x7FC1            # a NaN pattern no kernel writes
+
+
+def gpu_append_prefill(batch, layer=0, status=None):
+    dev = "cuda"
+    q = batch.q[layer].to(dev).clone()
+    ck = batch.cache_k[layer].to(dev).clone()
+    cv = batch.cache_v[layer].to(dev).clone()
+    pos0 = batch.pos0.to(dev)
+    n_new = batch.n_new.to(dev)
+    table = ops.rope_table(batch.T)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ops.ark_attn_append_rope(q, batch.k_new[layer].to(dev), batch.v_new[layer].to(dev), ck, cv, pos0, n_new,
+                             table, status)
+    B, S, Hq, D = q.shape
+    o = torch.empty_like(q).view(torch.int16).fill_(SENTINEL).view(torch.bfloat16)
+    lse = torch.full((B, Hq, S), float("nan"), dtype=torch.float32, device=dev)
+    ops.ark_attn_prefill(q, ck, cv, pos0, n_new, o, lse, SCALE, status)
+    torch.cuda.synchronize()
+    return q, ck, cv, o, lse, int(status.item())
+
+
+def oracle_append_prefill(batch, layer=0):
+    q_rot, ck, cv, skipped = oracle.append_rope(bits(batch.q[layer]), bits(batch.k_new[layer]),
+                                                bits(batch.v_new[layer]), bits(batch.cache_k[layer]),
+                                                bits(batch.cache_v[layer]), batch.pos0.numpy(), batch.n_new.numpy())
+    o, lse = oracle.prefill(q_rot, ck, cv, batch.pos0.numpy(), batch.n_new.numpy(), SCALE)
+    return q_rot, ck, cv, o, lse
+
+
+def compare(batch, layer=0, status_expected=0):
+    q, ck, cv, o, lse, st = gpu_append_prefill(batch, layer)
+    q_ref, ck_ref, cv_ref, o_ref, lse_ref = oracle_append_prefill(batch, layer)
+    assert st == status_expected
+    assert np.array_equal(bits(q), q_ref) and np.array_equal(bits(ck), ck_ref) and np.array_equal(bits(cv), cv_ref)
+    ob = bits(o)
+    of = f64(o)
+    lf = f64(lse)
+    for b in range(batch.B):
+        n = int(batch.n_new[b])
+        check_o(of[b, :n], o_ref[b, :n], f"o request {b}")
+        check_lse(lf[b, :, :n], lse_ref[b, :, :n], f"lse request {b}")
+        # rows past n_new are not written
+        assert np.all(ob[b, n:] == SENTINEL), f"request {b}: padded rows were written"
+        assert np.all(np.isnan(lf[b, :, n:]))
+
+
+@pytest.mark.parametrize("B,S,T,pos0,n_new", [
+    (3, 40, 256, [0, 30, 100], [40, 17, 1]),         # ragged tails, tiles of 16 positions
+    (2, 16, 64, [0, 48], [16, 16]),                  # exact one tile, cache ending at T
+    (1, 5, 8, [3], [5]),                             # smaller than a tile and than a KV block
+    (2, 130, 512, [0, 380], [130, 2]),               # two KV blocks, last one partial
+    (1, 200, 2048, [1700], [200]),                   # long context: 15 KV blocks
+])
+def test_prefill_small_cases(oracle_lib, B, S, T, pos0, n_new):
+    batch = W.make_batch(500 + S + T, B=B, S=S, T=T, pos0=pos0, n_new=n_new, garbage="nan")
+    compare(batch)
+
+
+def test_prefill_sweep_prompt(oracle_lib):
+    """The batch-1 prompt of the autoregressive sweep: 50 rows from position 0."""
+    batch = W.cfg_sweep_prefill(layers=2)
+    for layer in range(2):
+        compare(batch, layer)
+
+
+def test_prefill_coalesced_batch_full_size(oracle_lib):
+    """Coalesced prefill at its full size: 16 prompts of 20..387 rows, T=512."""
+    batch = W.cfg_prefill(layers=1)
+    compare(batch)
+
+
+def test_prefill_outliers(oracle_lib):
+    batch = W.make_batch(77, B=4, S=64, T=128, pos0=[0, 10, 60, 64], n_new=[64, 50, 3, 64], outliers="row")
+    compare(batch)
+
+
+def test_prefill_rows_match_decode(oracle_lib):
+    """Causal consistency on the GPU: prefill row t equals a decode over
+    pos0 + t + 1 rows of the same cache (both within tolerance of each other)."""
+    batch = W.make_batch(91, B=2, S=24, T=128, pos0=[0, 40], n_new=[24, 20])
+    q, ck, cv, o, lse, st = gpu_append_prefill(batch)
+    assert st == 0
+    dev = "cuda"
+    for b in range(2):
+        for t in range(int(batch.n_new[b])):
+            kv = torch.tensor([int(batch.pos0[b]) + t + 1], dtype=torch.int32, device=dev)
+            qd = q[b:b + 1, t:t + 1].contiguous()
+            od = torch.empty_like(qd)
+            ld = torch.empty(1, 16, dtype=torch.float32, device=dev)
+            ws = ops.decode_workspace(1, 16, 128, 128, 8, device=dev)
+            ops.ark_attn_decode(qd, ck[b:b + 1].contiguous(), cv[b:b + 1].contiguous(), kv, od, ld, SCALE,
+                                ops.ARK_LENGTH_AWARE, 8, ws)
+            torch.cuda.synchronize()
+            check_o(f64(o[b, t]), f64(od[0, 0]), "prefill vs decode")
+            check_lse(f64(lse[b, :, t]), f64(ld[0]), "prefill vs decode lse")
+
+
+def test_prefill_bad_lengths_set_status(oracle_lib):
+    batch = W.make_batch(92, B=2, S=8, T=16, pos0=[12, 0], n_new=[8, 4])   # 12 + 8 > 16
+    dev = "cuda"
+    q = batch.q[0].to(dev)
+    ck = batch.cache_k[0].to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(2, 16, 8, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ops.ark_attn_prefill(q, ck, ck, batch.pos0.to(dev), batch.n_new.to(dev), o, lse, SCALE, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & ops.ARK_DEV_BAD_POS
