@@ -174,10 +174,11 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
         }
     } else if (warp == 1) {
         // ================================================= MMA issuer
-        bool ok = mbar_wait(&bars[kBarQ], 0);
+        // waits are AND-ed over the warp so that the __syncwarp()s below are reached by all lanes
+        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarQ], 0));
         auto wait_kv = [&](int j) {
             // K/V block j landed; zero the V rows past the tile's causal range
-            if (!mbar_wait(&bars[kBarKvFull + (j & 1)], (j >> 1) & 1)) return false;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarKvFull + (j & 1)], (j >> 1) & 1))) return false;
             const int live = kv_end - j * kBN;
             if (live < kBN) {
                 uint8_t* vt = smem + kOffV + (j & 1) * kTile;
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
                 if (!(ok = wait_kv(j + 1))) break;
                 issue_qk(j + 1);
             }
-            if (!(ok = mbar_wait(&bars[kBarPFull], j & 1))) break;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPFull], j & 1)))) break;
             issue_pv(j);
         }
         if (!ok && lane == 0) {
@@ -248,8 +249,12 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
         float m_ref = -INFINITY, e_sum = 0.f, r_sum = 0.f;
         bool ok = true;
         uint8_t* prow_smem = smem + kOffP + r * 128;
+        // Every tcgen05.ld/st below is .sync.aligned: all 32 lanes of the warp
+        // execute it together, so all control flow around them is warp-uniform
+        // (ok is AND-ed over the warp; per-row choices become per-lane values).
         for (int j = 0; j < nblk && ok; ++j) {
-            if (!(ok = mbar_wait(&bars[kBarSFull + (j & 1)], (j >> 1) & 1))) break;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + (j & 1)], (j >> 1) & 1));
+            if (!ok) break;
             tc_fence_after();
             const uint32_t scol = lane_base + kColS + (j & 1) * kBN;
             const int kbase = j * kBN;
@@ -277,9 +282,12 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
             }
             const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
             // the P buffer and O are free once PV of block j-1 has completed
-            if (j >= 1 && !(ok = mbar_wait(&bars[kBarPvDone], (j - 1) & 1))) break;
+            if (j >= 1) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPvDone], (j - 1) & 1));
+                if (!ok) break;
+            }
             tc_fence_after();
-            if (rescale) {
+            if (__any_sync(0xffffffffu, rescale)) {       // lanes that need none scale by 1
                 e_sum *= alpha;
                 r_sum *= alpha;
 #pragma unroll
@@ -322,13 +330,15 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
             tc_fence_before();
             mbar_arrive(&bars[kBarPFull]);
         }
-        if (ok) ok = mbar_wait(&bars[kBarPvDone], (nblk - 1) & 1);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPvDone], (nblk - 1) & 1));
         tc_fence_after();
         if (!ok) {
             atomicExch(failed_flag, 1);
             if (lane == 0) report(p.status, ARK_DEV_TIMEOUT);
-        } else if (tr < nn) {
-            // epilogue: o row = O / sum of the bf16 weights; lse from the fp32 weights
+        } else {
+            // epilogue: o row = O / sum of the bf16 weights; lse from the fp32 weights.
+            // All lanes read TMEM; only rows of live positions are stored.
+            const bool live = tr < nn;
             const float inv = 1.f / r_sum;
             const int h = g * kGroup + hh;
             uint16_t* orow = p.o + ((static_cast<size_t>(b) * p.S + tr) * p.Hq + h) * kHeadDim;
@@ -337,17 +347,19 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
                 uint32_t v[32];
                 tmem_ld32(lane_base + kColO + c * 32, v);
                 tmem_wait_ld();
+                if (live) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint4 w;
-                    w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv);
-                    w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv);
-                    w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv);
-                    w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv);
-                    reinterpret_cast<uint4*>(orow + c * 32)[q] = w;
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv);
+                        w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv);
+                        w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv);
+                        w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv);
+                        reinterpret_cast<uint4*>(orow + c * 32)[q] = w;
+                    }
                 }
             }
-            p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + tr] = (m_ref + __log2f(e_sum)) * kLn2;
+            if (live) p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + tr] = (m_ref + __log2f(e_sum)) * kLn2;
         }
     }
 
