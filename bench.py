@@ -52,7 +52,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="ragged", choices=["ragged", "single", "long2048", "long1024"])
+    ap.add_argument("--config", default="ragged",
+                    choices=["ragged", "single", "long2048", "long1024", "prefill"])
     ap.add_argument("--mode", default="aware", choices=["aware", "masked"])
     ap.add_argument("--max-splits", type=int, default=8)
     ap.add_argument("--per-layer", action="store_true",
@@ -241,10 +242,118 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def prefill_bytes_flops(n_new):
+    """Causal prefill per layer: 9216 B per prompt row (q read 4096, o written
+    4096, K/V row 1024) and 4096 * L * (L + 1) FLOPs per request of L rows
+    (QK^T and PV over the causal half, 16 heads, head dim 128)."""
+    rows = sum(int(x) for x in n_new)
+    return rows * 9216, sum(4096 * int(x) * (int(x) + 1) for x in n_new)
+
+
+def measured_tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def run_prefill(args):
+    """Coalesced prefill: 16 prompts of 20..387 rows, 36 layers.  A step is
+    RoPE + delta write of all prompt rows of all layers, then the causal
+    prefill of every layer."""
+    import torch
+    from gqa_attention_static_b200 import ops
+    from gqa_attention_static_b200 import workloads as W
+    from gqa_attention_static_b200.step import PrefillStep
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+    ops.load()
+    batch = W.cfg_prefill(layers=N_LAYERS)
+    L = batch.layers
+    step = PrefillStep([x.to(dev) for x in batch.q], [x.to(dev) for x in batch.k_new],
+                       [x.to(dev) for x in batch.v_new], [x.to(dev) for x in batch.cache_k],
+                       [x.to(dev) for x in batch.cache_v], batch.pos0.to(dev), batch.n_new.to(dev))
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step.run(s)
+    torch.cuda.synchronize()
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=s):
+        step.run(s)
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+    g_inst = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_inst, stream=s):
+        ev[0].record(s)
+        step.append(s)
+        ev[1].record(s)
+        step.attention(s)
+        ev[2].record(s)
+    torch.cuda.synchronize()
+    for _ in range(max(3, args.warmup)):
+        g_step.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        e0.record(s)
+        for _ in range(args.steps):
+            g_step.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    ms_step = e0.elapsed_time(e1) / args.steps
+    with torch.cuda.stream(s):
+        g_inst.replay()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms_prefill = ev[1].elapsed_time(ev[2]) / L          # one prefill launch (one layer)
+    ms_append = ev[0].elapsed_time(ev[1])
+    if int(step.status.item()) != 0:
+        print(f"device status word set: {int(step.status.item())}", file=sys.stderr)
+    nb, nf = prefill_bytes_flops(batch.n_new.tolist())
+    hbm, hbm_kind = measured_peaks()
+    tc, tc_kind = measured_tensor_peak()
+    t_bytes = nb / (hbm * 1e9)
+    t_flops = nf / (tc * 1e12)
+    bound = "hbm" if t_bytes >= t_flops else "tensor"
+    achieved_gbs = nb / (ms_prefill * 1e-3) / 1e9
+    achieved_tf = nf / (ms_prefill * 1e-3) / 1e12
+    roof = {"kernel": "prefill_kernel (ark_attn_prefill, one layer)", "bound": bound,
+            "achieved": achieved_gbs if bound == "hbm" else achieved_tf,
+            "peak": hbm if bound == "hbm" else tc, "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+            "frac": (t_bytes if bound == "hbm" else t_flops) / (ms_prefill * 1e-3),
+            "peak_kind": hbm_kind if bound == "hbm" else tc_kind, "traffic": None,
+            "launch_ms": ms_prefill, "algorithmic_bytes_per_launch": nb, "flops_per_launch": nf,
+            "achieved_tflops": achieved_tf, "tensor_peak_tflops": tc,
+            "append_ms_per_step": ms_append}
+    value = nb * L / (ms_step * 1e-3) / 1e9
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "coalesced causal prefill B=16 L U[20,387] S=387 T=512, 36 layers",
+                       "layers": L, "rows": int(batch.n_new.sum()),
+                       "l2": "q/o of 36 layers (1.8 GB) larger than L2",
+                       "path": "layer-batched append + per-layer prefill replayed from one CUDA graph"},
+            "tokens_layers_per_s": int(batch.n_new.sum()) * L / (ms_step * 1e-3),
+            "roofline": roof, "gpu_launches": step.launches_per_step() * args.steps, "clocks": clk}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.config == "prefill":
+        run_prefill(args)
         return
     import torch
     import torch.distributed as dist
