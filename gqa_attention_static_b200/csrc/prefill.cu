@@ -14,16 +14,19 @@
 //     block is read once for all 8 heads (GQA packing).  The Q tile arrives
 //     by two 4-D TMA boxes (64 head-dim elements each, 128-byte swizzle),
 //     already in the K-major layout tcgen05 reads.
-//   - KV blocks of 128 keys stream through a 2-stage ring (TMA, 3-D boxes
-//     over the cache).  S = Q K^T for a block is 8 MMAs of 128x128x16 into a
-//     TMEM buffer (two buffers, so QK of block j+1 overlaps the softmax of
-//     block j); O += P V is 8 MMAs with V as an MN-major operand (no
-//     transpose), accumulated in TMEM.
+//   - KV blocks of 64 keys stream through a 2-stage ring (TMA, 3-D boxes over
+//     the cache).  S = Q K^T for a block is 8 MMAs of 128x64x16 into a TMEM
+//     buffer (two buffers, so QK of block j+1 overlaps the softmax of block
+//     j); O += P V is 4 MMAs of 128x128x16 with V as an MN-major operand (no
+//     transpose), accumulated in TMEM.  96 KB of shared memory and 256 TMEM
+//     columns per CTA: two CTAs share an SM, so one CTA's softmax overlaps the
+//     other's loads and MMAs.
 //   - Warp roles: warp 0 issues TMA (and owns the TMEM allocation), warp 1
 //     issues MMAs from one thread, warps 2..5 run the softmax: thread r owns
 //     TMEM lane r, i.e. one query row, so row max and row sum need no
-//     shuffles.  P (bf16) goes to shared memory in the swizzled K-major
-//     layout and feeds the PV MMA.
+//     shuffles; a block's 64 scores of a row sit in that thread's registers.
+//     P (bf16) is written, in the swizzled K-major layout, over the block's K
+//     tile (which the QK MMA has finished with) and feeds the PV MMA.
 //   - Softmax in the log2 domain with a lazily moved reference max: O is
 //     rescaled (read, scale, write back in TMEM) only when a row's block max
 //     exceeds its reference by more than 2^8, which for real data is almost
@@ -46,40 +49,40 @@ namespace pf {
 
 constexpr int kRows = 128;               // MMA M: 16 positions x 8 heads
 constexpr int kPos = 16;                 // query positions per tile
-constexpr int kBN = 128;                 // keys per KV block
-constexpr int kHalf = kRows * 128;       // one 64-element half of a 128-row tile (16 KB)
-constexpr int kTile = 2 * kHalf;         // a 128 x 128 bf16 tile (32 KB)
+constexpr int kBN = 64;                  // keys per KV block
+constexpr int kQHalf = kRows * 128;      // one 64-element half of the Q tile (16 KB)
+constexpr int kKHalf = kBN * 128;        // one 64-element half of a K or V block (8 KB)
+constexpr int kKV = 2 * kKHalf;          // a K or V block (16 KB); also holds P (128 rows x 64 keys)
 constexpr int kThreads = 192;            // warp 0: TMA, warp 1: MMA, warps 2..5: softmax
 
 // shared memory map (offsets from a 1024-aligned base)
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kTile;     // 2 stages
-constexpr int kOffV = kOffK + 2 * kTile; // 2 stages
-constexpr int kOffP = kOffV + 2 * kTile;
-constexpr int kOffBar = kOffP + kTile;
+constexpr int kOffK = kOffQ + 2 * kQHalf;   // 2 stages
+constexpr int kOffV = kOffK + 2 * kKV;      // 2 stages
+constexpr int kOffBar = kOffV + 2 * kKV;
 constexpr int kNumBars = 10;
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kOffFlag = kOffTmemPtr + 8;
 constexpr int kSmemBytes = 1024 + kOffFlag + 16;
 
 // bar indices
-constexpr int kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarSFull = 5, kBarPFull = 7, kBarPvDone = 8;
+constexpr int kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarSFull = 5, kBarPFull = 7, kBarPvDone = 9;
 
 // TMEM columns
-constexpr uint32_t kColS = 0;            // two S buffers: 0..127, 128..255
-constexpr uint32_t kColO = 256;          // O: 256..383
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;            // two S buffers: 0..63, 64..127
+constexpr uint32_t kColO = 128;          // O: 128..255
+constexpr uint32_t kTmemCols = 256;
 
-// instruction descriptors (kind::f16): D fp32, A/B bf16, M = 128, N = 128
-constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
-constexpr uint32_t kIdescQK = kIdescBase;               // A = Q (K-major), B = K (K-major)
-constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);  // A = P (K-major), B = V (MN-major)
+// instruction descriptors (kind::f16): D fp32, A/B bf16, M = 128
+constexpr uint32_t kIdescF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescQK = kIdescF16 | ((64u >> 3) << 17);                // N = 64 keys, B = K (K-major)
+constexpr uint32_t kIdescPV = kIdescF16 | ((128u >> 3) << 17) | (1u << 16);  // N = 128 dims, B = V (MN-major)
 
 constexpr float kLazyRescale = 8.0f;     // log2 units: rescale O only past a factor 2^8
 
 struct Params {
     CUtensorMap qmap;    // q as (128, 8, Hq/8, B*S), box (64, 8, 1, 16)
-    CUtensorMap kmap;    // cache_k as (128, Hkv, B*T), box (64, 1, 128)
+    CUtensorMap kmap;    // cache_k as (128, Hkv, B*T), box (64, 1, 64)
     CUtensorMap vmap;
     uint16_t* o;         // [B, S, Hq, 128]
     float* lse;          // [B, Hq, S]
@@ -92,7 +95,7 @@ struct Params {
 
 }  // namespace pf
 
-__global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_constant__ pf::Params p) {
+__global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_constant__ pf::Params p) {
     using namespace pf;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -124,13 +127,12 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[kBarQ], 1);
-        mbar_init(&bars[kBarKvFull], 1);
-        mbar_init(&bars[kBarKvFull + 1], 1);
-        mbar_init(&bars[kBarKvEmpty], 1);
-        mbar_init(&bars[kBarKvEmpty + 1], 1);
-        mbar_init(&bars[kBarSFull], 1);
-        mbar_init(&bars[kBarSFull + 1], 1);
-        mbar_init(&bars[kBarPFull], 128);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars[kBarKvFull + i], 1);
+            mbar_init(&bars[kBarKvEmpty + i], 1);
+            mbar_init(&bars[kBarSFull + i], 1);
+            mbar_init(&bars[kBarPFull + i], 128);
+        }
         mbar_init(&bars[kBarPvDone], 1);
         *failed_flag = 0;
         fence_mbar_init();
@@ -147,25 +149,26 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
         // ================================================= TMA producer
         if (lane == 0) {
             bool ok = true;
-            mbar_arrive_expect_tx(&bars[kBarQ], kTile);
+            mbar_arrive_expect_tx(&bars[kBarQ], 2 * kQHalf);
             const int qrow = b * p.S + t0;
             tma_load_4d(smem + kOffQ, &p.qmap, 0, 0, g, qrow, &bars[kBarQ]);
-            tma_load_4d(smem + kOffQ + kHalf, &p.qmap, 64, 0, g, qrow, &bars[kBarQ]);
-            for (int j = 0; j < nblk && ok; ++j) {
+            tma_load_4d(smem + kOffQ + kQHalf, &p.qmap, 64, 0, g, qrow, &bars[kBarQ]);
+            for (int j = 0; j < nblk; ++j) {
                 const int st = j & 1;
+                // stage st (K, V, and the P written over K) is free once PV of block j-2 is done
                 if (j >= 2 && !mbar_wait(&bars[kBarKvEmpty + st], ((j >> 1) - 1) & 1)) {
                     ok = false;
                     break;
                 }
                 uint64_t* full = &bars[kBarKvFull + st];
-                mbar_arrive_expect_tx(full, 2 * kTile);
+                mbar_arrive_expect_tx(full, 2 * kKV);
                 const int row = b * p.T + j * kBN;
-                uint8_t* kd = smem + kOffK + st * kTile;
-                uint8_t* vd = smem + kOffV + st * kTile;
+                uint8_t* kd = smem + kOffK + st * kKV;
+                uint8_t* vd = smem + kOffV + st * kKV;
                 tma_load_3d(kd, &p.kmap, 0, g, row, full);
-                tma_load_3d(kd + kHalf, &p.kmap, 64, g, row, full);
+                tma_load_3d(kd + kKHalf, &p.kmap, 64, g, row, full);
                 tma_load_3d(vd, &p.vmap, 0, g, row, full);
-                tma_load_3d(vd + kHalf, &p.vmap, 64, g, row, full);
+                tma_load_3d(vd + kKHalf, &p.vmap, 64, g, row, full);
             }
             if (!ok) {
                 atomicExch(failed_flag, 1);
@@ -181,10 +184,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarKvFull + (j & 1)], (j >> 1) & 1))) return false;
             const int live = kv_end - j * kBN;
             if (live < kBN) {
-                uint8_t* vt = smem + kOffV + (j & 1) * kTile;
+                uint8_t* vt = smem + kOffV + (j & 1) * kKV;
                 for (int i = lane; i < (kBN - live) * 16; i += 32) {
                     const int r = live + (i >> 4), part = i & 15;
-                    *reinterpret_cast<uint4*>(vt + (part >> 3) * kHalf + r * 128 + (part & 7) * 16) =
+                    *reinterpret_cast<uint4*>(vt + (part >> 3) * kKHalf + r * 128 + (part & 7) * 16) =
                         make_uint4(0, 0, 0, 0);
                 }
                 fence_proxy_async_smem();
@@ -196,12 +199,12 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
             if (lane == 0) {
                 tc_fence_after();
                 const uint32_t d = tmem + kColS + (j & 1) * kBN;
-                const uint32_t kb = sbase + kOffK + (j & 1) * kTile;
+                const uint32_t kb = sbase + kOffK + (j & 1) * kKV;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    umma_f16(d, umma_desc_sw128(sbase + kOffQ + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024),
-                             kIdescQK, kk > 0 ? 1u : 0u);
+                    const uint32_t sub = (kk & 3) * 32;
+                    umma_f16(d, umma_desc_sw128(sbase + kOffQ + (kk >> 2) * kQHalf + sub, 16, 1024),
+                             umma_desc_sw128(kb + (kk >> 2) * kKHalf + sub, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&bars[kBarSFull + (j & 1)]);
             }
@@ -210,12 +213,12 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
         auto issue_pv = [&](int j) {
             if (lane == 0) {
                 tc_fence_after();
-                const uint32_t vb = sbase + kOffV + (j & 1) * kTile;
+                const uint32_t pb = sbase + kOffK + (j & 1) * kKV;   // P of block j, over its K tile
+                const uint32_t vb = sbase + kOffV + (j & 1) * kKV;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t aoff = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    umma_f16(tmem + kColO, umma_desc_sw128(sbase + kOffP + aoff, 16, 1024),
-                             umma_desc_sw128(vb + kk * 16 * 128, kHalf, 1024), kIdescPV,
+                for (int kk = 0; kk < 4; ++kk) {
+                    umma_f16(tmem + kColO, umma_desc_sw128(pb + kk * 32, 16, 1024),
+                             umma_desc_sw128(vb + kk * 16 * 128, kKHalf, 1024), kIdescPV,
                              (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(&bars[kBarKvEmpty + (j & 1)]);
@@ -227,11 +230,11 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
         if (ok) issue_qk(0);
         for (int j = 0; j < nblk && ok; ++j) {
             if (j + 1 < nblk) {
-                // S buffer (j+1)&1 was last read by the softmax of block j-1 (waited below at j-1)
+                // S buffer (j+1)&1 was last read by the softmax of block j-1 (its P arrival was waited below)
                 if (!(ok = wait_kv(j + 1))) break;
                 issue_qk(j + 1);
             }
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPFull], j & 1)))) break;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPFull + (j & 1)], (j >> 1) & 1)))) break;
             issue_pv(j);
         }
         if (!ok && lane == 0) {
@@ -248,7 +251,6 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
         float m_ref = -INFINITY, e_sum = 0.f, r_sum = 0.f;
         bool ok = true;
-        uint8_t* prow_smem = smem + kOffP + r * 128;
         // Every tcgen05.ld/st below is .sync.aligned: all 32 lanes of the warp
         // execute it together, so all control flow around them is warp-uniform
         // (ok is AND-ed over the warp; per-row choices become per-lane values).
@@ -257,78 +259,76 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
             if (!ok) break;
             tc_fence_after();
             const uint32_t scol = lane_base + kColS + (j & 1) * kBN;
-            const int kbase = j * kBN;
-            const int nvalid = min(kBN, prow - kbase + 1);   // keys kbase .. prow of this block
-            // pass 1: block max of the visible scores
-            float bm = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t v[32];
-                tmem_ld32(scol + c * 32, v);
+            const int nvalid = min(kBN, prow - j * kBN + 1);   // keys j*64 .. prow of this block
+            uint32_t v[64];
+            {
+                uint32_t (&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+                uint32_t (&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+                tmem_ld32(scol, v0);
+                tmem_ld32(scol + 32, v1);
                 tmem_wait_ld();
+            }
+            float bm = -INFINITY;
+            if (nvalid >= kBN) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (c * 32 + i < nvalid) bm = fmaxf(bm, __uint_as_float(v[i]));
+                for (int i = 0; i < kBN; ++i) bm = fmaxf(bm, __uint_as_float(v[i]));
+            } else {
+#pragma unroll
+                for (int i = 0; i < kBN; ++i)
+                    if (i < nvalid) bm = fmaxf(bm, __uint_as_float(v[i]));
             }
             bm *= p.scale_log2;
             float alpha = 1.f;
             bool rescale = false;
             if (m_ref == -INFINITY) {
-                m_ref = bm;
+                m_ref = bm;                 // first visible block of this row: O is still empty
             } else if (bm > m_ref + kLazyRescale) {
                 alpha = fast_exp2(m_ref - bm);
                 m_ref = bm;
                 rescale = true;
             }
             const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-            // the P buffer and O are free once PV of block j-1 has completed
-            if (j >= 1) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPvDone], (j - 1) & 1));
-                if (!ok) break;
-            }
-            tc_fence_after();
-            if (__any_sync(0xffffffffu, rescale)) {       // lanes that need none scale by 1
+            if (__any_sync(0xffffffffu, rescale)) {
+                // O must hold PV of every earlier block before it is rescaled
+                if (j >= 1) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPvDone], (j - 1) & 1));
+                    if (!ok) break;
+                }
+                tc_fence_after();
                 e_sum *= alpha;
                 r_sum *= alpha;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(lane_base + kColO + c * 32, v);
+                for (int c = 0; c < 4; ++c) {         // lanes that need none scale by 1
+                    uint32_t o[32];
+                    tmem_ld32(lane_base + kColO + c * 32, o);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-                    tmem_st32(lane_base + kColO + c * 32, v);
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(lane_base + kColO + c * 32, o);
                 }
                 tmem_wait_st();
             }
-            // pass 2: P = exp2(s * scale_log2 - m_ref) as bf16 into the swizzled K-major P tile
+            // P = exp2(s * scale_log2 - m_ref) as bf16, written over this block's K tile
+            // (row r: 64 keys = one 128-byte swizzled row)
+            uint8_t* prow_smem = smem + kOffK + (j & 1) * kKV + r * 128;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t v[32];
-                tmem_ld32(scol + c * 32, v);
-                tmem_wait_ld();
-                uint32_t pk[16];
+            for (int q = 0; q < 8; ++q) {
+                uint32_t pk[4];
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const float s0 = (c * 32 + i < nvalid) ? fast_exp2(__uint_as_float(v[i]) * p.scale_log2 - mu) : 0.f;
-                    const float s1 =
-                        (c * 32 + i + 1 < nvalid) ? fast_exp2(__uint_as_float(v[i + 1]) * p.scale_log2 - mu) : 0.f;
+                for (int i = 0; i < 8; i += 2) {
+                    const int k0 = q * 8 + i;
+                    const float s0 = (k0 < nvalid) ? fast_exp2(__uint_as_float(v[k0]) * p.scale_log2 - mu) : 0.f;
+                    const float s1 = (k0 + 1 < nvalid) ? fast_exp2(__uint_as_float(v[k0 + 1]) * p.scale_log2 - mu) : 0.f;
                     const __nv_bfloat162 pb = __floats2bfloat162_rn(s0, s1);
                     e_sum += s0 + s1;
                     r_sum += __low2float(pb) + __high2float(pb);
                     pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&pb);
                 }
-                // keys c*32 .. c*32+31: half c/2, 16-byte chunks 4*(c&1) .. +3
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int chunk = 4 * (c & 1) + q;
-                    *reinterpret_cast<uint4*>(prow_smem + (c >> 1) * kHalf + ((chunk ^ (r & 7)) << 4)) =
-                        make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-                }
+                *reinterpret_cast<uint4*>(prow_smem + ((q ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
             fence_proxy_async_smem();      // P is read by the tensor core (async proxy)
             tc_fence_before();
-            mbar_arrive(&bars[kBarPFull]);
+            mbar_arrive(&bars[kBarPFull + (j & 1)]);
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPvDone], (nblk - 1) & 1));
         tc_fence_after();
@@ -344,17 +344,17 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const __grid_c
             uint16_t* orow = p.o + ((static_cast<size_t>(b) * p.S + tr) * p.Hq + h) * kHeadDim;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t v[32];
-                tmem_ld32(lane_base + kColO + c * 32, v);
+                uint32_t o[32];
+                tmem_ld32(lane_base + kColO + c * 32, o);
                 tmem_wait_ld();
                 if (live) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv);
-                        w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv);
-                        w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv);
-                        w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv);
+                        w.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
+                        w.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
+                        w.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
+                        w.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
                         reinterpret_cast<uint4*>(orow + c * 32)[q] = w;
                     }
                 }
