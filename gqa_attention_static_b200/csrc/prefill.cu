@@ -9,7 +9,8 @@
 // p = pos0[b] + t, attends to the cache rows j <= p of its KV head.
 //
 // Tiling (B200):
-//   - One CTA per (16 query positions, KV head g, request b).  Its 128 MMA
+//   - One CTA per (16 query positions, KV head g, request b), the tiles with
+//     the longest key ranges launched first.  Its 128 MMA
 //     rows are the 16 positions x the 8 query heads of group g, so every K/V
 //     block is read once for all 8 heads (GQA packing).  The Q tile arrives
 //     by two 4-D TMA boxes (64 head-dim elements each, 128-byte swizzle),
@@ -102,9 +103,11 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
                                                ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int qt = blockIdx.x;
-    const int g = blockIdx.y;
-    const int b = blockIdx.z;
+    // the grid runs the latest query tiles (longest key ranges) first, so the
+    // short tiles fill in behind them
+    const int qt = gridDim.z - 1 - blockIdx.z;
+    const int g = blockIdx.x;
+    const int b = blockIdx.y;
 
     // ---- lengths (device values: checked here)
     int nn = __ldg(p.n_new + b);
@@ -422,7 +425,8 @@ extern "C" ark_status ark_attn_prefill(const void* q, const void* cache_k, const
             return ARK_ERR_CUDA;
         g_prefill_attr[dev] = true;
     }
-    dim3 grid((S + pf::kPos - 1) / pf::kPos, Hkv, B);
+    if ((S + pf::kPos - 1) / pf::kPos > 65535) return ARK_ERR_UNSUPPORTED;
+    dim3 grid(Hkv, B, (S + pf::kPos - 1) / pf::kPos);
     prefill_kernel<<<grid, pf::kThreads, pf::kSmemBytes, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
 }
