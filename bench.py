@@ -97,6 +97,24 @@ def algorithmic_bytes(kv_len, B: int) -> int:
     return int(sum(int(x) for x in kv_len) * 1024 + B * 8192)
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's device time: every rank runs the same replica
+    workload, so the job takes as long as its slowest GPU."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job GB/s of N independent replicas (weak scaling): the bytes all
+    ranks processed over the slowest rank's time."""
+    return bytes_per_rank * world / (ms_max * 1e-3) / 1e9
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -441,12 +459,7 @@ def main():
                 fn()
             e1.record(s)
         barrier()
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return max_over_ranks(e0.elapsed_time(e1), world, dev)
 
     for _ in range(max(3, args.warmup)):
         g_step.replay()
@@ -471,7 +484,7 @@ def main():
     kvl = batch.kv_len.tolist()
     bytes_layer = algorithmic_bytes(kvl, B)
     step_bytes = bytes_layer * L
-    value = step_bytes * world / (ms_step * 1e-3) / 1e9
+    value = job_throughput(step_bytes, world, ms_step)
     tl = B * L * world / (ms_step * 1e-3)
     bytes_launch = bytes_layer * (L if step.batched else 1)
     peak, peak_kind = measured_peaks()
@@ -553,12 +566,8 @@ def main():
         s_h2d.wait_stream(s_d2h)
         e1.record(s_h2d)
         barrier()
-        ms_e2e = e0.elapsed_time(e1) / K2
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": step_bytes * world / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / K2, world, dev)
+        e2e = {"value": job_throughput(step_bytes, world, ms_e2e), "unit": "GB/s",
                "h2d_bytes_per_step": in_elems * 2, "d2h_bytes_per_step": L * osz * 2 + L * B * 16 * 4,
                "ms_per_step": ms_e2e,
                "how": "pinned host buffers, H2D of the step inputs and D2H of o/lse every step, "
