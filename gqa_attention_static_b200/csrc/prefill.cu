@@ -15,11 +15,12 @@
 //     block is read once for all 8 heads (GQA packing).  The Q tile arrives
 //     by two 4-D TMA boxes (64 head-dim elements each, 128-byte swizzle),
 //     already in the K-major layout tcgen05 reads.
-//   - KV blocks of 64 keys stream through a 2-stage ring (TMA, 3-D boxes over
-//     the cache).  S = Q K^T for a block is 8 MMAs of 128x64x16 into a TMEM
+//   - KV blocks of 64 keys stream in by TMA (3-D boxes over the cache): K
+//     through a 3-stage ring, V through a 2-stage ring, so both arrive about
+//     two blocks ahead of their use.  S = Q K^T for a block is 8 MMAs of 128x64x16 into a TMEM
 //     buffer (two buffers, so QK of block j+1 overlaps the softmax of block
 //     j); O += P V is 4 MMAs of 128x128x16 with V as an MN-major operand (no
-//     transpose), accumulated in TMEM.  96 KB of shared memory and 256 TMEM
+//     transpose), accumulated in TMEM.  112 KB of shared memory and 256 TMEM
 //     columns per CTA: two CTAs share an SM, so one CTA's softmax overlaps the
 //     other's loads and MMAs.
 //   - Warp roles: warp 0 issues TMA (and owns the TMEM allocation), warp 1
@@ -56,18 +57,26 @@ constexpr int kKHalf = kBN * 128;        // one 64-element half of a K or V bloc
 constexpr int kKV = 2 * kKHalf;          // a K or V block (16 KB); also holds P (128 rows x 64 keys)
 constexpr int kThreads = 192;            // warp 0: TMA, warp 1: MMA, warps 2..5: softmax
 
-// shared memory map (offsets from a 1024-aligned base)
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+
+// shared memory map (the dynamic shared memory base is 1024-aligned)
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + 2 * kQHalf;   // 2 stages
-constexpr int kOffV = kOffK + 2 * kKV;      // 2 stages
-constexpr int kOffBar = kOffV + 2 * kKV;
-constexpr int kNumBars = 10;
+constexpr int kOffK = kOffQ + 2 * kQHalf;          // kKStages stages (P of a block is written over its K)
+constexpr int kOffV = kOffK + kKStages * kKV;      // kVStages stages
+constexpr int kOffBar = kOffV + kVStages * kKV;
+constexpr int kBarQ = 0;
+constexpr int kBarKFull = 1;                       // kKStages
+constexpr int kBarKEmpty = kBarKFull + kKStages;   // kKStages
+constexpr int kBarVFull = kBarKEmpty + kKStages;   // kVStages
+constexpr int kBarVEmpty = kBarVFull + kVStages;   // kVStages
+constexpr int kBarSFull = kBarVEmpty + kVStages;   // 2
+constexpr int kBarPFull = kBarSFull + 2;           // 2
+constexpr int kBarPvDone = kBarPFull + 2;
+constexpr int kNumBars = kBarPvDone + 1;
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kOffFlag = kOffTmemPtr + 8;
-constexpr int kSmemBytes = 1024 + kOffFlag + 16;
-
-// bar indices
-constexpr int kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarSFull = 5, kBarPFull = 7, kBarPvDone = 9;
+constexpr int kSmemBytes = kOffFlag + 16;
 
 // TMEM columns
 constexpr uint32_t kColS = 0;            // two S buffers: 0..63, 64..127
@@ -98,9 +107,7 @@ struct Params {
 
 __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_constant__ pf::Params p) {
     using namespace pf;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~static_cast<uintptr_t>(1023));
+    extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     // the grid runs the latest query tiles (longest key ranges) first, so the
@@ -121,6 +128,10 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
     }
     const int t0 = qt * kPos;
     if (t0 >= nn) return;                                   // whole CTA: no live row
+    if (smem_u32(smem) & 1023u) {                           // the swizzled layouts need 1024-byte alignment
+        if (threadIdx.x == 0) report(p.status, ARK_DEV_TIMEOUT);
+        return;
+    }
     const int kv_end = p0 + min(t0 + kPos, nn);             // keys visible to the tile's last row
     const int nblk = (kv_end + kBN - 1) / kBN;
 
@@ -129,14 +140,7 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
     int* failed_flag = reinterpret_cast<int*>(smem + kOffFlag);
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars[kBarQ], 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars[kBarKvFull + i], 1);
-            mbar_init(&bars[kBarKvEmpty + i], 1);
-            mbar_init(&bars[kBarSFull + i], 1);
-            mbar_init(&bars[kBarPFull + i], 128);
-        }
-        mbar_init(&bars[kBarPvDone], 1);
+        for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? 128 : 1);
         *failed_flag = 0;
         fence_mbar_init();
     }
@@ -157,21 +161,27 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
             tma_load_4d(smem + kOffQ, &p.qmap, 0, 0, g, qrow, &bars[kBarQ]);
             tma_load_4d(smem + kOffQ + kQHalf, &p.qmap, 64, 0, g, qrow, &bars[kBarQ]);
             for (int j = 0; j < nblk; ++j) {
-                const int st = j & 1;
-                // stage st (K, V, and the P written over K) is free once PV of block j-2 is done
-                if (j >= 2 && !mbar_wait(&bars[kBarKvEmpty + st], ((j >> 1) - 1) & 1)) {
+                const int row = b * p.T + j * kBN;
+                // K stage (with the P written over it) is free once PV of block j-3 is done
+                const int ks = j % kKStages;
+                if (j >= kKStages && !mbar_wait(&bars[kBarKEmpty + ks], ((j / kKStages) - 1) & 1)) {
                     ok = false;
                     break;
                 }
-                uint64_t* full = &bars[kBarKvFull + st];
-                mbar_arrive_expect_tx(full, 2 * kKV);
-                const int row = b * p.T + j * kBN;
-                uint8_t* kd = smem + kOffK + st * kKV;
-                uint8_t* vd = smem + kOffV + st * kKV;
-                tma_load_3d(kd, &p.kmap, 0, g, row, full);
-                tma_load_3d(kd + kKHalf, &p.kmap, 64, g, row, full);
-                tma_load_3d(vd, &p.vmap, 0, g, row, full);
-                tma_load_3d(vd + kKHalf, &p.vmap, 64, g, row, full);
+                mbar_arrive_expect_tx(&bars[kBarKFull + ks], kKV);
+                uint8_t* kd = smem + kOffK + ks * kKV;
+                tma_load_3d(kd, &p.kmap, 0, g, row, &bars[kBarKFull + ks]);
+                tma_load_3d(kd + kKHalf, &p.kmap, 64, g, row, &bars[kBarKFull + ks]);
+                // V stage is free once PV of block j-2 is done
+                const int vs = j % kVStages;
+                if (j >= kVStages && !mbar_wait(&bars[kBarVEmpty + vs], ((j / kVStages) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&bars[kBarVFull + vs], kKV);
+                uint8_t* vd = smem + kOffV + vs * kKV;
+                tma_load_3d(vd, &p.vmap, 0, g, row, &bars[kBarVFull + vs]);
+                tma_load_3d(vd + kKHalf, &p.vmap, 64, g, row, &bars[kBarVFull + vs]);
             }
             if (!ok) {
                 atomicExch(failed_flag, 1);
@@ -182,12 +192,16 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
         // ================================================= MMA issuer
         // waits are AND-ed over the warp so that the __syncwarp()s below are reached by all lanes
         bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarQ], 0));
-        auto wait_kv = [&](int j) {
-            // K/V block j landed; zero the V rows past the tile's causal range
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarKvFull + (j & 1)], (j >> 1) & 1))) return false;
+        auto wait_k = [&](int j) {
+            return __all_sync(0xffffffffu, mbar_wait(&bars[kBarKFull + j % kKStages], (j / kKStages) & 1));
+        };
+        auto wait_v = [&](int j) {
+            // V block j landed; zero its rows past the tile's causal range
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarVFull + j % kVStages], (j / kVStages) & 1)))
+                return false;
             const int live = kv_end - j * kBN;
             if (live < kBN) {
-                uint8_t* vt = smem + kOffV + (j & 1) * kKV;
+                uint8_t* vt = smem + kOffV + (j % kVStages) * kKV;
                 for (int i = lane; i < (kBN - live) * 16; i += 32) {
                     const int r = live + (i >> 4), part = i & 15;
                     *reinterpret_cast<uint4*>(vt + (part >> 3) * kKHalf + r * 128 + (part & 7) * 16) =
@@ -202,7 +216,7 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
             if (lane == 0) {
                 tc_fence_after();
                 const uint32_t d = tmem + kColS + (j & 1) * kBN;
-                const uint32_t kb = sbase + kOffK + (j & 1) * kKV;
+                const uint32_t kb = sbase + kOffK + (j % kKStages) * kKV;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t sub = (kk & 3) * 32;
@@ -216,28 +230,30 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
         auto issue_pv = [&](int j) {
             if (lane == 0) {
                 tc_fence_after();
-                const uint32_t pb = sbase + kOffK + (j & 1) * kKV;   // P of block j, over its K tile
-                const uint32_t vb = sbase + kOffV + (j & 1) * kKV;
+                const uint32_t pb = sbase + kOffK + (j % kKStages) * kKV;   // P of block j, over its K tile
+                const uint32_t vb = sbase + kOffV + (j % kVStages) * kKV;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     umma_f16(tmem + kColO, umma_desc_sw128(pb + kk * 32, 16, 1024),
                              umma_desc_sw128(vb + kk * 16 * 128, kKHalf, 1024), kIdescPV,
                              (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(&bars[kBarKvEmpty + (j & 1)]);
+                umma_commit(&bars[kBarKEmpty + j % kKStages]);
+                umma_commit(&bars[kBarVEmpty + j % kVStages]);
                 umma_commit(&bars[kBarPvDone]);
             }
             __syncwarp();
         };
-        if (ok) ok = wait_kv(0);
+        if (ok) ok = wait_k(0);
         if (ok) issue_qk(0);
         for (int j = 0; j < nblk && ok; ++j) {
             if (j + 1 < nblk) {
                 // S buffer (j+1)&1 was last read by the softmax of block j-1 (its P arrival was waited below)
-                if (!(ok = wait_kv(j + 1))) break;
+                if (!(ok = wait_k(j + 1))) break;
                 issue_qk(j + 1);
             }
             if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPFull + (j & 1)], (j >> 1) & 1)))) break;
+            if (!(ok = wait_v(j))) break;
             issue_pv(j);
         }
         if (!ok && lane == 0) {
@@ -313,7 +329,7 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
             }
             // P = exp2(s * scale_log2 - m_ref) as bf16, written over this block's K tile
             // (row r: 64 keys = one 128-byte swizzled row)
-            uint8_t* prow_smem = smem + kOffK + (j & 1) * kKV + r * 128;
+            uint8_t* prow_smem = smem + kOffK + (j % kKStages) * kKV + r * 128;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 uint32_t pk[4];
@@ -371,7 +387,8 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
     if (warp == 0) {
         if (*failed_flag) {
             // do not release shared or tensor memory under copies or MMAs still in flight
-            for (int s = 0; s < 2; ++s) (void)mbar_wait(&bars[kBarKvFull + s], 0);
+            for (int s = 0; s < kKStages; ++s) (void)mbar_wait(&bars[kBarKFull + s], 0);
+            for (int s = 0; s < kVStages; ++s) (void)mbar_wait(&bars[kBarVFull + s], 0);
             (void)mbar_wait(&bars[kBarPvDone], (nblk - 1) & 1);
         }
         tc_fence_after();
