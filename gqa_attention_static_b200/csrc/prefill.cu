@@ -15,18 +15,18 @@
 //     block is read once for all 8 heads (GQA packing).  The Q tile arrives
 //     by two 4-D TMA boxes (64 head-dim elements each, 128-byte swizzle),
 //     already in the K-major layout tcgen05 reads.
-//   - KV blocks of 64 keys stream in by TMA (3-D boxes over the cache): K
-//     through a 3-stage ring, V through a 2-stage ring, so both arrive about
-//     two blocks ahead of their use.  S = Q K^T for a block is 8 MMAs of 128x64x16 into a TMEM
+//   - KV blocks of 64 keys stream in by TMA (3-D boxes over the cache)
+//     through 2-stage K and V rings with separate barriers.  S = Q K^T for a block is 8 MMAs of 128x64x16 into a TMEM
 //     buffer (two buffers, so QK of block j+1 overlaps the softmax of block
 //     j); O += P V is 4 MMAs of 128x128x16 with V as an MN-major operand (no
-//     transpose), accumulated in TMEM.  112 KB of shared memory and 256 TMEM
+//     transpose), accumulated in TMEM.  98 KB of shared memory and 256 TMEM
 //     columns per CTA: two CTAs share an SM, so one CTA's softmax overlaps the
 //     other's loads and MMAs.
 //   - Warp roles: warp 0 issues TMA (and owns the TMEM allocation), warp 1
-//     issues MMAs from one thread, warps 2..5 run the softmax: thread r owns
-//     TMEM lane r, i.e. one query row, so row max and row sum need no
-//     shuffles; a block's 64 scores of a row sit in that thread's registers.
+//     issues MMAs from one thread, warps 2..9 run the softmax: two threads
+//     per query row (TMEM lane), one for keys 0..31 and one for keys 32..63
+//     of each block, which trade their partial row maxima through shared
+//     memory behind one named barrier per block.
 //     P (bf16) is written, in the swizzled K-major layout, over the block's K
 //     tile (which the QK MMA has finished with) and feeds the PV MMA.
 //   - Softmax in the log2 domain with a lazily moved reference max: O is
@@ -55,9 +55,10 @@ constexpr int kBN = 64;                  // keys per KV block
 constexpr int kQHalf = kRows * 128;      // one 64-element half of the Q tile (16 KB)
 constexpr int kKHalf = kBN * 128;        // one 64-element half of a K or V block (8 KB)
 constexpr int kKV = 2 * kKHalf;          // a K or V block (16 KB); also holds P (128 rows x 64 keys)
-constexpr int kThreads = 192;            // warp 0: TMA, warp 1: MMA, warps 2..5: softmax
+constexpr int kThreads = 320;            // warp 0: TMA, warp 1: MMA, warps 2..9: softmax
+constexpr int kSoftmaxThreads = 256;     // two threads per row: keys 0..31 and 32..63 of a block
 
-constexpr int kKStages = 3;
+constexpr int kKStages = 2;
 constexpr int kVStages = 2;
 
 // shared memory map (the dynamic shared memory base is 1024-aligned)
@@ -74,7 +75,9 @@ constexpr int kBarSFull = kBarVEmpty + kVStages;   // 2
 constexpr int kBarPFull = kBarSFull + 2;           // 2
 constexpr int kBarPvDone = kBarPFull + 2;
 constexpr int kNumBars = kBarPvDone + 1;
-constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
+constexpr int kOffXchg = kOffBar + kNumBars * 8;   // [3][2 halves][128 rows] fp32: row max (by block
+                                                   // parity) and row sum exchange between a row's two threads
+constexpr int kOffTmemPtr = kOffXchg + 3 * 2 * kRows * 4;
 constexpr int kOffFlag = kOffTmemPtr + 8;
 constexpr int kSmemBytes = kOffFlag + 16;
 
@@ -104,6 +107,19 @@ struct Params {
 };
 
 }  // namespace pf
+
+// Named barrier 1 over the 256 softmax threads, returning the AND of `pred`
+// over all of them (so that decisions taken after it are the same everywhere).
+__device__ __forceinline__ bool bar_and_all(bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.and.pred po, 1, %2, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(out) : "r"(static_cast<uint32_t>(pred)), "n"(pf::kSoftmaxThreads) : "memory");
+    return out != 0;
+}
 
 __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_constant__ pf::Params p) {
     using namespace pf;
@@ -140,7 +156,8 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
     int* failed_flag = reinterpret_cast<int*>(smem + kOffFlag);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? 128 : 1);
+        for (int i = 0; i < kNumBars; ++i)
+            mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? kSoftmaxThreads : 1);
         *failed_flag = 0;
         fence_mbar_init();
     }
@@ -263,40 +280,45 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
     } else {
         // ================================================= softmax + epilogue
         const int quad = warp & 3;                      // TMEM lanes 32*quad .. +31
+        const int half = (warp - 2) >> 2;               // 0: keys 0..31 of a block, 1: keys 32..63
         const int r = quad * 32 + lane;                 // this thread's row of the tile
         const int tr = t0 + (r >> 3);                   // its query position (within the call)
         const int hh = r & 7;
         const int prow = p0 + tr;                       // its absolute position
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-        float m_ref = -INFINITY, e_sum = 0.f, r_sum = 0.f;
+        float* xchg = reinterpret_cast<float*>(smem + kOffXchg);   // [half][row]
+        float m_ref = -INFINITY, e_sum = 0.f, r_sum = 0.f;         // this half's share of the row sums
         bool ok = true;
         // Every tcgen05.ld/st below is .sync.aligned: all 32 lanes of the warp
-        // execute it together, so all control flow around them is warp-uniform
-        // (ok is AND-ed over the warp; per-row choices become per-lane values).
-        for (int j = 0; j < nblk && ok; ++j) {
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + (j & 1)], (j >> 1) & 1));
-            if (!ok) break;
+        // execute it together, so all control flow around them is warp-uniform;
+        // the loop itself is left by all 256 softmax threads together (its exit
+        // test is AND-reduced by the named barrier), so barrier 1 never deadlocks.
+        for (int j = 0; j < nblk; ++j) {
+            ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars[kBarSFull + (j & 1)], (j >> 1) & 1));
             tc_fence_after();
-            const uint32_t scol = lane_base + kColS + (j & 1) * kBN;
-            const int nvalid = min(kBN, prow - j * kBN + 1);   // keys j*64 .. prow of this block
-            uint32_t v[64];
-            {
-                uint32_t (&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
-                uint32_t (&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
-                tmem_ld32(scol, v0);
-                tmem_ld32(scol + 32, v1);
-                tmem_wait_ld();
-            }
-            float bm = -INFINITY;
-            if (nvalid >= kBN) {
+            const uint32_t scol = lane_base + kColS + (j & 1) * kBN + half * 32;
+            const int nvalid = min(32, prow - j * kBN - half * 32 + 1);   // visible keys of this half
+            uint32_t v[32];
+            tmem_ld32(scol, v);
+            tmem_wait_ld();
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (nvalid >= 32) {
 #pragma unroll
-                for (int i = 0; i < kBN; ++i) bm = fmaxf(bm, __uint_as_float(v[i]));
+                for (int i = 0; i < 32; ++i) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(v[i]));
             } else {
 #pragma unroll
-                for (int i = 0; i < kBN; ++i)
-                    if (i < nvalid) bm = fmaxf(bm, __uint_as_float(v[i]));
+                for (int i = 0; i < 32; ++i)
+                    if (i < nvalid) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(v[i]));
             }
-            bm *= p.scale_log2;
+            const float my_max = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            // trade partial maxima with the other half of the row (buffer chosen by block parity)
+            float* xm = xchg + (j & 1) * 2 * kRows;
+            xm[half * kRows + r] = my_max;
+            if (!bar_and_all(ok)) {
+                ok = false;
+                break;
+            }
+            const float bm = fmaxf(my_max, xm[(half ^ 1) * kRows + r]) * p.scale_log2;
             float alpha = 1.f;
             bool rescale = false;
             if (m_ref == -INFINITY) {
@@ -309,41 +331,43 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
             const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
             if (__any_sync(0xffffffffu, rescale)) {
                 // O must hold PV of every earlier block before it is rescaled
-                if (j >= 1) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPvDone], (j - 1) & 1));
-                    if (!ok) break;
-                }
+                if (j >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPvDone], (j - 1) & 1));
                 tc_fence_after();
                 e_sum *= alpha;
                 r_sum *= alpha;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {         // lanes that need none scale by 1
-                    uint32_t o[32];
-                    tmem_ld32(lane_base + kColO + c * 32, o);
+                for (int c = 0; c < 4; ++c) {         // this half rescales O columns 64*half .. +63
+                    uint32_t o[16];
+                    tmem_ld16(lane_base + kColO + half * 64 + c * 16, o);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(lane_base + kColO + c * 32, o);
+                    for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st16(lane_base + kColO + half * 64 + c * 16, o);
                 }
                 tmem_wait_st();
             }
-            // P = exp2(s * scale_log2 - m_ref) as bf16, written over this block's K tile
-            // (row r: 64 keys = one 128-byte swizzled row)
+            // P = exp2(s * scale_log2 - m_ref) as bf16, written over this block's K tile:
+            // row r is one 128-byte swizzled row; this half writes its 16-byte chunks 4*half .. +3
             uint8_t* prow_smem = smem + kOffK + (j % kKStages) * kKV + r * 128;
+            const bool full = nvalid >= 32;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int q = 0; q < 4; ++q) {
                 uint32_t pk[4];
 #pragma unroll
                 for (int i = 0; i < 8; i += 2) {
                     const int k0 = q * 8 + i;
-                    const float s0 = (k0 < nvalid) ? fast_exp2(__uint_as_float(v[k0]) * p.scale_log2 - mu) : 0.f;
-                    const float s1 = (k0 + 1 < nvalid) ? fast_exp2(__uint_as_float(v[k0 + 1]) * p.scale_log2 - mu) : 0.f;
+                    const float x0 = __uint_as_float(v[k0]) * p.scale_log2 - mu;
+                    const float x1 = __uint_as_float(v[k0 + 1]) * p.scale_log2 - mu;
+                    const float s0 = (full || k0 < nvalid) ? fast_exp2(x0) : 0.f;
+                    const float s1 = (full || k0 + 1 < nvalid) ? fast_exp2(x1) : 0.f;
                     const __nv_bfloat162 pb = __floats2bfloat162_rn(s0, s1);
                     e_sum += s0 + s1;
-                    r_sum += __low2float(pb) + __high2float(pb);
+                    const float2 pf2 = __bfloat1622float2(pb);
+                    r_sum += pf2.x + pf2.y;
                     pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&pb);
                 }
-                *reinterpret_cast<uint4*>(prow_smem + ((q ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                const int chunk = 4 * half + q;
+                *reinterpret_cast<uint4*>(prow_smem + ((chunk ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
             fence_proxy_async_smem();      // P is read by the tensor core (async proxy)
             tc_fence_before();
@@ -351,34 +375,44 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPvDone], (nblk - 1) & 1));
         tc_fence_after();
+        // the row sums of both halves (every softmax thread reaches these barriers)
+        float* xs = xchg + 2 * 2 * kRows;
+        xs[half * kRows + r] = e_sum;
+        ok = bar_and_all(ok);
+        const float e_tot = e_sum + xs[(half ^ 1) * kRows + r];
+        ok = bar_and_all(ok);
+        xs[half * kRows + r] = r_sum;
+        ok = bar_and_all(ok);
+        const float r_tot = r_sum + xs[(half ^ 1) * kRows + r];
         if (!ok) {
             atomicExch(failed_flag, 1);
             if (lane == 0) report(p.status, ARK_DEV_TIMEOUT);
         } else {
             // epilogue: o row = O / sum of the bf16 weights; lse from the fp32 weights.
-            // All lanes read TMEM; only rows of live positions are stored.
+            // This half writes dims 64*half .. +63.  All lanes read TMEM; only live rows are stored.
             const bool live = tr < nn;
-            const float inv = 1.f / r_sum;
+            const float inv = 1.f / r_tot;
             const int h = g * kGroup + hh;
-            uint16_t* orow = p.o + ((static_cast<size_t>(b) * p.S + tr) * p.Hq + h) * kHeadDim;
+            uint16_t* orow = p.o + ((static_cast<size_t>(b) * p.S + tr) * p.Hq + h) * kHeadDim + half * 64;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t o[32];
-                tmem_ld32(lane_base + kColO + c * 32, o);
+                uint32_t o[16];
+                tmem_ld16(lane_base + kColO + half * 64 + c * 16, o);
                 tmem_wait_ld();
                 if (live) {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
+                    for (int q = 0; q < 2; ++q) {
                         uint4 w;
                         w.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
                         w.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
                         w.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
                         w.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
-                        reinterpret_cast<uint4*>(orow + c * 32)[q] = w;
+                        reinterpret_cast<uint4*>(orow + c * 16)[q] = w;
                     }
                 }
             }
-            if (live) p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + tr] = (m_ref + __log2f(e_sum)) * kLn2;
+            if (live && half == 0)
+                p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + tr] = (m_ref + __log2f(e_tot)) * kLn2;
         }
     }
 
