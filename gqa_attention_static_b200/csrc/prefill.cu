@@ -26,7 +26,10 @@
 //     issues MMAs from one thread, warps 2..9 run the softmax: two threads
 //     per query row (TMEM lane), one for keys 0..31 and one for keys 32..63
 //     of each block, which trade their partial row maxima through shared
-//     memory behind one named barrier per block.
+//     memory behind one named barrier per block.  P (bf16) is stored back to
+//     tensor memory over the block's S columns and the PV MMA reads it from
+//     there (A operand in TMEM), so shared memory only stages Q, K and V and
+//     a K stage is released as soon as its QK MMA has completed.
 //     P (bf16) is written, in the swizzled K-major layout, over the block's K
 //     tile (which the QK MMA has finished with) and feeds the PV MMA.
 //   - Softmax in the log2 domain with a lazily moved reference max: O is
@@ -63,7 +66,7 @@ constexpr int kVStages = 2;
 
 // shared memory map (the dynamic shared memory base is 1024-aligned)
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + 2 * kQHalf;          // kKStages stages (P of a block is written over its K)
+constexpr int kOffK = kOffQ + 2 * kQHalf;          // kKStages stages
 constexpr int kOffV = kOffK + kKStages * kKV;      // kVStages stages
 constexpr int kOffBar = kOffV + kVStages * kKV;
 constexpr int kBarQ = 0;
@@ -179,7 +182,7 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
             tma_load_4d(smem + kOffQ + kQHalf, &p.qmap, 64, 0, g, qrow, &bars[kBarQ]);
             for (int j = 0; j < nblk; ++j) {
                 const int row = b * p.T + j * kBN;
-                // K stage (with the P written over it) is free once PV of block j-3 is done
+                // K stage is free once the QK MMA of block j - kKStages is done
                 const int ks = j % kKStages;
                 if (j >= kKStages && !mbar_wait(&bars[kBarKEmpty + ks], ((j / kKStages) - 1) & 1)) {
                     ok = false;
@@ -241,21 +244,21 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
                              umma_desc_sw128(kb + (kk >> 2) * kKHalf + sub, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&bars[kBarSFull + (j & 1)]);
+                umma_commit(&bars[kBarKEmpty + j % kKStages]);
             }
             __syncwarp();
         };
         auto issue_pv = [&](int j) {
             if (lane == 0) {
                 tc_fence_after();
-                const uint32_t pb = sbase + kOffK + (j % kKStages) * kKV;   // P of block j, over its K tile
+                // P of block j: bf16 pairs in the first 32 columns of its S buffer
+                const uint32_t pa = tmem + kColS + (j & 1) * kBN;
                 const uint32_t vb = sbase + kOffV + (j % kVStages) * kKV;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    umma_f16(tmem + kColO, umma_desc_sw128(pb + kk * 32, 16, 1024),
-                             umma_desc_sw128(vb + kk * 16 * 128, kKHalf, 1024), kIdescPV,
-                             (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_f16_ts(tmem + kColO, pa + kk * 8, umma_desc_sw128(vb + kk * 16 * 128, kKHalf, 1024),
+                                kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(&bars[kBarKEmpty + j % kKStages]);
                 umma_commit(&bars[kBarVEmpty + j % kVStages]);
                 umma_commit(&bars[kBarPvDone]);
             }
@@ -269,6 +272,7 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
                 if (!(ok = wait_k(j + 1))) break;
                 issue_qk(j + 1);
             }
+            // P of block j is in TMEM (and S buffer j&1 is not reused before PV(j): MMAs run in issue order)
             if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPFull + (j & 1)], (j >> 1) & 1)))) break;
             if (!(ok = wait_v(j))) break;
             issue_pv(j);
@@ -346,30 +350,25 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
                 }
                 tmem_wait_st();
             }
-            // P = exp2(s * scale_log2 - m_ref) as bf16, written over this block's K tile:
-            // row r is one 128-byte swizzled row; this half writes its 16-byte chunks 4*half .. +3
-            uint8_t* prow_smem = smem + kOffK + (j % kKStages) * kKV + r * 128;
+            // P = exp2(s * scale_log2 - m_ref) as bf16 pairs, stored over the block's S columns:
+            // keys 2c, 2c+1 in column c, this half's keys 32*half .. +31 in columns 16*half .. +15
+            // (both halves finished reading S before the barrier above)
             const bool full = nvalid >= 32;
+            uint32_t pk[16];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int i = 0; i < 8; i += 2) {
-                    const int k0 = q * 8 + i;
-                    const float x0 = __uint_as_float(v[k0]) * p.scale_log2 - mu;
-                    const float x1 = __uint_as_float(v[k0 + 1]) * p.scale_log2 - mu;
-                    const float s0 = (full || k0 < nvalid) ? fast_exp2(x0) : 0.f;
-                    const float s1 = (full || k0 + 1 < nvalid) ? fast_exp2(x1) : 0.f;
-                    const __nv_bfloat162 pb = __floats2bfloat162_rn(s0, s1);
-                    e_sum += s0 + s1;
-                    const float2 pf2 = __bfloat1622float2(pb);
-                    r_sum += pf2.x + pf2.y;
-                    pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&pb);
-                }
-                const int chunk = 4 * half + q;
-                *reinterpret_cast<uint4*>(prow_smem + ((chunk ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            for (int i = 0; i < 32; i += 2) {
+                const float x0 = __uint_as_float(v[i]) * p.scale_log2 - mu;
+                const float x1 = __uint_as_float(v[i + 1]) * p.scale_log2 - mu;
+                const float s0 = (full || i < nvalid) ? fast_exp2(x0) : 0.f;
+                const float s1 = (full || i + 1 < nvalid) ? fast_exp2(x1) : 0.f;
+                const __nv_bfloat162 pb = __floats2bfloat162_rn(s0, s1);
+                e_sum += s0 + s1;
+                const float2 pf2 = __bfloat1622float2(pb);
+                r_sum += pf2.x + pf2.y;
+                pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&pb);
             }
-            fence_proxy_async_smem();      // P is read by the tensor core (async proxy)
+            tmem_st16(lane_base + kColS + (j & 1) * kBN + half * 16, pk);
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars[kBarPFull + (j & 1)]);
         }
