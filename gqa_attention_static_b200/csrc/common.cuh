@@ -127,6 +127,20 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const void* map, int c0, 
         :: "r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)) : "memory");
 }
 
+// 4-D tiled TMA store of one box from shared memory (coordinates innermost
+// first).  The copy joins the issuing thread's bulk async-group: commit it
+// and wait (bulk_wait_read) before the shared memory is reused or released.
+__device__ __forceinline__ void tma_store_4d(const void* map, const void* src, int c0, int c1, int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+        :: "l"(map), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3) : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// wait until every committed bulk store of this thread has read its source
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
 // ---------------------------------------------- tcgen05 (5th-gen tensor core) ----
 
 // Allocate `cols` TMEM columns (power of two >= 32); the base address is

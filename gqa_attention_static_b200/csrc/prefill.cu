@@ -9,8 +9,12 @@
 // p = pos0[b] + t, attends to the cache rows j <= p of its KV head.
 //
 // Tiling (B200):
-//   - One CTA per (16 query positions, KV head g, request b), the tiles with
-//     the longest key ranges launched first.  Its 128 MMA
+//   - One CTA per live tile (16 query positions of request b, KV head g).
+//     The grid is the upper bound Hkv x B x ceil(S/16); CTA k takes the k-th
+//     live tile in order of decreasing absolute position (longest key range
+//     first), found on the device from pos0/n_new by a binary search over
+//     position levels, so the CTAs that have no tile are the last ones
+//     dispatched and never hold a slot ahead of real work.  Its 128 MMA
 //     rows are the 16 positions x the 8 query heads of group g, so every K/V
 //     block is read once for all 8 heads (GQA packing).  The Q tile arrives
 //     by two 4-D TMA boxes (64 head-dim elements each, 128-byte swizzle),
@@ -30,8 +34,6 @@
 //     tensor memory over the block's S columns and the PV MMA reads it from
 //     there (A operand in TMEM), so shared memory only stages Q, K and V and
 //     a K stage is released as soon as its QK MMA has completed.
-//     P (bf16) is written, in the swizzled K-major layout, over the block's K
-//     tile (which the QK MMA has finished with) and feeds the PV MMA.
 //   - Softmax in the log2 domain with a lazily moved reference max: O is
 //     rescaled (read, scale, write back in TMEM) only when a row's block max
 //     exceeds its reference by more than 2^8, which for real data is almost
@@ -100,6 +102,7 @@ struct Params {
     CUtensorMap qmap;    // q as (128, 8, Hq/8, B*S), box (64, 8, 1, 16)
     CUtensorMap kmap;    // cache_k as (128, Hkv, B*T), box (64, 1, 64)
     CUtensorMap vmap;
+    CUtensorMap omap;    // o as (128, 8, Hq/8, B*S), box (64, 8, 1, 1): one position, 8 heads, 64 dims
     uint16_t* o;         // [B, S, Hq, 128]
     float* lse;          // [B, Hq, S]
     const int32_t* pos0;
@@ -124,40 +127,111 @@ __device__ __forceinline__ bool bar_and_all(bool pred) {
     return out != 0;
 }
 
-__global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_constant__ pf::Params p) {
-    using namespace pf;
-    extern __shared__ __align__(1024) uint8_t smem[];
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    // the grid runs the latest query tiles (longest key ranges) first, so the
-    // short tiles fill in behind them
-    const int qt = gridDim.z - 1 - blockIdx.z;
-    const int g = blockIdx.x;
-    const int b = blockIdx.y;
+namespace pf {
 
-    // ---- lengths (device values: checked here)
+// Request b's lengths as the kernel uses them (device values, clamped into
+// range; `bad` when they had to be), and its tiles' position levels: tile qt
+// of request b sits at level (pos0 >> 4) + qt, and the request has
+// ceil(n_new / 16) tiles.
+struct ReqTiles {
+    int nn, p0, lev0, ntiles;
+    bool bad;
+};
+
+__device__ __forceinline__ ReqTiles req_tiles(const Params& p, int b) {
+    ReqTiles t;
     int nn = __ldg(p.n_new + b);
     int p0 = __ldg(p.pos0 + b);
-    if (nn < 0 || nn > p.S || p0 < 0 || p0 + (nn < 0 ? 0 : (nn > p.S ? p.S : nn)) > p.T) {
-        if (threadIdx.x == 0 && qt == 0 && g == 0) report(p.status, ARK_DEV_BAD_POS);
+    t.bad = nn < 0 || nn > p.S || p0 < 0 || p0 + (nn < 0 ? 0 : (nn > p.S ? p.S : nn)) > p.T;
+    if (t.bad) {
         nn = nn < 0 ? 0 : (nn > p.S ? p.S : nn);
         if (p0 < 0) p0 = 0;
         if (p0 > p.T) p0 = p.T;
         if (p0 + nn > p.T) nn = p.T - p0;
     }
-    const int t0 = qt * kPos;
-    if (t0 >= nn) return;                                   // whole CTA: no live row
+    t.nn = nn;
+    t.p0 = p0;
+    t.lev0 = p0 >> 4;
+    t.ntiles = (nn + kPos - 1) / kPos;
+    return t;
+}
+
+// tiles of a request at levels >= lam
+__device__ __forceinline__ int tiles_at_or_above(const ReqTiles& t, int lam) {
+    const int c = t.lev0 + t.ntiles - max(lam, t.lev0);
+    return c < 0 ? 0 : c;
+}
+
+// The j-th live tile in the order (level descending, request ascending),
+// computed by one warp (every lane returns the same result).  Lane l handles
+// requests l, l + 32, ...; C(lam) = tiles at levels >= lam is non-increasing,
+// and the tile's level is the largest lam with C(lam) > j.
+struct TilePick {
+    int b, qt, nn, p0;
+    bool live;
+};
+
+__device__ __forceinline__ TilePick pick_tile(const Params& p, int j, int lane, bool report_bad) {
+    const unsigned full = 0xffffffffu;
+    ReqTiles mine{0, 0, 0, 0, false};
+    if (lane < p.B) mine = req_tiles(p, lane);
+    bool bad = mine.bad;
+    auto count = [&](int lam) {
+        int c = lane < p.B ? tiles_at_or_above(mine, lam) : 0;
+        for (int bb = 32 + lane; bb < p.B; bb += 32) {
+            const ReqTiles t = req_tiles(p, bb);
+            c += tiles_at_or_above(t, lam);
+            bad |= t.bad;
+        }
+        return static_cast<int>(__reduce_add_sync(full, static_cast<unsigned>(c)));
+    };
+    TilePick r{0, 0, 0, 0, false};
+    const int total = count(0);
+    if (report_bad && __any_sync(full, bad) && lane == 0) report(p.status, ARK_DEV_BAD_POS);
+    if (j >= total) return r;
+    int lo = 0, hi = (p.T + kPos - 1) / kPos;     // C(lo) > j, C(hi) == 0
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (count(mid) > j) lo = mid;
+        else hi = mid;
+    }
+    int rank = j - count(lo + 1);                 // among the tiles at level lo, by request
+    for (int base = 0; base < p.B; base += 32) {
+        const ReqTiles t = base == 0 ? mine : (base + lane < p.B ? req_tiles(p, base + lane) : ReqTiles{0, 0, 0, 0, false});
+        const bool at = base + lane < p.B && t.lev0 <= lo && lo < t.lev0 + t.ntiles;
+        const unsigned m = __ballot_sync(full, at);
+        const int n = __popc(m);
+        if (rank < n) {
+            const int src = static_cast<int>(__fns(m, 0, rank + 1));
+            r.b = base + src;
+            r.nn = __shfl_sync(full, t.nn, src);
+            r.p0 = __shfl_sync(full, t.p0, src);
+            r.qt = lo - __shfl_sync(full, t.lev0, src);
+            r.live = true;
+            return r;
+        }
+        rank -= n;
+    }
+    return r;                                     // not reached for consistent counts
+}
+
+}  // namespace pf
+
+__global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_constant__ pf::Params p) {
+    using namespace pf;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = blockIdx.x % p.Hkv;
     if (smem_u32(smem) & 1023u) {                           // the swizzled layouts need 1024-byte alignment
         if (threadIdx.x == 0) report(p.status, ARK_DEV_TIMEOUT);
         return;
     }
-    const int kv_end = p0 + min(t0 + kPos, nn);             // keys visible to the tile's last row
-    const int nblk = (kv_end + kBN - 1) / kBN;
-
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
     int* failed_flag = reinterpret_cast<int*>(smem + kOffFlag);
 
+    // barrier init and the TMEM allocation overlap the tile search's loads
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNumBars; ++i)
             mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? kSoftmaxThreads : 1);
@@ -165,43 +239,69 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_ptr, kTmemCols);
+    // every warp finds the CTA's tile by itself (same inputs, same result)
+    const TilePick tile = pick_tile(p, blockIdx.x / p.Hkv, lane, blockIdx.x == 0 && warp == 0);
+    const int b = tile.b, qt = tile.qt, nn = tile.nn, p0 = tile.p0;
+    const int t0 = qt * kPos;
+    const int kv_end = p0 + min(t0 + kPos, nn);             // keys visible to the tile's last row
+    const int nblk = tile.live ? (kv_end + kBN - 1) / kBN : 0;
+
+    auto load_k = [&](int j) {
+        const int ks = j % kKStages;
+        mbar_arrive_expect_tx(&bars[kBarKFull + ks], kKV);
+        uint8_t* kd = smem + kOffK + ks * kKV;
+        tma_load_3d(kd, &p.kmap, 0, g, b * p.T + j * kBN, &bars[kBarKFull + ks]);
+        tma_load_3d(kd + kKHalf, &p.kmap, 64, g, b * p.T + j * kBN, &bars[kBarKFull + ks]);
+    };
+    auto load_v = [&](int j) {
+        const int vs = j % kVStages;
+        mbar_arrive_expect_tx(&bars[kBarVFull + vs], kKV);
+        uint8_t* vd = smem + kOffV + vs * kKV;
+        tma_load_3d(vd, &p.vmap, 0, g, b * p.T + j * kBN, &bars[kBarVFull + vs]);
+        tma_load_3d(vd + kKHalf, &p.vmap, 64, g, b * p.T + j * kBN, &bars[kBarVFull + vs]);
+    };
+    // the first blocks need no free stage: thread 0 (which initialised the
+    // barriers) issues them before the CTA barrier
+    constexpr int kPre = 2;
+    static_assert(kKStages >= kPre && kVStages >= kPre, "preloaded blocks need their own stages");
+    if (threadIdx.x == 0 && tile.live) {
+        mbar_arrive_expect_tx(&bars[kBarQ], 2 * kQHalf);
+        const int qrow = b * p.S + t0;
+        tma_load_4d(smem + kOffQ, &p.qmap, 0, 0, g, qrow, &bars[kBarQ]);
+        tma_load_4d(smem + kOffQ + kQHalf, &p.qmap, 64, 0, g, qrow, &bars[kBarQ]);
+        for (int j = 0; j < min(nblk, kPre); ++j) {
+            load_k(j);
+            load_v(j);
+        }
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_ptr;
+    if (!tile.live) {                                       // whole CTA: no live tile
+        if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+        return;
+    }
     const uint32_t sbase = smem_u32(smem);
 
     if (warp == 0) {
         // ================================================= TMA producer
         if (lane == 0) {
             bool ok = true;
-            mbar_arrive_expect_tx(&bars[kBarQ], 2 * kQHalf);
-            const int qrow = b * p.S + t0;
-            tma_load_4d(smem + kOffQ, &p.qmap, 0, 0, g, qrow, &bars[kBarQ]);
-            tma_load_4d(smem + kOffQ + kQHalf, &p.qmap, 64, 0, g, qrow, &bars[kBarQ]);
-            for (int j = 0; j < nblk; ++j) {
-                const int row = b * p.T + j * kBN;
+            for (int j = kPre; j < nblk; ++j) {
                 // K stage is free once the QK MMA of block j - kKStages is done
-                const int ks = j % kKStages;
-                if (j >= kKStages && !mbar_wait(&bars[kBarKEmpty + ks], ((j / kKStages) - 1) & 1)) {
+                if (!mbar_wait(&bars[kBarKEmpty + j % kKStages], ((j / kKStages) - 1) & 1)) {
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(&bars[kBarKFull + ks], kKV);
-                uint8_t* kd = smem + kOffK + ks * kKV;
-                tma_load_3d(kd, &p.kmap, 0, g, row, &bars[kBarKFull + ks]);
-                tma_load_3d(kd + kKHalf, &p.kmap, 64, g, row, &bars[kBarKFull + ks]);
-                // V stage is free once PV of block j-2 is done
-                const int vs = j % kVStages;
-                if (j >= kVStages && !mbar_wait(&bars[kBarVEmpty + vs], ((j / kVStages) - 1) & 1)) {
+                load_k(j);
+                // V stage is free once PV of block j - kVStages is done
+                if (!mbar_wait(&bars[kBarVEmpty + j % kVStages], ((j / kVStages) - 1) & 1)) {
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(&bars[kBarVFull + vs], kKV);
-                uint8_t* vd = smem + kOffV + vs * kKV;
-                tma_load_3d(vd, &p.vmap, 0, g, row, &bars[kBarVFull + vs]);
-                tma_load_3d(vd + kKHalf, &p.vmap, 64, g, row, &bars[kBarVFull + vs]);
+                load_v(j);
             }
             if (!ok) {
                 atomicExch(failed_flag, 1);
@@ -388,26 +488,37 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
             if (lane == 0) report(p.status, ARK_DEV_TIMEOUT);
         } else {
             // epilogue: o row = O / sum of the bf16 weights; lse from the fp32 weights.
-            // This half writes dims 64*half .. +63.  All lanes read TMEM; only live rows are stored.
+            // This half's 64 dims of the row go, as bf16, to the (finished) Q tile in shared
+            // memory, in the 128-byte-swizzled layout of a (64, 8 heads) TMA box per position;
+            // each warp then stores its 4 positions (its 32 rows) with TMA, live positions only.
             const bool live = tr < nn;
             const float inv = 1.f / r_tot;
             const int h = g * kGroup + hh;
-            uint16_t* orow = p.o + ((static_cast<size_t>(b) * p.S + tr) * p.Hq + h) * kHeadDim + half * 64;
+            uint8_t* stage = smem + kOffQ + half * kQHalf + r * 128;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[16];
                 tmem_ld16(lane_base + kColO + half * 64 + c * 16, o);
                 tmem_wait_ld();
-                if (live) {
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
-                        w.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
-                        w.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
-                        w.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
-                        reinterpret_cast<uint4*>(orow + c * 16)[q] = w;
-                    }
+                for (int q = 0; q < 2; ++q) {
+                    uint4 w;
+                    w.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
+                    w.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
+                    w.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
+                    w.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
+                    *reinterpret_cast<uint4*>(stage + (((2 * c + q) ^ (r & 7)) << 4)) = w;
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane < 4) {
+                const int pp = quad * 4 + lane;              // position of the tile
+                if (t0 + pp < nn) {
+                    tma_store_4d(&p.omap, smem + kOffQ + half * kQHalf + pp * 1024, half * 64, 0, g,
+                                 b * p.S + t0 + pp);
+                    bulk_commit();
+                    bulk_wait_read();
                 }
             }
             if (live && half == 0)
@@ -458,7 +569,8 @@ extern "C" ark_status ark_attn_prefill(const void* q, const void* cache_k, const
     pf::Params prm{};
     if (!q_group_tensor_map(&prm.qmap, q, static_cast<long long>(B) * S, Hq, 64, pf::kPos) ||
         !kv_tensor_map(&prm.kmap, cache_k, static_cast<long long>(B) * T, Hkv, 64, pf::kBN) ||
-        !kv_tensor_map(&prm.vmap, cache_v, static_cast<long long>(B) * T, Hkv, 64, pf::kBN))
+        !kv_tensor_map(&prm.vmap, cache_v, static_cast<long long>(B) * T, Hkv, 64, pf::kBN) ||
+        !q_group_tensor_map(&prm.omap, o, static_cast<long long>(B) * S, Hq, 64, 1))
         return ARK_ERR_CUDA;
     prm.o = static_cast<uint16_t*>(o);
     prm.lse = lse;
@@ -475,8 +587,8 @@ extern "C" ark_status ark_attn_prefill(const void* q, const void* cache_k, const
             return ARK_ERR_CUDA;
         g_prefill_attr[dev] = true;
     }
-    if ((S + pf::kPos - 1) / pf::kPos > 65535) return ARK_ERR_UNSUPPORTED;
-    dim3 grid(Hkv, B, (S + pf::kPos - 1) / pf::kPos);
-    prefill_kernel<<<grid, pf::kThreads, pf::kSmemBytes, stream>>>(prm);
+    const long long ctas = static_cast<long long>(Hkv) * B * ((S + pf::kPos - 1) / pf::kPos);
+    if (ctas >= (1LL << 31)) return ARK_ERR_UNSUPPORTED;
+    prefill_kernel<<<static_cast<unsigned>(ctas), pf::kThreads, pf::kSmemBytes, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
 }
