@@ -591,7 +591,7 @@ def main():
                        "path": ("per-layer calls" if args.per_layer else "layer-batched calls") +
                                " replayed from one CUDA graph"},
             "tokens_layers_per_s": tl,
-            "roofline": {"kernel": "decode_kernel (ark_attn_decode%s, merge fused)" %
+            "roofline": {"kernel": "decode_kernel + merge_kernel (one ark_attn_decode%s call)" %
                                    ("" if args.per_layer else "_layers"),
                          "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,

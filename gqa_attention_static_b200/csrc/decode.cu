@@ -36,10 +36,13 @@
 //     ldmatrix.trans on the same V tile.  fp32 online softmax in the log2
 //     domain; per-head maxima across positions by warp shuffles.
 //   - A warp that covers a whole segment writes o/lse directly.  A cut
-//     segment's pieces write normalised fp32 partials (at most two per warp)
-//     and bump a per-segment counter; the warp that arrives last merges the
-//     pieces by log-sum-exp (they are still in L2) and resets the counter to
-//     zero.  No warp ever waits for another.
+//     segment's pieces write normalised fp32 partials (at most two per warp,
+//     with an L2 evict-last hint while the K/V stream is marked evict-first)
+//     and the warp moves on: no fence, no counter, no warp ever waits for
+//     another.  A second, small kernel (merge_kernel, launched with
+//     programmatic dependent launch so that it is resident as soon as decode
+//     CTAs retire) recomputes the same partition and merges the pieces of
+//     every cut segment by log-sum-exp.
 //
 // Why tensor cores: per (position, KV head) the kernel reads 512 B and does
 // 2 x 8 x 128 multiply-adds, 4 FMA per byte.  At B200 HBM rates that needs
@@ -70,7 +73,6 @@ struct DecodeCore {
     uint32_t* status;
     float* part_o;       // [kMaxWarps][2][8][D]  two partial slots per warp
     float* part_lse;     // [kMaxWarps][2][8]
-    int* counters;       // [L][B][Hkv]
     int L, B, T, Hq, Hkv;
     int min_tiles;       // fewest tiles one warp takes (bounds the pieces per segment)
     int masked;
@@ -100,6 +102,49 @@ struct CombineParams {
 };
 
 __device__ __forceinline__ int clamp_len(int x, int T) { return x < 0 ? 0 : (x > T ? T : x); }
+
+// Prefix over the batch of the tiles per request (all KV heads of it):
+// s_pref[b] = first tile of request b within a layer, s_pref[B] = tiles per
+// layer.  Run by one warp; `report` flags lengths outside [0, T].
+__device__ __forceinline__ void tile_prefix(const DecodeCore& c, int* s_pref, int lane, bool report_bad) {
+    if (lane == 0) s_pref[0] = 0;
+    int run = 0;
+    for (int base = 0; base < c.B; base += 32) {
+        const int b = base + lane;
+        int n = 0;
+        if (b < c.B) {
+            const int raw = __ldg(c.kv_len + b);
+            if ((raw < 0 || raw > c.T) && report_bad) report(c.status, ARK_DEV_BAD_KVLEN);
+            const int hi = c.masked ? c.T : clamp_len(raw, c.T);
+            n = max(1, (hi + kTileRows - 1) / kTileRows) * c.Hkv;
+        }
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, n, off);
+            if (lane >= off) n += y;
+        }
+        if (b < c.B) s_pref[b + 1] = run + n;
+        run += __shfl_sync(0xffffffffu, n, 31);
+    }
+}
+
+// Warps of the decode partition: as many as give every warp at least
+// min_tiles tiles, at most the launch's warps.  Warp w takes tiles
+// [w N / W, (w + 1) N / W).
+__device__ __forceinline__ int partition_warps(const DecodeCore& c, int N, int launch_warps) {
+    int W = N / c.min_tiles;
+    if (W < 1) W = 1;
+    if (W > launch_warps) W = launch_warps;
+    return W;
+}
+
+template <int MaxL>
+struct MergeParamsT {
+    DecodeCore c;
+    uint16_t* o[MaxL];
+    float* lse[MaxL];
+    int decode_warps;    // warps of the decode launch whose partials are merged
+};
 
 // One segment = (layer, request, KV head): its tiles are s0 .. s0+n-1 of the
 // global tile list.  Tile indices fit in 32 bits (the host checks the size).
@@ -251,27 +296,9 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     int* s_pref = reinterpret_cast<int*>(smem + kRingBytes + kQBytes + kBarBytes);   // [B + 1]
 
     // ---- per CTA: prefix over the batch of the tiles per request (all KV heads)
-    if (warp == 0) {
-        if (lane == 0) s_pref[0] = 0;
-        int run = 0;
-        for (int base = 0; base < c.B; base += 32) {
-            const int b = base + lane;
-            int n = 0;
-            if (b < c.B) {
-                const int raw = __ldg(c.kv_len + b);
-                if ((raw < 0 || raw > c.T) && blockIdx.x == 0) report(c.status, ARK_DEV_BAD_KVLEN);
-                const int hi = c.masked ? c.T : clamp_len(raw, c.T);
-                n = max(1, (hi + kTileRows - 1) / kTileRows) * c.Hkv;
-            }
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, n, off);
-                if (lane >= off) n += y;
-            }
-            if (b < c.B) s_pref[b + 1] = run + n;
-            run += __shfl_sync(0xffffffffu, n, 31);
-        }
-    }
+    if (warp == 0) tile_prefix(c, s_pref, lane, blockIdx.x == 0);
+    // the merge grid may be scheduled from here on (it waits for this grid's completion)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (lane == 0) {
         for (int s = 0; s <= kStages; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
@@ -281,9 +308,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
 
     const int per_layer = s_pref[c.B];
     const int N = per_layer * c.L;
-    int W = N / c.min_tiles;
-    if (W < 1) W = 1;
-    if (W > static_cast<int>(gridDim.x) * kWarps) W = static_cast<int>(gridDim.x) * kWarps;
+    const int W = partition_warps(c, N, static_cast<int>(gridDim.x) * kWarps);
     const int w = blockIdx.x * kWarps + warp;
     if (w >= W) return;
     // warp w takes tiles [T0, T1); tile t belongs to warp floor(((t+1) W - 1) / N)
@@ -299,6 +324,10 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     const uint32_t v_row = kTileBytes + (lr + 8 * (lm >> 1)) * 128;   // V^T: rows 8*(lm>>1)
     const uint32_t v_x = (lm & 1) ^ lr;                        //      column chunk lm&1
 
+    // K/V rows are read once per launch; partials are read back by the merge
+    const uint64_t pol_stream = l2_policy_evict_first();
+    const uint64_t pol_keep = l2_policy_evict_last();
+
     // ---- producer cursor: next tile to issue
     int tp = T0;
     int pj;
@@ -310,10 +339,10 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
             uint8_t* dst = ring + st * kStageBytes;
             const int row = ps.b * c.T + pj * kTileRows;
             mbar_arrive_expect_tx(&bars[st], kStageBytes);
-            tma_load_3d(dst, &p.kmap[ps.l], 0, ps.g, row, &bars[st]);
-            tma_load_3d(dst + kHalfBytes, &p.kmap[ps.l], 64, ps.g, row, &bars[st]);
-            tma_load_3d(dst + kTileBytes, &p.vmap[ps.l], 0, ps.g, row, &bars[st]);
-            tma_load_3d(dst + kTileBytes + kHalfBytes, &p.vmap[ps.l], 64, ps.g, row, &bars[st]);
+            tma_load_3d_hint(dst, &p.kmap[ps.l], 0, ps.g, row, &bars[st], pol_stream);
+            tma_load_3d_hint(dst + kHalfBytes, &p.kmap[ps.l], 64, ps.g, row, &bars[st], pol_stream);
+            tma_load_3d_hint(dst + kTileBytes, &p.vmap[ps.l], 0, ps.g, row, &bars[st], pol_stream);
+            tma_load_3d_hint(dst + kTileBytes + kHalfBytes, &p.vmap[ps.l], 64, ps.g, row, &bars[st], pol_stream);
         }
         ++pseq;
         ++tp;
@@ -473,7 +502,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
         if (++cj < cs.n && t + 1 < T1) continue;
 
         // ---- the consumer leaves segment cs: publish its result
-        if (failed) m0 = m1 = -INFINITY;   // an empty result keeps the merge counters consistent
+        if (failed) m0 = m1 = -INFINITY;   // a timed-out piece publishes an empty result (lse -inf)
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
             e0 += __shfl_xor_sync(0xffffffffu, e0, o);
@@ -509,28 +538,14 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 const int d = 16 * mt + gid;
-                po[h0 * kHeadDim + d] = acc[mt][0] * inv0;
-                po[h1 * kHeadDim + d] = acc[mt][1] * inv1;
-                po[h0 * kHeadDim + d + 8] = acc[mt][2] * inv0;
-                po[h1 * kHeadDim + d + 8] = acc[mt][3] * inv1;
+                st_f32_hint(po + h0 * kHeadDim + d, acc[mt][0] * inv0, pol_keep);
+                st_f32_hint(po + h1 * kHeadDim + d, acc[mt][1] * inv1, pol_keep);
+                st_f32_hint(po + h0 * kHeadDim + d + 8, acc[mt][2] * inv0, pol_keep);
+                st_f32_hint(po + h1 * kHeadDim + d + 8, acc[mt][3] * inv1, pol_keep);
             }
             if (gid == 0) {
-                c.part_lse[(static_cast<size_t>(w) * 2 + slot) * kGroup + h0] = lse0;
-                c.part_lse[(static_cast<size_t>(w) * 2 + slot) * kGroup + h1] = lse1;
-            }
-            // warps whose ranges meet this segment: wa .. wb
-            const int wa = static_cast<int>((static_cast<long long>(cs.s0 + 1) * W - 1) / N);
-            const int wb = static_cast<int>((static_cast<long long>(cs.s0 + cs.n) * W - 1) / N);
-            __threadfence();
-            __syncwarp();
-            int last = 0;
-            int* cnt = c.counters + (static_cast<size_t>(cs.l) * c.B + cs.b) * c.Hkv + cs.g;
-            if (lane == 0) last = (atomicAdd(cnt, 1) == wb - wa);
-            last = __shfl_sync(0xffffffffu, last, 0);
-            if (last) {
-                __threadfence();
-                merge_pieces(c, p.o[cs.l], p.lse[cs.l], cs, wa, wb, W, N, lane, bh0);
-                if (lane == 0) atomicExch(cnt, 0);
+                st_f32_hint(c.part_lse + (static_cast<size_t>(w) * 2 + slot) * kGroup + h0, lse0, pol_keep);
+                st_f32_hint(c.part_lse + (static_cast<size_t>(w) * 2 + slot) * kGroup + h1, lse1, pol_keep);
             }
         }
         if (t + 1 < T1) {
@@ -546,6 +561,39 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
             (void)mbar_wait(&bars[q2 % kStages], (q2 / kStages) & 1);
         if (qissued > qseq) (void)mbar_wait(qbar, qseq & 1);
     }
+}
+
+// One warp per segment (layer, request, KV head): if the decode partition cut
+// it, merge its pieces.  Launched right after decode_kernel on the same
+// stream, possibly before it has finished (programmatic dependent launch):
+// the prefix only reads kv_len; griddepcontrol.wait then blocks until the
+// decode grid has completed and its writes are visible.
+template <int MaxL>
+__global__ void __launch_bounds__(kWarps * 32) merge_kernel(const __grid_constant__ MergeParamsT<MaxL> p) {
+    extern __shared__ int s_pref_m[];
+    const DecodeCore& c = p.c;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp == 0) tile_prefix(c, s_pref_m, lane, false);
+    __syncthreads();
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int per_layer = s_pref_m[c.B];
+    const int N = per_layer * c.L;
+    const int W = partition_warps(c, N, p.decode_warps);
+    const int sid = blockIdx.x * kWarps + warp;
+    if (sid >= c.L * c.B * c.Hkv) return;
+    Seg cs;
+    cs.l = sid / (c.B * c.Hkv);
+    const int rem = sid - cs.l * c.B * c.Hkv;
+    cs.b = rem / c.Hkv;
+    cs.g = rem - cs.b * c.Hkv;
+    cs.n = (s_pref_m[cs.b + 1] - s_pref_m[cs.b]) / c.Hkv;
+    cs.s0 = cs.l * per_layer + s_pref_m[cs.b] + cs.g * cs.n;
+    const int wa = static_cast<int>((static_cast<long long>(cs.s0 + 1) * W - 1) / N);
+    const int wb = static_cast<int>((static_cast<long long>(cs.s0 + cs.n) * W - 1) / N);
+    if (wa == wb) return;                    // one warp covered it and wrote o directly
+    const size_t bh0 = static_cast<size_t>(cs.b) * c.Hq + cs.g * kGroup;
+    merge_pieces(c, p.o[cs.l], p.lse[cs.l], cs, wa, wb, W, N, lane, bh0);
 }
 
 // One warp per (b, h): merge nsplit normalised partials by log-sum-exp.
@@ -600,15 +648,16 @@ int decode_min_tiles(int T, int max_splits) {
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct WsLayout {
-    size_t part_o, part_lse, counters, total;
+    size_t part_o, part_lse, total;
 };
 
-WsLayout ws_layout(int L, int B, int Hkv) {
+// Partials of up to kMaxWarps warps, two slots each; nothing in it needs
+// initialising and no call leaves state in it for the next.
+WsLayout ws_layout() {
     WsLayout w{};
     w.part_o = 0;
     w.part_lse = align256(static_cast<size_t>(kMaxWarps) * 2 * kGroup * kHeadDim * sizeof(float));
-    w.counters = w.part_lse + align256(static_cast<size_t>(kMaxWarps) * 2 * kGroup * sizeof(float));
-    w.total = w.counters + align256(static_cast<size_t>(L) * B * Hkv * sizeof(int));
+    w.total = w.part_lse + align256(static_cast<size_t>(kMaxWarps) * 2 * kGroup * sizeof(float));
     return w;
 }
 
@@ -622,6 +671,8 @@ ark_status check_decode_shape(int B, int T, int Hq, int Hkv, int D) {
 }
 
 size_t decode_smem(int B) { return 1024 + kRingBytes + kQBytes + kBarBytes + align256((B + 1) * sizeof(int)); }
+
+size_t merge_smem(int B) { return align256((B + 1) * sizeof(int)); }
 
 // SM count and resident CTAs per SM, queried once per device and kernel.
 struct DeviceInfo {
@@ -638,6 +689,9 @@ ark_status device_info(DeviceInfo& out) {
         if (cudaFuncSetAttribute(decode_kernel<MaxL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(decode_smem(kMaxBatch))) != cudaSuccess)
             return ARK_ERR_CUDA;
+        if (cudaFuncSetAttribute(merge_kernel<MaxL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(merge_smem(kMaxBatch))) != cudaSuccess)
+            return ARK_ERR_CUDA;
         int sms = 0, per = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ARK_ERR_CUDA;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_kernel<MaxL>, kWarps * 32,
@@ -647,6 +701,33 @@ ark_status device_info(DeviceInfo& out) {
         d.sms = sms;
     }
     out = d;
+    return ARK_OK;
+}
+
+// The merge of cut segments: one warp per segment, launched behind the decode
+// grid with programmatic stream serialisation (see merge_kernel).
+template <int MaxL>
+ark_status launch_merge(const DecodeParamsT<MaxL>& prm, int decode_warps, cudaStream_t stream) {
+    const DecodeCore& c = prm.c;
+    static thread_local MergeParamsT<MaxL> mp;
+    mp.c = c;
+    for (int l = 0; l < c.L; ++l) {
+        mp.o[l] = prm.o[l];
+        mp.lse[l] = prm.lse[l];
+    }
+    mp.decode_warps = decode_warps;
+    const long long segs = static_cast<long long>(c.L) * c.B * c.Hkv;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>((segs + kWarps - 1) / kWarps));
+    cfg.blockDim = dim3(kWarps * 32);
+    cfg.dynamicSmemBytes = merge_smem(c.B);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, merge_kernel<MaxL>, mp) != cudaSuccess) return ARK_ERR_CUDA;
     return ARK_OK;
 }
 
@@ -670,19 +751,19 @@ ark_status launch_decode_core(DecodeParamsT<MaxL>& prm, const void* const* k, co
     if (grid > max_warps / kWarps) grid = max_warps / kWarps;
     if (grid < 1) grid = 1;
     decode_kernel<MaxL><<<static_cast<unsigned>(grid), kWarps * 32, decode_smem(c.B), stream>>>(prm);
-    return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return ARK_ERR_CUDA;
+    return launch_merge<MaxL>(prm, static_cast<int>(grid) * kWarps, stream);
 }
 
 template <int MaxL>
 ark_status launch_decode(DecodeParamsT<MaxL>& prm, const void* const* k, const void* const* v, void* workspace,
                          size_t ws_bytes, int max_warps, cudaStream_t stream) {
     DecodeCore& c = prm.c;
-    const WsLayout w = ws_layout(c.L, c.B, c.Hkv);
+    const WsLayout w = ws_layout();
     if (!workspace || ws_bytes < w.total || !aligned16(workspace)) return ARK_ERR_WORKSPACE;
     uint8_t* base = static_cast<uint8_t*>(workspace);
     c.part_o = reinterpret_cast<float*>(base + w.part_o);
     c.part_lse = reinterpret_cast<float*>(base + w.part_lse);
-    c.counters = reinterpret_cast<int*>(base + w.counters);
     return launch_decode_core<MaxL>(prm, k, v, max_warps, stream);
 }
 
@@ -710,7 +791,7 @@ ark_status fill_common(DecodeCore& c, const int32_t* kv_len, int L, int B, int T
 
 extern "C" size_t ark_attn_decode_layers_workspace_size(int L, int B, int Hq, int D, int T, int max_splits) {
     if (L <= 0 || B <= 0 || Hq <= 0 || D <= 0 || T <= 0 || max_splits <= 0 || Hq % kGroup) return 0;
-    return ws_layout(L, B, Hq / kGroup).total;
+    return ws_layout().total;
 }
 
 extern "C" size_t ark_attn_decode_workspace_size(int B, int Hq, int D, int T, int max_splits) {
@@ -777,8 +858,7 @@ extern "C" ark_status ark_attn_combine(const float* o_part, const float* lse_par
 
 // ------------------------------------------------ decode without allocation ----
 // Scratch of ark_attn_decode_noalloc: partial results for up to
-// kNoAllocWarps warps and merge counters for up to kNoAllocMaxSegments
-// (request, KV head) pairs, in one file-scope device array that every GPU
+// kNoAllocWarps warps, in one file-scope device array that every GPU
 // loading this library holds until the process exits.  Host code must not pass
 // the array's name to a kernel (on the host it is a stand-in, not a device
 // address); each device's address is looked up once with
@@ -786,11 +866,9 @@ extern "C" ark_status ark_attn_combine(const float* o_part, const float* lse_par
 namespace {
 
 constexpr int kNoAllocWarps = 512;
-constexpr int kNoAllocMaxSegments = 4096;
 constexpr size_t kNoAllocPartO = static_cast<size_t>(kNoAllocWarps) * 2 * kGroup * kHeadDim * sizeof(float);
 constexpr size_t kNoAllocPartLse = static_cast<size_t>(kNoAllocWarps) * 2 * kGroup * sizeof(float);
-constexpr size_t kNoAllocCounters = static_cast<size_t>(kNoAllocMaxSegments) * sizeof(int);
-constexpr size_t kNoAllocBytes = kNoAllocPartO + kNoAllocPartLse + kNoAllocCounters;   // about 4.1 MB
+constexpr size_t kNoAllocBytes = kNoAllocPartO + kNoAllocPartLse;   // about 4.2 MB
 
 }  // namespace
 
@@ -826,7 +904,6 @@ extern "C" ark_status ark_attn_decode_noalloc(const void* q, const void* cache_k
     DecodeParamsT<1> prm{};
     ark_status st = fill_common(prm.c, kv_len, 1, B, T, Hq, Hkv, D, scale, mode, max_splits, d_status);
     if (st != ARK_OK) return st;
-    if (static_cast<long long>(B) * Hkv > kNoAllocMaxSegments) return ARK_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(cache_k) || !aligned16(cache_v) || !aligned16(o) ||
         (reinterpret_cast<uintptr_t>(lse) & 3u))
         return ARK_ERR_INVALID_ARG;
@@ -835,10 +912,6 @@ extern "C" ark_status ark_attn_decode_noalloc(const void* q, const void* cache_k
     uint8_t* b8 = static_cast<uint8_t*>(base);
     prm.c.part_o = reinterpret_cast<float*>(b8);
     prm.c.part_lse = reinterpret_cast<float*>(b8 + kNoAllocPartO);
-    prm.c.counters = reinterpret_cast<int*>(b8 + kNoAllocPartO + kNoAllocPartLse);
-    // the counters must start at zero; the array keeps whatever the last call left
-    if (cudaMemsetAsync(prm.c.counters, 0, static_cast<size_t>(B) * Hkv * sizeof(int), stream) != cudaSuccess)
-        return ARK_ERR_CUDA;
     prm.q[0] = static_cast<const uint16_t*>(q);
     prm.o[0] = static_cast<uint16_t*>(o);
     prm.lse[0] = lse;

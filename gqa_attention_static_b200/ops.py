@@ -221,10 +221,10 @@ def ark_attn_decode(q, cache_k, cache_v, kv_len, o, lse, scale: float, mode: int
 
 
 def decode_workspace(B: int, Hq: int, D: int, T: int, max_splits: int, device="cuda", layers: int = 1):
-    """Zero-filled decode workspace (its counters must start at zero), or None
-    when the call needs none."""
+    """Decode workspace (it needs no initialisation), or None when the call
+    needs none."""
     n = ark_attn_decode_layers_workspace_size(layers, B, Hq, D, T, max_splits)
-    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device) if n else None
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device) if n else None
 
 
 # --------------------------------------------------------------- combine ----

@@ -61,7 +61,8 @@ class DecodeStep:
         return max(1, -(-tiles // self.max_splits))
 
     def launches_per_step(self) -> int:
-        return 2 if self.batched else 2 * self.layers
+        """Kernels per step: append, decode and the merge of cut pieces."""
+        return 3 if self.batched else 3 * self.layers
 
     def append(self, stream=None) -> None:
         if self.batched:

@@ -136,19 +136,18 @@ ARK_API ark_status ark_attn_append_rope(void* q, const void* k_new, const void* 
  * request's rows may be cut into pieces processed in parallel; every warp
  * takes at least ceil(ceil(T/16) / max_splits) tiles, so one (request, KV
  * head) is cut into at most max_splits + 1 pieces.  Cut pieces leave fp32
- * partial results in `workspace` and are merged by log-sum-exp inside the
- * same launch (the last piece to finish merges).
+ * partial results in `workspace`; a second kernel, enqueued by the same call
+ * on the same stream (programmatic dependent launch, so it is resident as
+ * the first kernel's CTAs retire), merges them by log-sum-exp.
  * Layouts: q [B,1,Hq,D] bf16; cache_k, cache_v [B,T,Hkv,D] bf16; kv_len
  * int32[B] (device; the new row is already appended, so the query attends to
  * itself); o [B,1,Hq,D] bf16; lse [B,Hq] fp32 (natural log).
  * kv_len outside [0, T] is clamped and sets ARK_DEV_BAD_KVLEN; kv_len = 0
  * gives o = 0, lse = -inf.
  * Workspace: ark_attn_decode_workspace_size(...) bytes (about 16 MB: two
- * partial slots for each of up to 2048 warps, plus one counter per (request,
- * KV head)), 16-byte aligned, caller-owned, required.  The counters MUST be
- * zero before the first call (zero-fill the whole workspace once after
- * allocating it); every call leaves them at zero again.  Calls that can run
- * at the same time must not share a workspace.
+ * partial slots for each of up to 2048 warps), 16-byte aligned, caller-owned,
+ * required.  It needs no initialisation and carries nothing from one call to
+ * the next.  Calls that can run at the same time must not share a workspace.
  * Numerics: bf16 operands on the tensor cores with fp32 accumulation; the
  * softmax weights are rounded to bf16 before they multiply V, o is normalised
  * by the sum of those rounded weights and lse uses the fp32 weights.
@@ -188,7 +187,7 @@ ARK_API ark_status ark_attn_prefill(const void* q, const void* cache_k, const vo
  * the call returns).  All layers share B, S, T, the positions/lengths and the
  * rotary table.  Each layer's tensors follow the single-layer layouts above.
  * The decode workspace is ark_attn_decode_layers_workspace_size(L, ...) bytes
- * with the same zero-before-first-use rule.  Meant for callers that hold
+ * under the same rules.  Meant for callers that hold
  * several independent caches (the ARK-ASR-3B decoder has 36 layers), and for
  * measuring the kernels without per-launch overhead.
  */
@@ -229,18 +228,18 @@ ARK_API ark_status ark_attn_combine(const float* o_part, const float* lse_part, 
  * plugins whose host framework owns the allocator.  Such a caller still
  * passes its inputs and outputs, but no workspace.
  * Same operation, arguments, layouts and results as ark_attn_decode, without
- * the workspace arguments.  The scratch (partial results and merge counters)
+ * the workspace arguments.  The scratch (the partial results of cut pieces)
  * is a fixed array inside the library, ark_attn_decode_noalloc_scratch_bytes()
- * bytes (about 4.1 MB) on every GPU that loads the library, kept until the
- * process exits.  It limits a call to B * Hkv <= 4096 (request, KV head)
- * pairs (ARK_ERR_UNSUPPORTED beyond) and to at most 512 warps, so very large
- * batches run slower than with ark_attn_decode.
+ * bytes (about 4.2 MB) on every GPU that loads the library, kept until the
+ * process exits.  It holds the partials of at most 512 warps, so a call runs
+ * on at most 512 warps and very large batches run slower than with
+ * ark_attn_decode; the size limits are those of ark_attn_decode (B <= 4096,
+ * ARK_ERR_UNSUPPORTED beyond).
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress); make that first call before any stream capture.
- * Every call clears the counters it needs with cudaMemsetAsync on `stream`
- * and allocates nothing.  All calls share the one array, so calls that can
- * overlap on the GPU (different streams, or graphs replayed concurrently)
- * race: serialise them.
+ * Nothing in the scratch needs initialising and no call allocates.  All calls
+ * share the one array, so calls that can overlap on the GPU (different
+ * streams, or graphs replayed concurrently) race: serialise them.
  */
 ARK_API size_t ark_attn_decode_noalloc_scratch_bytes(void);
 ARK_API ark_status ark_attn_decode_noalloc(const void* q, const void* cache_k, const void* cache_v,

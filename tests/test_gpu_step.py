@@ -73,14 +73,16 @@ def test_step_ragged_batch_full_size(oracle_lib, batched):
 
 
 def test_step_repeated_calls_reuse_workspace(oracle_lib):
-    """The merge counters return to zero after every call: the same workspace
-    serves consecutive steps (here: the same step three times, with q restored)."""
+    """The workspace carries nothing from one call to the next: consecutive
+    steps give the same results (the same step three times, with q restored),
+    also after the workspace has been overwritten with NaN bytes."""
     batch = W.cfg_ragged_decode(layers=3, seed=21)
     step = run_step(batch)
     o1 = [x.clone() for x in step.o]
     for _ in range(2):
         for l in range(3):
             step.q[l].copy_(batch.q[l].cuda())
+        step.workspace.fill_(0xFF)
         step.run()
     torch.cuda.synchronize()
     for l in range(3):

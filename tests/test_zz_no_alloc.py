@@ -76,10 +76,10 @@ def test_no_alloc_matches_workspace_decode_twice(case):
             check_lse(f64(lse), f64(lse_ref), "lse (no-alloc vs workspace)")
 
 
-def test_no_alloc_rejects_batches_beyond_its_scratch():
+def test_no_alloc_rejects_batches_beyond_its_limits():
     lib = ops.load()
     dev = "cuda"
-    B, T = 2049, 16          # 2049 requests x 2 KV heads > 4096 counters
+    B, T = 4097, 16          # more requests than decode takes
     q = torch.zeros(B, 1, 16, 128, dtype=torch.bfloat16, device=dev)
     ck = torch.zeros(B, T, 2, 128, dtype=torch.bfloat16, device=dev)
     kv = torch.ones(B, dtype=torch.int32, device=dev)
