@@ -192,16 +192,71 @@ __device__ __forceinline__ void seg_next(Seg& s, const int* s_pref, const Decode
     }
 }
 
-// Log-sum-exp merge of the pieces of one cut segment, run by the warp that
-// finished last.  Pieces come from warps wa..wb; warp wi keeps a piece of this
-// segment in slot 0 if the segment began before its range (T0(wi) > s0), in
-// slot 1 otherwise.  Lane i first reads the 8 heads' lse of piece wa + i
-// (32 pieces at a time), the warp reduces max and sum per head with
-// shuffles, then every lane accumulates dims 4*lane .. 4*lane+3 of all 8
-// heads, two pieces per iteration so that 16 loads are in flight.
+// Log-sum-exp merge of the pieces of one cut segment (one warp).  Pieces
+// come from warps wa..wb; warp wi keeps a piece of this segment in slot 0 if
+// the segment began before its range (T0(wi) > s0), in slot 1 otherwise.
+// Every lane produces dims 4*lane .. 4*lane+3 of all 8 heads.  Up to
+// kFastPieces pieces are read in one round of loads; beyond that, lane i
+// first reads the 8 heads' lse of piece wa + i (32 pieces at a time), the
+// warp reduces max and sum per head with shuffles, then the pieces' o rows
+// are accumulated two pieces per iteration so that 16 loads are in flight.
+constexpr int kFastPieces = 3;
 __device__ __forceinline__ void merge_pieces(const DecodeCore& c, uint16_t* o, float* lse_out, const Seg& cs, int wa,
                                           int wb, int W, int N, int lane, size_t bh0) {
     const int count = wb - wa + 1;
+    auto slot_of = [&](int wi) -> size_t {   // first row of piece wi's 8 heads
+        const int sl = (static_cast<long long>(wi) * N >= static_cast<long long>(cs.s0 + 1) * W) ? 0 : 1;
+        return (static_cast<size_t>(wi) * 2 + sl) * kGroup;
+    };
+    if (count <= kFastPieces) {
+        // the common case (a segment cut once or twice): every load in one round
+        float4 x[kFastPieces][kGroup];
+        float lz[kFastPieces][kGroup];
+#pragma unroll
+        for (int u = 0; u < kFastPieces; ++u) {
+            if (u < count) {
+                const size_t row = slot_of(wa + u);
+                const float4* lsrc = reinterpret_cast<const float4*>(c.part_lse + row);
+                const float4 y0 = __ldcg(lsrc), y1 = __ldcg(lsrc + 1);
+                lz[u][0] = y0.x; lz[u][1] = y0.y; lz[u][2] = y0.z; lz[u][3] = y0.w;
+                lz[u][4] = y1.x; lz[u][5] = y1.y; lz[u][6] = y1.z; lz[u][7] = y1.w;
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h)
+                    x[u][h] = __ldcg(reinterpret_cast<const float4*>(c.part_o + (row + h) * kHeadDim) + lane);
+            } else {
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) {
+                    lz[u][h] = -INFINITY;
+                    x[u][h] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) {
+            float m = lz[0][h];
+#pragma unroll
+            for (int u = 1; u < kFastPieces; ++u) m = fmaxf(m, lz[u][h]);
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+            float sum = 0.f;
+            if (m != -INFINITY) {
+#pragma unroll
+                for (int u = 0; u < kFastPieces; ++u) {
+                    if (lz[u][h] == -INFINITY) continue;   // empty piece: its o is not used
+                    const float wgt = fast_exp2((lz[u][h] - m) * kLog2e);
+                    sum += wgt;
+                    a.x += wgt * x[u][h].x; a.y += wgt * x[u][h].y;
+                    a.z += wgt * x[u][h].z; a.w += wgt * x[u][h].w;
+                }
+            }
+            const float iw = (m == -INFINITY) ? 0.f : 1.f / sum;
+            uint2 pk;
+            pk.x = pack_bf16x2(a.x * iw, a.y * iw);
+            pk.y = pack_bf16x2(a.z * iw, a.w * iw);
+            reinterpret_cast<uint2*>(o + (bh0 + h) * kHeadDim)[lane] = pk;
+            if (lane == 0) lse_out[bh0 + h] = (m == -INFINITY) ? -INFINITY : m + __logf(sum);
+        }
+        return;
+    }
     float M[kGroup], S[kGroup];
 #pragma unroll
     for (int h = 0; h < kGroup; ++h) { M[h] = -INFINITY; S[h] = 0.f; }
@@ -569,7 +624,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
 // the prefix only reads kv_len; griddepcontrol.wait then blocks until the
 // decode grid has completed and its writes are visible.
 template <int MaxL>
-__global__ void __launch_bounds__(kWarps * 32) merge_kernel(const __grid_constant__ MergeParamsT<MaxL> p) {
+__global__ void __launch_bounds__(kWarps * 32, 4) merge_kernel(const __grid_constant__ MergeParamsT<MaxL> p) {
     extern __shared__ int s_pref_m[];
     const DecodeCore& c = p.c;
     const int warp = threadIdx.x >> 5;
