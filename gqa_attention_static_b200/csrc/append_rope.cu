@@ -39,6 +39,10 @@ struct AppendParams {
 };
 
 __global__ void __launch_bounds__(128) append_rope_kernel(const __grid_constant__ AppendParams p) {
+    // a kernel launched behind this one with programmatic stream serialisation
+    // (the decode) may start its own prologue now; it waits for this grid's
+    // completion (griddepcontrol.wait) before it reads q or the cache
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int t = blockIdx.x;
     const int b = blockIdx.y;
     const AppendLayer& L = p.layer[blockIdx.z];

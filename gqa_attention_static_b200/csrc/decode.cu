@@ -360,6 +360,11 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     }
     fence_proxy_async_smem();
     __syncthreads();   // the last block-wide barrier: warps run independently from here
+    // q and the cache rows may come from the kernel before this one in the
+    // stream (the append): with programmatic dependent launch this grid may be
+    // running already, so wait here for that grid's completion and its writes
+    // (a no-op when there is no such dependency); the prefix above only read kv_len
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     const int per_layer = s_pref[c.B];
     const int N = per_layer * c.L;
@@ -805,8 +810,19 @@ ark_status launch_decode_core(DecodeParamsT<MaxL>& prm, const void* const* k, co
     if (need < grid) grid = need;
     if (grid > max_warps / kWarps) grid = max_warps / kWarps;
     if (grid < 1) grid = 1;
-    decode_kernel<MaxL><<<static_cast<unsigned>(grid), kWarps * 32, decode_smem(c.B), stream>>>(prm);
-    if (cudaGetLastError() != cudaSuccess) return ARK_ERR_CUDA;
+    // programmatic stream serialisation: the prologue (prefix over kv_len)
+    // overlaps the tail of the previous kernel; see griddepcontrol.wait
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kWarps * 32);
+    cfg.dynamicSmemBytes = decode_smem(c.B);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, decode_kernel<MaxL>, prm) != cudaSuccess) return ARK_ERR_CUDA;
     return launch_merge<MaxL>(prm, static_cast<int>(grid) * kWarps, stream);
 }
 
