@@ -44,8 +44,10 @@ N_LAYERS = 36
 # sha256 of the kernel source it was taken on; reported as null once the source
 # has changed.
 DECODE_TRAFFIC = {
-    # ncu --set full, one launch of the ragged decode workload (see profiles/)
-    "284d27e5f29adca128c040fe5339a87ceef98ed8f3eb9125e6eed61196e9e764": 336.002304e6 + 10.370048e6,
+    # ncu, one call of the ragged decode workload: decode_kernel (--set full) plus
+    # merge_kernel (dram bytes), read + write (see profiles/)
+    "f7a1da552b684995569ecc1bd9f9489abae906c47d9b1b1550bb2b7a9bce5fee":
+        329.750784e6 + 4.109312e6 + 13.198592e6 + 256,
 }
 
 
