@@ -51,6 +51,13 @@ DECODE_TRAFFIC = {
 }
 
 
+# Per-launch DRAM traffic of the prefill kernel (one layer of the coalesced
+# prefill workload) from an ncu --set full capture, keyed the same way.
+PREFILL_TRAFFIC = {
+    "140f02fa222ad28528f71bc5d4aa3343e3c9092a1c033aede617ebbebd746419": 17.877504e6 + 256,
+}
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -352,7 +359,8 @@ def run_prefill(args):
             "achieved": achieved_gbs if bound == "hbm" else achieved_tf,
             "peak": hbm if bound == "hbm" else tc, "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
             "frac": (t_bytes if bound == "hbm" else t_flops) / (ms_prefill * 1e-3),
-            "peak_kind": hbm_kind if bound == "hbm" else tc_kind, "traffic": None,
+            "peak_kind": hbm_kind if bound == "hbm" else tc_kind,
+            "traffic": PREFILL_TRAFFIC.get(src_hash("gqa_attention_static_b200/csrc/prefill.cu")),
             "launch_ms": ms_prefill, "algorithmic_bytes_per_launch": nb, "flops_per_launch": nf,
             "achieved_tflops": achieved_tf, "tensor_peak_tflops": tc,
             "append_ms_per_step": ms_append}
