@@ -13,6 +13,13 @@
 // subtraction/addition rounded once to bf16 with cvt.rn.bf16.f64.  The result
 // is therefore bit-reproducible.
 //
+// fp8 cache variant (ark_attn_append_rope_fp8): the caches hold OCP E4M3
+// codes with one fp32 scale per (layer, KV head) for K and one for V (a cache
+// format the pages do not have; they quantise weights only).  The rotated key
+// is divided by its scale in double (not rounded to bf16 first), rounded to
+// fp32 and converted to e4m3 with cvt.rn.satfinite; values likewise.  q is
+// rotated to bf16 exactly as above.
+//
 // Work: one CTA per (t, b, layer) row; 128 threads cover (Hq + Hkv) heads x 16
 // groups of 4 rotary pairs, plus Hkv x 16 16-byte pieces of the V copy.  The op
 // moves ~10 KB per row and is latency-bound; it exists so the caller never
@@ -25,8 +32,10 @@ struct AppendLayer {
     uint16_t* q;
     const uint16_t* k_new;
     const uint16_t* v_new;
-    uint16_t* cache_k;
-    uint16_t* cache_v;
+    void* cache_k;           // bf16 or fp8 codes
+    void* cache_v;
+    const float* k_scale;    // fp8 only: [Hkv]
+    const float* v_scale;
 };
 
 struct AppendParams {
@@ -38,6 +47,7 @@ struct AppendParams {
     AppendLayer layer[ARK_MAX_LAYERS];
 };
 
+template <bool Fp8>
 __global__ void __launch_bounds__(128) append_rope_kernel(const __grid_constant__ AppendParams p) {
     // a kernel launched behind this one with programmatic stream serialisation
     // (the decode) may start its own prologue now; it waits for this grid's
@@ -68,7 +78,9 @@ __global__ void __launch_bounds__(128) append_rope_kernel(const __grid_constant_
             const int head = it >> 4;
             const int pg = it & 15;           // pairs 4pg .. 4pg+3
             const uint16_t* src;
-            uint16_t* dst;
+            uint16_t* dst = nullptr;
+            uint8_t* dst8 = nullptr;
+            double kscale = 1.0;
             if (head < p.Hq) {
                 uint16_t* row = L.q + ((static_cast<size_t>(b) * p.S + t) * p.Hq + head) * kHeadDim;
                 src = row;
@@ -76,7 +88,13 @@ __global__ void __launch_bounds__(128) append_rope_kernel(const __grid_constant_
             } else {
                 const int g = head - p.Hq;
                 src = L.k_new + ((static_cast<size_t>(b) * p.S + t) * p.Hkv + g) * kHeadDim;
-                dst = L.cache_k + ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + g) * kHeadDim;
+                const size_t off = ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + g) * kHeadDim;
+                if (Fp8) {
+                    dst8 = static_cast<uint8_t*>(L.cache_k) + off;
+                    kscale = static_cast<double>(__ldg(L.k_scale + g));
+                } else {
+                    dst = static_cast<uint16_t*>(L.cache_k) + off;
+                }
             }
             const uint2 lo = *reinterpret_cast<const uint2*>(src + 4 * pg);
             const uint2 hi = *reinterpret_cast<const uint2*>(src + 64 + 4 * pg);
@@ -89,6 +107,7 @@ __global__ void __launch_bounds__(128) append_rope_kernel(const __grid_constant_
             const float cc[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
             const float ss[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
             uint16_t yl[4], yh[4];
+            double dl[4], dh[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const double a = bf16_bits_to_f64(xl[i]);
@@ -96,8 +115,24 @@ __global__ void __launch_bounds__(128) append_rope_kernel(const __grid_constant_
                 const double c = static_cast<double>(cc[i]);
                 const double s = static_cast<double>(ss[i]);
                 // both products are exact in double, so contraction cannot change the result
-                yl[i] = f64_to_bf16_rn(a * c - h * s);
-                yh[i] = f64_to_bf16_rn(h * c + a * s);
+                dl[i] = a * c - h * s;
+                dh[i] = h * c + a * s;
+                yl[i] = f64_to_bf16_rn(dl[i]);
+                yh[i] = f64_to_bf16_rn(dh[i]);
+            }
+            if (Fp8 && dst8) {
+                // the key into the fp8 cache: e4m3(fp32(y / scale)), two codes per conversion
+                uint32_t cl = 0, ch = 0;
+#pragma unroll
+                for (int i = 0; i < 4; i += 2) {
+                    cl |= static_cast<uint32_t>(f32x2_to_e4m3x2(__double2float_rn(dl[i] / kscale),
+                                                                __double2float_rn(dl[i + 1] / kscale))) << (8 * i);
+                    ch |= static_cast<uint32_t>(f32x2_to_e4m3x2(__double2float_rn(dh[i] / kscale),
+                                                                __double2float_rn(dh[i + 1] / kscale))) << (8 * i);
+                }
+                *reinterpret_cast<uint32_t*>(dst8 + 4 * pg) = cl;
+                *reinterpret_cast<uint32_t*>(dst8 + 64 + 4 * pg) = ch;
+                continue;
             }
             uint2 ol, oh;
             ol.x = static_cast<uint32_t>(yl[0]) | (static_cast<uint32_t>(yl[1]) << 16);
@@ -112,9 +147,24 @@ __global__ void __launch_bounds__(128) append_rope_kernel(const __grid_constant_
             const int piece = c & 15;
             const uint4* src = reinterpret_cast<const uint4*>(
                 L.v_new + ((static_cast<size_t>(b) * p.S + t) * p.Hkv + g) * kHeadDim);
-            uint4* dst = reinterpret_cast<uint4*>(
-                L.cache_v + ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + g) * kHeadDim);
-            dst[piece] = src[piece];
+            const size_t off = ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + g) * kHeadDim;
+            if (Fp8) {
+                // 8 values -> 8 codes: e4m3(fp32(v / scale))
+                const double vscale = static_cast<double>(__ldg(L.v_scale + g));
+                const uint4 x = src[piece];
+                const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+                uint32_t out[2] = {0, 0};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float f0 = __double2float_rn(bf16_bits_to_f64(static_cast<uint16_t>(w[i] & 0xffff)) / vscale);
+                    const float f1 = __double2float_rn(bf16_bits_to_f64(static_cast<uint16_t>(w[i] >> 16)) / vscale);
+                    out[i >> 1] |= static_cast<uint32_t>(f32x2_to_e4m3x2(f0, f1)) << (16 * (i & 1));
+                }
+                *reinterpret_cast<uint2*>(static_cast<uint8_t*>(L.cache_v) + off + 8 * piece) = make_uint2(out[0], out[1]);
+            } else {
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(L.cache_v) + off);
+                dst[piece] = src[piece];
+            }
         }
     }
 }
@@ -136,11 +186,16 @@ ark_status check_common(int B, int S, int T, int Hq, int Hkv, int D) {
     return ARK_OK;
 }
 
-ark_status launch_append(AppendParams& prm, int L, cudaStream_t stream) {
+ark_status launch_append(AppendParams& prm, int L, bool fp8, cudaStream_t stream) {
     dim3 grid(prm.S, prm.B, L);
-    append_rope_kernel<<<grid, 128, 0, stream>>>(prm);
+    if (fp8)
+        append_rope_kernel<true><<<grid, 128, 0, stream>>>(prm);
+    else
+        append_rope_kernel<false><<<grid, 128, 0, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
 }
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 }  // namespace
 
@@ -165,9 +220,8 @@ extern "C" ark_status ark_attn_append_rope(void* q, const void* k_new, const voi
     prm.status = d_status;
     prm.B = B; prm.S = S; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
     prm.layer[0] = AppendLayer{static_cast<uint16_t*>(q), static_cast<const uint16_t*>(k_new),
-                               static_cast<const uint16_t*>(v_new), static_cast<uint16_t*>(cache_k),
-                               static_cast<uint16_t*>(cache_v)};
-    return launch_append(prm, 1, stream);
+                               static_cast<const uint16_t*>(v_new), cache_k, cache_v, nullptr, nullptr};
+    return launch_append(prm, 1, false, stream);
 }
 
 extern "C" ark_status ark_attn_append_rope_layers(int L, void* const* q, const void* const* k_new,
@@ -196,8 +250,52 @@ extern "C" ark_status ark_attn_append_rope_layers(int L, void* const* q, const v
             !aligned16(cache_v[l]))
             return ARK_ERR_INVALID_ARG;
         prm.layer[l] = AppendLayer{static_cast<uint16_t*>(q[l]), static_cast<const uint16_t*>(k_new[l]),
-                                   static_cast<const uint16_t*>(v_new[l]), static_cast<uint16_t*>(cache_k[l]),
-                                   static_cast<uint16_t*>(cache_v[l])};
+                                   static_cast<const uint16_t*>(v_new[l]), cache_k[l], cache_v[l], nullptr, nullptr};
     }
-    return launch_append(prm, L, stream);
+    return launch_append(prm, L, false, stream);
+}
+
+extern "C" ark_status ark_attn_append_rope_fp8_layers(int L, void* const* q, const void* const* k_new,
+                                                      const void* const* v_new, void* const* cache_k,
+                                                      void* const* cache_v, const float* const* k_scale,
+                                                      const float* const* v_scale, const int32_t* pos0,
+                                                      const int32_t* n_new, int B, int S, int T, int Hq, int Hkv,
+                                                      int D, const float* d_table, uint32_t* d_status,
+                                                      cudaStream_t stream) {
+    if (!q || !k_new || !v_new || !cache_k || !cache_v || !k_scale || !v_scale || !pos0 || !n_new || !d_table)
+        return ARK_ERR_INVALID_ARG;
+    if (L <= 0) return ARK_ERR_INVALID_ARG;
+    if (L > ARK_MAX_LAYERS) return ARK_ERR_UNSUPPORTED;
+    ark_status st = check_common(B, S, T, Hq, Hkv, D);
+    if (st != ARK_OK) return st;
+    if (S > 65535) return ARK_ERR_UNSUPPORTED;
+    if (!aligned16(d_table)) return ARK_ERR_INVALID_ARG;
+    AppendParams prm{};
+    prm.pos0 = pos0;
+    prm.n_new = n_new;
+    prm.table = reinterpret_cast<const float2*>(d_table);
+    prm.status = d_status;
+    prm.B = B; prm.S = S; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
+    for (int l = 0; l < L; ++l) {
+        if (!q[l] || !k_new[l] || !v_new[l] || !cache_k[l] || !cache_v[l] || !k_scale[l] || !v_scale[l])
+            return ARK_ERR_INVALID_ARG;
+        if (!aligned16(q[l]) || !aligned16(k_new[l]) || !aligned16(v_new[l]) || !aligned16(cache_k[l]) ||
+            !aligned16(cache_v[l]) || !aligned4(k_scale[l]) || !aligned4(v_scale[l]))
+            return ARK_ERR_INVALID_ARG;
+        prm.layer[l] = AppendLayer{static_cast<uint16_t*>(q[l]), static_cast<const uint16_t*>(k_new[l]),
+                                   static_cast<const uint16_t*>(v_new[l]), cache_k[l], cache_v[l], k_scale[l],
+                                   v_scale[l]};
+    }
+    return launch_append(prm, L, true, stream);
+}
+
+extern "C" ark_status ark_attn_append_rope_fp8(void* q, const void* k_new, const void* v_new, void* cache_k,
+                                               void* cache_v, const float* k_scale, const float* v_scale,
+                                               const int32_t* pos0, const int32_t* n_new, int B, int S, int T,
+                                               int Hq, int Hkv, int D, const float* d_table, uint32_t* d_status,
+                                               cudaStream_t stream) {
+    const void* kn = k_new;
+    const void* vn = v_new;
+    return ark_attn_append_rope_fp8_layers(1, &q, &kn, &vn, &cache_k, &cache_v, &k_scale, &v_scale, pos0, n_new,
+                                           B, S, T, Hq, Hkv, D, d_table, d_status, stream);
 }

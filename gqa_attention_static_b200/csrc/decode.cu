@@ -64,7 +64,12 @@ constexpr int kWarpRing = kStages * kStageBytes;
 constexpr int kRingBytes = kWarps * kWarpRing;
 constexpr int kQSlotBytes = kGroup * kHeadDim * 2;   // the 8 query rows of one group
 constexpr int kQBytes = kWarps * kQSlotBytes;
-constexpr int kBarBytes = kWarps * (kStages + 1) * 8;
+// fp8 cache: 16-row tiles of 128-byte rows, twice as many stages in the same ring
+constexpr int kStages8 = 4;
+constexpr int kTileBytes8 = kTileRows * 128;         // one 16-row fp8 K or V tile (2 KB)
+constexpr int kStageBytes8 = 2 * kTileBytes8;
+static_assert(kStages8 * kStageBytes8 == kWarpRing, "both cache formats use the same ring");
+constexpr int kBarBytes = kWarps * (kStages8 + 1) * 8;
 constexpr int kMaxBatch = 4096;
 constexpr int kMaxWarps = 2048;                      // upper bound on warps per launch (sizes the partials)
 
@@ -81,12 +86,14 @@ struct DecodeCore {
 
 template <int MaxL>
 struct DecodeParamsT {
-    CUtensorMap kmap[MaxL];   // per layer: cache_k as (128 dims, Hkv, B*T rows), box (64, 1, 16)
-    CUtensorMap vmap[MaxL];
+    CUtensorMap kmap[MaxL];   // per layer: cache_k as (128 dims, Hkv, B*T rows), box (64, 1, 16);
+    CUtensorMap vmap[MaxL];   // fp8 cache: box (128, 1, 16) of bytes
     DecodeCore c;
     const uint16_t* q[MaxL];
     uint16_t* o[MaxL];
     float* lse[MaxL];
+    const float* k_scale[MaxL];   // fp8 cache only: per layer [Hkv]
+    const float* v_scale[MaxL];
 };
 
 struct CombineLayer {
@@ -335,8 +342,18 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
 }
 
-template <int MaxL>
+// Fp8: the cache holds e4m3 codes (one fp32 scale per layer and KV head for K
+// and for V).  Tiles are 16 rows of 128 bytes; the MMA fragments are built in
+// registers (ld.shared, byte permutes, cvt e4m3x2 -> f16x2, exact) and the MMAs
+// run on f16 operands (q converted from bf16 once per segment, P rounded to
+// f16).  The head dimension is permuted so that each lane's fragment bytes are
+// contiguous: the score dot products are sums over all 128 dims (any common
+// order of Q's and K's dims gives the same S), and O's dims are put back in
+// place when o is written.
+template <int MaxL, bool Fp8>
 __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_constant__ DecodeParamsT<MaxL> p) {
+    constexpr int kSt = Fp8 ? kStages8 : kStages;          // ring stages
+    constexpr int kStB = Fp8 ? kStageBytes8 : kStageBytes;  // bytes per stage (K tile + V tile)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     const DecodeCore& c = p.c;
@@ -346,8 +363,8 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     const int tig = lane & 3;
     uint8_t* ring = smem + warp * kWarpRing;
     uint8_t* qslot = smem + kRingBytes + warp * kQSlotBytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRingBytes + kQBytes) + warp * (kStages + 1);
-    uint64_t* qbar = bars + kStages;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRingBytes + kQBytes) + warp * (kSt + 1);
+    uint64_t* qbar = bars + kSt;
     int* s_pref = reinterpret_cast<int*>(smem + kRingBytes + kQBytes + kBarBytes);   // [B + 1]
 
     // ---- per CTA: prefix over the batch of the tiles per request (all KV heads)
@@ -355,7 +372,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     // the merge grid may be scheduled from here on (it waits for this grid's completion)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (lane == 0) {
-        for (int s = 0; s <= kStages; ++s) mbar_init(&bars[s], 1);
+        for (int s = 0; s <= kSt; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
     }
     fence_proxy_async_smem();
@@ -394,15 +411,21 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     Seg ps = locate(T0, s_pref, per_layer, c, pj);
     uint32_t pseq = 0;
     auto issue_next = [&]() {
-        const int st = pseq % kStages;
+        const int st = pseq % kSt;
         if (lane == 0) {
-            uint8_t* dst = ring + st * kStageBytes;
+            uint8_t* dst = ring + st * kStB;
             const int row = ps.b * c.T + pj * kTileRows;
-            mbar_arrive_expect_tx(&bars[st], kStageBytes);
-            tma_load_3d_hint(dst, &p.kmap[ps.l], 0, ps.g, row, &bars[st], pol_stream);
-            tma_load_3d_hint(dst + kHalfBytes, &p.kmap[ps.l], 64, ps.g, row, &bars[st], pol_stream);
-            tma_load_3d_hint(dst + kTileBytes, &p.vmap[ps.l], 0, ps.g, row, &bars[st], pol_stream);
-            tma_load_3d_hint(dst + kTileBytes + kHalfBytes, &p.vmap[ps.l], 64, ps.g, row, &bars[st], pol_stream);
+            mbar_arrive_expect_tx(&bars[st], kStB);
+            if constexpr (Fp8) {
+                tma_load_3d_hint(dst, &p.kmap[ps.l], 0, ps.g, row, &bars[st], pol_stream);
+                tma_load_3d_hint(dst + kTileBytes8, &p.vmap[ps.l], 0, ps.g, row, &bars[st], pol_stream);
+            } else {
+                tma_load_3d_hint(dst, &p.kmap[ps.l], 0, ps.g, row, &bars[st], pol_stream);
+                tma_load_3d_hint(dst + kHalfBytes, &p.kmap[ps.l], 64, ps.g, row, &bars[st], pol_stream);
+                tma_load_3d_hint(dst + kTileBytes, &p.vmap[ps.l], 0, ps.g, row, &bars[st], pol_stream);
+                tma_load_3d_hint(dst + kTileBytes + kHalfBytes, &p.vmap[ps.l], 64, ps.g, row, &bars[st],
+                                 pol_stream);
+            }
         }
         ++pseq;
         ++tp;
@@ -411,7 +434,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
             pj = 0;
         }
     };
-    for (int s = 0; s < kStages && tp < T1; ++s) issue_next();
+    for (int s = 0; s < kSt && tp < T1; ++s) issue_next();
 
     // ---- query rows of a segment: one 2 KB bulk copy into this warp's slot
     auto issue_q = [&](const Seg& s) {
@@ -433,17 +456,38 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     uint32_t qf[8][2];
     float acc[8][4];
     float m0, m1, e0, e1, r0s, r1s;
+    float sl2 = c.scale_log2;   // score scale (log2 domain), times the K scale for an fp8 cache
+    float vsc = 1.f;            // V scale of an fp8 cache
     auto begin_segment = [&]() {
         if (!failed && !mbar_wait(qbar, qseq & 1)) {
             failed = true;
             if (lane == 0) report(c.status, ARK_DEV_TIMEOUT);
         }
         ++qseq;
-        // B fragments of Q [8 heads][128 dims]: block (heads 0-7, dims 8k..8k+7) -> b0/b1 of k-step k/2
-        const uint32_t qa = smem_u32(qslot) + lr * 256 + lm * 16;
+        if constexpr (Fp8) {
+            // B fragments of Q^T in f16, head dims permuted: k-step kk of lane (gid, tig) takes
+            // dims 32 tig + 4 kk + {0,1} (b0) and + {2,3} (b1) of head gid
+            const uint4* qrow = reinterpret_cast<const uint4*>(qslot + gid * 256 + tig * 64);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            ldsm_x4(qa + i * 64, qf[2 * i][0], qf[2 * i][1], qf[2 * i + 1][0], qf[2 * i + 1][1]);
+            for (int i = 0; i < 4; ++i) {
+                const uint4 x = qrow[i];
+                const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float lo = __uint_as_float(w[j] << 16), hi = __uint_as_float(w[j] & 0xffff0000u);
+                    const __half2 h = __floats2half2_rn(lo, hi);
+                    qf[2 * i + (j >> 1)][j & 1] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+            }
+            sl2 = c.scale_log2 * __ldg(p.k_scale[cs.l] + cs.g);
+            vsc = __ldg(p.v_scale[cs.l] + cs.g);
+        } else {
+            // B fragments of Q [8 heads][128 dims]: block (heads 0-7, dims 8k..8k+7) -> b0/b1 of k-step k/2
+            const uint32_t qa = smem_u32(qslot) + lr * 256 + lm * 16;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                ldsm_x4(qa + i * 64, qf[2 * i][0], qf[2 * i][1], qf[2 * i + 1][0], qf[2 * i + 1][1]);
+        }
         __syncwarp();
         // fetch the next segment's rows into the slot once the fragments above
         // have been consumed by the first tile's MMAs
@@ -462,24 +506,32 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
 
     for (int t = T0; t < T1; ++t) {
         const uint32_t seq = static_cast<uint32_t>(t - T0);
-        const int s = seq % kStages;
-        if (!failed && !mbar_wait(&bars[s], (seq / kStages) & 1)) {
+        const int s = seq % kSt;
+        if (!failed && !mbar_wait(&bars[s], (seq / kSt) & 1)) {
             failed = true;
             if (lane == 0) report(c.status, ARK_DEV_TIMEOUT);
         }
         if (!failed) {
             const int r0 = cj * kTileRows;
-            const uint32_t st = ring_u32 + s * kStageBytes;
+            const uint32_t st = ring_u32 + s * kStB;
+            const uint8_t* kt8 = ring + s * kStB;              // fp8: K tile, then the V tile
+            const uint8_t* vt8 = kt8 + kTileBytes8;
             const int live = cs.hi - r0;   // rows of this tile that belong to the request's read range
             if (live < kTileRows) {
                 // the box also brought rows past the range (next request, or garbage):
                 // zero their V rows so that their zero weights never meet a NaN
-                uint8_t* vt = ring + s * kStageBytes + kTileBytes;
                 const int z0 = max(live, 0);
-                for (int i = lane; i < (kTileRows - z0) * 16; i += 32) {
-                    const int r = z0 + (i >> 4), part = i & 15;
-                    *reinterpret_cast<uint4*>(vt + (part >> 3) * kHalfBytes + r * 128 + (part & 7) * 16) =
-                        make_uint4(0, 0, 0, 0);
+                if constexpr (Fp8) {
+                    uint8_t* vt = ring + s * kStB + kTileBytes8;
+                    for (int i = lane; i < (kTileRows - z0) * 8; i += 32)
+                        *reinterpret_cast<uint4*>(vt + (z0 + (i >> 3)) * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+                } else {
+                    uint8_t* vt = ring + s * kStB + kTileBytes;
+                    for (int i = lane; i < (kTileRows - z0) * 16; i += 32) {
+                        const int r = z0 + (i >> 4), part = i & 15;
+                        *reinterpret_cast<uint4*>(vt + (part >> 3) * kHalfBytes + r * 128 + (part & 7) * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
                 }
                 fence_proxy_async_smem();
             }
@@ -487,23 +539,43 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
             // two independent accumulation chains over the head dim, summed at the end
             float sc[4] = {0.f, 0.f, 0.f, 0.f};
             float sd[4] = {0.f, 0.f, 0.f, 0.f};
+            if constexpr (Fp8) {
+                // K rows gid and gid+8: bytes (dims) 32 tig .. 32 tig + 31, chunks 2 tig and 2 tig + 1
+                // of the 128-byte swizzled rows; word kk holds dims 32 tig + 4 kk .. + 3
+                const uint32_t x0 = (2 * tig) ^ (gid & 7), x1 = (2 * tig + 1) ^ (gid & 7);
+                const uint4 g0 = *reinterpret_cast<const uint4*>(kt8 + gid * 128 + x0 * 16);
+                const uint4 g1 = *reinterpret_cast<const uint4*>(kt8 + gid * 128 + x1 * 16);
+                const uint4 h0 = *reinterpret_cast<const uint4*>(kt8 + (gid + 8) * 128 + x0 * 16);
+                const uint4 h1 = *reinterpret_cast<const uint4*>(kt8 + (gid + 8) * 128 + x1 * 16);
+                const uint32_t wg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                const uint32_t wh[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
-            for (int kk = 0; kk < 8; kk += 2) {
-                uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-                ldsm_x4(st + (kk >> 2) * kHalfBytes + k_row + (((2 * (kk & 3)) ^ k_x) << 4), a0, a1, a2, a3);
-                ldsm_x4(st + ((kk + 1) >> 2) * kHalfBytes + k_row + (((2 * ((kk + 1) & 3)) ^ k_x) << 4),
-                        b0, b1, b2, b3);
-                mma_bf16_16816(sc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-                mma_bf16_16816(sd, b0, b1, b2, b3, qf[kk + 1][0], qf[kk + 1][1]);
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t a0 = e4m3x2_to_f16x2(static_cast<uint16_t>(wg[kk] & 0xffff));
+                    const uint32_t a1 = e4m3x2_to_f16x2(static_cast<uint16_t>(wh[kk] & 0xffff));
+                    const uint32_t a2 = e4m3x2_to_f16x2(static_cast<uint16_t>(wg[kk] >> 16));
+                    const uint32_t a3 = e4m3x2_to_f16x2(static_cast<uint16_t>(wh[kk] >> 16));
+                    mma_f16_16816((kk & 1) ? sd : sc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+                }
+            } else {
+#pragma unroll
+                for (int kk = 0; kk < 8; kk += 2) {
+                    uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+                    ldsm_x4(st + (kk >> 2) * kHalfBytes + k_row + (((2 * (kk & 3)) ^ k_x) << 4), a0, a1, a2, a3);
+                    ldsm_x4(st + ((kk + 1) >> 2) * kHalfBytes + k_row + (((2 * ((kk + 1) & 3)) ^ k_x) << 4),
+                            b0, b1, b2, b3);
+                    mma_bf16_16816(sc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+                    mma_bf16_16816(sd, b0, b1, b2, b3, qf[kk + 1][0], qf[kk + 1][1]);
+                }
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) sc[i] += sd[i];
             const bool v0 = (r0 + gid) < cs.kvl;
             const bool v1 = (r0 + gid + 8) < cs.kvl;
-            sc[0] = v0 ? sc[0] * c.scale_log2 : -INFINITY;
-            sc[1] = v0 ? sc[1] * c.scale_log2 : -INFINITY;
-            sc[2] = v1 ? sc[2] * c.scale_log2 : -INFINITY;
-            sc[3] = v1 ? sc[3] * c.scale_log2 : -INFINITY;
+            sc[0] = v0 ? sc[0] * sl2 : -INFINITY;
+            sc[1] = v0 ? sc[1] * sl2 : -INFINITY;
+            sc[2] = v1 ? sc[2] * sl2 : -INFINITY;
+            sc[3] = v1 ? sc[3] * sl2 : -INFINITY;
 
             float t0 = fmaxf(sc[0], sc[2]);
             float t1 = fmaxf(sc[1], sc[3]);
@@ -525,12 +597,24 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
 
             const float p0 = fast_exp2(sc[0] - u0), p1 = fast_exp2(sc[1] - u1);
             const float p2 = fast_exp2(sc[2] - u0), p3 = fast_exp2(sc[3] - u1);
-            const __nv_bfloat162 p01 = __floats2bfloat162_rn(p0, p1);
-            const __nv_bfloat162 p23 = __floats2bfloat162_rn(p2, p3);
+            // P rounded to the MMA's operand type (bf16, or f16 for an fp8 cache)
+            uint32_t p01, p23;
+            float q0, q1, q2, q3;   // the rounded weights
+            if constexpr (Fp8) {
+                const __half2 h01 = __floats2half2_rn(p0, p1), h23 = __floats2half2_rn(p2, p3);
+                p01 = *reinterpret_cast<const uint32_t*>(&h01);
+                p23 = *reinterpret_cast<const uint32_t*>(&h23);
+                q0 = __low2float(h01); q1 = __high2float(h01); q2 = __low2float(h23); q3 = __high2float(h23);
+            } else {
+                const __nv_bfloat162 b01 = __floats2bfloat162_rn(p0, p1), b23 = __floats2bfloat162_rn(p2, p3);
+                p01 = *reinterpret_cast<const uint32_t*>(&b01);
+                p23 = *reinterpret_cast<const uint32_t*>(&b23);
+                q0 = __low2float(b01); q1 = __high2float(b01); q2 = __low2float(b23); q3 = __high2float(b23);
+            }
             e0 = e0 * alpha0 + (p0 + p2);
             e1 = e1 * alpha1 + (p1 + p3);
-            r0s = r0s * alpha0 + (__low2float(p01) + __low2float(p23));
-            r1s = r1s * alpha1 + (__high2float(p01) + __high2float(p23));
+            r0s = r0s * alpha0 + (q0 + q2);
+            r1s = r1s * alpha1 + (q1 + q3);
             if (moved) {
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
@@ -540,13 +624,37 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
                     acc[mt][3] *= alpha1;
                 }
             }
-            const uint32_t pb0 = movmatrix_t(*reinterpret_cast<const uint32_t*>(&p01));
-            const uint32_t pb1 = movmatrix_t(*reinterpret_cast<const uint32_t*>(&p23));
+            const uint32_t pb0 = movmatrix_t(p01);
+            const uint32_t pb1 = movmatrix_t(p23);
+            if constexpr (Fp8) {
+                // V^T fragments: output dims permuted so that lane gid's rows (gid, gid+8) of
+                // block mt are dims 16 gid + 2 mt and 16 gid + 2 mt + 1: one 16-byte chunk
+                // (chunk gid) of each of the rows 2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9
+                const int ra = 2 * tig;
+                const uint4 va = *reinterpret_cast<const uint4*>(vt8 + ra * 128 + ((gid ^ (ra & 7)) << 4));
+                const uint4 vb = *reinterpret_cast<const uint4*>(vt8 + (ra + 1) * 128 + ((gid ^ ((ra + 1) & 7)) << 4));
+                const uint4 vc = *reinterpret_cast<const uint4*>(vt8 + (ra + 8) * 128 + ((gid ^ (ra & 7)) << 4));
+                const uint4 vd = *reinterpret_cast<const uint4*>(vt8 + (ra + 9) * 128 + ((gid ^ ((ra + 1) & 7)) << 4));
+                const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+                const uint32_t wc[4] = {vc.x, vc.y, vc.z, vc.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4_t(st + v_row + (mt >> 2) * kHalfBytes + (((2 * (mt & 3)) ^ v_x) << 4), a0, a1, a2, a3);
-                mma_bf16_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
+                for (int mt = 0; mt < 8; ++mt) {
+                    // bytes 2mt, 2mt+1 of the two rows interleaved: (row a, row b) pairs per dim
+                    const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+                    const uint32_t ab = __byte_perm(wa[mt >> 1], wb[mt >> 1], sel);
+                    const uint32_t cd = __byte_perm(wc[mt >> 1], wd[mt >> 1], sel);
+                    mma_f16_16816(acc[mt], e4m3x2_to_f16x2(static_cast<uint16_t>(ab & 0xffff)),
+                                  e4m3x2_to_f16x2(static_cast<uint16_t>(ab >> 16)),
+                                  e4m3x2_to_f16x2(static_cast<uint16_t>(cd & 0xffff)),
+                                  e4m3x2_to_f16x2(static_cast<uint16_t>(cd >> 16)), pb0, pb1);
+                }
+            } else {
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4_t(st + v_row + (mt >> 2) * kHalfBytes + (((2 * (mt & 3)) ^ v_x) << 4), a0, a1, a2, a3);
+                    mma_bf16_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
+                }
             }
             __syncwarp();
             if (tp < T1) issue_next();     // refill the stage just consumed
@@ -571,14 +679,48 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
             r1s += __shfl_xor_sync(0xffffffffu, r1s, o);
         }
         const bool empty0 = (m0 == -INFINITY), empty1 = (m1 == -INFINITY);
-        const float inv0 = empty0 ? 0.f : 1.f / r0s;
-        const float inv1 = empty1 ? 0.f : 1.f / r1s;
+        const float inv0 = empty0 ? 0.f : vsc / r0s;    // vsc = 1 for a bf16 cache
+        const float inv1 = empty1 ? 0.f : vsc / r1s;
         const float lse0 = empty0 ? -INFINITY : (m0 + __log2f(e0)) * kLn2;
         const float lse1 = empty1 ? -INFINITY : (m1 + __log2f(e1)) * kLn2;
         const int h0 = 2 * tig, h1 = 2 * tig + 1;
         const size_t bh0 = static_cast<size_t>(cs.b) * c.Hq + cs.g * kGroup;   // row of the group's head 0
         const bool whole = (cs.s0 >= T0) && (cs.s0 + cs.n <= T1);
-        if (whole) {
+        if (Fp8 && whole) {
+            // lane (gid, tig) holds dims 16 gid .. 16 gid + 15 of heads h0, h1 (the permuted order)
+            uint32_t w0[8], w1[8];
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                w0[mt] = pack_bf16x2(acc[mt][0] * inv0, acc[mt][2] * inv0);
+                w1[mt] = pack_bf16x2(acc[mt][1] * inv1, acc[mt][3] * inv1);
+            }
+            uint4* d0 = reinterpret_cast<uint4*>(p.o[cs.l] + (bh0 + h0) * kHeadDim + 16 * gid);
+            uint4* d1 = reinterpret_cast<uint4*>(p.o[cs.l] + (bh0 + h1) * kHeadDim + 16 * gid);
+            d0[0] = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+            d0[1] = make_uint4(w0[4], w0[5], w0[6], w0[7]);
+            d1[0] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+            d1[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
+            if (gid == 0) {
+                p.lse[cs.l][bh0 + h0] = lse0;
+                p.lse[cs.l][bh0 + h1] = lse1;
+            }
+        } else if (Fp8) {
+            const int slot = (cs.s0 < T0) ? 0 : 1;
+            float* po = c.part_o + (static_cast<size_t>(w) * 2 + slot) * kGroup * kHeadDim;
+            float* p0r = po + h0 * kHeadDim + 16 * gid;
+            float* p1r = po + h1 * kHeadDim + 16 * gid;
+#pragma unroll
+            for (int mt = 0; mt < 8; mt += 2) {
+                st_f32x4_hint(p0r + 2 * mt, acc[mt][0] * inv0, acc[mt][2] * inv0, acc[mt + 1][0] * inv0,
+                              acc[mt + 1][2] * inv0, pol_keep);
+                st_f32x4_hint(p1r + 2 * mt, acc[mt][1] * inv1, acc[mt][3] * inv1, acc[mt + 1][1] * inv1,
+                              acc[mt + 1][3] * inv1, pol_keep);
+            }
+            if (gid == 0) {
+                st_f32_hint(c.part_lse + (static_cast<size_t>(w) * 2 + slot) * kGroup + h0, lse0, pol_keep);
+                st_f32_hint(c.part_lse + (static_cast<size_t>(w) * 2 + slot) * kGroup + h1, lse1, pol_keep);
+            }
+        } else if (whole) {
             __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(p.o[cs.l] + bh0 * kHeadDim);
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
@@ -617,8 +759,8 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     // Never leave with copies in flight: a timed-out warp stops consuming, so
     // wait (bounded) for the tiles and query rows it issued but did not consume.
     if (failed) {
-        for (uint32_t q2 = pseq > kStages ? pseq - kStages : 0; q2 < pseq; ++q2)
-            (void)mbar_wait(&bars[q2 % kStages], (q2 / kStages) & 1);
+        for (uint32_t q2 = pseq > kSt ? pseq - kSt : 0; q2 < pseq; ++q2)
+            (void)mbar_wait(&bars[q2 % kSt], (q2 / kSt) & 1);
         if (qissued > qseq) (void)mbar_wait(qbar, qseq & 1);
     }
 }
@@ -739,14 +881,14 @@ struct DeviceInfo {
     int sms = 0, ctas_per_sm = 0;
 };
 
-template <int MaxL>
+template <int MaxL, bool Fp8>
 ark_status device_info(DeviceInfo& out) {
     static DeviceInfo table[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARK_ERR_CUDA;
     DeviceInfo& d = table[dev];
     if (d.sms == 0) {
-        if (cudaFuncSetAttribute(decode_kernel<MaxL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(decode_kernel<MaxL, Fp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(decode_smem(kMaxBatch))) != cudaSuccess)
             return ARK_ERR_CUDA;
         if (cudaFuncSetAttribute(merge_kernel<MaxL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -754,7 +896,7 @@ ark_status device_info(DeviceInfo& out) {
             return ARK_ERR_CUDA;
         int sms = 0, per = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ARK_ERR_CUDA;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_kernel<MaxL>, kWarps * 32,
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_kernel<MaxL, Fp8>, kWarps * 32,
                                                           decode_smem(64)) != cudaSuccess)
             return ARK_ERR_CUDA;
         d.ctas_per_sm = per > 0 ? per : 1;
@@ -791,17 +933,20 @@ ark_status launch_merge(const DecodeParamsT<MaxL>& prm, int decode_warps, cudaSt
     return ARK_OK;
 }
 
-template <int MaxL>
+template <int MaxL, bool Fp8>
 ark_status launch_decode_core(DecodeParamsT<MaxL>& prm, const void* const* k, const void* const* v, int max_warps,
                               cudaStream_t stream) {
     DecodeCore& c = prm.c;
     for (int l = 0; l < c.L; ++l) {
-        if (!kv_tensor_map(&prm.kmap[l], k[l], static_cast<long long>(c.B) * c.T, c.Hkv, 64, kTileRows) ||
-            !kv_tensor_map(&prm.vmap[l], v[l], static_cast<long long>(c.B) * c.T, c.Hkv, 64, kTileRows))
-            return ARK_ERR_CUDA;
+        const long long rows = static_cast<long long>(c.B) * c.T;
+        const bool ok = Fp8 ? (kv8_tensor_map(&prm.kmap[l], k[l], rows, c.Hkv, kTileRows) &&
+                               kv8_tensor_map(&prm.vmap[l], v[l], rows, c.Hkv, kTileRows))
+                            : (kv_tensor_map(&prm.kmap[l], k[l], rows, c.Hkv, 64, kTileRows) &&
+                               kv_tensor_map(&prm.vmap[l], v[l], rows, c.Hkv, 64, kTileRows));
+        if (!ok) return ARK_ERR_CUDA;
     }
     DeviceInfo d;
-    ark_status st = device_info<MaxL>(d);
+    ark_status st = device_info<MaxL, Fp8>(d);
     if (st != ARK_OK) return st;
     // tiles in the largest case the device lengths can produce
     const long long max_tiles = static_cast<long long>(c.L) * c.B * c.Hkv * ((c.T + kTileRows - 1) / kTileRows);
@@ -822,11 +967,11 @@ ark_status launch_decode_core(DecodeParamsT<MaxL>& prm, const void* const* k, co
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, decode_kernel<MaxL>, prm) != cudaSuccess) return ARK_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, decode_kernel<MaxL, Fp8>, prm) != cudaSuccess) return ARK_ERR_CUDA;
     return launch_merge<MaxL>(prm, static_cast<int>(grid) * kWarps, stream);
 }
 
-template <int MaxL>
+template <int MaxL, bool Fp8 = false>
 ark_status launch_decode(DecodeParamsT<MaxL>& prm, const void* const* k, const void* const* v, void* workspace,
                          size_t ws_bytes, int max_warps, cudaStream_t stream) {
     DecodeCore& c = prm.c;
@@ -835,7 +980,7 @@ ark_status launch_decode(DecodeParamsT<MaxL>& prm, const void* const* k, const v
     uint8_t* base = static_cast<uint8_t*>(workspace);
     c.part_o = reinterpret_cast<float*>(base + w.part_o);
     c.part_lse = reinterpret_cast<float*>(base + w.part_lse);
-    return launch_decode_core<MaxL>(prm, k, v, max_warps, stream);
+    return launch_decode_core<MaxL, Fp8>(prm, k, v, max_warps, stream);
 }
 
 ark_status fill_common(DecodeCore& c, const int32_t* kv_len, int L, int B, int T, int Hq, int Hkv, int D,
@@ -908,6 +1053,55 @@ extern "C" ark_status ark_attn_decode_layers(int L, const void* const* q, const 
         prm.lse[l] = lse[l];
     }
     return launch_decode<ARK_MAX_LAYERS>(prm, cache_k, cache_v, workspace, workspace_bytes, kMaxWarps, stream);
+}
+
+extern "C" ark_status ark_attn_decode_fp8_layers(int L, const void* const* q, const void* const* cache_k,
+                                                 const void* const* cache_v, const float* const* k_scale,
+                                                 const float* const* v_scale, const int32_t* kv_len, int B, int T,
+                                                 int Hq, int Hkv, int D, float scale, ark_decode_mode mode,
+                                                 int max_splits, void* workspace, size_t workspace_bytes,
+                                                 void* const* o, float* const* lse, uint32_t* d_status,
+                                                 cudaStream_t stream) {
+    if (!q || !cache_k || !cache_v || !k_scale || !v_scale || !o || !lse) return ARK_ERR_INVALID_ARG;
+    static thread_local DecodeParamsT<ARK_MAX_LAYERS> prm;
+    prm = DecodeParamsT<ARK_MAX_LAYERS>{};
+    ark_status st = fill_common(prm.c, kv_len, L, B, T, Hq, Hkv, D, scale, mode, max_splits, d_status);
+    if (st != ARK_OK) return st;
+    for (int l = 0; l < L; ++l) {
+        if (!q[l] || !cache_k[l] || !cache_v[l] || !o[l] || !lse[l] || !k_scale[l] || !v_scale[l])
+            return ARK_ERR_INVALID_ARG;
+        if (!aligned16(q[l]) || !aligned16(cache_k[l]) || !aligned16(cache_v[l]) || !aligned16(o[l]) ||
+            (reinterpret_cast<uintptr_t>(lse[l]) & 3u) || (reinterpret_cast<uintptr_t>(k_scale[l]) & 3u) ||
+            (reinterpret_cast<uintptr_t>(v_scale[l]) & 3u))
+            return ARK_ERR_INVALID_ARG;
+        prm.q[l] = static_cast<const uint16_t*>(q[l]);
+        prm.o[l] = static_cast<uint16_t*>(o[l]);
+        prm.lse[l] = lse[l];
+        prm.k_scale[l] = k_scale[l];
+        prm.v_scale[l] = v_scale[l];
+    }
+    return launch_decode<ARK_MAX_LAYERS, true>(prm, cache_k, cache_v, workspace, workspace_bytes, kMaxWarps, stream);
+}
+
+extern "C" ark_status ark_attn_decode_fp8(const void* q, const void* cache_k, const void* cache_v,
+                                          const float* k_scale, const float* v_scale, const int32_t* kv_len, int B,
+                                          int T, int Hq, int Hkv, int D, float scale, ark_decode_mode mode,
+                                          int max_splits, void* workspace, size_t workspace_bytes, void* o,
+                                          float* lse, uint32_t* d_status, cudaStream_t stream) {
+    if (!q || !cache_k || !cache_v || !k_scale || !v_scale || !o || !lse) return ARK_ERR_INVALID_ARG;
+    DecodeParamsT<1> prm{};
+    ark_status st = fill_common(prm.c, kv_len, 1, B, T, Hq, Hkv, D, scale, mode, max_splits, d_status);
+    if (st != ARK_OK) return st;
+    if (!aligned16(q) || !aligned16(cache_k) || !aligned16(cache_v) || !aligned16(o) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(k_scale) & 3u) ||
+        (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+        return ARK_ERR_INVALID_ARG;
+    prm.q[0] = static_cast<const uint16_t*>(q);
+    prm.o[0] = static_cast<uint16_t*>(o);
+    prm.lse[0] = lse;
+    prm.k_scale[0] = k_scale;
+    prm.v_scale[0] = v_scale;
+    return launch_decode<1, true>(prm, &cache_k, &cache_v, workspace, workspace_bytes, kMaxWarps, stream);
 }
 
 extern "C" ark_status ark_attn_combine(const float* o_part, const float* lse_part, int B, int Hq,
@@ -986,5 +1180,5 @@ extern "C" ark_status ark_attn_decode_noalloc(const void* q, const void* cache_k
     prm.q[0] = static_cast<const uint16_t*>(q);
     prm.o[0] = static_cast<uint16_t*>(o);
     prm.lse[0] = lse;
-    return launch_decode_core<1>(prm, &cache_k, &cache_v, kNoAllocWarps, stream);
+    return launch_decode_core<1, false>(prm, &cache_k, &cache_v, kNoAllocWarps, stream);
 }

@@ -53,7 +53,8 @@ std::unordered_map<Key, CUtensorMap, KeyHash>& cache() {
 }
 
 bool cached_encode(const Key& key, CUtensorMap* out, cuuint32_t rank, const cuuint64_t* dims,
-                   const cuuint64_t* strides, const cuuint32_t* box) {
+                   const cuuint64_t* strides, const cuuint32_t* box,
+                   CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     {
         std::lock_guard<std::mutex> lk(g_mu);
         auto it = cache().find(key);
@@ -66,7 +67,7 @@ bool cached_encode(const Key& key, CUtensorMap* out, cuuint32_t rank, const cuui
     if (!fn) return false;
     const cuuint32_t es[5] = {1, 1, 1, 1, 1};
     CUtensorMap m;
-    if (fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, reinterpret_cast<void*>(key.base), dims, strides, box, es,
+    if (fn(&m, dtype, rank, reinterpret_cast<void*>(key.base), dims, strides, box, es,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return false;
@@ -85,6 +86,14 @@ bool kv_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv, 
     const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(Hkv) * 256};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 1, static_cast<cuuint32_t>(box_rows)};
     return cached_encode(key, out, 3, dims, strides, box);
+}
+
+bool kv8_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv, int box_rows) {
+    const Key key{reinterpret_cast<uintptr_t>(base), rows, 3, Hkv, 128, box_rows};
+    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(Hkv) * 128};
+    const cuuint32_t box[3] = {128, 1, static_cast<cuuint32_t>(box_rows)};
+    return cached_encode(key, out, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8);
 }
 
 bool q_group_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hq, int box_inner, int box_rows) {

@@ -15,6 +15,10 @@ bool kv_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv, 
 
 // 2-D tiled map over a row-major [rows, 128] bf16 matrix (row pitch 256 B),
 // box (box_inner elements, box_rows rows), 128-byte swizzle.
+// fp8 (one byte per element) cache [B*T rows][Hkv][128], 128-byte rows:
+// dims (128, Hkv, rows), box (128, 1, box_rows), 128-byte swizzle.
+bool kv8_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv, int box_rows);
+
 bool rows_tensor_map(CUtensorMap* out, const void* base, long long rows, int box_inner, int box_rows);
 
 // 4-D tiled map over q [B, S, Hq, 128] bf16 viewed as (dim 0: 128 head-dim

@@ -48,6 +48,10 @@ EXPORTS = (
     "ark_attn_decode_layers",
     "ark_attn_decode_noalloc_scratch_bytes",
     "ark_attn_decode_noalloc",
+    "ark_attn_append_rope_fp8",
+    "ark_attn_append_rope_fp8_layers",
+    "ark_attn_decode_fp8",
+    "ark_attn_decode_fp8_layers",
 )
 
 
@@ -98,6 +102,16 @@ def load() -> ctypes.CDLL:
     lib.ark_attn_decode_noalloc_scratch_bytes.restype = Z
     lib.ark_attn_decode_noalloc.argtypes = [P, P, P, P, I, I, I, I, I, ctypes.c_float, I, I, P, P, P, P]
     lib.ark_attn_decode_noalloc.restype = I
+    lib.ark_attn_append_rope_fp8.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P]
+    lib.ark_attn_append_rope_fp8.restype = I
+    lib.ark_attn_append_rope_fp8_layers.argtypes = [I, PP, PP, PP, PP, PP, PP, PP, P, P, I, I, I, I, I, I, P, P,
+                                                    P]
+    lib.ark_attn_append_rope_fp8_layers.restype = I
+    lib.ark_attn_decode_fp8.argtypes = [P, P, P, P, P, P, I, I, I, I, I, ctypes.c_float, I, I, P, Z, P, P, P, P]
+    lib.ark_attn_decode_fp8.restype = I
+    lib.ark_attn_decode_fp8_layers.argtypes = [I, PP, PP, PP, PP, PP, P, I, I, I, I, I, ctypes.c_float, I, I, P,
+                                               Z, PP, PP, P, P]
+    lib.ark_attn_decode_fp8_layers.restype = I
     _lib = lib
     return lib
 
@@ -374,3 +388,134 @@ def ark_attn_decode_noalloc(q, cache_k, cache_v, kv_len, o, lse, scale: float, m
                                           float(scale), int(mode), int(max_splits), _ptr(o), _ptr(lse), _ptr(status),
                                           _stream(stream)),
            "ark_attn_decode_noalloc")
+
+
+# --------------------------------------------------------- fp8 KV cache ----
+# Caches of e4m3 codes (torch.uint8, [B,T,Hkv,D]) with fp32 scales per KV head
+# (torch.float32 [Hkv] per layer); see the header for the format.
+
+def _fp8_cache_checks(cache_k, cache_v, k_scale, v_scale, Hkv_expected=None):
+    _need(cache_k, "cache_k", torch.uint8, 4)
+    _need(cache_v, "cache_v", torch.uint8, 4)
+    _need(k_scale, "k_scale", torch.float32, 1)
+    _need(v_scale, "v_scale", torch.float32, 1)
+    if cache_v.shape != cache_k.shape:
+        raise ValueError("cache_k and cache_v must have the same shape")
+    Hkv = cache_k.shape[2]
+    if k_scale.numel() != Hkv or v_scale.numel() != Hkv:
+        raise ValueError("one K scale and one V scale per KV head")
+
+
+def ark_attn_append_rope_fp8_layers(q: Sequence[torch.Tensor], k_new, v_new, cache_k, cache_v, k_scale, v_scale,
+                                    pos0, n_new, table, status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """ark_attn_append_rope into fp8 caches, L layers in one launch."""
+    L = len(q)
+    if not (len(k_new) == len(v_new) == len(cache_k) == len(cache_v) == len(k_scale) == len(v_scale) == L) \
+            or L == 0:
+        raise ValueError("per-layer lists must have the same non-zero length")
+    for i in range(L):
+        for name, t in (("q", q[i]), ("k_new", k_new[i]), ("v_new", v_new[i])):
+            _need(t, name, torch.bfloat16, 4)
+        _fp8_cache_checks(cache_k[i], cache_v[i], k_scale[i], v_scale[i])
+        if q[i].shape != q[0].shape or cache_k[i].shape != cache_k[0].shape or \
+                k_new[i].shape != k_new[0].shape or v_new[i].shape != k_new[0].shape:
+            raise ValueError("all layers must have the same shapes")
+    _need(pos0, "pos0", torch.int32, 1)
+    _need(n_new, "n_new", torch.int32, 1)
+    _need(table, "table", torch.float32)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    B, S, Hq, D = q[0].shape
+    T, Hkv = cache_k[0].shape[1], cache_k[0].shape[2]
+    if tuple(k_new[0].shape) != (B, S, Hkv, D) or cache_k[0].shape[0] != B or cache_k[0].shape[3] != D:
+        raise ValueError("shapes")
+    if table.numel() < T * (D // 2) * 2:
+        raise ValueError("rotary table has fewer than T rows")
+    _raise(load().ark_attn_append_rope_fp8_layers(L, _ptr_array(q), _ptr_array(k_new), _ptr_array(v_new),
+                                                  _ptr_array(cache_k), _ptr_array(cache_v), _ptr_array(k_scale),
+                                                  _ptr_array(v_scale), _ptr(pos0), _ptr(n_new), B, S, T, Hq, Hkv,
+                                                  D, _ptr(table), _ptr(status), _stream(stream)),
+           "ark_attn_append_rope_fp8_layers")
+
+
+def ark_attn_append_rope_fp8(q, k_new, v_new, cache_k, cache_v, k_scale, v_scale, pos0, n_new, table,
+                             status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """RoPE + delta write into one layer's fp8 cache."""
+    for name, t in (("q", q), ("k_new", k_new), ("v_new", v_new)):
+        _need(t, name, torch.bfloat16, 4)
+    _fp8_cache_checks(cache_k, cache_v, k_scale, v_scale)
+    _need(pos0, "pos0", torch.int32, 1)
+    _need(n_new, "n_new", torch.int32, 1)
+    _need(table, "table", torch.float32)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    B, S, Hq, D = q.shape
+    T, Hkv = cache_k.shape[1], cache_k.shape[2]
+    if tuple(k_new.shape) != (B, S, Hkv, D) or tuple(v_new.shape) != (B, S, Hkv, D) or cache_k.shape[0] != B:
+        raise ValueError("shapes")
+    if table.numel() < T * (D // 2) * 2:
+        raise ValueError("rotary table has fewer than T rows")
+    _raise(load().ark_attn_append_rope_fp8(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(cache_k), _ptr(cache_v),
+                                           _ptr(k_scale), _ptr(v_scale), _ptr(pos0), _ptr(n_new), B, S, T, Hq,
+                                           Hkv, D, _ptr(table), _ptr(status), _stream(stream)),
+           "ark_attn_append_rope_fp8")
+
+
+def ark_attn_decode_fp8(q, cache_k, cache_v, k_scale, v_scale, kv_len, o, lse, scale: float,
+                        mode: int = ARK_LENGTH_AWARE, max_splits: int = 8, workspace: Optional[torch.Tensor] = None,
+                        status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """ark_attn_decode over one layer's fp8 cache."""
+    _need(q, "q", torch.bfloat16, 4)
+    _fp8_cache_checks(cache_k, cache_v, k_scale, v_scale)
+    _need(kv_len, "kv_len", torch.int32, 1)
+    _need(o, "o", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32)
+    B, S, Hq, D = q.shape
+    if S != 1:
+        raise ValueError("decode takes one query row per request")
+    T, Hkv = cache_k.shape[1], cache_k.shape[2]
+    ws_bytes = 0
+    if workspace is not None:
+        _need(workspace, "workspace", workspace.dtype)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    if status is not None:
+        _need(status, "status", torch.int32)
+    _raise(load().ark_attn_decode_fp8(_ptr(q), _ptr(cache_k), _ptr(cache_v), _ptr(k_scale), _ptr(v_scale),
+                                      _ptr(kv_len), B, T, Hq, Hkv, D, float(scale), int(mode), int(max_splits),
+                                      _ptr(workspace), ws_bytes, _ptr(o), _ptr(lse), _ptr(status),
+                                      _stream(stream)),
+           "ark_attn_decode_fp8")
+
+
+def ark_attn_decode_fp8_layers(q: Sequence[torch.Tensor], cache_k, cache_v, k_scale, v_scale, kv_len, o, lse,
+                               scale: float, mode: int = ARK_LENGTH_AWARE, max_splits: int = 8,
+                               workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                               stream=None) -> None:
+    """ark_attn_decode_fp8 over L independent layers in one launch."""
+    L = len(q)
+    if not (len(cache_k) == len(cache_v) == len(k_scale) == len(v_scale) == len(o) == len(lse) == L) or L == 0:
+        raise ValueError("per-layer lists must have the same non-zero length")
+    for i in range(L):
+        _need(q[i], "q", torch.bfloat16, 4)
+        _fp8_cache_checks(cache_k[i], cache_v[i], k_scale[i], v_scale[i])
+        _need(o[i], "o", torch.bfloat16, 4)
+        _need(lse[i], "lse", torch.float32)
+        if q[i].shape != q[0].shape or cache_k[i].shape != cache_k[0].shape or o[i].shape != q[0].shape or \
+                lse[i].numel() != q[0].shape[0] * q[0].shape[2]:
+            raise ValueError("all layers must have the same shapes")
+    _need(kv_len, "kv_len", torch.int32, 1)
+    B, S, Hq, D = q[0].shape
+    if S != 1:
+        raise ValueError("decode takes one query row per request")
+    T, Hkv = cache_k[0].shape[1], cache_k[0].shape[2]
+    ws_bytes = 0
+    if workspace is not None:
+        _need(workspace, "workspace", workspace.dtype)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    if status is not None:
+        _need(status, "status", torch.int32)
+    _raise(load().ark_attn_decode_fp8_layers(L, _ptr_array(q), _ptr_array(cache_k), _ptr_array(cache_v),
+                                             _ptr_array(k_scale), _ptr_array(v_scale), _ptr(kv_len), B, T, Hq, Hkv,
+                                             D, float(scale), int(mode), int(max_splits), _ptr(workspace), ws_bytes,
+                                             _ptr_array(o), _ptr_array(lse), _ptr(status), _stream(stream)),
+           "ark_attn_decode_fp8_layers")

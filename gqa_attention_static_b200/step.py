@@ -28,14 +28,21 @@ class DecodeStep:
       q [B,1,Hq,D] (rotated in place), k_new/v_new [B,1,Hkv,D],
       cache_k/cache_v [B,T,Hkv,D], o [B,1,Hq,D], lse [B,Hq];
     shared: pos0, n_new, kv_len int32[B], rotary table, workspace, status.
+    With k_scale/v_scale (per layer fp32 [Hkv]) the caches are fp8 (uint8 e4m3
+    codes) and the step uses the fp8 entry points.
     """
 
     def __init__(self, q: List[torch.Tensor], k_new: List[torch.Tensor], v_new: List[torch.Tensor],
                  cache_k: List[torch.Tensor], cache_v: List[torch.Tensor], pos0: torch.Tensor,
                  n_new: torch.Tensor, kv_len: torch.Tensor, max_splits: int = 8,
                  mode: int = ops.ARK_LENGTH_AWARE, rope_theta: float = 1e6,
-                 scale: Optional[float] = None, batched: bool = True):
+                 scale: Optional[float] = None, batched: bool = True,
+                 k_scale: Optional[List[torch.Tensor]] = None, v_scale: Optional[List[torch.Tensor]] = None):
         self.q, self.k_new, self.v_new = q, k_new, v_new
+        self.fp8 = cache_k[0].dtype == torch.uint8
+        if self.fp8 and (k_scale is None or v_scale is None):
+            raise ValueError("an fp8 cache needs k_scale and v_scale")
+        self.k_scale, self.v_scale = k_scale, v_scale
         self.cache_k, self.cache_v = cache_k, cache_v
         self.pos0, self.n_new, self.kv_len = pos0, n_new, kv_len
         self.layers = len(q)
@@ -65,6 +72,17 @@ class DecodeStep:
         return 3 if self.batched else 3 * self.layers
 
     def append(self, stream=None) -> None:
+        if self.fp8:
+            if self.batched:
+                ops.ark_attn_append_rope_fp8_layers(self.q, self.k_new, self.v_new, self.cache_k, self.cache_v,
+                                                    self.k_scale, self.v_scale, self.pos0, self.n_new, self.table,
+                                                    self.status, stream)
+            else:
+                for l in range(self.layers):
+                    ops.ark_attn_append_rope_fp8(self.q[l], self.k_new[l], self.v_new[l], self.cache_k[l],
+                                                 self.cache_v[l], self.k_scale[l], self.v_scale[l], self.pos0,
+                                                 self.n_new, self.table, self.status, stream)
+            return
         if self.batched:
             ops.ark_attn_append_rope_layers(self.q, self.k_new, self.v_new, self.cache_k, self.cache_v,
                                             self.pos0, self.n_new, self.table, self.status, stream)
@@ -75,6 +93,17 @@ class DecodeStep:
                                          stream)
 
     def attention(self, stream=None) -> None:
+        if self.fp8:
+            if self.batched:
+                ops.ark_attn_decode_fp8_layers(self.q, self.cache_k, self.cache_v, self.k_scale, self.v_scale,
+                                               self.kv_len, self.o, self.lse, self.scale, self.mode, self.max_splits,
+                                               self.workspace, self.status, stream)
+            else:
+                for l in range(self.layers):
+                    ops.ark_attn_decode_fp8(self.q[l], self.cache_k[l], self.cache_v[l], self.k_scale[l],
+                                            self.v_scale[l], self.kv_len, self.o[l], self.lse[l], self.scale,
+                                            self.mode, self.max_splits, self.workspace, self.status, stream)
+            return
         if self.batched:
             ops.ark_attn_decode_layers(self.q, self.cache_k, self.cache_v, self.kv_len, self.o, self.lse,
                                        self.scale, self.mode, self.max_splits, self.workspace, self.status,

@@ -224,3 +224,53 @@ def cfg_long_decode(seed: int = 5, layers: int = N_LAYERS, T: int = 2048, B: int
                    layers=layers, garbage="big", device=device)
     b.meta["name"] = f"long decode B={B} T={T}"
     return b
+
+
+# ---------------------------------------------------------- fp8 caches ----
+# Caches of OCP E4M3 codes (uint8) for the 8-bit cache format.  Drawn as codes
+# directly (random sign, exponent field and mantissa bits), so nothing here
+# quantises anything.
+
+@dataclass
+class Fp8Cache:
+    cache_k: List[torch.Tensor]      # per layer [B, T, Hkv, D] uint8 codes
+    cache_v: List[torch.Tensor]
+    k_scale: List[torch.Tensor]      # per layer [Hkv] fp32
+    v_scale: List[torch.Tensor]
+
+
+def e4m3_codes(shape, gen: torch.Generator, exp_lo: int = 3, exp_hi: int = 10) -> torch.Tensor:
+    """Finite e4m3 codes with exponent field in [exp_lo, exp_hi] (magnitudes
+    2^(exp_lo-7) .. 1.875 * 2^(exp_hi-7)), random sign and mantissa."""
+    sign = torch.randint(0, 2, shape, generator=gen, dtype=torch.int32) << 7
+    expo = torch.randint(exp_lo, exp_hi + 1, shape, generator=gen, dtype=torch.int32) << 3
+    mant = torch.randint(0, 8, shape, generator=gen, dtype=torch.int32)
+    return (sign | expo | mant).to(torch.uint8)
+
+
+def make_fp8_cache(seed: int, B: int, T: int, valid, layers: int = 1, garbage: str = "nan",
+                   Hkv: int = HKV, D: int = HEAD_DIM) -> Fp8Cache:
+    """fp8 caches whose rows j < valid[b] hold codes of moderate magnitude and
+    whose later rows hold `garbage`: "nan" (NaN codes 0x7F/0xFF mixed with the
+    largest finite codes), "big" (finite codes of magnitude 256..448) or
+    "none" (the same distribution as the valid rows).  Scales: uniform in
+    [0.02, 0.2], one per KV head for K and for V."""
+    g = _gen(seed)
+    valid = torch.as_tensor(valid, dtype=torch.int32).view(B)
+    out = Fp8Cache([], [], [], [])
+    j = torch.arange(T).view(1, T, 1, 1)
+    past = j >= valid.view(B, 1, 1, 1)
+    for _ in range(layers):
+        for lst in (out.cache_k, out.cache_v):
+            x = e4m3_codes((B, T, Hkv, D), g)
+            if garbage == "nan":
+                bad = torch.where(torch.rand((B, T, Hkv, D), generator=g) < 0.5,
+                                  torch.randint(0, 2, (B, T, Hkv, D), generator=g, dtype=torch.int32) * 0x80 + 0x7F,
+                                  torch.randint(0, 2, (B, T, Hkv, D), generator=g, dtype=torch.int32) * 0x80 + 0x7E)
+                x = torch.where(past, bad.to(torch.uint8), x)
+            elif garbage == "big":
+                x = torch.where(past, e4m3_codes((B, T, Hkv, D), g, 14, 14), x)
+            lst.append(x.contiguous())
+        out.k_scale.append((0.02 + 0.18 * torch.rand(Hkv, generator=g)).float())
+        out.v_scale.append((0.02 + 0.18 * torch.rand(Hkv, generator=g)).float())
+    return out

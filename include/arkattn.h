@@ -247,6 +247,54 @@ ARK_API ark_status ark_attn_decode_noalloc(const void* q, const void* cache_k, c
                                            float scale, ark_decode_mode mode, int max_splits, void* o,
                                            float* lse, uint32_t* d_status, cudaStream_t stream);
 
+/* ------------------------------------------------------- fp8 KV cache ----
+ * A cache of 8-bit codes, half the bytes of the bf16 cache, for the same
+ * attention.  The pages quantise weights only (the int8/int4 tiers of the
+ * "ARK-ASR-3B -- INT8 ONNX" model card); the cache format here is this
+ * library's own:
+ *   - codes are OCP FP8 E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa
+ *     bits; no infinities; S.1111.111 is NaN; largest finite value 448);
+ *   - k_scale, v_scale: one fp32 scale per KV head for K and for V (device
+ *     arrays [Hkv] per layer, caller-owned, 4-byte aligned); a stored code c
+ *     stands for c * scale;
+ *   - the append stores e4m3(fp32(x / scale)) for the rotated key x (formed
+ *     in fp64 as for the bf16 cache, not rounded to bf16 first) and for the
+ *     value row: the quotient in fp64, rounded to fp32, then to e4m3 with
+ *     round-to-nearest-even, finite values beyond +-448 and infinities
+ *     saturating to +-448, NaN kept.  q is rotated to bf16 in place as by
+ *     ark_attn_append_rope.  Bit-reproducible.
+ * Layouts: cache_k, cache_v [B,T,Hkv,D] of uint8 codes (16-byte aligned);
+ * everything else, the arguments, the status bits and the errors as for the
+ * bf16 entry points.  The decode computes Q K^T and P V on f16 tensor-core
+ * operands (every e4m3 value is an f16 value; q is converted from bf16 to
+ * f16, exact for |q| in [2^-14, 65504]; the softmax weights are rounded to
+ * f16) with fp32 accumulation, and uses the workspace of ark_attn_decode.
+ */
+ARK_API ark_status ark_attn_append_rope_fp8(void* q, const void* k_new, const void* v_new, void* cache_k,
+                                            void* cache_v, const float* k_scale, const float* v_scale,
+                                            const int32_t* pos0, const int32_t* n_new, int B, int S, int T,
+                                            int Hq, int Hkv, int D, const float* d_table, uint32_t* d_status,
+                                            cudaStream_t stream);
+ARK_API ark_status ark_attn_append_rope_fp8_layers(int L, void* const* q, const void* const* k_new,
+                                                   const void* const* v_new, void* const* cache_k,
+                                                   void* const* cache_v, const float* const* k_scale,
+                                                   const float* const* v_scale, const int32_t* pos0,
+                                                   const int32_t* n_new, int B, int S, int T, int Hq, int Hkv,
+                                                   int D, const float* d_table, uint32_t* d_status,
+                                                   cudaStream_t stream);
+ARK_API ark_status ark_attn_decode_fp8(const void* q, const void* cache_k, const void* cache_v,
+                                       const float* k_scale, const float* v_scale, const int32_t* kv_len, int B,
+                                       int T, int Hq, int Hkv, int D, float scale, ark_decode_mode mode,
+                                       int max_splits, void* workspace, size_t workspace_bytes, void* o,
+                                       float* lse, uint32_t* d_status, cudaStream_t stream);
+ARK_API ark_status ark_attn_decode_fp8_layers(int L, const void* const* q, const void* const* cache_k,
+                                              const void* const* cache_v, const float* const* k_scale,
+                                              const float* const* v_scale, const int32_t* kv_len, int B, int T,
+                                              int Hq, int Hkv, int D, float scale, ark_decode_mode mode,
+                                              int max_splits, void* workspace, size_t workspace_bytes,
+                                              void* const* o, float* const* lse, uint32_t* d_status,
+                                              cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

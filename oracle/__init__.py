@@ -64,6 +64,16 @@ def _load():
         lib.ora_combine.restype = None
         lib.ora_num_threads.argtypes = []
         lib.ora_num_threads.restype = I
+        lib.ora_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        lib.ora_e4m3_to_f64.restype = ctypes.c_double
+        lib.ora_f32_to_e4m3.argtypes = [ctypes.c_float]
+        lib.ora_f32_to_e4m3.restype = ctypes.c_uint8
+        lib.ora_quantize_e4m3.argtypes = [ctypes.c_double, ctypes.c_float]
+        lib.ora_quantize_e4m3.restype = ctypes.c_uint8
+        lib.ora_append_rope_fp8.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, P]
+        lib.ora_append_rope_fp8.restype = I
+        lib.ora_attention_fp8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, ctypes.c_double, I, P, P]
+        lib.ora_attention_fp8.restype = None
         _lib = lib
     return _lib
 
@@ -237,3 +247,80 @@ def combine(o_part, lse_part):
     lse = np.zeros(1, dtype=np.float64)
     lib.ora_combine(_ptr(op), _ptr(lp), n, D, _ptr(o), _ptr(lse))
     return o, float(lse[0])
+
+
+# ---------------------------------------------------------- fp8 KV cache ----
+# An 8-bit cache format that is not on the pages (they quantise weights only);
+# the reading is stated in arkattn_oracle.c: OCP E4M3 codes, one fp32 scale per
+# (layer, KV head) for K and for V, code = e4m3(fp32(x / scale)).
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """Exact values of e4m3 codes (uint8); NaN for the NaN codes."""
+    lib = _load()
+    c = np.asarray(codes, dtype=np.uint8)
+    return np.array([lib.ora_e4m3_to_f64(int(x)) for x in c.reshape(-1)], dtype=np.float64).reshape(c.shape)
+
+
+def f32_to_e4m3(x) -> np.ndarray:
+    """fp32 values -> e4m3 codes (nearest even, saturating to +-448)."""
+    lib = _load()
+    a = np.asarray(x, dtype=np.float32)
+    return np.array([lib.ora_f32_to_e4m3(float(v)) for v in a.reshape(-1)], dtype=np.uint8).reshape(a.shape)
+
+
+def quantize_e4m3(x, scale: float) -> np.ndarray:
+    """e4m3(fp32(x / scale)) for fp64 values x."""
+    lib = _load()
+    a = np.asarray(x, dtype=np.float64)
+    return np.array([lib.ora_quantize_e4m3(float(v), float(scale)) for v in a.reshape(-1)],
+                    dtype=np.uint8).reshape(a.shape)
+
+
+def append_rope_fp8(q, k_new, v_new, cache_k, cache_v, k_scale, v_scale, pos0, n_new, theta: float = 1e6):
+    """RoPE + delta write into an fp8 cache of one layer: q rotated to bf16 in
+    place, rotated keys and values quantised with the per-KV-head scales.
+    Works on copies; returns (q_rot, cache_k_new, cache_v_new, skipped)."""
+    lib = _load()
+    q = np.array(q, dtype=np.uint16, copy=True, order="C")
+    ck = np.array(cache_k, dtype=np.uint8, copy=True, order="C")
+    cv = np.array(cache_v, dtype=np.uint8, copy=True, order="C")
+    kn = _c(k_new, np.uint16)
+    vn = _c(v_new, np.uint16)
+    ks = _c(k_scale, np.float32)
+    vs = _c(v_scale, np.float32)
+    p0 = _c(pos0, np.int32)
+    nn = _c(n_new, np.int32)
+    B, S, Hq, D = q.shape
+    T, Hkv = ck.shape[1], ck.shape[2]
+    cos_t, sin_t = rope_table(T, D, theta)
+    skipped = lib.ora_append_rope_fp8(_ptr(q), _ptr(kn), _ptr(vn), _ptr(ck), _ptr(cv), _ptr(ks), _ptr(vs),
+                                      _ptr(p0), _ptr(nn), B, S, T, Hq, Hkv, D, _ptr(cos_t), _ptr(sin_t))
+    return q, ck, cv, int(skipped)
+
+
+def attention_fp8(q, cache_k, cache_v, k_scale, v_scale, first_vis, n_rows, scale: float,
+                  static_mode: bool = False):
+    """attention() over an fp8 cache (uint8 codes, per-KV-head scales)."""
+    lib = _load()
+    q = _c(q, np.uint16)
+    ck = _c(cache_k, np.uint8)
+    cv = _c(cache_v, np.uint8)
+    ks = _c(k_scale, np.float32)
+    vs = _c(v_scale, np.float32)
+    fv = _c(first_vis, np.int32)
+    nr = _c(n_rows, np.int32)
+    B, S, Hq, D = q.shape
+    T, Hkv = ck.shape[1], ck.shape[2]
+    o = np.full((B, S, Hq, D), np.nan, dtype=np.float64)
+    lse = np.full((B, Hq, S), np.nan, dtype=np.float64)
+    lib.ora_attention_fp8(_ptr(q), _ptr(ck), _ptr(cv), _ptr(ks), _ptr(vs), _ptr(fv), _ptr(nr),
+                          B, S, T, Hq, Hkv, D, float(scale), 1 if static_mode else 0, _ptr(o), _ptr(lse))
+    return o, lse
+
+
+def decode_fp8(q, cache_k, cache_v, k_scale, v_scale, kv_len, scale: float, static_mode: bool = False):
+    """Single-token decode over an fp8 cache.  Returns o [B,1,Hq,D], lse [B,Hq]."""
+    B = q.shape[0]
+    o, lse = attention_fp8(q, cache_k, cache_v, k_scale, v_scale, kv_len, np.ones(B, dtype=np.int32),
+                           scale, static_mode)
+    return o, lse[:, :, 0]

@@ -333,3 +333,171 @@ void ora_combine(const double* o_part, const double* lse_part, int n, int D,
     for (int d = 0; d < D; ++d) o[d] /= wsum;
     *lse = M + log(wsum);
 }
+
+/* ------------------------------------------------------- fp8 KV cache ---- */
+/*
+ * An fp8 variant of the cache format.  The pages quantise weights only (the
+ * int8/int4 tiers of the "ARK-ASR-3B -- INT8 ONNX" model card); keeping the
+ * cache itself in 8 bits is not on them.  Reading taken for it:
+ *   - element format: OCP FP8 E4M3 ("fn"): 1 sign bit, 4 exponent bits (bias
+ *     7), 3 mantissa bits, no infinities, S.1111.111 is NaN, largest finite
+ *     value 448, subnormals down to 2^-9;
+ *   - one fp32 scale per (layer, KV head) for K and one for V, given by the
+ *     caller; the stored code of a value x is e4m3(fp32(x / scale)): the
+ *     quotient formed in fp64, rounded to fp32 (nearest even), then to e4m3
+ *     (nearest even, finite values beyond +-448 and infinities saturate to
+ *     +-448, NaN stays NaN);
+ *   - x is the rotated key (formed in fp64 as for the bf16 cache, not rounded
+ *     to bf16 first) or the bf16 value row;
+ *   - attention reads code * scale.
+ */
+
+/* e4m3 code -> its exact value (as double); NaN for S.1111.111. */
+double ora_e4m3_to_f64(uint8_t code) {
+    int sign = code >> 7;
+    int e = (code >> 3) & 15;
+    int m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);                 /* subnormal: m/8 * 2^-6 */
+    else
+        v = ldexp(8.0 + m, e - 10);               /* (1 + m/8) * 2^(e-7) */
+    return sign ? -v : v;
+}
+
+/*
+ * fp32 value -> e4m3 code, nearest-even, saturating: the plain definition,
+ * a search over the 127 non-negative finite codes for the nearest value, a
+ * tie going to the code with an even mantissa (its low bit clear).
+ */
+uint8_t ora_f32_to_e4m3(float f) {
+    double x = (double)f;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    if (isnan(x)) return (uint8_t)(sign | 0x7F);
+    double a = fabs(x);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);   /* saturate, infinities included */
+    int best = 0;
+    double best_err = a;                               /* code 0 is +0 */
+    for (int c = 1; c <= 0x7E; ++c) {
+        double err = fabs(ora_e4m3_to_f64((uint8_t)c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* x (fp64) quantised with `scale`: e4m3(fp32(x / scale)) */
+uint8_t ora_quantize_e4m3(double x, float scale) {
+    float y = (float)(x / (double)scale);
+    return ora_f32_to_e4m3(y);
+}
+
+/*
+ * RoPE + delta write into an fp8 cache (same rows, positions and skipping as
+ * ora_append_rope): q is rotated in place to bf16 as before; the rotated key
+ * (fp64) and the value row are quantised with the scales of their KV head,
+ * k_scale[g] and v_scale[g] (this layer's).
+ */
+int ora_append_rope_fp8(uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                        uint8_t* cache_k, uint8_t* cache_v, const float* k_scale, const float* v_scale,
+                        const int32_t* pos0, const int32_t* n_new,
+                        int B, int S, int T, int Hq, int Hkv, int D,
+                        const float* cos_tab, const float* sin_tab) {
+    int skipped = 0;
+    int half = D / 2;
+    for (int b = 0; b < B; ++b) {
+        for (int t = 0; t < S && t < n_new[b]; ++t) {
+            int p = pos0[b] + t;
+            if (p < 0 || p >= T) { ++skipped; continue; }
+            for (int h = 0; h < Hq; ++h) {
+                uint16_t* row = q + (((size_t)b * S + t) * Hq + h) * D;
+                uint16_t tmp[512];
+                rope_row_bf16(row, tmp, p, D, cos_tab, sin_tab);
+                memcpy(row, tmp, sizeof(uint16_t) * (size_t)D);
+            }
+            for (int g = 0; g < Hkv; ++g) {
+                const uint16_t* krow = k_new + (((size_t)b * S + t) * Hkv + g) * D;
+                const uint16_t* vrow = v_new + (((size_t)b * S + t) * Hkv + g) * D;
+                uint8_t* kdst = cache_k + (((size_t)b * T + p) * Hkv + g) * D;
+                uint8_t* vdst = cache_v + (((size_t)b * T + p) * Hkv + g) * D;
+                double x[512], c[256], s[256], y[512];
+                for (int d = 0; d < D; ++d) x[d] = ora_bf16_to_f64(krow[d]);
+                for (int i = 0; i < half; ++i) {
+                    c[i] = (double)cos_tab[(size_t)p * half + i];
+                    s[i] = (double)sin_tab[(size_t)p * half + i];
+                }
+                ora_rope_rotate(x, c, s, D, y);
+                for (int d = 0; d < D; ++d) kdst[d] = ora_quantize_e4m3(y[d], k_scale[g]);
+                for (int d = 0; d < D; ++d) vdst[d] = ora_quantize_e4m3(ora_bf16_to_f64(vrow[d]), v_scale[g]);
+            }
+        }
+    }
+    return skipped;
+}
+
+/*
+ * Attention over an fp8 cache: the definition of ora_attention with key row j
+ * read as code * k_scale[g] and value row j as code * v_scale[g] (exact in
+ * double).  Each (b, h) dequantises its KV head's rows into double arrays and
+ * takes the same two-pass softmax (or the masked static form).
+ */
+static void attend_rows_f64(const double* q, const double* k, const double* v, int n_rows_total,
+                            int n_valid, int static_form, int D, double scale, double* o, double* lse) {
+    int n = static_form ? n_rows_total : n_valid;
+    double m = -INFINITY;
+    double* sc = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    for (int j = 0; j < n; ++j) {
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += q[d] * k[(size_t)j * D + d];
+        sc[j] = (j < n_valid) ? scale * dot : -INFINITY;
+        if (sc[j] > m) m = sc[j];
+    }
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    if (m == -INFINITY) { *lse = -INFINITY; free(sc); return; }
+    double l = 0.0;
+    for (int j = 0; j < n; ++j) {
+        double w = exp(sc[j] - m);
+        l += w;
+        for (int d = 0; d < D; ++d) o[d] += w * v[(size_t)j * D + d];
+    }
+    for (int d = 0; d < D; ++d) o[d] /= l;
+    *lse = m + log(l);
+    free(sc);
+}
+
+void ora_attention_fp8(const uint16_t* q, const uint8_t* cache_k, const uint8_t* cache_v,
+                       const float* k_scale, const float* v_scale,
+                       const int32_t* first_vis, const int32_t* n_rows,
+                       int B, int S, int T, int Hq, int Hkv, int D, double scale, int static_mode,
+                       double* o, double* lse) {
+    int group = Hq / Hkv;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < Hq; ++h) {
+            int g = h / group;
+            double* kd = (double*)malloc(sizeof(double) * (size_t)T * D);
+            double* vd = (double*)malloc(sizeof(double) * (size_t)T * D);
+            for (int j = 0; j < T; ++j)
+                for (int d = 0; d < D; ++d) {
+                    size_t idx = (((size_t)b * T + j) * Hkv + g) * D + d;
+                    kd[(size_t)j * D + d] = ora_e4m3_to_f64(cache_k[idx]) * (double)k_scale[g];
+                    vd[(size_t)j * D + d] = ora_e4m3_to_f64(cache_v[idx]) * (double)v_scale[g];
+                }
+            for (int t = 0; t < S && t < n_rows[b]; ++t) {
+                int vis = first_vis[b] + t;
+                if (vis < 0) vis = 0;
+                if (vis > T) vis = T;
+                double qd[512];
+                const uint16_t* qrow = q + (((size_t)b * S + t) * Hq + h) * D;
+                for (int d = 0; d < D; ++d) qd[d] = ora_bf16_to_f64(qrow[d]);
+                attend_rows_f64(qd, kd, vd, T, vis, static_mode, D, scale,
+                                o + (((size_t)b * S + t) * Hq + h) * D, lse + ((size_t)b * Hq + h) * S + t);
+            }
+            free(kd);
+            free(vd);
+        }
+    }
+}

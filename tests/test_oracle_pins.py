@@ -422,3 +422,127 @@ def test_audio_slots_golden():
         assert max(W.audio_slots_from_mel(mel), 1) == slots
     assert W.sweep_prompt_len() == 50
     assert W.audio_slots(30 * 16000) + 12 == 387
+
+
+# ----------------------------------------------------------- fp8 (e4m3) ----
+# The 8-bit cache format is a reading of its own (the pages quantise weights
+# only): OCP E4M3 codes, one fp32 scale per (layer, KV head), code =
+# e4m3(fp32(x / scale)).  The pins tie the oracle's encoder and decoder to
+# torch's float8_e4m3fn conversions and to the format's defining constants,
+# and the fp8 attention to the bf16 attention pinned above.
+
+def test_e4m3_decode_all_codes_matches_torch(oracle_lib):
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_to_f64(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    assert np.array_equal(ours[fin], ref[fin])
+    assert np.isnan(ours).sum() == 2                       # S.1111.111 only: no infinities
+
+
+def test_e4m3_defining_constants(oracle_lib):
+    v = oracle.e4m3_to_f64(np.array([0x7E, 0x01, 0x08, 0x07, 0x38, 0x80], np.uint8))
+    assert v[0] == 448.0                                   # largest finite: 1.75 * 2^8
+    assert v[1] == 2.0 ** -9                               # smallest subnormal
+    assert v[2] == 2.0 ** -6                               # smallest normal
+    assert v[3] == 7 * 2.0 ** -9                           # largest subnormal
+    assert v[4] == 1.0 and v[5] == 0.0 and np.signbit(v[5])
+    pos = oracle.e4m3_to_f64(np.arange(0x7F, dtype=np.uint8))
+    assert np.all(np.diff(pos) > 0)                        # codes 0..126 increase strictly
+
+
+def test_e4m3_encode_roundtrip_ties_and_saturation(oracle_lib):
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    vals = oracle.e4m3_to_f64(codes).astype(np.float32)
+    assert np.array_equal(oracle.f32_to_e4m3(vals), codes)                 # every finite code round-trips
+    pos = oracle.e4m3_to_f64(np.arange(0x7F, dtype=np.uint8))
+    mids = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)                   # exact in fp32
+    got = oracle.f32_to_e4m3(mids).astype(int)
+    lo = np.arange(0x7E)
+    assert np.array_equal(got, np.where(lo % 2 == 0, lo, lo + 1))          # ties to the even code
+    assert np.array_equal(oracle.f32_to_e4m3(np.nextafter(mids, np.float32(0))), lo)
+    assert np.array_equal(oracle.f32_to_e4m3(np.nextafter(mids, np.float32(1e9))), lo + 1)
+    sat = oracle.f32_to_e4m3(np.array([448.5, 463.9, 464.0, 1e30, np.inf, -np.inf, -1e9], np.float32))
+    assert list(sat) == [0x7E] * 5 + [0xFE, 0xFE]
+    assert oracle.f32_to_e4m3(np.array([np.nan], np.float32))[0] & 0x7F == 0x7F
+
+
+def test_e4m3_encode_matches_torch_in_range(oracle_lib):
+    g = torch.Generator().manual_seed(31)
+    x = torch.cat([torch.randn(4000, generator=g) * s for s in (0.003, 0.1, 1.0, 30.0)])
+    x = torch.clamp(x, -448.0, 448.0).float()
+    ref = x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.f32_to_e4m3(x.numpy()), ref)
+
+
+def test_append_fp8_within_half_code_of_fp64_rotation(oracle_lib):
+    """Dequantised fp8 keys sit within half an e4m3 step of the fp64 rotation
+    (then divided by the scale); values reproduce exactly when they are
+    representable; rows outside the written range keep their codes."""
+    B, S, T = 2, 3, 16
+    q = rand_bits((B, S, 16, 128), 40)
+    kn = rand_bits((B, S, 2, 128), 41)
+    g = torch.Generator().manual_seed(42)
+    rep = oracle.e4m3_to_f64(torch.randint(0x18, 0x58, (B, S, 2, 128), generator=g).to(torch.uint8).numpy())
+    vscale = np.array([0.25, 2.0], np.float32)
+    vn = bf16_bits(torch.from_numpy(rep * vscale[None, None, :, None]))   # exact: power-of-two scales
+    ck = torch.randint(0, 0x70, (B, T, 2, 128), generator=g).to(torch.uint8).numpy()
+    cv = torch.randint(0, 0x70, (B, T, 2, 128), generator=g).to(torch.uint8).numpy()
+    kscale = np.array([0.05, 0.013], np.float32)
+    pos0 = np.array([2, 9], np.int32)
+    n_new = np.array([3, 2], np.int32)
+    q2, ck2, cv2, skipped = oracle.append_rope_fp8(q, kn, vn, ck, cv, kscale, vscale, pos0, n_new)
+    assert skipped == 0
+    q_ref, _, _, _ = oracle.append_rope(q, kn, vn, np.zeros((B, T, 2, 128), np.uint16),
+                                        np.zeros((B, T, 2, 128), np.uint16), pos0, n_new)
+    assert np.array_equal(q2, q_ref)                       # q is rotated exactly as on the bf16 path
+    cos_t, sin_t = oracle.rope_table(T)
+    for b in range(B):
+        for t in range(n_new[b]):
+            p = pos0[b] + t
+            for h in range(2):
+                y = oracle.rope_rotate(oracle.bf16_array_to_f64(kn[b, t, h]), cos_t[p].astype(np.float64),
+                                       sin_t[p].astype(np.float64)) / kscale[h]
+                d = oracle.e4m3_to_f64(ck2[b, p, h])
+                step = np.maximum(2.0 ** (np.floor(np.log2(np.maximum(np.abs(y), 2.0 ** -6))) - 3), 2.0 ** -9)
+                assert np.all(np.abs(d - np.clip(y, -448, 448)) <= step / 2 + 1e-12)
+                assert np.array_equal(oracle.e4m3_to_f64(cv2[b, p, h]), rep[b, t, h])
+        written = set(range(pos0[b], pos0[b] + n_new[b]))
+        for j in range(T):
+            if j not in written:
+                assert np.array_equal(ck2[b, j], ck[b, j]) and np.array_equal(cv2[b, j], cv[b, j])
+
+
+def test_fp8_attention_equals_bf16_attention_of_dequantised_cache(oracle_lib):
+    """With power-of-two scales every dequantised code is a bf16 value, so the
+    fp8 attention must give exactly the bf16 attention of those values (length
+    aware and masked static); NaN codes past the valid length change nothing."""
+    B, T = 3, 40
+    g = torch.Generator().manual_seed(50)
+    codes_k = torch.randint(0x10, 0x60, (B, T, 2, 128), generator=g).to(torch.uint8)
+    codes_v = torch.randint(0x10, 0x60, (B, T, 2, 128), generator=g).to(torch.uint8)
+    sign_k = torch.randint(0, 2, codes_k.shape, generator=g).to(torch.uint8) << 7
+    codes_k = (codes_k | sign_k).numpy()
+    codes_v = codes_v.numpy()
+    ks = np.array([0.125, 0.5], np.float32)
+    vs = np.array([0.25, 1.0], np.float32)
+    q = rand_bits((B, 1, 16, 128), 51)
+    kv = np.array([1, 17, 40], np.int32)
+    kd = oracle.e4m3_to_f64(codes_k) * ks[None, None, :, None]
+    vd = oracle.e4m3_to_f64(codes_v) * vs[None, None, :, None]
+    kb = bf16_bits(torch.from_numpy(kd))
+    vb = bf16_bits(torch.from_numpy(vd))
+    assert np.array_equal(oracle.bf16_array_to_f64(kb), kd)   # exact in bf16
+    for static in (False, True):
+        o8, l8 = oracle.decode_fp8(q, codes_k, codes_v, ks, vs, kv, 0.0884, static)
+        o16, l16 = oracle.decode(q, kb, vb, kv, 0.0884, static)
+        assert np.array_equal(o8, o16) and np.array_equal(l8, l16)
+    garbage_k = codes_k.copy()
+    garbage_v = codes_v.copy()
+    for b in range(B):
+        garbage_k[b, kv[b]:] = 0x7F
+        garbage_v[b, kv[b]:] = 0xFF
+    o8g, l8g = oracle.decode_fp8(q, garbage_k, garbage_v, ks, vs, kv, 0.0884)
+    o8, l8 = oracle.decode_fp8(q, codes_k, codes_v, ks, vs, kv, 0.0884)
+    assert np.array_equal(o8g, o8) and np.array_equal(l8g, l8)
