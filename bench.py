@@ -67,6 +67,8 @@ def parse():
     ap.add_argument("--config", default="ragged",
                     choices=["ragged", "single", "long2048", "long1024", "prefill"])
     ap.add_argument("--mode", default="aware", choices=["aware", "masked"])
+    ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
+                    help="cache format of the decode configurations: bf16, or fp8 E4M3 codes with per-head scales")
     ap.add_argument("--max-splits", type=int, default=8)
     ap.add_argument("--per-layer", action="store_true",
                     help="issue the single-layer calls layer by layer instead of the layer-batched calls")
@@ -100,10 +102,21 @@ def make_workload(name: str, layers: int, device: str):
     return b, desc
 
 
-def algorithmic_bytes(kv_len, B: int) -> int:
+def algorithmic_bytes(kv_len, B: int, kv: str = "bf16") -> int:
     """Decode attention per layer: K+V rows read (1024 B per position for the
-    2 KV heads) + q read (4096 B) + o written (4096 B), per request."""
-    return int(sum(int(x) for x in kv_len) * 1024 + B * 8192)
+    2 KV heads, 512 B for an fp8 cache) + q read (4096 B) + o written (4096 B),
+    per request."""
+    per_pos = 512 if kv == "fp8" else 1024
+    return int(sum(int(x) for x in kv_len) * per_pos + B * 8192)
+
+
+def fp8_cache_for(batch, mode: str):
+    """fp8 caches (e4m3 codes, per-head scales) for a decode workload: valid
+    rows before each request's cache_position, garbage after it (NaN codes for
+    the length-aware mode, large finite codes for the masked one)."""
+    from gqa_attention_static_b200 import workloads as W
+    return W.make_fp8_cache(1000 + batch.B, batch.B, batch.T, batch.pos0, layers=batch.layers,
+                            garbage="big" if mode == "masked" else "nan")
 
 
 def max_over_ranks(ms: float, world: int, device) -> float:
@@ -198,7 +211,7 @@ class OracleRunner:
     layer-steps (RoPE + delta write + attention) over a bounded sample of the
     workload's layers.  OpenMP threads = all host cores."""
 
-    def __init__(self, workload: str, mode: str, layers: int = 4):
+    def __init__(self, workload: str, mode: str, layers: int = 4, kv: str = "bf16"):
         import numpy as np
         import torch
         cores = os.cpu_count() or 1
@@ -212,19 +225,33 @@ class OracleRunner:
         def bits(x):
             return x.contiguous().view(torch.int16).numpy().view(np.uint16)
 
-        self.inputs = [(bits(batch.q[l]), bits(batch.k_new[l]), bits(batch.v_new[l]),
-                        bits(batch.cache_k[l]), bits(batch.cache_v[l])) for l in range(layers)]
+        self.fp8 = (kv == "fp8")
+        if self.fp8:
+            fc = fp8_cache_for(batch, mode)
+            self.inputs = [(bits(batch.q[l]), bits(batch.k_new[l]), bits(batch.v_new[l]),
+                            fc.cache_k[l].numpy(), fc.cache_v[l].numpy(), fc.k_scale[l].numpy(),
+                            fc.v_scale[l].numpy()) for l in range(layers)]
+            self.desc = self.desc.replace(" 1% x8 K/V row outliers", "") + ", fp8 E4M3 cache"
+        else:
+            self.inputs = [(bits(batch.q[l]), bits(batch.k_new[l]), bits(batch.v_new[l]),
+                            bits(batch.cache_k[l]), bits(batch.cache_v[l])) for l in range(layers)]
         self.pos0 = batch.pos0.numpy()
         self.n_new = batch.n_new.numpy()
         self.kv = batch.kv_len.numpy()
         self.B = batch.B
         self.static = (mode == "masked")
-        self.bytes_per_layer = algorithmic_bytes(self.kv, self.B)
+        self.bytes_per_layer = algorithmic_bytes(self.kv, self.B, kv)
         self.i = 0
 
     def layer_step(self):
-        q, kn, vn, ck, cv = self.inputs[self.i % len(self.inputs)]
+        x = self.inputs[self.i % len(self.inputs)]
         self.i += 1
+        if self.fp8:
+            q, kn, vn, ck, cv, ks, vs = x
+            qr, ck2, cv2, _ = self.oracle.append_rope_fp8(q, kn, vn, ck, cv, ks, vs, self.pos0, self.n_new)
+            self.oracle.decode_fp8(qr, ck2, cv2, ks, vs, self.kv, 1.0 / math.sqrt(128), static_mode=self.static)
+            return
+        q, kn, vn, ck, cv = x
         qr, ck2, cv2, _ = self.oracle.append_rope(q, kn, vn, ck, cv, self.pos0, self.n_new)
         self.oracle.decode(qr, ck2, cv2, self.kv, 1.0 / math.sqrt(128), static_mode=self.static)
 
@@ -239,8 +266,8 @@ class OracleRunner:
                 return n, el
 
 
-def cpu_baseline(workload: str, seconds: float, mode: str):
-    r = OracleRunner(workload, mode)
+def cpu_baseline(workload: str, seconds: float, mode: str, kv: str = "bf16"):
+    r = OracleRunner(workload, mode, kv=kv)
     r.timed(0.0, 1)   # warm
     n, el = r.timed(seconds, 1)
     return {"value": r.bytes_per_layer * n / el / 1e9, "unit": "GB/s", "cores": r.cores, "kind": "oracle",
@@ -253,7 +280,7 @@ def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
         return
-    r = OracleRunner(args.config, args.mode)
+    r = OracleRunner(args.config, args.mode, kv=args.kv)
     for _ in range(max(1, args.warmup)):
         r.layer_step()
     t0 = time.perf_counter()
@@ -266,7 +293,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": r.desc, "mode": args.mode},
+            "data": "synthetic", "config": {"workload": r.desc, "mode": args.mode, "kv_cache": args.kv},
             "cpu_baseline": {"value": v, "unit": "GB/s", "cores": r.cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -417,14 +444,24 @@ def main():
         qv[l].copy_(batch.q[l])
         kv_[l].copy_(batch.k_new[l])
         vv[l].copy_(batch.v_new[l])
-    ck = [x.to(dev) for x in batch.cache_k]
-    cv = [x.to(dev) for x in batch.cache_v]
+    fp8 = (args.kv == "fp8")
+    ks = vs = None
+    if fp8:
+        fc = fp8_cache_for(batch, args.mode)
+        ck = [x.to(dev) for x in fc.cache_k]
+        cv = [x.to(dev) for x in fc.cache_v]
+        ks = [x.to(dev) for x in fc.k_scale]
+        vs = [x.to(dev) for x in fc.v_scale]
+        desc = desc.replace(" 1% x8 K/V row outliers", "") + ", fp8 E4M3 cache (per-head scales)"
+    else:
+        ck = [x.to(dev) for x in batch.cache_k]
+        cv = [x.to(dev) for x in batch.cache_v]
     pos0 = batch.pos0.to(dev)
     n_new = batch.n_new.to(dev)
     kv_len = batch.kv_len.to(dev)
     step = DecodeStep([qv[l] for l in range(L)], [kv_[l] for l in range(L)], [vv[l] for l in range(L)],
                       ck, cv, pos0, n_new, kv_len, max_splits=args.max_splits, mode=mode,
-                      batched=not args.per_layer)
+                      batched=not args.per_layer, k_scale=ks, v_scale=vs)
     # outputs packed for the device->host read of the e2e leg
     osz = B * 16 * 128
     d_out_o = torch.empty(L * osz, dtype=torch.bfloat16, device=dev)
@@ -492,7 +529,7 @@ def main():
     per_launch_ms = sum(attn_ms) / len(attn_ms) / calls_per_group
 
     kvl = batch.kv_len.tolist()
-    bytes_layer = algorithmic_bytes(kvl, B)
+    bytes_layer = algorithmic_bytes(kvl, B, args.kv)
     step_bytes = bytes_layer * L
     value = job_throughput(step_bytes, world, ms_step)
     tl = B * L * world / (ms_step * 1e-3)
@@ -501,8 +538,8 @@ def main():
     achieved = bytes_launch / (per_launch_ms * 1e-3) / 1e9
     h = src_hash("gqa_attention_static_b200/csrc/decode.cu")
     # the capture is of the default workload's batched launch
-    traffic = (DECODE_TRAFFIC.get(h) if (not args.per_layer and args.config == "ragged" and args.mode == "aware")
-               else None)
+    traffic = (DECODE_TRAFFIC.get(h) if (not args.per_layer and args.config == "ragged" and args.mode == "aware"
+                                         and not fp8) else None)
 
     e2e = None
     if not args.no_e2e:
@@ -525,7 +562,7 @@ def main():
                 v2 = di[L * (qsz + ksz):].view(L, B, 1, 2, 128)
                 st_k = DecodeStep([q2[l] for l in range(L)], [k2[l] for l in range(L)], [v2[l] for l in range(L)],
                                   ck, cv, pos0, n_new, kv_len, max_splits=args.max_splits, mode=mode,
-                                  batched=not args.per_layer)
+                                  batched=not args.per_layer, k_scale=ks, v_scale=vs)
                 st_k.o = [do[l * osz:(l + 1) * osz].view(B, 1, 16, 128) for l in range(L)]
                 st_k.lse = [dl[l * B * 16:(l + 1) * B * 16].view(B, 16) for l in range(L)]
                 with torch.cuda.stream(s):
@@ -585,18 +622,18 @@ def main():
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_baseline(args.config, args.cpu_seconds, args.mode)
+        cb = cpu_baseline(args.config, args.cpu_seconds, args.mode, args.kv)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": desc, "batch": B, "max_total_len": T, "layers": L,
+            "vs_baseline": None, "dtype": "e4m3 cache, f16 MMA" if fp8 else "bf16", "data": "synthetic",
+            "config": {"workload": desc, "batch": B, "max_total_len": T, "layers": L, "kv_cache": args.kv,
                        "mode": "masked-static" if args.mode == "masked" else "length-aware",
                        "max_splits": args.max_splits, "min_tiles_per_warp": step.min_tiles,
                        "l2": "inputs larger than L2 (%.0f MB of caches streamed per step)" %
-                             (2 * L * B * T * 2 * 128 * 2 / 1e6),
+                             (2 * L * B * T * 2 * 128 * (1 if fp8 else 2) / 1e6),
                        "parallelism": f"replicas x{world}",
                        "path": ("per-layer calls" if args.per_layer else "layer-batched calls") +
                                " replayed from one CUDA graph"},
