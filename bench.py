@@ -370,7 +370,7 @@ def run_prefill(args):
         g_inst.replay()
     torch.cuda.synchronize()
     clk = clocks.stop()
-    ms_prefill = ev[1].elapsed_time(ev[2]) / L          # one prefill launch (one layer)
+    ms_prefill = ev[1].elapsed_time(ev[2]) / L          # per layer: the layer-batched prefill call / L
     ms_append = ev[0].elapsed_time(ev[1])
     if int(step.status.item()) != 0:
         print(f"device status word set: {int(step.status.item())}", file=sys.stderr)
@@ -382,7 +382,7 @@ def run_prefill(args):
     bound = "hbm" if t_bytes >= t_flops else "tensor"
     achieved_gbs = nb / (ms_prefill * 1e-3) / 1e9
     achieved_tf = nf / (ms_prefill * 1e-3) / 1e12
-    roof = {"kernel": "prefill_kernel (ark_attn_prefill, one layer)", "bound": bound,
+    roof = {"kernel": "prefill_kernel (ark_attn_prefill_layers, per layer)", "bound": bound,
             "achieved": achieved_gbs if bound == "hbm" else achieved_tf,
             "peak": hbm if bound == "hbm" else tc, "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
             "frac": (t_bytes if bound == "hbm" else t_flops) / (ms_prefill * 1e-3),
@@ -398,7 +398,8 @@ def run_prefill(args):
             "config": {"workload": "coalesced causal prefill B=16 L U[20,387] S=387 T=512, 36 layers",
                        "layers": L, "rows": int(batch.n_new.sum()),
                        "l2": "q/o of 36 layers (1.8 GB) larger than L2",
-                       "path": "layer-batched append + per-layer prefill replayed from one CUDA graph"},
+                       "path": "layer-batched append + layer-batched prefill (16 layers per launch) "
+                               "replayed from one CUDA graph"},
             "tokens_layers_per_s": int(batch.n_new.sum()) * L / (ms_step * 1e-3),
             "roofline": roof, "gpu_launches": step.launches_per_step() * args.steps, "clocks": clk}
     if rank == 0:

@@ -9,12 +9,15 @@
 // p = pos0[b] + t, attends to the cache rows j <= p of its KV head.
 //
 // Tiling (B200):
-//   - One CTA per live tile (16 query positions of request b, KV head g).
-//     The grid is the upper bound Hkv x B x ceil(S/16); CTA k takes the k-th
-//     live tile in order of decreasing absolute position (longest key range
-//     first), found on the device from pos0/n_new by a binary search over
-//     position levels, so the CTAs that have no tile are the last ones
-//     dispatched and never hold a slot ahead of real work.  Its 128 MMA
+//   - One CTA per live tile (16 query positions of request b, KV head g, in
+//     one of the launch's layers: up to 16 independent layers per launch).
+//     The grid is the upper bound Hkv x B x ceil(S/16) x L; CTA k takes the
+//     k-th live tile in order of decreasing absolute position (longest key
+//     range first; the layers' copies of a tile next to each other), found on
+//     the device from pos0/n_new by a binary search over position levels, so
+//     the CTAs that have no tile are the last ones dispatched and never hold a
+//     slot ahead of real work, and one launch keeps the SMs busy across
+//     layers instead of draining at every layer.  Its 128 MMA
 //     rows are the 16 positions x the 8 query heads of group g, so every K/V
 //     block is read once for all 8 heads (GQA packing).  The Q tile arrives
 //     by two 4-D TMA boxes (64 head-dim elements each, 128-byte swizzle),
@@ -98,17 +101,20 @@ constexpr uint32_t kIdescPV = kIdescF16 | ((128u >> 3) << 17) | (1u << 16);  // 
 
 constexpr float kLazyRescale = 8.0f;     // log2 units: rescale O only past a factor 2^8
 
+// layers per launch: four tensor maps per layer in the kernel parameters
+// (which hold at most 32 KB)
+constexpr int kLayersPerLaunch = 16;
+
 struct Params {
-    CUtensorMap qmap;    // q as (128, 8, Hq/8, B*S), box (64, 8, 1, 16)
-    CUtensorMap kmap;    // cache_k as (128, Hkv, B*T), box (64, 1, 64)
-    CUtensorMap vmap;
-    CUtensorMap omap;    // o as (128, 8, Hq/8, B*S), box (64, 8, 1, 1): one position, 8 heads, 64 dims
-    uint16_t* o;         // [B, S, Hq, 128]
-    float* lse;          // [B, Hq, S]
+    CUtensorMap qmap[kLayersPerLaunch];   // q as (128, 8, Hq/8, B*S), box (64, 8, 1, 16)
+    CUtensorMap kmap[kLayersPerLaunch];   // cache_k as (128, Hkv, B*T), box (64, 1, 64)
+    CUtensorMap vmap[kLayersPerLaunch];
+    CUtensorMap omap[kLayersPerLaunch];   // o as q, box (64, 8, 1, 1): one position, 8 heads, 64 dims
+    float* lse[kLayersPerLaunch];         // [B, Hq, S]
     const int32_t* pos0;
     const int32_t* n_new;
     uint32_t* status;
-    int B, S, T, Hq, Hkv;
+    int B, S, T, Hq, Hkv, L;
     float scale_log2;
 };
 
@@ -239,8 +245,11 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_ptr, kTmemCols);
-    // every warp finds the CTA's tile by itself (same inputs, same result)
-    const TilePick tile = pick_tile(p, blockIdx.x / p.Hkv, lane, blockIdx.x == 0 && warp == 0);
+    // every warp finds the CTA's tile by itself (same inputs, same result);
+    // consecutive CTAs take the same tile of consecutive layers
+    const int lt = static_cast<int>(blockIdx.x / p.Hkv);
+    const int l = lt % p.L;
+    const TilePick tile = pick_tile(p, lt / p.L, lane, blockIdx.x == 0 && warp == 0);
     const int b = tile.b, qt = tile.qt, nn = tile.nn, p0 = tile.p0;
     const int t0 = qt * kPos;
     const int kv_end = p0 + min(t0 + kPos, nn);             // keys visible to the tile's last row
@@ -250,15 +259,15 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
         const int ks = j % kKStages;
         mbar_arrive_expect_tx(&bars[kBarKFull + ks], kKV);
         uint8_t* kd = smem + kOffK + ks * kKV;
-        tma_load_3d(kd, &p.kmap, 0, g, b * p.T + j * kBN, &bars[kBarKFull + ks]);
-        tma_load_3d(kd + kKHalf, &p.kmap, 64, g, b * p.T + j * kBN, &bars[kBarKFull + ks]);
+        tma_load_3d(kd, &p.kmap[l], 0, g, b * p.T + j * kBN, &bars[kBarKFull + ks]);
+        tma_load_3d(kd + kKHalf, &p.kmap[l], 64, g, b * p.T + j * kBN, &bars[kBarKFull + ks]);
     };
     auto load_v = [&](int j) {
         const int vs = j % kVStages;
         mbar_arrive_expect_tx(&bars[kBarVFull + vs], kKV);
         uint8_t* vd = smem + kOffV + vs * kKV;
-        tma_load_3d(vd, &p.vmap, 0, g, b * p.T + j * kBN, &bars[kBarVFull + vs]);
-        tma_load_3d(vd + kKHalf, &p.vmap, 64, g, b * p.T + j * kBN, &bars[kBarVFull + vs]);
+        tma_load_3d(vd, &p.vmap[l], 0, g, b * p.T + j * kBN, &bars[kBarVFull + vs]);
+        tma_load_3d(vd + kKHalf, &p.vmap[l], 64, g, b * p.T + j * kBN, &bars[kBarVFull + vs]);
     };
     // the first blocks need no free stage: thread 0 (which initialised the
     // barriers) issues them before the CTA barrier
@@ -267,8 +276,8 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
     if (threadIdx.x == 0 && tile.live) {
         mbar_arrive_expect_tx(&bars[kBarQ], 2 * kQHalf);
         const int qrow = b * p.S + t0;
-        tma_load_4d(smem + kOffQ, &p.qmap, 0, 0, g, qrow, &bars[kBarQ]);
-        tma_load_4d(smem + kOffQ + kQHalf, &p.qmap, 64, 0, g, qrow, &bars[kBarQ]);
+        tma_load_4d(smem + kOffQ, &p.qmap[l], 0, 0, g, qrow, &bars[kBarQ]);
+        tma_load_4d(smem + kOffQ + kQHalf, &p.qmap[l], 64, 0, g, qrow, &bars[kBarQ]);
         for (int j = 0; j < min(nblk, kPre); ++j) {
             load_k(j);
             load_v(j);
@@ -515,14 +524,14 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
             if (lane < 4) {
                 const int pp = quad * 4 + lane;              // position of the tile
                 if (t0 + pp < nn) {
-                    tma_store_4d(&p.omap, smem + kOffQ + half * kQHalf + pp * 1024, half * 64, 0, g,
+                    tma_store_4d(&p.omap[l], smem + kOffQ + half * kQHalf + pp * 1024, half * 64, 0, g,
                                  b * p.S + t0 + pp);
                     bulk_commit();
                     bulk_wait_read();
                 }
             }
             if (live && half == 0)
-                p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + tr] = (m_ref + __log2f(e_tot)) * kLn2;
+                p.lse[l][(static_cast<size_t>(b) * p.Hq + h) * p.S + tr] = (m_ref + __log2f(e_tot)) * kLn2;
         }
     }
 
@@ -552,32 +561,42 @@ bool g_prefill_attr[64];
 
 }  // namespace
 
-extern "C" ark_status ark_attn_prefill(const void* q, const void* cache_k, const void* cache_v,
-                                       const int32_t* pos0, const int32_t* n_new, int B, int S, int T, int Hq,
-                                       int Hkv, int D, float scale, void* o, float* lse, uint32_t* d_status,
-                                       cudaStream_t stream) {
-    if (!q || !cache_k || !cache_v || !pos0 || !n_new || !o || !lse) return ARK_ERR_INVALID_ARG;
+namespace {
+
+ark_status prefill_checks(int B, int S, int T, int Hq, int Hkv, int D, float scale) {
     if (B <= 0 || S <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || !(scale > 0.f)) return ARK_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return ARK_ERR_INVALID_ARG;
     if (D != kHeadDim || Hq / Hkv != kGroup) return ARK_ERR_UNSUPPORTED;
     if (T > ARK_MAX_T || B > 65535 || Hkv > 65535) return ARK_ERR_UNSUPPORTED;
     if (static_cast<long long>(B) * S >= (1LL << 31) || static_cast<long long>(B) * T >= (1LL << 31))
         return ARK_ERR_UNSUPPORTED;
-    if (!aligned16(q) || !aligned16(cache_k) || !aligned16(cache_v) || !aligned16(o) ||
-        (reinterpret_cast<uintptr_t>(lse) & 3u))
-        return ARK_ERR_INVALID_ARG;
-    pf::Params prm{};
-    if (!q_group_tensor_map(&prm.qmap, q, static_cast<long long>(B) * S, Hq, 64, pf::kPos) ||
-        !kv_tensor_map(&prm.kmap, cache_k, static_cast<long long>(B) * T, Hkv, 64, pf::kBN) ||
-        !kv_tensor_map(&prm.vmap, cache_v, static_cast<long long>(B) * T, Hkv, 64, pf::kBN) ||
-        !q_group_tensor_map(&prm.omap, o, static_cast<long long>(B) * S, Hq, 64, 1))
-        return ARK_ERR_CUDA;
-    prm.o = static_cast<uint16_t*>(o);
-    prm.lse = lse;
+    return ARK_OK;
+}
+
+// one launch over layers [l0, l0 + n) of the per-layer arrays
+ark_status launch_prefill(const void* const* q, const void* const* cache_k, const void* const* cache_v,
+                          void* const* o, float* const* lse, int l0, int n, const int32_t* pos0,
+                          const int32_t* n_new, int B, int S, int T, int Hq, int Hkv, float scale,
+                          uint32_t* d_status, cudaStream_t stream) {
+    static thread_local pf::Params prm;
+    prm = pf::Params{};
+    for (int i = 0; i < n; ++i) {
+        const int l = l0 + i;
+        if (!q[l] || !cache_k[l] || !cache_v[l] || !o[l] || !lse[l]) return ARK_ERR_INVALID_ARG;
+        if (!aligned16(q[l]) || !aligned16(cache_k[l]) || !aligned16(cache_v[l]) || !aligned16(o[l]) ||
+            (reinterpret_cast<uintptr_t>(lse[l]) & 3u))
+            return ARK_ERR_INVALID_ARG;
+        if (!q_group_tensor_map(&prm.qmap[i], q[l], static_cast<long long>(B) * S, Hq, 64, pf::kPos) ||
+            !kv_tensor_map(&prm.kmap[i], cache_k[l], static_cast<long long>(B) * T, Hkv, 64, pf::kBN) ||
+            !kv_tensor_map(&prm.vmap[i], cache_v[l], static_cast<long long>(B) * T, Hkv, 64, pf::kBN) ||
+            !q_group_tensor_map(&prm.omap[i], o[l], static_cast<long long>(B) * S, Hq, 64, 1))
+            return ARK_ERR_CUDA;
+        prm.lse[i] = lse[l];
+    }
     prm.pos0 = pos0;
     prm.n_new = n_new;
     prm.status = d_status;
-    prm.B = B; prm.S = S; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
+    prm.B = B; prm.S = S; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv; prm.L = n;
     prm.scale_log2 = scale * kLog2e;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARK_ERR_CUDA;
@@ -587,8 +606,40 @@ extern "C" ark_status ark_attn_prefill(const void* q, const void* cache_k, const
             return ARK_ERR_CUDA;
         g_prefill_attr[dev] = true;
     }
-    const long long ctas = static_cast<long long>(Hkv) * B * ((S + pf::kPos - 1) / pf::kPos);
+    const long long ctas = static_cast<long long>(Hkv) * B * ((S + pf::kPos - 1) / pf::kPos) * n;
     if (ctas >= (1LL << 31)) return ARK_ERR_UNSUPPORTED;
     prefill_kernel<<<static_cast<unsigned>(ctas), pf::kThreads, pf::kSmemBytes, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" ark_status ark_attn_prefill(const void* q, const void* cache_k, const void* cache_v,
+                                       const int32_t* pos0, const int32_t* n_new, int B, int S, int T, int Hq,
+                                       int Hkv, int D, float scale, void* o, float* lse, uint32_t* d_status,
+                                       cudaStream_t stream) {
+    if (!q || !cache_k || !cache_v || !pos0 || !n_new || !o || !lse) return ARK_ERR_INVALID_ARG;
+    ark_status st = prefill_checks(B, S, T, Hq, Hkv, D, scale);
+    if (st != ARK_OK) return st;
+    return launch_prefill(&q, &cache_k, &cache_v, &o, &lse, 0, 1, pos0, n_new, B, S, T, Hq, Hkv, scale, d_status,
+                          stream);
+}
+
+extern "C" ark_status ark_attn_prefill_layers(int L, const void* const* q, const void* const* cache_k,
+                                              const void* const* cache_v, const int32_t* pos0,
+                                              const int32_t* n_new, int B, int S, int T, int Hq, int Hkv, int D,
+                                              float scale, void* const* o, float* const* lse, uint32_t* d_status,
+                                              cudaStream_t stream) {
+    if (!q || !cache_k || !cache_v || !pos0 || !n_new || !o || !lse) return ARK_ERR_INVALID_ARG;
+    if (L <= 0) return ARK_ERR_INVALID_ARG;
+    if (L > ARK_MAX_LAYERS) return ARK_ERR_UNSUPPORTED;
+    ark_status st = prefill_checks(B, S, T, Hq, Hkv, D, scale);
+    if (st != ARK_OK) return st;
+    for (int l0 = 0; l0 < L; l0 += pf::kLayersPerLaunch) {
+        const int n = (L - l0 < pf::kLayersPerLaunch) ? L - l0 : pf::kLayersPerLaunch;
+        st = launch_prefill(q, cache_k, cache_v, o, lse, l0, n, pos0, n_new, B, S, T, Hq, Hkv, scale, d_status,
+                            stream);
+        if (st != ARK_OK) return st;
+    }
+    return ARK_OK;
 }

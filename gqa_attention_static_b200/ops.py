@@ -52,6 +52,7 @@ EXPORTS = (
     "ark_attn_append_rope_fp8_layers",
     "ark_attn_decode_fp8",
     "ark_attn_decode_fp8_layers",
+    "ark_attn_prefill_layers",
 )
 
 
@@ -112,6 +113,8 @@ def load() -> ctypes.CDLL:
     lib.ark_attn_decode_fp8_layers.argtypes = [I, PP, PP, PP, PP, PP, P, I, I, I, I, I, ctypes.c_float, I, I, P,
                                                Z, PP, PP, P, P]
     lib.ark_attn_decode_fp8_layers.restype = I
+    lib.ark_attn_prefill_layers.argtypes = [I, PP, PP, PP, P, P, I, I, I, I, I, I, ctypes.c_float, PP, PP, P, P]
+    lib.ark_attn_prefill_layers.restype = I
     _lib = lib
     return lib
 
@@ -519,3 +522,32 @@ def ark_attn_decode_fp8_layers(q: Sequence[torch.Tensor], cache_k, cache_v, k_sc
                                              D, float(scale), int(mode), int(max_splits), _ptr(workspace), ws_bytes,
                                              _ptr_array(o), _ptr_array(lse), _ptr(status), _stream(stream)),
            "ark_attn_decode_fp8_layers")
+
+
+def ark_attn_prefill_layers(q: Sequence[torch.Tensor], cache_k, cache_v, pos0, n_new, o, lse, scale: float,
+                            status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """ark_attn_prefill over L independent layers (up to 16 layers per launch)."""
+    L = len(q)
+    if not (len(cache_k) == len(cache_v) == len(o) == len(lse) == L) or L == 0:
+        raise ValueError("per-layer lists must have the same non-zero length")
+    for i in range(L):
+        _need(q[i], "q", torch.bfloat16, 4)
+        _need(cache_k[i], "cache_k", torch.bfloat16, 4)
+        _need(cache_v[i], "cache_v", torch.bfloat16, 4)
+        _need(o[i], "o", torch.bfloat16, 4)
+        _need(lse[i], "lse", torch.float32, 3)
+        if q[i].shape != q[0].shape or cache_k[i].shape != cache_k[0].shape or cache_v[i].shape != cache_k[0].shape \
+                or o[i].shape != q[0].shape or lse[i].shape != lse[0].shape:
+            raise ValueError("all layers must have the same shapes")
+    _need(pos0, "pos0", torch.int32, 1)
+    _need(n_new, "n_new", torch.int32, 1)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    B, S, Hq, D = q[0].shape
+    T, Hkv = cache_k[0].shape[1], cache_k[0].shape[2]
+    if tuple(lse[0].shape) != (B, Hq, S):
+        raise ValueError("lse must be [B, Hq, S]")
+    _raise(load().ark_attn_prefill_layers(L, _ptr_array(q), _ptr_array(cache_k), _ptr_array(cache_v), _ptr(pos0),
+                                          _ptr(n_new), B, S, T, Hq, Hkv, D, float(scale), _ptr_array(o),
+                                          _ptr_array(lse), _ptr(status), _stream(stream)),
+           "ark_attn_prefill_layers")

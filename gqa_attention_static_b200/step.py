@@ -127,7 +127,8 @@ class DecodeStep:
 class PrefillStep:
     """Prefill of one prompt batch over L independent layers: RoPE + delta
     write of the prompt rows for all layers (one launch), then the causal
-    tcgen05 prefill of each layer (one launch per layer).
+    tcgen05 prefill of all layers (one launch per 16 layers; one launch per
+    layer with batched=False).
 
     Buffers (per layer lists): q [B,S,Hq,D] (rotated in place), k_new/v_new
     [B,S,Hkv,D], cache_k/cache_v [B,T,Hkv,D]; outputs o [B,S,Hq,D] bf16 and
@@ -135,7 +136,8 @@ class PrefillStep:
     """
 
     def __init__(self, q, k_new, v_new, cache_k, cache_v, pos0, n_new, rope_theta: float = 1e6,
-                 scale: Optional[float] = None):
+                 scale: Optional[float] = None, batched: bool = True):
+        self.batched = batched
         self.q, self.k_new, self.v_new = q, k_new, v_new
         self.cache_k, self.cache_v = cache_k, cache_v
         self.pos0, self.n_new = pos0, n_new
@@ -150,16 +152,20 @@ class PrefillStep:
         self.lse = [torch.empty(self.B, self.Hq, self.S, dtype=torch.float32, device=dev) for _ in q]
 
     def launches_per_step(self) -> int:
-        return 1 + self.layers
+        return 1 + ((self.layers + 15) // 16 if self.batched else self.layers)
 
     def append(self, stream=None) -> None:
         ops.ark_attn_append_rope_layers(self.q, self.k_new, self.v_new, self.cache_k, self.cache_v, self.pos0,
                                         self.n_new, self.table, self.status, stream)
 
     def attention(self, stream=None) -> None:
-        for l in range(self.layers):
-            ops.ark_attn_prefill(self.q[l], self.cache_k[l], self.cache_v[l], self.pos0, self.n_new, self.o[l],
-                                 self.lse[l], self.scale, self.status, stream)
+        if self.batched:
+            ops.ark_attn_prefill_layers(self.q, self.cache_k, self.cache_v, self.pos0, self.n_new, self.o, self.lse,
+                                        self.scale, self.status, stream)
+        else:
+            for l in range(self.layers):
+                ops.ark_attn_prefill(self.q[l], self.cache_k[l], self.cache_v[l], self.pos0, self.n_new, self.o[l],
+                                     self.lse[l], self.scale, self.status, stream)
 
     def run(self, stream=None) -> None:
         self.append(stream)

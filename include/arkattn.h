@@ -186,11 +186,19 @@ ARK_API ark_status ark_attn_prefill(const void* q, const void* cache_k, const vo
  * device pointers (read during the call; the array itself may be freed when
  * the call returns).  All layers share B, S, T, the positions/lengths and the
  * rotary table.  Each layer's tensors follow the single-layer layouts above.
+ * ark_attn_prefill_layers runs the tiles of up to 16 layers in one launch
+ * (longer lists take several launches, in order on `stream`), so that the GPU
+ * does not drain at every layer boundary.
  * The decode workspace is ark_attn_decode_layers_workspace_size(L, ...) bytes
  * under the same rules.  Meant for callers that hold
  * several independent caches (the ARK-ASR-3B decoder has 36 layers), and for
  * measuring the kernels without per-launch overhead.
  */
+ARK_API ark_status ark_attn_prefill_layers(int L, const void* const* q, const void* const* cache_k,
+                                           const void* const* cache_v, const int32_t* pos0, const int32_t* n_new,
+                                           int B, int S, int T, int Hq, int Hkv, int D, float scale,
+                                           void* const* o, float* const* lse, uint32_t* d_status,
+                                           cudaStream_t stream);
 ARK_API ark_status ark_attn_append_rope_layers(int L, void* const* q, const void* const* k_new,
                                                const void* const* v_new, void* const* cache_k,
                                                void* const* cache_v, const int32_t* pos0,

@@ -128,3 +128,56 @@ def test_prefill_bad_lengths_set_status(oracle_lib):
     ops.ark_attn_prefill(q, ck, ck, batch.pos0.to(dev), batch.n_new.to(dev), o, lse, SCALE, status)
     torch.cuda.synchronize()
     assert int(status.item()) & ops.ARK_DEV_BAD_POS
+
+
+def test_prefill_layers_matches_oracle(oracle_lib):
+    """ark_attn_prefill_layers: three layers with their own caches in one
+    launch, each against the oracle (the same causal prefill per layer)."""
+    L = 3
+    batch = W.make_batch(510, B=3, S=40, T=256, pos0=[0, 30, 100], n_new=[40, 17, 5], layers=L, garbage="nan")
+    dev = "cuda"
+    q = [x.to(dev).clone() for x in batch.q]
+    ck = [x.to(dev).clone() for x in batch.cache_k]
+    cv = [x.to(dev).clone() for x in batch.cache_v]
+    pos0, n_new = batch.pos0.to(dev), batch.n_new.to(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ops.ark_attn_append_rope_layers(q, [x.to(dev) for x in batch.k_new], [x.to(dev) for x in batch.v_new], ck, cv,
+                                    pos0, n_new, ops.rope_table(batch.T), status)
+    B, S, Hq, D = q[0].shape
+    o = [torch.empty_like(x).view(torch.int16).fill_(SENTINEL).view(torch.bfloat16) for x in q]
+    lse = [torch.full((B, Hq, S), float("nan"), dtype=torch.float32, device=dev) for _ in q]
+    ops.ark_attn_prefill_layers(q, ck, cv, pos0, n_new, o, lse, SCALE, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for l in range(L):
+        q_ref, ck_ref, cv_ref, o_ref, lse_ref = oracle_append_prefill(batch, l)
+        for b in range(B):
+            n = int(batch.n_new[b])
+            check_o(f64(o[l])[b, :n], o_ref[b, :n], f"o layer {l} request {b}")
+            check_lse(f64(lse[l])[b, :, :n], lse_ref[b, :, :n], f"lse layer {l} request {b}")
+            assert np.all(bits(o[l])[b, n:] == SENTINEL)
+
+
+def test_prefill_layers_across_launches_equals_single_layer_calls(oracle_lib):
+    """18 layers take two launches (16 + 2); every layer's output is bit for bit
+    the single-layer call's (the same tile arithmetic), padded rows untouched."""
+    L = 18
+    batch = W.make_batch(511, B=2, S=20, T=64, pos0=[0, 37], n_new=[20, 9], layers=L)
+    dev = "cuda"
+    q = [x.to(dev).clone() for x in batch.q]
+    ck = [x.to(dev).clone() for x in batch.cache_k]
+    cv = [x.to(dev).clone() for x in batch.cache_v]
+    pos0, n_new = batch.pos0.to(dev), batch.n_new.to(dev)
+    ops.ark_attn_append_rope_layers(q, [x.to(dev) for x in batch.k_new], [x.to(dev) for x in batch.v_new], ck, cv,
+                                    pos0, n_new, ops.rope_table(batch.T))
+    B, S, Hq, D = q[0].shape
+    o = [torch.empty_like(x).view(torch.int16).fill_(SENTINEL).view(torch.bfloat16) for x in q]
+    lse = [torch.full((B, Hq, S), float("nan"), dtype=torch.float32, device=dev) for _ in q]
+    ops.ark_attn_prefill_layers(q, ck, cv, pos0, n_new, o, lse, SCALE)
+    for l in range(L):
+        o1 = torch.empty_like(q[l]).view(torch.int16).fill_(SENTINEL).view(torch.bfloat16)
+        l1 = torch.full((B, Hq, S), float("nan"), dtype=torch.float32, device=dev)
+        ops.ark_attn_prefill(q[l], ck[l], cv[l], pos0, n_new, o1, l1, SCALE)
+        torch.cuda.synchronize()
+        assert torch.equal(o[l].view(torch.int16), o1.view(torch.int16)), f"layer {l}"
+        assert torch.equal(torch.nan_to_num(lse[l], nan=-7.0), torch.nan_to_num(l1, nan=-7.0)), f"layer {l}"
