@@ -72,6 +72,8 @@ def parse():
     ap.add_argument("--max-splits", type=int, default=8)
     ap.add_argument("--per-layer", action="store_true",
                     help="issue the single-layer calls layer by layer instead of the layer-batched calls")
+    ap.add_argument("--rope-on-load", action="store_true",
+                    help="prefill: K/V-only append, RoPE applied by the prefill kernel as it loads q")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -333,7 +335,8 @@ def run_prefill(args):
     L = batch.layers
     step = PrefillStep([x.to(dev) for x in batch.q], [x.to(dev) for x in batch.k_new],
                        [x.to(dev) for x in batch.v_new], [x.to(dev) for x in batch.cache_k],
-                       [x.to(dev) for x in batch.cache_v], batch.pos0.to(dev), batch.n_new.to(dev))
+                       [x.to(dev) for x in batch.cache_v], batch.pos0.to(dev), batch.n_new.to(dev),
+                       fused_rope=args.rope_on_load)
     s = torch.cuda.Stream(device=dev)
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
@@ -382,7 +385,8 @@ def run_prefill(args):
     bound = "hbm" if t_bytes >= t_flops else "tensor"
     achieved_gbs = nb / (ms_prefill * 1e-3) / 1e9
     achieved_tf = nf / (ms_prefill * 1e-3) / 1e12
-    roof = {"kernel": "prefill_kernel (ark_attn_prefill_layers, per layer)", "bound": bound,
+    roof = {"kernel": "prefill_kernel (ark_attn_prefill%s_layers, per layer)" % ("_rope" if args.rope_on_load else ""),
+            "bound": bound,
             "achieved": achieved_gbs if bound == "hbm" else achieved_tf,
             "peak": hbm if bound == "hbm" else tc, "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
             "frac": (t_bytes if bound == "hbm" else t_flops) / (ms_prefill * 1e-3),
@@ -398,8 +402,9 @@ def run_prefill(args):
             "config": {"workload": "coalesced causal prefill B=16 L U[20,387] S=387 T=512, 36 layers",
                        "layers": L, "rows": int(batch.n_new.sum()),
                        "l2": "q/o of 36 layers (1.8 GB) larger than L2",
-                       "path": "layer-batched append + layer-batched prefill (16 layers per launch) "
-                               "replayed from one CUDA graph"},
+                       "path": ("layer-batched K/V append + layer-batched prefill rotating q as it loads it"
+                                if args.rope_on_load else "layer-batched append + layer-batched prefill") +
+                               " (16 layers per launch), replayed from one CUDA graph"},
             "tokens_layers_per_s": int(batch.n_new.sum()) * L / (ms_step * 1e-3),
             "roofline": roof, "gpu_launches": step.launches_per_step() * args.steps, "clocks": clk}
     if rank == 0:

@@ -20,10 +20,12 @@
 // fp32 and converted to e4m3 with cvt.rn.satfinite; values likewise.  q is
 // rotated to bf16 exactly as above.
 //
-// Work: one CTA per (t, b, layer) row; 128 threads cover (Hq + Hkv) heads x 16
-// groups of 4 rotary pairs, plus Hkv x 16 16-byte pieces of the V copy.  The op
-// moves ~10 KB per row and is latency-bound; it exists so the caller never
-// crosses to the host between the projection and the attention.
+// Work: one CTA per (request, layer) and group of rows (one row for a decode
+// step, 8 consecutive rows of a prompt, so that a long padded prompt batch
+// does not launch a CTA per padded row); 128 threads cover, per row, (Hq +
+// Hkv) heads x 16 groups of 4 rotary pairs plus Hkv x 16 16-byte pieces of the
+// V copy.  The op is small next to the attention; it exists so the caller
+// never crosses to the host between the projection and the attention.
 #include "common.cuh"
 
 namespace ark {
@@ -44,6 +46,8 @@ struct AppendParams {
     const float2* table;  // [T][64] {cos, sin}
     uint32_t* status;
     int B, S, T, Hq, Hkv;
+    int rotate_q;         // 0: K/V rows only (q is rotated where it is read, by the prefill)
+    int rows_per_cta;     // consecutive rows t of one (request, layer) per CTA
     AppendLayer layer[ARK_MAX_LAYERS];
 };
 
@@ -53,117 +57,129 @@ __global__ void __launch_bounds__(128) append_rope_kernel(const __grid_constant_
     // (the decode) may start its own prologue now; it waits for this grid's
     // completion (griddepcontrol.wait) before it reads q or the cache
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int t = blockIdx.x;
     const int b = blockIdx.y;
     const AppendLayer& L = p.layer[blockIdx.z];
 
     int nn = __ldg(p.n_new + b);
     if (nn < 0 || nn > p.S) {
-        if (threadIdx.x == 0 && t == 0 && blockIdx.z == 0) report(p.status, ARK_DEV_BAD_KVLEN);
+        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) report(p.status, ARK_DEV_BAD_KVLEN);
         nn = nn < 0 ? 0 : p.S;
     }
-    if (t >= nn) return;
-    const int pos = __ldg(p.pos0 + b) + t;
-    if (pos < 0 || pos >= p.T) {
-        if (threadIdx.x == 0 && blockIdx.z == 0) report(p.status, ARK_DEV_BAD_POS);
-        return;
-    }
+    const int p0 = __ldg(p.pos0 + b);
+    const int t_end = min(nn, (static_cast<int>(blockIdx.x) + 1) * p.rows_per_cta);
+    for (int t = blockIdx.x * p.rows_per_cta; t < t_end; ++t) {
+        const int pos = p0 + t;
+        if (pos < 0 || pos >= p.T) {
+            if (threadIdx.x == 0 && blockIdx.z == 0) report(p.status, ARK_DEV_BAD_POS);
+            continue;
+        }
 
-    const int nrot = (p.Hq + p.Hkv) * 16;    // items of 4 rotary pairs
-    const int ncopy = p.Hkv * 16;            // 16-byte pieces of V rows
-    const float4* trow = reinterpret_cast<const float4*>(p.table + static_cast<size_t>(pos) * 64);
+        const int qh = p.rotate_q ? p.Hq : 0;    // query heads this call rotates
+        const int nrot = (qh + p.Hkv) * 16;      // items of 4 rotary pairs
+        const int ncopy = p.Hkv * 16;            // 16-byte pieces of V rows
+        const float4* trow = reinterpret_cast<const float4*>(p.table + static_cast<size_t>(pos) * 64);
 
-    for (int it = threadIdx.x; it < nrot + ncopy; it += blockDim.x) {
-        if (it < nrot) {
-            const int head = it >> 4;
-            const int pg = it & 15;           // pairs 4pg .. 4pg+3
-            const uint16_t* src;
-            uint16_t* dst = nullptr;
-            uint8_t* dst8 = nullptr;
-            double kscale = 1.0;
-            if (head < p.Hq) {
-                uint16_t* row = L.q + ((static_cast<size_t>(b) * p.S + t) * p.Hq + head) * kHeadDim;
-                src = row;
-                dst = row;
-            } else {
-                const int g = head - p.Hq;
-                src = L.k_new + ((static_cast<size_t>(b) * p.S + t) * p.Hkv + g) * kHeadDim;
-                const size_t off = ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + g) * kHeadDim;
-                if (Fp8) {
-                    dst8 = static_cast<uint8_t*>(L.cache_k) + off;
-                    kscale = static_cast<double>(__ldg(L.k_scale + g));
+        for (int it = threadIdx.x; it < nrot + ncopy; it += blockDim.x) {
+            if (it < nrot) {
+                const int head = it >> 4;
+                const int pg = it & 15;           // pairs 4pg .. 4pg+3
+                const uint16_t* src;
+                uint16_t* dst = nullptr;
+                uint8_t* dst8 = nullptr;
+                double kscale = 1.0;
+                if (head < qh) {
+                    uint16_t* row = L.q + ((static_cast<size_t>(b) * p.S + t) * p.Hq + head) * kHeadDim;
+                    src = row;
+                    dst = row;
                 } else {
-                    dst = static_cast<uint16_t*>(L.cache_k) + off;
+                    const int g = head - qh;
+                    src = L.k_new + ((static_cast<size_t>(b) * p.S + t) * p.Hkv + g) * kHeadDim;
+                    const size_t off = ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + g) * kHeadDim;
+                    if (Fp8) {
+                        dst8 = static_cast<uint8_t*>(L.cache_k) + off;
+                        kscale = static_cast<double>(__ldg(L.k_scale + g));
+                    } else {
+                        dst = static_cast<uint16_t*>(L.cache_k) + off;
+                    }
                 }
-            }
-            const uint2 lo = *reinterpret_cast<const uint2*>(src + 4 * pg);
-            const uint2 hi = *reinterpret_cast<const uint2*>(src + 64 + 4 * pg);
-            const float4 cs01 = __ldg(trow + 2 * pg);      // c0 s0 c1 s1
-            const float4 cs23 = __ldg(trow + 2 * pg + 1);  // c2 s2 c3 s3
-            const uint16_t xl[4] = {static_cast<uint16_t>(lo.x & 0xffff), static_cast<uint16_t>(lo.x >> 16),
-                                    static_cast<uint16_t>(lo.y & 0xffff), static_cast<uint16_t>(lo.y >> 16)};
-            const uint16_t xh[4] = {static_cast<uint16_t>(hi.x & 0xffff), static_cast<uint16_t>(hi.x >> 16),
-                                    static_cast<uint16_t>(hi.y & 0xffff), static_cast<uint16_t>(hi.y >> 16)};
-            const float cc[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
-            const float ss[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
-            uint16_t yl[4], yh[4];
-            double dl[4], dh[4];
+                const uint2 lo = *reinterpret_cast<const uint2*>(src + 4 * pg);
+                const uint2 hi = *reinterpret_cast<const uint2*>(src + 64 + 4 * pg);
+                const float4 cs01 = __ldg(trow + 2 * pg);      // c0 s0 c1 s1
+                const float4 cs23 = __ldg(trow + 2 * pg + 1);  // c2 s2 c3 s3
+                const uint16_t xl[4] = {static_cast<uint16_t>(lo.x & 0xffff), static_cast<uint16_t>(lo.x >> 16),
+                                        static_cast<uint16_t>(lo.y & 0xffff), static_cast<uint16_t>(lo.y >> 16)};
+                const uint16_t xh[4] = {static_cast<uint16_t>(hi.x & 0xffff), static_cast<uint16_t>(hi.x >> 16),
+                                        static_cast<uint16_t>(hi.y & 0xffff), static_cast<uint16_t>(hi.y >> 16)};
+                const float cc[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
+                const float ss[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
+                if (Fp8 && dst8) {
+                    // the key for the fp8 cache is quantised from the unrounded rotation, in double
+                    double dl[4], dh[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const double a = bf16_bits_to_f64(xl[i]);
-                const double h = bf16_bits_to_f64(xh[i]);
-                const double c = static_cast<double>(cc[i]);
-                const double s = static_cast<double>(ss[i]);
-                // both products are exact in double, so contraction cannot change the result
-                dl[i] = a * c - h * s;
-                dh[i] = h * c + a * s;
-                yl[i] = f64_to_bf16_rn(dl[i]);
-                yh[i] = f64_to_bf16_rn(dh[i]);
-            }
-            if (Fp8 && dst8) {
-                // the key into the fp8 cache: e4m3(fp32(y / scale)), two codes per conversion
-                uint32_t cl = 0, ch = 0;
+                    for (int i = 0; i < 4; ++i) {
+                        const double a = bf16_bits_to_f64(xl[i]);
+                        const double h = bf16_bits_to_f64(xh[i]);
+                        const double c = static_cast<double>(cc[i]);
+                        const double s = static_cast<double>(ss[i]);
+                        // both products are exact in double, so contraction cannot change the result
+                        dl[i] = a * c - h * s;
+                        dh[i] = h * c + a * s;
+                    }
+                    // the key into the fp8 cache: e4m3(fp32(y / scale)), two codes per conversion
+                    uint32_t cl = 0, ch = 0;
 #pragma unroll
-                for (int i = 0; i < 4; i += 2) {
-                    cl |= static_cast<uint32_t>(f32x2_to_e4m3x2(__double2float_rn(dl[i] / kscale),
-                                                                __double2float_rn(dl[i + 1] / kscale))) << (8 * i);
-                    ch |= static_cast<uint32_t>(f32x2_to_e4m3x2(__double2float_rn(dh[i] / kscale),
-                                                                __double2float_rn(dh[i + 1] / kscale))) << (8 * i);
+                    for (int i = 0; i < 4; i += 2) {
+                        cl |= static_cast<uint32_t>(f32x2_to_e4m3x2(__double2float_rn(dl[i] / kscale),
+                                                                    __double2float_rn(dl[i + 1] / kscale))) << (8 * i);
+                        ch |= static_cast<uint32_t>(f32x2_to_e4m3x2(__double2float_rn(dh[i] / kscale),
+                                                                    __double2float_rn(dh[i + 1] / kscale))) << (8 * i);
+                    }
+                    *reinterpret_cast<uint32_t*>(dst8 + 4 * pg) = cl;
+                    *reinterpret_cast<uint32_t*>(dst8 + 64 + 4 * pg) = ch;
+                    continue;
                 }
-                *reinterpret_cast<uint32_t*>(dst8 + 4 * pg) = cl;
-                *reinterpret_cast<uint32_t*>(dst8 + 64 + 4 * pg) = ch;
-                continue;
-            }
-            uint2 ol, oh;
-            ol.x = static_cast<uint32_t>(yl[0]) | (static_cast<uint32_t>(yl[1]) << 16);
-            ol.y = static_cast<uint32_t>(yl[2]) | (static_cast<uint32_t>(yl[3]) << 16);
-            oh.x = static_cast<uint32_t>(yh[0]) | (static_cast<uint32_t>(yh[1]) << 16);
-            oh.y = static_cast<uint32_t>(yh[2]) | (static_cast<uint32_t>(yh[3]) << 16);
-            *reinterpret_cast<uint2*>(dst + 4 * pg) = ol;
-            *reinterpret_cast<uint2*>(dst + 64 + 4 * pg) = oh;
-        } else {
-            const int c = it - nrot;
-            const int g = c >> 4;
-            const int piece = c & 15;
-            const uint4* src = reinterpret_cast<const uint4*>(
-                L.v_new + ((static_cast<size_t>(b) * p.S + t) * p.Hkv + g) * kHeadDim);
-            const size_t off = ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + g) * kHeadDim;
-            if (Fp8) {
-                // 8 values -> 8 codes: e4m3(fp32(v / scale))
-                const double vscale = static_cast<double>(__ldg(L.v_scale + g));
-                const uint4 x = src[piece];
-                const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-                uint32_t out[2] = {0, 0};
+                uint16_t yl[4], yh[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const float f0 = __double2float_rn(bf16_bits_to_f64(static_cast<uint16_t>(w[i] & 0xffff)) / vscale);
-                    const float f1 = __double2float_rn(bf16_bits_to_f64(static_cast<uint16_t>(w[i] >> 16)) / vscale);
-                    out[i >> 1] |= static_cast<uint32_t>(f32x2_to_e4m3x2(f0, f1)) << (16 * (i & 1));
+                    const double a = bf16_bits_to_f64(xl[i]);
+                    const double h = bf16_bits_to_f64(xh[i]);
+                    const double c = static_cast<double>(cc[i]);
+                    const double s = static_cast<double>(ss[i]);
+                    // both products are exact in double, so contraction cannot change the result
+                    yl[i] = f64_to_bf16_rn(a * c - h * s);
+                    yh[i] = f64_to_bf16_rn(h * c + a * s);
                 }
-                *reinterpret_cast<uint2*>(static_cast<uint8_t*>(L.cache_v) + off + 8 * piece) = make_uint2(out[0], out[1]);
+                uint2 ol, oh;
+                ol.x = static_cast<uint32_t>(yl[0]) | (static_cast<uint32_t>(yl[1]) << 16);
+                ol.y = static_cast<uint32_t>(yl[2]) | (static_cast<uint32_t>(yl[3]) << 16);
+                oh.x = static_cast<uint32_t>(yh[0]) | (static_cast<uint32_t>(yh[1]) << 16);
+                oh.y = static_cast<uint32_t>(yh[2]) | (static_cast<uint32_t>(yh[3]) << 16);
+                *reinterpret_cast<uint2*>(dst + 4 * pg) = ol;
+                *reinterpret_cast<uint2*>(dst + 64 + 4 * pg) = oh;
             } else {
-                uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(L.cache_v) + off);
-                dst[piece] = src[piece];
+                const int c = it - nrot;
+                const int g = c >> 4;
+                const int piece = c & 15;
+                const uint4* src = reinterpret_cast<const uint4*>(
+                    L.v_new + ((static_cast<size_t>(b) * p.S + t) * p.Hkv + g) * kHeadDim);
+                const size_t off = ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + g) * kHeadDim;
+                if (Fp8) {
+                    // 8 values -> 8 codes: e4m3(fp32(v / scale))
+                    const double vscale = static_cast<double>(__ldg(L.v_scale + g));
+                    const uint4 x = src[piece];
+                    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+                    uint32_t out[2] = {0, 0};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float f0 = __double2float_rn(bf16_bits_to_f64(static_cast<uint16_t>(w[i] & 0xffff)) / vscale);
+                        const float f1 = __double2float_rn(bf16_bits_to_f64(static_cast<uint16_t>(w[i] >> 16)) / vscale);
+                        out[i >> 1] |= static_cast<uint32_t>(f32x2_to_e4m3x2(f0, f1)) << (16 * (i & 1));
+                    }
+                    *reinterpret_cast<uint2*>(static_cast<uint8_t*>(L.cache_v) + off + 8 * piece) = make_uint2(out[0], out[1]);
+                } else {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(L.cache_v) + off);
+                    dst[piece] = src[piece];
+                }
             }
         }
     }
@@ -187,7 +203,11 @@ ark_status check_common(int B, int S, int T, int Hq, int Hkv, int D) {
 }
 
 ark_status launch_append(AppendParams& prm, int L, bool fp8, cudaStream_t stream) {
-    dim3 grid(prm.S, prm.B, L);
+    // K/V rows only, of a long prompt: several rows per CTA, so that the grid
+    // is not a CTA per (mostly padded) row; with the query rows each row is
+    // enough work for its own CTA
+    prm.rows_per_cta = (prm.S >= 64 && !prm.rotate_q) ? 8 : 1;
+    dim3 grid((prm.S + prm.rows_per_cta - 1) / prm.rows_per_cta, prm.B, L);
     if (fp8)
         append_rope_kernel<true><<<grid, 128, 0, stream>>>(prm);
     else
@@ -219,6 +239,7 @@ extern "C" ark_status ark_attn_append_rope(void* q, const void* k_new, const voi
     prm.table = reinterpret_cast<const float2*>(d_table);
     prm.status = d_status;
     prm.B = B; prm.S = S; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
+    prm.rotate_q = 1;
     prm.layer[0] = AppendLayer{static_cast<uint16_t*>(q), static_cast<const uint16_t*>(k_new),
                                static_cast<const uint16_t*>(v_new), cache_k, cache_v, nullptr, nullptr};
     return launch_append(prm, 1, false, stream);
@@ -244,6 +265,7 @@ extern "C" ark_status ark_attn_append_rope_layers(int L, void* const* q, const v
     prm.table = reinterpret_cast<const float2*>(d_table);
     prm.status = d_status;
     prm.B = B; prm.S = S; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
+    prm.rotate_q = 1;
     for (int l = 0; l < L; ++l) {
         if (!q[l] || !k_new[l] || !v_new[l] || !cache_k[l] || !cache_v[l]) return ARK_ERR_INVALID_ARG;
         if (!aligned16(q[l]) || !aligned16(k_new[l]) || !aligned16(v_new[l]) || !aligned16(cache_k[l]) ||
@@ -276,6 +298,7 @@ extern "C" ark_status ark_attn_append_rope_fp8_layers(int L, void* const* q, con
     prm.table = reinterpret_cast<const float2*>(d_table);
     prm.status = d_status;
     prm.B = B; prm.S = S; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
+    prm.rotate_q = 1;
     for (int l = 0; l < L; ++l) {
         if (!q[l] || !k_new[l] || !v_new[l] || !cache_k[l] || !cache_v[l] || !k_scale[l] || !v_scale[l])
             return ARK_ERR_INVALID_ARG;
@@ -298,4 +321,41 @@ extern "C" ark_status ark_attn_append_rope_fp8(void* q, const void* k_new, const
     const void* vn = v_new;
     return ark_attn_append_rope_fp8_layers(1, &q, &kn, &vn, &cache_k, &cache_v, &k_scale, &v_scale, pos0, n_new,
                                            B, S, T, Hq, Hkv, D, d_table, d_status, stream);
+}
+
+extern "C" ark_status ark_attn_append_rope_kv_layers(int L, const void* const* k_new, const void* const* v_new,
+                                                     void* const* cache_k, void* const* cache_v, const int32_t* pos0,
+                                                     const int32_t* n_new, int B, int S, int T, int Hq, int Hkv,
+                                                     int D, const float* d_table, uint32_t* d_status,
+                                                     cudaStream_t stream) {
+    if (!k_new || !v_new || !cache_k || !cache_v || !pos0 || !n_new || !d_table) return ARK_ERR_INVALID_ARG;
+    if (L <= 0) return ARK_ERR_INVALID_ARG;
+    if (L > ARK_MAX_LAYERS) return ARK_ERR_UNSUPPORTED;
+    ark_status st = check_common(B, S, T, Hq, Hkv, D);
+    if (st != ARK_OK) return st;
+    if (S > 65535) return ARK_ERR_UNSUPPORTED;
+    if (!aligned16(d_table)) return ARK_ERR_INVALID_ARG;
+    AppendParams prm{};
+    prm.pos0 = pos0;
+    prm.n_new = n_new;
+    prm.table = reinterpret_cast<const float2*>(d_table);
+    prm.status = d_status;
+    prm.B = B; prm.S = S; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv;
+    prm.rotate_q = 0;
+    for (int l = 0; l < L; ++l) {
+        if (!k_new[l] || !v_new[l] || !cache_k[l] || !cache_v[l]) return ARK_ERR_INVALID_ARG;
+        if (!aligned16(k_new[l]) || !aligned16(v_new[l]) || !aligned16(cache_k[l]) || !aligned16(cache_v[l]))
+            return ARK_ERR_INVALID_ARG;
+        prm.layer[l] = AppendLayer{nullptr, static_cast<const uint16_t*>(k_new[l]),
+                                   static_cast<const uint16_t*>(v_new[l]), cache_k[l], cache_v[l], nullptr, nullptr};
+    }
+    return launch_append(prm, L, false, stream);
+}
+
+extern "C" ark_status ark_attn_append_rope_kv(const void* k_new, const void* v_new, void* cache_k, void* cache_v,
+                                              const int32_t* pos0, const int32_t* n_new, int B, int S, int T,
+                                              int Hq, int Hkv, int D, const float* d_table, uint32_t* d_status,
+                                              cudaStream_t stream) {
+    return ark_attn_append_rope_kv_layers(1, &k_new, &v_new, &cache_k, &cache_v, pos0, n_new, B, S, T, Hq, Hkv, D,
+                                          d_table, d_status, stream);
 }

@@ -82,7 +82,8 @@ constexpr int kBarVEmpty = kBarVFull + kVStages;   // kVStages
 constexpr int kBarSFull = kBarVEmpty + kVStages;   // 2
 constexpr int kBarPFull = kBarSFull + 2;           // 2
 constexpr int kBarPvDone = kBarPFull + 2;
-constexpr int kNumBars = kBarPvDone + 1;
+constexpr int kBarQRot = kBarPvDone + 1;           // rotated Q tile in place (count: softmax threads)
+constexpr int kNumBars = kBarQRot + 1;
 constexpr int kOffXchg = kOffBar + kNumBars * 8;   // [3][2 halves][128 rows] fp32: row max (by block
                                                    // parity) and row sum exchange between a row's two threads
 constexpr int kOffTmemPtr = kOffXchg + 3 * 2 * kRows * 4;
@@ -114,6 +115,7 @@ struct Params {
     const int32_t* pos0;
     const int32_t* n_new;
     uint32_t* status;
+    const float4* table;                  // rotary table [T][64] {cos, sin} (fp32), for the fused-RoPE form
     int B, S, T, Hq, Hkv, L;
     float scale_log2;
 };
@@ -223,6 +225,11 @@ __device__ __forceinline__ TilePick pick_tile(const Params& p, int j, int lane, 
 
 }  // namespace pf
 
+// Rope: q arrives unrotated and the softmax warps rotate the Q tile in shared
+// memory (Qwen2 rotate-half at the row's absolute position, the products in
+// double from the bf16 input and the fp32 table, one rounding to bf16: the
+// same values ark_attn_append_rope writes), before the first QK MMA.
+template <bool Rope>
 __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_constant__ pf::Params p) {
     using namespace pf;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -240,7 +247,7 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
     // barrier init and the TMEM allocation overlap the tile search's loads
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNumBars; ++i)
-            mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? kSoftmaxThreads : 1);
+            mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1 || i == kBarQRot) ? kSoftmaxThreads : 1);
         *failed_flag = 0;
         fence_mbar_init();
     }
@@ -320,7 +327,7 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
     } else if (warp == 1) {
         // ================================================= MMA issuer
         // waits are AND-ed over the warp so that the __syncwarp()s below are reached by all lanes
-        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarQ], 0));
+        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[Rope ? kBarQRot : kBarQ], 0));
         auto wait_k = [&](int j) {
             return __all_sync(0xffffffffu, mbar_wait(&bars[kBarKFull + j % kKStages], (j / kKStages) & 1));
         };
@@ -402,6 +409,42 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
         float* xchg = reinterpret_cast<float*>(smem + kOffXchg);   // [half][row]
         float m_ref = -INFINITY, e_sum = 0.f, r_sum = 0.f;         // this half's share of the row sums
         bool ok = true;
+        if constexpr (Rope) {
+            // rotate the Q tile in place: item = (row, 16-byte chunk); the chunk holds dims 8c..8c+7
+            // in the first half and their rotary partners 64 + 8c.. in the second, at the same offset
+            ok = mbar_wait(&bars[kBarQ], 0);
+            if (ok) {
+                for (int it = threadIdx.x - 64; it < kRows * 8; it += kSoftmaxThreads) {
+                    const int rr = it >> 3, cch = it & 7;
+                    if (t0 + (rr >> 3) >= nn) continue;                 // padded rows are never stored
+                    const int pos = p0 + t0 + (rr >> 3);
+                    const uint32_t off = rr * 128 + ((cch ^ (rr & 7)) << 4);
+                    uint4* plo = reinterpret_cast<uint4*>(smem + kOffQ + off);
+                    uint4* phi = reinterpret_cast<uint4*>(smem + kOffQ + kQHalf + off);
+                    const uint4 xlo = *plo, xhi = *phi;
+                    const uint32_t wl[4] = {xlo.x, xlo.y, xlo.z, xlo.w}, wh[4] = {xhi.x, xhi.y, xhi.z, xhi.w};
+                    uint32_t ol[4], oh[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float4 cs = __ldg(p.table + static_cast<size_t>(pos) * 32 + 4 * cch + j);  // pairs 2j, 2j+1
+                        const double c0 = cs.x, s0 = cs.y, c1 = cs.z, s1 = cs.w;
+                        const double a0 = bf16_bits_to_f64(static_cast<uint16_t>(wl[j] & 0xffff));
+                        const double a1 = bf16_bits_to_f64(static_cast<uint16_t>(wl[j] >> 16));
+                        const double h0 = bf16_bits_to_f64(static_cast<uint16_t>(wh[j] & 0xffff));
+                        const double h1 = bf16_bits_to_f64(static_cast<uint16_t>(wh[j] >> 16));
+                        // both products are exact in double, so contraction cannot change the result
+                        ol[j] = static_cast<uint32_t>(f64_to_bf16_rn(a0 * c0 - h0 * s0)) |
+                                (static_cast<uint32_t>(f64_to_bf16_rn(a1 * c1 - h1 * s1)) << 16);
+                        oh[j] = static_cast<uint32_t>(f64_to_bf16_rn(h0 * c0 + a0 * s0)) |
+                                (static_cast<uint32_t>(f64_to_bf16_rn(h1 * c1 + a1 * s1)) << 16);
+                    }
+                    *plo = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+                    *phi = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+                }
+            }
+            fence_proxy_async_smem();                          // the MMA reads the tile through the async proxy
+            mbar_arrive(&bars[kBarQRot]);
+        }
         // Every tcgen05.ld/st below is .sync.aligned: all 32 lanes of the warp
         // execute it together, so all control flow around them is warp-uniform;
         // the loop itself is left by all 256 softmax threads together (its exit
@@ -577,7 +620,7 @@ ark_status prefill_checks(int B, int S, int T, int Hq, int Hkv, int D, float sca
 ark_status launch_prefill(const void* const* q, const void* const* cache_k, const void* const* cache_v,
                           void* const* o, float* const* lse, int l0, int n, const int32_t* pos0,
                           const int32_t* n_new, int B, int S, int T, int Hq, int Hkv, float scale,
-                          uint32_t* d_status, cudaStream_t stream) {
+                          const float* table, uint32_t* d_status, cudaStream_t stream) {
     static thread_local pf::Params prm;
     prm = pf::Params{};
     for (int i = 0; i < n; ++i) {
@@ -597,18 +640,24 @@ ark_status launch_prefill(const void* const* q, const void* const* cache_k, cons
     prm.n_new = n_new;
     prm.status = d_status;
     prm.B = B; prm.S = S; prm.T = T; prm.Hq = Hq; prm.Hkv = Hkv; prm.L = n;
+    prm.table = reinterpret_cast<const float4*>(table);
     prm.scale_log2 = scale * kLog2e;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARK_ERR_CUDA;
     if (!g_prefill_attr[dev]) {
-        if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::kSmemBytes) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 pf::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 pf::kSmemBytes) != cudaSuccess)
             return ARK_ERR_CUDA;
         g_prefill_attr[dev] = true;
     }
     const long long ctas = static_cast<long long>(Hkv) * B * ((S + pf::kPos - 1) / pf::kPos) * n;
     if (ctas >= (1LL << 31)) return ARK_ERR_UNSUPPORTED;
-    prefill_kernel<<<static_cast<unsigned>(ctas), pf::kThreads, pf::kSmemBytes, stream>>>(prm);
+    if (table)
+        prefill_kernel<true><<<static_cast<unsigned>(ctas), pf::kThreads, pf::kSmemBytes, stream>>>(prm);
+    else
+        prefill_kernel<false><<<static_cast<unsigned>(ctas), pf::kThreads, pf::kSmemBytes, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
 }
 
@@ -621,8 +670,8 @@ extern "C" ark_status ark_attn_prefill(const void* q, const void* cache_k, const
     if (!q || !cache_k || !cache_v || !pos0 || !n_new || !o || !lse) return ARK_ERR_INVALID_ARG;
     ark_status st = prefill_checks(B, S, T, Hq, Hkv, D, scale);
     if (st != ARK_OK) return st;
-    return launch_prefill(&q, &cache_k, &cache_v, &o, &lse, 0, 1, pos0, n_new, B, S, T, Hq, Hkv, scale, d_status,
-                          stream);
+    return launch_prefill(&q, &cache_k, &cache_v, &o, &lse, 0, 1, pos0, n_new, B, S, T, Hq, Hkv, scale, nullptr,
+                          d_status, stream);
 }
 
 extern "C" ark_status ark_attn_prefill_layers(int L, const void* const* q, const void* const* cache_k,
@@ -637,9 +686,37 @@ extern "C" ark_status ark_attn_prefill_layers(int L, const void* const* q, const
     if (st != ARK_OK) return st;
     for (int l0 = 0; l0 < L; l0 += pf::kLayersPerLaunch) {
         const int n = (L - l0 < pf::kLayersPerLaunch) ? L - l0 : pf::kLayersPerLaunch;
-        st = launch_prefill(q, cache_k, cache_v, o, lse, l0, n, pos0, n_new, B, S, T, Hq, Hkv, scale, d_status,
-                            stream);
+        st = launch_prefill(q, cache_k, cache_v, o, lse, l0, n, pos0, n_new, B, S, T, Hq, Hkv, scale, nullptr,
+                            d_status, stream);
         if (st != ARK_OK) return st;
     }
     return ARK_OK;
+}
+
+extern "C" ark_status ark_attn_prefill_rope_layers(int L, const void* const* q, const void* const* cache_k,
+                                                   const void* const* cache_v, const int32_t* pos0,
+                                                   const int32_t* n_new, int B, int S, int T, int Hq, int Hkv,
+                                                   int D, float scale, const float* d_table, void* const* o,
+                                                   float* const* lse, uint32_t* d_status, cudaStream_t stream) {
+    if (!q || !cache_k || !cache_v || !pos0 || !n_new || !o || !lse || !d_table) return ARK_ERR_INVALID_ARG;
+    if (L <= 0) return ARK_ERR_INVALID_ARG;
+    if (L > ARK_MAX_LAYERS) return ARK_ERR_UNSUPPORTED;
+    ark_status st = prefill_checks(B, S, T, Hq, Hkv, D, scale);
+    if (st != ARK_OK) return st;
+    if (!aligned16(d_table)) return ARK_ERR_INVALID_ARG;
+    for (int l0 = 0; l0 < L; l0 += pf::kLayersPerLaunch) {
+        const int n = (L - l0 < pf::kLayersPerLaunch) ? L - l0 : pf::kLayersPerLaunch;
+        st = launch_prefill(q, cache_k, cache_v, o, lse, l0, n, pos0, n_new, B, S, T, Hq, Hkv, scale, d_table,
+                            d_status, stream);
+        if (st != ARK_OK) return st;
+    }
+    return ARK_OK;
+}
+
+extern "C" ark_status ark_attn_prefill_rope(const void* q, const void* cache_k, const void* cache_v,
+                                            const int32_t* pos0, const int32_t* n_new, int B, int S, int T, int Hq,
+                                            int Hkv, int D, float scale, const float* d_table, void* o, float* lse,
+                                            uint32_t* d_status, cudaStream_t stream) {
+    return ark_attn_prefill_rope_layers(1, &q, &cache_k, &cache_v, pos0, n_new, B, S, T, Hq, Hkv, D, scale, d_table,
+                                        &o, &lse, d_status, stream);
 }

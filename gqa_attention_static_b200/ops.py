@@ -53,6 +53,10 @@ EXPORTS = (
     "ark_attn_decode_fp8",
     "ark_attn_decode_fp8_layers",
     "ark_attn_prefill_layers",
+    "ark_attn_append_rope_kv",
+    "ark_attn_append_rope_kv_layers",
+    "ark_attn_prefill_rope",
+    "ark_attn_prefill_rope_layers",
 )
 
 
@@ -115,6 +119,15 @@ def load() -> ctypes.CDLL:
     lib.ark_attn_decode_fp8_layers.restype = I
     lib.ark_attn_prefill_layers.argtypes = [I, PP, PP, PP, P, P, I, I, I, I, I, I, ctypes.c_float, PP, PP, P, P]
     lib.ark_attn_prefill_layers.restype = I
+    lib.ark_attn_append_rope_kv.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, P, P]
+    lib.ark_attn_append_rope_kv.restype = I
+    lib.ark_attn_append_rope_kv_layers.argtypes = [I, PP, PP, PP, PP, P, P, I, I, I, I, I, I, P, P, P]
+    lib.ark_attn_append_rope_kv_layers.restype = I
+    lib.ark_attn_prefill_rope.argtypes = [P, P, P, P, P, I, I, I, I, I, I, ctypes.c_float, P, P, P, P, P]
+    lib.ark_attn_prefill_rope.restype = I
+    lib.ark_attn_prefill_rope_layers.argtypes = [I, PP, PP, PP, P, P, I, I, I, I, I, I, ctypes.c_float, P, PP, PP,
+                                                 P, P]
+    lib.ark_attn_prefill_rope_layers.restype = I
     _lib = lib
     return lib
 
@@ -551,3 +564,69 @@ def ark_attn_prefill_layers(q: Sequence[torch.Tensor], cache_k, cache_v, pos0, n
                                           _ptr(n_new), B, S, T, Hq, Hkv, D, float(scale), _ptr_array(o),
                                           _ptr_array(lse), _ptr(status), _stream(stream)),
            "ark_attn_prefill_layers")
+
+
+# -------------------------------------------- prefill with RoPE on load ----
+# The prefill rotates q itself as it loads each tile (the same bf16 values the
+# append writes), so the append only has to write the K/V rows.
+
+def ark_attn_append_rope_kv_layers(k_new: Sequence[torch.Tensor], v_new, cache_k, cache_v, pos0, n_new, table,
+                                   Hq: int = 16, status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """ark_attn_append_rope without the query rows: rotated keys and the
+    values written into the cache at cache_position, L layers in one launch."""
+    L = len(k_new)
+    if not (len(v_new) == len(cache_k) == len(cache_v) == L) or L == 0:
+        raise ValueError("per-layer lists must have the same non-zero length")
+    for i in range(L):
+        for name, t in (("k_new", k_new[i]), ("v_new", v_new[i]), ("cache_k", cache_k[i]), ("cache_v", cache_v[i])):
+            _need(t, name, torch.bfloat16, 4)
+        if k_new[i].shape != k_new[0].shape or v_new[i].shape != k_new[0].shape or \
+                cache_k[i].shape != cache_k[0].shape or cache_v[i].shape != cache_k[0].shape:
+            raise ValueError("all layers must have the same shapes")
+    _need(pos0, "pos0", torch.int32, 1)
+    _need(n_new, "n_new", torch.int32, 1)
+    _need(table, "table", torch.float32)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    B, S, Hkv, D = k_new[0].shape
+    T = cache_k[0].shape[1]
+    if table.numel() < T * (D // 2) * 2:
+        raise ValueError("rotary table has fewer than T rows")
+    _raise(load().ark_attn_append_rope_kv_layers(L, _ptr_array(k_new), _ptr_array(v_new), _ptr_array(cache_k),
+                                                 _ptr_array(cache_v), _ptr(pos0), _ptr(n_new), B, S, T, int(Hq),
+                                                 Hkv, D, _ptr(table), _ptr(status), _stream(stream)),
+           "ark_attn_append_rope_kv_layers")
+
+
+def ark_attn_prefill_rope_layers(q: Sequence[torch.Tensor], cache_k, cache_v, pos0, n_new, o, lse, scale: float,
+                                 table: torch.Tensor, status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """ark_attn_prefill with q given unrotated: each tile is rotated as it is
+    loaded, with the append's arithmetic (q itself is not modified)."""
+    L = len(q)
+    if not (len(cache_k) == len(cache_v) == len(o) == len(lse) == L) or L == 0:
+        raise ValueError("per-layer lists must have the same non-zero length")
+    for i in range(L):
+        _need(q[i], "q", torch.bfloat16, 4)
+        _need(cache_k[i], "cache_k", torch.bfloat16, 4)
+        _need(cache_v[i], "cache_v", torch.bfloat16, 4)
+        _need(o[i], "o", torch.bfloat16, 4)
+        _need(lse[i], "lse", torch.float32, 3)
+        if q[i].shape != q[0].shape or cache_k[i].shape != cache_k[0].shape or cache_v[i].shape != cache_k[0].shape \
+                or o[i].shape != q[0].shape or lse[i].shape != lse[0].shape:
+            raise ValueError("all layers must have the same shapes")
+    _need(pos0, "pos0", torch.int32, 1)
+    _need(n_new, "n_new", torch.int32, 1)
+    _need(table, "table", torch.float32)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    B, S, Hq, D = q[0].shape
+    T, Hkv = cache_k[0].shape[1], cache_k[0].shape[2]
+    if tuple(lse[0].shape) != (B, Hq, S):
+        raise ValueError("lse must be [B, Hq, S]")
+    if table.numel() < T * (D // 2) * 2:
+        raise ValueError("rotary table has fewer than T rows")
+    _raise(load().ark_attn_prefill_rope_layers(L, _ptr_array(q), _ptr_array(cache_k), _ptr_array(cache_v),
+                                               _ptr(pos0), _ptr(n_new), B, S, T, Hq, Hkv, D, float(scale),
+                                               _ptr(table), _ptr_array(o), _ptr_array(lse), _ptr(status),
+                                               _stream(stream)),
+           "ark_attn_prefill_rope_layers")

@@ -136,8 +136,11 @@ class PrefillStep:
     """
 
     def __init__(self, q, k_new, v_new, cache_k, cache_v, pos0, n_new, rope_theta: float = 1e6,
-                 scale: Optional[float] = None, batched: bool = True):
+                 scale: Optional[float] = None, batched: bool = True, fused_rope: bool = False):
         self.batched = batched
+        # fused_rope: the append writes only the K/V rows and the prefill rotates
+        # q as it loads it (q is then left unrotated in memory)
+        self.fused_rope = fused_rope
         self.q, self.k_new, self.v_new = q, k_new, v_new
         self.cache_k, self.cache_v = cache_k, cache_v
         self.pos0, self.n_new = pos0, n_new
@@ -155,10 +158,18 @@ class PrefillStep:
         return 1 + ((self.layers + 15) // 16 if self.batched else self.layers)
 
     def append(self, stream=None) -> None:
+        if self.fused_rope:
+            ops.ark_attn_append_rope_kv_layers(self.k_new, self.v_new, self.cache_k, self.cache_v, self.pos0,
+                                               self.n_new, self.table, self.Hq, self.status, stream)
+            return
         ops.ark_attn_append_rope_layers(self.q, self.k_new, self.v_new, self.cache_k, self.cache_v, self.pos0,
                                         self.n_new, self.table, self.status, stream)
 
     def attention(self, stream=None) -> None:
+        if self.fused_rope:
+            ops.ark_attn_prefill_rope_layers(self.q, self.cache_k, self.cache_v, self.pos0, self.n_new, self.o,
+                                             self.lse, self.scale, self.table, self.status, stream)
+            return
         if self.batched:
             ops.ark_attn_prefill_layers(self.q, self.cache_k, self.cache_v, self.pos0, self.n_new, self.o, self.lse,
                                         self.scale, self.status, stream)

@@ -255,6 +255,36 @@ ARK_API ark_status ark_attn_decode_noalloc(const void* q, const void* cache_k, c
                                            float scale, ark_decode_mode mode, int max_splits, void* o,
                                            float* lse, uint32_t* d_status, cudaStream_t stream);
 
+/* ------------------------------------- prefill with RoPE on the q load ----
+ * The same prefill for a caller that leaves q unrotated:
+ * ark_attn_append_rope_kv(_layers) rotates and writes only the K rows and
+ * copies the V rows into the cache (as ark_attn_append_rope does, q not
+ * touched; the q argument is absent and Hq only sizes the checks), and
+ * ark_attn_prefill_rope(_layers) rotates each q tile as it loads it, with the
+ * append's arithmetic (products in double from the bf16 input and the fp32
+ * table d_table of ark_attn_rope_table_init, one rounding to bf16), so its o
+ * and lse equal those of ark_attn_append_rope + ark_attn_prefill bit for bit.
+ * q is read only.  This saves the append's read and write of every prompt q
+ * row.
+ */
+ARK_API ark_status ark_attn_append_rope_kv(const void* k_new, const void* v_new, void* cache_k, void* cache_v,
+                                           const int32_t* pos0, const int32_t* n_new, int B, int S, int T, int Hq,
+                                           int Hkv, int D, const float* d_table, uint32_t* d_status,
+                                           cudaStream_t stream);
+ARK_API ark_status ark_attn_append_rope_kv_layers(int L, const void* const* k_new, const void* const* v_new,
+                                                  void* const* cache_k, void* const* cache_v, const int32_t* pos0,
+                                                  const int32_t* n_new, int B, int S, int T, int Hq, int Hkv, int D,
+                                                  const float* d_table, uint32_t* d_status, cudaStream_t stream);
+ARK_API ark_status ark_attn_prefill_rope(const void* q, const void* cache_k, const void* cache_v,
+                                         const int32_t* pos0, const int32_t* n_new, int B, int S, int T, int Hq,
+                                         int Hkv, int D, float scale, const float* d_table, void* o, float* lse,
+                                         uint32_t* d_status, cudaStream_t stream);
+ARK_API ark_status ark_attn_prefill_rope_layers(int L, const void* const* q, const void* const* cache_k,
+                                                const void* const* cache_v, const int32_t* pos0,
+                                                const int32_t* n_new, int B, int S, int T, int Hq, int Hkv, int D,
+                                                float scale, const float* d_table, void* const* o,
+                                                float* const* lse, uint32_t* d_status, cudaStream_t stream);
+
 /* ------------------------------------------------------- fp8 KV cache ----
  * A cache of 8-bit codes, half the bytes of the bf16 cache, for the same
  * attention.  The pages quantise weights only (the int8/int4 tiers of the

@@ -181,3 +181,61 @@ def test_prefill_layers_across_launches_equals_single_layer_calls(oracle_lib):
         torch.cuda.synchronize()
         assert torch.equal(o[l].view(torch.int16), o1.view(torch.int16)), f"layer {l}"
         assert torch.equal(torch.nan_to_num(lse[l], nan=-7.0), torch.nan_to_num(l1, nan=-7.0)), f"layer {l}"
+
+
+def _two_paths(batch, L):
+    """(a) append_rope + prefill_layers, (b) append_rope_kv + prefill_rope_layers,
+    on identical inputs; returns both results and the untouched q of (b)."""
+    dev = "cuda"
+    out = []
+    for fused in (False, True):
+        q = [x.to(dev).clone() for x in batch.q[:L]]
+        ck = [x.to(dev).clone() for x in batch.cache_k[:L]]
+        cv = [x.to(dev).clone() for x in batch.cache_v[:L]]
+        pos0, n_new = batch.pos0.to(dev), batch.n_new.to(dev)
+        kn = [x.to(dev) for x in batch.k_new[:L]]
+        vn = [x.to(dev) for x in batch.v_new[:L]]
+        table = ops.rope_table(batch.T)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        B, S, Hq, D = q[0].shape
+        o = [torch.empty_like(x).view(torch.int16).fill_(SENTINEL).view(torch.bfloat16) for x in q]
+        lse = [torch.full((B, Hq, S), float("nan"), dtype=torch.float32, device=dev) for _ in q]
+        if fused:
+            ops.ark_attn_append_rope_kv_layers(kn, vn, ck, cv, pos0, n_new, table, Hq, status)
+            ops.ark_attn_prefill_rope_layers(q, ck, cv, pos0, n_new, o, lse, SCALE, table, status)
+        else:
+            ops.ark_attn_append_rope_layers(q, kn, vn, ck, cv, pos0, n_new, table, status)
+            ops.ark_attn_prefill_layers(q, ck, cv, pos0, n_new, o, lse, SCALE, status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        out.append((q, ck, cv, o, lse))
+    return out
+
+
+@pytest.mark.parametrize("B,S,T,pos0,n_new", [
+    (3, 40, 256, [0, 30, 100], [40, 17, 1]),
+    (1, 5, 8, [3], [5]),
+    (1, 200, 2048, [1700], [200]),
+])
+def test_prefill_rope_on_load_equals_append_then_prefill(oracle_lib, B, S, T, pos0, n_new):
+    """RoPE applied by the prefill as it loads q gives the same o and lse, bit
+    for bit, as rotating q in the append first; the K/V-only append writes the
+    same cache bytes and leaves q untouched."""
+    L = 2
+    batch = W.make_batch(520 + S, B=B, S=S, T=T, pos0=pos0, n_new=n_new, layers=L, garbage="nan")
+    (qa, cka, cva, oa, la), (qb, ckb, cvb, ob, lb) = _two_paths(batch, L)
+    for l in range(L):
+        assert torch.equal(cka[l].view(torch.int16), ckb[l].view(torch.int16))
+        assert torch.equal(cva[l].view(torch.int16), cvb[l].view(torch.int16))
+        assert torch.equal(qb[l].view(torch.int16), batch.q[l].cuda().view(torch.int16))
+        assert torch.equal(oa[l].view(torch.int16), ob[l].view(torch.int16)), f"layer {l}: o differs"
+        assert torch.equal(torch.nan_to_num(la[l], nan=-7.0), torch.nan_to_num(lb[l], nan=-7.0)), f"layer {l}"
+
+
+def test_prefill_rope_on_load_coalesced_full_size(oracle_lib):
+    batch = W.cfg_prefill(layers=2)
+    (qa, cka, cva, oa, la), (qb, ckb, cvb, ob, lb) = _two_paths(batch, 2)
+    for l in range(2):
+        assert torch.equal(oa[l].view(torch.int16), ob[l].view(torch.int16)), f"layer {l}: o differs"
+        assert torch.equal(torch.nan_to_num(la[l], nan=-7.0), torch.nan_to_num(lb[l], nan=-7.0))
+        assert torch.equal(cka[l].view(torch.int16), ckb[l].view(torch.int16))
