@@ -65,7 +65,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="ragged",
-                    choices=["ragged", "single", "long2048", "long1024", "prefill"])
+                    choices=["ragged", "single", "long2048", "long1024", "prefill", "encoder"])
     ap.add_argument("--mode", default="aware", choices=["aware", "masked"])
     ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
                     help="cache format of the decode configurations: bf16, or fp8 E4M3 codes with per-head scales")
@@ -278,9 +278,66 @@ def cpu_baseline(workload: str, seconds: float, mode: str, kv: str = "bf16"):
             "tokens_layers_per_s": r.B * n / el}
 
 
+class EncoderOracleRunner:
+    """The fp64 oracle's encoder attention on this host's cores over a bounded
+    sample: one clip of the encoder batch per step (clips cycled, 4 layers)."""
+
+    def __init__(self, layers: int = 4):
+        import numpy as np
+        import torch
+        cores = os.cpu_count() or 1
+        os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+        import oracle
+        from gqa_attention_static_b200 import workloads as W
+        oracle.build()
+        self.oracle = oracle
+        self.cores = oracle.num_threads()
+        e = W.cfg_encoder(layers=layers)
+        bits = lambda x: x.contiguous().view(torch.int16).numpy().view(np.uint16)
+        self.items = [(bits(e.q[l][b:b + 1]), bits(e.k[l][b:b + 1]), bits(e.v[l][b:b + 1]),
+                       e.length[b:b + 1].numpy()) for l in range(layers) for b in range(e.B)]
+        self.scale = 1.0 / math.sqrt(W.ENC_HEAD_DIM)
+        self.i = 0
+        self.flops = 0
+
+    def step(self):
+        q, k, v, n = self.items[self.i % len(self.items)]
+        self.i += 1
+        self.oracle.attention_bidir(q, k, v, n, self.scale)
+        self.flops += encoder_flops(n.tolist())
+
+
+def run_reference_encoder(args):
+    r = EncoderOracleRunner()
+    r.step()
+    r.flops = 0
+    for _ in range(max(0, args.warmup - 1)):
+        r.step()
+    r.flops = 0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r.step()
+    el = time.perf_counter() - t0
+    v = r.flops / el / 1e12
+    sample = (f"each step = encoder attention of ONE clip (all 20 heads) of one layer of the encoder batch "
+              f"(8 clips x 4 layers cycled); fp64 oracle; TFLOP/s by the GPU line's FLOP count")
+    line = {"impl": "reference", "metric": "encoder attention TFLOP/s (1xB200); % of bf16 tensor roofline",
+            "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "encoder attention B=8 clips of 150..1500 frames (S=1500), 20 heads x 64, "
+                                   "32 layers"},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": r.cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
+        return
+    if args.config == "encoder":
+        run_reference_encoder(args)
         return
     r = OracleRunner(args.config, args.mode, kv=args.kv)
     for _ in range(max(1, args.warmup)):
@@ -411,6 +468,85 @@ def run_prefill(args):
         print(json.dumps(line), flush=True)
 
 
+def encoder_flops(lengths, H: int = 20, D: int = 64) -> int:
+    """Encoder attention per layer: 4 * D FLOPs per (query frame, key frame)
+    pair of a clip (QK^T and PV), len^2 pairs per clip and head."""
+    return sum(4 * D * H * int(n) * int(n) for n in lengths)
+
+
+def run_encoder(args):
+    """The audio encoder's bidirectional attention: 8 clips of 3..30 s (150..1500
+    frames, padded to 1500), 20 heads of 64 dims, 32 layers; a step is the
+    attention of all 32 layers (one launch each), replayed from a CUDA graph."""
+    import torch
+    from gqa_attention_static_b200 import ops
+    from gqa_attention_static_b200 import workloads as W
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+    ops.load()
+    e = W.cfg_encoder()
+    L = len(e.q)
+    q = [x.to(dev) for x in e.q]
+    k = [x.to(dev) for x in e.k]
+    v = [x.to(dev) for x in e.v]
+    length = e.length.to(dev)
+    o = [torch.empty_like(x) for x in q]
+    lse = [torch.empty((e.B, x.shape[2], e.S), dtype=torch.float32, device=dev) for x in q]
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(W.ENC_HEAD_DIM)
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+
+    def step():
+        for l in range(L):
+            ops.ark_attn_encoder(q[l], k[l], v[l], length, o[l], lse[l], scale, status, stream=s)
+
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    torch.cuda.synchronize()
+    for _ in range(max(3, args.warmup)):
+        g.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        e0.record(s)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms_step = e0.elapsed_time(e1) / args.steps
+    if int(status.item()) != 0:
+        print(f"device status word set: {int(status.item())}", file=sys.stderr)
+    nf = encoder_flops(e.length.tolist())
+    tc, tc_kind = measured_tensor_peak()
+    ms_launch = ms_step / L
+    achieved = nf / (ms_launch * 1e-3) / 1e12
+    roof = {"kernel": "encoder_attn_kernel (ark_attn_encoder, one layer per launch)", "bound": "tensor",
+            "achieved": achieved, "peak": tc, "unit": "TFLOP/s", "frac": achieved / tc, "peak_kind": tc_kind,
+            "traffic": None, "launch_ms": ms_launch, "flops_per_launch": nf}
+    value = achieved
+    line = {"metric": "encoder attention TFLOP/s (1xB200); % of bf16 tensor roofline", "value": value,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "encoder attention B=8 clips of 150..1500 frames (S=1500), 20 heads x 64, "
+                                   "32 layers", "lengths": e.length.tolist(),
+                       "l2": "q/k/v/o of 32 layers (3.9 GB) larger than L2"},
+            "roofline": roof, "gpu_launches": L * args.steps, "clocks": clk}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -418,6 +554,9 @@ def main():
         return
     if args.config == "prefill":
         run_prefill(args)
+        return
+    if args.config == "encoder":
+        run_encoder(args)
         return
     import torch
     import torch.distributed as dist

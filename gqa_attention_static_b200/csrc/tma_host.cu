@@ -96,6 +96,14 @@ bool kv8_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv,
     return cached_encode(key, out, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8);
 }
 
+bool hd64_tensor_map(CUtensorMap* out, const void* base, long long rows, int H, int box_rows) {
+    const Key key{reinterpret_cast<uintptr_t>(base), rows, 4, H, 64, box_rows};
+    const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(H) * 128};
+    const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+    return cached_encode(key, out, 3, dims, strides, box);
+}
+
 bool q_group_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hq, int box_inner, int box_rows) {
     const Key key{reinterpret_cast<uintptr_t>(base), rows, 2, Hq, box_inner, box_rows};
     const cuuint64_t dims[4] = {128, 8, static_cast<cuuint64_t>(Hq / 8), static_cast<cuuint64_t>(rows)};

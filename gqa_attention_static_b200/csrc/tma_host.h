@@ -19,6 +19,10 @@ bool kv_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv, 
 // dims (128, Hkv, rows), box (128, 1, box_rows), 128-byte swizzle.
 bool kv8_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv, int box_rows);
 
+// [rows][H][64] bf16 (heads of 64 dims): dims (64, H, rows), box (64, 1, box_rows),
+// 128-byte swizzle.
+bool hd64_tensor_map(CUtensorMap* out, const void* base, long long rows, int H, int box_rows);
+
 bool rows_tensor_map(CUtensorMap* out, const void* base, long long rows, int box_inner, int box_rows);
 
 // 4-D tiled map over q [B, S, Hq, 128] bf16 viewed as (dim 0: 128 head-dim

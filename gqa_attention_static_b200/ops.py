@@ -57,6 +57,7 @@ EXPORTS = (
     "ark_attn_append_rope_kv_layers",
     "ark_attn_prefill_rope",
     "ark_attn_prefill_rope_layers",
+    "ark_attn_encoder",
 )
 
 
@@ -128,6 +129,8 @@ def load() -> ctypes.CDLL:
     lib.ark_attn_prefill_rope_layers.argtypes = [I, PP, PP, PP, P, P, I, I, I, I, I, I, ctypes.c_float, P, PP, PP,
                                                  P, P]
     lib.ark_attn_prefill_rope_layers.restype = I
+    lib.ark_attn_encoder.argtypes = [P, P, P, P, I, I, I, I, ctypes.c_float, P, P, P, P]
+    lib.ark_attn_encoder.restype = I
     _lib = lib
     return lib
 
@@ -630,3 +633,23 @@ def ark_attn_prefill_rope_layers(q: Sequence[torch.Tensor], cache_k, cache_v, po
                                                _ptr(table), _ptr_array(o), _ptr_array(lse), _ptr(status),
                                                _stream(stream)),
            "ark_attn_prefill_rope_layers")
+
+
+# ------------------------------------------------------ encoder attention ----
+
+def ark_attn_encoder(q, k, v, length, o, lse, scale: float, status: Optional[torch.Tensor] = None,
+                     stream=None) -> None:
+    """Bidirectional multi-head attention of the audio encoder: q, k, v, o
+    [B,S,H,64] bf16, length int32[B], lse [B,H,S] fp32."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _need(t, name, torch.bfloat16, 4)
+    _need(length, "len", torch.int32, 1)
+    _need(lse, "lse", torch.float32, 3)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    B, S, H, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape or o.shape != q.shape or tuple(lse.shape) != (B, H, S):
+        raise ValueError("shapes")
+    _raise(load().ark_attn_encoder(_ptr(q), _ptr(k), _ptr(v), _ptr(length), B, S, H, D, float(scale), _ptr(o),
+                                   _ptr(lse), _ptr(status), _stream(stream)),
+           "ark_attn_encoder")

@@ -274,3 +274,61 @@ def make_fp8_cache(seed: int, B: int, T: int, valid, layers: int = 1, garbage: s
         out.k_scale.append((0.02 + 0.18 * torch.rand(Hkv, generator=g)).float())
         out.v_scale.append((0.02 + 0.18 * torch.rand(Hkv, generator=g)).float())
     return out
+
+
+# ------------------------------------------------------- encoder batches ----
+# The audio encoder's attention: clips of 3..30 s at 16 kHz, 50 encoder frames
+# per second after the stride-2 convolution (1500 frames at the 30-second
+# Whisper boundary), encoded 8 at a time (SGLang-Omni cookbook "ARK-ASR-3B",
+# audio handling: 30 s truncation, encoder_max_batch_size 8); heads of the
+# 1280-wide Whisper-large geometry (20 x 64).
+
+ENC_HEADS = 20
+ENC_HEAD_DIM = 64
+ENC_LAYERS = 32
+
+
+def encoder_frames(seconds: float) -> int:
+    """Encoder frames of a clip: 100 mel frames per second, halved by the
+    stride-2 convolution, at most 1500."""
+    return max(1, min(1500, int(seconds * 100) // 2))
+
+
+@dataclass
+class EncoderBatch:
+    q: List[torch.Tensor]          # per layer [B, S, H, D] bf16
+    k: List[torch.Tensor]
+    v: List[torch.Tensor]
+    length: torch.Tensor           # int32 [B]
+
+    @property
+    def B(self) -> int:
+        return self.q[0].shape[0]
+
+    @property
+    def S(self) -> int:
+        return self.q[0].shape[1]
+
+
+def make_encoder_batch(seed: int, B: int, S: int, lengths, H: int = ENC_HEADS, D: int = ENC_HEAD_DIM,
+                       layers: int = 1, garbage: str = "nan") -> EncoderBatch:
+    """bf16 N(0,1) q/k/v per layer; frames past each clip's length hold
+    garbage ("nan": NaN/inf, "big": +-1e4, "none": N(0,1))."""
+    g = _gen(seed)
+    length = torch.as_tensor(lengths, dtype=torch.int32).view(B)
+    out = EncoderBatch([], [], [], length)
+    for _ in range(layers):
+        for lst in (out.q, out.k, out.v):
+            x = randn_bf16((B, S, H, D), g)
+            if garbage != "none":
+                fill_garbage_(x, length, g, garbage)
+            lst.append(x.contiguous())
+    return out
+
+
+def cfg_encoder(seed: int = 6, layers: int = ENC_LAYERS, B: int = 8) -> EncoderBatch:
+    """8 clips of 3..30 s (150..1500 frames), padded to 1500."""
+    g = _gen(seed)
+    secs = 3.0 + 27.0 * torch.rand(B, generator=g)
+    lengths = [encoder_frames(float(s)) for s in secs]
+    return make_encoder_batch(seed + 1, B, 1500, lengths, layers=layers)

@@ -333,6 +333,26 @@ ARK_API ark_status ark_attn_decode_fp8_layers(int L, const void* const* q, const
                                               void* const* o, float* const* lse, uint32_t* d_status,
                                               cudaStream_t stream);
 
+/* --------------------------------------------------- encoder attention ----
+ * Bidirectional multi-head self-attention of the audio encoder.  The pages
+ * describe a Whisper-style audio tower with rotary self-attention whose output
+ * is 1280 wide ("ARK-ASR-3B -- INT8 ONNX", Inference step 1; "Inside
+ * ARK-ASR-3B's Whisper and Qwen architecture", components) but give neither its
+ * head count nor its rotary parameters; the reading taken is the Whisper-large
+ * geometry of a 1280-wide model, H heads of D = 64 (H = 20), with q and k
+ * already rotated.  For clip b, head h and frame i < len[b]:
+ *   o[b,i,h,:] = sum_{j < len[b]} softmax_j(scale <q[b,i,h,:], k[b,j,h,:]>) v[b,j,h,:]
+ *   lse[b,h,i] = ln sum_{j < len[b]} exp(scale <q[b,i,h,:], k[b,j,h,:]>)
+ * Layouts: q, k, v [B,S,H,D] bf16 (16-byte aligned); len int32[B] (device);
+ * o [B,S,H,D] bf16; lse [B,H,S] fp32.  Rows i >= len[b] are not written; len
+ * outside [0, S] is clamped and sets ARK_DEV_BAD_KVLEN.  D != 64 returns
+ * ARK_ERR_UNSUPPORTED.  tcgen05 MMAs (bf16 operands, fp32 accumulation in
+ * tensor memory); the softmax weights are rounded to bf16 before P V.
+ */
+ARK_API ark_status ark_attn_encoder(const void* q, const void* k, const void* v, const int32_t* len, int B, int S,
+                                    int H, int D, float scale, void* o, float* lse, uint32_t* d_status,
+                                    cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

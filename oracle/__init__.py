@@ -74,6 +74,8 @@ def _load():
         lib.ora_append_rope_fp8.restype = I
         lib.ora_attention_fp8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, ctypes.c_double, I, P, P]
         lib.ora_attention_fp8.restype = None
+        lib.ora_attention_bidir.argtypes = [P, P, P, P, I, I, I, I, ctypes.c_double, P, P]
+        lib.ora_attention_bidir.restype = None
         _lib = lib
     return _lib
 
@@ -324,3 +326,22 @@ def decode_fp8(q, cache_k, cache_v, k_scale, v_scale, kv_len, scale: float, stat
     o, lse = attention_fp8(q, cache_k, cache_v, k_scale, v_scale, kv_len, np.ones(B, dtype=np.int32),
                            scale, static_mode)
     return o, lse[:, :, 0]
+
+
+# ------------------------------------------------------ encoder attention ----
+
+def attention_bidir(q, k, v, length, scale: float):
+    """Bidirectional multi-head attention of the audio encoder: row i < len[b]
+    of clip b and head h attends to rows j < len[b] of the same clip and head.
+    q, k, v [B,S,H,D] uint16 (bf16 bits).  Returns o [B,S,H,D] float64 and lse
+    [B,H,S] float64, NaN for rows i >= len[b]."""
+    lib = _load()
+    q = _c(q, np.uint16)
+    k = _c(k, np.uint16)
+    v = _c(v, np.uint16)
+    ln = _c(length, np.int32)
+    B, S, H, D = q.shape
+    o = np.full((B, S, H, D), np.nan, dtype=np.float64)
+    lse = np.full((B, H, S), np.nan, dtype=np.float64)
+    lib.ora_attention_bidir(_ptr(q), _ptr(k), _ptr(v), _ptr(ln), B, S, H, D, float(scale), _ptr(o), _ptr(lse))
+    return o, lse

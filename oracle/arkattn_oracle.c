@@ -501,3 +501,33 @@ void ora_attention_fp8(const uint16_t* q, const uint8_t* cache_k, const uint8_t*
         }
     }
 }
+
+/* ------------------------------------------------- encoder attention ---- */
+/*
+ * Bidirectional multi-head self-attention of the audio encoder (the pages
+ * give a Whisper-style encoder with rotary self-attention and a 1280-wide
+ * output; reading: every frame of a clip attends to every frame of the same
+ * clip, q and k already rotated).  Layouts: q, k, v [B, S, H, D] (bf16 bits),
+ * len[B] valid frames per clip; o [B, S, H, D] double, lse [B, H, S] double;
+ * rows i >= len[b] are not written.  Each (b, h, i) is ora_attend_one over the
+ * clip's rows [0, len[b]) of head h.
+ */
+void ora_attention_bidir(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* len,
+                         int B, int S, int H, int D, double scale, double* o, double* lse) {
+    long row_stride = (long)H * D;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            int n = len[b];
+            if (n < 0) n = 0;
+            if (n > S) n = S;
+            const uint16_t* kb = k + ((size_t)b * S * H + h) * D;
+            const uint16_t* vb = v + ((size_t)b * S * H + h) * D;
+            for (int i = 0; i < n; ++i) {
+                const uint16_t* qrow = q + (((size_t)b * S + i) * H + h) * D;
+                ora_attend_one(qrow, kb, vb, row_stride, 0, n, D, scale,
+                               o + (((size_t)b * S + i) * H + h) * D, lse + ((size_t)b * H + h) * S + i);
+            }
+        }
+    }
+}

@@ -124,3 +124,17 @@ def test_binding_refuses_cpu_tensors(lib):
     q = torch.zeros(1, 1, 16, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         ops.ark_attn_decode(q, q, q, torch.zeros(1, dtype=torch.int32), q, torch.zeros(16), 0.1)
+
+
+def test_encoder_arg_checks(lib):
+    def enc(q=FAKE, k=FAKE, v=FAKE, ln=FAKE, B=2, S=100, H=20, D=64, scale=0.125, o=FAKE, lse=FAKE):
+        return lib.ark_attn_encoder(q, k, v, ln, B, S, H, D, scale, o, lse, None, None)
+    assert enc(q=None) == ops.ARK_ERR_INVALID_ARG
+    assert enc(lse=None) == ops.ARK_ERR_INVALID_ARG
+    assert enc(B=0) == ops.ARK_ERR_INVALID_ARG
+    assert enc(S=-3) == ops.ARK_ERR_INVALID_ARG
+    assert enc(scale=0.0) == ops.ARK_ERR_INVALID_ARG
+    assert enc(D=128) == ops.ARK_ERR_UNSUPPORTED
+    assert enc(H=70000) == ops.ARK_ERR_UNSUPPORTED
+    assert enc(v=FAKE_MIS) == ops.ARK_ERR_INVALID_ARG
+    assert enc(lse=FAKE + 2) == ops.ARK_ERR_INVALID_ARG

@@ -546,3 +546,48 @@ def test_fp8_attention_equals_bf16_attention_of_dequantised_cache(oracle_lib):
     o8g, l8g = oracle.decode_fp8(q, garbage_k, garbage_v, ks, vs, kv, 0.0884)
     o8, l8 = oracle.decode_fp8(q, codes_k, codes_v, ks, vs, kv, 0.0884)
     assert np.array_equal(o8g, o8) and np.array_equal(l8g, l8)
+
+
+# ------------------------------------------------------ encoder attention ----
+
+def test_encoder_attention_matches_torch_sdpa_fp64(oracle_lib):
+    """Bidirectional multi-head attention per clip against torch's SDPA in
+    fp64 (no mask inside the clip's length), and against a pure-Python loop on
+    one row."""
+    B, S, H, D = 3, 20, 4, 64
+    q = rand_bits((B, S, H, D), 60)
+    k = rand_bits((B, S, H, D), 61)
+    v = rand_bits((B, S, H, D), 62)
+    length = np.array([20, 7, 1], np.int32)
+    scale = 1 / 8.0
+    o, lse = oracle.attention_bidir(q, k, v, length, scale)
+    qd, kd, vd = (torch.from_numpy(oracle.bf16_array_to_f64(x)) for x in (q, k, v))
+    for b in range(B):
+        n = int(length[b])
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            qd[b, :n].transpose(0, 1), kd[b, :n].transpose(0, 1), vd[b, :n].transpose(0, 1), scale=scale)
+        assert np.allclose(o[b, :n], ref.transpose(0, 1).numpy(), rtol=1e-12, atol=1e-12)
+        assert np.all(np.isnan(o[b, n:])) and np.all(np.isnan(lse[b, :, n:]))
+    b, i, h = 1, 3, 2
+    n = int(length[b])
+    s = [scale * sum(float(qd[b, i, h, d]) * float(kd[b, j, h, d]) for d in range(D)) for j in range(n)]
+    m = max(s)
+    w = [math.exp(x - m) for x in s]
+    l = sum(w)
+    assert abs(lse[b, h, i] - (m + math.log(l))) < 1e-12
+    for d in (0, 31, 63):
+        assert abs(o[b, i, h, d] - sum(w[j] * float(vd[b, j, h, d]) for j in range(n)) / l) < 1e-12
+
+
+def test_encoder_attention_ignores_frames_past_length(oracle_lib):
+    B, S, H, D = 2, 16, 2, 64
+    q = rand_bits((B, S, H, D), 63)
+    k = rand_bits((B, S, H, D), 64)
+    v = rand_bits((B, S, H, D), 65)
+    length = np.array([9, 16], np.int32)
+    o, lse = oracle.attention_bidir(q, k, v, length, 0.125)
+    k2, v2 = k.copy(), v.copy()
+    k2[0, 9:] = 0x7FC0           # NaN
+    v2[0, 9:] = 0x7F80           # +inf
+    o2, lse2 = oracle.attention_bidir(q, k2, v2, length, 0.125)
+    assert np.array_equal(o[0, :9], o2[0, :9]) and np.array_equal(lse[0, :, :9], lse2[0, :, :9])
