@@ -74,6 +74,8 @@ def parse():
                     help="issue the single-layer calls layer by layer instead of the layer-batched calls")
     ap.add_argument("--rope-on-load", action="store_true",
                     help="prefill: K/V-only append, RoPE applied by the prefill kernel as it loads q")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="encoder: layers per step (default 32; fewer only for profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -486,7 +488,7 @@ def run_encoder(args):
     torch.cuda.set_device(local)
     dev = f"cuda:{local}"
     ops.load()
-    e = W.cfg_encoder()
+    e = W.cfg_encoder(layers=args.layers or W.ENC_LAYERS)
     L = len(e.q)
     q = [x.to(dev) for x in e.q]
     k = [x.to(dev) for x in e.k]
@@ -540,7 +542,7 @@ def run_encoder(args):
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "encoder attention B=8 clips of 150..1500 frames (S=1500), 20 heads x 64, "
-                                   "32 layers", "lengths": e.length.tolist(),
+                                   f"{L} layers", "lengths": e.length.tolist(),
                        "l2": "q/k/v/o of 32 layers (3.9 GB) larger than L2"},
             "roofline": roof, "gpu_launches": L * args.steps, "clocks": clk}
     if rank == 0:

@@ -83,7 +83,8 @@ constexpr int kBarSFull = kBarVEmpty + kVStages;   // 2
 constexpr int kBarPFull = kBarSFull + 2;           // 2
 constexpr int kBarPvDone = kBarPFull + 2;
 constexpr int kBarQRot = kBarPvDone + 1;           // rotated Q tile in place (count: softmax threads)
-constexpr int kNumBars = kBarQRot + 1;
+constexpr int kBarODone = kBarQRot + 1;            // every MMA of the tile done (one phase)
+constexpr int kNumBars = kBarODone + 1;
 constexpr int kOffXchg = kOffBar + kNumBars * 8;   // [3][2 halves][128 rows] fp32: row max (by block
                                                    // parity) and row sum exchange between a row's two threads
 constexpr int kOffTmemPtr = kOffXchg + 3 * 2 * kRows * 4;
@@ -393,6 +394,8 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
             if (!(ok = wait_v(j))) break;
             issue_pv(j);
         }
+        if (ok && lane == 0) umma_commit(&bars[kBarODone]);
+        __syncwarp();
         if (!ok && lane == 0) {
             atomicExch(failed_flag, 1);
             report(p.status, ARK_DEV_TIMEOUT);
@@ -524,7 +527,9 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
             tc_fence_before();
             mbar_arrive(&bars[kBarPFull + (j & 1)]);
         }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPvDone], (nblk - 1) & 1));
+        // O is complete once every MMA of the tile is (a barrier of its own: the per-block one
+        // may still be a phase short of PV(nblk-2) here, and its parity would not tell)
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarODone], 0));
         tc_fence_after();
         // the row sums of both halves (every softmax thread reaches these barriers)
         float* xs = xchg + 2 * 2 * kRows;
@@ -585,7 +590,7 @@ __global__ void __launch_bounds__(pf::kThreads, 2) prefill_kernel(const __grid_c
             // do not release shared or tensor memory under copies or MMAs still in flight
             for (int s = 0; s < kKStages; ++s) (void)mbar_wait(&bars[kBarKFull + s], 0);
             for (int s = 0; s < kVStages; ++s) (void)mbar_wait(&bars[kBarVFull + s], 0);
-            (void)mbar_wait(&bars[kBarPvDone], (nblk - 1) & 1);
+            (void)mbar_wait(&bars[kBarODone], 0);
         }
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
