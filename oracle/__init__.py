@@ -75,6 +75,8 @@ def _load():
         lib.ora_attention_fp8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, ctypes.c_double, I, P, P]
         lib.ora_attention_fp8.restype = None
         lib.ora_attention_bidir.argtypes = [P, P, P, P, I, I, I, I, ctypes.c_double, P, P]
+        lib.ora_qkv_proj.argtypes = [P, P, P, I, I, I, P]
+        lib.ora_qkv_proj.restype = None
         lib.ora_attention_bidir.restype = None
         _lib = lib
     return _lib
@@ -345,3 +347,38 @@ def attention_bidir(q, k, v, length, scale: float):
     lse = np.full((B, H, S), np.nan, dtype=np.float64)
     lib.ora_attention_bidir(_ptr(q), _ptr(k), _ptr(v), _ptr(ln), B, S, H, D, float(scale), _ptr(o), _ptr(lse))
     return o, lse
+
+
+# ------------------------------------------------------ Q/K/V projection ----
+
+def qkv_proj(x, w, bias=None):
+    """The Q/K/V projections of a decoder layer as one Linear over the
+    concatenated weight [Wq; Wk; Wv] ("ARK-ASR-3B -- INT8 ONNX", model card:
+    Q/K/V projections of the Qwen2 decoder, hidden 2048): x [M, K], w [N, K],
+    bias [N] or None (bf16 bits) -> out [M, N] bf16 bits, each the bf16 rounding
+    of the double-precision sum plus bias."""
+    lib = _load()
+    x = _c(x, np.uint16)
+    w = _c(w, np.uint16)
+    M, K = x.shape
+    N = w.shape[0]
+    assert w.shape[1] == K
+    b = None if bias is None else _c(bias, np.uint16)
+    out = np.zeros((M, N), dtype=np.uint16)
+    lib.ora_qkv_proj(_ptr(x), _ptr(w), None if b is None else _ptr(b), M, K, N, _ptr(out))
+    return out
+
+
+def qkv_rope_append(x, w, bias, cache_k, cache_v, pos0, n_new, Hq: int, Hkv: int, D: int = 128,
+                    theta: float = 1e6):
+    """The projection step in front of the attention, then RoPE and the delta
+    write: x [B, S, K] token rows; q, k, v = the three column blocks of
+    qkv_proj(x); then append_rope.  Returns (q_rot [B,S,Hq,D], cache_k,
+    cache_v, skipped)."""
+    x = _c(x, np.uint16)
+    B, S, K = x.shape
+    out = qkv_proj(x.reshape(B * S, K), w, bias)
+    q = out[:, :Hq * D].reshape(B, S, Hq, D)
+    k = out[:, Hq * D:(Hq + Hkv) * D].reshape(B, S, Hkv, D)
+    v = out[:, (Hq + Hkv) * D:].reshape(B, S, Hkv, D)
+    return append_rope(q, k, v, cache_k, cache_v, pos0, n_new, theta)

@@ -531,3 +531,32 @@ void ora_attention_bidir(const uint16_t* q, const uint16_t* k, const uint16_t* v
         }
     }
 }
+
+/* ------------------------------------------- Q/K/V projection (Linear) ---- */
+/*
+ * The Q/K/V projections of a Qwen2 decoder layer, the step in front of the
+ * attention: three dense layers hidden -> Hq*D, Hkv*D, Hkv*D
+ * ("ARK-ASR-3B -- INT8 ONNX", model card: Q/K/V projections of the Qwen2
+ * decoder, hidden 2048).  Written as one Linear over the concatenated weight
+ * W = [Wq; Wk; Wv] of shape [N, K] (N = (Hq + 2 Hkv) * D, K = hidden):
+ *   out[m, n] = bf16_rne( sum_k x[m, k] * W[n, k] + bias[n] )
+ * Reading for precision (the pages give bf16 serving, nothing finer): the
+ * products of two bf16 values are exact in double; the sum is taken in double
+ * in k order, the bias (bf16, may be absent) added in double, and the result
+ * rounded once to bf16 -- the bf16 value of the exact Linear output up to the
+ * double rounding of the sum.
+ * Layouts: x [M, K], W [N, K], bias [N] or NULL (bf16 bits); out [M, N].
+ */
+void ora_qkv_proj(const uint16_t* x, const uint16_t* w, const uint16_t* bias, int M, int K, int N,
+                  uint16_t* out) {
+#pragma omp parallel for schedule(static)
+    for (int m = 0; m < M; ++m) {
+        for (int n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int k = 0; k < K; ++k)
+                acc += ora_bf16_to_f64(x[(size_t)m * K + k]) * ora_bf16_to_f64(w[(size_t)n * K + k]);
+            if (bias) acc += ora_bf16_to_f64(bias[n]);
+            out[(size_t)m * N + n] = ora_f64_to_bf16_rne(acc);
+        }
+    }
+}

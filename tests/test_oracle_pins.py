@@ -591,3 +591,83 @@ def test_encoder_attention_ignores_frames_past_length(oracle_lib):
     v2[0, 9:] = 0x7F80           # +inf
     o2, lse2 = oracle.attention_bidir(q, k2, v2, length, 0.125)
     assert np.array_equal(o[0, :9], o2[0, :9]) and np.array_equal(lse[0, :, :9], lse2[0, :, :9])
+
+
+# ------------------------------------------------------ Q/K/V projection ----
+
+def _bf16_value(bits):
+    """Exact value of a bf16 bit pattern as a Fraction (no float arithmetic)."""
+    from fractions import Fraction
+    b = int(bits)
+    sign = -1 if b >> 15 else 1
+    e = (b >> 7) & 0xFF
+    m = b & 0x7F
+    assert e != 0xFF
+    if e == 0:
+        return sign * Fraction(m, 1 << 7) * Fraction(1, 1 << 126)
+    return sign * (1 + Fraction(m, 1 << 7)) * (Fraction(2) ** (e - 127))
+
+
+def _bf16_round_exact(v):
+    """Nearest bf16 to the rational v, ties to even mantissa, by exact
+    comparison among the candidates around float(v)."""
+    import struct
+    f = float(v)
+    u = struct.unpack("<I", struct.pack("<f", f))[0] >> 16 if f == f else 0x7FC0
+    cands = set()
+    for d in range(-3, 4):
+        c = (u + d) & 0xFFFF
+        if ((c >> 7) & 0xFF) != 0xFF:
+            cands.add(c)
+    best = min(cands, key=lambda c: (abs(_bf16_value(c) - v), c & 1))
+    return best
+
+
+def test_qkv_proj_matches_exact_rational_sum():
+    """Every output of a small Linear equals the bf16 nearest to the exact
+    rational sum + bias (brute force in Fractions, independent rounding)."""
+    rng = np.random.default_rng(5)
+    M, K, N = 3, 37, 5
+    x = oracle.f64_to_bf16(rng.standard_normal((M, K)))
+    w = oracle.f64_to_bf16(rng.standard_normal((N, K)) * 0.3)
+    b = oracle.f64_to_bf16(rng.standard_normal(N))
+    got = oracle.qkv_proj(x, w, b)
+    got_nb = oracle.qkv_proj(x, w, None)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(_bf16_value(x[m, k]) * _bf16_value(w[n, k]) for k in range(K))
+            assert got_nb[m, n] == _bf16_round_exact(exact), (m, n)
+            assert got[m, n] == _bf16_round_exact(exact + _bf16_value(b[n])), (m, n)
+
+
+def test_qkv_proj_selection_matrix_copies_inputs():
+    """W[n, k] = [k == perm[n]] selects input columns: out[m, n] is x[m, perm[n]]
+    bit for bit (fixes the operand orientation and the indexing)."""
+    rng = np.random.default_rng(6)
+    M, K = 4, 64
+    x = oracle.f64_to_bf16(rng.standard_normal((M, K)))
+    perm = rng.permutation(K)[:40]
+    w = np.zeros((40, K), dtype=np.uint16)
+    w[np.arange(40), perm] = 0x3F80           # 1.0
+    assert np.array_equal(oracle.qkv_proj(x, w), x[:, perm])
+
+
+def test_qkv_rope_append_splits_columns_q_k_v():
+    """With W the identity the projection is the input itself, so the fused
+    step equals RoPE + delta write of the input's three column blocks
+    (q: heads 0..Hq-1, then k, then v)."""
+    rng = np.random.default_rng(7)
+    Hq, Hkv, D, B, S, T = 2, 1, 128, 2, 3, 16
+    N = (Hq + 2 * Hkv) * D
+    x = oracle.f64_to_bf16(rng.standard_normal((B, S, N)))
+    w = np.zeros((N, N), dtype=np.uint16)
+    w[np.arange(N), np.arange(N)] = 0x3F80
+    ck = oracle.f64_to_bf16(rng.standard_normal((B, T, Hkv, D)))
+    cv = oracle.f64_to_bf16(rng.standard_normal((B, T, Hkv, D)))
+    pos0, n_new = np.array([0, 9], np.int32), np.array([3, 2], np.int32)
+    got = oracle.qkv_rope_append(x, w, None, ck, cv, pos0, n_new, Hq, Hkv, D)
+    want = oracle.append_rope(x[:, :, :Hq * D].reshape(B, S, Hq, D),
+                              x[:, :, Hq * D:(Hq + Hkv) * D].reshape(B, S, Hkv, D),
+                              x[:, :, (Hq + Hkv) * D:].reshape(B, S, Hkv, D), ck, cv, pos0, n_new)
+    for a, b_ in zip(got[:3], want[:3]):
+        assert np.array_equal(a, b_)
