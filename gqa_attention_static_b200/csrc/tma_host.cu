@@ -112,6 +112,14 @@ bool q_group_tensor_map(CUtensorMap* out, const void* base, long long rows, int 
     return cached_encode(key, out, 4, dims, strides, box);
 }
 
+bool kmajor_tensor_map(CUtensorMap* out, const void* base, long long rows, int K, int box_rows) {
+    const Key key{reinterpret_cast<uintptr_t>(base), rows, 5, K, 64, box_rows};
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    return cached_encode(key, out, 2, dims, strides, box);
+}
+
 bool rows_tensor_map(CUtensorMap* out, const void* base, long long rows, int box_inner, int box_rows) {
     const Key key{reinterpret_cast<uintptr_t>(base), rows, 1, 0, box_inner, box_rows};
     const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};

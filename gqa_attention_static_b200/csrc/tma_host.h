@@ -23,6 +23,10 @@ bool kv8_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv,
 // 128-byte swizzle.
 bool hd64_tensor_map(CUtensorMap* out, const void* base, long long rows, int H, int box_rows);
 
+// [rows][K] bf16, K contiguous (a K-major GEMM operand): dims (K, rows), box
+// (64, box_rows), 128-byte swizzle.  K * 2 bytes must be a multiple of 16.
+bool kmajor_tensor_map(CUtensorMap* out, const void* base, long long rows, int K, int box_rows);
+
 bool rows_tensor_map(CUtensorMap* out, const void* base, long long rows, int box_inner, int box_rows);
 
 // 4-D tiled map over q [B, S, Hq, 128] bf16 viewed as (dim 0: 128 head-dim

@@ -58,6 +58,8 @@ EXPORTS = (
     "ark_attn_prefill_rope",
     "ark_attn_prefill_rope_layers",
     "ark_attn_encoder",
+    "ark_attn_qkv_proj",
+    "ark_attn_qkv_rope_append",
 )
 
 
@@ -131,6 +133,10 @@ def load() -> ctypes.CDLL:
     lib.ark_attn_prefill_rope_layers.restype = I
     lib.ark_attn_encoder.argtypes = [P, P, P, P, I, I, I, I, ctypes.c_float, P, P, P, P]
     lib.ark_attn_encoder.restype = I
+    lib.ark_attn_qkv_proj.argtypes = [P, P, P, I, I, I, P, P, P]
+    lib.ark_attn_qkv_proj.restype = I
+    lib.ark_attn_qkv_rope_append.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P, P]
+    lib.ark_attn_qkv_rope_append.restype = I
     _lib = lib
     return lib
 
@@ -653,3 +659,48 @@ def ark_attn_encoder(q, k, v, length, o, lse, scale: float, status: Optional[tor
     _raise(load().ark_attn_encoder(_ptr(q), _ptr(k), _ptr(v), _ptr(length), B, S, H, D, float(scale), _ptr(o),
                                    _ptr(lse), _ptr(status), _stream(stream)),
            "ark_attn_encoder")
+
+
+# ------------------------------------------------------ Q/K/V projection ----
+
+def ark_attn_qkv_proj(x, w, bias, out, status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """out [M, N] = bf16(x [M, K] @ w [N, K]^T + bias [N]); bias may be None."""
+    _need(x, "x", torch.bfloat16, 2)
+    _need(w, "w", torch.bfloat16, 2)
+    _need(out, "out", torch.bfloat16, 2)
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    M, K = x.shape
+    N = w.shape[0]
+    if w.shape[1] != K or tuple(out.shape) != (M, N) or (bias is not None and bias.shape[0] != N):
+        raise ValueError("shapes")
+    _raise(load().ark_attn_qkv_proj(_ptr(x), _ptr(w), _ptr(bias), M, K, N, _ptr(out), _ptr(status),
+                                    _stream(stream)), "ark_attn_qkv_proj")
+
+
+def ark_attn_qkv_rope_append(x, w, bias, pos0, n_new, table, q, cache_k, cache_v,
+                             status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Projection of x [B, S, K] by w [(Hq + 2 Hkv) * 128, K] (+ bias), then RoPE
+    and the delta write: q [B, S, Hq, 128], caches [B, T, Hkv, 128]."""
+    _need(x, "x", torch.bfloat16, 3)
+    _need(w, "w", torch.bfloat16, 2)
+    for name, t in (("q", q), ("cache_k", cache_k), ("cache_v", cache_v)):
+        _need(t, name, torch.bfloat16, 4)
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1)
+    _need(pos0, "pos0", torch.int32, 1)
+    _need(n_new, "n_new", torch.int32, 1)
+    _need(table, "table", torch.float32)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    B, S, K = x.shape
+    Hq, D = q.shape[2], q.shape[3]
+    T, Hkv = cache_k.shape[1], cache_k.shape[2]
+    if tuple(q.shape[:2]) != (B, S) or w.shape != ((Hq + 2 * Hkv) * D, K) or cache_v.shape != cache_k.shape:
+        raise ValueError("shapes")
+    _raise(load().ark_attn_qkv_rope_append(_ptr(x), _ptr(w), _ptr(bias), _ptr(pos0), _ptr(n_new), B, S, T, Hq,
+                                           Hkv, D, K, _ptr(table), _ptr(q), _ptr(cache_k), _ptr(cache_v),
+                                           _ptr(status), _stream(stream)),
+           "ark_attn_qkv_rope_append")

@@ -332,3 +332,24 @@ def cfg_encoder(seed: int = 6, layers: int = ENC_LAYERS, B: int = 8) -> EncoderB
     secs = 3.0 + 27.0 * torch.rand(B, generator=g)
     lengths = [encoder_frames(float(s)) for s in secs]
     return make_encoder_batch(seed + 1, B, 1500, lengths, layers=layers)
+
+
+# ----------------------------------------------- projection weights (synthetic) ----
+# The decoder's Q/K/V projections (hidden 2048 -> 16 q heads, 2 k, 2 v heads of
+# 128; "ARK-ASR-3B -- INT8 ONNX" model card).  No trained weights: W ~ N(0, 1/K)
+# (the scale of an initialised Linear), bias ~ N(0, 0.1^2), hidden states
+# ~ N(0, 1) (the scale after the RMSNorm in front of the projection).
+
+HIDDEN = 2048
+
+
+def make_qkv_weights(seed: int, K: int = HIDDEN, Hq: int = 16, Hkv: int = 2, D: int = 128, bias: bool = True):
+    g = _gen(seed)
+    N = (Hq + 2 * Hkv) * D
+    w = (torch.randn((N, K), generator=g, dtype=torch.float32) / (K ** 0.5)).to(torch.bfloat16)
+    b = (torch.randn((N,), generator=g, dtype=torch.float32) * 0.1).to(torch.bfloat16) if bias else None
+    return w, b
+
+
+def make_hidden(seed: int, B: int, S: int, K: int = HIDDEN) -> torch.Tensor:
+    return randn_bf16((B, S, K), _gen(seed))

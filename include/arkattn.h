@@ -353,6 +353,38 @@ ARK_API ark_status ark_attn_encoder(const void* q, const void* k, const void* v,
                                     int H, int D, float scale, void* o, float* lse, uint32_t* d_status,
                                     cudaStream_t stream);
 
+/* ------------------------------------------ Q/K/V projection (+ RoPE) ----
+ * The step in front of the attention: the Q/K/V projections of a decoder
+ * layer ("ARK-ASR-3B -- INT8 ONNX" model card: Qwen2 decoder, hidden 2048,
+ * 16 query and 2 KV heads of 128 dims) as one Linear over the concatenated
+ * weight W = [Wq; Wk; Wv], optionally with the RoPE + delta write of
+ * ark_attn_append_rope fused into its epilogue (tcgen05 MMAs, fp32
+ * accumulation).
+ *
+ * ark_attn_qkv_proj: out[m, n] = bf16(sum_k x[m, k] W[n, k] + bias[n]).
+ *   x [M, K], W [N, K], out [M, N] bf16 row-major (16-byte aligned); bias [N]
+ *   bf16 or NULL.  K % 64 == 0, N % 128 == 0, else ARK_ERR_INVALID_ARG.  The
+ *   fp32 accumulator and the bias are added in double and rounded once to bf16.
+ *
+ * ark_attn_qkv_rope_append: x [B, S, K] token rows of B requests (row t of
+ *   request b is live when t < n_new[b], at position pos0[b] + t); W [(Hq + 2
+ *   Hkv) * 128, K] with the q heads first, then k, then v; bias as above.  For
+ *   every live row: q[b, t] = RoPE(p_q) (q [B, S, Hq, 128]), cache_k[b, pos] =
+ *   RoPE(p_k), cache_v[b, pos] = p_v (caches [B, T, Hkv, 128]), with p the
+ *   bf16 projection above and RoPE exactly as in ark_attn_append_rope (table
+ *   from ark_attn_rope_table_init).  Bit-identical to ark_attn_qkv_proj
+ *   followed by ark_attn_append_rope.  Padded rows, and rows whose position
+ *   falls outside [0, T) (ARK_DEV_BAD_POS), are not written; n_new outside
+ *   [0, S] is clamped (ARK_DEV_BAD_KVLEN).  D != 128 returns ARK_ERR_UNSUPPORTED.
+ */
+ARK_API ark_status ark_attn_qkv_proj(const void* x, const void* w, const void* bias, int M, int K, int N, void* out,
+                                     uint32_t* d_status, cudaStream_t stream);
+
+ARK_API ark_status ark_attn_qkv_rope_append(const void* x, const void* w, const void* bias, const int32_t* pos0,
+                                            const int32_t* n_new, int B, int S, int T, int Hq, int Hkv, int D, int K,
+                                            const float* d_table, void* q, void* cache_k, void* cache_v,
+                                            uint32_t* d_status, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
