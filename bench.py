@@ -65,7 +65,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="ragged",
-                    choices=["ragged", "single", "long2048", "long1024", "prefill", "encoder"])
+                    choices=["ragged", "single", "long2048", "long1024", "prefill", "encoder", "qkv_decode",
+                             "qkv_prefill"])
     ap.add_argument("--mode", default="aware", choices=["aware", "masked"])
     ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
                     help="cache format of the decode configurations: bf16, or fp8 E4M3 codes with per-head scales")
@@ -75,7 +76,7 @@ def parse():
     ap.add_argument("--rope-on-load", action="store_true",
                     help="prefill: K/V-only append, RoPE applied by the prefill kernel as it loads q")
     ap.add_argument("--layers", type=int, default=None,
-                    help="encoder: layers per step (default 32; fewer only for profiler captures)")
+                    help="encoder / qkv: layers per step (default 32 / 36; fewer only for profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -549,6 +550,103 @@ def run_encoder(args):
         print(json.dumps(line), flush=True)
 
 
+def run_qkv(args):
+    """The projection step in front of the attention, fused with RoPE and the
+    delta write (ark_attn_qkv_rope_append), for 36 layers each with its own
+    synthetic weights [2560, 2048] (+ bias).  qkv_decode: one decode step of the
+    ragged batch (32 token rows); qkv_prefill: the coalesced prefill batch
+    (16 prompts of 20..387 rows, padded to 387)."""
+    import torch
+    from gqa_attention_static_b200 import ops
+    from gqa_attention_static_b200 import workloads as W
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+    ops.load()
+    L = args.layers or N_LAYERS
+    if args.config == "qkv_decode":
+        base = W.cfg_ragged_decode(layers=1)
+        desc = "decode step B=32 (ragged batch), hidden 2048 -> 16+2+2 heads x 128, 36 layers"
+    else:
+        base = W.cfg_prefill(layers=1)
+        desc = "coalesced prefill B=16 L U[20,387] S=387, hidden 2048 -> 16+2+2 heads x 128, 36 layers"
+    B, S, T = base.B, base.q[0].shape[1], base.T
+    pos0, n_new = base.pos0.to(dev), base.n_new.to(dev)
+    ws, bs, xs, qs, cks, cvs = [], [], [], [], [], []
+    for l in range(L):
+        w, b = W.make_qkv_weights(1000 + l)
+        ws.append(w.to(dev))
+        bs.append(b.to(dev))
+        xs.append(W.make_hidden(2000 + l, B, S).to(dev))
+        qs.append(torch.empty((B, S, 16, 128), dtype=torch.bfloat16, device=dev))
+        cks.append(torch.zeros((B, T, 2, 128), dtype=torch.bfloat16, device=dev))
+        cvs.append(torch.zeros((B, T, 2, 128), dtype=torch.bfloat16, device=dev))
+    table = ops.rope_table(T, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+
+    def step():
+        for l in range(L):
+            ops.ark_attn_qkv_rope_append(xs[l], ws[l], bs[l], pos0, n_new, table, qs[l], cks[l], cvs[l], status,
+                                         stream=s)
+
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    torch.cuda.synchronize()
+    for _ in range(max(3, args.warmup)):
+        g.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        e0.record(s)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms_step = e0.elapsed_time(e1) / args.steps
+    if int(status.item()) != 0:
+        print(f"device status word set: {int(status.item())}", file=sys.stderr)
+    rows = int(base.n_new.sum())
+    N, K = 2560, 2048
+    # algorithmic bytes per layer: W + bias, the live x rows, the q / k / v rows written
+    nbytes = N * K * 2 + N * 2 + rows * K * 2 + rows * N * 2
+    nflops = 2 * rows * K * N
+    ms_launch = ms_step / L
+    hbm, hbm_kind = measured_peaks()
+    tc, tc_kind = measured_tensor_peak()
+    t_bytes = nbytes / (hbm * 1e9)
+    t_flops = nflops / (tc * 1e12)
+    bound = "hbm" if t_bytes >= t_flops else "tensor"
+    achieved = (nbytes / 1e9 if bound == "hbm" else nflops / 1e12) / (ms_launch * 1e-3)
+    roof = {"kernel": "qkv_proj_kernel (ark_attn_qkv_rope_append, one layer per launch)", "bound": bound,
+            "achieved": achieved, "peak": hbm if bound == "hbm" else tc, "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+            "frac": (t_bytes if bound == "hbm" else t_flops) / (ms_launch * 1e-3),
+            "peak_kind": hbm_kind if bound == "hbm" else tc_kind, "traffic": None, "launch_ms": ms_launch,
+            "algorithmic_bytes_per_launch": nbytes, "flops_per_launch": nflops,
+            "achieved_gbs": nbytes / (ms_launch * 1e-3) / 1e9, "achieved_tflops": nflops / (ms_launch * 1e-3) / 1e12}
+    value = rows * L / (ms_step * 1e-3)
+    line = {"metric": "fused Q/K/V projection + RoPE + delta write, token-layers/s (1xB200); % of roofline",
+            "value": value, "unit": "token-layers/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (random-init weights)",
+            "config": {"workload": desc.replace("36 layers", f"{L} layers"), "rows": rows,
+                       "l2": "weights of %d layers (%.0f MB) larger than L2" % (L, L * N * K * 2 / 1e6)},
+            "roofline": roof, "gpu_launches": L * args.steps, "clocks": clk}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -559,6 +657,9 @@ def main():
         return
     if args.config == "encoder":
         run_encoder(args)
+        return
+    if args.config in ("qkv_decode", "qkv_prefill"):
+        run_qkv(args)
         return
     import torch
     import torch.distributed as dist

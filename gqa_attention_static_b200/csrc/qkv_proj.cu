@@ -13,13 +13,21 @@
 // rotate-half RoPE, the same table and the same double-precision formula as
 // ark_attn_append_rope) and to store q, and k and v into the caches at pos.
 //
-// Tiling: one CTA per (128 token rows, one head = 128 output features).  The
-// K dimension streams through a 4-stage ring of 64-wide chunks (x tile 16 KB,
-// W tile 16 KB, 128-byte swizzle) loaded by TMA; one thread issues 4 MMAs of
-// 128x128x16 per chunk into a 128-column TMEM accumulator.  Epilogue: 4 warps,
-// one token row per thread, so the rotary partners i and i + 64 of a head are
-// in the same thread.  The projection value is the fp32 accumulator plus the
-// bias, added in double and rounded once to bf16; the rotation then works on
+// Tiling: one CTA per (128 token rows, one head = 128 output features), two
+// CTAs per SM.  The K dimension streams through a 3-stage ring of 64-wide
+// chunks (x tile 16 KB, W tile 16 KB, 128-byte swizzle) loaded by TMA; one
+// thread issues 4 MMAs of 128x128x16 per chunk into a 128-column TMEM
+// accumulator.  When the tiles are too few to fill the GPU (a decode step: 20
+// tiles of a few token rows, bound by streaming the 10.5 MB weight), K is split
+// over a thread-block cluster of up to 8 CTAs: each sums its share of K, the
+// others leave their fp32 partial tiles in shared memory, and the cluster's
+// rank-0 CTA adds them in rank order over distributed shared memory (so the
+// result does not depend on timing) before its epilogue.  Epilogue: 4 warps
+// move the accumulator tile (one token row per thread) into shared memory; all
+// 128 threads then take (row, 4 rotary pairs) items, the partners i and i + 64
+// of a head being in the same row.  The projection value is the fp32
+// accumulator plus the bias, added in double and rounded once to bf16; the
+// rotation then works on
 // that bf16 value exactly as the append kernel does, so the fused result is
 // bit-identical to ark_attn_qkv_proj followed by ark_attn_append_rope.
 #include "common.cuh"
@@ -31,7 +39,7 @@ namespace qp {
 constexpr int kBM = 128;                 // token rows per tile (MMA M)
 constexpr int kBN = 128;                 // output features per tile: one head (MMA N)
 constexpr int kBK = 64;                  // K chunk: 64 bf16 = one 128-byte swizzle row
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kTileA = kBM * 128;        // 16 KB
 constexpr int kTileB = kBN * 128;        // 16 KB
 constexpr int kStageBytes = kTileA + kTileB;
@@ -42,9 +50,15 @@ constexpr int kBarFull = 0;              // [kStages]
 constexpr int kBarEmpty = kBarFull + kStages;
 constexpr int kBarDone = kBarEmpty + kStages;
 constexpr int kNumBars = kBarDone + 1;
-constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
+constexpr int kOffRows = kOffBar + kNumBars * 8;    // per tile row: int2 {destination offset / 8 or -1, pos}
+constexpr int kOffBias = kOffRows + kBM * 8;           // this head's 128 bias values, fp32
+constexpr int kOffTmemPtr = kOffBias + kBN * 4;
 constexpr int kOffFlag = kOffTmemPtr + 8;
 constexpr int kSmemBytes = kOffFlag + 8;
+constexpr int kPartStride = 132;         // floats per row of a partial tile in shared memory (16-byte rows,
+                                         // conflict-free float4 stores of 8 consecutive rows)
+static_assert(kBM * kPartStride * 4 <= kOffBar, "partial tile fits in the stage buffers");
+constexpr int kMaxSplit = 8;             // portable cluster size
 constexpr uint32_t kTmemCols = 128;
 
 // kind::f16, bf16 x bf16 -> fp32, M = 128, N = 128, A and B K-major
@@ -67,26 +81,51 @@ struct Params {
     int B, S, T, Hq, Hkv;
 };
 
+// Every thread of every CTA of the cluster, at the same program point.
+__device__ __forceinline__ void cluster_sync_all() {
+    __syncwarp();
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 16 bytes of another CTA's shared memory at this CTA's offset `local`.
+__device__ __forceinline__ float4 ld_dsmem_f4(const void* local, uint32_t rank) {
+    uint32_t raddr;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(smem_u32(local)), "r"(rank));
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(raddr) : "memory");
+    return v;
+}
+
 }  // namespace qp
 
-__global__ void __launch_bounds__(qp::kThreads, 1) qkv_proj_kernel(const __grid_constant__ qp::Params p) {
+__global__ void __launch_bounds__(qp::kThreads, 2) qkv_proj_kernel(const __grid_constant__ qp::Params p) {
     using namespace qp;
     extern __shared__ __align__(1024) uint8_t smem[];
+    // the next launch (the next layer's projection, launched with programmatic stream
+    // serialisation) may start streaming its weights now; it reads its x and writes its
+    // outputs only after griddepcontrol.wait, i.e. after this grid has completed
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int head = blockIdx.x;                 // output features 128*head .. +127
     const int m0 = blockIdx.y * kBM;
-    const int nk = p.K / kBK;
-    if (smem_u32(smem) & 1023u) {
-        if (threadIdx.x == 0) report(p.status, ARK_DEV_TIMEOUT);
-        return;
-    }
+    // K split: this CTA sums chunks [c_begin, c_end); blockIdx.z is its rank in the cluster
+    // (cluster dims (1, 1, gridDim.z)); no CTA returns early, every thread reaches the
+    // cluster barriers below
+    const int split = gridDim.z;
+    const int rank = blockIdx.z;
+    const int nk_all = p.K / kBK;
+    const int c_begin = rank * nk_all / split;
+    const int nk = (rank + 1) * nk_all / split - c_begin;
+    const bool misaligned = (smem_u32(smem) & 1023u) != 0;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
     int* failed_flag = reinterpret_cast<int*>(smem + kOffFlag);
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], 1);
-        *failed_flag = 0;
+        *failed_flag = misaligned ? 1 : 0;
+        if (misaligned) report(p.status, ARK_DEV_TIMEOUT);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_ptr, kTmemCols);
@@ -101,12 +140,26 @@ __global__ void __launch_bounds__(qp::kThreads, 1) qkv_proj_kernel(const __grid_
         if (lane == 0) {
             int last = -1;
             bool ok = true;
-            for (int c = 0; c < nk; ++c) {
+            const int n_run = misaligned ? 0 : nk;
+            // the weight tiles of the first stages do not depend on the previous kernel: they go first
+            const int pre = min(n_run, kStages);
+            for (int c = 0; c < pre; ++c) {
+                mbar_arrive_expect_tx(&bars[kBarFull + c], kStageBytes);
+                tma_load_2d(smem + c * kStageBytes + kTileA, &p.wmap, (c_begin + c) * kBK, head * kBN,
+                            &bars[kBarFull + c]);
+            }
+            asm volatile("griddepcontrol.wait;" ::: "memory");    // x may be the previous kernel's output
+            for (int c = 0; c < pre; ++c) {
+                tma_load_2d(smem + c * kStageBytes, &p.xmap, (c_begin + c) * kBK, m0, &bars[kBarFull + c]);
+                last = c;
+            }
+            for (int c = pre; c < n_run; ++c) {
                 const int st = c % kStages;
-                if (c >= kStages && !(ok = mbar_wait(&bars[kBarEmpty + st], ((c / kStages) - 1) & 1))) break;
+                if (!(ok = mbar_wait(&bars[kBarEmpty + st], ((c / kStages) - 1) & 1))) break;
                 mbar_arrive_expect_tx(&bars[kBarFull + st], kStageBytes);
-                tma_load_2d(smem + st * kStageBytes, &p.xmap, c * kBK, m0, &bars[kBarFull + st]);
-                tma_load_2d(smem + st * kStageBytes + kTileA, &p.wmap, c * kBK, head * kBN, &bars[kBarFull + st]);
+                const int kc = (c_begin + c) * kBK;
+                tma_load_2d(smem + st * kStageBytes, &p.xmap, kc, m0, &bars[kBarFull + st]);
+                tma_load_2d(smem + st * kStageBytes + kTileA, &p.wmap, kc, head * kBN, &bars[kBarFull + st]);
                 last = c;
             }
             if (!ok) {
@@ -120,7 +173,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1) qkv_proj_kernel(const __grid_
     } else if (warp == 1) {
         // ================================================= MMA issuer
         bool ok = true;
-        for (int c = 0; c < nk; ++c) {
+        for (int c = 0; c < (misaligned ? 0 : nk); ++c) {
             const int st = c % kStages;
             if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarFull + st], (c / kStages) & 1)))) break;
             if (lane == 0) {
@@ -142,45 +195,33 @@ __global__ void __launch_bounds__(qp::kThreads, 1) qkv_proj_kernel(const __grid_
         __syncwarp();
         if (lane == 0) umma_commit(&bars[kBarDone]);     // also when the loop gave up: MMAs issued so far
         __syncwarp();
-    } else {
-        // ================================================= epilogue: one token row per thread
-        const int quad = warp & 3;               // TMEM lanes 32*quad .. +31
-        const int r = quad * 32 + lane;
-        const int m = m0 + r;
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarDone], 0)) &&
-                        !*reinterpret_cast<volatile int*>(failed_flag);
-        tc_fence_after();
-        if (!ok) {
-            if (lane == 0) report(p.status, ARK_DEV_TIMEOUT);
-        } else if (!p.fused) {
-            // p = bf16(acc + bias) -> out[m][128*head ..]
-            uint16_t* dst = p.out + static_cast<size_t>(m) * p.N + head * kBN;
-            for (int c16 = 0; c16 < kBN / 16; ++c16) {
-                uint32_t a[16];
-                tmem_ld16(lane_base + c16 * 16, a);
-                tmem_wait_ld();
-                if (m < p.M) {
-                    uint32_t w[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int n = head * kBN + c16 * 16 + 2 * i;
-                        const double b0 = p.bias ? bf16_bits_to_f64(p.bias[n]) : 0.0;
-                        const double b1 = p.bias ? bf16_bits_to_f64(p.bias[n + 1]) : 0.0;
-                        w[i] = static_cast<uint32_t>(f64_to_bf16_rn(static_cast<double>(__uint_as_float(a[2 * i])) + b0)) |
-                               (static_cast<uint32_t>(f64_to_bf16_rn(static_cast<double>(__uint_as_float(a[2 * i + 1])) + b1)) << 16);
-                    }
-                    uint4* d4 = reinterpret_cast<uint4*>(dst + c16 * 16);
-                    d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                    d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                }
-            }
-        } else {
-            // which row of which request, and where it goes
-            uint16_t* dst = nullptr;
-            bool rotate = false;
+    }
+
+    // ================================================= epilogue
+    // (1) every epilogue thread moves its TMEM row (a token row) into shared memory, over the
+    // stage buffers, which are free once every MMA is done; (2) in a split cluster, rank 0 adds
+    // the other ranks' tiles to its own, in rank order; (3) all 128 epilogue threads share the
+    // live rows x 16 groups of 4 rotary pairs.  Every epilogue thread reaches every barrier.
+    const int quad = warp & 3;               // TMEM lanes 32*quad .. +31
+    const int r = quad * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    float* part = reinterpret_cast<float*>(smem);          // [kBM][kPartStride] fp32
+    const int rows = min(kBM, p.M - m0);                   // live token rows of this tile
+    int2* rowinfo = reinterpret_cast<int2*>(smem + kOffRows);
+    float* sbias = reinterpret_cast<float*>(smem + kOffBias);
+    if (warp >= 2) {
+        // the outputs may still be read by the previous kernel, and its pos0 / n_new / table writes
+        // must be visible: nothing global is touched before it has completed
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        // while the MMAs run: where this thread's row goes (destination in 8-byte units, or -1),
+        // its position, the head's bias, and the row's rotary table pulled toward L2
+        {
+            const int et = threadIdx.x - 64;
+            sbias[et] = p.bias ? static_cast<float>(bf16_bits_to_f64(p.bias[head * kBN + et])) : 0.f;
+            long long off = -1;
             int pos = 0;
-            if (m < p.M) {
+            if (p.fused && et < rows && rank == 0) {
+                const int m = m0 + et;
                 const int b = m / p.S, t = m - b * p.S;
                 int nn = __ldg(p.n_new + b);
                 if (nn < 0 || nn > p.S) {
@@ -192,64 +233,144 @@ __global__ void __launch_bounds__(qp::kThreads, 1) qkv_proj_kernel(const __grid_
                     if (pos < 0 || pos >= p.T) {
                         if (head == 0) report(p.status, ARK_DEV_BAD_POS);
                     } else if (head < p.Hq) {
-                        dst = p.q + (static_cast<size_t>(m) * p.Hq + head) * kHeadDim;
-                        rotate = true;
+                        off = (static_cast<long long>(m) * p.Hq + head) * kHeadDim;
                     } else if (head < p.Hq + p.Hkv) {
-                        dst = p.cache_k + ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + (head - p.Hq)) * kHeadDim;
-                        rotate = true;
+                        off = ((static_cast<long long>(b) * p.T + pos) * p.Hkv + (head - p.Hq)) * kHeadDim;
                     } else {
-                        dst = p.cache_v +
-                              ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + (head - p.Hq - p.Hkv)) * kHeadDim;
+                        off = ((static_cast<long long>(b) * p.T + pos) * p.Hkv + (head - p.Hq - p.Hkv)) * kHeadDim;
+                    }
+                    if (off >= 0 && head < p.Hq + p.Hkv) {
+                        const char* tr = reinterpret_cast<const char*>(p.table + static_cast<size_t>(pos) * 64);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) asm volatile("prefetch.global.L2 [%0];" :: "l"(tr + 128 * i));
                     }
                 }
             }
-            const float4* trow = reinterpret_cast<const float4*>(p.table + static_cast<size_t>(rotate ? pos : 0) * 64);
-            // rotary pairs (i, i + 64) for i in 16-wide groups; every warp runs every tcgen05.ld
-            for (int g16 = 0; g16 < 4; ++g16) {
-                uint32_t lo[16], hi[16];
-                tmem_ld16(lane_base + g16 * 16, lo);
-                tmem_ld16(lane_base + 64 + g16 * 16, hi);
-                tmem_wait_ld();
-                if (!dst) continue;
-                uint16_t yl[16], yh[16];
+            // offsets are multiples of 128 elements; stored in 8-byte units they fit an int
+            rowinfo[et] = make_int2(off < 0 ? -1 : static_cast<int>(off >> 2), pos);
+        }
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarDone], 0));
+        tc_fence_after();
+        if (!ok) {
+            atomicExch(failed_flag, 1);
+            if (lane == 0) report(p.status, ARK_DEV_TIMEOUT);
+        }
+        for (int c16 = 0; c16 < kBN / 16; ++c16) {
+            uint32_t a[16];
+            tmem_ld16(lane_base + c16 * 16, a);
+            tmem_wait_ld();
+            if (ok && r < rows) {
+                float4* d4 = reinterpret_cast<float4*>(part + r * kPartStride + c16 * 16);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int d = g16 * 16 + i;
-                    const int n = head * kBN + d;
-                    const double bl = p.bias ? bf16_bits_to_f64(p.bias[n]) : 0.0;
-                    const double bh = p.bias ? bf16_bits_to_f64(p.bias[n + 64]) : 0.0;
+                for (int i = 0; i < 4; ++i)
+                    d4[i] = make_float4(__uint_as_float(a[4 * i]), __uint_as_float(a[4 * i + 1]),
+                                        __uint_as_float(a[4 * i + 2]), __uint_as_float(a[4 * i + 3]));
+            }
+        }
+    }
+    if (split > 1) cluster_sync_all();       // the tiles of every rank are in place
+    if (warp >= 2) {
+        const int et = threadIdx.x - 64;     // 0 .. 127
+        if (split > 1 && rank == 0) {
+            // own + rank 1 + rank 2 + ..., each thread's remote loads issued before its adds
+            const int items = rows * (kBN / 4);
+            for (int it0 = et; it0 < items; it0 += 256) {
+                // two pieces per pass: every remote load of both is in flight before the first add
+                float* loc[2];
+                float4 t[2][kMaxSplit - 1];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int it = min(it0 + 128 * u, items - 1);
+                    loc[u] = part + (it / (kBN / 4)) * kPartStride + (it % (kBN / 4)) * 4;
+#pragma unroll
+                    for (int z = 1; z < kMaxSplit; ++z)
+                        if (z < split) t[u][z - 1] = ld_dsmem_f4(loc[u], static_cast<uint32_t>(z));
+                }
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    if (it0 + 128 * u >= items) continue;
+                    float4 sum = *reinterpret_cast<const float4*>(loc[u]);
+#pragma unroll
+                    for (int z = 1; z < kMaxSplit; ++z)
+                        if (z < split) {
+                            sum.x += t[u][z - 1].x;
+                            sum.y += t[u][z - 1].y;
+                            sum.z += t[u][z - 1].z;
+                            sum.w += t[u][z - 1].w;
+                        }
+                    *reinterpret_cast<float4*>(loc[u]) = sum;
+                }
+            }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");     // the tile's sums are complete
+        const bool failed = *reinterpret_cast<volatile int*>(failed_flag) != 0;
+        if (rank == 0 && !failed && !p.fused) {
+            // p = bf16(acc + bias) -> out[m][128*head ..]: items of 8 columns
+            for (int it = et; it < rows * (kBN / 8); it += 128) {
+                const int row = it / (kBN / 8), c8 = (it % (kBN / 8)) * 8;
+                const float* src = part + row * kPartStride + c8;
+                uint32_t w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const double b0 = static_cast<double>(sbias[c8 + 2 * i]);
+                    const double b1 = static_cast<double>(sbias[c8 + 2 * i + 1]);
+                    w[i] = static_cast<uint32_t>(f64_to_bf16_rn(static_cast<double>(src[2 * i]) + b0)) |
+                           (static_cast<uint32_t>(f64_to_bf16_rn(static_cast<double>(src[2 * i + 1]) + b1)) << 16);
+                }
+                *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(m0 + row) * p.N + head * kBN + c8) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        } else if (rank == 0 && !failed) {
+            // items (row, group g of rotary pairs 4g .. 4g+3): the projection value is the
+            // accumulator plus the bias rounded once to bf16, then the append kernel's rotation
+            for (int it = et; it < rows * 16; it += 128) {
+                const int row = it >> 4, g = it & 15;
+                const int2 info = rowinfo[row];
+                if (info.x < 0) continue;                         // padded or out-of-range row: not written
+                const int pos = info.y;
+                uint16_t* base = head < p.Hq ? p.q : (head < p.Hq + p.Hkv ? p.cache_k : p.cache_v);
+                uint16_t* dst = base + (static_cast<size_t>(info.x) << 2);
+                const bool rotate = head < p.Hq + p.Hkv;
+                const float4 lo = *reinterpret_cast<const float4*>(part + row * kPartStride + 4 * g);
+                const float4 hi = *reinterpret_cast<const float4*>(part + row * kPartStride + 64 + 4 * g);
+                const float al[4] = {lo.x, lo.y, lo.z, lo.w};
+                const float ah[4] = {hi.x, hi.y, hi.z, hi.w};
+                const float4* trow = reinterpret_cast<const float4*>(p.table + static_cast<size_t>(pos) * 64);
+                const float4 cs01 = __ldg(trow + 2 * g);          // c0 s0 c1 s1 of pairs 4g, 4g+1
+                const float4 cs23 = __ldg(trow + 2 * g + 1);      // c2 s2 c3 s3
+                const float cc[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
+                const float ss[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
+                uint16_t yl[4], yh[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const double bl = static_cast<double>(sbias[4 * g + i]);
+                    const double bh = static_cast<double>(sbias[64 + 4 * g + i]);
                     // the projection output (the Linear's bf16 value)
-                    const uint16_t xl = f64_to_bf16_rn(static_cast<double>(__uint_as_float(lo[i])) + bl);
-                    const uint16_t xh = f64_to_bf16_rn(static_cast<double>(__uint_as_float(hi[i])) + bh);
+                    const uint16_t xl = f64_to_bf16_rn(static_cast<double>(al[i]) + bl);
+                    const uint16_t xh = f64_to_bf16_rn(static_cast<double>(ah[i]) + bh);
                     if (rotate) {
-                        const float4 cs = __ldg(trow + (d >> 1));        // {c, s} of pairs d & ~1 and d | 1
-                        const double c = static_cast<double>((d & 1) ? cs.z : cs.x);
-                        const double s = static_cast<double>((d & 1) ? cs.w : cs.y);
                         const double a = bf16_bits_to_f64(xl);
                         const double h = bf16_bits_to_f64(xh);
+                        const double c = static_cast<double>(cc[i]);
+                        const double sn = static_cast<double>(ss[i]);
                         // both products are exact in double, so contraction cannot change the result
-                        yl[i] = f64_to_bf16_rn(a * c - h * s);
-                        yh[i] = f64_to_bf16_rn(h * c + a * s);
+                        yl[i] = f64_to_bf16_rn(a * c - h * sn);
+                        yh[i] = f64_to_bf16_rn(h * c + a * sn);
                     } else {
                         yl[i] = xl;
                         yh[i] = xh;
                     }
                 }
-                uint32_t wl[8], wh[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    wl[i] = static_cast<uint32_t>(yl[2 * i]) | (static_cast<uint32_t>(yl[2 * i + 1]) << 16);
-                    wh[i] = static_cast<uint32_t>(yh[2 * i]) | (static_cast<uint32_t>(yh[2 * i + 1]) << 16);
-                }
-                uint4* dl = reinterpret_cast<uint4*>(dst + g16 * 16);
-                uint4* dh = reinterpret_cast<uint4*>(dst + 64 + g16 * 16);
-                dl[0] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-                dl[1] = make_uint4(wl[4], wl[5], wl[6], wl[7]);
-                dh[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-                dh[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
+                *reinterpret_cast<uint2*>(dst + 4 * g) =
+                    make_uint2(static_cast<uint32_t>(yl[0]) | (static_cast<uint32_t>(yl[1]) << 16),
+                               static_cast<uint32_t>(yl[2]) | (static_cast<uint32_t>(yl[3]) << 16));
+                *reinterpret_cast<uint2*>(dst + 64 + 4 * g) =
+                    make_uint2(static_cast<uint32_t>(yh[0]) | (static_cast<uint32_t>(yh[1]) << 16),
+                               static_cast<uint32_t>(yh[2]) | (static_cast<uint32_t>(yh[3]) << 16));
             }
         }
     }
+    if (split > 1) cluster_sync_all();       // rank 0 has read every other rank's tile: they may exit
 
     tc_fence_before();
     __syncthreads();
@@ -268,6 +389,8 @@ namespace {
 bool qp_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool g_qp_attr[64];
+int g_qp_sms[64];
+int g_qp_clusters[64][4];    // clusters of 2, 4, 8 CTAs that can be resident at once (0: unknown)
 
 ark_status launch_qkv(qp::Params& prm, const void* x, const void* w, int M, int K, int N, cudaStream_t stream) {
     if (!kmajor_tensor_map(&prm.xmap, x, M, K, qp::kBM) || !kmajor_tensor_map(&prm.wmap, w, N, K, qp::kBN))
@@ -281,10 +404,50 @@ ark_status launch_qkv(qp::Params& prm, const void* x, const void* w, int M, int 
         if (cudaFuncSetAttribute(qkv_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, qp::kSmemBytes) !=
             cudaSuccess)
             return ARK_ERR_CUDA;
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            return ARK_ERR_CUDA;
+        g_qp_sms[dev] = sms;
         g_qp_attr[dev] = true;
     }
-    const dim3 grid(N / qp::kBN, (M + qp::kBM - 1) / qp::kBM);
-    qkv_proj_kernel<<<grid, qp::kThreads, qp::kSmemBytes, stream>>>(prm);
+    const int tiles = (N / qp::kBN) * ((M + qp::kBM - 1) / qp::kBM);
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(qp::kThreads);
+    cfg.dynamicSmemBytes = qp::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = 1;
+    // split K over a cluster while every cluster of the launch can be resident at once (one wave),
+    // the CTAs fit two per SM and the chunks divide evenly
+    int split = 1;
+    const int nk = K / qp::kBK;
+    for (int cand = 2, ci = 0; cand <= qp::kMaxSplit; cand *= 2, ++ci) {
+        if (nk % cand != 0 || static_cast<long long>(tiles) * cand > 2LL * g_qp_sms[dev]) break;
+        if (g_qp_clusters[dev][ci] == 0) {
+            cudaLaunchConfig_t occ = cfg;
+            occ.gridDim = dim3(1, 1, cand);
+            attr[1].val.clusterDim.z = static_cast<unsigned>(cand);
+            occ.attrs = attr + 1;
+            occ.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, qkv_proj_kernel, &occ) != cudaSuccess) {
+                (void)cudaGetLastError();
+                n = -1;
+            }
+            g_qp_clusters[dev][ci] = n > 0 ? n : -1;
+        }
+        if (g_qp_clusters[dev][ci] < tiles) break;
+        split = cand;
+    }
+    cfg.gridDim = dim3(N / qp::kBN, (M + qp::kBM - 1) / qp::kBM, split);
+    attr[1].val.clusterDim.z = static_cast<unsigned>(split);
+    cfg.attrs = attr;
+    cfg.numAttrs = split > 1 ? 2 : 1;
+    if (cudaLaunchKernelEx(&cfg, qkv_proj_kernel, prm) != cudaSuccess) return ARK_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
 }
 
@@ -313,8 +476,10 @@ extern "C" ark_status ark_attn_qkv_rope_append(const void* x, const void* w, con
     if (B <= 0 || S <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || K <= 0 || K % qp::kBK != 0) return ARK_ERR_INVALID_ARG;
     if (D != kHeadDim) return ARK_ERR_UNSUPPORTED;
     const long long M = static_cast<long long>(B) * S;
+    // row destinations are kept as 32-bit counts of 8-byte units
     if (M >= (1LL << 31) || static_cast<long long>(B) * T >= (1LL << 31) || Hq + 2 * Hkv > 65535 ||
-        (M + qp::kBM - 1) / qp::kBM > 65535)
+        (M + qp::kBM - 1) / qp::kBM > 65535 || M * Hq * (kHeadDim / 4) >= (1LL << 31) ||
+        static_cast<long long>(B) * T * Hkv * (kHeadDim / 4) >= (1LL << 31))
         return ARK_ERR_UNSUPPORTED;
     if (!qp_aligned16(x) || !qp_aligned16(w) || !qp_aligned16(q) || !qp_aligned16(cache_k) ||
         !qp_aligned16(cache_v) || !qp_aligned16(d_table) || (reinterpret_cast<uintptr_t>(bias) & 1u))
