@@ -58,6 +58,13 @@ PREFILL_TRAFFIC = {
 }
 
 
+# Per-launch DRAM traffic of the encoder attention kernel (one layer of the encoder batch)
+# from an ncu --set full capture, keyed the same way.
+ENCODER_TRAFFIC = {
+    "1c03b40e4781186eaf749a42e344400882142a09be1bd50caa849ab8ddb7ce20": 62.4896e6 + 2.68032e6,
+}
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -537,7 +544,8 @@ def run_encoder(args):
     achieved = nf / (ms_launch * 1e-3) / 1e12
     roof = {"kernel": "encoder_attn_kernel (ark_attn_encoder, one layer per launch)", "bound": "tensor",
             "achieved": achieved, "peak": tc, "unit": "TFLOP/s", "frac": achieved / tc, "peak_kind": tc_kind,
-            "traffic": None, "launch_ms": ms_launch, "flops_per_launch": nf}
+            "traffic": ENCODER_TRAFFIC.get(src_hash("gqa_attention_static_b200/csrc/encoder.cu")),
+            "launch_ms": ms_launch, "flops_per_launch": nf}
     value = achieved
     line = {"metric": "encoder attention TFLOP/s (1xB200); % of bf16 tensor roofline", "value": value,
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
