@@ -46,15 +46,24 @@ N_LAYERS = 36
 DECODE_TRAFFIC = {
     # ncu, one call of the ragged decode workload: decode_kernel (--set full) plus
     # merge_kernel (dram bytes), read + write (see profiles/)
-    "f7a1da552b684995569ecc1bd9f9489abae906c47d9b1b1550bb2b7a9bce5fee":
-        329.750784e6 + 4.109312e6 + 13.198592e6 + 256,
+    "79d6a2dbdddefa6947b568ea05b6e92b19c54f1d75f952faafdef48dae35a988":
+        329.755392e6 + 4.086016e6 + 13.198848e6 + 0,
 }
 
 
 # Per-launch DRAM traffic of the prefill kernel (one layer of the coalesced
 # prefill workload) from an ncu --set full capture, keyed the same way.
 PREFILL_TRAFFIC = {
-    "140f02fa222ad28528f71bc5d4aa3343e3c9092a1c033aede617ebbebd746419": 17.877504e6 + 256,
+    # one 16-layer launch of the coalesced prefill (read 332.35 MB + write 185.23 MB) / 16
+    "82d36dee9a26219530cce144be51941b9b67aa54cb2d787cce86b47d539d46fb": (332.350976e6 + 185.234688e6) / 16,
+}
+
+
+# Per-launch DRAM traffic of the projection kernel (one layer) from ncu --set full
+# captures of the two projection workloads, keyed by source hash and workload.
+QKV_TRAFFIC = {
+    ("7ba1c3300cd72423b0759df4608c6a375ea573145e282d46291568ca38ad809d", "qkv_decode"): 10.668288e6 + 0,
+    ("7ba1c3300cd72423b0759df4608c6a375ea573145e282d46291568ca38ad809d", "qkv_prefill"): 36.077568e6 + 0.54272e6,
 }
 
 
@@ -640,7 +649,9 @@ def run_qkv(args):
     roof = {"kernel": "qkv_proj_kernel (ark_attn_qkv_rope_append, one layer per launch)", "bound": bound,
             "achieved": achieved, "peak": hbm if bound == "hbm" else tc, "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
             "frac": (t_bytes if bound == "hbm" else t_flops) / (ms_launch * 1e-3),
-            "peak_kind": hbm_kind if bound == "hbm" else tc_kind, "traffic": None, "launch_ms": ms_launch,
+            "peak_kind": hbm_kind if bound == "hbm" else tc_kind,
+            "traffic": QKV_TRAFFIC.get((src_hash("gqa_attention_static_b200/csrc/qkv_proj.cu"), args.config)),
+            "launch_ms": ms_launch,
             "algorithmic_bytes_per_launch": nbytes, "flops_per_launch": nflops,
             "achieved_gbs": nbytes / (ms_launch * 1e-3) / 1e9, "achieved_tflops": nflops / (ms_launch * 1e-3) / 1e12}
     value = rows * L / (ms_step * 1e-3)

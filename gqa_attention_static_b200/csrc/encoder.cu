@@ -17,84 +17,81 @@
 //   o[b,i,h,:] = sum_{j < len[b]} softmax_j(scale <q[b,i,h,:], k[b,j,h,:]>) v[b,j,h,:]
 //   lse[b,h,i] = ln sum_{j < len[b]} exp(scale <q[b,i,h,:], k[b,j,h,:]>)
 //
-// Work: a tile is 128 consecutive frames of one (clip, head); only tiles with
-// a frame inside their clip exist.  The kernel is persistent: two CTAs per SM,
-// each walking the tile list (clips longest first) in snake order, so that
-// the long tiles spread evenly and no CTA is launched for padding.  Inside a
-// CTA the tiles run as one pipeline: Q is double-buffered, K and V blocks of
-// 64 frames (8 KB each) stream through 4-stage rings, and the first QK^T of
-// the next tile is issued before the last PV of the current one.
+// Work: a unit is 256 consecutive frames of one (clip, head), two Q tiles A
+// and B of 128 rows (MMA M = 128) that share every K/V block; only units with
+// a frame inside their clip exist, and tile B is skipped when it has none.
+// The kernel is persistent, one CTA per SM walking the unit list (clips with
+// more key blocks first) in snake order.  K and V blocks of 128 frames (16 KB
+// each) stream through 3-stage TMA rings, Q through 2 buffers.
 //
-// Per block: S = Q K^T is 4 MMAs of 128x64x16 into a double-buffered TMEM S.
-// Warp 0 issues the TMA copies, warp 1 the MMAs (one thread), warps 2..9 run
-// the softmax with two threads per row, one for each half of a block's keys.
-// The halves are independent: each keeps its own running maximum (lazily
-// rescaled), sum and O accumulator in TMEM and stores its P (bf16) over its
-// own scores, and O_half += P_half V_half is 2 MMAs of 128x64x16 with P read
-// from TMEM and V an MN-major operand.  The two partial results are merged
-// once per tile in the epilogue (the rule of a split-KV combine).  Keys past
-// len[b] get score -inf (and their V rows are zeroed) in the last block only.
-// Rows past len[b] are computed on whatever q holds and are not written.
+// Per block and tile X: S_X = Q_X K^T is 4 MMAs of 128x128x16 into 128 TMEM
+// columns; the tile's softmax warpgroup (one thread per row, all 128 keys of
+// the block) stores P (bf16) over the first 64 columns of S_X, and O_X +=
+// P_X V is 8 MMAs of 128x64x16 with P read from TMEM and V an MN-major
+// operand.  The MMA warp interleaves the tiles (QK_A, QK_B, PV_A, QK_A next,
+// PV_B, QK_B next, ...), so one tile's softmax runs while the tensor cores
+// work for the other.  Because QK_X(j+1) is issued after PV_X(j), a softmax
+// that finds S_X(j+1) ready also knows O_X holds PV_X(j): the lazy rescale of
+// O_X needs no wait of its own.  Keys past len[b] get score -inf (and their V
+// rows are zeroed) in the last block only.  Rows past len[b] are computed on
+// whatever q holds and are not written.  Warps: 0 TMA, 1 MMA (one thread),
+// 2..5 softmax of tile A, 6..9 softmax of tile B.
 #include "common.cuh"
 #include "tma_host.h"
 
 namespace ark {
 namespace enc {
 
-constexpr int kRows = 128;               // frames per tile (MMA M)
+constexpr int kRows = 128;               // frames per Q tile (MMA M)
+constexpr int kUnitRows = 2 * kRows;     // frames per unit (tiles A and B)
 constexpr int kD = 64;                   // head dim
-constexpr int kBN = 64;                  // keys per block
-constexpr int kQBytes = kRows * 128;     // 128 rows x 64 dims bf16
-constexpr int kKV = kBN * 128;           // a K or V block (8 KB)
+constexpr int kBN = 128;                 // keys per block
+constexpr int kQBytes = kRows * 128;     // one Q tile: 128 rows x 64 dims bf16 (16 KB)
+constexpr int kKV = kBN * 128;           // a K or V block (16 KB)
 constexpr int kThreads = 320;
-constexpr int kHalfThreads = 128;        // softmax threads of one half (one thread per row)
-constexpr int kSoftmaxThreads = 2 * kHalfThreads;
-constexpr int kQStages = 2;
-constexpr int kStages = 4;               // K and V ring depth
+constexpr int kWgThreads = 128;          // softmax threads of one tile (one per row)
+constexpr int kQStages = 2;              // units in flight (each 2 tiles)
+constexpr int kStages = 3;               // K and V ring depth
 constexpr int kMaxClips = 256;
 
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQStages * kQBytes;
+constexpr int kOffK = kOffQ + kQStages * 2 * kQBytes;
 constexpr int kOffV = kOffK + kStages * kKV;
 constexpr int kOffBar = kOffV + kStages * kKV;
 constexpr int kBarQFull = 0;                       // [kQStages]
-constexpr int kBarQEmpty = kBarQFull + kQStages;   // [kQStages]: every QK of the tile done
+constexpr int kBarQEmpty = kBarQFull + kQStages;   // [kQStages]: every QK of the unit done
 constexpr int kBarKFull = kBarQEmpty + kQStages;   // [kStages]
 constexpr int kBarKEmpty = kBarKFull + kStages;
 constexpr int kBarVFull = kBarKEmpty + kStages;
 constexpr int kBarVEmpty = kBarVFull + kStages;
-constexpr int kBarSFull = kBarVEmpty + kStages;    // [2]: S buffer
-constexpr int kBarPFull = kBarSFull + 2;           // [half][2]: P of a half in TMEM (count 128)
-constexpr int kBarPvDone = kBarPFull + 4;          // [half]: PV of a half's keys done (one phase per block)
-constexpr int kBarODone = kBarPvDone + 2;          // every MMA of a tile done (one phase per tile)
-constexpr int kBarOEmpty = kBarODone + 1;          // O read out by the epilogue (count 256, one phase per tile)
-constexpr int kBarDrain = kBarOEmpty + 1;          // MMAs in flight when the MMA warp gives up
-constexpr int kBarXchg = kBarDrain + 1;            // [tile parity]: both halves' (max, sum) in shared memory (count 256)
-constexpr int kNumBars = kBarXchg + 2;
-constexpr int kOffXchg = kOffBar + kNumBars * 8;   // [tile parity][half][max, sum][128] fp32
-constexpr int kOffClips = kOffXchg + 2 * 2 * 2 * kRows * 4;
-//   int len[kMaxClips] (clamped), order[kMaxClips] (clips, longest first), cum[kMaxClips + 1] (tile prefix)
+constexpr int kBarSFull = kBarVEmpty + kStages;    // [tile]: S_X of the next block (one phase per block)
+constexpr int kBarPFull = kBarSFull + 2;           // [tile]: P_X in TMEM (count 128, one phase per block)
+constexpr int kBarODone = kBarPFull + 2;           // [tile]: every MMA of the unit done (one phase per unit)
+constexpr int kBarOEmpty = kBarODone + 2;          // [tile]: O_X read out (count 128, one phase per unit)
+constexpr int kBarDrain = kBarOEmpty + 2;          // MMAs in flight when the MMA warp gives up
+constexpr int kNumBars = kBarDrain + 1;
+constexpr int kOffClips = kOffBar + kNumBars * 8;
+//   int len[kMaxClips] (clamped), order[kMaxClips] (clips, most key blocks first), cum[kMaxClips + 1]
 constexpr int kOffTmemPtr = kOffClips + (3 * kMaxClips + 1) * 4 + 12;
 constexpr int kOffFlag = kOffTmemPtr + 8;
 constexpr int kSmemBytes = kOffFlag + 16;
 static_assert(kOffBar % 8 == 0 && kOffTmemPtr % 8 == 0, "alignment");
 
-// TMEM columns: S buffers 0..63 and 64..127 (fp32 scores; half h's P, bf16
-// pairs, over columns 32h..32h+15 of its own scores), O of the keys of half 0
-// at 128..191 and of half 1 at 192..255.
+// TMEM columns: S_A 0..127, S_B 128..255 (fp32 scores; P as bf16 pairs over the
+// first 64 columns of its own S), O_A 256..319, O_B 320..383.
 constexpr uint32_t kColS = 0;
-constexpr uint32_t kColO = 128;
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColO = 256;
+constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kIdescF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 4) << 24);
-constexpr uint32_t kIdescQK = kIdescF16 | ((64u >> 3) << 17);                // N = 64 keys, K-major B
+constexpr uint32_t kIdescQK = kIdescF16 | ((128u >> 3) << 17);               // N = 128 keys, K-major B
 constexpr uint32_t kIdescPV = kIdescF16 | ((64u >> 3) << 17) | (1u << 16);   // N = 64 dims, MN-major B
 
 constexpr float kLazyRescale = 8.0f;
 
 struct Params {
     CUtensorMap qmap;    // q as (64, H, B*S), box (64, 1, 128)
-    CUtensorMap kmap;    // k as (64, H, B*S), box (64, 1, 64)
+    CUtensorMap kmap;    // k as (64, H, B*S), box (64, 1, 128)
     CUtensorMap vmap;
     uint16_t* o;         // [B, S, H, 64]
     float* lse;          // [B, H, S]
@@ -137,35 +134,36 @@ __device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-// The k-th tile of CTA c among G CTAs: snake order over the tile list.
-__device__ __forceinline__ int snake_tile(int k, int c, int G) { return k * G + ((k & 1) ? G - 1 - c : c); }
+// The k-th unit of CTA c among G CTAs: snake order over the unit list.
+__device__ __forceinline__ int snake_unit(int k, int c, int G) { return k * G + ((k & 1) ? G - 1 - c : c); }
 
-// A tile of the list, by the clip tables in shared memory.
-struct Tile {
-    int b, h, qt, len, nblk;
+struct Unit {
+    int b, h, u, len, nblk;
+    bool live_b;         // tile B has a frame inside the clip
 };
 
-// Tile t: clip order[r] with cum[r] <= t < cum[r + 1] (r only grows along a
-// CTA's walk), frames fastest, heads next.  False past the list.
-__device__ __forceinline__ bool tile_at(int t, int& r, const int* slen, const int* order, const int* cum, int B,
-                                        Tile& out) {
+// Unit t: clip order[r] with cum[r] <= t < cum[r + 1] (r only grows along a
+// CTA's walk), frame ranges fastest, heads next.  False past the list.
+__device__ __forceinline__ bool unit_at(int t, int& r, const int* slen, const int* order, const int* cum, int B,
+                                        Unit& out) {
     while (r < B && cum[r + 1] <= t) ++r;
     if (r >= B) return false;
     const int b = order[r];
     const int len = slen[b];
-    const int nt = ceil_div(len, kRows);
-    const int u = t - cum[r];
+    const int nt = ceil_div(len, kUnitRows);
+    const int v = t - cum[r];
     out.b = b;
-    out.h = u / nt;
-    out.qt = u - out.h * nt;
+    out.h = v / nt;
+    out.u = v - out.h * nt;
     out.len = len;
     out.nblk = ceil_div(len, kBN);
+    out.live_b = out.u * kUnitRows + kRows < len;
     return true;
 }
 
 }  // namespace enc
 
-__global__ void __launch_bounds__(enc::kThreads, 2) encoder_attn_kernel(const __grid_constant__ enc::Params p) {
+__global__ void __launch_bounds__(enc::kThreads, 1) encoder_attn_kernel(const __grid_constant__ enc::Params p) {
     using namespace enc;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
@@ -182,7 +180,7 @@ __global__ void __launch_bounds__(enc::kThreads, 2) encoder_attn_kernel(const __
     int* cum = order + kMaxClips;
     const int B = p.B, H = p.H, G = gridDim.x, c = blockIdx.x;
 
-    // ---- clip tables: clamped lengths, clips by decreasing block count, tile prefix sums
+    // ---- clip tables: clamped lengths, clips by decreasing block count, unit prefix sums
     if (threadIdx.x < B) {
         int len = __ldg(p.len + threadIdx.x);
         if (len < 0 || len > p.S) {
@@ -204,17 +202,16 @@ __global__ void __launch_bounds__(enc::kThreads, 2) encoder_attn_kernel(const __
     __syncthreads();
     if (threadIdx.x == 0) {
         cum[0] = 0;
-        for (int r = 0; r < B; ++r) cum[r + 1] = cum[r] + ceil_div(slen[order[r]], kRows) * H;
+        for (int r = 0; r < B; ++r) cum[r + 1] = cum[r] + ceil_div(slen[order[r]], kUnitRows) * H;
     }
     __syncthreads();
     const int total = cum[B];
-    if (c >= total) return;                                  // no tile for this CTA
+    if (c >= total) return;                                  // no unit for this CTA
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNumBars; ++i) {
             uint32_t cnt = 1;
-            if (i >= kBarPFull && i < kBarPFull + 4) cnt = kHalfThreads;
-            if (i == kBarOEmpty || i == kBarXchg || i == kBarXchg + 1) cnt = kSoftmaxThreads;
+            if ((i >= kBarPFull && i < kBarPFull + 2) || (i >= kBarOEmpty && i < kBarOEmpty + 2)) cnt = kWgThreads;
             mbar_init(&bars[i], cnt);
         }
         *failed_flag = 0;
@@ -232,29 +229,31 @@ __global__ void __launch_bounds__(enc::kThreads, 2) encoder_attn_kernel(const __
         if (lane == 0) {
             bool ok = true;
             int r = 0, g = 0;
-            int last_q[kQStages] = {-1, -1};        // last tile whose Q went into each buffer
-            int last_k[kStages] = {-1, -1, -1, -1};   // last block whose K (V) went into each stage
-            int last_v[kStages] = {-1, -1, -1, -1};
+            int last_q[kQStages] = {-1, -1};        // last unit whose Q went into each buffer
+            int last_k[kStages] = {-1, -1, -1};     // last block whose K (V) went into each stage
+            int last_v[kStages] = {-1, -1, -1};
             for (int k = 0; ok; ++k) {
-                const int t = snake_tile(k, c, G);
-                Tile tl;
-                if (t >= total || !tile_at(t, r, slen, order, cum, B, tl)) break;
-                const int row0 = tl.b * p.S;
+                const int t = snake_unit(k, c, G);
+                Unit un;
+                if (t >= total || !unit_at(t, r, slen, order, cum, B, un)) break;
+                const int row0 = un.b * p.S;
                 const int qs = k & 1;
                 if (k >= kQStages && !(ok = mbar_wait(&bars[kBarQEmpty + qs], ((k >> 1) - 1) & 1))) break;
-                mbar_arrive_expect_tx(&bars[kBarQFull + qs], kQBytes);
-                tma_load_3d(smem + kOffQ + qs * kQBytes, &p.qmap, 0, tl.h, row0 + tl.qt * kRows, &bars[kBarQFull + qs]);
+                mbar_arrive_expect_tx(&bars[kBarQFull + qs], 2 * kQBytes);
+                uint8_t* qd = smem + kOffQ + qs * 2 * kQBytes;
+                tma_load_3d(qd, &p.qmap, 0, un.h, row0 + un.u * kUnitRows, &bars[kBarQFull + qs]);
+                tma_load_3d(qd + kQBytes, &p.qmap, 0, un.h, row0 + un.u * kUnitRows + kRows, &bars[kBarQFull + qs]);
                 last_q[qs] = k;
-                for (int j = 0; j < tl.nblk; ++j, ++g) {
+                for (int j = 0; j < un.nblk; ++j, ++g) {
                     const int st = g % kStages;
                     const uint32_t par = ((g / kStages) - 1) & 1;
                     if (g >= kStages && !(ok = mbar_wait(&bars[kBarKEmpty + st], par))) break;
                     mbar_arrive_expect_tx(&bars[kBarKFull + st], kKV);
-                    tma_load_3d(smem + kOffK + st * kKV, &p.kmap, 0, tl.h, row0 + j * kBN, &bars[kBarKFull + st]);
+                    tma_load_3d(smem + kOffK + st * kKV, &p.kmap, 0, un.h, row0 + j * kBN, &bars[kBarKFull + st]);
                     last_k[st] = g;
                     if (g >= kStages && !(ok = mbar_wait(&bars[kBarVEmpty + st], par))) break;
                     mbar_arrive_expect_tx(&bars[kBarVFull + st], kKV);
-                    tma_load_3d(smem + kOffV + st * kKV, &p.vmap, 0, tl.h, row0 + j * kBN, &bars[kBarVFull + st]);
+                    tma_load_3d(smem + kOffV + st * kKV, &p.vmap, 0, un.h, row0 + j * kBN, &bars[kBarVFull + st]);
                     last_v[st] = g;
                 }
             }
@@ -262,103 +261,108 @@ __global__ void __launch_bounds__(enc::kThreads, 2) encoder_attn_kernel(const __
                 atomicExch(failed_flag, 1);
                 report(p.status, ARK_DEV_TIMEOUT);
             }
-            {
-                // every copy issued has landed before the shared memory can go away (on the normal
-                // path the consumers have seen all of them already)
-                for (int s = 0; s < kQStages; ++s)
-                    if (last_q[s] >= 0) (void)mbar_wait(&bars[kBarQFull + s], (last_q[s] >> 1) & 1);
-                for (int s = 0; s < kStages; ++s) {
-                    if (last_k[s] >= 0) (void)mbar_wait(&bars[kBarKFull + s], (last_k[s] / kStages) & 1);
-                    if (last_v[s] >= 0) (void)mbar_wait(&bars[kBarVFull + s], (last_v[s] / kStages) & 1);
-                }
+            // every copy issued has landed before the shared memory can go away (on the normal
+            // path the consumers have seen all of them already)
+            for (int s = 0; s < kQStages; ++s)
+                if (last_q[s] >= 0) (void)mbar_wait(&bars[kBarQFull + s], (last_q[s] >> 1) & 1);
+            for (int s = 0; s < kStages; ++s) {
+                if (last_k[s] >= 0) (void)mbar_wait(&bars[kBarKFull + s], (last_k[s] / kStages) & 1);
+                if (last_v[s] >= 0) (void)mbar_wait(&bars[kBarVFull + s], (last_v[s] / kStages) & 1);
             }
         }
     } else if (warp == 1) {
         // ================================================= MMA issuer
         bool ok = true;
-        // S = Q K^T of block g (block j of tile k)
-        auto issue_qk = [&](int k, int j, int g, const Tile& tl) {
-            const int qs = k & 1, st = g % kStages;
-            if (j == 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarQFull + qs], (k >> 1) & 1)))) return;
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarKFull + st], (g / kStages) & 1)))) return;
+        int gx[2] = {0, 0};       // blocks issued per tile (S_X / P_X phases)
+        int kx[2] = {0, 0};       // units finished per tile (O_X phases)
+        // S_X = Q_X K^T of block j (the block's K in stage st)
+        auto issue_qk = [&](int x, int qs, int st) {
             if (lane == 0) {
                 tc_fence_after();
-                const uint32_t d = tmem + kColS + (g & 1) * kBN;
-                const uint32_t qa = sbase + kOffQ + qs * kQBytes;
+                const uint32_t qa = sbase + kOffQ + qs * 2 * kQBytes + x * kQBytes;
                 const uint32_t kb = sbase + kOffK + st * kKV;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(d, umma_desc_sw128(qa + kk * 32, 16, 1024), umma_desc_sw128(kb + kk * 32, 16, 1024),
-                             kIdescQK, kk > 0 ? 1u : 0u);
-                umma_commit(&bars[kBarSFull + (g & 1)]);
-                umma_commit(&bars[kBarKEmpty + st]);
-                if (j == tl.nblk - 1) umma_commit(&bars[kBarQEmpty + qs]);
+                    umma_f16(tmem + kColS + x * kBN, umma_desc_sw128(qa + kk * 32, 16, 1024),
+                             umma_desc_sw128(kb + kk * 32, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+                umma_commit(&bars[kBarSFull + x]);
             }
             __syncwarp();
         };
-        // O_half += P_half V_half for both halves of block g (block j of tile k)
-        auto issue_pv = [&](int k, int j, int g, const Tile& tl) {
-            const int st = g % kStages;
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarVFull + st], (g / kStages) & 1)))) return;
-            const int live = tl.len - j * kBN;               // frames of the clip in this block
-            if (live < kBN) {
-                // rows past the clip may hold anything (NaN included): P is 0 there, 0 * NaN is not
-                uint8_t* vt = smem + kOffV + st * kKV;
-                for (int i = lane; i < (kBN - live) * 8; i += 32)
-                    *reinterpret_cast<uint4*>(vt + (live + (i >> 3)) * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
-                fence_proxy_async_smem();
+        // O_X += P_X V of block j (the block's V in stage st); the first block overwrites O_X
+        auto issue_pv = [&](int x, int j, int st) -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarPFull + x], gx[x] & 1))) return false;
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t pa = tmem + kColS + x * kBN;
+                const uint32_t vb = sbase + kOffV + st * kKV;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_f16_ts(tmem + kColO + x * kD, pa + kk * 8, umma_desc_sw128(vb + kk * 16 * 128, kKV, 1024),
+                                kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
             }
             __syncwarp();
-            // the first PV of a tile overwrites O: the previous tile's epilogue must have read it
-            if (j == 0 && k > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarOEmpty], (k - 1) & 1)))) return;
-            for (int half = 0; half < 2; ++half) {
-                if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPFull + 2 * half + (g & 1)], (g >> 1) & 1))))
-                    return;
+            ++gx[x];
+            return true;
+        };
+        int r = 0, g = 0;
+        for (int k = 0; ok; ++k) {
+            const int t = snake_unit(k, c, G);
+            Unit un;
+            if (t >= total || !unit_at(t, r, slen, order, cum, B, un)) break;
+            const int qs = k & 1;
+            const int ntile = un.live_b ? 2 : 1;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarQFull + qs], (k >> 1) & 1)))) break;
+            // S of block 0 for each tile (S_X is free: the previous unit's PV_X were issued before)
+            {
+                const int st = g % kStages;
+                if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarKFull + st], (g / kStages) & 1)))) break;
+                for (int x = 0; x < ntile; ++x) issue_qk(x, qs, st);
                 if (lane == 0) {
-                    tc_fence_after();
-                    const uint32_t pa = tmem + kColS + (g & 1) * kBN + half * 32;
-                    const uint32_t vb = sbase + kOffV + st * kKV + half * 32 * 128;
-#pragma unroll
-                    for (int kk = 0; kk < 2; ++kk)
-                        umma_f16_ts(tmem + kColO + half * kD, pa + kk * 8,
-                                    umma_desc_sw128(vb + kk * 16 * 128, kKV, 1024), kIdescPV,
-                                    (j > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(&bars[kBarPvDone + half]);
+                    umma_commit(&bars[kBarKEmpty + st]);
+                    if (un.nblk == 1) umma_commit(&bars[kBarQEmpty + qs]);
                 }
                 __syncwarp();
             }
-            if (lane == 0) {
-                umma_commit(&bars[kBarVEmpty + st]);
-                if (j == tl.nblk - 1) umma_commit(&bars[kBarODone]);
-            }
-            __syncwarp();
-        };
-        // walk the blocks of all tiles of this CTA, QK one block ahead of PV
-        int r = 0, k = 0, j = 0, g = 0;
-        Tile cur, nt;
-        bool have = tile_at(snake_tile(0, c, G), r, slen, order, cum, B, cur);
-        if (have) issue_qk(0, 0, 0, cur);
-        while (have && ok) {
-            int nk = k, nj = j + 1;
-            bool more = true;
-            if (nj == cur.nblk) {
-                nk = k + 1;
-                nj = 0;
-                const int t = snake_tile(nk, c, G);
-                more = t < total && tile_at(t, r, slen, order, cum, B, nt);
-            } else {
-                nt = cur;
-            }
-            if (more) {
-                issue_qk(nk, nj, g + 1, nt);
+            // per block j: PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1) -- tile A's next scores are on their
+            // way while tile B's softmax still runs (QK_X(j+1) reuses S_X after PV_X(j) read P_X(j))
+            for (int j = 0; j < un.nblk && ok; ++j, ++g) {
+                const int st = g % kStages;
+                const int st1 = (g + 1) % kStages;
+                const bool more = j + 1 < un.nblk;
+                if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarVFull + st], (g / kStages) & 1)))) break;
+                const int live = un.len - j * kBN;           // frames of the clip in this block
+                if (live < kBN) {
+                    // rows past the clip may hold anything (NaN included): P is 0 there, 0 * NaN is not
+                    uint8_t* vt = smem + kOffV + st * kKV;
+                    for (int i = lane; i < (kBN - live) * 8; i += 32)
+                        *reinterpret_cast<uint4*>(vt + (live + (i >> 3)) * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+                    fence_proxy_async_smem();
+                }
+                __syncwarp();
+                if (more && !(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarKFull + st1], ((g + 1) / kStages) & 1))))
+                    break;
+                for (int x = 0; x < ntile && ok; ++x) {
+                    // the first PV of a unit overwrites O_X: the previous unit's epilogue must have read it
+                    if (j == 0 && kx[x] > 0 &&
+                        !(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarOEmpty + x], (kx[x] - 1) & 1))))
+                        break;
+                    if (!(ok = issue_pv(x, j, st))) break;
+                    if (more) issue_qk(x, qs, st1);
+                }
                 if (!ok) break;
+                if (lane == 0) {
+                    umma_commit(&bars[kBarVEmpty + st]);
+                    if (more) {
+                        umma_commit(&bars[kBarKEmpty + st1]);
+                        if (j + 1 == un.nblk - 1) umma_commit(&bars[kBarQEmpty + qs]);
+                    } else {
+                        for (int x = 0; x < ntile; ++x) umma_commit(&bars[kBarODone + x]);
+                    }
+                }
+                __syncwarp();
             }
-            issue_pv(k, j, g, cur);
-            if (!ok || !more) break;
-            k = nk;
-            j = nj;
-            cur = nt;
-            ++g;
+            for (int x = 0; x < ntile; ++x) ++kx[x];
         }
         if (!ok) {
             atomicExch(failed_flag, 1);
@@ -370,51 +374,75 @@ __global__ void __launch_bounds__(enc::kThreads, 2) encoder_attn_kernel(const __
             __syncwarp();
         }
     } else {
-        // ================================================= softmax + epilogue
+        // ================================================= softmax + epilogue of tile X
+        const int x = (warp - 2) >> 2;                  // 0: tile A (warps 2..5), 1: tile B (warps 6..9)
         const int quad = warp & 3;
-        const int half = (warp - 2) >> 2;               // keys 32*half .. +31 of every block
         const int rr = quad * 32 + lane;                // this thread's row of the tile
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-        const uint32_t col_o = kColO + half * kD;
+        const uint32_t col_s = kColS + x * kBN;
+        const uint32_t col_o = kColO + x * kD;
         const float sl2 = p.scale_log2;
-        float* xchg = reinterpret_cast<float*>(smem + kOffXchg);
         bool ok = true;
-        int r = 0, g = 0;
+        int r = 0, gxx = 0, kxx = 0;
         for (int k = 0; ok; ++k) {
-            const int t = snake_tile(k, c, G);
-            Tile tl;
-            if (t >= total || !tile_at(t, r, slen, order, cum, B, tl)) break;
+            const int t = snake_unit(k, c, G);
+            Unit un;
+            if (t >= total || !unit_at(t, r, slen, order, cum, B, un)) break;
+            if (x == 1 && !un.live_b) continue;          // tile B of this unit has no frame: not computed
             float m_ref = -INFINITY, e0 = 0.f, e1 = 0.f;
             // every tcgen05.ld/st is .sync.aligned and sits on warp-uniform control flow
-            for (int j = 0; j < tl.nblk; ++j, ++g) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + (g & 1)], (g >> 1) & 1));
+            for (int j = 0; j < un.nblk; ++j, ++gxx) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + x], gxx & 1));
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t col_s = kColS + (g & 1) * kBN + half * 32;
-                uint32_t v[32];
-                tmem_ld32(lane_base + col_s, v);
+                // keys 0..63 stay in registers; keys 64..127 are read twice (max, then exponentials), 32
+                // columns at a time, so no more than 96 scores are live.  P (keys 0..63 -> columns 0..31,
+                // keys 64..127 -> columns 32..63) only overwrites scores already held in registers.
+                const int nvalid = un.len - j * kBN;      // keys of the block inside the clip
+                uint32_t v[64];
+                tmem_ld32(lane_base + col_s, *reinterpret_cast<uint32_t(*)[32]>(v));
+                tmem_ld32(lane_base + col_s + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
                 tmem_wait_ld();
-                const int nvalid = tl.len - j * kBN - half * 32;   // keys of this half inside the clip
-                if (nvalid < 32) {
-                    // the last block: keys past the clip get score -inf, hence P = 0
+                // the last block: keys past the clip get score -inf, hence P = 0
+                auto mask32 = [&](uint32_t* w, int key0) {
+                    if (nvalid < key0 + 32) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (i >= nvalid) v[i] = 0xff800000u;
-                }
-                float mx[4];
+                        for (int i = 0; i < 32; ++i)
+                            if (key0 + i >= nvalid) w[i] = 0xff800000u;
+                    }
+                };
+                auto max32 = [&](const uint32_t* w) {
+                    float y[2];
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const uint32_t* w = v + 8 * q4;
-                    float x = max3(__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2]));
-                    x = max3(x, __uint_as_float(w[3]), __uint_as_float(w[4]));
-                    x = max3(x, __uint_as_float(w[5]), __uint_as_float(w[6]));
-                    mx[q4] = fmaxf(x, __uint_as_float(w[7]));
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const uint32_t* z = w + 16 * hh;
+                        float t = max3(__uint_as_float(z[0]), __uint_as_float(z[1]), __uint_as_float(z[2]));
+                        t = max3(t, __uint_as_float(z[3]), __uint_as_float(z[4]));
+                        t = max3(t, __uint_as_float(z[5]), __uint_as_float(z[6]));
+                        t = max3(t, __uint_as_float(z[7]), __uint_as_float(z[8]));
+                        t = max3(t, __uint_as_float(z[9]), __uint_as_float(z[10]));
+                        t = max3(t, __uint_as_float(z[11]), __uint_as_float(z[12]));
+                        t = max3(t, __uint_as_float(z[13]), __uint_as_float(z[14]));
+                        y[hh] = fmaxf(t, __uint_as_float(z[15]));
+                    }
+                    return fmaxf(y[0], y[1]);
+                };
+                mask32(v, 0);
+                mask32(v + 32, 32);
+                float bmax = fmaxf(max32(v), max32(v + 32));
+#pragma unroll
+                for (int c2 = 2; c2 < 4; ++c2) {
+                    uint32_t w[32];
+                    tmem_ld32(lane_base + col_s + 32 * c2, w);
+                    tmem_wait_ld();
+                    mask32(w, 32 * c2);
+                    bmax = fmaxf(bmax, max32(w));
                 }
-                const float bm = fmaxf(max3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
+                const float bm = bmax * sl2;
                 float alpha = 1.f;
                 bool rescale = false;
                 if (m_ref == -INFINITY) {
-                    m_ref = bm;              // first block with a key of this half: O_half is still empty
+                    m_ref = bm;              // first block: O_X is still empty
                 } else if (bm > m_ref + kLazyRescale) {
                     alpha = fast_exp2(m_ref - bm);
                     m_ref = bm;
@@ -422,11 +450,7 @@ __global__ void __launch_bounds__(enc::kThreads, 2) encoder_attn_kernel(const __
                 }
                 const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
                 if (__any_sync(0xffffffffu, rescale)) {
-                    // O_half must hold the PV of every earlier block of the tile before it is
-                    // rescaled (m_ref was finite before, so j >= 1; PV(g-2) is known complete)
-                    ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPvDone + half], (g - 1) & 1));
-                    if (!ok) break;
-                    tc_fence_after();
+                    // O_X holds PV_X of every earlier block: PV_X(j-1) was issued before QK_X(j)
                     e0 *= alpha;
                     e1 *= alpha;
 #pragma unroll
@@ -440,64 +464,60 @@ __global__ void __launch_bounds__(enc::kThreads, 2) encoder_attn_kernel(const __
                     }
                     tmem_wait_st();
                 }
-                uint32_t pk[16];
+                // P = 2^(s * scale_log2 - mu) as bf16 pairs; 32 keys -> 16 columns
+                auto exp32 = [&](const uint32_t* w, uint32_t col) {
+                    uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    float x0, x1;
-                    fma2(x0, x1, __uint_as_float(v[i]), __uint_as_float(v[i + 1]), sl2, sl2, -mu, -mu);
-                    const float s0 = fast_exp2(x0);
-                    const float s1 = fast_exp2(x1);
-                    add2(e0, e1, s0, s1);
-                    pk[i >> 1] = pack_bf16x2(s0, s1);
+                    for (int i = 0; i < 32; i += 2) {
+                        float x0, x1;
+                        fma2(x0, x1, __uint_as_float(w[i]), __uint_as_float(w[i + 1]), sl2, sl2, -mu, -mu);
+                        const float s0 = fast_exp2(x0);
+                        const float s1 = fast_exp2(x1);
+                        add2(e0, e1, s0, s1);
+                        pk[i >> 1] = pack_bf16x2(s0, s1);
+                    }
+                    tmem_st16(lane_base + col, pk);
+                };
+                exp32(v, col_s);
+                exp32(v + 32, col_s + 16);
+#pragma unroll
+                for (int c2 = 2; c2 < 4; ++c2) {
+                    uint32_t w[32];
+                    tmem_ld32(lane_base + col_s + 32 * c2, w);
+                    tmem_wait_ld();
+                    mask32(w, 32 * c2);
+                    exp32(w, col_s + 16 * c2);
                 }
-                tmem_st16(lane_base + col_s, pk);
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&bars[kBarPFull + 2 * half + (g & 1)]);
+                mbar_arrive(&bars[kBarPFull + x]);
             }
             if (!ok) break;
-            // ---- epilogue: O_0 and O_1 are complete once every MMA of the tile is
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarODone], k & 1));
+            // ---- epilogue: O_X is complete once every MMA of the unit is
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarODone + x], kxx & 1));
             if (!ok) break;
             tc_fence_after();
-            uint32_t oa[32], ob[32];
-            tmem_ld32(lane_base + kColO + half * 32, oa);          // dims 32*half .. +31 from O_0
-            tmem_ld32(lane_base + kColO + kD + half * 32, ob);     // and from O_1
+            uint32_t oa[64];
+            tmem_ld32(lane_base + col_o, *reinterpret_cast<uint32_t(*)[32]>(oa));
+            tmem_ld32(lane_base + col_o + 32, *reinterpret_cast<uint32_t(*)[32]>(oa + 32));
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(&bars[kBarOEmpty]);                        // the next tile may overwrite O
-            float* xm = xchg + (k & 1) * 2 * 2 * kRows;             // [half][max, sum][row]
-            xm[(half * 2 + 0) * kRows + rr] = m_ref;
-            xm[(half * 2 + 1) * kRows + rr] = e0 + e1;
-            // a bounded wait (not a named barrier): a softmax warp that gave up never hangs the others
-            mbar_arrive(&bars[kBarXchg + (k & 1)]);
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarXchg + (k & 1)], (k >> 1) & 1));
-            if (!ok) break;
-            const float m_oth = xm[((half ^ 1) * 2 + 0) * kRows + rr];
-            const float e_oth = xm[((half ^ 1) * 2 + 1) * kRows + rr];
-            const int tt = tl.qt * kRows + rr;
-            if (tt < tl.len) {
-                // O = (2^(m0-M) O_0 + 2^(m1-M) O_1) / (2^(m0-M) l_0 + 2^(m1-M) l_1)
-                const float m0 = half == 0 ? m_ref : m_oth, m1 = half == 0 ? m_oth : m_ref;
-                const float l0 = half == 0 ? e0 + e1 : e_oth, l1 = half == 0 ? e_oth : e0 + e1;
-                const float M = fmaxf(m0, m1);                  // finite for a live row (key 0 is in half 0)
-                const float a0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - M);
-                const float a1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - M);
-                const float l = l0 * a0 + l1 * a1;
+            mbar_arrive(&bars[kBarOEmpty + x]);                    // the next unit may overwrite O_X
+            ++kxx;
+            const int tt = un.u * kUnitRows + x * kRows + rr;
+            if (tt < un.len) {
+                const float l = e0 + e1;
                 const float inv = 1.f / l;
-                const float c0 = a0 * inv, c1 = a1 * inv;
-                uint4* orow = reinterpret_cast<uint4*>(
-                    p.o + ((static_cast<size_t>(tl.b) * p.S + tt) * H + tl.h) * kD + half * 32);
+                uint4* orow = reinterpret_cast<uint4*>(p.o + ((static_cast<size_t>(un.b) * p.S + tt) * H + un.h) * kD);
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    float f[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        f[i] = __uint_as_float(oa[8 * q4 + i]) * c0 + __uint_as_float(ob[8 * q4 + i]) * c1;
-                    orow[q4] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                                          pack_bf16x2(f[6], f[7]));
+                for (int q8 = 0; q8 < 8; ++q8) {
+                    const uint32_t* w = oa + 8 * q8;
+                    orow[q8] = make_uint4(pack_bf16x2(__uint_as_float(w[0]) * inv, __uint_as_float(w[1]) * inv),
+                                          pack_bf16x2(__uint_as_float(w[2]) * inv, __uint_as_float(w[3]) * inv),
+                                          pack_bf16x2(__uint_as_float(w[4]) * inv, __uint_as_float(w[5]) * inv),
+                                          pack_bf16x2(__uint_as_float(w[6]) * inv, __uint_as_float(w[7]) * inv));
                 }
-                if (half == 0) p.lse[(static_cast<size_t>(tl.b) * H + tl.h) * p.S + tt] = (M + __log2f(l)) * kLn2;
+                p.lse[(static_cast<size_t>(un.b) * H + un.h) * p.S + tt] = (m_ref + __log2f(l)) * kLn2;
             }
         }
         if (!ok) {
@@ -533,9 +553,9 @@ extern "C" ark_status ark_attn_encoder(const void* q, const void* k, const void*
     if (!q || !k || !v || !len || !o || !lse) return ARK_ERR_INVALID_ARG;
     if (B <= 0 || S <= 0 || H <= 0 || D <= 0 || !(scale > 0.f)) return ARK_ERR_INVALID_ARG;
     if (D != enc::kD || B > enc::kMaxClips) return ARK_ERR_UNSUPPORTED;
-    const long long qt = (S + enc::kRows - 1) / enc::kRows;
+    const long long units = (S + enc::kUnitRows - 1) / enc::kUnitRows;
     if (static_cast<long long>(B) * S >= (1LL << 31) || H > 65535 ||
-        static_cast<long long>(B) * H * qt >= (1LL << 31))
+        static_cast<long long>(B) * H * units >= (1LL << 31))
         return ARK_ERR_UNSUPPORTED;
     if (!enc_aligned16(q) || !enc_aligned16(k) || !enc_aligned16(v) || !enc_aligned16(o) ||
         (reinterpret_cast<uintptr_t>(lse) & 3u))
@@ -563,9 +583,9 @@ extern "C" ark_status ark_attn_encoder(const void* q, const void* k, const void*
         g_encoder_sms[dev] = sms;
         g_encoder_attr[dev] = true;
     }
-    // persistent: two CTAs per SM, at most one per possible tile
-    const long long tiles_max = static_cast<long long>(B) * H * qt;
-    const int grid = static_cast<int>(tiles_max < 2LL * g_encoder_sms[dev] ? tiles_max : 2LL * g_encoder_sms[dev]);
+    // persistent: one CTA per SM, at most one per possible unit
+    const long long units_max = static_cast<long long>(B) * H * units;
+    const int grid = static_cast<int>(units_max < g_encoder_sms[dev] ? units_max : g_encoder_sms[dev]);
     encoder_attn_kernel<<<grid, enc::kThreads, enc::kSmemBytes, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
 }
