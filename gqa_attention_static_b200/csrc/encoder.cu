@@ -395,8 +395,8 @@ __global__ void __launch_bounds__(enc::kThreads, 1) encoder_attn_kernel(const __
                 ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + x], gxx & 1));
                 if (!ok) break;
                 tc_fence_after();
-                // keys 0..63 stay in registers; keys 64..127 are read twice (max, then exponentials), 32
-                // columns at a time, so no more than 96 scores are live.  P (keys 0..63 -> columns 0..31,
+                // keys 0..63 stay in registers; keys 64..127 are read twice (for the max 32 columns at a
+                // time, then for the exponentials), so no more than 96 scores are live.  P (keys 0..63 -> columns 0..31,
                 // keys 64..127 -> columns 32..63) only overwrites scores already held in registers.
                 const int nvalid = un.len - j * kBN;      // keys of the block inside the clip
                 uint32_t v[64];
@@ -480,13 +480,16 @@ __global__ void __launch_bounds__(enc::kThreads, 1) encoder_attn_kernel(const __
                 };
                 exp32(v, col_s);
                 exp32(v + 32, col_s + 16);
-#pragma unroll
-                for (int c2 = 2; c2 < 4; ++c2) {
-                    uint32_t w[32];
-                    tmem_ld32(lane_base + col_s + 32 * c2, w);
+                {
+                    // keys 64..127 again, both chunks behind one wait (keys 0..63 are no longer live)
+                    uint32_t w[64];
+                    tmem_ld32(lane_base + col_s + 64, *reinterpret_cast<uint32_t(*)[32]>(w));
+                    tmem_ld32(lane_base + col_s + 96, *reinterpret_cast<uint32_t(*)[32]>(w + 32));
                     tmem_wait_ld();
-                    mask32(w, 32 * c2);
-                    exp32(w, col_s + 16 * c2);
+                    mask32(w, 64);
+                    mask32(w + 32, 96);
+                    exp32(w, col_s + 32);
+                    exp32(w + 32, col_s + 48);
                 }
                 tmem_wait_st();
                 tc_fence_before();
