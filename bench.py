@@ -70,7 +70,7 @@ QKV_TRAFFIC = {
 # Per-launch DRAM traffic of the encoder attention kernel (one layer of the encoder batch)
 # from an ncu --set full capture, keyed the same way.
 ENCODER_TRAFFIC = {
-    "1c03b40e4781186eaf749a42e344400882142a09be1bd50caa849ab8ddb7ce20": 62.4896e6 + 2.68032e6,
+    "f6de4adf9ccc481b5f7f0ffc735ae7e41ecb4b29e7b1ca4b1f9b5e15324fa659": 64.04736e6 + 2.65472e6,
 }
 
 
