@@ -351,12 +351,73 @@ def run_reference_encoder(args):
     print(json.dumps(line), flush=True)
 
 
+def run_reference_qkv(args):
+    """The oracle's projection + RoPE + delta write on the host cores: each step is
+    one layer over a bounded sample of the workload's live token rows (all 32 of a
+    decode step; 64 of the prefill batch), layers cycled."""
+    import numpy as np
+    import torch
+    cores = os.cpu_count() or 1
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    import oracle
+    from gqa_attention_static_b200 import workloads as W
+    oracle.build()
+    bits = lambda x: x.contiguous().view(torch.int16).numpy().view(np.uint16)
+    if args.config == "qkv_decode":
+        base = W.cfg_ragged_decode(layers=1)
+        rows = [(b, 0) for b in range(base.B)]
+        desc = "decode step B=32 (ragged batch), hidden 2048 -> 16+2+2 heads x 128, 36 layers"
+    else:
+        base = W.cfg_prefill(layers=1)
+        live = [(b, t) for b in range(base.B) for t in range(int(base.n_new[b]))]
+        rng = np.random.default_rng(0)
+        rows = [live[i] for i in rng.choice(len(live), 64, replace=False)]
+        desc = "coalesced prefill B=16 L U[20,387] S=387, hidden 2048 -> 16+2+2 heads x 128, 36 layers"
+    B, S, T = base.B, base.q[0].shape[1], base.T
+    pos = np.array([int(base.pos0[b]) + t for b, t in rows], np.int32)
+    layers = []
+    for l in range(4):
+        w, bias = W.make_qkv_weights(1000 + l)
+        x = bits(W.make_hidden(2000 + l, B, S))
+        xs = np.stack([x[b, t] for b, t in rows])[:, None, :]
+        layers.append((xs, bits(w), bits(bias)))
+    ck = np.zeros((len(rows), T, 2, 128), np.uint16)
+    cv = np.zeros((len(rows), T, 2, 128), np.uint16)
+    ones = np.ones(len(rows), np.int32)
+
+    def step(i):
+        xs, w, bias = layers[i % len(layers)]
+        oracle.qkv_rope_append(xs, w, bias, ck, cv, pos, ones, 16, 2)
+
+    for i in range(max(1, args.warmup)):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    el = time.perf_counter() - t0
+    v = len(rows) * args.steps / el
+    sample = (f"each step = projection + RoPE + delta write of ONE layer over {len(rows)} live token rows of: "
+              f"{desc} (4 distinct layers cycled); fp64 oracle; token-layers/s")
+    line = {"impl": "reference",
+            "metric": "fused Q/K/V projection + RoPE + delta write, token-layers/s (1xB200); % of roofline",
+            "value": v, "unit": "token-layers/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic (random-init weights)", "config": {"workload": desc},
+            "cpu_baseline": {"value": v, "unit": "token-layers/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": "token-layers/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
         return
     if args.config == "encoder":
         run_reference_encoder(args)
+        return
+    if args.config in ("qkv_decode", "qkv_prefill"):
+        run_reference_qkv(args)
         return
     r = OracleRunner(args.config, args.mode, kv=args.kv)
     for _ in range(max(1, args.warmup)):
