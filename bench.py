@@ -55,22 +55,22 @@ DECODE_TRAFFIC = {
 # prefill workload) from an ncu --set full capture, keyed the same way.
 PREFILL_TRAFFIC = {
     # one 16-layer launch of the coalesced prefill (read 332.35 MB + write 185.23 MB) / 16
-    "82d36dee9a26219530cce144be51941b9b67aa54cb2d787cce86b47d539d46fb": (332.350976e6 + 185.234688e6) / 16,
+    "2c8173635d520a21840a02bbb4ccc3d051ffc242c7595b1d02691730f9a13e6c": (332.350976e6 + 185.234688e6) / 16,
 }
 
 
 # Per-launch DRAM traffic of the projection kernel (one layer) from ncu --set full
 # captures of the two projection workloads, keyed by source hash and workload.
 QKV_TRAFFIC = {
-    ("7ba1c3300cd72423b0759df4608c6a375ea573145e282d46291568ca38ad809d", "qkv_decode"): 10.668288e6 + 0,
-    ("7ba1c3300cd72423b0759df4608c6a375ea573145e282d46291568ca38ad809d", "qkv_prefill"): 36.077568e6 + 0.54272e6,
+    ("49e18cbfa343066580088a60cf12d45db947e4a0f28b0d0a44eaf3934a14eaed", "qkv_decode"): 10.668288e6 + 0,
+    ("49e18cbfa343066580088a60cf12d45db947e4a0f28b0d0a44eaf3934a14eaed", "qkv_prefill"): 36.077568e6 + 0.54272e6,
 }
 
 
 # Per-launch DRAM traffic of the encoder attention kernel (one layer of the encoder batch)
 # from an ncu --set full capture, keyed the same way.
 ENCODER_TRAFFIC = {
-    "f6de4adf9ccc481b5f7f0ffc735ae7e41ecb4b29e7b1ca4b1f9b5e15324fa659": 64.04736e6 + 2.65472e6,
+    "c9a95e526155cc2b96648ff6961d41d4db8aa6cb1fc2d46f91b176f748b1f761": 64.04736e6 + 2.65472e6,
 }
 
 

@@ -39,6 +39,8 @@
 #include "common.cuh"
 #include "tma_host.h"
 
+#include <mutex>
+
 namespace ark {
 namespace enc {
 
@@ -545,6 +547,7 @@ namespace {
 
 bool enc_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+std::mutex g_encoder_mu;       // guards the per-device set-up below (first calls may come from several threads)
 bool g_encoder_attr[64];
 int g_encoder_sms[64];
 
@@ -576,19 +579,24 @@ extern "C" ark_status ark_attn_encoder(const void* q, const void* k, const void*
     prm.scale_log2 = scale * kLog2e;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARK_ERR_CUDA;
-    if (!g_encoder_attr[dev]) {
-        if (cudaFuncSetAttribute(encoder_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, enc::kSmemBytes) !=
-            cudaSuccess)
-            return ARK_ERR_CUDA;
-        int sms = 0;
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-            return ARK_ERR_CUDA;
-        g_encoder_sms[dev] = sms;
-        g_encoder_attr[dev] = true;
+    int sms = 0;
+    {
+        std::lock_guard<std::mutex> lk(g_encoder_mu);
+        if (!g_encoder_attr[dev]) {
+            if (cudaFuncSetAttribute(encoder_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     enc::kSmemBytes) != cudaSuccess)
+                return ARK_ERR_CUDA;
+            int n = 0;
+            if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+                return ARK_ERR_CUDA;
+            g_encoder_sms[dev] = n;
+            g_encoder_attr[dev] = true;
+        }
+        sms = g_encoder_sms[dev];
     }
     // persistent: one CTA per SM, at most one per possible unit
     const long long units_max = static_cast<long long>(B) * H * units;
-    const int grid = static_cast<int>(units_max < g_encoder_sms[dev] ? units_max : g_encoder_sms[dev]);
+    const int grid = static_cast<int>(units_max < sms ? units_max : sms);
     encoder_attn_kernel<<<grid, enc::kThreads, enc::kSmemBytes, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
 }

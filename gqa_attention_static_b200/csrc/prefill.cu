@@ -54,6 +54,8 @@
 #include "common.cuh"
 #include "tma_host.h"
 
+#include <mutex>
+
 namespace ark {
 namespace pf {
 
@@ -605,6 +607,7 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+std::mutex g_prefill_mu;       // guards the per-device set-up below (first calls may come from several threads)
 bool g_prefill_attr[64];
 
 }  // namespace
@@ -649,13 +652,16 @@ ark_status launch_prefill(const void* const* q, const void* const* cache_k, cons
     prm.scale_log2 = scale * kLog2e;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARK_ERR_CUDA;
-    if (!g_prefill_attr[dev]) {
-        if (cudaFuncSetAttribute(prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 pf::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 pf::kSmemBytes) != cudaSuccess)
-            return ARK_ERR_CUDA;
-        g_prefill_attr[dev] = true;
+    {
+        std::lock_guard<std::mutex> lk(g_prefill_mu);
+        if (!g_prefill_attr[dev]) {
+            if (cudaFuncSetAttribute(prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     pf::kSmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     pf::kSmemBytes) != cudaSuccess)
+                return ARK_ERR_CUDA;
+            g_prefill_attr[dev] = true;
+        }
     }
     const long long ctas = static_cast<long long>(Hkv) * B * ((S + pf::kPos - 1) / pf::kPos) * n;
     if (ctas >= (1LL << 31)) return ARK_ERR_UNSUPPORTED;

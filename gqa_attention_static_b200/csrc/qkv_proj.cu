@@ -33,6 +33,8 @@
 #include "common.cuh"
 #include "tma_host.h"
 
+#include <mutex>
+
 namespace ark {
 namespace qp {
 
@@ -388,6 +390,7 @@ namespace {
 
 bool qp_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+std::mutex g_qp_mu;            // guards the per-device set-up below (first calls may come from several threads)
 bool g_qp_attr[64];
 int g_qp_sms[64];
 int g_qp_clusters[64][4];    // clusters of 2, 4, 8 CTAs that can be resident at once (0: unknown)
@@ -400,6 +403,7 @@ ark_status launch_qkv(qp::Params& prm, const void* x, const void* w, int M, int 
     prm.N = N;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARK_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_qp_mu);     // held through the split choice (it fills g_qp_clusters)
     if (!g_qp_attr[dev]) {
         if (cudaFuncSetAttribute(qkv_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, qp::kSmemBytes) !=
             cudaSuccess)
