@@ -35,6 +35,15 @@
  * to bf16, round-to-nearest-even.  With bf16 inputs and fp32 table entries the
  * products are exact in fp64.
  *
+ * Two neighbours of the decoder attention, for the tests of their kernels:
+ *   - ora_attention_bidir: the audio encoder's bidirectional multi-head
+ *     attention ("Inside ARK-ASR-3B's Whisper and Qwen architecture",
+ *     components; reading: 20 heads of 64, every frame of a clip attends to
+ *     every frame of the same clip, q and k already rotated).
+ *   - ora_qkv_proj: the Q/K/V projections in front of the attention ("ARK-ASR-3B
+ *     -- INT8 ONNX" model card, Qwen2 decoder, hidden 2048) as one Linear over
+ *     the concatenated weight, the sum in double and one rounding to bf16.
+ *
  * Every function here is a direct, unblocked statement of its definition.
  */
 #include <math.h>
