@@ -41,25 +41,33 @@ namespace qp {
 constexpr int kBM = 128;                 // token rows per tile (MMA M)
 constexpr int kBN = 128;                 // output features per tile: one head (MMA N)
 constexpr int kBK = 64;                  // K chunk: 64 bf16 = one 128-byte swizzle row
-constexpr int kStages = 3;
 constexpr int kTileA = kBM * 128;        // 16 KB
 constexpr int kTileB = kBN * 128;        // 16 KB
 constexpr int kStageBytes = kTileA + kTileB;
 constexpr int kThreads = 192;            // warp 0: TMA, warp 1: MMA, warps 2..5: epilogue
 
-constexpr int kOffBar = kStages * kStageBytes;
-constexpr int kBarFull = 0;              // [kStages]
-constexpr int kBarEmpty = kBarFull + kStages;
-constexpr int kBarDone = kBarEmpty + kStages;
-constexpr int kNumBars = kBarDone + 1;
-constexpr int kOffRows = kOffBar + kNumBars * 8;    // per tile row: int2 {destination offset / 8 or -1, pos}
-constexpr int kOffBias = kOffRows + kBM * 8;           // this head's 128 bias values, fp32
-constexpr int kOffTmemPtr = kOffBias + kBN * 4;
-constexpr int kOffFlag = kOffTmemPtr + 8;
-constexpr int kSmemBytes = kOffFlag + 8;
 constexpr int kPartStride = 132;         // floats per row of a partial tile in shared memory (16-byte rows,
                                          // conflict-free float4 stores of 8 consecutive rows)
-static_assert(kBM * kPartStride * 4 <= kOffBar, "partial tile fits in the stage buffers");
+
+// Shared memory of a CTA with an S-stage ring: 3 stages (two CTAs per SM) when the tiles fill the
+// GPU, 6 stages (one CTA per SM, more of a CTA's share of K in flight at once) when K is split.
+template <int S>
+struct Layout {
+    static constexpr int kStages = S;
+    static constexpr int kOffBar = S * kStageBytes;
+    static constexpr int kBarFull = 0;                          // [S]
+    static constexpr int kBarEmpty = kBarFull + S;              // [S]
+    static constexpr int kBarDone = kBarEmpty + S;
+    static constexpr int kNumBars = kBarDone + 1;
+    static constexpr int kOffRows = kOffBar + kNumBars * 8;     // per tile row: int2 {destination / 8 or -1, pos}
+    static constexpr int kOffBias = kOffRows + kBM * 8;         // this head's 128 bias values, fp32
+    static constexpr int kOffTmemPtr = kOffBias + kBN * 4;
+    static constexpr int kOffFlag = kOffTmemPtr + 8;
+    static constexpr int kSmemBytes = kOffFlag + 8;
+    static_assert(kBM * kPartStride * 4 <= kOffBar, "partial tile fits in the stage buffers");
+};
+constexpr int kStagesWide = 3;           // many tiles
+constexpr int kStagesSplit = 6;          // K split over a cluster
 constexpr int kMaxSplit = 8;             // portable cluster size
 constexpr uint32_t kTmemCols = 128;
 
@@ -101,8 +109,19 @@ __device__ __forceinline__ float4 ld_dsmem_f4(const void* local, uint32_t rank) 
 
 }  // namespace qp
 
-__global__ void __launch_bounds__(qp::kThreads, 2) qkv_proj_kernel(const __grid_constant__ qp::Params p) {
+template <int S>
+__global__ void __launch_bounds__(qp::kThreads, S <= 3 ? 2 : 1) qkv_proj_kernel(const __grid_constant__ qp::Params p) {
     using namespace qp;
+    constexpr int kStages = Layout<S>::kStages;
+    constexpr int kOffBar = Layout<S>::kOffBar;
+    constexpr int kBarFull = Layout<S>::kBarFull;
+    constexpr int kBarEmpty = Layout<S>::kBarEmpty;
+    constexpr int kBarDone = Layout<S>::kBarDone;
+    constexpr int kNumBars = Layout<S>::kNumBars;
+    constexpr int kOffRows = Layout<S>::kOffRows;
+    constexpr int kOffBias = Layout<S>::kOffBias;
+    constexpr int kOffTmemPtr = Layout<S>::kOffTmemPtr;
+    constexpr int kOffFlag = Layout<S>::kOffFlag;
     extern __shared__ __align__(1024) uint8_t smem[];
     // the next launch (the next layer's projection, launched with programmatic stream
     // serialisation) may start streaming its weights now; it reads its x and writes its
@@ -393,7 +412,27 @@ bool qp_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u)
 std::mutex g_qp_mu;            // guards the per-device set-up below (first calls may come from several threads)
 bool g_qp_attr[64];
 int g_qp_sms[64];
-int g_qp_clusters[64][4];    // clusters of 2, 4, 8 CTAs that can be resident at once (0: unknown)
+int g_qp_clusters[64][4];    // clusters of 2, 4, 8 six-stage CTAs that can be resident at once (0: unknown)
+
+template <int S>
+ark_status launch_kernel(const qp::Params& prm, int M, int N, int split, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(N / qp::kBN, (M + qp::kBM - 1) / qp::kBM, split);
+    cfg.blockDim = dim3(qp::kThreads);
+    cfg.dynamicSmemBytes = qp::Layout<S>::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = static_cast<unsigned>(split);
+    cfg.attrs = attr;
+    cfg.numAttrs = split > 1 ? 2 : 1;
+    if (cudaLaunchKernelEx(&cfg, qkv_proj_kernel<S>, prm) != cudaSuccess) return ARK_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
+}
 
 ark_status launch_qkv(qp::Params& prm, const void* x, const void* w, int M, int K, int N, cudaStream_t stream) {
     if (!kmajor_tensor_map(&prm.xmap, x, M, K, qp::kBM) || !kmajor_tensor_map(&prm.wmap, w, N, K, qp::kBN))
@@ -405,8 +444,10 @@ ark_status launch_qkv(qp::Params& prm, const void* x, const void* w, int M, int 
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARK_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_qp_mu);     // held through the split choice (it fills g_qp_clusters)
     if (!g_qp_attr[dev]) {
-        if (cudaFuncSetAttribute(qkv_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, qp::kSmemBytes) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(qkv_proj_kernel<qp::kStagesWide>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 qp::Layout<qp::kStagesWide>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(qkv_proj_kernel<qp::kStagesSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 qp::Layout<qp::kStagesSplit>::kSmemBytes) != cudaSuccess)
             return ARK_ERR_CUDA;
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
@@ -415,30 +456,26 @@ ark_status launch_qkv(qp::Params& prm, const void* x, const void* w, int M, int 
         g_qp_attr[dev] = true;
     }
     const int tiles = (N / qp::kBN) * ((M + qp::kBM - 1) / qp::kBM);
-    cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(qp::kThreads);
-    cfg.dynamicSmemBytes = qp::kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = 1;
-    attr[1].val.clusterDim.y = 1;
-    // split K over a cluster while every cluster of the launch can be resident at once (one wave),
-    // the CTAs fit two per SM and the chunks divide evenly
+    // split K over a cluster of six-stage CTAs (one per SM) while the split CTAs fit on the SMs, every
+    // cluster of the launch can be resident at once (one wave) and the chunks divide evenly
     int split = 1;
     const int nk = K / qp::kBK;
     for (int cand = 2, ci = 0; cand <= qp::kMaxSplit; cand *= 2, ++ci) {
-        if (nk % cand != 0 || static_cast<long long>(tiles) * cand > 2LL * g_qp_sms[dev]) break;
+        if (nk % cand != 0 || static_cast<long long>(tiles) * cand > g_qp_sms[dev]) break;
         if (g_qp_clusters[dev][ci] == 0) {
-            cudaLaunchConfig_t occ = cfg;
+            cudaLaunchConfig_t occ = {};
             occ.gridDim = dim3(1, 1, cand);
-            attr[1].val.clusterDim.z = static_cast<unsigned>(cand);
-            occ.attrs = attr + 1;
+            occ.blockDim = dim3(qp::kThreads);
+            occ.dynamicSmemBytes = qp::Layout<qp::kStagesSplit>::kSmemBytes;
+            cudaLaunchAttribute ca[1];
+            ca[0].id = cudaLaunchAttributeClusterDimension;
+            ca[0].val.clusterDim.x = 1;
+            ca[0].val.clusterDim.y = 1;
+            ca[0].val.clusterDim.z = static_cast<unsigned>(cand);
+            occ.attrs = ca;
             occ.numAttrs = 1;
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, qkv_proj_kernel, &occ) != cudaSuccess) {
+            if (cudaOccupancyMaxActiveClusters(&n, qkv_proj_kernel<qp::kStagesSplit>, &occ) != cudaSuccess) {
                 (void)cudaGetLastError();
                 n = -1;
             }
@@ -447,12 +484,8 @@ ark_status launch_qkv(qp::Params& prm, const void* x, const void* w, int M, int 
         if (g_qp_clusters[dev][ci] < tiles) break;
         split = cand;
     }
-    cfg.gridDim = dim3(N / qp::kBN, (M + qp::kBM - 1) / qp::kBM, split);
-    attr[1].val.clusterDim.z = static_cast<unsigned>(split);
-    cfg.attrs = attr;
-    cfg.numAttrs = split > 1 ? 2 : 1;
-    if (cudaLaunchKernelEx(&cfg, qkv_proj_kernel, prm) != cudaSuccess) return ARK_ERR_CUDA;
-    return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
+    if (split > 1) return launch_kernel<qp::kStagesSplit>(prm, M, N, split, stream);
+    return launch_kernel<qp::kStagesWide>(prm, M, N, 1, stream);
 }
 
 }  // namespace
