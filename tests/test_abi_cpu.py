@@ -138,3 +138,26 @@ def test_encoder_arg_checks(lib):
     assert enc(H=70000) == ops.ARK_ERR_UNSUPPORTED
     assert enc(v=FAKE_MIS) == ops.ARK_ERR_INVALID_ARG
     assert enc(lse=FAKE + 2) == ops.ARK_ERR_INVALID_ARG
+
+
+def test_qkv_arg_checks(lib):
+    def proj(x=FAKE, w=FAKE, bias=None, M=32, K=2048, N=2560, out=FAKE):
+        return lib.ark_attn_qkv_proj(x, w, bias, M, K, N, out, None, None)
+    assert proj(x=None) == ops.ARK_ERR_INVALID_ARG
+    assert proj(out=None) == ops.ARK_ERR_INVALID_ARG
+    assert proj(M=0) == ops.ARK_ERR_INVALID_ARG
+    assert proj(K=2000) == ops.ARK_ERR_INVALID_ARG          # K % 64
+    assert proj(N=2500) == ops.ARK_ERR_INVALID_ARG          # N % 128
+    assert proj(w=FAKE_MIS) == ops.ARK_ERR_INVALID_ARG
+    assert proj(bias=FAKE + 1) == ops.ARK_ERR_INVALID_ARG   # bf16 bias must be 2-byte aligned
+
+    def fused(x=FAKE, w=FAKE, pos0=FAKE, n_new=FAKE, B=32, S=1, T=512, Hq=16, Hkv=2, D=128, K=2048,
+              table=FAKE, q=FAKE, ck=FAKE, cv=FAKE):
+        return lib.ark_attn_qkv_rope_append(x, w, None, pos0, n_new, B, S, T, Hq, Hkv, D, K, table, q, ck, cv,
+                                            None, None)
+    assert fused(table=None) == ops.ARK_ERR_INVALID_ARG
+    assert fused(n_new=None) == ops.ARK_ERR_INVALID_ARG
+    assert fused(B=0) == ops.ARK_ERR_INVALID_ARG
+    assert fused(K=100) == ops.ARK_ERR_INVALID_ARG
+    assert fused(D=64) == ops.ARK_ERR_UNSUPPORTED
+    assert fused(ck=FAKE_MIS) == ops.ARK_ERR_INVALID_ARG
