@@ -345,8 +345,8 @@ ARK_API ark_status ark_attn_decode_fp8_layers(int L, const void* const* q, const
  *   lse[b,h,i] = ln sum_{j < len[b]} exp(scale <q[b,i,h,:], k[b,j,h,:]>)
  * Layouts: q, k, v [B,S,H,D] bf16 (16-byte aligned); len int32[B] (device);
  * o [B,S,H,D] bf16; lse [B,H,S] fp32.  Rows i >= len[b] are not written; len
- * outside [0, S] is clamped and sets ARK_DEV_BAD_KVLEN.  D != 64 returns
- * ARK_ERR_UNSUPPORTED.  tcgen05 MMAs (bf16 operands, fp32 accumulation in
+ * outside [0, S] is clamped and sets ARK_DEV_BAD_KVLEN.  D != 64 or more than
+ * 256 clips (B > 256) returns ARK_ERR_UNSUPPORTED.  tcgen05 MMAs (bf16 operands, fp32 accumulation in
  * tensor memory); the softmax weights are rounded to bf16 before P V.
  */
 ARK_API ark_status ark_attn_encoder(const void* q, const void* k, const void* v, const int32_t* len, int B, int S,
@@ -376,6 +376,11 @@ ARK_API ark_status ark_attn_encoder(const void* q, const void* k, const void* v,
  *   followed by ark_attn_append_rope.  Padded rows, and rows whose position
  *   falls outside [0, T) (ARK_DEV_BAD_POS), are not written; n_new outside
  *   [0, S] is clamped (ARK_DEV_BAD_KVLEN).  D != 128 returns ARK_ERR_UNSUPPORTED.
+ *
+ * Both are launched with programmatic stream serialisation: a launch may start
+ * streaming W while the kernel before it in the stream finishes, and reads x
+ * and writes its outputs only after that kernel has completed, so stream order
+ * is kept.  Few tiles (a decode step) split K over a thread-block cluster.
  */
 ARK_API ark_status ark_attn_qkv_proj(const void* x, const void* w, const void* bias, int M, int K, int N, void* out,
                                      uint32_t* d_status, cudaStream_t stream);
