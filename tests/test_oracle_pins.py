@@ -9,6 +9,7 @@ SGLang-Omni cookbook "ARK-ASR-3B" (introduction, Audio Handling, dtype).
 import math
 import os
 
+
 import numpy as np
 import pytest
 import torch
@@ -474,6 +475,89 @@ def test_e4m3_encode_matches_torch_in_range(oracle_lib):
     x = torch.clamp(x, -448.0, 448.0).float()
     ref = x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     assert np.array_equal(oracle.f32_to_e4m3(x.numpy()), ref)
+
+
+def _rn_binary(q, mant_bits: int, min_exp: int):
+    """Exact round-to-nearest-even of the rational q onto a binary grid with
+    mant_bits bits after the point and exponents >= min_exp (subnormals below
+    2^min_exp); no overflow handling.  Plain exponent/ulp arithmetic, written
+    from the IEEE definition, not a search."""
+    from fractions import Fraction
+    if q == 0:
+        return Fraction(0)
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1                                   # now 2^e <= a < 2^(e+1)
+    e = max(e, min_exp)
+    ulp = Fraction(2) ** (e - mant_bits)
+    m = a / ulp
+    lo = m.numerator // m.denominator
+    rem = m - lo
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and lo % 2 == 1):
+        lo += 1
+    v = lo * ulp
+    return v if q > 0 else -v
+
+
+def _e4m3_reference(x: float, scale: float) -> int:
+    """e4m3(fp32(x / scale)) by exact rational arithmetic: the fp64 quotient
+    (Python's correctly rounded float division), rounded to fp32, rounded to
+    e4m3 (nearest even, saturating at +-448), encoded from its exponent and
+    mantissa."""
+    from fractions import Fraction
+    q64 = x / float(np.float32(scale))
+    y = _rn_binary(Fraction(q64), 23, -126)              # fp32 (the quotients here stay in range)
+    sign = 0x80 if (y < 0 or (y == 0 and math.copysign(1.0, q64) < 0)) else 0
+    a = abs(y)
+    if a >= 448:
+        return sign | 0x7E
+    v = _rn_binary(a, 3, -6)
+    if v == 0:
+        return sign
+    if v >= 448:
+        return sign | 0x7E
+    e = v.numerator.bit_length() - v.denominator.bit_length()
+    if Fraction(2) ** e > v:
+        e -= 1
+    if e < -6:                                           # subnormal: multiples of 2^-9
+        return sign | int(v / Fraction(2) ** -9)
+    mant = int((v / Fraction(2) ** e - 1) * 8)
+    return sign | ((e + 7) << 3) | mant
+
+
+def test_quantize_e4m3_exact_including_double_rounding(oracle_lib):
+    """ora_quantize_e4m3 equals the exact e4m3(fp32(x / scale)) everywhere
+    tested, including quotients that sit within half an fp32 step of an e4m3
+    midpoint: there the fp32 rounding lands ON the midpoint and the tie goes
+    to the even code, while rounding the fp64 quotient straight to e4m3 would
+    go the other way -- a version that skipped the fp32 step fails here."""
+    from fractions import Fraction
+    pos = oracle.e4m3_to_f64(np.arange(0x7F, dtype=np.uint8))
+    xs, scales, flips = [], [], 0
+    for c in range(0x7E):
+        mid = (pos[c] + pos[c + 1]) / 2                  # exact in fp64 and fp32
+        for sc in (1.0, 0.5, 4.0):
+            for sgn in (1.0, -1.0):
+                for d in (2.0 ** -30, -(2.0 ** -30)):
+                    x = sgn * (mid + d * max(mid, 2.0 ** -9)) * sc    # power-of-two scale: exact quotient
+                    xs.append(x)
+                    scales.append(sc)
+                    # the exact quotient is off the midpoint, its fp32 rounding is the midpoint
+                    direct = _rn_binary(Fraction(x / sc), 3, -6)
+                    via32 = _rn_binary(_rn_binary(Fraction(x / sc), 23, -126), 3, -6)
+                    flips += int(direct != via32)
+    assert flips > 100                                   # the cases really discriminate
+    g = np.random.default_rng(17)
+    for sc in (0.0371, 0.1, 0.2, 1.7, 3.0e-3):
+        for v in np.concatenate([g.standard_normal(300) * m for m in (1e-4, 0.01, 1.0, 30.0)]):
+            xs.append(float(v))
+            scales.append(sc)
+    xs += [500.0, -1e6, 0.0, -0.0, 2.0 ** -12]
+    scales += [1.0, 1.0, 1.0, 1.0, 1.0]
+    for x, sc in zip(xs, scales):
+        got = int(oracle.quantize_e4m3(np.array([x]), sc)[0])
+        assert got == _e4m3_reference(x, sc), (x, sc, got, _e4m3_reference(x, sc))
 
 
 def test_append_fp8_within_half_code_of_fp64_rotation(oracle_lib):
