@@ -72,6 +72,7 @@ def compare(batch, layer=0, status_expected=0):
     (1, 5, 8, [3], [5]),                             # smaller than a tile and than a KV block
     (2, 130, 512, [0, 380], [130, 2]),               # two KV blocks, last one partial
     (1, 200, 2048, [1700], [200]),                   # long context: 15 KV blocks
+    (5, 33, 96, [0, 7, 31, 63, 40], [33, 0, 32, 33, 17]),   # empty request, unit = 32 rows + 1, odd positions
 ])
 def test_prefill_small_cases(oracle_lib, B, S, T, pos0, n_new):
     batch = W.make_batch(500 + S + T, B=B, S=S, T=T, pos0=pos0, n_new=n_new, garbage="nan")
@@ -88,6 +89,16 @@ def test_prefill_sweep_prompt(oracle_lib):
 def test_prefill_coalesced_batch_full_size(oracle_lib):
     """Coalesced prefill at its full size: 16 prompts of 20..387 rows, T=512."""
     batch = W.cfg_prefill(layers=1)
+    compare(batch)
+
+
+def test_prefill_many_requests(oracle_lib):
+    """More requests than a warp has lanes (the unit list's per-request counts
+    take two rounds), lengths of every residue mod 16 and 32."""
+    g = torch.Generator().manual_seed(93)
+    n_new = torch.randint(1, 70, (45,), generator=g).tolist()
+    pos0 = torch.randint(0, 60, (45,), generator=g).tolist()
+    batch = W.make_batch(93, B=45, S=70, T=130, pos0=pos0, n_new=n_new, garbage="nan")
     compare(batch)
 
 
@@ -159,9 +170,9 @@ def test_prefill_layers_matches_oracle(oracle_lib):
 
 
 def test_prefill_layers_across_launches_equals_single_layer_calls(oracle_lib):
-    """18 layers take two launches (16 + 2); every layer's output is bit for bit
+    """40 layers take two launches (20 + 20); every layer's output is bit for bit
     the single-layer call's (the same tile arithmetic), padded rows untouched."""
-    L = 18
+    L = 40
     batch = W.make_batch(511, B=2, S=20, T=64, pos0=[0, 37], n_new=[20, 9], layers=L)
     dev = "cuda"
     q = [x.to(dev).clone() for x in batch.q]
@@ -239,3 +250,58 @@ def test_prefill_rope_on_load_coalesced_full_size(oracle_lib):
         assert torch.equal(oa[l].view(torch.int16), ob[l].view(torch.int16)), f"layer {l}: o differs"
         assert torch.equal(torch.nan_to_num(la[l], nan=-7.0), torch.nan_to_num(lb[l], nan=-7.0))
         assert torch.equal(cka[l].view(torch.int16), ckb[l].view(torch.int16))
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_prefill_36_layers_one_launch_equals_single_layer_calls(oracle_lib, fused):
+    """The coalesced batch at full size over 36 layers in one launch, where every
+    CTA walks some 54 units through its rings (Q slots, K/V stages, the list
+    entries, the output staging), equals 36 single-layer calls (a CTA walks at
+    most two units there) bit for bit, padded rows untouched; two layers are
+    also compared with the oracle.  Both forms: q rotated by the append, and q
+    rotated as the prefill loads it."""
+    L = 36
+    batch = W.cfg_prefill(layers=L, device="cuda")
+    dev = "cuda"
+    B, S, Hq, D = batch.q[0].shape
+    table = ops.rope_table(batch.T)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ck = [x.clone() for x in batch.cache_k]
+    cv = [x.clone() for x in batch.cache_v]
+    q = [x.clone() for x in batch.q]
+    if fused:
+        ops.ark_attn_append_rope_kv_layers(batch.k_new, batch.v_new, ck, cv, batch.pos0, batch.n_new, table, Hq,
+                                           status)
+    else:
+        ops.ark_attn_append_rope_layers(q, batch.k_new, batch.v_new, ck, cv, batch.pos0, batch.n_new, table, status)
+    o = [torch.empty_like(x).view(torch.int16).fill_(SENTINEL).view(torch.bfloat16) for x in q]
+    lse = [torch.full((B, Hq, S), float("nan"), dtype=torch.float32, device=dev) for _ in q]
+    if fused:
+        ops.ark_attn_prefill_rope_layers(q, ck, cv, batch.pos0, batch.n_new, o, lse, SCALE, table, status)
+    else:
+        ops.ark_attn_prefill_layers(q, ck, cv, batch.pos0, batch.n_new, o, lse, SCALE, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for l in range(L):
+        o1 = torch.empty_like(q[l]).view(torch.int16).fill_(SENTINEL).view(torch.bfloat16)
+        l1 = torch.full((B, Hq, S), float("nan"), dtype=torch.float32, device=dev)
+        if fused:
+            ops.ark_attn_prefill_rope_layers([q[l]], [ck[l]], [cv[l]], batch.pos0, batch.n_new, [o1], [l1], SCALE,
+                                             table, status)
+        else:
+            ops.ark_attn_prefill(q[l], ck[l], cv[l], batch.pos0, batch.n_new, o1, l1, SCALE, status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert torch.equal(o[l].view(torch.int16), o1.view(torch.int16)), f"layer {l}"
+        assert torch.equal(torch.nan_to_num(lse[l], nan=-7.0), torch.nan_to_num(l1, nan=-7.0)), f"layer {l}"
+    for l in (0, 35):
+        cpu = lambda x: x.cpu()
+        one = W.Batch([cpu(batch.q[l])], [cpu(batch.k_new[l])], [cpu(batch.v_new[l])], [cpu(batch.cache_k[l])],
+                      [cpu(batch.cache_v[l])], cpu(batch.pos0), cpu(batch.n_new), batch.T, batch.S)
+        q_ref, ck_ref, cv_ref, o_ref, lse_ref = oracle_append_prefill(one)
+        assert np.array_equal(bits(ck[l]), ck_ref) and np.array_equal(bits(cv[l]), cv_ref)
+        for b in range(B):
+            n = int(batch.n_new[b])
+            check_o(f64(o[l])[b, :n], o_ref[b, :n], f"o layer {l} request {b}")
+            check_lse(f64(lse[l])[b, :, :n], lse_ref[b, :, :n], f"lse layer {l} request {b}")
+            assert np.all(bits(o[l])[b, n:] == SENTINEL)
