@@ -367,21 +367,22 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     uint64_t* qbar = bars + kSt;
     int* s_pref = reinterpret_cast<int*>(smem + kRingBytes + kQBytes + kBarBytes);   // [B + 1]
 
-    // ---- per CTA: prefix over the batch of the tiles per request (all KV heads)
-    if (warp == 0) tile_prefix(c, s_pref, lane, blockIdx.x == 0);
-    // the merge grid may be scheduled from here on (it waits for this grid's completion)
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (lane == 0) {
         for (int s = 0; s <= kSt; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
     }
+    // q, the cache rows and kv_len may come from the kernel before this one in
+    // the stream (the append, or a kernel that advances the lengths): with
+    // programmatic dependent launch this grid may be running already, so wait
+    // for that grid's completion and its writes before reading any of them (a
+    // no-op when there is no such dependency)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // ---- per CTA: prefix over the batch of the tiles per request (all KV heads)
+    if (warp == 0) tile_prefix(c, s_pref, lane, blockIdx.x == 0);
+    // the merge grid may be scheduled from here on (it waits for this grid's completion)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     fence_proxy_async_smem();
     __syncthreads();   // the last block-wide barrier: warps run independently from here
-    // q and the cache rows may come from the kernel before this one in the
-    // stream (the append): with programmatic dependent launch this grid may be
-    // running already, so wait here for that grid's completion and its writes
-    // (a no-op when there is no such dependency); the prefix above only read kv_len
-    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     const int per_layer = s_pref[c.B];
     const int N = per_layer * c.L;
@@ -758,10 +759,12 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_kernel(const __grid_con
     }
     // Never leave with copies in flight: a timed-out warp stops consuming, so
     // wait (bounded) for the tiles and query rows it issued but did not consume.
+    // (At most one query copy is in flight at a time, so waiting for the last
+    // one issued covers them all; a completed phase returns at once.)
     if (failed) {
         for (uint32_t q2 = pseq > kSt ? pseq - kSt : 0; q2 < pseq; ++q2)
             (void)mbar_wait(&bars[q2 % kSt], (q2 / kSt) & 1);
-        if (qissued > qseq) (void)mbar_wait(qbar, qseq & 1);
+        (void)mbar_wait(qbar, (qissued - 1) & 1);
     }
 }
 
@@ -881,11 +884,14 @@ struct DeviceInfo {
     int sms = 0, ctas_per_sm = 0;
 };
 
+std::mutex g_device_info_mu;    // guards the per-device tables below (first calls may come from several threads)
+
 template <int MaxL, bool Fp8>
 ark_status device_info(DeviceInfo& out) {
     static DeviceInfo table[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARK_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_device_info_mu);
     DeviceInfo& d = table[dev];
     if (d.sms == 0) {
         if (cudaFuncSetAttribute(decode_kernel<MaxL, Fp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1141,17 +1147,51 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocBytes];
 
 namespace {
 
+// The array's address belongs to the module loaded in one CUDA context: after
+// a device reset the next context loads the module again, possibly elsewhere.
+// So the cached address is keyed by the current context's unique id (driver
+// entry points looked up through the runtime; the library links no libcuda).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
 std::mutex g_scratch_mu;
 void* g_scratch_addr[64];
+unsigned long long g_scratch_ctx[64];
+
+bool current_context_id(unsigned long long* id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 ark_status scratch_address(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARK_ERR_CUDA;
+    // no context may be current yet on this thread's first CUDA call; the symbol
+    // lookup below makes the device's primary context current
+    unsigned long long ctx = 0;
+    const bool have_ctx = current_context_id(&ctx);
     std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
+    if (!have_ctx || !g_scratch_addr[dev] || g_scratch_ctx[dev] != ctx) {
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) return ARK_ERR_CUDA;
+        if (!have_ctx && !current_context_id(&ctx)) return ARK_ERR_CUDA;
         g_scratch_addr[dev] = ptr;
+        g_scratch_ctx[dev] = ctx;
     }
     *out = g_scratch_addr[dev];
     return ARK_OK;

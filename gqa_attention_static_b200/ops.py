@@ -548,7 +548,7 @@ def ark_attn_decode_fp8_layers(q: Sequence[torch.Tensor], cache_k, cache_v, k_sc
 
 def ark_attn_prefill_layers(q: Sequence[torch.Tensor], cache_k, cache_v, pos0, n_new, o, lse, scale: float,
                             status: Optional[torch.Tensor] = None, stream=None) -> None:
-    """ark_attn_prefill over L independent layers (up to 16 layers per launch)."""
+    """ark_attn_prefill over L independent layers (up to 36 layers per launch)."""
     L = len(q)
     if not (len(cache_k) == len(cache_v) == len(o) == len(lse) == L) or L == 0:
         raise ValueError("per-layer lists must have the same non-zero length")

@@ -27,7 +27,9 @@ class DecodeStep:
     Buffers (per layer lists, all on ``device``):
       q [B,1,Hq,D] (rotated in place), k_new/v_new [B,1,Hkv,D],
       cache_k/cache_v [B,T,Hkv,D], o [B,1,Hq,D], lse [B,Hq];
-    shared: pos0, n_new, kv_len int32[B], rotary table, workspace, status.
+    shared: pos0, n_new, kv_len int32[B], rotary table, workspace, status
+    (table, workspace, status and the o/lse lists are allocated here unless
+    passed in).
     With k_scale/v_scale (per layer fp32 [Hkv]) the caches are fp8 (uint8 e4m3
     codes) and the step uses the fp8 entry points.
     """
@@ -37,7 +39,10 @@ class DecodeStep:
                  n_new: torch.Tensor, kv_len: torch.Tensor, max_splits: int = 8,
                  mode: int = ops.ARK_LENGTH_AWARE, rope_theta: float = 1e6,
                  scale: Optional[float] = None, batched: bool = True,
-                 k_scale: Optional[List[torch.Tensor]] = None, v_scale: Optional[List[torch.Tensor]] = None):
+                 k_scale: Optional[List[torch.Tensor]] = None, v_scale: Optional[List[torch.Tensor]] = None,
+                 table: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                 status: Optional[torch.Tensor] = None, o: Optional[List[torch.Tensor]] = None,
+                 lse: Optional[List[torch.Tensor]] = None):
         self.q, self.k_new, self.v_new = q, k_new, v_new
         self.fp8 = cache_k[0].dtype == torch.uint8
         if self.fp8 and (k_scale is None or v_scale is None):
@@ -54,12 +59,15 @@ class DecodeStep:
         self.mode = mode
         self.batched = batched
         self.scale = scale if scale is not None else 1.0 / math.sqrt(self.D)
-        self.table = ops.rope_table(self.T, self.D, rope_theta, device=dev)
-        self.workspace = ops.decode_workspace(self.B, self.Hq, self.D, self.T, max_splits, device=dev,
-                                              layers=self.layers if batched else 1)
-        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
-        self.o = [torch.empty_like(x) for x in q]
-        self.lse = [torch.empty(self.B, self.Hq, dtype=torch.float32, device=dev) for _ in q]
+        # table, workspace, status and outputs may be shared between steps that run one after
+        # another on one stream (a decode loop over many positions)
+        self.table = table if table is not None else ops.rope_table(self.T, self.D, rope_theta, device=dev)
+        self.workspace = workspace if workspace is not None else ops.decode_workspace(
+            self.B, self.Hq, self.D, self.T, max_splits, device=dev, layers=self.layers if batched else 1)
+        self.status = status if status is not None else torch.zeros(1, dtype=torch.int32, device=dev)
+        self.o = o if o is not None else [torch.empty_like(x) for x in q]
+        self.lse = lse if lse is not None else [torch.empty(self.B, self.Hq, dtype=torch.float32, device=dev)
+                                                for _ in q]
 
     @property
     def min_tiles(self) -> int:
@@ -127,7 +135,7 @@ class DecodeStep:
 class PrefillStep:
     """Prefill of one prompt batch over L independent layers: RoPE + delta
     write of the prompt rows for all layers (one launch), then the causal
-    tcgen05 prefill of all layers (one launch per 16 layers; one launch per
+    tcgen05 prefill of all layers (one launch per 36 layers; one launch per
     layer with batched=False).
 
     Buffers (per layer lists): q [B,S,Hq,D] (rotated in place), k_new/v_new
@@ -154,8 +162,16 @@ class PrefillStep:
         self.o = [torch.empty_like(x) for x in q]
         self.lse = [torch.empty(self.B, self.Hq, self.S, dtype=torch.float32, device=dev) for _ in q]
 
+    # layers the library's prefill kernel takes per launch (kernel-parameter space)
+    LAYERS_PER_LAUNCH = 36
+
     def launches_per_step(self) -> int:
-        return 1 + ((self.layers + 15) // 16 if self.batched else self.layers)
+        """The append (one launch) and the prefill (one launch per 36 layers,
+        or one per layer with batched=False; the RoPE-on-load form is always
+        layer-batched)."""
+        if self.batched or self.fused_rope:
+            return 1 + -(-self.layers // self.LAYERS_PER_LAUNCH)
+        return 1 + self.layers
 
     def append(self, stream=None) -> None:
         if self.fused_rope:

@@ -19,7 +19,11 @@
  *     pointer must be 16-byte aligned.
  *   - The caller owns and allocates every buffer (tensors, workspace, RoPE
  *     table, status word).  The library allocates no device memory and keeps
- *     no per-call state.
+ *     no per-call state, with two stated exceptions: ark_attn_decode_noalloc
+ *     uses one fixed, file-scope device array (see there), and the host keeps
+ *     a process-wide cache of the TMA tensor maps it encodes, keyed by buffer
+ *     address and shape (a map describes only the address and shape, so a
+ *     buffer freed and reallocated at the same address reuses a valid map).
  *   - Calls are asynchronous on `stream` and enqueue kernels only (except
  *     ark_attn_rope_table_init, which copies from the host and synchronises).
  *   - Arguments the host can see are checked before anything is launched; a
@@ -143,7 +147,11 @@ ARK_API ark_status ark_attn_append_rope(void* q, const void* k_new, const void* 
  * int32[B] (device; the new row is already appended, so the query attends to
  * itself); o [B,1,Hq,D] bf16; lse [B,Hq] fp32 (natural log).
  * kv_len outside [0, T] is clamped and sets ARK_DEV_BAD_KVLEN; kv_len = 0
- * gives o = 0, lse = -inf.
+ * gives o = 0, lse = -inf.  The decode kernel is launched with programmatic
+ * dependent launch behind whatever kernel precedes it on `stream`; it waits
+ * for that kernel's completion before it reads q, the caches or kv_len, so
+ * the preceding kernel may write any of them (an append, or a kernel that
+ * advances the lengths on the device).
  * Workspace: ark_attn_decode_workspace_size(...) bytes (about 16 MB: two
  * partial slots for each of up to 2048 warps), 16-byte aligned, caller-owned,
  * required.  It needs no initialisation and carries nothing from one call to
@@ -186,9 +194,10 @@ ARK_API ark_status ark_attn_prefill(const void* q, const void* cache_k, const vo
  * device pointers (read during the call; the array itself may be freed when
  * the call returns).  All layers share B, S, T, the positions/lengths and the
  * rotary table.  Each layer's tensors follow the single-layer layouts above.
- * ark_attn_prefill_layers runs the tiles of up to 16 layers in one launch
- * (longer lists take several launches, in order on `stream`), so that the GPU
- * does not drain at every layer boundary.
+ * ark_attn_prefill_layers runs the work of up to 36 layers in one launch of
+ * its persistent kernel (longer lists take several launches of near-equal
+ * size, in order on `stream`), so that the GPU does not drain at every layer
+ * boundary.
  * The decode workspace is ark_attn_decode_layers_workspace_size(L, ...) bytes
  * under the same rules.  Meant for callers that hold
  * several independent caches (the ARK-ASR-3B decoder has 36 layers), and for
@@ -245,6 +254,8 @@ ARK_API ark_status ark_attn_combine(const float* o_part, const float* lse_part, 
  * ARK_ERR_UNSUPPORTED beyond).
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * The address is cached per CUDA context: after a device reset the next call
+ * looks it up again (make that call, too, before any capture).
  * Nothing in the scratch needs initialising and no call allocates.  All calls
  * share the one array, so calls that can overlap on the GPU (different
  * streams, or graphs replayed concurrently) race: serialise them.
