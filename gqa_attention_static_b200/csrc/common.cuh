@@ -76,13 +76,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // Bounded wait for the phase with the given parity to complete.  Returns
-// false if it did not complete within kWaitLimitNs (or kMaxPolls polls).
+// false if it did not complete within LimitNs of the global timer (kWaitLimitNs
+// in every kernel of the library) or kMaxPolls polls, whichever comes first.
+template <uint64_t LimitNs = kWaitLimitNs>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1; i < kMaxPolls; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+        if ((i & 63) == 0 && globaltimer_ns() - t0 > LimitNs) return false;
     }
     return false;
 }
