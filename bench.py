@@ -1,7 +1,8 @@
 """Benchmark of the decode hot path: GQA attention over the static KV cache.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config ragged|single|long2048|long1024|prefill] [--mode aware|masked]
+                    [--config ragged|single|long2048|long1024|sweep|prefill|encoder|qkv_decode|qkv_prefill]
+                    [--mode aware|masked] [--kv bf16|fp8]
 
 A step is one pass of the whole decode path over one batch: for each of the
 36 layers, RoPE on the new q/k rows with the delta write into that layer's
@@ -11,11 +12,20 @@ valid lengths uniform in [40, 511] before the append (41..512 rows read),
 K/V with 1% x8 row outliers, 36 independent layers (604 MB of caches, larger
 than the 126 MB L2, so every step streams from HBM).
 
+The default run (N = 1) also measures the other workloads of the decoder's
+attention and reports them under "configs" in the same JSON line: the single
+decode step (B = 1), the batch-1 autoregressive sweep (50-row prefill, then
+461 decode steps), the coalesced prefill (16 prompts of 20..387 rows), and the
+long-cache batches (T = 2048 ragged, T = 1024 full) in the length-aware and
+masked-static modes side by side.  Each of them can also be run alone with
+--config.
+
 Timing: W untimed warm-up steps, then exactly K steps replayed from one CUDA
 graph, bracketed by a barrier and a device synchronisation, timed with CUDA
 events on the launching stream; max over ranks.  Rank 0 prints one JSON line.
 Multi-GPU runs are independent replicas (weak scaling, no collective on the
-data path).
+data path).  Roofline fractions are given against the measured copy
+bandwidth (MEASURED_PEAKS.json) and against the 8 TB/s HBM3e figure.
 
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload (the oracle is the only reference implementation there is).
@@ -38,7 +48,9 @@ if ROOT not in sys.path:
 
 METRIC = "decode-attn KV GB/s & tokens·layers/s (1×B200); % of HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0          # B200 HBM3e figure the decode target is stated against
 N_LAYERS = 36
+DECODE_CONFIGS = ("ragged", "single", "long2048", "long1024")
 
 # Per-launch DRAM traffic of the decode kernel from an ncu capture, keyed by the
 # sha256 of the kernel source it was taken on; reported as null once the source
@@ -54,8 +66,6 @@ DECODE_TRAFFIC = {
 # Per-launch DRAM traffic of the prefill kernel (one layer of the coalesced
 # prefill workload) from an ncu --set full capture, keyed the same way.
 PREFILL_TRAFFIC = {
-    # one 16-layer launch of the coalesced prefill (read 332.35 MB + write 185.23 MB) / 16
-    "2c8173635d520a21840a02bbb4ccc3d051ffc242c7595b1d02691730f9a13e6c": (332.350976e6 + 185.234688e6) / 16,
 }
 
 
@@ -75,29 +85,31 @@ ENCODER_TRAFFIC = {
 }
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="ragged",
-                    choices=["ragged", "single", "long2048", "long1024", "prefill", "encoder", "qkv_decode",
-                             "qkv_prefill"])
+                    choices=list(DECODE_CONFIGS) + ["sweep", "prefill", "encoder", "qkv_decode", "qkv_prefill"])
     ap.add_argument("--mode", default="aware", choices=["aware", "masked"])
     ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
                     help="cache format of the decode configurations: bf16, or fp8 E4M3 codes with per-head scales")
     ap.add_argument("--max-splits", type=int, default=8)
     ap.add_argument("--per-layer", action="store_true",
                     help="issue the single-layer calls layer by layer instead of the layer-batched calls")
-    ap.add_argument("--rope-on-load", action="store_true",
-                    help="prefill: K/V-only append, RoPE applied by the prefill kernel as it loads q")
+    ap.add_argument("--two-call-prefill", action="store_true",
+                    help="prefill: rotate q in the append (q read and written) instead of in the prefill kernel")
     ap.add_argument("--layers", type=int, default=None,
-                    help="encoder / qkv: layers per step (default 32 / 36; fewer only for profiler captures)")
+                    help="encoder / qkv / prefill: layers per step (default 32 / 36 / 36; fewer only for profiler "
+                         "captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="default run: skip the other workloads reported under \"configs\"")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def dist_env():
@@ -107,21 +119,42 @@ def dist_env():
     return world, rank, local
 
 
+WORKLOAD_DESC = {
+    "ragged": "ragged decode B=32 T=512 kv_len U[41,512] 1% x8 K/V row outliers, 36 layers",
+    "single": "single decode B=1 T=512 kv_len 65, 36 layers",
+    "long2048": "long decode B=32 T=2048 kv_len U[1501,2048], 36 layers",
+    "long1024": "long decode B=32 T=1024 full (kv_len 1024), 36 layers",
+    "sweep": "autoregressive sweep B=1 T=512: prefill of 50 rows (37 audio + 13 text), then 461 decode steps "
+             "(positions 50..510), fresh q/k/v per step, 36 layers",
+    "prefill": "coalesced causal prefill B=16 L U[20,387] S=387 T=512, 36 layers",
+}
+
+
 def make_workload(name: str, layers: int, device: str):
     from gqa_attention_static_b200 import workloads as W
     if name == "ragged":
         b = W.cfg_ragged_decode(layers=layers, device=device)
-        desc = "ragged decode B=32 T=512 kv_len U[41,512] 1% x8 K/V row outliers, 36 layers"
     elif name == "single":
         b = W.cfg_single_decode(layers=layers, device=device)
-        desc = "single decode B=1 T=512 kv_len 65, 36 layers"
     elif name == "long2048":
         b = W.cfg_long_decode(layers=layers, T=2048, device=device)
-        desc = "long decode B=32 T=2048 kv_len U[1501,2048], 36 layers"
-    else:
+    elif name == "long1024":
         b = W.cfg_long_decode(layers=layers, T=1024, device=device)
-        desc = "long decode B=32 T=1024 full (kv_len 1024), 36 layers"
-    return b, desc
+    else:
+        raise ValueError(f"not a decode workload: {name}")
+    return b, WORKLOAD_DESC[name]
+
+
+def decode_config(name: str, B: int, T: int, L: int, kv: str, mode: str, world: int) -> dict:
+    """The `config` of a decode workload's JSON line, the same for both arms."""
+    desc = WORKLOAD_DESC[name]
+    if kv == "fp8":
+        desc = desc.replace(" 1% x8 K/V row outliers", "") + ", fp8 E4M3 cache (per-head scales)"
+    return {"workload": desc, "batch": B, "max_total_len": T, "layers": L, "kv_cache": kv,
+            "mode": "masked-static" if mode == "masked" else "length-aware",
+            "l2": "inputs larger than L2 (%.0f MB of caches per step)" %
+                  (2 * L * B * T * 2 * 128 * (1 if kv == "fp8" else 2) / 1e6),
+            "parallelism": f"replicas x{world}"}
 
 
 def algorithmic_bytes(kv_len, B: int, kv: str = "bf16") -> int:
@@ -167,6 +200,23 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def hbm_roofline(achieved_gbs: float) -> dict:
+    """An HBM-bound kernel's fractions: of the measured copy bandwidth (or the
+    fallback when no measurement is present) and of the 8 TB/s HBM3e figure."""
+    peak, kind = measured_peaks()
+    return {"bound": "hbm", "achieved": achieved_gbs, "peak": peak, "unit": "GB/s", "frac": achieved_gbs / peak,
+            "peak_kind": kind, "spec_peak": SPEC_HBM_GBS, "frac_spec": achieved_gbs / SPEC_HBM_GBS}
 
 
 def src_hash(rel: str) -> str:
@@ -228,39 +278,58 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def encoder_config(L: int, lengths) -> dict:
+    return {"workload": "encoder attention B=8 clips of 150..1500 frames (S=1500), 20 heads x 64, %d layers" % L,
+            "lengths": list(lengths), "l2": "q/k/v/o of the layers (%.1f GB) larger than L2" % (L * 0.123)}
+
+
+def qkv_config(desc: str, rows: int, L: int) -> dict:
+    return {"workload": desc.replace("36 layers", f"{L} layers"), "rows": rows,
+            "l2": "weights of %d layers (%.0f MB) larger than L2" % (L, L * 2560 * 2048 * 2 / 1e6)}
+
+
+# ------------------------------------------------------------ the oracle arms ----
+# The fp64 oracle (test infrastructure) timed as it stands on this host's cores:
+# the cpu_baseline of the GPU line and the --impl reference arm.  Nothing here
+# runs on the GPU.
+
+def _bits(x):
+    import numpy as np
+    import torch
+    return x.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _oracle():
+    cores = os.cpu_count() or 1
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    import oracle
+    oracle.build()
+    return oracle
+
+
 class OracleRunner:
     """The fp64 oracle (as it stands) on this host's cores: whole decode
     layer-steps (RoPE + delta write + attention) over a bounded sample of the
     workload's layers.  OpenMP threads = all host cores."""
 
     def __init__(self, workload: str, mode: str, layers: int = 4, kv: str = "bf16"):
-        import numpy as np
-        import torch
-        cores = os.cpu_count() or 1
-        os.environ.setdefault("OMP_NUM_THREADS", str(cores))
-        import oracle
-        oracle.build()
-        self.oracle = oracle
-        self.cores = oracle.num_threads()
+        self.oracle = _oracle()
+        self.cores = self.oracle.num_threads()
         batch, self.desc = make_workload(workload, layers, "cpu")
-
-        def bits(x):
-            return x.contiguous().view(torch.int16).numpy().view(np.uint16)
-
         self.fp8 = (kv == "fp8")
         if self.fp8:
             fc = fp8_cache_for(batch, mode)
-            self.inputs = [(bits(batch.q[l]), bits(batch.k_new[l]), bits(batch.v_new[l]),
+            self.inputs = [(_bits(batch.q[l]), _bits(batch.k_new[l]), _bits(batch.v_new[l]),
                             fc.cache_k[l].numpy(), fc.cache_v[l].numpy(), fc.k_scale[l].numpy(),
                             fc.v_scale[l].numpy()) for l in range(layers)]
             self.desc = self.desc.replace(" 1% x8 K/V row outliers", "") + ", fp8 E4M3 cache"
         else:
-            self.inputs = [(bits(batch.q[l]), bits(batch.k_new[l]), bits(batch.v_new[l]),
-                            bits(batch.cache_k[l]), bits(batch.cache_v[l])) for l in range(layers)]
+            self.inputs = [(_bits(batch.q[l]), _bits(batch.k_new[l]), _bits(batch.v_new[l]),
+                            _bits(batch.cache_k[l]), _bits(batch.cache_v[l])) for l in range(layers)]
         self.pos0 = batch.pos0.numpy()
         self.n_new = batch.n_new.numpy()
         self.kv = batch.kv_len.numpy()
-        self.B = batch.B
+        self.B, self.T = batch.B, batch.T
         self.static = (mode == "masked")
         self.bytes_per_layer = algorithmic_bytes(self.kv, self.B, kv)
         self.i = 0
@@ -298,6 +367,112 @@ def cpu_baseline(workload: str, seconds: float, mode: str, kv: str = "bf16"):
             "tokens_layers_per_s": r.B * n / el}
 
 
+def _reference_line(args, metric, value, unit, el, config, sample, cores, dtype="f64", data="synthetic"):
+    return {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": data,
+            "config": config,
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def run_reference_decode(args):
+    r = OracleRunner(args.config, args.mode, kv=args.kv)
+    for _ in range(max(1, args.warmup)):
+        r.layer_step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r.layer_step()          # one step = one layer of the workload (bounded sample)
+    el = time.perf_counter() - t0
+    v = r.bytes_per_layer * args.steps / el / 1e9
+    sample = (f"each step = RoPE + delta write + decode attention of ONE of the 36 layers of: {r.desc} "
+              f"(4 distinct layers cycled); fp64 oracle; GB/s by the GPU line's algorithmic-byte count")
+    cfg = decode_config(args.config, r.B, r.T, N_LAYERS, args.kv, args.mode, args.gpus)
+    print(json.dumps(_reference_line(args, METRIC, v, "GB/s", el, cfg, sample, r.cores)), flush=True)
+
+
+def run_reference_prefill(args):
+    """The oracle's RoPE + delta write + causal prefill on the host cores: each
+    step is one request of the coalesced prefill batch in one layer (requests
+    and 4 layers cycled); GB/s by the GPU line's prefill byte count."""
+    import numpy as np
+    from gqa_attention_static_b200 import workloads as W
+    oracle = _oracle()
+    batch = W.cfg_prefill(layers=4)
+    items = []
+    for l in range(4):
+        for b in range(batch.B):
+            n = int(batch.n_new[b])
+            items.append((_bits(batch.q[l][b:b + 1]), _bits(batch.k_new[l][b:b + 1]), _bits(batch.v_new[l][b:b + 1]),
+                          _bits(batch.cache_k[l][b:b + 1]), _bits(batch.cache_v[l][b:b + 1]), n))
+    scale = 1.0 / math.sqrt(128)
+    zero = np.zeros(1, np.int32)
+    state = {"i": 0, "bytes": 0}
+
+    def step():
+        q, kn, vn, ck, cv, n = items[state["i"] % len(items)]
+        state["i"] += 1
+        nn = np.array([n], np.int32)
+        qr, ck2, cv2, _ = oracle.append_rope(q, kn, vn, ck, cv, zero, nn)
+        oracle.prefill(qr, ck2, cv2, zero, nn, scale)
+        state["bytes"] += 9216 * n
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    state["bytes"] = 0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    v = state["bytes"] / el / 1e9
+    sample = (f"each step = RoPE + delta write + causal prefill of ONE request (all 16 heads) of one layer of: "
+              f"{WORKLOAD_DESC['prefill']} (16 requests x 4 layers cycled); fp64 oracle; GB/s by the GPU line's "
+              f"prefill byte count (9216 B per prompt row)")
+    cfg = prefill_config(N_LAYERS, int(batch.n_new.sum()), args.gpus)
+    print(json.dumps(_reference_line(args, PREFILL_METRIC, v, "GB/s", el, cfg, sample, oracle.num_threads())),
+          flush=True)
+
+
+def run_reference_sweep(args):
+    """The oracle's sweep on the host cores: each step is the whole sweep of ONE
+    layer (prefill of the 50-row prompt, then 461 decode steps, each with its
+    RoPE + delta write); tokens·layers/s."""
+    import numpy as np
+    from gqa_attention_static_b200 import workloads as W
+    oracle = _oracle()
+    pre = W.cfg_sweep_prefill(layers=1)
+    L0 = pre.S
+    nsteps = pre.T - 1 - L0
+    qa, ka, va = W.sweep_all_step_inputs(2, nsteps, 1)
+    scale = 1.0 / math.sqrt(128)
+    one = np.ones(1, np.int32)
+
+    def sweep():
+        qr, ck, cv, _ = oracle.append_rope(_bits(pre.q[0]), _bits(pre.k_new[0]), _bits(pre.v_new[0]),
+                                           _bits(pre.cache_k[0]), _bits(pre.cache_v[0]), pre.pos0.numpy(),
+                                           pre.n_new.numpy())
+        oracle.prefill(qr, ck, cv, pre.pos0.numpy(), pre.n_new.numpy(), scale)
+        for i in range(nsteps):
+            p = L0 + i
+            qd, ck, cv, _ = oracle.append_rope(_bits(qa[i, 0]), _bits(ka[i, 0]), _bits(va[i, 0]), ck, cv,
+                                               np.array([p], np.int32), one)
+            oracle.decode(qd, ck, cv, np.array([p + 1], np.int32), scale)
+
+    for _ in range(max(1, args.warmup)):
+        sweep()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        sweep()
+    el = time.perf_counter() - t0
+    v = (L0 + nsteps) * args.steps / el
+    sample = (f"each step = the whole sweep of ONE layer (of the 36) of: {WORKLOAD_DESC['sweep']}; fp64 oracle; "
+              f"tokens·layers/s")
+    cfg = {"workload": WORKLOAD_DESC["sweep"], "batch": 1, "max_total_len": pre.T, "layers": N_LAYERS,
+           "prompt_rows": L0, "decode_steps": nsteps, "parallelism": f"replicas x{args.gpus}"}
+    print(json.dumps(_reference_line(args, SWEEP_METRIC, v, "tokens·layers/s", el, cfg, sample,
+                                     oracle.num_threads())), flush=True)
+
+
 class EncoderOracleRunner:
     """The fp64 oracle's encoder attention on this host's cores over a bounded
     sample: one clip of the encoder batch per step (clips cycled, 4 layers)."""
@@ -313,6 +488,7 @@ class EncoderOracleRunner:
         self.oracle = oracle
         self.cores = oracle.num_threads()
         e = W.cfg_encoder(layers=layers)
+        self.lengths = e.length.tolist()
         bits = lambda x: x.contiguous().view(torch.int16).numpy().view(np.uint16)
         self.items = [(bits(e.q[l][b:b + 1]), bits(e.k[l][b:b + 1]), bits(e.v[l][b:b + 1]),
                        e.length[b:b + 1].numpy()) for l in range(layers) for b in range(e.B)]
@@ -345,8 +521,7 @@ def run_reference_encoder(args):
             "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "encoder attention B=8 clips of 150..1500 frames (S=1500), 20 heads x 64, "
-                                   "32 layers"},
+            "config": encoder_config(32, [int(x) for x in r.lengths]),
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": r.cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -403,40 +578,185 @@ def run_reference_qkv(args):
             "metric": "fused Q/K/V projection + RoPE + delta write, token-layers/s (1xB200); % of roofline",
             "value": v, "unit": "token-layers/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64", "data": "synthetic (random-init weights)", "config": {"workload": desc},
+            "dtype": "f64", "data": "synthetic (random-init weights)", "config": qkv_config(desc, int(base.n_new.sum()) if args.config == "qkv_prefill" else base.B, N_LAYERS),
             "cpu_baseline": {"value": v, "unit": "token-layers/s", "cores": oracle.num_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": v, "unit": "token-layers/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def run_reference(args):
-    world, rank, _ = dist_env()
-    if rank != 0:
-        return
-    if args.config == "encoder":
-        run_reference_encoder(args)
-        return
-    if args.config in ("qkv_decode", "qkv_prefill"):
-        run_reference_qkv(args)
-        return
-    r = OracleRunner(args.config, args.mode, kv=args.kv)
-    for _ in range(max(1, args.warmup)):
-        r.layer_step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        r.layer_step()          # one step = one layer of the workload (bounded sample)
-    el = time.perf_counter() - t0
-    v = r.bytes_per_layer * args.steps / el / 1e9
-    sample = (f"each step = RoPE + delta write + decode attention of ONE of the 36 layers of: {r.desc} "
-              f"(4 distinct layers cycled); fp64 oracle; GB/s by the GPU line's algorithmic-byte count")
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": r.desc, "mode": args.mode, "kv_cache": args.kv},
-            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": r.cores, "kind": "oracle", "sample": sample},
-            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- the GPU arm ----
+
+PREFILL_METRIC = "coalesced causal prefill GB/s (1×B200); % of HBM roofline"
+SWEEP_METRIC = "autoregressive sweep tokens·layers/s (1×B200)"
+
+
+def _capture(fn, s):
+    """A CUDA graph of fn(s) (run once eagerly first: loads kernels, sets attributes)."""
+    import torch
+    with torch.cuda.stream(s):
+        fn(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        fn(s)
+    torch.cuda.synchronize()
+    return g
+
+
+def _replay_ms(g, s, n: int) -> float:
+    """Device time per replay of graph g, n replays back to back on stream s,
+    CUDA events on s with a synchronisation on both sides."""
+    import torch
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        e0.record(s)
+        for _ in range(n):
+            g.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / n
+
+
+def _instrumented(append_fn, attn_fn, s, U: int):
+    """A graph of U steps with event-record nodes around each step's two kernel
+    groups, so per-launch durations are read on the launching stream."""
+    import torch
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(U)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for u in range(U):
+            ev[u][0].record(s)
+            append_fn(s)
+            ev[u][1].record(s)
+            attn_fn(s)
+            ev[u][2].record(s)
+    torch.cuda.synchronize()
+    return g, ev
+
+
+def _launch_times(g, ev, s, U: int, step_ms: float, min_calls: int = 200, min_s: float = 0.5):
+    """Replay the instrumented graph for at least min_calls calls and min_s
+    seconds; mean (append ms, attention ms) per call over the last replay's U
+    calls (every replay overwrites the same events)."""
+    import torch
+    reps = max(-(-min_calls // U), int(math.ceil(min_s * 1e3 / max(step_ms * U, 1e-3))))
+    with torch.cuda.stream(s):
+        for _ in range(reps):
+            g.replay()
+    torch.cuda.synchronize()
+    app = [ev[u][0].elapsed_time(ev[u][1]) for u in range(U)]
+    att = [ev[u][1].elapsed_time(ev[u][2]) for u in range(U)]
+    return sum(app) / U, sum(att) / U, reps * U
+
+
+def decode_measure(name: str, mode_name: str, dev: str, s, steps: int, batched: bool = True, max_splits: int = 8,
+                   kv: str = "bf16"):
+    """One decode workload on this GPU: step time (graph replays), the decode
+    call's duration (instrumented graph), algorithmic GB/s and roofline
+    fractions.  Inputs are generated on the device."""
+    import torch
+    from gqa_attention_static_b200 import ops
+    from gqa_attention_static_b200.step import DecodeStep
+    batch, desc = make_workload(name, N_LAYERS, dev)
+    mode = ops.ARK_MASKED_STATIC if mode_name == "masked" else ops.ARK_LENGTH_AWARE
+    ks = vs = None
+    if kv == "fp8":
+        fc = fp8_cache_for(batch, mode_name)
+        ck, cv = [x.to(dev) for x in fc.cache_k], [x.to(dev) for x in fc.cache_v]
+        ks, vs = [x.to(dev) for x in fc.k_scale], [x.to(dev) for x in fc.v_scale]
+    else:
+        ck, cv = batch.cache_k, batch.cache_v
+    step = DecodeStep(batch.q, batch.k_new, batch.v_new, ck, cv, batch.pos0, batch.n_new, batch.kv_len,
+                      max_splits=max_splits, mode=mode, batched=batched, k_scale=ks, v_scale=vs)
+    g = _capture(step.run, s)
+    for _ in range(3):
+        g.replay()
+    ms_step = _replay_ms(g, s, steps)
+    U = 8 if batched else 2
+    gi, ev = _instrumented(step.append, step.attention, s, U)
+    app_ms, attn_ms, calls = _launch_times(gi, ev, s, U, ms_step)
+    per_call = attn_ms / (1 if batched else N_LAYERS)
+    L = batch.layers
+    bytes_layer = algorithmic_bytes(batch.kv_len.tolist(), batch.B, kv)
+    bytes_call = bytes_layer * (L if batched else 1)
+    out = {"workload": desc, "mode": "masked-static" if mode_name == "masked" else "length-aware",
+           "ms_per_step": ms_step, "gbs": bytes_layer * L / (ms_step * 1e-3) / 1e9,
+           "tokens_layers_per_s": batch.B * L / (ms_step * 1e-3),
+           "decode_call_us": per_call * 1e3, "append_us_per_step": app_ms * 1e3,
+           "algorithmic_bytes_per_step": bytes_layer * L, "timed_calls": calls,
+           "status": int(step.status.item())}
+    out.update({"decode_" + k: v for k, v in hbm_roofline(bytes_call / (per_call * 1e-3) / 1e9).items()
+                if k in ("achieved", "frac", "frac_spec", "peak", "peak_kind")})
+    return out, step, batch, g, ms_step, per_call, bytes_layer
+
+
+def sweep_measure(dev: str, s, reps: int = 3, fused_rope: bool = True):
+    """The batch-1 autoregressive sweep over 36 layers: prefill of the 50-row
+    prompt, then 461 decode steps at positions 50..510, each appending its fresh
+    k/v row and attending to every valid row.  The prefill and the 461 steps
+    are each one CUDA graph (the decode graph holds 461 x 3 launches)."""
+    import torch
+    from gqa_attention_static_b200 import ops
+    from gqa_attention_static_b200 import workloads as W
+    from gqa_attention_static_b200.step import DecodeStep, PrefillStep
+    L = N_LAYERS
+    pre = W.cfg_sweep_prefill(layers=L, device=dev)
+    L0, T = pre.S, pre.T
+    nsteps = T - 1 - L0
+    ps = PrefillStep(pre.q, pre.k_new, pre.v_new, pre.cache_k, pre.cache_v, pre.pos0, pre.n_new,
+                     fused_rope=fused_rope)
+    qa, ka, va = W.sweep_all_step_inputs(2, nsteps, L, device=dev)
+    pos_all = torch.arange(L0, L0 + nsteps, dtype=torch.int32, device=dev)
+    kv_all = pos_all + 1
+    one = torch.ones(1, dtype=torch.int32, device=dev)
+    ws = ops.decode_workspace(1, 16, 128, T, 8, device=dev, layers=L)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    o = [torch.empty(1, 1, 16, 128, dtype=torch.bfloat16, device=dev) for _ in range(L)]
+    lse = [torch.empty(1, 16, dtype=torch.float32, device=dev) for _ in range(L)]
+    steps = [DecodeStep([qa[i, l] for l in range(L)], [ka[i, l] for l in range(L)], [va[i, l] for l in range(L)],
+                        pre.cache_k, pre.cache_v, pos_all[i:i + 1], one, kv_all[i:i + 1], table=ps.table,
+                        workspace=ws, status=status, o=o, lse=lse) for i in range(nsteps)]
+
+    def decode_all(st):
+        for x in steps:
+            x.run(st)
+
+    g_pre = _capture(ps.run, s)
+    g_dec = _capture(decode_all, s)
+    for _ in range(2):
+        g_pre.replay()
+        g_dec.replay()
+    torch.cuda.synchronize()
+    ms_pre = _replay_ms(g_pre, s, max(3, reps))
+    ms_dec = _replay_ms(g_dec, s, reps)
+    # the whole sweep: prefill then decode, back to back
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        e0.record(s)
+        for _ in range(reps):
+            g_pre.replay()
+            g_dec.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    ms_sweep = e0.elapsed_time(e1) / reps
+    positions = sum(range(L0 + 1, L0 + nsteps + 1))
+    dec_bytes = (positions * 1024 + nsteps * 8192) * L
+    st = int(status.item()) | int(ps.status.item())
+    res = {"workload": WORKLOAD_DESC["sweep"], "ms_per_sweep": ms_sweep,
+           "tokens_layers_per_s": (L0 + nsteps) * L / (ms_sweep * 1e-3),
+           "prefill_ms": ms_pre, "decode_ms": ms_dec, "decode_us_per_step": ms_dec * 1e3 / nsteps,
+           "decode_tokens_layers_per_s": nsteps * L / (ms_dec * 1e-3),
+           "decode_kv_gbs": dec_bytes / (ms_dec * 1e-3) / 1e9, "decode_algorithmic_bytes": dec_bytes,
+           "prefill_path": "K/V append + prefill rotating q on load" if fused_rope else "append + prefill",
+           "launches_per_sweep": ps.launches_per_step() + 3 * nsteps, "status": st}
+    return res, ps.launches_per_step() + 3 * nsteps
 
 
 def prefill_bytes_flops(n_new):
@@ -447,104 +767,382 @@ def prefill_bytes_flops(n_new):
     return rows * 9216, sum(4096 * int(x) * (int(x) + 1) for x in n_new)
 
 
-def measured_tensor_peak():
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            d = json.load(f)
-        return float(d["bf16_tflops"]), "measured"
-    except Exception:
-        return 1590.0, "fallback"
+def prefill_config(L: int, rows: int, world: int) -> dict:
+    return {"workload": WORKLOAD_DESC["prefill"].replace("36 layers", f"{L} layers"), "layers": L, "rows": rows,
+            "l2": "q/o of the layers (%.1f GB) larger than L2" % (L * 16 * 387 * 16 * 128 * 2 * 2 / 1e9),
+            "parallelism": f"replicas x{world}"}
 
 
-def run_prefill(args):
-    """Coalesced prefill: 16 prompts of 20..387 rows, 36 layers.  A step is
-    RoPE + delta write of all prompt rows of all layers, then the causal
-    prefill of every layer."""
+def prefill_measure(dev: str, s, steps: int, fused_rope: bool = True, layers: int = N_LAYERS):
+    """Coalesced prefill: 16 prompts of 20..387 rows, 36 layers.  A step is the
+    K/V append (RoPE on k, delta write) of every prompt row of every layer, then
+    the causal prefill of every layer (rotating q as it loads it); with
+    fused_rope False the append also rotates q in place."""
     import torch
-    from gqa_attention_static_b200 import ops
     from gqa_attention_static_b200 import workloads as W
     from gqa_attention_static_b200.step import PrefillStep
+    batch = W.cfg_prefill(layers=layers, device=dev)
+    L = batch.layers
+    step = PrefillStep(batch.q, batch.k_new, batch.v_new, batch.cache_k, batch.cache_v, batch.pos0, batch.n_new,
+                       fused_rope=fused_rope)
+    g = _capture(step.run, s)
+    for _ in range(3):
+        g.replay()
+    ms_step = _replay_ms(g, s, steps)
+    U = 4
+    gi, ev = _instrumented(step.append, step.attention, s, U)
+    ms_append, ms_attn, calls = _launch_times(gi, ev, s, U, ms_step, min_calls=40, min_s=0.3)
+    ms_layer = ms_attn / L
+    nb, nf = prefill_bytes_flops(batch.n_new.tolist())
+    tc, tc_kind = measured_tensor_peak()
+    hb = hbm_roofline(nb / (ms_layer * 1e-3) / 1e9)
+    achieved_tf = nf / (ms_layer * 1e-3) / 1e12
+    roof = dict(hb)
+    roof.update({"kernel": "prefill_kernel (ark_attn_prefill%s_layers: one launch of 36 layers), per layer" %
+                           ("_rope" if fused_rope else ""),
+                 "traffic": PREFILL_TRAFFIC.get(src_hash("gqa_attention_static_b200/csrc/prefill.cu")),
+                 "launch_ms_per_layer": ms_layer, "algorithmic_bytes_per_layer": nb, "flops_per_layer": nf,
+                 "achieved_tflops": achieved_tf, "tensor_peak_tflops": tc, "tensor_peak_kind": tc_kind,
+                 "frac_tensor": achieved_tf / tc, "append_ms_per_step": ms_append, "timed_calls": calls})
+    res = {"workload": WORKLOAD_DESC["prefill"], "ms_per_step": ms_step, "gbs": nb * L / (ms_step * 1e-3) / 1e9,
+           "tokens_layers_per_s": int(batch.n_new.sum()) * L / (ms_step * 1e-3),
+           "prefill_ms_per_layer": ms_layer, "append_ms_per_step": ms_append,
+           "frac": hb["frac"], "frac_spec": hb["frac_spec"], "frac_tensor": achieved_tf / tc,
+           "path": ("K/V-only append + prefill rotating q as it loads it" if fused_rope else
+                    "append rotating q in place + prefill"),
+           "status": int(step.status.item())}
+    return res, roof, step, batch, ms_step
 
+
+def e2e_measure(step_factory, d_in, d_out_o, d_out_lse, g_step, step, s, dev, steps: int):
+    """End to end through the public calls: every step copies its inputs
+    (q/k_new/v_new of all layers) from pinned host memory and reads o/lse back
+    into pinned host memory.  Two buffer sets let the copy engines move step
+    i+1's inputs and step i-1's outputs while the kernels run step i (three
+    streams, events between them).  U pipelined steps are captured in one CUDA
+    graph (copies and kernels), replayed until at least `steps` steps and 0.3 s;
+    the copies alone are timed too, for the breakdown."""
+    import torch
+    sets = []
+    for k in range(2):
+        if k == 0:
+            di, do, dl, st_k = d_in, d_out_o, d_out_lse, step
+        else:
+            di, do, dl = torch.empty_like(d_in), torch.empty_like(d_out_o), torch.empty_like(d_out_lse)
+            st_k = step_factory(di, do, dl)
+        ho = torch.empty(do.numel(), dtype=do.dtype, pin_memory=True)
+        hl = torch.empty(dl.numel(), dtype=dl.dtype, pin_memory=True)
+        sets.append((di, do, dl, st_k, ho, hl))
+    h_in = torch.empty(d_in.numel(), dtype=d_in.dtype, pin_memory=True)
+    h_in.copy_(d_in.cpu())
+    s_h2d = torch.cuda.Stream(device=dev)
+    s_d2h = torch.cuda.Stream(device=dev)
+    for _, _, _, st_k, _, _ in sets:          # eager run: kernels loaded, tensor maps cached
+        with torch.cuda.stream(s):
+            st_k.run(s)
+    torch.cuda.synchronize()
+    U = 8
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        s_h2d.wait_stream(s)
+        s_d2h.wait_stream(s)
+        for i in range(U):
+            k = i % 2
+            di, do, dl, st_k, ho, hl = sets[k]
+            if i >= 2:
+                s_h2d.wait_event(ev_comp[k])           # step i-2 no longer reads this input set
+            with torch.cuda.stream(s_h2d):
+                di.copy_(h_in, non_blocking=True)
+            ev_in[k].record(s_h2d)
+            s.wait_event(ev_in[k])
+            if i >= 2:
+                s.wait_event(ev_out[k])                # step i-2's outputs were read back
+            st_k.run(s)
+            ev_comp[k].record(s)
+            s_d2h.wait_event(ev_comp[k])
+            with torch.cuda.stream(s_d2h):
+                ho.copy_(do, non_blocking=True)
+                hl.copy_(dl, non_blocking=True)
+            ev_out[k].record(s_d2h)
+        s.wait_stream(s_h2d)
+        s.wait_stream(s_d2h)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        g.replay()
+    ms_u = _replay_ms(g, s, 1)
+    reps = max(-(-steps // U), int(math.ceil(300.0 / max(ms_u, 1e-3))))
+    ms_e2e = _replay_ms(g, s, reps) / U
+    # breakdown: the copies alone, the compute alone
+    ho, hl = sets[0][4], sets[0][5]
+
+    def h2d_only(st):
+        d_in.copy_(h_in, non_blocking=True)
+
+    def d2h_only(st):
+        ho.copy_(d_out_o, non_blocking=True)
+        hl.copy_(d_out_lse, non_blocking=True)
+
+    g_h = _capture(h2d_only, s)
+    g_d = _capture(d2h_only, s)
+    ms_h2d = _replay_ms(g_h, s, 20)
+    ms_d2h = _replay_ms(g_d, s, 20)
+    ms_comp = _replay_ms(g_step, s, 20)
+    h2d_bytes = d_in.numel() * d_in.element_size()
+    d2h_bytes = d_out_o.numel() * d_out_o.element_size() + d_out_lse.numel() * d_out_lse.element_size()
+    return {"ms_per_step": ms_e2e, "timed_steps": reps * U, "h2d_bytes_per_step": h2d_bytes,
+            "d2h_bytes_per_step": d2h_bytes,
+            "breakdown_ms": {"h2d": ms_h2d, "compute": ms_comp, "d2h": ms_d2h,
+                             "h2d_gbs": h2d_bytes / (ms_h2d * 1e-3) / 1e9, "d2h_gbs": d2h_bytes / (ms_d2h * 1e-3) / 1e9},
+            "how": "pinned host buffers, H2D of the step inputs and D2H of o/lse every step, double-buffered on "
+                   "separate copy streams; %d pipelined steps per CUDA graph (copies and kernels)" % U}
+
+
+def run_decode(args):
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = f"cuda:{local}"
+
+    from gqa_attention_static_b200 import ops
+    from gqa_attention_static_b200.step import DecodeStep
+
+    ops.load()
+    mode = ops.ARK_MASKED_STATIC if args.mode == "masked" else ops.ARK_LENGTH_AWARE
+    batch, desc = make_workload(args.config, N_LAYERS, "cpu")
+    B, T = batch.B, batch.T
+    L = batch.layers
+
+    # device buffers: one packed input buffer (q | k_new | v_new) and one packed output (o | lse)
+    qsz = B * 16 * 128
+    ksz = B * 2 * 128
+    in_elems = L * (qsz + 2 * ksz)
+    d_in = torch.empty(in_elems, dtype=torch.bfloat16, device=dev)
+
+    def views(di):
+        qv = di[:L * qsz].view(L, B, 1, 16, 128)
+        kv_ = di[L * qsz:L * (qsz + ksz)].view(L, B, 1, 2, 128)
+        vv = di[L * (qsz + ksz):].view(L, B, 1, 2, 128)
+        return [qv[l] for l in range(L)], [kv_[l] for l in range(L)], [vv[l] for l in range(L)]
+
+    qv, kv_, vv = views(d_in)
+    for l in range(L):
+        qv[l].copy_(batch.q[l])
+        kv_[l].copy_(batch.k_new[l])
+        vv[l].copy_(batch.v_new[l])
+    fp8 = (args.kv == "fp8")
+    ks = vs = None
+    if fp8:
+        fc = fp8_cache_for(batch, args.mode)
+        ck = [x.to(dev) for x in fc.cache_k]
+        cv = [x.to(dev) for x in fc.cache_v]
+        ks = [x.to(dev) for x in fc.k_scale]
+        vs = [x.to(dev) for x in fc.v_scale]
+    else:
+        ck = [x.to(dev) for x in batch.cache_k]
+        cv = [x.to(dev) for x in batch.cache_v]
+    pos0 = batch.pos0.to(dev)
+    n_new = batch.n_new.to(dev)
+    kv_len = batch.kv_len.to(dev)
+    osz = B * 16 * 128
+    d_out_o = torch.empty(L * osz, dtype=torch.bfloat16, device=dev)
+    d_out_lse = torch.empty(L * B * 16, dtype=torch.float32, device=dev)
+
+    def make_step(di, do, dl):
+        q_, k_, v_ = views(di)
+        return DecodeStep(q_, k_, v_, ck, cv, pos0, n_new, kv_len, max_splits=args.max_splits, mode=mode,
+                          batched=not args.per_layer, k_scale=ks, v_scale=vs,
+                          o=[do[l * osz:(l + 1) * osz].view(B, 1, 16, 128) for l in range(L)],
+                          lse=[dl[l * B * 16:(l + 1) * B * 16].view(B, 16) for l in range(L)])
+
+    step = make_step(d_in, d_out_o, d_out_lse)
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    g_step = _capture(step.run, s)
+    U = 8 if step.batched else 2
+    g_inst, ev = _instrumented(step.append, step.attention, s, U)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed(fn, K):
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            e0.record(s)
+            for _ in range(K):
+                fn()
+            e1.record(s)
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1), world, dev)
+
+    for _ in range(max(3, args.warmup)):
+        g_step.replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ms_total = timed(g_step.replay, args.steps)
+    ms_step = ms_total / args.steps
+    # kernel durations: the instrumented graph, replayed right after on the same stream, for at
+    # least 200 decode calls and 0.5 s whatever --steps is
+    app_ms, attn_ms, inst_calls = _launch_times(g_inst, ev, s, U, ms_step)
+    clk = clocks.stop()
+    if int(step.status.item()) != 0:
+        print(f"device status word set: {int(step.status.item())}", file=sys.stderr)
+    calls_per_group = 1 if step.batched else L          # decode launches per attention group
+    per_launch_ms = attn_ms / calls_per_group
+
+    kvl = batch.kv_len.tolist()
+    bytes_layer = algorithmic_bytes(kvl, B, args.kv)
+    step_bytes = bytes_layer * L
+    value = job_throughput(step_bytes, world, ms_step)
+    tl = B * L * world / (ms_step * 1e-3)
+    bytes_launch = bytes_layer * (L if step.batched else 1)
+    achieved = bytes_launch / (per_launch_ms * 1e-3) / 1e9
+    h = src_hash("gqa_attention_static_b200/csrc/decode.cu")
+    # the capture is of the default workload's batched launch
+    traffic = (DECODE_TRAFFIC.get(h) if (not args.per_layer and args.config == "ragged" and args.mode == "aware"
+                                         and not fp8) else None)
+    roof = {"kernel": "decode_kernel + merge_kernel (one ark_attn_decode%s call)" % ("" if args.per_layer else
+                                                                                     "_layers")}
+    roof.update(hbm_roofline(achieved))
+    roof.update({"traffic": traffic, "launch_ms": per_launch_ms, "algorithmic_bytes_per_launch": bytes_launch,
+                 "timed_calls": inst_calls, "append_ms_per_step": app_ms})
+
+    e2e = None
+    if not args.no_e2e:
+        r = e2e_measure(make_step, d_in, d_out_o, d_out_lse, g_step, step, s, dev, max(100, args.steps))
+        ms_e2e = max_over_ranks(r["ms_per_step"], world, dev)
+        e2e = {"value": job_throughput(step_bytes, world, ms_e2e), "unit": "GB/s",
+               "h2d_bytes_per_step": r["h2d_bytes_per_step"], "d2h_bytes_per_step": r["d2h_bytes_per_step"],
+               "ms_per_step": ms_e2e, "timed_steps": r["timed_steps"], "breakdown_ms": r["breakdown_ms"],
+               "how": r["how"]}
+
+    extras = None
+    if (world == 1 and not args.no_extras and args.config == "ragged" and args.mode == "aware" and not fp8
+            and not args.per_layer):
+        del g_step, g_inst
+        extras = measure_extras(dev, s, args)
+
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(args.config, args.cpu_seconds, args.mode, args.kv)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3 cache, f16 MMA" if fp8 else "bf16", "data": "synthetic",
+            "config": decode_config(args.config, B, T, L, args.kv, args.mode, world),
+            "impl_details": {"max_splits": args.max_splits, "min_tiles_per_warp": step.min_tiles,
+                             "path": ("per-layer calls" if args.per_layer else "layer-batched calls") +
+                                     " replayed from one CUDA graph"},
+            "tokens_layers_per_s": tl,
+            "roofline": roof,
+            "cpu_baseline": cb,
+            "e2e": e2e,
+            "gpu_launches": step.launches_per_step() * args.steps,
+            "clocks": clk,
+        }
+        if extras is not None:
+            line["configs"] = extras
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def measure_extras(dev, s, args):
+    """The decoder's other attention workloads, each measured on this GPU in a
+    few seconds (inputs generated on the device, freed after each)."""
+    import torch
+    out = {}
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    for name, mode in (("single", "aware"), ("ragged", "masked"), ("long2048", "aware"), ("long2048", "masked"),
+                       ("long1024", "aware"), ("long1024", "masked")):
+        r = decode_measure(name, mode, dev, s, 50)[0]
+        out[f"{name}_{mode}"] = r
+        torch.cuda.empty_cache()
+    out["single_aware"]["us_per_step"] = out["single_aware"]["ms_per_step"] * 1e3
+    for T in ("long2048", "long1024"):
+        a, m = out[f"{T}_aware"], out[f"{T}_masked"]
+        m["masked_over_aware_time"] = m["ms_per_step"] / a["ms_per_step"]
+    sw, _ = sweep_measure(dev, s, reps=3, fused_rope=not args.two_call_prefill)
+    out["sweep"] = sw
+    torch.cuda.empty_cache()
+    pr = prefill_measure(dev, s, 20, fused_rope=not args.two_call_prefill)[0]
+    out["prefill"] = pr
+    torch.cuda.empty_cache()
+    out["clocks"] = clocks.stop()
+    return out
+
+
+def run_sweep(args):
+    import torch
+    from gqa_attention_static_b200 import ops
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
     dev = f"cuda:{local}"
     ops.load()
-    batch = W.cfg_prefill(layers=N_LAYERS)
-    L = batch.layers
-    step = PrefillStep([x.to(dev) for x in batch.q], [x.to(dev) for x in batch.k_new],
-                       [x.to(dev) for x in batch.v_new], [x.to(dev) for x in batch.cache_k],
-                       [x.to(dev) for x in batch.cache_v], batch.pos0.to(dev), batch.n_new.to(dev),
-                       fused_rope=args.rope_on_load)
     s = torch.cuda.Stream(device=dev)
     s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        step.run(s)
-    torch.cuda.synchronize()
-    g_step = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step, stream=s):
-        step.run(s)
-    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
-    g_inst = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_inst, stream=s):
-        ev[0].record(s)
-        step.append(s)
-        ev[1].record(s)
-        step.attention(s)
-        ev[2].record(s)
-    torch.cuda.synchronize()
-    for _ in range(max(3, args.warmup)):
-        g_step.replay()
-    torch.cuda.synchronize()
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(s):
-        e0.record(s)
-        for _ in range(args.steps):
-            g_step.replay()
-        e1.record(s)
-    torch.cuda.synchronize()
-    ms_step = e0.elapsed_time(e1) / args.steps
-    with torch.cuda.stream(s):
-        g_inst.replay()
-    torch.cuda.synchronize()
+    res, launches = sweep_measure(dev, s, reps=max(3, args.steps), fused_rope=not args.two_call_prefill)
     clk = clocks.stop()
-    ms_prefill = ev[1].elapsed_time(ev[2]) / L          # per layer: the layer-batched prefill call / L
-    ms_append = ev[0].elapsed_time(ev[1])
-    if int(step.status.item()) != 0:
-        print(f"device status word set: {int(step.status.item())}", file=sys.stderr)
-    nb, nf = prefill_bytes_flops(batch.n_new.tolist())
-    hbm, hbm_kind = measured_peaks()
-    tc, tc_kind = measured_tensor_peak()
-    t_bytes = nb / (hbm * 1e9)
-    t_flops = nf / (tc * 1e12)
-    bound = "hbm" if t_bytes >= t_flops else "tensor"
-    achieved_gbs = nb / (ms_prefill * 1e-3) / 1e9
-    achieved_tf = nf / (ms_prefill * 1e-3) / 1e12
-    roof = {"kernel": "prefill_kernel (ark_attn_prefill%s_layers, per layer)" % ("_rope" if args.rope_on_load else ""),
-            "bound": bound,
-            "achieved": achieved_gbs if bound == "hbm" else achieved_tf,
-            "peak": hbm if bound == "hbm" else tc, "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
-            "frac": (t_bytes if bound == "hbm" else t_flops) / (ms_prefill * 1e-3),
-            "peak_kind": hbm_kind if bound == "hbm" else tc_kind,
-            "traffic": PREFILL_TRAFFIC.get(src_hash("gqa_attention_static_b200/csrc/prefill.cu")),
-            "launch_ms": ms_prefill, "algorithmic_bytes_per_launch": nb, "flops_per_launch": nf,
-            "achieved_tflops": achieved_tf, "tensor_peak_tflops": tc,
-            "append_ms_per_step": ms_append}
-    value = nb * L / (ms_step * 1e-3) / 1e9
-    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "coalesced causal prefill B=16 L U[20,387] S=387 T=512, 36 layers",
-                       "layers": L, "rows": int(batch.n_new.sum()),
-                       "l2": "q/o of 36 layers (1.8 GB) larger than L2",
-                       "path": ("layer-batched K/V append + layer-batched prefill rotating q as it loads it"
-                                if args.rope_on_load else "layer-batched append + layer-batched prefill") +
-                               " (16 layers per launch), replayed from one CUDA graph"},
-            "tokens_layers_per_s": int(batch.n_new.sum()) * L / (ms_step * 1e-3),
-            "roofline": roof, "gpu_launches": step.launches_per_step() * args.steps, "clocks": clk}
+    if res["status"]:
+        print(f"device status word set: {res['status']}", file=sys.stderr)
+    roof = {"kernel": "decode_kernel + merge_kernel, one call per sweep position (latency-bound at B=1)"}
+    roof.update(hbm_roofline(res["decode_kv_gbs"]))
+    line = {"metric": SWEEP_METRIC, "value": res["tokens_layers_per_s"], "unit": "tokens·layers/s", "n_gpus": world,
+            "steps": max(3, args.steps), "warmup": 2, "ms_per_step": res["ms_per_sweep"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD_DESC["sweep"], "batch": 1, "max_total_len": 512, "layers": N_LAYERS,
+                       "prompt_rows": 50, "decode_steps": 461, "parallelism": f"replicas x{world}"},
+            "sweep": res, "roofline": roof, "gpu_launches": launches * max(3, args.steps), "clocks": clk}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_prefill(args):
+    import torch
+    from gqa_attention_static_b200 import ops
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+    ops.load()
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    res, roof, step, batch, ms_step = prefill_measure(dev, s, args.steps, fused_rope=not args.two_call_prefill,
+                                                      layers=args.layers or N_LAYERS)
+    clk = clocks.stop()
+    if res["status"]:
+        print(f"device status word set: {res['status']}", file=sys.stderr)
+    L = batch.layers
+    nb, _ = prefill_bytes_flops(batch.n_new.tolist())
+    line = {"metric": PREFILL_METRIC, "value": nb * L * world / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": prefill_config(L, int(batch.n_new.sum()), world),
+            "impl_details": {"path": res["path"] + " (one launch of 36 layers), replayed from one CUDA graph"},
+            "tokens_layers_per_s": res["tokens_layers_per_s"], "prefill": res, "roofline": roof,
+            "gpu_launches": step.launches_per_step() * args.steps, "clocks": clk}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -621,9 +1219,7 @@ def run_encoder(args):
     line = {"metric": "encoder attention TFLOP/s (1xB200); % of bf16 tensor roofline", "value": value,
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "encoder attention B=8 clips of 150..1500 frames (S=1500), 20 heads x 64, "
-                                   f"{L} layers", "lengths": e.length.tolist(),
-                       "l2": "q/k/v/o of 32 layers (3.9 GB) larger than L2"},
+            "config": encoder_config(L, e.length.tolist()),
             "roofline": roof, "gpu_launches": L * args.steps, "clocks": clk}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -721,11 +1317,28 @@ def run_qkv(args):
             "value": value, "unit": "token-layers/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic (random-init weights)",
-            "config": {"workload": desc.replace("36 layers", f"{L} layers"), "rows": rows,
-                       "l2": "weights of %d layers (%.0f MB) larger than L2" % (L, L * N * K * 2 / 1e6)},
+            "config": qkv_config(desc, rows, L),
             "roofline": roof, "gpu_launches": L * args.steps, "clocks": clk}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    if args.config == "encoder":
+        run_reference_encoder(args)
+    elif args.config in ("qkv_decode", "qkv_prefill"):
+        run_reference_qkv(args)
+    elif args.config == "prefill":
+        run_reference_prefill(args)
+    elif args.config == "sweep":
+        run_reference_sweep(args)
+    else:
+        run_reference_decode(args)
 
 
 def main():
@@ -735,253 +1348,14 @@ def main():
         return
     if args.config == "prefill":
         run_prefill(args)
-        return
-    if args.config == "encoder":
+    elif args.config == "sweep":
+        run_sweep(args)
+    elif args.config == "encoder":
         run_encoder(args)
-        return
-    if args.config in ("qkv_decode", "qkv_prefill"):
+    elif args.config in ("qkv_decode", "qkv_prefill"):
         run_qkv(args)
-        return
-    import torch
-    import torch.distributed as dist
-
-    world, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    dev = f"cuda:{local}"
-
-    from gqa_attention_static_b200 import ops
-    from gqa_attention_static_b200.step import DecodeStep
-
-    ops.load()
-    mode = ops.ARK_MASKED_STATIC if args.mode == "masked" else ops.ARK_LENGTH_AWARE
-    batch, desc = make_workload(args.config, N_LAYERS, "cpu")
-    B, T = batch.B, batch.T
-    L = batch.layers
-
-    # device buffers: one packed input buffer (q | k_new | v_new) and one packed output (o | lse)
-    qsz = B * 16 * 128
-    ksz = B * 2 * 128
-    in_elems = L * (qsz + 2 * ksz)
-    d_in = torch.empty(in_elems, dtype=torch.bfloat16, device=dev)
-    qv = d_in[:L * qsz].view(L, B, 1, 16, 128)
-    kv_ = d_in[L * qsz:L * (qsz + ksz)].view(L, B, 1, 2, 128)
-    vv = d_in[L * (qsz + ksz):].view(L, B, 1, 2, 128)
-    for l in range(L):
-        qv[l].copy_(batch.q[l])
-        kv_[l].copy_(batch.k_new[l])
-        vv[l].copy_(batch.v_new[l])
-    fp8 = (args.kv == "fp8")
-    ks = vs = None
-    if fp8:
-        fc = fp8_cache_for(batch, args.mode)
-        ck = [x.to(dev) for x in fc.cache_k]
-        cv = [x.to(dev) for x in fc.cache_v]
-        ks = [x.to(dev) for x in fc.k_scale]
-        vs = [x.to(dev) for x in fc.v_scale]
-        desc = desc.replace(" 1% x8 K/V row outliers", "") + ", fp8 E4M3 cache (per-head scales)"
     else:
-        ck = [x.to(dev) for x in batch.cache_k]
-        cv = [x.to(dev) for x in batch.cache_v]
-    pos0 = batch.pos0.to(dev)
-    n_new = batch.n_new.to(dev)
-    kv_len = batch.kv_len.to(dev)
-    step = DecodeStep([qv[l] for l in range(L)], [kv_[l] for l in range(L)], [vv[l] for l in range(L)],
-                      ck, cv, pos0, n_new, kv_len, max_splits=args.max_splits, mode=mode,
-                      batched=not args.per_layer, k_scale=ks, v_scale=vs)
-    # outputs packed for the device->host read of the e2e leg
-    osz = B * 16 * 128
-    d_out_o = torch.empty(L * osz, dtype=torch.bfloat16, device=dev)
-    d_out_lse = torch.empty(L * B * 16, dtype=torch.float32, device=dev)
-    step.o = [d_out_o[l * osz:(l + 1) * osz].view(B, 1, 16, 128) for l in range(L)]
-    step.lse = [d_out_lse[l * B * 16:(l + 1) * B * 16].view(B, 16) for l in range(L)]
-
-    s = torch.cuda.Stream(device=dev)
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        step.run(s)                 # eager run before capture (loads kernels, sets attributes)
-    torch.cuda.synchronize()
-    g_step = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step, stream=s):
-        step.run(s)
-    # The same steps with event-record nodes around each kernel group, to read
-    # per-launch kernel durations from inside the timed stream.
-    U = 8 if step.batched else 2
-    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(U)]
-    g_inst = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_inst, stream=s):
-        for u in range(U):
-            ev[u][0].record(s)
-            step.append(s)
-            ev[u][1].record(s)
-            step.attention(s)
-            ev[u][2].record(s)
-    torch.cuda.synchronize()
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    def timed(fn, K):
-        barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(s):
-            e0.record(s)
-            for _ in range(K):
-                fn()
-            e1.record(s)
-        barrier()
-        return max_over_ranks(e0.elapsed_time(e1), world, dev)
-
-    for _ in range(max(3, args.warmup)):
-        g_step.replay()
-    torch.cuda.synchronize()
-
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
-    ms_total = timed(g_step.replay, args.steps)
-    # kernel durations: the instrumented graph, replayed right after, same stream
-    reps = max(1, args.steps // U)
-    timed(g_inst.replay, reps)
-    clk = clocks.stop()
-    ms_step = ms_total / args.steps
-    if int(step.status.item()) != 0:
-        print(f"device status word set: {int(step.status.item())}", file=sys.stderr)
-    attn_ms = [ev[u][1].elapsed_time(ev[u][2]) for u in range(U)]
-    app_ms = [ev[u][0].elapsed_time(ev[u][1]) for u in range(U)]
-    calls_per_group = 1 if step.batched else L          # decode launches per attention group
-    per_launch_ms = sum(attn_ms) / len(attn_ms) / calls_per_group
-
-    kvl = batch.kv_len.tolist()
-    bytes_layer = algorithmic_bytes(kvl, B, args.kv)
-    step_bytes = bytes_layer * L
-    value = job_throughput(step_bytes, world, ms_step)
-    tl = B * L * world / (ms_step * 1e-3)
-    bytes_launch = bytes_layer * (L if step.batched else 1)
-    peak, peak_kind = measured_peaks()
-    achieved = bytes_launch / (per_launch_ms * 1e-3) / 1e9
-    h = src_hash("gqa_attention_static_b200/csrc/decode.cu")
-    # the capture is of the default workload's batched launch
-    traffic = (DECODE_TRAFFIC.get(h) if (not args.per_layer and args.config == "ragged" and args.mode == "aware"
-                                         and not fp8) else None)
-
-    e2e = None
-    if not args.no_e2e:
-        # End to end through the public calls: every step copies its q/k_new/v_new
-        # from pinned host memory and reads o/lse back.  Two buffer sets let the
-        # copy engines work on step i+1's inputs and step i-1's outputs while the
-        # kernels run step i (three streams, events between them).
-        h_in = torch.empty(in_elems, dtype=torch.bfloat16, pin_memory=True)
-        h_in.copy_(d_in.cpu())
-        sets = []
-        for k in range(2):
-            di = d_in if k == 0 else torch.empty_like(d_in)
-            do = d_out_o if k == 0 else torch.empty_like(d_out_o)
-            dl = d_out_lse if k == 0 else torch.empty_like(d_out_lse)
-            if k == 0:
-                st_k, g_k = step, g_step
-            else:
-                q2 = di[:L * qsz].view(L, B, 1, 16, 128)
-                k2 = di[L * qsz:L * (qsz + ksz)].view(L, B, 1, 2, 128)
-                v2 = di[L * (qsz + ksz):].view(L, B, 1, 2, 128)
-                st_k = DecodeStep([q2[l] for l in range(L)], [k2[l] for l in range(L)], [v2[l] for l in range(L)],
-                                  ck, cv, pos0, n_new, kv_len, max_splits=args.max_splits, mode=mode,
-                                  batched=not args.per_layer, k_scale=ks, v_scale=vs)
-                st_k.o = [do[l * osz:(l + 1) * osz].view(B, 1, 16, 128) for l in range(L)]
-                st_k.lse = [dl[l * B * 16:(l + 1) * B * 16].view(B, 16) for l in range(L)]
-                with torch.cuda.stream(s):
-                    st_k.run(s)
-                torch.cuda.synchronize()
-                g_k = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g_k, stream=s):
-                    st_k.run(s)
-            ho = torch.empty(L * osz, dtype=torch.bfloat16, pin_memory=True)
-            hl = torch.empty(L * B * 16, dtype=torch.float32, pin_memory=True)
-            sets.append((di, do, dl, g_k, ho, hl))
-        s_h2d = torch.cuda.Stream(device=dev)
-        s_d2h = torch.cuda.Stream(device=dev)
-        ev_in = [torch.cuda.Event() for _ in range(2)]
-        ev_comp = [torch.cuda.Event() for _ in range(2)]
-        ev_out = [torch.cuda.Event() for _ in range(2)]
-        for k in range(2):
-            ev_comp[k].record(s)
-            ev_out[k].record(s)
-        torch.cuda.synchronize()
-
-        def run_e2e(K):
-            for i in range(K):
-                k = i % 2
-                di, do, dl, g_k, ho, hl = sets[k]
-                s_h2d.wait_event(ev_comp[k])          # step i-2 no longer reads this input set
-                with torch.cuda.stream(s_h2d):
-                    di.copy_(h_in, non_blocking=True)
-                ev_in[k].record(s_h2d)
-                s.wait_event(ev_in[k])
-                s.wait_event(ev_out[k])                # step i-2's outputs were read back
-                with torch.cuda.stream(s):
-                    g_k.replay()
-                ev_comp[k].record(s)
-                s_d2h.wait_event(ev_comp[k])
-                with torch.cuda.stream(s_d2h):
-                    ho.copy_(do, non_blocking=True)
-                    hl.copy_(dl, non_blocking=True)
-                ev_out[k].record(s_d2h)
-
-        run_e2e(4)
-        K2 = max(10, args.steps // 2)
-        barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(s_h2d)
-        run_e2e(K2)
-        s_h2d.wait_stream(s_d2h)
-        e1.record(s_h2d)
-        barrier()
-        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / K2, world, dev)
-        e2e = {"value": job_throughput(step_bytes, world, ms_e2e), "unit": "GB/s",
-               "h2d_bytes_per_step": in_elems * 2, "d2h_bytes_per_step": L * osz * 2 + L * B * 16 * 4,
-               "ms_per_step": ms_e2e,
-               "how": "pinned host buffers, H2D of the step inputs and D2H of o/lse every step, "
-                      "double-buffered on separate copy streams"}
-
-    cb = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_baseline(args.config, args.cpu_seconds, args.mode, args.kv)
-
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "e4m3 cache, f16 MMA" if fp8 else "bf16", "data": "synthetic",
-            "config": {"workload": desc, "batch": B, "max_total_len": T, "layers": L, "kv_cache": args.kv,
-                       "mode": "masked-static" if args.mode == "masked" else "length-aware",
-                       "max_splits": args.max_splits, "min_tiles_per_warp": step.min_tiles,
-                       "l2": "inputs larger than L2 (%.0f MB of caches streamed per step)" %
-                             (2 * L * B * T * 2 * 128 * (1 if fp8 else 2) / 1e6),
-                       "parallelism": f"replicas x{world}",
-                       "path": ("per-layer calls" if args.per_layer else "layer-batched calls") +
-                               " replayed from one CUDA graph"},
-            "tokens_layers_per_s": tl,
-            "roofline": {"kernel": "decode_kernel + merge_kernel (one ark_attn_decode%s call)" %
-                                   ("" if args.per_layer else "_layers"),
-                         "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
-                         "launch_ms": per_launch_ms, "algorithmic_bytes_per_launch": bytes_launch,
-                         "append_ms_per_step": sum(app_ms) / len(app_ms)},
-            "cpu_baseline": cb,
-            "e2e": e2e,
-            "gpu_launches": step.launches_per_step() * args.steps,
-            "clocks": clk,
-        }
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        del g_step, g_inst
-        dist.destroy_process_group()
+        run_decode(args)
 
 
 if __name__ == "__main__":

@@ -181,6 +181,18 @@ def sweep_step_inputs(seed: int, step: int, layers: int = N_LAYERS, device: str 
     return qs, ks, vs
 
 
+def sweep_all_step_inputs(seed: int, steps: int, layers: int = N_LAYERS, device: str = "cpu"):
+    """Fresh N(0,1) q/k/v for every decode step of the sweep at once, as three
+    tensors q [steps, layers, 1, 1, 16, 128], k/v [steps, layers, 1, 1, 2, 128]
+    whose [step, layer] slices are one step's per-layer inputs (for the
+    benchmark, which replays the whole sweep from device memory)."""
+    gen = _gen(seed * 100003 + 7, device)
+    q = randn_bf16((steps, layers, 1, 1, HQ, HEAD_DIM), gen, device)
+    k = randn_bf16((steps, layers, 1, 1, HKV, HEAD_DIM), gen, device)
+    v = randn_bf16((steps, layers, 1, 1, HKV, HEAD_DIM), gen, device)
+    return q, k, v
+
+
 def ragged_lengths(seed: int, B: int, lo: int, hi: int) -> torch.Tensor:
     g = _gen(seed + 7919)
     return torch.randint(lo, hi + 1, (B,), generator=g, dtype=torch.int32)
