@@ -819,62 +819,68 @@ def e2e_measure(step_factory, d_in, d_out_o, d_out_lse, g_step, step, s, dev, st
     (q/k_new/v_new of all layers) from pinned host memory and reads o/lse back
     into pinned host memory.  Two buffer sets let the copy engines move step
     i+1's inputs and step i-1's outputs while the kernels run step i (three
-    streams, events between them).  U pipelined steps are captured in one CUDA
-    graph (copies and kernels), replayed until at least `steps` steps and 0.3 s;
-    the copies alone are timed too, for the breakdown."""
+    streams, events between them; the kernels of a step replay its CUDA
+    graph).  Timed over at least `steps` steps and 0.3 s; the copies alone and
+    the compute alone are timed too, for the breakdown."""
     import torch
     sets = []
     for k in range(2):
         if k == 0:
-            di, do, dl, st_k = d_in, d_out_o, d_out_lse, step
+            di, do, dl, g_k = d_in, d_out_o, d_out_lse, g_step
         else:
             di, do, dl = torch.empty_like(d_in), torch.empty_like(d_out_o), torch.empty_like(d_out_lse)
-            st_k = step_factory(di, do, dl)
+            g_k = _capture(step_factory(di, do, dl).run, s)
         ho = torch.empty(do.numel(), dtype=do.dtype, pin_memory=True)
         hl = torch.empty(dl.numel(), dtype=dl.dtype, pin_memory=True)
-        sets.append((di, do, dl, st_k, ho, hl))
+        sets.append((di, do, dl, g_k, ho, hl))
     h_in = torch.empty(d_in.numel(), dtype=d_in.dtype, pin_memory=True)
     h_in.copy_(d_in.cpu())
     s_h2d = torch.cuda.Stream(device=dev)
     s_d2h = torch.cuda.Stream(device=dev)
-    for _, _, _, st_k, _, _ in sets:          # eager run: kernels loaded, tensor maps cached
-        with torch.cuda.stream(s):
-            st_k.run(s)
-    torch.cuda.synchronize()
-    U = 8
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_comp = [torch.cuda.Event() for _ in range(2)]
     ev_out = [torch.cuda.Event() for _ in range(2)]
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=s):
-        s_h2d.wait_stream(s)
-        s_d2h.wait_stream(s)
-        for i in range(U):
+    for k in range(2):
+        ev_comp[k].record(s)
+        ev_out[k].record(s)
+    torch.cuda.synchronize()
+
+    def run_e2e(K):
+        for i in range(K):
             k = i % 2
-            di, do, dl, st_k, ho, hl = sets[k]
-            if i >= 2:
-                s_h2d.wait_event(ev_comp[k])           # step i-2 no longer reads this input set
+            di, do, dl, g_k, ho, hl = sets[k]
+            s_h2d.wait_event(ev_comp[k])          # step i-2 no longer reads this input set
             with torch.cuda.stream(s_h2d):
                 di.copy_(h_in, non_blocking=True)
             ev_in[k].record(s_h2d)
             s.wait_event(ev_in[k])
-            if i >= 2:
-                s.wait_event(ev_out[k])                # step i-2's outputs were read back
-            st_k.run(s)
+            s.wait_event(ev_out[k])                # step i-2's outputs were read back
+            with torch.cuda.stream(s):
+                g_k.replay()
             ev_comp[k].record(s)
             s_d2h.wait_event(ev_comp[k])
             with torch.cuda.stream(s_d2h):
                 ho.copy_(do, non_blocking=True)
                 hl.copy_(dl, non_blocking=True)
             ev_out[k].record(s_d2h)
-        s.wait_stream(s_h2d)
-        s.wait_stream(s_d2h)
+
+    run_e2e(8)
     torch.cuda.synchronize()
-    for _ in range(2):
-        g.replay()
-    ms_u = _replay_ms(g, s, 1)
-    reps = max(-(-steps // U), int(math.ceil(300.0 / max(ms_u, 1e-3))))
-    ms_e2e = _replay_ms(g, s, reps) / U
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s_h2d)
+    run_e2e(10)
+    s_h2d.wait_stream(s_d2h)
+    e1.record(s_h2d)
+    torch.cuda.synchronize()
+    ms10 = e0.elapsed_time(e1) / 10
+    K = max(steps, int(math.ceil(300.0 / max(ms10, 1e-3))))
+    e0.record(s_h2d)
+    run_e2e(K)
+    s_h2d.wait_stream(s_d2h)
+    e1.record(s_h2d)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1) / K
     # breakdown: the copies alone, the compute alone
     ho, hl = sets[0][4], sets[0][5]
 
@@ -892,12 +898,12 @@ def e2e_measure(step_factory, d_in, d_out_o, d_out_lse, g_step, step, s, dev, st
     ms_comp = _replay_ms(g_step, s, 20)
     h2d_bytes = d_in.numel() * d_in.element_size()
     d2h_bytes = d_out_o.numel() * d_out_o.element_size() + d_out_lse.numel() * d_out_lse.element_size()
-    return {"ms_per_step": ms_e2e, "timed_steps": reps * U, "h2d_bytes_per_step": h2d_bytes,
+    return {"ms_per_step": ms_e2e, "timed_steps": K, "h2d_bytes_per_step": h2d_bytes,
             "d2h_bytes_per_step": d2h_bytes,
             "breakdown_ms": {"h2d": ms_h2d, "compute": ms_comp, "d2h": ms_d2h,
                              "h2d_gbs": h2d_bytes / (ms_h2d * 1e-3) / 1e9, "d2h_gbs": d2h_bytes / (ms_d2h * 1e-3) / 1e9},
             "how": "pinned host buffers, H2D of the step inputs and D2H of o/lse every step, double-buffered on "
-                   "separate copy streams; %d pipelined steps per CUDA graph (copies and kernels)" % U}
+                   "separate copy streams, the step's kernels replayed from its CUDA graph"}
 
 
 def run_decode(args):
