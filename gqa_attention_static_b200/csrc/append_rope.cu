@@ -22,9 +22,10 @@
 //
 // Work: one CTA per (request, layer) and group of rows (one row for a decode
 // step, 8 consecutive rows of a prompt, so that a long padded prompt batch
-// does not launch a CTA per padded row); 128 threads cover, per row, (Hq +
-// Hkv) heads x 16 groups of 4 rotary pairs plus Hkv x 16 16-byte pieces of the
-// V copy.  The op is small next to the attention; it exists so the caller
+// does not launch a CTA per padded row).  A row's items are (Hq + Hkv) heads
+// x 16 groups of 4 rotary pairs plus Hkv x 16 16-byte pieces of the V copy;
+// the CTA's (row, item) pairs share one index space over its threads (one
+// item per thread for a decode row).  The op is small next to the attention; it exists so the caller
 // never crosses to the host between the projection and the attention.
 #include "common.cuh"
 
@@ -52,7 +53,7 @@ struct AppendParams {
 };
 
 template <bool Fp8>
-__global__ void __launch_bounds__(128) append_rope_kernel(const __grid_constant__ AppendParams p) {
+__global__ void __launch_bounds__(512) append_rope_kernel(const __grid_constant__ AppendParams p) {
     // a kernel launched behind this one with programmatic stream serialisation
     // (the decode) may start its own prologue now; it waits for this grid's
     // completion (griddepcontrol.wait) before it reads q or the cache
@@ -66,20 +67,24 @@ __global__ void __launch_bounds__(128) append_rope_kernel(const __grid_constant_
         nn = nn < 0 ? 0 : p.S;
     }
     const int p0 = __ldg(p.pos0 + b);
-    const int t_end = min(nn, (static_cast<int>(blockIdx.x) + 1) * p.rows_per_cta);
-    for (int t = blockIdx.x * p.rows_per_cta; t < t_end; ++t) {
+    const int t_first = static_cast<int>(blockIdx.x) * p.rows_per_cta;
+    const int nrows = min(nn, t_first + p.rows_per_cta) - t_first;
+    const int qh = p.rotate_q ? p.Hq : 0;    // query heads this call rotates
+    const int nrot = (qh + p.Hkv) * 16;      // items of 4 rotary pairs per row
+    const int ncopy = p.Hkv * 16;            // 16-byte pieces of V rows per row
+    const int nitems = nrot + ncopy;
+    // (row, item) pairs of the CTA's rows in one index space, so that every
+    // thread has at most a couple of items and their loads are in flight together
+    for (int idx = threadIdx.x; idx < nrows * nitems; idx += blockDim.x) {
+        const int t = t_first + idx / nitems;
+        const int it = idx - (t - t_first) * nitems;
         const int pos = p0 + t;
         if (pos < 0 || pos >= p.T) {
-            if (threadIdx.x == 0 && blockIdx.z == 0) report(p.status, ARK_DEV_BAD_POS);
+            if (it == 0 && blockIdx.z == 0) report(p.status, ARK_DEV_BAD_POS);
             continue;
         }
-
-        const int qh = p.rotate_q ? p.Hq : 0;    // query heads this call rotates
-        const int nrot = (qh + p.Hkv) * 16;      // items of 4 rotary pairs
-        const int ncopy = p.Hkv * 16;            // 16-byte pieces of V rows
         const float4* trow = reinterpret_cast<const float4*>(p.table + static_cast<size_t>(pos) * 64);
-
-        for (int it = threadIdx.x; it < nrot + ncopy; it += blockDim.x) {
+        {
             if (it < nrot) {
                 const int head = it >> 4;
                 const int pg = it & 15;           // pairs 4pg .. 4pg+3
@@ -208,10 +213,15 @@ ark_status launch_append(AppendParams& prm, int L, bool fp8, cudaStream_t stream
     // enough work for its own CTA
     prm.rows_per_cta = (prm.S >= 64 && !prm.rotate_q) ? 8 : 1;
     dim3 grid((prm.S + prm.rows_per_cta - 1) / prm.rows_per_cta, prm.B, L);
+    // one thread per item of a row with the query heads ((Hq + 2 Hkv) x 16 = 320 for the
+    // decoder's heads), two per item of the eight K/V-only rows of a CTA otherwise
+    const int items = ((prm.rotate_q ? prm.Hq : 0) + 2 * prm.Hkv) * 16 * prm.rows_per_cta;
+    int threads = items < 512 ? ((items + 31) / 32) * 32 : 256;
+    if (threads > 512) threads = 512;
     if (fp8)
-        append_rope_kernel<true><<<grid, 128, 0, stream>>>(prm);
+        append_rope_kernel<true><<<grid, threads, 0, stream>>>(prm);
     else
-        append_rope_kernel<false><<<grid, 128, 0, stream>>>(prm);
+        append_rope_kernel<false><<<grid, threads, 0, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
 }
 
