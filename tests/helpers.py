@@ -9,12 +9,21 @@ Tolerances (fp64 oracle as reference):
         an absolute floor near lse = 0 where a relative bound is undefined).
   RoPE outputs and cache writes: bit-exact.
 """
+import os
+
 import numpy as np
 import torch
 
 O_ABS = 1e-2
 O_REL = 2.0 ** -8
 LSE_REL = 1e-3
+# below this magnitude the bf16 rounding of o alone (at most 2^-8 |o|) stays
+# under the literal 1e-2 bound, so there the literal bound is the meaningful one
+O_LITERAL_BELOW = 2.56
+
+# per check_o call: (test, what, max |o - o_ref|, elements with |o_ref| < 2.56 and
+# |o - o_ref| > 1e-2, elements with |o_ref| < 2.56); printed at the end of the run
+MARGINS = []
 
 
 def bits(x: torch.Tensor) -> np.ndarray:
@@ -32,6 +41,10 @@ def check_o(got: np.ndarray, ref: np.ndarray, what: str = "o") -> float:
     assert got.shape == ref.shape, (got.shape, ref.shape)
     assert np.isfinite(ref).all(), f"{what}: oracle produced non-finite values"
     err = np.abs(got - ref)
+    small = np.abs(ref) < O_LITERAL_BELOW
+    MARGINS.append((os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0], what,
+                    float(np.nanmax(err)) if err.size else 0.0, int(np.sum(small & ~(err <= O_ABS))),
+                    int(np.sum(small))))
     bound = O_ABS + O_REL * np.abs(ref)
     bad = ~(err <= bound)
     if bad.any():

@@ -4,9 +4,10 @@ reserved all memory up front, or in a plugin whose framework owns the
 allocator).  It takes no workspace and uses the library's own fixed scratch.
 
 Called here through the C ABI (ctypes, raw device pointers) and checked
-against ark_attn_decode, the entry point with a caller workspace, within the
-same tolerances as every other decode test, on two calls in a row (the second
-call finds the scratch as the first one left it).  This file is collected
+against ark_attn_decode, the entry point with a caller workspace, and against
+the fp64 oracle, within the same tolerances as every other decode test, on
+two calls in a row (the second call finds the scratch as the first one left
+it).  This file is collected
 last so that a stop-at-first-failure run has run every other test first; it
 also passes alone in a fresh process, where its first call sets the scratch
 up on the device.
@@ -17,9 +18,10 @@ import math
 import pytest
 import torch
 
+import oracle
 from gqa_attention_static_b200 import ops
 from gqa_attention_static_b200 import workloads as W
-from tests.helpers import check_lse, check_o, f64
+from tests.helpers import bits, check_lse, check_o, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -51,7 +53,7 @@ def no_alloc_c_abi(lib, q, ck, cv, kv, mode, max_splits, status):
 
 
 @pytest.mark.parametrize("case", ["ragged512", "long2048", "masked"])
-def test_no_alloc_matches_workspace_decode_twice(case):
+def test_no_alloc_matches_workspace_decode_twice(oracle_lib, case):
     lib = ops.load()
     assert lib.ark_attn_decode_noalloc_scratch_bytes() < 8 << 20
     dev = "cuda"
@@ -66,6 +68,8 @@ def test_no_alloc_matches_workspace_decode_twice(case):
     cv = batch.cache_v[0].to(dev)
     kv = batch.pos0.to(dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
+    o_or, lse_or = oracle.decode(bits(batch.q[0]), bits(batch.cache_k[0]), bits(batch.cache_v[0]),
+                                 batch.pos0.numpy(), SCALE, static_mode=(mode == ops.ARK_MASKED_STATIC))
     for max_splits in (8, 32):
         o_ref, lse_ref = with_workspace(q, ck, cv, kv, mode, max_splits)
         for _ in range(2):
@@ -74,6 +78,8 @@ def test_no_alloc_matches_workspace_decode_twice(case):
             assert int(status.item()) == 0
             check_o(f64(o), f64(o_ref), "o (no-alloc vs workspace)")
             check_lse(f64(lse), f64(lse_ref), "lse (no-alloc vs workspace)")
+            check_o(f64(o), o_or, "o (no-alloc vs oracle)")
+            check_lse(f64(lse), lse_or, "lse (no-alloc vs oracle)")
 
 
 def test_no_alloc_rejects_batches_beyond_its_limits():
