@@ -18,32 +18,40 @@
 //     first), then request, KV head and layer, and the kernel is persistent:
 //     one CTA per SM walks its units in snake order over that list, so the
 //     SMs never drain between layers or tiles.
+//   - The units of a CTA form one stream of steps (unit, 64-key block) with no
+//     break at unit boundaries: the score MMAs run ahead of the P V MMAs by up
+//     to the two S buffers of each tile (possibly into the next unit), and each
+//     unit's epilogue runs after the softmax of the next unit's first block, so
+//     neither the tensor cores nor the softmax warps wait for a unit to drain.
 //   - Warp roles.  Warp 10 computes the unit list entries (a binary search
 //     over position levels, from pos0/n_new on the device), publishes them in
-//     a 4-entry ring, loads each unit's Q tiles by TMA into one of two Q slots
-//     (so the next unit's Q streams in while this one computes), and issues
-//     the TMA stores of each finished unit's output.  Warp 0 streams the K and
-//     V blocks (64 keys, 16 KB each) through 3-stage rings.  Warp 1 issues the
-//     MMAs from one thread.  Warps 2..5 run the softmax and epilogue of tile A,
-//     warps 6..9 those of tile B, one thread per row.  With RoPE on load, warps
-//     11..14 rotate the landed Q tiles in shared memory before the first MMA.
+//     a 4-entry ring and loads each unit's Q tiles by TMA into one of two Q
+//     slots; a slot is reloaded as soon as the last score MMA that reads it has
+//     completed.  Warp 0 streams the K and V blocks (64 keys, 16 KB each)
+//     through 3-stage rings.  Two warps issue the MMAs, each from one thread:
+//     warp 1 the scores S = Q K^T, warp 11 the products O += P V, so that the
+//     waits of one chain do not hold up the other (each thread's MMAs complete
+//     in issue order, and its commits track only its own).  Warps 2..5 run the
+//     softmax and epilogue of tile A, warps 6..9 those of tile B, one thread
+//     per row.  With RoPE on load, warps 12..15 rotate the landed Q tiles in
+//     shared memory before the first MMA.
 //   - Tensor memory (512 columns): for each tile two S buffers of 64 columns
 //     (S = Q K^T of a block: 8 MMAs of 128x64x16) and an O accumulator of 128
 //     columns (O += P V: 4 MMAs of 128x128x16 with P, bf16, read from tensor
 //     memory over its own S columns and V an MN-major shared-memory operand).
-//     The MMA warp runs QK of block j+1 ahead of PV of block j, so the softmax
-//     of one block overlaps the scores of the next and the other tile's work.
+//     A unit's last block computes only the 16-key groups that reach into its
+//     causal range (fewer score columns, fewer P V steps).
 //   - Softmax in the log2 domain with a lazily moved reference max: O is
 //     rescaled in tensor memory only when a row's block max exceeds its
 //     reference by more than 2^8.  Only blocks that reach past a row's
 //     position are masked; V rows past the unit's causal range are zeroed in
 //     shared memory before their (zero-weight) use, so garbage past the valid
 //     rows cannot turn into NaN.  Rows past n_new[b] are computed on whatever
-//     the padded q holds and never written.
-//   - Epilogue: O / (sum of the bf16 weights) as bf16 into the unit's finished
-//     Q tile in shared memory (the layout of the Q load), then warp 10 stores
-//     it by TMA: one box per 64-dim half for a tile whose 16 positions are all
-//     live, one box per live position otherwise.  lse by plain stores.
+//     the padded q holds and never written.  The exponent arguments and the
+//     row sums are computed on packed fp32 pairs.
+//   - Epilogue: O / (sum of the bf16 weights) as bf16, written by each row's
+//     thread straight to its 256-byte output row (16-byte stores); lse by plain
+//     stores.
 //
 // Roofline: per request of L prompt rows and per layer, 4096 * L * (L + 1)
 // FLOPs (the causal half of QK^T and PV for 16 heads) against 9216 * L bytes
@@ -72,12 +80,13 @@ constexpr int kDescs = 4;                // unit-list entries in flight
 
 // warps
 constexpr int kWarpKV = 0;
-constexpr int kWarpMMA = 1;
+constexpr int kWarpMMA = 1;              // score MMAs (S = Q K^T); allocates the tensor memory
 constexpr int kWarpSoft0 = 2;            // 2..5 tile A, 6..9 tile B
 constexpr int kWarpQ = 10;
-constexpr int kWarpRot0 = 11;            // 11..14 (RoPE on load only)
-constexpr int kThreads = 352;
-constexpr int kThreadsRope = 480;
+constexpr int kWarpPV = 11;              // P V MMAs
+constexpr int kWarpRot0 = 12;            // 12..15 (RoPE on load only)
+constexpr int kThreads = 384;
+constexpr int kThreadsRope = 512;
 constexpr int kRotThreads = 128;
 
 // shared memory map (the dynamic shared memory base is 1024-aligned)
@@ -89,7 +98,8 @@ constexpr int kBarDesc = 0;                          // [kDescs] unit-list entry
 constexpr int kBarDescFree = kBarDesc + kDescs;      // [kDescs] entry read by every consumer warp
 constexpr int kBarQFull = kBarDescFree + kDescs;     // [kQSlots] Q tiles landed (tx)
 constexpr int kBarQRot = kBarQFull + kQSlots;        // [kQSlots] Q tiles rotated (RoPE on load)
-constexpr int kBarKFull = kBarQRot + kQSlots;        // [kStages]
+constexpr int kBarQEmpty = kBarQRot + kQSlots;       // [kQSlots] every score MMA of the slot's unit done
+constexpr int kBarKFull = kBarQEmpty + kQSlots;      // [kStages]
 constexpr int kBarKEmpty = kBarKFull + kStages;
 constexpr int kBarVFull = kBarKEmpty + kStages;
 constexpr int kBarVEmpty = kBarVFull + kStages;
@@ -98,14 +108,9 @@ constexpr int kBarPFull = kBarSFull + 4;             // [tile][buffer] P of a bl
 constexpr int kBarPvDone = kBarPFull + 4;            // [tile] one phase per PV
 constexpr int kBarODone = kBarPvDone + 2;            // [tile] one phase per unit: every MMA of the tile done
 constexpr int kBarOEmpty = kBarODone + 2;            // [tile] O read out of TMEM (count 128)
-// [tile][Q slot] O staged in shared memory (count 128).  One per slot: the
-// softmax warps may finish two consecutive units before warp 10 flushes the
-// first, but never two units of the same slot (the slot's next unit needs Q
-// tiles that are loaded only after the flush), so each barrier stays within
-// one phase of its waiter.
-constexpr int kBarStaged = kBarOEmpty + 2;
-constexpr int kBarDrain = kBarStaged + 4;            // MMAs in flight when the MMA warp gives up
-constexpr int kNumBars = kBarDrain + 1;
+constexpr int kBarSFree = kBarOEmpty + 2;           // [tile][buffer] the PV that read a block's P is done
+constexpr int kBarDrain = kBarSFree + 4;             // [issuing warp] MMAs in flight when it gives up
+constexpr int kNumBars = kBarDrain + 2;
 constexpr int kOffDesc = (kOffBar + kNumBars * 8 + 15) & ~15;
 struct UnitDesc {
     int l, b, g, t0;      // layer (of the launch), request, KV head, first position of tile A (call index)
@@ -126,12 +131,12 @@ constexpr uint32_t kTmemCols = 512;
 
 // instruction descriptors (kind::f16): D fp32, A/B bf16, M = 128
 constexpr uint32_t kIdescF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 4) << 24);
-constexpr uint32_t kIdescQK = kIdescF16 | ((64u >> 3) << 17);                // N = 64 keys, B = K (K-major)
+// QK: N = keys of the block (64, or fewer 16-key groups on a unit's last block), B = K (K-major)
 constexpr uint32_t kIdescPV = kIdescF16 | ((128u >> 3) << 17) | (1u << 16);  // N = 128 dims, B = V (MN-major)
 
 constexpr float kLazyRescale = 8.0f;     // log2 units: rescale O only past a factor 2^8
 
-// layers per launch: five tensor maps per layer in the kernel parameters
+// layers per launch: three tensor maps per layer in the kernel parameters
 constexpr int kLayersPerLaunch = 36;
 // layers per chunk of the unit order (the K/V rows of a chunk stay in L2 while its units run)
 constexpr int kLayerChunk = 12;
@@ -140,14 +145,14 @@ struct Params {
     CUtensorMap qmap[kLayersPerLaunch];   // q as (128, 8, Hq/8, B*S), box (64, 8, 1, 16)
     CUtensorMap kmap[kLayersPerLaunch];   // cache_k as (128, Hkv, B*T), box (64, 1, 64)
     CUtensorMap vmap[kLayersPerLaunch];
-    CUtensorMap omap[kLayersPerLaunch];   // o as q, box (64, 8, 1, 16): a tile's 64-dim half
-    CUtensorMap omap1[kLayersPerLaunch];  // o as q, box (64, 8, 1, 1): one position
+    __nv_bfloat16* o[kLayersPerLaunch];   // [B, S, Hq, 128]
     float* lse[kLayersPerLaunch];         // [B, Hq, S]
     const int32_t* pos0;
     const int32_t* n_new;
     uint32_t* status;
     const float4* table;                  // rotary table [T][64] {cos, sin} (fp32), for RoPE on load
     int B, S, T, Hq, Hkv, L, Lc;
+    int o_align32;                        // every o[l] 32-byte aligned: 32-byte stores
     float scale_log2;
 };
 static_assert(sizeof(Params) <= 32000, "kernel parameter space");
@@ -286,6 +291,7 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const unsigned full = 0xffffffffu;
     if (smem_u32(smem) & 1023u) {                           // the swizzled layouts need 1024-byte alignment
         if (threadIdx.x == 0) report(p.status, ARK_DEV_TIMEOUT);
         return;
@@ -298,12 +304,10 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNumBars; ++i) {
             uint32_t cnt = 1;
-            if ((i >= kBarPFull && i < kBarPFull + 4) || (i >= kBarOEmpty && i < kBarOEmpty + 2) ||
-                (i >= kBarStaged && i < kBarStaged + 4))
-                cnt = kRows;
+            if ((i >= kBarPFull && i < kBarPFull + 4) || (i >= kBarOEmpty && i < kBarOEmpty + 2)) cnt = kRows;
             if (i >= kBarQRot && i < kBarQRot + kQSlots) cnt = kRotThreads;
-            // readers of an entry: the K/V producer, the MMA warp, 8 softmax warps (+4 rotation warps)
-            if (i >= kBarDescFree && i < kBarDescFree + kDescs) cnt = Rope ? 14 : 10;
+            // readers of an entry: the K/V producer, the two MMA warps, 8 softmax warps (+4 rotation warps)
+            if (i >= kBarDescFree && i < kBarDescFree + kDescs) cnt = Rope ? 15 : 11;
             mbar_init(&bars[i], cnt);
         }
         fence_mbar_init();
@@ -329,44 +333,16 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
     auto fail = [&]() { report(p.status, ARK_DEV_TIMEOUT); };
 
     if (warp == kWarpQ) {
-        // ================================================= unit list, Q loads, O stores
+        // ================================================= unit list, Q loads
         bool ok = true, bad = false;
         const int per_head = count_units(p, 0, lane, bad);
-        const bool any_bad = __any_sync(0xffffffffu, bad);
+        const bool any_bad = __any_sync(full, bad);
         if (c == 0 && lane == 0 && any_bad) report(p.status, ARK_DEV_BAD_POS);
         const long long total = static_cast<long long>(p.L) * p.Hkv * per_head;
-        int staged[4] = {0, 0, 0, 0};         // [tile][slot]: stagings of tile X in slot s consumed
-        UnitDesc prev[2];                     // entries of units k-1, k-2 (ring by k & 1)
-        // store the finished output of unit u (its Q slot u & 1), then free that slot
-        auto flush = [&](int u, const UnitDesc& d) {
-            const int ntile = d.nblk_b > 0 ? 2 : 1;
-            for (int x = 0; x < ntile && ok; ++x) {
-                const int sb = x * 2 + (u & 1);
-                if (!(ok = mbar_wait(&bars[kBarStaged + sb], staged[sb] & 1))) break;
-                ++staged[sb];
-                const int t0 = d.t0 + x * kPos;
-                const int live = min(kPos, d.nn - t0);
-                const uint8_t* st = smem + kOffQ + (u & 1) * kQSlot + x * kQTile;
-                const int row = d.b * p.S + t0;
-                if (live == kPos) {
-                    tma_store_4d(&p.omap[d.l], st, 0, 0, d.g, row);
-                    tma_store_4d(&p.omap[d.l], st + kQHalf, 64, 0, d.g, row);
-                } else {
-                    for (int pp = 0; pp < live; ++pp) {
-                        tma_store_4d(&p.omap1[d.l], st + pp * 1024, 0, 0, d.g, row + pp);
-                        tma_store_4d(&p.omap1[d.l], st + kQHalf + pp * 1024, 64, 0, d.g, row + pp);
-                    }
-                }
-            }
-            bulk_commit();
-            bulk_wait_read();                 // the slot may take the next Q tiles
-        };
-        int k = 0;
         int q_issued = -1;                    // last unit whose Q was loaded
-        for (;; ++k) {
+        for (int k = 0;; ++k) {
             const UnitDesc d = unit_desc(p, snake_unit(k, c, G), per_head, total, lane);
             if (lane == 0) {
-                if (k >= 2 && ok) flush(k - 2, prev[k & 1]);
                 // entry slot k % 4 last held unit k - 4: every consumer warp has read it
                 if (k >= kDescs && ok)
                     ok = mbar_wait(&bars[kBarDescFree + (k & (kDescs - 1))], ((k / kDescs) - 1) & 1);
@@ -379,8 +355,10 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
                     descs[k & (kDescs - 1)] = d;
                 }
                 mbar_arrive(&bars[kBarDesc + (k & (kDescs - 1))]);
+                const int qs = k & 1;
+                // the slot last held unit k - 2: its score MMAs have completed
+                if (ok && !d.end && k >= 2) ok = mbar_wait(&bars[kBarQEmpty + qs], ((k - 2) >> 1) & 1);
                 if (ok && !d.end) {
-                    const int qs = k & 1;
                     const int ntile = d.nblk_b > 0 ? 2 : 1;
                     mbar_arrive_expect_tx(&bars[kBarQFull + qs], ntile * kQTile);
                     uint8_t* qd = smem + kOffQ + qs * kQSlot;
@@ -391,21 +369,16 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
                     }
                     q_issued = k;
                 }
-                prev[k & 1] = d;
             }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            ok = __shfl_sync(full, ok ? 1 : 0, 0) != 0;
             if (d.end || !ok) break;
         }
-        if (lane == 0) {
-            if (ok && k >= 1 && !prev[(k - 1) & 1].end) flush(k - 1, prev[(k - 1) & 1]);
-            if (!ok) {
-                fail();
-                // every Q copy issued has landed before the shared memory can go away
-                if (q_issued >= 0) (void)mbar_wait(&bars[kBarQFull + (q_issued & 1)], (q_issued >> 1) & 1);
-                if (q_issued >= 1)
-                    (void)mbar_wait(&bars[kBarQFull + ((q_issued - 1) & 1)], ((q_issued - 1) >> 1) & 1);
-            }
-            bulk_wait_read();
+        if (lane == 0 && !ok) {
+            fail();
+            // every Q copy issued has landed before the shared memory can go away
+            if (q_issued >= 0) (void)mbar_wait(&bars[kBarQFull + (q_issued & 1)], (q_issued >> 1) & 1);
+            if (q_issued >= 1)
+                (void)mbar_wait(&bars[kBarQFull + ((q_issued - 1) & 1)], ((q_issued - 1) >> 1) & 1);
         }
         __syncwarp();
     } else if (warp == kWarpKV) {
@@ -448,64 +421,99 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
             }
         }
     } else if (warp == kWarpMMA) {
-        // ================================================= MMA issuer
-        // waits are AND-ed over the warp so that the __syncwarp()s below are reached by all lanes
+        // ================================================= score MMAs (S = Q K^T)
+        // Runs ahead of the softmax by up to the two S buffers of each tile: a buffer is reused once
+        // the PV that read its P has completed.  Waits are AND-ed over the warp so that the
+        // __syncwarp()s below are reached by all lanes.
         bool ok = true;
         int sq[2] = {0, 0};       // QK blocks issued per tile (S buffer = sq & 1)
-        int pv[2] = {0, 0};       // PV blocks issued per tile (P buffer = pv & 1)
-        int uo[2] = {0, 0};       // units finished per tile (O phases)
-        int gk = 0;               // K/V blocks consumed
+        int g = 0;                // K/V blocks consumed
+        // descriptors of the shared-memory operands at the region bases; offsets are added in 16-byte units
+        const uint64_t dq0 = umma_desc_sw128(sbase + kOffQ, 16, 1024);
+        const uint64_t dk0 = umma_desc_sw128(sbase + kOffK, 16, 1024);
         for (int k = 0; ok; ++k) {
             UnitDesc d;
-            if (!(ok = __all_sync(0xffffffffu, wait_desc(k, d)))) break;
+            if (!(ok = __all_sync(full, wait_desc(k, d)))) break;
             free_desc(k);
             if (d.end) break;
-            const int qs = k & 1;
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[(Rope ? kBarQRot : kBarQFull) + qs], (k >> 1) & 1))))
+            if (!(ok = __all_sync(full, mbar_wait(&bars[(Rope ? kBarQRot : kBarQFull) + (k & 1)], (k >> 1) & 1))))
                 break;
             const int nbx[2] = {d.nblk_a, d.nblk_b};
             const int nb = max(d.nblk_a, d.nblk_b);
             const int kv_end = d.p0 + min(d.t0 + (d.nblk_b > 0 ? kUnitPos : kPos), d.nn);
-            const int g0 = gk;
-            auto issue_qk = [&](int j) -> bool {
-                const int st = (g0 + j) % kStages;
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarKFull + st], ((g0 + j) / kStages) & 1)))
-                    return false;
+            const uint64_t qslot = dq0 + static_cast<uint64_t>(((k & 1) * kQSlot) >> 4);
+            for (int j = 0; j < nb && ok; ++j, ++g) {
+                const int st = g % kStages;
+                if (!(ok = __all_sync(full, mbar_wait(&bars[kBarKFull + st], (g / kStages) & 1)))) break;
+                for (int x = 0; x < 2 && ok; ++x)
+                    if (j < nbx[x] && sq[x] >= 2)
+                        ok = __all_sync(full, mbar_wait(&bars[kBarSFree + x * 2 + (sq[x] & 1)],
+                                                        ((sq[x] >> 1) - 1) & 1));
+                if (!ok) break;
+                // scores past the unit's causal range are masked by the softmax: the last block computes
+                // only the 16-key groups that reach into the range (the columns past them are never used
+                // unmasked)
+                const int n16 = min(kBN, (kv_end - j * kBN + 15) & ~15);
+                const uint32_t idesc = kIdescF16 | (static_cast<uint32_t>(n16 >> 3) << 17);
                 if (lane == 0) {
                     tc_fence_after();
-                    const uint32_t kb = sbase + kOffK + st * kKV;
+                    const uint64_t kb = dk0 + static_cast<uint64_t>((st * kKV) >> 4);
+#pragma unroll
                     for (int x = 0; x < 2; ++x) {
                         if (j >= nbx[x]) continue;
                         const uint32_t dcol = tmem + kColS + x * 128 + (sq[x] & 1) * kBN;
-                        const uint32_t qa = sbase + kOffQ + qs * kQSlot + x * kQTile;
+                        const uint64_t qa = qslot + static_cast<uint64_t>((x * kQTile) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t sub = (kk & 3) * 32;
-                            umma_f16(dcol, umma_desc_sw128(qa + (kk >> 2) * kQHalf + sub, 16, 1024),
-                                     umma_desc_sw128(kb + (kk >> 2) * kKHalf + sub, 16, 1024), kIdescQK,
-                                     kk > 0 ? 1u : 0u);
+                            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4);
+                            const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * kKHalf + (kk & 3) * 32) >> 4);
+                            umma_f16(dcol, qa + off, kb + koff, idesc, kk > 0 ? 1u : 0u);
                         }
                         umma_commit(&bars[kBarSFull + x * 2 + (sq[x] & 1)]);
                     }
                     umma_commit(&bars[kBarKEmpty + st]);
+                    // the unit's last score MMAs: its Q slot may take another unit once they complete
+                    if (j == nb - 1) umma_commit(&bars[kBarQEmpty + (k & 1)]);
                 }
                 __syncwarp();
                 for (int x = 0; x < 2; ++x)
                     if (j < nbx[x]) ++sq[x];
-                return true;
-            };
-            if (!(ok = issue_qk(0))) break;
-            for (int j = 0; j < nb && ok; ++j) {
-                if (j + 1 < nb && !(ok = issue_qk(j + 1))) break;
-                const int st = (g0 + j) % kStages;
-                if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarVFull + st], ((g0 + j) / kStages) & 1))))
-                    break;
-                const int live = kv_end - j * kBN;            // rows of the block inside the causal range
-                if (live < kBN) {
-                    // rows past it may hold anything (NaN included): P is 0 there, 0 * NaN is not
+            }
+        }
+        if (!ok) {
+            if (lane == 0) {
+                fail();
+                umma_commit(&bars[kBarDrain]);
+                (void)mbar_wait(&bars[kBarDrain], 0);            // MMAs issued so far have completed
+            }
+            __syncwarp();
+        }
+    } else if (warp == kWarpPV) {
+        // ================================================= P V MMAs (O += P V)
+        bool ok = true;
+        int pv[2] = {0, 0};       // PV blocks issued per tile (P buffer = pv & 1)
+        int uo[2] = {0, 0};       // units whose last PV was issued, per tile (O phases)
+        int g = 0;                // K/V blocks consumed
+        const uint64_t dv0 = umma_desc_sw128(sbase + kOffV, kKHalf, 1024);
+        for (int k = 0; ok; ++k) {
+            UnitDesc d;
+            if (!(ok = __all_sync(full, wait_desc(k, d)))) break;
+            free_desc(k);
+            if (d.end) break;
+            const int nbx[2] = {d.nblk_a, d.nblk_b};
+            const int nb = max(d.nblk_a, d.nblk_b);
+            const int kv_end = d.p0 + min(d.t0 + (d.nblk_b > 0 ? kUnitPos : kPos), d.nn);
+            for (int j = 0; j < nb && ok; ++j, ++g) {
+                const int st = g % kStages;
+                if (!(ok = __all_sync(full, mbar_wait(&bars[kBarVFull + st], (g / kStages) & 1)))) break;
+                const int live = min(kBN, kv_end - j * kBN);      // rows of the block inside the causal range
+                const int ksteps = min(kBN, (live + 15) & ~15) >> 4;   // 16-row groups that reach into it
+                if (live < ksteps * 16) {
+                    // the rows of the last group past the range may hold anything (NaN included): P is 0
+                    // there, 0 * NaN is not
                     uint8_t* vt = smem + kOffV + st * kKV;
-                    for (int i = lane; i < (kBN - max(live, 0)) * 16; i += 32) {
-                        const int r = max(live, 0) + (i >> 4), part = i & 15;
+                    for (int i = lane; i < (ksteps * 16 - live) * 16; i += 32) {
+                        const int r = live + (i >> 4), part = i & 15;
                         *reinterpret_cast<uint4*>(vt + (part >> 3) * kKHalf + r * 128 + (part & 7) * 16) =
                             make_uint4(0, 0, 0, 0);
                     }
@@ -516,43 +524,42 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
                     if (j >= nbx[x]) continue;
                     // the first PV of a unit overwrites O_x: the previous unit's epilogue must have read it
                     if (j == 0 && uo[x] > 0 &&
-                        !(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarOEmpty + x], (uo[x] - 1) & 1))))
+                        !(ok = __all_sync(full, mbar_wait(&bars[kBarOEmpty + x], (uo[x] - 1) & 1))))
                         break;
-                    if (!(ok = __all_sync(0xffffffffu,
-                                          mbar_wait(&bars[kBarPFull + x * 2 + (pv[x] & 1)], (pv[x] >> 1) & 1))))
+                    if (!(ok = __all_sync(full, mbar_wait(&bars[kBarPFull + x * 2 + (pv[x] & 1)], (pv[x] >> 1) & 1))))
                         break;
+                    const bool last = j == nbx[x] - 1;
                     if (lane == 0) {
                         tc_fence_after();
                         const uint32_t pa = tmem + kColS + x * 128 + (pv[x] & 1) * kBN;   // P: 32 columns
-                        const uint32_t vb = sbase + kOffV + st * kKV;
+                        const uint64_t vb = dv0 + static_cast<uint64_t>((st * kKV) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            umma_f16_ts(tmem + kColO + x * 128, pa + kk * 8,
-                                        umma_desc_sw128(vb + kk * 16 * 128, kKHalf, 1024), kIdescPV,
-                                        (j > 0 || kk > 0) ? 1u : 0u);
+                            if (kk < ksteps)
+                                umma_f16_ts(tmem + kColO + x * 128, pa + kk * 8, vb + static_cast<uint64_t>(kk * 128),
+                                            kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);   // 16 V rows = 2048 bytes
                         umma_commit(&bars[kBarPvDone + x]);
-                        if (j == nbx[x] - 1) umma_commit(&bars[kBarODone + x]);
+                        umma_commit(&bars[kBarSFree + x * 2 + (pv[x] & 1)]);
+                        if (last) umma_commit(&bars[kBarODone + x]);
                     }
                     __syncwarp();
                     ++pv[x];
+                    if (last) ++uo[x];
                 }
                 if (!ok) break;
                 if (lane == 0) umma_commit(&bars[kBarVEmpty + st]);
                 __syncwarp();
             }
-            gk = g0 + nb;
-            for (int x = 0; x < 2; ++x)
-                if (nbx[x] > 0) ++uo[x];
         }
         if (!ok) {
             if (lane == 0) {
                 fail();
-                umma_commit(&bars[kBarDrain]);
-                (void)mbar_wait(&bars[kBarDrain], 0);            // MMAs issued so far have completed
+                umma_commit(&bars[kBarDrain + 1]);
+                (void)mbar_wait(&bars[kBarDrain + 1], 0);        // MMAs issued so far have completed
             }
             __syncwarp();
         }
-    } else if (warp < kWarpQ) {
+    } else if (warp >= kWarpSoft0 && warp < kWarpQ) {
         // ================================================= softmax + epilogue of tile x
         const int x = (warp - kWarpSoft0) >> 2;         // 0: tile A (warps 2..5), 1: tile B (warps 6..9)
         const int quad = warp & 3;                      // TMEM lanes 32*quad .. +31
@@ -562,24 +569,63 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
         const uint32_t col_s = kColS + x * 128;
         const uint32_t col_o = kColO + x * 128;
         const float sl2 = p.scale_log2;
+        const uint64_t sl2x2 = f2_make(sl2, sl2);
         bool ok = true;
         int sq = 0;               // blocks processed (S/P buffer = sq & 1; also the PV count)
         int uo = 0;               // units finished (O phases)
+        // the unit whose output still sits in O_x: its epilogue runs after the next unit's first block
+        bool pend = false;
+        int e_l = 0, e_b = 0, e_g = 0, e_tr = 0, e_nn = 0;
+        float e_m = 0.f, e_sum = 0.f, e_rsum = 1.f;
+        auto epilogue = [&]() -> bool {
+            if (!__all_sync(full, mbar_wait(&bars[kBarODone + x], uo & 1))) return false;
+            ++uo;
+            tc_fence_after();
+            const float inv = 1.f / e_rsum;
+            // O row as bf16 pairs: read all of it before releasing O_x to the next unit's first PV
+            uint32_t w[64];
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+                uint32_t o[64];
+                tmem_ld32(lane_base + col_o + 64 * c2, *reinterpret_cast<uint32_t(*)[32]>(o));
+                tmem_ld32(lane_base + col_o + 64 * c2 + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    w[32 * c2 + i] = cvt_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+            }
+            tc_fence_before();
+            mbar_arrive(&bars[kBarOEmpty + x]);                // the next unit may overwrite O_x
+            if (e_tr < e_nn) {
+                const int h = e_g * kGroup + hh;
+                uint8_t* dst = reinterpret_cast<uint8_t*>(p.o[e_l]) +
+                               ((static_cast<size_t>(e_b) * p.S + e_tr) * p.Hq + h) * (kHeadDim * 2);
+                if (p.o_align32) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) st_global_v8(dst + 32 * q, &w[8 * q]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) st_global_v4(dst + 16 * q, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                }
+                p.lse[e_l][(static_cast<size_t>(e_b) * p.Hq + h) * p.S + e_tr] = (e_m + __log2f(e_sum)) * kLn2;
+            }
+            return true;
+        };
         for (int k = 0; ok; ++k) {
             UnitDesc d;
-            if (!(ok = __all_sync(0xffffffffu, wait_desc(k, d)))) break;
+            if (!(ok = __all_sync(full, wait_desc(k, d)))) break;
             free_desc(k);
             if (d.end) break;
             const int nbl = x ? d.nblk_b : d.nblk_a;
             if (nbl == 0) continue;                      // tile B of this unit has no live row
-            const int t0 = d.t0 + x * kPos;
-            const int tr = t0 + (r >> 3);                // this row's position (call index)
+            const int tr = d.t0 + x * kPos + (r >> 3);   // this row's position (call index)
             const int prow = d.p0 + tr;                  // and its absolute position
-            float m_ref = -INFINITY, e0 = 0.f, e1 = 0.f, r0 = 0.f, r1 = 0.f;
+            float m_ref = -INFINITY;
+            uint64_t esum = f2_make(0.f, 0.f), rsum = f2_make(0.f, 0.f);
             // every tcgen05.ld/st is .sync.aligned and sits on warp-uniform control flow
             for (int j = 0; j < nbl; ++j, ++sq) {
                 const int buf = sq & 1;
-                if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + x * 2 + buf], (sq >> 1) & 1)))) break;
+                if (!(ok = __all_sync(full, mbar_wait(&bars[kBarSFull + x * 2 + buf], (sq >> 1) & 1)))) break;
                 tc_fence_after();
                 const uint32_t scol = lane_base + col_s + buf * kBN;
                 uint32_t v[64];
@@ -594,7 +640,12 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
                 }
                 float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(v[i]));
+                for (int i = 0; i < 64; i += 8) {
+                    mx[0] = fmax3(mx[0], __uint_as_float(v[i + 0]), __uint_as_float(v[i + 1]));
+                    mx[1] = fmax3(mx[1], __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+                    mx[2] = fmax3(mx[2], __uint_as_float(v[i + 4]), __uint_as_float(v[i + 5]));
+                    mx[3] = fmax3(mx[3], __uint_as_float(v[i + 6]), __uint_as_float(v[i + 7]));
+                }
                 const float bm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
                 float alpha = 1.f;
                 bool rescale = false;
@@ -606,15 +657,37 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
                     rescale = true;
                 }
                 const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-                if (__any_sync(0xffffffffu, rescale)) {
-                    // O must hold the PV of every earlier block of the unit (the one before this
-                    // block may still run: QK of this block was issued before it)
-                    if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPvDone + x], (sq - 1) & 1)))) break;
+                const bool any_rescale = __any_sync(full, rescale);
+                if (any_rescale) {
+                    const uint64_t a2 = f2_make(alpha, alpha), z2 = f2_make(0.f, 0.f);
+                    esum = f2_fma(esum, a2, z2);
+                    rsum = f2_fma(rsum, a2, z2);
+                }
+                // P = exp2(s * scale_log2 - mu) as bf16 pairs: keys 2c, 2c+1 in column c of the block's S
+                // buffer (columns 0..31; the scores there are already in registers)
+                const uint64_t nmu = f2_make(-mu, -mu);
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float a0, a1;
+                        f2_split(f2_fma(f2_make(__uint_as_float(v[32 * h2 + 2 * i]),
+                                                __uint_as_float(v[32 * h2 + 2 * i + 1])), sl2x2, nmu), a0, a1);
+                        const float s0 = fast_exp2(a0), s1 = fast_exp2(a1);
+                        const uint32_t w = cvt_bf16x2(s0, s1);
+                        esum = f2_add(esum, f2_make(s0, s1));
+                        rsum = f2_add(rsum, f2_make(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)));
+                        pk[i] = w;
+                    }
+                    tmem_st16(scol + 16 * h2, pk);
+                }
+                if (any_rescale) {
+                    // O must hold the PV of every earlier block of the unit (the one before this block
+                    // may still run: QK of this block was issued before it) and is rescaled before
+                    // this block's P is released to the MMA warp
+                    if (!(ok = __all_sync(full, mbar_wait(&bars[kBarPvDone + x], (sq - 1) & 1)))) break;
                     tc_fence_after();
-                    e0 *= alpha;
-                    e1 *= alpha;
-                    r0 *= alpha;
-                    r1 *= alpha;
 #pragma unroll
                     for (int q4 = 0; q4 < 8; ++q4) {
                         uint32_t o[16];
@@ -624,66 +697,31 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
                         for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
                         tmem_st16(lane_base + col_o + q4 * 16, o);
                     }
-                    tmem_wait_st();
-                }
-                // P = exp2(s * scale_log2 - mu) as bf16 pairs: keys 2c, 2c+1 in column c of the block's S
-                // buffer (columns 0..31; the scores there are already in registers)
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const float s0 = fast_exp2(__uint_as_float(v[32 * h2 + i]) * sl2 - mu);
-                        const float s1 = fast_exp2(__uint_as_float(v[32 * h2 + i + 1]) * sl2 - mu);
-                        const __nv_bfloat162 pb = __floats2bfloat162_rn(s0, s1);
-                        e0 += s0;
-                        e1 += s1;
-                        const float2 pf2 = __bfloat1622float2(pb);
-                        r0 += pf2.x;
-                        r1 += pf2.y;
-                        pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&pb);
-                    }
-                    tmem_st16(scol + 16 * h2, pk);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&bars[kBarPFull + x * 2 + buf]);
+                // the previous unit's output, now that this unit's first P is on its way
+                if (j == 0 && pend) {
+                    if (!(ok = epilogue())) break;
+                    pend = false;
+                }
             }
             if (!ok) break;
-            // ---- epilogue: O_x is complete once every MMA of the tile is
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarODone + x], uo & 1)))) break;
-            ++uo;
-            tc_fence_after();
-            const float inv = 1.f / (r0 + r1);
-            // bf16 row into the unit's finished Q tile, in the 128-byte-swizzled layout of the Q load
-            uint8_t* stage = smem + kOffQ + (k & 1) * kQSlot + x * kQTile + r * 128;
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                uint32_t o[32];
-                tmem_ld32(lane_base + col_o + 32 * c4, o);
-                tmem_wait_ld();
-                if (c4 == 3) {
-                    tc_fence_before();
-                    mbar_arrive(&bars[kBarOEmpty + x]);            // the next unit may overwrite O_x
-                }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint4 w;
-                    w.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
-                    w.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
-                    w.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
-                    w.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
-                    const int chunk = (c4 & 1) * 4 + q;                   // 16-byte chunk within the half
-                    *reinterpret_cast<uint4*>(stage + (c4 >> 1) * kQHalf + ((chunk ^ (r & 7)) << 4)) = w;
-                }
-            }
-            fence_proxy_async_smem();                    // the TMA store reads the tile through the async proxy
-            mbar_arrive(&bars[kBarStaged + x * 2 + (k & 1)]);
-            if (tr < d.nn) {
-                const int h = d.g * kGroup + hh;
-                p.lse[d.l][(static_cast<size_t>(d.b) * p.Hq + h) * p.S + tr] = (m_ref + __log2f(e0 + e1)) * kLn2;
-            }
+            float e0, e1, r0, r1;
+            f2_split(esum, e0, e1);
+            f2_split(rsum, r0, r1);
+            pend = true;
+            e_l = d.l;
+            e_b = d.b;
+            e_g = d.g;
+            e_tr = tr;
+            e_nn = d.nn;
+            e_m = m_ref;
+            e_sum = e0 + e1;
+            e_rsum = r0 + r1;
         }
+        if (ok && pend) ok = epilogue();
         if (!ok && lane == 0) fail();
     } else if (Rope) {
         // ================================================= RoPE on the landed Q tiles
@@ -792,12 +830,14 @@ ark_status launch_prefill(const void* const* q, const void* const* cache_k, cons
             return ARK_ERR_INVALID_ARG;
         if (!q_group_tensor_map(&prm.qmap[i], q[l], static_cast<long long>(B) * S, Hq, 64, pf::kPos) ||
             !kv_tensor_map(&prm.kmap[i], cache_k[l], static_cast<long long>(B) * T, Hkv, 64, pf::kBN) ||
-            !kv_tensor_map(&prm.vmap[i], cache_v[l], static_cast<long long>(B) * T, Hkv, 64, pf::kBN) ||
-            !q_group_tensor_map(&prm.omap[i], o[l], static_cast<long long>(B) * S, Hq, 64, pf::kPos) ||
-            !q_group_tensor_map(&prm.omap1[i], o[l], static_cast<long long>(B) * S, Hq, 64, 1))
+            !kv_tensor_map(&prm.vmap[i], cache_v[l], static_cast<long long>(B) * T, Hkv, 64, pf::kBN))
             return ARK_ERR_CUDA;
+        prm.o[i] = static_cast<__nv_bfloat16*>(o[l]);
         prm.lse[i] = lse[l];
     }
+    prm.o_align32 = 1;
+    for (int i = 0; i < n; ++i)
+        if (reinterpret_cast<uintptr_t>(o[l0 + i]) & 31u) prm.o_align32 = 0;
     prm.pos0 = pos0;
     prm.n_new = n_new;
     prm.status = d_status;
