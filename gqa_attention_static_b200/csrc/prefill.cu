@@ -284,6 +284,20 @@ __device__ __forceinline__ UnitDesc unit_desc(const Params& p, long long i, int 
 
 }  // namespace pf
 
+namespace pf {
+// the unit-list fields an MMA warp computes descriptors from, made warp-uniform (broadcast from
+// lane 0) so that every lane derives the same descriptor values and one elected lane issues
+__device__ __forceinline__ void uniform_desc(UnitDesc& d) {
+    d.l = __shfl_sync(0xffffffffu, d.l, 0);
+    d.t0 = __shfl_sync(0xffffffffu, d.t0, 0);
+    d.nn = __shfl_sync(0xffffffffu, d.nn, 0);
+    d.p0 = __shfl_sync(0xffffffffu, d.p0, 0);
+    d.nblk_a = __shfl_sync(0xffffffffu, d.nblk_a, 0);
+    d.nblk_b = __shfl_sync(0xffffffffu, d.nblk_b, 0);
+    d.end = __shfl_sync(0xffffffffu, d.end, 0);
+}
+}  // namespace pf
+
 template <bool Rope>
 __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
     prefill_kernel(const __grid_constant__ pf::Params p) {
@@ -435,6 +449,7 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
             UnitDesc d;
             if (!(ok = __all_sync(full, wait_desc(k, d)))) break;
             free_desc(k);
+            uniform_desc(d);
             if (d.end) break;
             if (!(ok = __all_sync(full, mbar_wait(&bars[(Rope ? kBarQRot : kBarQFull) + (k & 1)], (k >> 1) & 1))))
                 break;
@@ -455,26 +470,25 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
                 // unmasked)
                 const int n16 = min(kBN, (kv_end - j * kBN + 15) & ~15);
                 const uint32_t idesc = kIdescF16 | (static_cast<uint32_t>(n16 >> 3) << 17);
-                if (lane == 0) {
-                    tc_fence_after();
-                    const uint64_t kb = dk0 + static_cast<uint64_t>((st * kKV) >> 4);
+                // the whole warp computes the (uniform) descriptors; one elected lane issues each instruction
+                tc_fence_after();
+                const uint64_t kb = dk0 + static_cast<uint64_t>((st * kKV) >> 4);
 #pragma unroll
-                    for (int x = 0; x < 2; ++x) {
-                        if (j >= nbx[x]) continue;
-                        const uint32_t dcol = tmem + kColS + x * 128 + (sq[x] & 1) * kBN;
-                        const uint64_t qa = qslot + static_cast<uint64_t>((x * kQTile) >> 4);
+                for (int x = 0; x < 2; ++x) {
+                    if (j >= nbx[x]) continue;
+                    const uint32_t dcol = tmem + kColS + x * 128 + (sq[x] & 1) * kBN;
+                    const uint64_t qa = qslot + static_cast<uint64_t>((x * kQTile) >> 4);
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4);
-                            const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * kKHalf + (kk & 3) * 32) >> 4);
-                            umma_f16(dcol, qa + off, kb + koff, idesc, kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit(&bars[kBarSFull + x * 2 + (sq[x] & 1)]);
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4);
+                        const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * kKHalf + (kk & 3) * 32) >> 4);
+                        if (elect_one()) umma_f16(dcol, qa + off, kb + koff, idesc, kk > 0 ? 1u : 0u);
                     }
-                    umma_commit(&bars[kBarKEmpty + st]);
-                    // the unit's last score MMAs: its Q slot may take another unit once they complete
-                    if (j == nb - 1) umma_commit(&bars[kBarQEmpty + (k & 1)]);
+                    if (elect_one()) umma_commit(&bars[kBarSFull + x * 2 + (sq[x] & 1)]);
                 }
+                if (elect_one()) umma_commit(&bars[kBarKEmpty + st]);
+                // the unit's last score MMAs: its Q slot may take another unit once they complete
+                if (j == nb - 1 && elect_one()) umma_commit(&bars[kBarQEmpty + (k & 1)]);
                 __syncwarp();
                 for (int x = 0; x < 2; ++x)
                     if (j < nbx[x]) ++sq[x];
@@ -499,6 +513,7 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
             UnitDesc d;
             if (!(ok = __all_sync(full, wait_desc(k, d)))) break;
             free_desc(k);
+            uniform_desc(d);
             if (d.end) break;
             const int nbx[2] = {d.nblk_a, d.nblk_b};
             const int nb = max(d.nblk_a, d.nblk_b);
@@ -529,15 +544,15 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
                     if (!(ok = __all_sync(full, mbar_wait(&bars[kBarPFull + x * 2 + (pv[x] & 1)], (pv[x] >> 1) & 1))))
                         break;
                     const bool last = j == nbx[x] - 1;
-                    if (lane == 0) {
-                        tc_fence_after();
-                        const uint32_t pa = tmem + kColS + x * 128 + (pv[x] & 1) * kBN;   // P: 32 columns
-                        const uint64_t vb = dv0 + static_cast<uint64_t>((st * kKV) >> 4);
+                    tc_fence_after();
+                    const uint32_t pa = tmem + kColS + x * 128 + (pv[x] & 1) * kBN;   // P: 32 columns
+                    const uint64_t vb = dv0 + static_cast<uint64_t>((st * kKV) >> 4);
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            if (kk < ksteps)
-                                umma_f16_ts(tmem + kColO + x * 128, pa + kk * 8, vb + static_cast<uint64_t>(kk * 128),
-                                            kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);   // 16 V rows = 2048 bytes
+                    for (int kk = 0; kk < 4; ++kk)
+                        if (kk < ksteps && elect_one())
+                            umma_f16_ts(tmem + kColO + x * 128, pa + kk * 8, vb + static_cast<uint64_t>(kk * 128),
+                                        kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);   // 16 V rows = 2048 bytes
+                    if (elect_one()) {
                         umma_commit(&bars[kBarPvDone + x]);
                         umma_commit(&bars[kBarSFree + x * 2 + (pv[x] & 1)]);
                         if (last) umma_commit(&bars[kBarODone + x]);
@@ -547,7 +562,7 @@ __global__ void __launch_bounds__(Rope ? pf::kThreadsRope : pf::kThreads, 1)
                     if (last) ++uo[x];
                 }
                 if (!ok) break;
-                if (lane == 0) umma_commit(&bars[kBarVEmpty + st]);
+                if (elect_one()) umma_commit(&bars[kBarVEmpty + st]);
                 __syncwarp();
             }
         }
