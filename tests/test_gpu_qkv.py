@@ -113,14 +113,16 @@ def check_fused_against_oracle(x, w, b, pos0, n_new, ck0, cv0, q, ck, cv, rows=N
                                                        np.asarray(pos0, np.int32), np.asarray(n_new, np.int32),
                                                        HQ, HKV, D)
         q_ref = np.stack([qa[i, t] for i, t in live])[:, None]
-        ck_ref = [cka[i] for i, _ in live]
-        cv_ref = [cva[i] for i, _ in live]
+        rk = np.stack([cka[i, int(pos0[i]) + t] for i, t in live])
+        rv = np.stack([cva[i, int(pos0[i]) + t] for i, t in live])
     else:
         ones = np.ones(len(live), np.int32)
         ck_rows = np.stack([bits(ck0)[i] for i, _ in live])
         cv_rows = np.stack([bits(cv0)[i] for i, _ in live])
         q_ref, ck_ref, cv_ref, skipped = oracle.qkv_rope_append(xs, bits(w), bb, ck_rows, cv_rows, p0, ones, HQ,
                                                                 HKV, D)
+        rk = np.stack([ck_ref[r, p0[r]] for r in range(len(live))])
+        rv = np.stack([cv_ref[r, p0[r]] for r in range(len(live))])
     assert skipped == 0
     # error scale of each projection value, then of each rotated value (|c|, |s| <= 1)
     s = abs_dot(xs[:, 0], bits(w), bb) * (2048 * 2.0 ** -24)                # [R, N]
@@ -139,8 +141,6 @@ def check_fused_against_oracle(x, w, b, pos0, n_new, ck0, cv0, q, ck, cv, rows=N
     gk = np.stack([kb[i, int(pos0[i]) + t] for i, t in live])
     gv = np.stack([vb[i, int(pos0[i]) + t] for i, t in live])
     rq = q_ref[:, 0]
-    rk = np.stack([ck_ref[r, p0[r]] for r in range(len(live))])
-    rv = np.stack([cv_ref[r, p0[r]] for r in range(len(live))])
     check_close_bf16(gq, rq, rot(pq + uq), "q")
     check_close_bf16(gk, rk, rot(pk + uk), "cache_k")
     check_close_bf16(gv, rv, pv, "cache_v")
