@@ -58,23 +58,28 @@ DECODE_CONFIGS = ("ragged", "single", "long2048", "long1024")
 DECODE_TRAFFIC = {
     # ncu, one call of the ragged decode workload: decode_kernel (--set full) plus
     # merge_kernel (dram bytes), read + write (see profiles/)
-    "79d6a2dbdddefa6947b568ea05b6e92b19c54f1d75f952faafdef48dae35a988":
-        329.755392e6 + 4.086016e6 + 13.198848e6 + 0,
+    "897eda01dc002b0828394c98dd54fc30527c34eb69bb38b58a6fed55f875d66d":
+        329.750784e6 + 4.175616e6 + 13.199104e6 + 0,
 }
 
 
 # Per-launch DRAM traffic of the prefill kernel (one layer of the coalesced
 # prefill workload) from an ncu --set full capture, keyed the same way.
 PREFILL_TRAFFIC = {
+    # ncu --set full of one 4-layer launch of the workload (RoPE on load), read + write, / 4:
+    # reads 17.92 MB per layer (q rows, K/V rows); most of o is still in L2 when the kernel
+    # ends, so DRAM writes (2.93 MB per layer) stay below the 13.5 MB written (see profiles/)
+    "3ba101752de68b41be5d43962949cc44d37ede4c00e20bccf4cb897a3b498984": (71.671552e6 + 11.726848e6) / 4,
 }
 
 
 # Per-launch DRAM traffic of the projection kernel (one layer) from ncu --set full
 # captures of the two projection workloads, keyed by source hash and workload.
 QKV_TRAFFIC = {
-    # the 3-stage instantiation (many tiles); the 6-stage split-K instantiation used for a decode
-    # step has not been captured since it changed, so that workload reports null
+    # the 3-stage instantiation (many tiles) for the prompt rows; the 6-stage split-K one for a
+    # decode step
     ("cde2e14ac2c31091a231005ee3800a1c5b6ed3f7342cfb4061ca0ee650e6b0ef", "qkv_prefill"): 36.077568e6 + 0.54272e6,
+    ("cde2e14ac2c31091a231005ee3800a1c5b6ed3f7342cfb4061ca0ee650e6b0ef", "qkv_decode"): 10.670336e6 + 0,
 }
 
 
