@@ -63,6 +63,29 @@ def test_step_single_decode_36_layers(oracle_lib, batched):
     compare(step, batch, range(36))
 
 
+def test_step_with_lengths_advanced_on_the_device(oracle_lib):
+    """Lengths kept on the device and advanced there by a kernel on the same
+    stream right before the step (a serving loop that never copies kv_len back
+    to the host): the decode reads kv_len only after the kernels before it on
+    the stream are done, so it attends over the advanced lengths."""
+    batch = W.cfg_ragged_decode(layers=4)
+    dev = "cuda"
+    q = [x.to(dev).clone() for x in batch.q]
+    kn = [x.to(dev) for x in batch.k_new]
+    vn = [x.to(dev) for x in batch.v_new]
+    ck = [x.to(dev).clone() for x in batch.cache_k]
+    cv = [x.to(dev).clone() for x in batch.cache_v]
+    kv_dev = batch.pos0.to(dev).clone()          # the lengths before this step's new row
+    step = DecodeStep(q, kn, vn, ck, cv, batch.pos0.to(dev), batch.n_new.to(dev), kv_dev,
+                      max_splits=BENCH_MAX_SPLITS, batched=True)
+    torch.cuda.synchronize()
+    kv_dev.add_(batch.n_new.to(dev))             # advanced on the device, on the step's stream
+    step.run()
+    torch.cuda.synchronize()
+    assert torch.equal(kv_dev.cpu(), batch.kv_len)
+    compare(step, batch, range(4))
+
+
 @pytest.mark.parametrize("batched", [True, False])
 def test_step_ragged_batch_full_size(oracle_lib, batched):
     """Ragged batch of 32, 36 layers, T = 512: the benchmark's workload at its
