@@ -26,16 +26,17 @@
 //
 // Per block and tile X: S_X = Q_X K^T is 4 MMAs of 128x128x16 into 128 TMEM
 // columns; the tile's softmax warpgroup (one thread per row, all 128 keys of
-// the block) stores P (bf16) over the first 64 columns of S_X, and O_X +=
-// P_X V is 8 MMAs of 128x64x16 with P read from TMEM and V an MN-major
-// operand.  The MMA warp interleaves the tiles (QK_A, QK_B, PV_A, QK_A next,
-// PV_B, QK_B next, ...), so one tile's softmax runs while the tensor cores
-// work for the other.  Because QK_X(j+1) is issued after PV_X(j), a softmax
-// that finds S_X(j+1) ready also knows O_X holds PV_X(j): the lazy rescale of
-// O_X needs no wait of its own.  Keys past len[b] get score -inf (and their V
-// rows are zeroed) in the last block only.  Rows past len[b] are computed on
-// whatever q holds and are not written.  Warps: 0 TMA, 1 MMA (one thread),
-// 2..5 softmax of tile A, 6..9 softmax of tile B.
+// the block, read in two passes of 32 keys: the row max, then the
+// exponentials) stores P (bf16) in 64 TMEM columns of its own, and O_X += P_X
+// V is 8 MMAs of 128x64x16 with P read from TMEM and V an MN-major operand.
+// Two warps issue the MMAs, each from one thread: warp 1 the scores, warp 10
+// the products.  S_X of the next block is computed as soon as the softmax has
+// read the current scores out of tensor memory; before it overwrites P_X (and
+// before a lazy rescale of O_X) the softmax waits for the tile's previous
+// product.  Keys past len[b] get score -inf (and their V rows are zeroed) in
+// the last block only.  Rows past len[b] are computed on whatever q holds and
+// are not written.  Warps: 0 TMA, 1 score MMAs, 2..5 softmax of tile A, 6..9
+// softmax of tile B, 10 P V MMAs.
 #include "common.cuh"
 #include "tma_host.h"
 
@@ -50,7 +51,7 @@ constexpr int kD = 64;                   // head dim
 constexpr int kBN = 128;                 // keys per block
 constexpr int kQBytes = kRows * 128;     // one Q tile: 128 rows x 64 dims bf16 (16 KB)
 constexpr int kKV = kBN * 128;           // a K or V block (16 KB)
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;            // warp 0 TMA, 1 score MMAs, 2..9 softmax, 10 P V MMAs
 constexpr int kWgThreads = 128;          // softmax threads of one tile (one per row)
 constexpr int kQStages = 2;              // units in flight (each 2 tiles)
 constexpr int kStages = 3;               // K and V ring depth
@@ -67,11 +68,13 @@ constexpr int kBarKEmpty = kBarKFull + kStages;
 constexpr int kBarVFull = kBarKEmpty + kStages;
 constexpr int kBarVEmpty = kBarVFull + kStages;
 constexpr int kBarSFull = kBarVEmpty + kStages;    // [tile]: S_X of the next block (one phase per block)
-constexpr int kBarPFull = kBarSFull + 2;           // [tile]: P_X in TMEM (count 128, one phase per block)
-constexpr int kBarODone = kBarPFull + 2;           // [tile]: every MMA of the unit done (one phase per unit)
+constexpr int kBarSRead = kBarSFull + 2;           // [tile]: S_X read out by the softmax (count 128, per block)
+constexpr int kBarPFull = kBarSRead + 2;           // [tile]: P_X in TMEM (count 128, one phase per block)
+constexpr int kBarPvDone = kBarPFull + 2;          // [tile]: PV_X of a block done (one phase per block)
+constexpr int kBarODone = kBarPvDone + 2;          // [tile]: every MMA of the unit done (one phase per unit)
 constexpr int kBarOEmpty = kBarODone + 2;          // [tile]: O_X read out (count 128, one phase per unit)
-constexpr int kBarDrain = kBarOEmpty + 2;          // MMAs in flight when the MMA warp gives up
-constexpr int kNumBars = kBarDrain + 1;
+constexpr int kBarDrain = kBarOEmpty + 2;          // [issuing warp]: MMAs in flight when it gives up
+constexpr int kNumBars = kBarDrain + 2;
 constexpr int kOffClips = kOffBar + kNumBars * 8;
 //   int len[kMaxClips] (clamped), order[kMaxClips] (clips, most key blocks first), cum[kMaxClips + 1]
 constexpr int kOffTmemPtr = kOffClips + (3 * kMaxClips + 1) * 4 + 12;
@@ -79,10 +82,11 @@ constexpr int kOffFlag = kOffTmemPtr + 8;
 constexpr int kSmemBytes = kOffFlag + 16;
 static_assert(kOffBar % 8 == 0 && kOffTmemPtr % 8 == 0, "alignment");
 
-// TMEM columns: S_A 0..127, S_B 128..255 (fp32 scores; P as bf16 pairs over the
-// first 64 columns of its own S), O_A 256..319, O_B 320..383.
+// TMEM columns: S_A 0..127, S_B 128..255 (fp32 scores), O_A 256..319, O_B
+// 320..383, P_A 384..447, P_B 448..511 (bf16 pairs: keys 2c, 2c+1 in column c).
 constexpr uint32_t kColS = 0;
 constexpr uint32_t kColO = 256;
+constexpr uint32_t kColP = 384;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kIdescF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 4) << 24);
@@ -213,7 +217,9 @@ __global__ void __launch_bounds__(enc::kThreads, 1) encoder_attn_kernel(const __
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNumBars; ++i) {
             uint32_t cnt = 1;
-            if ((i >= kBarPFull && i < kBarPFull + 2) || (i >= kBarOEmpty && i < kBarOEmpty + 2)) cnt = kWgThreads;
+            if ((i >= kBarPFull && i < kBarPFull + 2) || (i >= kBarOEmpty && i < kBarOEmpty + 2) ||
+                (i >= kBarSRead && i < kBarSRead + 2))
+                cnt = kWgThreads;
             mbar_init(&bars[i], cnt);
         }
         *failed_flag = 0;
@@ -273,40 +279,11 @@ __global__ void __launch_bounds__(enc::kThreads, 1) encoder_attn_kernel(const __
             }
         }
     } else if (warp == 1) {
-        // ================================================= MMA issuer
+        // ================================================= score MMAs: S_X = Q_X K^T
+        // S_X of the next block is computed as soon as the softmax has read the current one out of
+        // tensor memory (P has columns of its own).  Waits are AND-ed over the warp.
         bool ok = true;
-        int gx[2] = {0, 0};       // blocks issued per tile (S_X / P_X phases)
-        int kx[2] = {0, 0};       // units finished per tile (O_X phases)
-        // S_X = Q_X K^T of block j (the block's K in stage st)
-        auto issue_qk = [&](int x, int qs, int st) {
-            if (lane == 0) {
-                tc_fence_after();
-                const uint32_t qa = sbase + kOffQ + qs * 2 * kQBytes + x * kQBytes;
-                const uint32_t kb = sbase + kOffK + st * kKV;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + kColS + x * kBN, umma_desc_sw128(qa + kk * 32, 16, 1024),
-                             umma_desc_sw128(kb + kk * 32, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
-                umma_commit(&bars[kBarSFull + x]);
-            }
-            __syncwarp();
-        };
-        // O_X += P_X V of block j (the block's V in stage st); the first block overwrites O_X
-        auto issue_pv = [&](int x, int j, int st) -> bool {
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarPFull + x], gx[x] & 1))) return false;
-            if (lane == 0) {
-                tc_fence_after();
-                const uint32_t pa = tmem + kColS + x * kBN;
-                const uint32_t vb = sbase + kOffV + st * kKV;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_f16_ts(tmem + kColO + x * kD, pa + kk * 8, umma_desc_sw128(vb + kk * 16 * 128, kKV, 1024),
-                                kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
-            }
-            __syncwarp();
-            ++gx[x];
-            return true;
-        };
+        int sx[2] = {0, 0};       // score blocks issued per tile
         int r = 0, g = 0;
         for (int k = 0; ok; ++k) {
             const int t = snake_unit(k, c, G);
@@ -315,23 +292,56 @@ __global__ void __launch_bounds__(enc::kThreads, 1) encoder_attn_kernel(const __
             const int qs = k & 1;
             const int ntile = un.live_b ? 2 : 1;
             if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarQFull + qs], (k >> 1) & 1)))) break;
-            // S of block 0 for each tile (S_X is free: the previous unit's PV_X were issued before)
-            {
+            for (int j = 0; j < un.nblk && ok; ++j, ++g) {
                 const int st = g % kStages;
                 if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarKFull + st], (g / kStages) & 1)))) break;
-                for (int x = 0; x < ntile; ++x) issue_qk(x, qs, st);
+                for (int x = 0; x < ntile && ok; ++x) {
+                    if (sx[x] > 0 &&
+                        !(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSRead + x], (sx[x] - 1) & 1))))
+                        break;
+                    if (lane == 0) {
+                        tc_fence_after();
+                        const uint32_t qa = sbase + kOffQ + qs * 2 * kQBytes + x * kQBytes;
+                        const uint32_t kb = sbase + kOffK + st * kKV;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_f16(tmem + kColS + x * kBN, umma_desc_sw128(qa + kk * 32, 16, 1024),
+                                     umma_desc_sw128(kb + kk * 32, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+                        umma_commit(&bars[kBarSFull + x]);
+                    }
+                    __syncwarp();
+                    ++sx[x];
+                }
+                if (!ok) break;
                 if (lane == 0) {
                     umma_commit(&bars[kBarKEmpty + st]);
-                    if (un.nblk == 1) umma_commit(&bars[kBarQEmpty + qs]);
+                    if (j == un.nblk - 1) umma_commit(&bars[kBarQEmpty + qs]);
                 }
                 __syncwarp();
             }
-            // per block j: PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1) -- tile A's next scores are on their
-            // way while tile B's softmax still runs (QK_X(j+1) reuses S_X after PV_X(j) read P_X(j))
+        }
+        if (!ok) {
+            atomicExch(failed_flag, 1);
+            if (lane == 0) {
+                report(p.status, ARK_DEV_TIMEOUT);
+                umma_commit(&bars[kBarDrain]);
+                (void)mbar_wait(&bars[kBarDrain], 0);            // MMAs issued so far have completed
+            }
+            __syncwarp();
+        }
+    } else if (warp == 10) {
+        // ================================================= P V MMAs: O_X += P_X V
+        bool ok = true;
+        int gx[2] = {0, 0};       // P V blocks issued per tile
+        int kx[2] = {0, 0};       // units finished per tile (O_X phases)
+        int r = 0, g = 0;
+        for (int k = 0; ok; ++k) {
+            const int t = snake_unit(k, c, G);
+            Unit un;
+            if (t >= total || !unit_at(t, r, slen, order, cum, B, un)) break;
+            const int ntile = un.live_b ? 2 : 1;
             for (int j = 0; j < un.nblk && ok; ++j, ++g) {
                 const int st = g % kStages;
-                const int st1 = (g + 1) % kStages;
-                const bool more = j + 1 < un.nblk;
                 if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarVFull + st], (g / kStages) & 1)))) break;
                 const int live = un.len - j * kBN;           // frames of the clip in this block
                 if (live < kBN) {
@@ -342,26 +352,30 @@ __global__ void __launch_bounds__(enc::kThreads, 1) encoder_attn_kernel(const __
                     fence_proxy_async_smem();
                 }
                 __syncwarp();
-                if (more && !(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarKFull + st1], ((g + 1) / kStages) & 1))))
-                    break;
+                const bool last = j == un.nblk - 1;
                 for (int x = 0; x < ntile && ok; ++x) {
                     // the first PV of a unit overwrites O_X: the previous unit's epilogue must have read it
                     if (j == 0 && kx[x] > 0 &&
                         !(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarOEmpty + x], (kx[x] - 1) & 1))))
                         break;
-                    if (!(ok = issue_pv(x, j, st))) break;
-                    if (more) issue_qk(x, qs, st1);
+                    if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPFull + x], gx[x] & 1)))) break;
+                    if (lane == 0) {
+                        tc_fence_after();
+                        const uint32_t pa = tmem + kColP + x * 64;
+                        const uint32_t vb = sbase + kOffV + st * kKV;
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            umma_f16_ts(tmem + kColO + x * kD, pa + kk * 8,
+                                        umma_desc_sw128(vb + kk * 16 * 128, kKV, 1024), kIdescPV,
+                                        (j > 0 || kk > 0) ? 1u : 0u);
+                        umma_commit(&bars[kBarPvDone + x]);
+                        if (last) umma_commit(&bars[kBarODone + x]);
+                    }
+                    __syncwarp();
+                    ++gx[x];
                 }
                 if (!ok) break;
-                if (lane == 0) {
-                    umma_commit(&bars[kBarVEmpty + st]);
-                    if (more) {
-                        umma_commit(&bars[kBarKEmpty + st1]);
-                        if (j + 1 == un.nblk - 1) umma_commit(&bars[kBarQEmpty + qs]);
-                    } else {
-                        for (int x = 0; x < ntile; ++x) umma_commit(&bars[kBarODone + x]);
-                    }
-                }
+                if (lane == 0) umma_commit(&bars[kBarVEmpty + st]);
                 __syncwarp();
             }
             for (int x = 0; x < ntile; ++x) ++kx[x];
@@ -370,8 +384,8 @@ __global__ void __launch_bounds__(enc::kThreads, 1) encoder_attn_kernel(const __
             atomicExch(failed_flag, 1);
             if (lane == 0) {
                 report(p.status, ARK_DEV_TIMEOUT);
-                umma_commit(&bars[kBarDrain]);
-                (void)mbar_wait(&bars[kBarDrain], 0);            // MMAs issued so far have completed
+                umma_commit(&bars[kBarDrain + 1]);
+                (void)mbar_wait(&bars[kBarDrain + 1], 0);        // MMAs issued so far have completed
             }
             __syncwarp();
         }
@@ -383,6 +397,7 @@ __global__ void __launch_bounds__(enc::kThreads, 1) encoder_attn_kernel(const __
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
         const uint32_t col_s = kColS + x * kBN;
         const uint32_t col_o = kColO + x * kD;
+        const uint32_t col_p = kColP + x * 64;
         const float sl2 = p.scale_log2;
         bool ok = true;
         int r = 0, gxx = 0, kxx = 0;
@@ -397,50 +412,33 @@ __global__ void __launch_bounds__(enc::kThreads, 1) encoder_attn_kernel(const __
                 ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + x], gxx & 1));
                 if (!ok) break;
                 tc_fence_after();
-                // keys 0..63 stay in registers; keys 64..127 are read twice (for the max 32 columns at a
-                // time, then for the exponentials), so no more than 96 scores are live.  P (keys 0..63 -> columns 0..31,
-                // keys 64..127 -> columns 32..63) only overwrites scores already held in registers.
+                // two passes over the block's scores, 32 at a time: the row max, then the exponentials;
+                // S_X goes back to the score warp once its last chunk has been read again
                 const int nvalid = un.len - j * kBN;      // keys of the block inside the clip
-                uint32_t v[64];
-                tmem_ld32(lane_base + col_s, *reinterpret_cast<uint32_t(*)[32]>(v));
-                tmem_ld32(lane_base + col_s + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-                tmem_wait_ld();
                 // the last block: keys past the clip get score -inf, hence P = 0
-                auto mask32 = [&](uint32_t* w, int key0) {
-                    if (nvalid < key0 + 32) {
+                auto mask32 = [&](uint32_t* w, int k0) {
+                    if (nvalid < k0 + 32) {
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
-                            if (key0 + i >= nvalid) w[i] = 0xff800000u;
+                            if (k0 + i >= nvalid) w[i] = 0xff800000u;
                     }
                 };
-                auto max32 = [&](const uint32_t* w) {
-                    float y[2];
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const uint32_t* z = w + 16 * hh;
-                        float t = max3(__uint_as_float(z[0]), __uint_as_float(z[1]), __uint_as_float(z[2]));
-                        t = max3(t, __uint_as_float(z[3]), __uint_as_float(z[4]));
-                        t = max3(t, __uint_as_float(z[5]), __uint_as_float(z[6]));
-                        t = max3(t, __uint_as_float(z[7]), __uint_as_float(z[8]));
-                        t = max3(t, __uint_as_float(z[9]), __uint_as_float(z[10]));
-                        t = max3(t, __uint_as_float(z[11]), __uint_as_float(z[12]));
-                        t = max3(t, __uint_as_float(z[13]), __uint_as_float(z[14]));
-                        y[hh] = fmaxf(t, __uint_as_float(z[15]));
-                    }
-                    return fmaxf(y[0], y[1]);
-                };
-                mask32(v, 0);
-                mask32(v + 32, 32);
-                float bmax = fmaxf(max32(v), max32(v + 32));
-#pragma unroll
-                for (int c2 = 2; c2 < 4; ++c2) {
+                for (int c4 = 0; c4 < 4; ++c4) {
                     uint32_t w[32];
-                    tmem_ld32(lane_base + col_s + 32 * c2, w);
+                    tmem_ld32(lane_base + col_s + 32 * c4, w);
                     tmem_wait_ld();
-                    mask32(w, 32 * c2);
-                    bmax = fmaxf(bmax, max32(w));
+                    mask32(w, 32 * c4);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        mx[0] = max3(mx[0], __uint_as_float(w[i + 0]), __uint_as_float(w[i + 1]));
+                        mx[1] = max3(mx[1], __uint_as_float(w[i + 2]), __uint_as_float(w[i + 3]));
+                        mx[2] = max3(mx[2], __uint_as_float(w[i + 4]), __uint_as_float(w[i + 5]));
+                        mx[3] = max3(mx[3], __uint_as_float(w[i + 6]), __uint_as_float(w[i + 7]));
+                    }
                 }
-                const float bm = bmax * sl2;
+                const float bm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
                 float alpha = 1.f;
                 bool rescale = false;
                 if (m_ref == -INFINITY) {
@@ -451,23 +449,28 @@ __global__ void __launch_bounds__(enc::kThreads, 1) encoder_attn_kernel(const __
                     rescale = true;
                 }
                 const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-                if (__any_sync(0xffffffffu, rescale)) {
-                    // O_X holds PV_X of every earlier block: PV_X(j-1) was issued before QK_X(j)
+                // P_X is overwritten below and O_X may be rescaled: the previous PV of the tile must be done
+                if (gxx > 0) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarPvDone + x], (gxx - 1) & 1));
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                const bool any_rescale = __any_sync(0xffffffffu, rescale);
+                if (any_rescale) {
                     e0 *= alpha;
                     e1 *= alpha;
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint32_t o[16];
-                        tmem_ld16(lane_base + col_o + q4 * 16, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st16(lane_base + col_o + q4 * 16, o);
-                    }
-                    tmem_wait_st();
                 }
-                // P = 2^(s * scale_log2 - mu) as bf16 pairs; 32 keys -> 16 columns
-                auto exp32 = [&](const uint32_t* w, uint32_t col) {
+                // P = 2^(s * scale_log2 - mu) as bf16 pairs; 32 keys -> 16 columns of P_X
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    uint32_t w[32];
+                    tmem_ld32(lane_base + col_s + 32 * c4, w);
+                    tmem_wait_ld();
+                    if (c4 == 3) {
+                        tc_fence_before();
+                        mbar_arrive(&bars[kBarSRead + x]);     // every score of the block has been read
+                    }
+                    mask32(w, 32 * c4);
                     uint32_t pk[16];
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
@@ -478,20 +481,20 @@ __global__ void __launch_bounds__(enc::kThreads, 1) encoder_attn_kernel(const __
                         add2(e0, e1, s0, s1);
                         pk[i >> 1] = pack_bf16x2(s0, s1);
                     }
-                    tmem_st16(lane_base + col, pk);
-                };
-                exp32(v, col_s);
-                exp32(v + 32, col_s + 16);
-                {
-                    // keys 64..127 again, both chunks behind one wait (keys 0..63 are no longer live)
-                    uint32_t w[64];
-                    tmem_ld32(lane_base + col_s + 64, *reinterpret_cast<uint32_t(*)[32]>(w));
-                    tmem_ld32(lane_base + col_s + 96, *reinterpret_cast<uint32_t(*)[32]>(w + 32));
-                    tmem_wait_ld();
-                    mask32(w, 64);
-                    mask32(w + 32, 96);
-                    exp32(w, col_s + 32);
-                    exp32(w + 32, col_s + 48);
+                    tmem_st16(lane_base + col_p + 16 * c4, pk);
+                }
+                if (any_rescale) {
+                    // O_X holds the PV of every earlier block (waited for above); rescaled before this
+                    // block's P is released to the PV warp, with the scores no longer live
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint32_t o[16];
+                        tmem_ld16(lane_base + col_o + q4 * 16, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st16(lane_base + col_o + q4 * 16, o);
+                    }
                 }
                 tmem_wait_st();
                 tc_fence_before();
