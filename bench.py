@@ -86,7 +86,7 @@ QKV_TRAFFIC = {
 # Per-launch DRAM traffic of the encoder attention kernel (one layer of the encoder batch)
 # from an ncu --set full capture, keyed the same way.
 ENCODER_TRAFFIC = {
-    "c9a95e526155cc2b96648ff6961d41d4db8aa6cb1fc2d46f91b176f748b1f761": 64.04736e6 + 2.65472e6,
+    "80df227913d295a8609e6a3f910c9fec15f5022b9b6a5ccd51b8841d3da00579": 64.049152e6 + 2.81856e6,
 }
 
 
