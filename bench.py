@@ -323,9 +323,12 @@ class OracleRunner:
         batch, self.desc = make_workload(workload, layers, "cpu")
         self.fp8 = (kv == "fp8")
         if self.fp8:
+            from gqa_attention_static_b200 import workloads as W
             fc = fp8_cache_for(batch, mode)
+            # the oracle takes caches in [B,T,Hkv,D] order; the library's fp8 cache is head-major
             self.inputs = [(_bits(batch.q[l]), _bits(batch.k_new[l]), _bits(batch.v_new[l]),
-                            fc.cache_k[l].numpy(), fc.cache_v[l].numpy(), fc.k_scale[l].numpy(),
+                            W.to_btkd(fc.cache_k[l]).contiguous().numpy(),
+                            W.to_btkd(fc.cache_v[l]).contiguous().numpy(), fc.k_scale[l].numpy(),
                             fc.v_scale[l].numpy()) for l in range(layers)]
             self.desc = self.desc.replace(" 1% x8 K/V row outliers", "") + ", fp8 E4M3 cache"
         else:

@@ -14,8 +14,9 @@
 // is therefore bit-reproducible.
 //
 // fp8 cache variant (ark_attn_append_rope_fp8): the caches hold OCP E4M3
-// codes with one fp32 scale per (layer, KV head) for K and one for V (a cache
-// format the pages do not have; they quantise weights only).  The rotated key
+// codes with one fp32 scale per (layer, KV head) for K and one for V, stored
+// head-major (a cache format the pages do not have; they quantise weights
+// only).  The rotated key
 // is divided by its scale in double (not rounded to bf16 first), rounded to
 // fp32 and converted to e4m3 with cvt.rn.satfinite; values likewise.  q is
 // rotated to bf16 exactly as above.
@@ -51,6 +52,13 @@ struct AppendParams {
     int rows_per_cta;     // consecutive rows t of one (request, layer) per CTA
     AppendLayer layer[ARK_MAX_LAYERS];
 };
+
+// Byte offset of (request b, KV head g, position pos) in an fp8 cache, which
+// is head-major [B][Hkv][T][128]: one head's positions are consecutive
+// 128-byte rows, so a tile of positions is one contiguous block.
+__device__ __forceinline__ size_t fp8_row_offset(int b, int g, int pos, int T, int Hkv) {
+    return ((static_cast<size_t>(b) * Hkv + g) * T + pos) * kHeadDim;
+}
 
 template <bool Fp8>
 __global__ void __launch_bounds__(512) append_rope_kernel(const __grid_constant__ AppendParams p) {
@@ -99,12 +107,11 @@ __global__ void __launch_bounds__(512) append_rope_kernel(const __grid_constant_
                 } else {
                     const int g = head - qh;
                     src = L.k_new + ((static_cast<size_t>(b) * p.S + t) * p.Hkv + g) * kHeadDim;
-                    const size_t off = ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + g) * kHeadDim;
                     if (Fp8) {
-                        dst8 = static_cast<uint8_t*>(L.cache_k) + off;
+                        dst8 = static_cast<uint8_t*>(L.cache_k) + fp8_row_offset(b, g, pos, p.T, p.Hkv);
                         kscale = static_cast<double>(__ldg(L.k_scale + g));
                     } else {
-                        dst = static_cast<uint16_t*>(L.cache_k) + off;
+                        dst = static_cast<uint16_t*>(L.cache_k) + ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + g) * kHeadDim;
                     }
                 }
                 const uint2 lo = *reinterpret_cast<const uint2*>(src + 4 * pg);
@@ -167,7 +174,6 @@ __global__ void __launch_bounds__(512) append_rope_kernel(const __grid_constant_
                 const int piece = c & 15;
                 const uint4* src = reinterpret_cast<const uint4*>(
                     L.v_new + ((static_cast<size_t>(b) * p.S + t) * p.Hkv + g) * kHeadDim);
-                const size_t off = ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + g) * kHeadDim;
                 if (Fp8) {
                     // 8 values -> 8 codes: e4m3(fp32(v / scale))
                     const double vscale = static_cast<double>(__ldg(L.v_scale + g));
@@ -180,9 +186,11 @@ __global__ void __launch_bounds__(512) append_rope_kernel(const __grid_constant_
                         const float f1 = __double2float_rn(bf16_bits_to_f64(static_cast<uint16_t>(w[i] >> 16)) / vscale);
                         out[i >> 1] |= static_cast<uint32_t>(f32x2_to_e4m3x2(f0, f1)) << (16 * (i & 1));
                     }
-                    *reinterpret_cast<uint2*>(static_cast<uint8_t*>(L.cache_v) + off + 8 * piece) = make_uint2(out[0], out[1]);
+                    *reinterpret_cast<uint2*>(static_cast<uint8_t*>(L.cache_v) + fp8_row_offset(b, g, pos, p.T, p.Hkv) +
+                                              8 * piece) = make_uint2(out[0], out[1]);
                 } else {
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(L.cache_v) + off);
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(L.cache_v) +
+                                                          ((static_cast<size_t>(b) * p.T + pos) * p.Hkv + g) * kHeadDim);
                     dst[piece] = src[piece];
                 }
             }

@@ -88,11 +88,12 @@ bool kv_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv, 
     return cached_encode(key, out, 3, dims, strides, box);
 }
 
-bool kv8_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv, int box_rows) {
-    const Key key{reinterpret_cast<uintptr_t>(base), rows, 3, Hkv, 128, box_rows};
-    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(rows)};
-    const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(Hkv) * 128};
-    const cuuint32_t box[3] = {128, 1, static_cast<cuuint32_t>(box_rows)};
+bool kv8_tensor_map(CUtensorMap* out, const void* base, int B, int T, int Hkv, int box_rows) {
+    // the key's `inner` slot holds T here: the map depends on how B*T splits into B and T
+    const Key key{reinterpret_cast<uintptr_t>(base), static_cast<long long>(B) * T, 3, Hkv, T, box_rows};
+    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B) * Hkv};
+    const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(T) * 128};
+    const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), 1};
     return cached_encode(key, out, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8);
 }
 

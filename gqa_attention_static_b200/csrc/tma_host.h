@@ -15,9 +15,11 @@ bool kv_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv, 
 
 // 2-D tiled map over a row-major [rows, 128] bf16 matrix (row pitch 256 B),
 // box (box_inner elements, box_rows rows), 128-byte swizzle.
-// fp8 (one byte per element) cache [B*T rows][Hkv][128], 128-byte rows:
-// dims (128, Hkv, rows), box (128, 1, box_rows), 128-byte swizzle.
-bool kv8_tensor_map(CUtensorMap* out, const void* base, long long rows, int Hkv, int box_rows);
+// fp8 (one byte per element) cache, head-major [B][Hkv][T][128], 128-byte
+// rows: dims (128, T, B*Hkv), box (128, box_rows, 1), 128-byte swizzle; a box
+// is box_rows consecutive positions of one (request, KV head), contiguous in
+// memory; positions past T read as zero.
+bool kv8_tensor_map(CUtensorMap* out, const void* base, int B, int T, int Hkv, int box_rows);
 
 // [rows][H][64] bf16 (heads of 64 dims): dims (64, H, rows), box (64, 1, box_rows),
 // 128-byte swizzle.

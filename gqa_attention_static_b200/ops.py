@@ -416,8 +416,9 @@ def ark_attn_decode_noalloc(q, cache_k, cache_v, kv_len, o, lse, scale: float, m
 
 
 # --------------------------------------------------------- fp8 KV cache ----
-# Caches of e4m3 codes (torch.uint8, [B,T,Hkv,D]) with fp32 scales per KV head
-# (torch.float32 [Hkv] per layer); see the header for the format.
+# Caches of e4m3 codes (torch.uint8, head-major [B,Hkv,T,D], unlike the bf16
+# cache) with fp32 scales per KV head (torch.float32 [Hkv] per layer); see the
+# header for the format.
 
 def _fp8_cache_checks(cache_k, cache_v, k_scale, v_scale, Hkv_expected=None):
     _need(cache_k, "cache_k", torch.uint8, 4)
@@ -426,7 +427,7 @@ def _fp8_cache_checks(cache_k, cache_v, k_scale, v_scale, Hkv_expected=None):
     _need(v_scale, "v_scale", torch.float32, 1)
     if cache_v.shape != cache_k.shape:
         raise ValueError("cache_k and cache_v must have the same shape")
-    Hkv = cache_k.shape[2]
+    Hkv = cache_k.shape[1]
     if k_scale.numel() != Hkv or v_scale.numel() != Hkv:
         raise ValueError("one K scale and one V scale per KV head")
 
@@ -451,7 +452,7 @@ def ark_attn_append_rope_fp8_layers(q: Sequence[torch.Tensor], k_new, v_new, cac
     if status is not None:
         _need(status, "status", torch.int32)
     B, S, Hq, D = q[0].shape
-    T, Hkv = cache_k[0].shape[1], cache_k[0].shape[2]
+    Hkv, T = cache_k[0].shape[1], cache_k[0].shape[2]
     if tuple(k_new[0].shape) != (B, S, Hkv, D) or cache_k[0].shape[0] != B or cache_k[0].shape[3] != D:
         raise ValueError("shapes")
     if table.numel() < T * (D // 2) * 2:
@@ -475,7 +476,7 @@ def ark_attn_append_rope_fp8(q, k_new, v_new, cache_k, cache_v, k_scale, v_scale
     if status is not None:
         _need(status, "status", torch.int32)
     B, S, Hq, D = q.shape
-    T, Hkv = cache_k.shape[1], cache_k.shape[2]
+    Hkv, T = cache_k.shape[1], cache_k.shape[2]
     if tuple(k_new.shape) != (B, S, Hkv, D) or tuple(v_new.shape) != (B, S, Hkv, D) or cache_k.shape[0] != B:
         raise ValueError("shapes")
     if table.numel() < T * (D // 2) * 2:
@@ -498,7 +499,7 @@ def ark_attn_decode_fp8(q, cache_k, cache_v, k_scale, v_scale, kv_len, o, lse, s
     B, S, Hq, D = q.shape
     if S != 1:
         raise ValueError("decode takes one query row per request")
-    T, Hkv = cache_k.shape[1], cache_k.shape[2]
+    Hkv, T = cache_k.shape[1], cache_k.shape[2]
     ws_bytes = 0
     if workspace is not None:
         _need(workspace, "workspace", workspace.dtype)
@@ -532,7 +533,7 @@ def ark_attn_decode_fp8_layers(q: Sequence[torch.Tensor], cache_k, cache_v, k_sc
     B, S, Hq, D = q[0].shape
     if S != 1:
         raise ValueError("decode takes one query row per request")
-    T, Hkv = cache_k[0].shape[1], cache_k[0].shape[2]
+    Hkv, T = cache_k[0].shape[1], cache_k[0].shape[2]
     ws_bytes = 0
     if workspace is not None:
         _need(workspace, "workspace", workspace.dtype)

@@ -31,7 +31,7 @@ class DecodeStep:
     (table, workspace, status and the o/lse lists are allocated here unless
     passed in).
     With k_scale/v_scale (per layer fp32 [Hkv]) the caches are fp8 (uint8 e4m3
-    codes) and the step uses the fp8 entry points.
+    codes, head-major [B,Hkv,T,D]) and the step uses the fp8 entry points.
     """
 
     def __init__(self, q: List[torch.Tensor], k_new: List[torch.Tensor], v_new: List[torch.Tensor],
@@ -52,8 +52,9 @@ class DecodeStep:
         self.pos0, self.n_new, self.kv_len = pos0, n_new, kv_len
         self.layers = len(q)
         self.B, _, self.Hq, self.D = q[0].shape
-        self.T = cache_k[0].shape[1]
-        self.Hkv = cache_k[0].shape[2]
+        # the fp8 cache is head-major [B,Hkv,T,D], the bf16 cache [B,T,Hkv,D]
+        self.Hkv, self.T = (cache_k[0].shape[1], cache_k[0].shape[2]) if self.fp8 else \
+            (cache_k[0].shape[2], cache_k[0].shape[1])
         dev = q[0].device
         self.max_splits = max_splits
         self.mode = mode

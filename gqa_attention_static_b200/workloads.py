@@ -260,10 +260,23 @@ def e4m3_codes(shape, gen: torch.Generator, exp_lo: int = 3, exp_hi: int = 10) -
     return (sign | expo | mant).to(torch.uint8)
 
 
+def to_btkd(x):
+    """A head-major [B,Hkv,T,D] fp8 cache as [B,T,Hkv,D] (a permuted view;
+    works for torch tensors and numpy arrays)."""
+    return x.permute(0, 2, 1, 3) if hasattr(x, "permute") else x.transpose(0, 2, 1, 3)
+
+
+def to_bhtd(x):
+    """The inverse of to_btkd: [B,T,Hkv,D] as head-major [B,Hkv,T,D]."""
+    return to_btkd(x)
+
+
 def make_fp8_cache(seed: int, B: int, T: int, valid, layers: int = 1, garbage: str = "nan",
                    Hkv: int = HKV, D: int = HEAD_DIM) -> Fp8Cache:
-    """fp8 caches whose rows j < valid[b] hold codes of moderate magnitude and
-    whose later rows hold `garbage`: "nan" (NaN codes 0x7F/0xFF mixed with the
+    """fp8 caches (head-major [B,Hkv,T,D] uint8, the library's fp8 layout;
+    `to_btkd` gives the [B,T,Hkv,D] view) whose rows j < valid[b] hold codes
+    of moderate magnitude and whose later rows hold `garbage`: "nan" (NaN
+    codes 0x7F/0xFF mixed with the
     largest finite codes), "big" (finite codes of magnitude 256..448) or
     "none" (the same distribution as the valid rows).  Scales: uniform in
     [0.02, 0.2], one per KV head for K and for V."""
@@ -282,7 +295,9 @@ def make_fp8_cache(seed: int, B: int, T: int, valid, layers: int = 1, garbage: s
                 x = torch.where(past, bad.to(torch.uint8), x)
             elif garbage == "big":
                 x = torch.where(past, e4m3_codes((B, T, Hkv, D), g, 14, 14), x)
-            lst.append(x.contiguous())
+            # the library's fp8 cache is head-major [B,Hkv,T,D]; the draws above run in
+            # [B,T,Hkv,D] order so that the values stay those of the same seed
+            lst.append(x.permute(0, 2, 1, 3).contiguous())
         out.k_scale.append((0.02 + 0.18 * torch.rand(Hkv, generator=g)).float())
         out.v_scale.append((0.02 + 0.18 * torch.rand(Hkv, generator=g)).float())
     return out

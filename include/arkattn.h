@@ -312,9 +312,10 @@ ARK_API ark_status ark_attn_prefill_rope_layers(int L, const void* const* q, con
  *     round-to-nearest-even, finite values beyond +-448 and infinities
  *     saturating to +-448, NaN kept.  q is rotated to bf16 in place as by
  *     ark_attn_append_rope.  Bit-reproducible.
- * Layouts: cache_k, cache_v [B,T,Hkv,D] of uint8 codes (16-byte aligned);
- * everything else, the arguments, the status bits and the errors as for the
- * bf16 entry points.  The decode computes Q K^T and P V on f16 tensor-core
+ * Layouts: cache_k, cache_v head-major [B,Hkv,T,D] of uint8 codes (16-byte
+ * aligned; unlike the bf16 cache's [B,T,Hkv,D], so that the positions of one
+ * KV head are consecutive 128-byte rows); everything else, the arguments, the
+ * status bits and the errors as for the bf16 entry points.  The decode computes Q K^T and P V on f16 tensor-core
  * operands (every e4m3 value is an f16 value; q is converted from bf16 to
  * f16, exact for |q| in [2^-14, 65504]; the softmax weights are rounded to
  * f16) with fp32 accumulation, and uses the workspace of ark_attn_decode.

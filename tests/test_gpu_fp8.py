@@ -24,7 +24,9 @@ SCALE = 1.0 / math.sqrt(128)
 
 
 def u8(x: torch.Tensor) -> np.ndarray:
-    return x.detach().cpu().contiguous().numpy()
+    """An fp8 cache (the library's head-major [B,Hkv,T,D]) as a uint8 array in
+    the oracle's [B,T,Hkv,D] order."""
+    return W.to_btkd(x.detach().cpu()).contiguous().numpy()
 
 
 def test_append_fp8_bit_exact(oracle_lib):
@@ -79,7 +81,7 @@ def test_append_fp8_saturates_and_single_layer_entry(oracle_lib):
 def gpu_decode_fp8(q, fc, kv, mode=ops.ARK_LENGTH_AWARE, max_splits=8, layer=0):
     dev = "cuda"
     B, _, Hq, D = q.shape
-    T = fc.cache_k[layer].shape[1]
+    T = fc.cache_k[layer].shape[2]
     o = torch.full((B, 1, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
     lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=dev)
     ws = ops.decode_workspace(B, Hq, D, T, max_splits, device=dev)
