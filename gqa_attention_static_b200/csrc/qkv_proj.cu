@@ -74,6 +74,42 @@ constexpr uint32_t kTmemCols = 128;
 // kind::f16, bf16 x bf16 -> fp32, M = 128, N = 128, A and B K-major
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
+// The narrow form, for a few token rows (a decode step): the operands swap roles, so that the
+// 128 output features of a head are the MMA's M and the token rows its N (nt = 16 .. 64).  A
+// stage is then a 16 KB weight tile and a small x tile (room for XR rows), and the ring holds a
+// cluster rank's whole share of K (hidden 2048 split 8 ways: 4 stages, two CTAs per SM): every
+// weight copy is issued before the wait for the previous kernel, only the x copies after it,
+// and the next layer's CTAs are resident beside this one's.  The split's partial tiles meet
+// in `recv`: rank r owns token rows [r nt / split, (r+1) nt / split), and every rank pushes
+// those rows of its fp32 tile into rank r's recv[rank] with st.async, which completes bytes on
+// r's mbarrier -- no cluster-wide barrier sits between the MMAs and the epilogue.
+constexpr int kNarrowMaxM = 64;
+template <int NS, int XR>
+struct NarrowLayout {
+    static constexpr int kNStages = NS;
+    static constexpr int kStage = kTileB + XR * 128;           // W tile + x tile of up to XR rows
+    static constexpr int kOffRecv = NS * kStage;               // [split][128 features][nt / split] fp32
+    static constexpr int kRecvBytes = XR * kBN * 4;
+    static constexpr int kOffBar = kOffRecv + kRecvBytes;
+    static constexpr int kBarFull = 0;                          // [NS]
+    static constexpr int kBarEmpty = kBarFull + NS;             // [NS]
+    static constexpr int kBarDone = kBarEmpty + NS;
+    static constexpr int kBarRecv = kBarDone + 1;
+    static constexpr int kNumBars = kBarRecv + 1;
+    static constexpr int kOffRows = kOffBar + kNumBars * 8;     // per token row of this rank: int2
+    static constexpr int kOffBias = kOffRows + XR * 8;
+    static constexpr int kOffTmemPtr = kOffBias + kBN * 4;
+    static constexpr int kOffFlag = kOffTmemPtr + 8;
+    static constexpr int kSmemBytes = kOffFlag + 8;
+    static_assert(kStage % 1024 == 0 && kTileB % 1024 == 0, "128-byte swizzled tiles start on 1 KB");
+    static_assert(XR <= kNarrowMaxM && XR % 16 == 0, "x tile rows");
+};
+constexpr uint32_t kNarrowTmemCols = 64;
+// kind::f16, bf16 x bf16 -> fp32, M = 128, N = n, A and B K-major
+__host__ __device__ constexpr uint32_t idesc_m128(uint32_t n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
+}
+
 struct Params {
     CUtensorMap xmap;          // x [M][K] as (K, M), box (64, 128)
     CUtensorMap wmap;          // W [N][K] as (K, N), box (64, 128)
@@ -89,6 +125,7 @@ struct Params {
     const float2* table;       // [T][64] {cos, sin}
     uint32_t* status;
     int B, S, T, Hq, Hkv;
+    int nt;                    // narrow form only: token rows per tile (MMA N), 16 .. 64
 };
 
 // Every thread of every CTA of the cluster, at the same program point.
@@ -105,6 +142,143 @@ __device__ __forceinline__ float4 ld_dsmem_f4(const void* local, uint32_t rank) 
     asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
                  : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(raddr) : "memory");
     return v;
+}
+
+// 4 fp32 values (or one) into another CTA's shared memory at `raddr` (a shared::cluster
+// address), completing their bytes on that CTA's mbarrier at `rbar`.
+__device__ __forceinline__ void st_async_v4(uint32_t raddr, float a, float b, float c, float d, uint32_t rbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+                 :: "r"(raddr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(rbar) : "memory");
+}
+__device__ __forceinline__ void st_async_f32(uint32_t raddr, float a, uint32_t rbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+                 :: "r"(raddr), "r"(__float_as_uint(a)), "r"(rbar) : "memory");
+}
+__device__ __forceinline__ uint32_t map_rank(uint32_t local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+// The narrow form's receive wait.  Every sender sends after at most one bounded wait of its
+// own (kWaitLimitNs, in its epilogue), so a limit four times as long (on the global timer only)
+// keeps a receiver from leaving while another rank may still write into its shared memory.
+__device__ __forceinline__ bool mbar_wait_recv(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 0;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63) == 63 && globaltimer_ns() - t0 > 4 * kWaitLimitNs) return false;
+    }
+}
+
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    __syncwarp();
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    __syncwarp();
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// The plain projection of 8 output features of one token row: p = bf16(acc + bias), the sum in
+// double and rounded once, stored as one 16-byte write at `dst`.
+__device__ __forceinline__ void emit_plain8(uint16_t* dst, const float* sbias, int c8, float4 a0, float4 a1) {
+    const float v[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const double b0 = static_cast<double>(sbias[c8 + 2 * i]);
+        const double b1 = static_cast<double>(sbias[c8 + 2 * i + 1]);
+        w[i] = static_cast<uint32_t>(f64_to_bf16_rn(static_cast<double>(v[2 * i]) + b0)) |
+               (static_cast<uint32_t>(f64_to_bf16_rn(static_cast<double>(v[2 * i + 1]) + b1)) << 16);
+    }
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// The fused form for one token row and rotary pairs 4g .. 4g+3 of one head: the projection
+// value is the accumulator (lo: features 4g.., hi: features 64+4g..) plus the bias rounded once
+// to bf16; q and k heads are then rotated exactly as by the append kernel (products exact in
+// double, one rounding), v heads stored as they are.  info = {destination in 8-byte units, pos}.
+// cs01, cs23: {cos, sin} of pairs 4g, 4g+1 and 4g+2, 4g+3 at the row's position (rope_pairs).
+__device__ __forceinline__ void emit_rope_group(const Params& p, int head, int g, int2 info, const float* sbias,
+                                                float4 lo, float4 hi, float4 cs01, float4 cs23) {
+    uint16_t* base = head < p.Hq ? p.q : (head < p.Hq + p.Hkv ? p.cache_k : p.cache_v);
+    uint16_t* dst = base + (static_cast<size_t>(info.x) << 2);
+    const bool rotate = head < p.Hq + p.Hkv;
+    const float al[4] = {lo.x, lo.y, lo.z, lo.w};
+    const float ah[4] = {hi.x, hi.y, hi.z, hi.w};
+    const float cc[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
+    const float ss[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
+    uint16_t yl[4], yh[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const double bl = static_cast<double>(sbias[4 * g + i]);
+        const double bh = static_cast<double>(sbias[64 + 4 * g + i]);
+        // the projection output (the Linear's bf16 value)
+        const uint16_t xl = f64_to_bf16_rn(static_cast<double>(al[i]) + bl);
+        const uint16_t xh = f64_to_bf16_rn(static_cast<double>(ah[i]) + bh);
+        if (rotate) {
+            const double a = bf16_bits_to_f64(xl);
+            const double h = bf16_bits_to_f64(xh);
+            const double c = static_cast<double>(cc[i]);
+            const double sn = static_cast<double>(ss[i]);
+            // both products are exact in double, so contraction cannot change the result
+            yl[i] = f64_to_bf16_rn(a * c - h * sn);
+            yh[i] = f64_to_bf16_rn(h * c + a * sn);
+        } else {
+            yl[i] = xl;
+            yh[i] = xh;
+        }
+    }
+    *reinterpret_cast<uint2*>(dst + 4 * g) =
+        make_uint2(static_cast<uint32_t>(yl[0]) | (static_cast<uint32_t>(yl[1]) << 16),
+                   static_cast<uint32_t>(yl[2]) | (static_cast<uint32_t>(yl[3]) << 16));
+    *reinterpret_cast<uint2*>(dst + 64 + 4 * g) =
+        make_uint2(static_cast<uint32_t>(yh[0]) | (static_cast<uint32_t>(yh[1]) << 16),
+                   static_cast<uint32_t>(yh[2]) | (static_cast<uint32_t>(yh[3]) << 16));
+}
+
+// The rotary table entries of pairs 4g .. 4g+3 at position pos (zeros when the head is not
+// rotated or pos is outside the table: such rows are not written).
+__device__ __forceinline__ void rope_pairs(const Params& p, int head, int g, int pos, float4& cs01, float4& cs23) {
+    if (head < p.Hq + p.Hkv && pos >= 0 && pos < p.T) {
+        const float4* trow = reinterpret_cast<const float4*>(p.table + static_cast<size_t>(pos) * 64);
+        cs01 = __ldg(trow + 2 * g);
+        cs23 = __ldg(trow + 2 * g + 1);
+    } else {
+        cs01 = cs23 = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+// Where token row m of a tile goes: {destination in 8-byte units or -1, position}; reports bad
+// n_new / positions, and pulls the row's rotary table toward L2.
+__device__ __forceinline__ int2 row_destination(const Params& p, int m, int head) {
+    long long off = -1;
+    int pos = 0;
+    const int b = m / p.S, t = m - b * p.S;
+    int nn = __ldg(p.n_new + b);
+    if (nn < 0 || nn > p.S) {
+        if (t == 0 && head == 0) report(p.status, ARK_DEV_BAD_KVLEN);
+        nn = nn < 0 ? 0 : p.S;
+    }
+    pos = __ldg(p.pos0 + b) + t;
+    if (t < nn) {
+        if (pos < 0 || pos >= p.T) {
+            if (head == 0) report(p.status, ARK_DEV_BAD_POS);
+        } else if (head < p.Hq) {
+            off = (static_cast<long long>(m) * p.Hq + head) * kHeadDim;
+        } else if (head < p.Hq + p.Hkv) {
+            off = ((static_cast<long long>(b) * p.T + pos) * p.Hkv + (head - p.Hq)) * kHeadDim;
+        } else {
+            off = ((static_cast<long long>(b) * p.T + pos) * p.Hkv + (head - p.Hq - p.Hkv)) * kHeadDim;
+        }
+        if (off >= 0 && head < p.Hq + p.Hkv) {
+            const char* tr = reinterpret_cast<const char*>(p.table + static_cast<size_t>(pos) * 64);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) asm volatile("prefetch.global.L2 [%0];" :: "l"(tr + 128 * i));
+        }
+    }
+    // offsets are multiples of 128 elements; stored in 8-byte units they fit an int
+    return make_int2(off < 0 ? -1 : static_cast<int>(off >> 2), pos);
 }
 
 }  // namespace qp
@@ -239,36 +413,7 @@ __global__ void __launch_bounds__(qp::kThreads, S <= 3 ? 2 : 1) qkv_proj_kernel(
         {
             const int et = threadIdx.x - 64;
             sbias[et] = p.bias ? static_cast<float>(bf16_bits_to_f64(p.bias[head * kBN + et])) : 0.f;
-            long long off = -1;
-            int pos = 0;
-            if (p.fused && et < rows && rank == 0) {
-                const int m = m0 + et;
-                const int b = m / p.S, t = m - b * p.S;
-                int nn = __ldg(p.n_new + b);
-                if (nn < 0 || nn > p.S) {
-                    if (t == 0 && head == 0) report(p.status, ARK_DEV_BAD_KVLEN);
-                    nn = nn < 0 ? 0 : p.S;
-                }
-                pos = __ldg(p.pos0 + b) + t;
-                if (t < nn) {
-                    if (pos < 0 || pos >= p.T) {
-                        if (head == 0) report(p.status, ARK_DEV_BAD_POS);
-                    } else if (head < p.Hq) {
-                        off = (static_cast<long long>(m) * p.Hq + head) * kHeadDim;
-                    } else if (head < p.Hq + p.Hkv) {
-                        off = ((static_cast<long long>(b) * p.T + pos) * p.Hkv + (head - p.Hq)) * kHeadDim;
-                    } else {
-                        off = ((static_cast<long long>(b) * p.T + pos) * p.Hkv + (head - p.Hq - p.Hkv)) * kHeadDim;
-                    }
-                    if (off >= 0 && head < p.Hq + p.Hkv) {
-                        const char* tr = reinterpret_cast<const char*>(p.table + static_cast<size_t>(pos) * 64);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) asm volatile("prefetch.global.L2 [%0];" :: "l"(tr + 128 * i));
-                    }
-                }
-            }
-            // offsets are multiples of 128 elements; stored in 8-byte units they fit an int
-            rowinfo[et] = make_int2(off < 0 ? -1 : static_cast<int>(off >> 2), pos);
+            rowinfo[et] = (p.fused && et < rows && rank == 0) ? row_destination(p, m0 + et, head) : make_int2(-1, 0);
         }
         const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarDone], 0));
         tc_fence_after();
@@ -330,64 +475,20 @@ __global__ void __launch_bounds__(qp::kThreads, S <= 3 ? 2 : 1) qkv_proj_kernel(
             for (int it = et; it < rows * (kBN / 8); it += 128) {
                 const int row = it / (kBN / 8), c8 = (it % (kBN / 8)) * 8;
                 const float* src = part + row * kPartStride + c8;
-                uint32_t w[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const double b0 = static_cast<double>(sbias[c8 + 2 * i]);
-                    const double b1 = static_cast<double>(sbias[c8 + 2 * i + 1]);
-                    w[i] = static_cast<uint32_t>(f64_to_bf16_rn(static_cast<double>(src[2 * i]) + b0)) |
-                           (static_cast<uint32_t>(f64_to_bf16_rn(static_cast<double>(src[2 * i + 1]) + b1)) << 16);
-                }
-                *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(m0 + row) * p.N + head * kBN + c8) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
+                emit_plain8(p.out + static_cast<size_t>(m0 + row) * p.N + head * kBN + c8, sbias, c8,
+                            *reinterpret_cast<const float4*>(src), *reinterpret_cast<const float4*>(src + 4));
             }
         } else if (rank == 0 && !failed) {
-            // items (row, group g of rotary pairs 4g .. 4g+3): the projection value is the
-            // accumulator plus the bias rounded once to bf16, then the append kernel's rotation
+            // items (row, group g of rotary pairs 4g .. 4g+3)
             for (int it = et; it < rows * 16; it += 128) {
                 const int row = it >> 4, g = it & 15;
                 const int2 info = rowinfo[row];
                 if (info.x < 0) continue;                         // padded or out-of-range row: not written
-                const int pos = info.y;
-                uint16_t* base = head < p.Hq ? p.q : (head < p.Hq + p.Hkv ? p.cache_k : p.cache_v);
-                uint16_t* dst = base + (static_cast<size_t>(info.x) << 2);
-                const bool rotate = head < p.Hq + p.Hkv;
-                const float4 lo = *reinterpret_cast<const float4*>(part + row * kPartStride + 4 * g);
-                const float4 hi = *reinterpret_cast<const float4*>(part + row * kPartStride + 64 + 4 * g);
-                const float al[4] = {lo.x, lo.y, lo.z, lo.w};
-                const float ah[4] = {hi.x, hi.y, hi.z, hi.w};
-                const float4* trow = reinterpret_cast<const float4*>(p.table + static_cast<size_t>(pos) * 64);
-                const float4 cs01 = __ldg(trow + 2 * g);          // c0 s0 c1 s1 of pairs 4g, 4g+1
-                const float4 cs23 = __ldg(trow + 2 * g + 1);      // c2 s2 c3 s3
-                const float cc[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
-                const float ss[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
-                uint16_t yl[4], yh[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const double bl = static_cast<double>(sbias[4 * g + i]);
-                    const double bh = static_cast<double>(sbias[64 + 4 * g + i]);
-                    // the projection output (the Linear's bf16 value)
-                    const uint16_t xl = f64_to_bf16_rn(static_cast<double>(al[i]) + bl);
-                    const uint16_t xh = f64_to_bf16_rn(static_cast<double>(ah[i]) + bh);
-                    if (rotate) {
-                        const double a = bf16_bits_to_f64(xl);
-                        const double h = bf16_bits_to_f64(xh);
-                        const double c = static_cast<double>(cc[i]);
-                        const double sn = static_cast<double>(ss[i]);
-                        // both products are exact in double, so contraction cannot change the result
-                        yl[i] = f64_to_bf16_rn(a * c - h * sn);
-                        yh[i] = f64_to_bf16_rn(h * c + a * sn);
-                    } else {
-                        yl[i] = xl;
-                        yh[i] = xh;
-                    }
-                }
-                *reinterpret_cast<uint2*>(dst + 4 * g) =
-                    make_uint2(static_cast<uint32_t>(yl[0]) | (static_cast<uint32_t>(yl[1]) << 16),
-                               static_cast<uint32_t>(yl[2]) | (static_cast<uint32_t>(yl[3]) << 16));
-                *reinterpret_cast<uint2*>(dst + 64 + 4 * g) =
-                    make_uint2(static_cast<uint32_t>(yh[0]) | (static_cast<uint32_t>(yh[1]) << 16),
-                               static_cast<uint32_t>(yh[2]) | (static_cast<uint32_t>(yh[3]) << 16));
+                float4 cs01, cs23;
+                rope_pairs(p, head, g, info.y, cs01, cs23);
+                emit_rope_group(p, head, g, info, sbias,
+                                *reinterpret_cast<const float4*>(part + row * kPartStride + 4 * g),
+                                *reinterpret_cast<const float4*>(part + row * kPartStride + 64 + 4 * g), cs01, cs23);
             }
         }
     }
@@ -398,6 +499,262 @@ __global__ void __launch_bounds__(qp::kThreads, S <= 3 ? 2 : 1) qkv_proj_kernel(
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// The narrow form (see qp::NarrowLayout): D^T[128 features][nt tokens] = W_tile . x_tile^T in
+// TMEM, one feature per TMEM lane.  Each epilogue thread sends its feature's values of rank r's
+// token rows to rank r (its own rows by plain stores); rank r sums the split partials in rank
+// order (rank 0's first, as the wide form adds), so the result does not depend on timing, and
+// emits its rows with the wide form's arithmetic.  Every rank sends all its rows unconditionally
+// (after bounded waits), so each owner's receive wait ends, and a CTA leaves only after the
+// bytes sent to it have landed.
+template <int NS, int XR>
+__global__ void __launch_bounds__(qp::kThreads, NS <= 4 ? 2 : 1) qkv_proj_narrow_kernel(const __grid_constant__ qp::Params p) {
+    using namespace qp;
+    using Lay = NarrowLayout<NS, XR>;
+    constexpr int kNStages = NS;
+    constexpr int kStage = Lay::kStage;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    // the next launch may start streaming its weights now (see qkv_proj_kernel)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int head = blockIdx.x;
+    const int nt = p.nt;
+    const int m0 = blockIdx.y * nt;
+    const int split = gridDim.z;
+    const int rank = blockIdx.z;
+    const int nk_all = p.K / kBK;
+    const int c_begin = rank * nk_all / split;
+    const int nk = (rank + 1) * nk_all / split - c_begin;
+    const int my_rows = nt / split;                    // token rows per rank (the host makes split divide nt)
+    const uint32_t stage_tx = static_cast<uint32_t>(kTileB + nt * 128);
+    const bool misaligned = (smem_u32(smem) & 1023u) != 0;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
+    uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + Lay::kOffTmemPtr);
+    int* failed_flag = reinterpret_cast<int*>(smem + Lay::kOffFlag);
+    float* recv = reinterpret_cast<float*>(smem + Lay::kOffRecv);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < Lay::kNumBars; ++i) mbar_init(&bars[i], 1);
+        *failed_flag = misaligned ? 1 : 0;
+        if (misaligned) report(p.status, ARK_DEV_TIMEOUT);
+        // the other ranks' rows of this rank's tile: one arrival now, the bytes as they land
+        mbar_arrive_expect_tx(&bars[Lay::kBarRecv], static_cast<uint32_t>((split - 1) * kBN * my_rows * 4));
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_ptr, kNarrowTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // every rank's receive barrier is initialised before any rank sends (the wait comes before the sends)
+    if (split > 1) cluster_arrive_relaxed();
+    const uint32_t tmem = *tmem_ptr;
+    const uint32_t sbase = smem_u32(smem);
+
+    if (warp == 0) {
+        // ================================================= TMA producer
+        if (lane == 0) {
+            int last = -1;
+            bool ok = true;
+            const int n_run = misaligned ? 0 : nk;
+            // every weight tile that has a stage goes before the wait: they do not depend on the
+            // previous kernel
+            const int pre = min(n_run, kNStages);
+            for (int c = 0; c < pre; ++c) {
+                mbar_arrive_expect_tx(&bars[Lay::kBarFull + c], stage_tx);
+                tma_load_2d(smem + c * kStage, &p.wmap, (c_begin + c) * kBK, head * kBN, &bars[Lay::kBarFull + c]);
+            }
+            asm volatile("griddepcontrol.wait;" ::: "memory");    // x may be the previous kernel's output
+            for (int c = 0; c < pre; ++c) {
+                tma_load_2d(smem + c * kStage + kTileB, &p.xmap, (c_begin + c) * kBK, m0, &bars[Lay::kBarFull + c]);
+                last = c;
+            }
+            for (int c = pre; c < n_run; ++c) {
+                const int st = c % kNStages;
+                if (!(ok = mbar_wait(&bars[Lay::kBarEmpty + st], ((c / kNStages) - 1) & 1))) break;
+                mbar_arrive_expect_tx(&bars[Lay::kBarFull + st], stage_tx);
+                const int kc = (c_begin + c) * kBK;
+                tma_load_2d(smem + st * kStage, &p.wmap, kc, head * kBN, &bars[Lay::kBarFull + st]);
+                tma_load_2d(smem + st * kStage + kTileB, &p.xmap, kc, m0, &bars[Lay::kBarFull + st]);
+                last = c;
+            }
+            if (!ok) {
+                atomicExch(failed_flag, 1);
+                report(p.status, ARK_DEV_TIMEOUT);
+            }
+            // the copies of the last stages have landed before the shared memory can go away
+            for (int c = last - kNStages + 1; c <= last; ++c)
+                if (c >= 0) (void)mbar_wait(&bars[Lay::kBarFull + c % kNStages], (c / kNStages) & 1);
+        }
+    } else if (warp == 1) {
+        // ================================================= MMA issuer
+        const uint32_t idesc = idesc_m128(static_cast<uint32_t>(nt));
+        bool ok = true;
+        if (nk <= kNStages) {
+            // the whole share is in the ring: wait for all of it, then issue every MMA back to back
+            for (int c = 0; c < (misaligned ? 0 : nk); ++c)
+                if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[Lay::kBarFull + c], 0)))) break;
+            if (ok && !misaligned && lane == 0) {
+                tc_fence_after();
+                for (int c = 0; c < nk; ++c) {
+                    const uint32_t a = sbase + c * kStage;       // W tile: A, 128 features x 64 K
+                    const uint32_t b = a + kTileB;                // x tile: B, nt tokens x 64 K
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem, umma_desc_sw128(a + kk * 32, 16, 1024), umma_desc_sw128(b + kk * 32, 16, 1024),
+                                 idesc, (c > 0 || kk > 0) ? 1u : 0u);
+                }
+            }
+            __syncwarp();
+        } else {
+            for (int c = 0; c < (misaligned ? 0 : nk); ++c) {
+                const int st = c % kNStages;
+                if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[Lay::kBarFull + st], (c / kNStages) & 1)))) break;
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint32_t a = sbase + st * kStage;
+                    const uint32_t b = a + kTileB;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem, umma_desc_sw128(a + kk * 32, 16, 1024), umma_desc_sw128(b + kk * 32, 16, 1024),
+                                 idesc, (c > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&bars[Lay::kBarEmpty + st]);
+                }
+                __syncwarp();
+            }
+        }
+        if (!ok) {
+            atomicExch(failed_flag, 1);
+            if (lane == 0) report(p.status, ARK_DEV_TIMEOUT);
+        }
+        __syncwarp();
+        if (lane == 0) umma_commit(&bars[Lay::kBarDone]);     // also when the loop gave up
+        __syncwarp();
+    }
+
+    // ================================================= epilogue
+    const int quad = warp & 3;
+    const int f = quad * 32 + lane;                        // this thread's feature (its TMEM lane)
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const int rows = min(nt, p.M - m0);
+    const int t0 = rank * my_rows;
+    int2* rowinfo = reinterpret_cast<int2*>(smem + Lay::kOffRows);
+    float* sbias = reinterpret_cast<float*>(smem + Lay::kOffBias);
+    if (warp >= 2) {
+        // nothing global is read before the previous kernel has completed (see qkv_proj_kernel)
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        {
+            const int et = threadIdx.x - 64;
+            sbias[et] = p.bias ? static_cast<float>(bf16_bits_to_f64(p.bias[head * kBN + et])) : 0.f;
+            if (et < my_rows)
+                rowinfo[et] = (p.fused && t0 + et < rows) ? row_destination(p, m0 + t0 + et, head)
+                                                          : make_int2(-1, 0);
+        }
+        // the rotary table entries of this thread's first item (token row t0 + et / 16, group
+        // et % 16), loaded while the MMAs run; any further items load theirs when they come
+        float4 pre01 = make_float4(0.f, 0.f, 0.f, 0.f), pre23 = pre01;
+        {
+            const int et = threadIdx.x - 64;
+            const int t = t0 + (et >> 4);
+            if (p.fused && et < my_rows * 16 && t < rows) {
+                const int m = m0 + t;
+                const int b = m / p.S;
+                rope_pairs(p, head, et & 15, __ldg(p.pos0 + b) + (m - b * p.S), pre01, pre23);
+            }
+        }
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[Lay::kBarDone], 0));
+        tc_fence_after();
+        if (!ok) {
+            atomicExch(failed_flag, 1);
+            if (lane == 0) report(p.status, ARK_DEV_TIMEOUT);
+        }
+        if (split > 1) cluster_wait();                     // every rank's receive barrier is set up
+        // send: token t of this feature goes to recv[rank][f][t % my_rows] of rank t / my_rows
+        const uint32_t my_slot = static_cast<uint32_t>((rank * kBN + f) * my_rows) * 4u;
+        const uint32_t recv_local = smem_u32(recv) + my_slot;
+        const uint32_t rbar_local = smem_u32(&bars[Lay::kBarRecv]);
+        for (int c16 = 0; c16 < nt / 16; ++c16) {
+            uint32_t a[16];
+            tmem_ld16(lane_base + c16 * 16, a);
+            tmem_wait_ld();
+            if ((my_rows & 3) == 0) {
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int t = c16 * 16 + 4 * q4;
+                    const int z = t / my_rows;
+                    const uint32_t off = static_cast<uint32_t>(t - z * my_rows) * 4u;
+                    const float v0 = __uint_as_float(a[4 * q4]), v1 = __uint_as_float(a[4 * q4 + 1]);
+                    const float v2 = __uint_as_float(a[4 * q4 + 2]), v3 = __uint_as_float(a[4 * q4 + 3]);
+                    if (z == rank)
+                        *reinterpret_cast<float4*>(smem + Lay::kOffRecv + my_slot + off) = make_float4(v0, v1, v2, v3);
+                    else
+                        st_async_v4(map_rank(recv_local + off, static_cast<uint32_t>(z)), v0, v1, v2, v3,
+                                    map_rank(rbar_local, static_cast<uint32_t>(z)));
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int t = c16 * 16 + i;
+                    const int z = t / my_rows;
+                    const uint32_t off = static_cast<uint32_t>(t - z * my_rows) * 4u;
+                    if (z == rank)
+                        *reinterpret_cast<float*>(smem + Lay::kOffRecv + my_slot + off) = __uint_as_float(a[i]);
+                    else
+                        st_async_f32(map_rank(recv_local + off, static_cast<uint32_t>(z)), __uint_as_float(a[i]),
+                                     map_rank(rbar_local, static_cast<uint32_t>(z)));
+                }
+            }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");     // this rank's own rows are in recv
+        bool got = true;
+        if (split > 1) got = __all_sync(0xffffffffu, mbar_wait_recv(&bars[Lay::kBarRecv], 0));
+        if (!got) {
+            atomicExch(failed_flag, 1);
+            if (lane == 0) report(p.status, ARK_DEV_TIMEOUT);
+        }
+        const bool failed = *reinterpret_cast<volatile int*>(failed_flag) != 0;
+        const int et = threadIdx.x - 64;
+        // items (token row of this rank, group g): fused, features 4g.. and 64+4g..; plain, 8g .. 8g+7
+        for (int it = et; it < my_rows * 16 && !failed; it += 128) {
+            const int tl = it >> 4, g = it & 15;
+            if (t0 + tl >= rows) continue;
+            if (p.fused && rowinfo[tl].x < 0) continue;    // padded or out-of-range row: not written
+            const int fa = p.fused ? 4 * g : 8 * g;
+            const int fb = p.fused ? 64 + 4 * g : 8 * g + 4;
+            float va[4], vb[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                va[i] = recv[(fa + i) * my_rows + tl];
+                vb[i] = recv[(fb + i) * my_rows + tl];
+            }
+            for (int z = 1; z < split; ++z) {
+                const float* rz = recv + z * kBN * my_rows;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    va[i] += rz[(fa + i) * my_rows + tl];
+                    vb[i] += rz[(fb + i) * my_rows + tl];
+                }
+            }
+            const float4 sa = make_float4(va[0], va[1], va[2], va[3]);
+            const float4 sb = make_float4(vb[0], vb[1], vb[2], vb[3]);
+            if (p.fused) {
+                const int2 info = rowinfo[tl];
+                if (it >= 128) rope_pairs(p, head, g, info.y, pre01, pre23);
+                emit_rope_group(p, head, g, info, sbias, sa, sb, pre01, pre23);
+            } else {
+                emit_plain8(p.out + static_cast<size_t>(m0 + t0 + tl) * p.N + head * kBN + 8 * g, sbias, 8 * g, sa, sb);
+            }
+        }
+    } else if (split > 1) {
+        cluster_wait();                                    // (pairs with the arrival above)
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kNarrowTmemCols);
     }
 }
 
@@ -434,20 +791,110 @@ ark_status launch_kernel(const qp::Params& prm, int M, int N, int split, cudaStr
     return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
 }
 
-ark_status launch_qkv(qp::Params& prm, const void* x, const void* w, int M, int K, int N, cudaStream_t stream) {
-    if (!kmajor_tensor_map(&prm.xmap, x, M, K, qp::kBM) || !kmajor_tensor_map(&prm.wmap, w, N, K, qp::kBN))
+// Clusters of `split` CTAs of `kernel` (with `smem` bytes) that can be resident at once, or -1.
+int max_clusters(const void* kernel, int smem, int split) {
+    cudaLaunchConfig_t occ = {};
+    occ.gridDim = dim3(1, 1, split);
+    occ.blockDim = dim3(qp::kThreads);
+    occ.dynamicSmemBytes = smem;
+    cudaLaunchAttribute ca[1];
+    ca[0].id = cudaLaunchAttributeClusterDimension;
+    ca[0].val.clusterDim.x = 1;
+    ca[0].val.clusterDim.y = 1;
+    ca[0].val.clusterDim.z = static_cast<unsigned>(split);
+    occ.attrs = ca;
+    occ.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &occ) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return -1;
+    }
+    return n > 0 ? n : -1;
+}
+
+// The narrow form for M <= 64 token rows: nt = M rounded up to 16; K split 8 ways (4-stage
+// ring, two CTAs per SM) when the hidden size allows it and the grid fits two CTAs per SM, else
+// over the largest cluster whose clusters are all resident at once; the split divides nt.
+template <int NS, int XR>
+ark_status launch_narrow_ns(const qp::Params& prm, int tiles, int split, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(tiles, 1, split);
+    cfg.blockDim = dim3(qp::kThreads);
+    cfg.dynamicSmemBytes = qp::NarrowLayout<NS, XR>::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = static_cast<unsigned>(split);
+    cfg.attrs = attr;
+    cfg.numAttrs = split > 1 ? 2 : 1;
+    if (cudaLaunchKernelEx(&cfg, qkv_proj_narrow_kernel<NS, XR>, prm) != cudaSuccess) return ARK_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? ARK_OK : ARK_ERR_CUDA;
+}
+
+template <int NS, int XR>
+cudaError_t narrow_smem_attr() {
+    return cudaFuncSetAttribute(qkv_proj_narrow_kernel<NS, XR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                qp::NarrowLayout<NS, XR>::kSmemBytes);
+}
+
+int g_qp_nclusters[64][4];   // clusters of 2, 4, 8 narrow CTAs (8-stage form) resident at once (0: unknown)
+int g_qp_n8[64];             // clusters of 8 of the 4-stage form resident at once (0: unknown)
+
+ark_status launch_narrow(qp::Params& prm, const void* x, const void* w, int M, int K, int N, int dev,
+                         cudaStream_t stream) {
+    const int nt = (M + 15) / 16 * 16;
+    if (!kmajor_tensor_map(&prm.xmap, x, M, K, nt) || !kmajor_tensor_map(&prm.wmap, w, N, K, qp::kBN))
         return ARK_ERR_CUDA;
     prm.M = M;
     prm.K = K;
     prm.N = N;
+    prm.nt = nt;
+    const int tiles = N / qp::kBN;
+    const int nk = K / qp::kBK;
+    const bool wide_x = nt > 32;
+    int split = 1;
+    if (nk % 8 == 0 && nk / 8 <= 4 && tiles * 8 <= 2 * g_qp_sms[dev]) {
+        if (g_qp_n8[dev] == 0)
+            g_qp_n8[dev] = wide_x ? max_clusters(reinterpret_cast<const void*>(qkv_proj_narrow_kernel<4, 64>),
+                                                 qp::NarrowLayout<4, 64>::kSmemBytes, 8)
+                                  : max_clusters(reinterpret_cast<const void*>(qkv_proj_narrow_kernel<4, 32>),
+                                                 qp::NarrowLayout<4, 32>::kSmemBytes, 8);
+        if (g_qp_n8[dev] > 0) split = 8;
+    }
+    if (split == 1) {
+        for (int cand = 2, ci = 0; cand <= 4; cand *= 2, ++ci) {
+            if (nk % cand != 0) break;
+            if (g_qp_nclusters[dev][ci] == 0)
+                g_qp_nclusters[dev][ci] =
+                    wide_x ? max_clusters(reinterpret_cast<const void*>(qkv_proj_narrow_kernel<6, 64>),
+                                          qp::NarrowLayout<6, 64>::kSmemBytes, cand)
+                           : max_clusters(reinterpret_cast<const void*>(qkv_proj_narrow_kernel<8, 32>),
+                                          qp::NarrowLayout<8, 32>::kSmemBytes, cand);
+            if (g_qp_nclusters[dev][ci] < tiles) break;
+            split = cand;
+        }
+    }
+    const bool small = nk / split <= 4;
+    if (wide_x)
+        return small ? launch_narrow_ns<4, 64>(prm, tiles, split, stream) : launch_narrow_ns<6, 64>(prm, tiles, split, stream);
+    return small ? launch_narrow_ns<4, 32>(prm, tiles, split, stream) : launch_narrow_ns<8, 32>(prm, tiles, split, stream);
+}
+
+ark_status launch_qkv(qp::Params& prm, const void* x, const void* w, int M, int K, int N, cudaStream_t stream) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARK_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_qp_mu);     // held through the split choice (it fills g_qp_clusters)
+    std::lock_guard<std::mutex> lk(g_qp_mu);     // held through the split choice (it fills the cluster tables)
     if (!g_qp_attr[dev]) {
         if (cudaFuncSetAttribute(qkv_proj_kernel<qp::kStagesWide>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  qp::Layout<qp::kStagesWide>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(qkv_proj_kernel<qp::kStagesSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 qp::Layout<qp::kStagesSplit>::kSmemBytes) != cudaSuccess)
+                                 qp::Layout<qp::kStagesSplit>::kSmemBytes) != cudaSuccess ||
+            narrow_smem_attr<4, 32>() != cudaSuccess || narrow_smem_attr<8, 32>() != cudaSuccess ||
+            narrow_smem_attr<4, 64>() != cudaSuccess || narrow_smem_attr<6, 64>() != cudaSuccess)
             return ARK_ERR_CUDA;
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
@@ -455,6 +902,12 @@ ark_status launch_qkv(qp::Params& prm, const void* x, const void* w, int M, int 
         g_qp_sms[dev] = sms;
         g_qp_attr[dev] = true;
     }
+    if (M <= qp::kNarrowMaxM) return launch_narrow(prm, x, w, M, K, N, dev, stream);
+    if (!kmajor_tensor_map(&prm.xmap, x, M, K, qp::kBM) || !kmajor_tensor_map(&prm.wmap, w, N, K, qp::kBN))
+        return ARK_ERR_CUDA;
+    prm.M = M;
+    prm.K = K;
+    prm.N = N;
     const int tiles = (N / qp::kBN) * ((M + qp::kBM - 1) / qp::kBM);
     // split K over a cluster of six-stage CTAs (one per SM) while the split CTAs fit on the SMs, every
     // cluster of the launch can be resident at once (one wave) and the chunks divide evenly
@@ -462,25 +915,9 @@ ark_status launch_qkv(qp::Params& prm, const void* x, const void* w, int M, int 
     const int nk = K / qp::kBK;
     for (int cand = 2, ci = 0; cand <= qp::kMaxSplit; cand *= 2, ++ci) {
         if (nk % cand != 0 || static_cast<long long>(tiles) * cand > g_qp_sms[dev]) break;
-        if (g_qp_clusters[dev][ci] == 0) {
-            cudaLaunchConfig_t occ = {};
-            occ.gridDim = dim3(1, 1, cand);
-            occ.blockDim = dim3(qp::kThreads);
-            occ.dynamicSmemBytes = qp::Layout<qp::kStagesSplit>::kSmemBytes;
-            cudaLaunchAttribute ca[1];
-            ca[0].id = cudaLaunchAttributeClusterDimension;
-            ca[0].val.clusterDim.x = 1;
-            ca[0].val.clusterDim.y = 1;
-            ca[0].val.clusterDim.z = static_cast<unsigned>(cand);
-            occ.attrs = ca;
-            occ.numAttrs = 1;
-            int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, qkv_proj_kernel<qp::kStagesSplit>, &occ) != cudaSuccess) {
-                (void)cudaGetLastError();
-                n = -1;
-            }
-            g_qp_clusters[dev][ci] = n > 0 ? n : -1;
-        }
+        if (g_qp_clusters[dev][ci] == 0)
+            g_qp_clusters[dev][ci] = max_clusters(reinterpret_cast<const void*>(qkv_proj_kernel<qp::kStagesSplit>),
+                                                  qp::Layout<qp::kStagesSplit>::kSmemBytes, cand);
         if (g_qp_clusters[dev][ci] < tiles) break;
         split = cand;
     }

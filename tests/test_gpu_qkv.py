@@ -63,9 +63,10 @@ def check_close_bf16(got_bits, ref_bits, err_bound, what):
     assert exact > 0.98, f"{what}: only {exact:.4f} bit-identical"
 
 
-@pytest.mark.parametrize("M,bias", [(200, True), (128, False), (37, True)])
+@pytest.mark.parametrize("M,bias", [(200, True), (128, False), (37, True), (64, False), (1, True)])
 def test_qkv_proj_against_oracle(oracle_lib, M, bias):
-    """Ragged M (several 128-row tiles and a tail), K = 2048, N = 2560."""
+    """Ragged M (several 128-row tiles and a tail; and up to 64 rows, the
+    narrow form with the token rows on the MMA's N), K = 2048, N = 2560."""
     w, b = W.make_qkv_weights(11 + M, bias=bias)
     x = W.make_hidden(12 + M, 1, M)[0]
     out = torch.full((M, w.shape[0]), 0, dtype=torch.bfloat16, device="cuda")
@@ -172,10 +173,15 @@ def test_qkv_rope_append_against_oracle(oracle_lib, B, S, T, pos0, n_new):
         assert np.all(qb[i, int(nn[i]):] == U16_NAN)
 
 
-def test_qkv_fused_equals_projection_then_append(oracle_lib):
+@pytest.mark.parametrize("B,S,pos0,n_new", [
+    (4, 70, [0, 100, 441, 7], [70, 33, 70, 1]),   # 128-row tiles
+    (32, 1, list(range(3, 480, 15)), [1] * 32),   # a decode step: the narrow form
+    (5, 3, [0, 9, 500, 77, 1], [3, 1, 2, 0, 3]),  # 15 token rows, padded ones among them
+])
+def test_qkv_fused_equals_projection_then_append(oracle_lib, B, S, pos0, n_new):
     """Bit for bit: the fused epilogue == ark_attn_qkv_proj + ark_attn_append_rope."""
-    B, S, T = 4, 70, 512
-    x, w, b, p0, nn, ck0, cv0 = make_case(77, B, S, T, [0, 100, 441, 7], [70, 33, 70, 1])
+    T = 512
+    x, w, b, p0, nn, ck0, cv0 = make_case(77 + B, B, S, T, pos0, n_new)
     q, ck, cv, st = run_fused(x, w, b, p0, nn, T, ck0, cv0)
     assert st == 0
     dev = "cuda"
