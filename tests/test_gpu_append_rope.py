@@ -105,3 +105,62 @@ def test_append_rope_bad_n_new_sets_status(oracle_lib):
     q_ref, ck_ref, cv_ref, _ = run_oracle_append(fixed)
     assert_bits_equal(q, q_ref, "q")
     assert_bits_equal(ck, ck_ref, "cache_k")
+
+
+def _bf16_from_bits(u16: np.ndarray) -> np.ndarray:
+    return (u16.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _midpoint_distance(v: np.ndarray) -> np.ndarray:
+    """|v - nearest bf16 rounding midpoint| / |v| (v float64, nonzero)."""
+    _, e = np.frexp(v)
+    spacing = np.ldexp(1.0, e - 8)                   # bf16 keeps 8 significant bits
+    frac = np.abs(v) / spacing
+    return np.abs(frac - np.floor(frac) - 0.5) * spacing / np.abs(v)
+
+
+def _near_midpoint_rows(table: np.ndarray, S: int, heads: int, n_cand: int, rng) -> np.ndarray:
+    """bf16 rows [S, heads, 128] whose rotations x_i c - x_{i+64} s at position t
+    (= the row index) land as close to a bf16 rounding midpoint as n_cand random
+    candidate pairs allow."""
+    out = np.zeros((S, heads, 128), np.uint16)
+    for t in range(S):
+        c, s = table[t, :, 0][:, None], table[t, :, 1][:, None]
+        for h in range(heads):
+            sign = rng.integers(0, 2, (64, n_cand, 2), dtype=np.uint16) << 15
+            expo = rng.integers(120, 134, (64, n_cand, 2), dtype=np.uint16) << 7
+            mant = rng.integers(0, 128, (64, n_cand, 2), dtype=np.uint16)
+            cand = sign | expo | mant
+            a, z = _bf16_from_bits(cand[..., 0]), _bf16_from_bits(cand[..., 1])
+            v = a * c - z * s                          # products exact in double, one rounding
+            d = np.where(v != 0, _midpoint_distance(np.where(v != 0, v, 1.0)), 1.0)
+            pick = np.argmin(d, axis=1)
+            out[t, h, :64] = cand[np.arange(64), pick, 0]
+            out[t, h, 64:] = cand[np.arange(64), pick, 1]
+    return out
+
+
+def test_rotation_near_bf16_midpoints(oracle_lib):
+    """Rotations whose double result lies within a few fp32 ulps of a bf16
+    rounding midpoint (where any shortcut through fp32 would round the wrong
+    way) and ones just outside that zone: q and k rows bit-exact against the
+    oracle's double-precision rotation."""
+    B, S, T = 1, 24, 64
+    rng = np.random.default_rng(20261203)
+    table = ops.rope_table(T).cpu().numpy().astype(np.float64)     # [T, 64, 2] {cos, sin}
+    batch = W.make_batch(77, B=B, S=S, T=T, pos0=[0], n_new=[S])
+    q_rows = _near_midpoint_rows(table, S, 16, 4096, rng)
+    k_rows = _near_midpoint_rows(table, S, 2, 4096, rng)
+    batch.q[0] = torch.from_numpy(q_rows.view(np.int16)).view(torch.bfloat16).view(B, S, 16, 128).clone()
+    batch.k_new[0] = torch.from_numpy(k_rows.view(np.int16)).view(torch.bfloat16).view(B, S, 2, 128).clone()
+    # how close the first outputs came: some within 2^-22 of a midpoint, most just outside
+    a, z = _bf16_from_bits(q_rows[..., :64]), _bf16_from_bits(q_rows[..., 64:])
+    v = a * table[:S, None, :, 0] - z * table[:S, None, :, 1]
+    d = _midpoint_distance(v[v != 0])
+    assert (d < 2.0 ** -22).sum() > 20 and (d > 2.0 ** -19).sum() > 1000
+    q, ck, cv, st = run_gpu_append(batch)
+    assert st == 0
+    q_ref, ck_ref, cv_ref, skipped = run_oracle_append(batch)
+    assert skipped == 0
+    assert np.array_equal(bits(q), q_ref), f"q differs at {np.argwhere(bits(q) != q_ref)[:5]}"
+    assert np.array_equal(bits(ck), ck_ref) and np.array_equal(bits(cv), cv_ref)
