@@ -56,10 +56,15 @@ DECODE_CONFIGS = ("ragged", "single", "long2048", "long1024")
 # sha256 of the kernel source it was taken on; reported as null once the source
 # has changed.
 DECODE_TRAFFIC = {
-    # ncu, one call of the ragged decode workload: decode_kernel (--set full) plus
-    # merge_kernel (dram bytes), read + write (see profiles/)
-    "897eda01dc002b0828394c98dd54fc30527c34eb69bb38b58a6fed55f875d66d":
-        329.750784e6 + 4.175616e6 + 13.199104e6 + 0,
+    # ncu dram bytes, one call of the ragged decode workload: decode_kernel plus
+    # merge_kernel, read + write (see profiles/)
+    "09c8f33c6fa5b1855d6c89b8aca0676a6d501d7e5059e7b4c2d4dd0dfb6ba281":
+        329.766656e6 + 3.29088e6 + 13.198336e6 + 0,
+}
+# The same for the fp8 cache (the ragged workload with --kv fp8).
+DECODE_TRAFFIC_FP8 = {
+    "09c8f33c6fa5b1855d6c89b8aca0676a6d501d7e5059e7b4c2d4dd0dfb6ba281":
+        167.267072e6 + 3.617536e6 + 13.19808e6 + 0,
 }
 
 
@@ -76,10 +81,10 @@ PREFILL_TRAFFIC = {
 # Per-launch DRAM traffic of the projection kernel (one layer) from ncu --set full
 # captures of the two projection workloads, keyed by source hash and workload.
 QKV_TRAFFIC = {
-    # the 3-stage instantiation (many tiles) for the prompt rows; the 6-stage split-K one for a
-    # decode step
-    ("cde2e14ac2c31091a231005ee3800a1c5b6ed3f7342cfb4061ca0ee650e6b0ef", "qkv_prefill"): 36.077568e6 + 0.54272e6,
-    ("cde2e14ac2c31091a231005ee3800a1c5b6ed3f7342cfb4061ca0ee650e6b0ef", "qkv_decode"): 10.670336e6 + 0,
+    # the 3-stage instantiation (many tiles) for the prompt rows (dram bytes); the narrow form
+    # (token rows on the MMA's N, K split 8 ways) for a decode step (--set full)
+    ("0a08bed75d20bc0d45e4704b032ede1509714699f2ec5b8cb1205bd094be9717", "qkv_prefill"): 36.07808e6 + 0.306176e6,
+    ("0a08bed75d20bc0d45e4704b032ede1509714699f2ec5b8cb1205bd094be9717", "qkv_decode"): 10.684672e6 + 0,
 }
 
 
@@ -1035,8 +1040,8 @@ def run_decode(args):
     achieved = bytes_launch / (per_launch_ms * 1e-3) / 1e9
     h = src_hash("gqa_attention_static_b200/csrc/decode.cu")
     # the capture is of the default workload's batched launch
-    traffic = (DECODE_TRAFFIC.get(h) if (not args.per_layer and args.config == "ragged" and args.mode == "aware"
-                                         and not fp8) else None)
+    traffic = ((DECODE_TRAFFIC_FP8 if fp8 else DECODE_TRAFFIC).get(h)
+               if (not args.per_layer and args.config == "ragged" and args.mode == "aware") else None)
     roof = {"kernel": "decode_kernel + merge_kernel (one ark_attn_decode%s call)" % ("" if args.per_layer else
                                                                                      "_layers")}
     roof.update(hbm_roofline(achieved))
@@ -1326,7 +1331,8 @@ def run_qkv(args):
     t_flops = nflops / (tc * 1e12)
     bound = "hbm" if t_bytes >= t_flops else "tensor"
     achieved = (nbytes / 1e9 if bound == "hbm" else nflops / 1e12) / (ms_launch * 1e-3)
-    roof = {"kernel": "qkv_proj_kernel (ark_attn_qkv_rope_append, one layer per launch)", "bound": bound,
+    kname = "qkv_proj_narrow_kernel" if args.config == "qkv_decode" else "qkv_proj_kernel"
+    roof = {"kernel": kname + " (ark_attn_qkv_rope_append, one layer per launch)", "bound": bound,
             "achieved": achieved, "peak": hbm if bound == "hbm" else tc, "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
             "frac": (t_bytes if bound == "hbm" else t_flops) / (ms_launch * 1e-3),
             "peak_kind": hbm_kind if bound == "hbm" else tc_kind,
