@@ -841,8 +841,10 @@ cudaError_t narrow_smem_attr() {
                                 qp::NarrowLayout<NS, XR>::kSmemBytes);
 }
 
-int g_qp_nclusters[64][4];   // clusters of 2, 4, 8 narrow CTAs (8-stage form) resident at once (0: unknown)
-int g_qp_n8[64];             // clusters of 8 of the 4-stage form resident at once (0: unknown)
+// clusters of the narrow form resident at once (0: unknown), per device and x tile size (32 or
+// 64 rows): of 2 and 4 CTAs of the deep-ring form, and of 8 CTAs of the 4-stage form
+int g_qp_nclusters[64][2][4];
+int g_qp_n8[64][2];
 
 ark_status launch_narrow(qp::Params& prm, const void* x, const void* w, int M, int K, int N, int dev,
                          cudaStream_t stream) {
@@ -858,23 +860,24 @@ ark_status launch_narrow(qp::Params& prm, const void* x, const void* w, int M, i
     const bool wide_x = nt > 32;
     int split = 1;
     if (nk % 8 == 0 && nk / 8 <= 4 && tiles * 8 <= 2 * g_qp_sms[dev]) {
-        if (g_qp_n8[dev] == 0)
-            g_qp_n8[dev] = wide_x ? max_clusters(reinterpret_cast<const void*>(qkv_proj_narrow_kernel<4, 64>),
-                                                 qp::NarrowLayout<4, 64>::kSmemBytes, 8)
-                                  : max_clusters(reinterpret_cast<const void*>(qkv_proj_narrow_kernel<4, 32>),
-                                                 qp::NarrowLayout<4, 32>::kSmemBytes, 8);
-        if (g_qp_n8[dev] > 0) split = 8;
+        int& n8 = g_qp_n8[dev][wide_x ? 1 : 0];
+        if (n8 == 0)
+            n8 = wide_x ? max_clusters(reinterpret_cast<const void*>(qkv_proj_narrow_kernel<4, 64>),
+                                       qp::NarrowLayout<4, 64>::kSmemBytes, 8)
+                        : max_clusters(reinterpret_cast<const void*>(qkv_proj_narrow_kernel<4, 32>),
+                                       qp::NarrowLayout<4, 32>::kSmemBytes, 8);
+        if (n8 > 0) split = 8;
     }
     if (split == 1) {
         for (int cand = 2, ci = 0; cand <= 4; cand *= 2, ++ci) {
             if (nk % cand != 0) break;
-            if (g_qp_nclusters[dev][ci] == 0)
-                g_qp_nclusters[dev][ci] =
-                    wide_x ? max_clusters(reinterpret_cast<const void*>(qkv_proj_narrow_kernel<6, 64>),
-                                          qp::NarrowLayout<6, 64>::kSmemBytes, cand)
-                           : max_clusters(reinterpret_cast<const void*>(qkv_proj_narrow_kernel<8, 32>),
-                                          qp::NarrowLayout<8, 32>::kSmemBytes, cand);
-            if (g_qp_nclusters[dev][ci] < tiles) break;
+            int& nc = g_qp_nclusters[dev][wide_x ? 1 : 0][ci];
+            if (nc == 0)
+                nc = wide_x ? max_clusters(reinterpret_cast<const void*>(qkv_proj_narrow_kernel<6, 64>),
+                                           qp::NarrowLayout<6, 64>::kSmemBytes, cand)
+                            : max_clusters(reinterpret_cast<const void*>(qkv_proj_narrow_kernel<8, 32>),
+                                           qp::NarrowLayout<8, 32>::kSmemBytes, cand);
+            if (nc < tiles) break;
             split = cand;
         }
     }

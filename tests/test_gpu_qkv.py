@@ -78,6 +78,21 @@ def test_qkv_proj_against_oracle(oracle_lib, M, bias):
     check_close_bf16(bits(out), ref, bound, "projection")
 
 
+@pytest.mark.parametrize("M,K", [(32, 4096), (48, 1024), (20, 512)])
+def test_qkv_proj_narrow_other_hidden_sizes(oracle_lib, M, K):
+    """The narrow form (up to 64 token rows) at other hidden sizes: K = 4096
+    gives each cluster rank more K chunks than its ring has stages (the ring is
+    reused), K = 1024 and 512 the 4-stage form with one and two chunks a rank."""
+    w, b = W.make_qkv_weights(500 + K, K=K)
+    x = W.make_hidden(501 + K, 1, M, K=K)[0]
+    out = torch.full((M, w.shape[0]), 0, dtype=torch.bfloat16, device="cuda")
+    ops.ark_attn_qkv_proj(x.cuda(), w.cuda(), b.cuda(), out)
+    torch.cuda.synchronize()
+    ref = oracle.qkv_proj(bits(x), bits(w), bits(b))
+    bound = K * 2.0 ** -24 * abs_dot(bits(x), bits(w), bits(b))
+    check_close_bf16(bits(out), ref, bound, f"projection M={M} K={K}")
+
+
 def run_fused(x, w, b, pos0, n_new, T, ck0, cv0):
     dev = "cuda"
     B, S, _ = x.shape
