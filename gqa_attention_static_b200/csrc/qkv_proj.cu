@@ -103,6 +103,7 @@ struct NarrowLayout {
     static constexpr int kSmemBytes = kOffFlag + 8;
     static_assert(kStage % 1024 == 0 && kTileB % 1024 == 0, "128-byte swizzled tiles start on 1 KB");
     static_assert(XR <= kNarrowMaxM && XR % 16 == 0, "x tile rows");
+    static_assert(XR * kBN * 4 <= NS * kStage, "the summed rows fit over the stage buffers");
 };
 constexpr uint32_t kNarrowTmemCols = 64;
 // kind::f16, bf16 x bf16 -> fp32, M = 128, N = n, A and B K-major
@@ -714,30 +715,46 @@ __global__ void __launch_bounds__(qp::kThreads, NS <= 4 ? 2 : 1) qkv_proj_narrow
             if (lane == 0) report(p.status, ARK_DEV_TIMEOUT);
         }
         const bool failed = *reinterpret_cast<volatile int*>(failed_flag) != 0;
+        // the split's partials of this thread's feature, summed for each of this rank's token rows
+        // in rank order (rank 0's first), into sums[row][feature] over the stage buffers (free now
+        // that every MMA has completed): 16-byte loads of 4 rows at a time, consecutive features
+        // in consecutive threads, so the loads and stores are free of bank conflicts
+        float* sums = reinterpret_cast<float*>(smem);
+        if ((my_rows & 3) == 0) {
+            for (int t4 = 0; t4 < my_rows; t4 += 4) {
+                float4 acc = *reinterpret_cast<const float4*>(recv + f * my_rows + t4);
+#pragma unroll
+                for (int z = 1; z < kMaxSplit; ++z) {
+                    if (z >= split) break;
+                    const float4 v = *reinterpret_cast<const float4*>(recv + (z * kBN + f) * my_rows + t4);
+                    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+                }
+                sums[(t4 + 0) * kBN + f] = acc.x;
+                sums[(t4 + 1) * kBN + f] = acc.y;
+                sums[(t4 + 2) * kBN + f] = acc.z;
+                sums[(t4 + 3) * kBN + f] = acc.w;
+            }
+        } else {
+            for (int tl = 0; tl < my_rows; ++tl) {
+                float acc = recv[f * my_rows + tl];
+#pragma unroll
+                for (int z = 1; z < kMaxSplit; ++z) {
+                    if (z >= split) break;
+                    acc += recv[(z * kBN + f) * my_rows + tl];
+                }
+                sums[tl * kBN + f] = acc;
+            }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");     // every row's sums are in place
         const int et = threadIdx.x - 64;
         // items (token row of this rank, group g): fused, features 4g.. and 64+4g..; plain, 8g .. 8g+7
         for (int it = et; it < my_rows * 16 && !failed; it += 128) {
             const int tl = it >> 4, g = it & 15;
             if (t0 + tl >= rows) continue;
             if (p.fused && rowinfo[tl].x < 0) continue;    // padded or out-of-range row: not written
-            const int fa = p.fused ? 4 * g : 8 * g;
-            const int fb = p.fused ? 64 + 4 * g : 8 * g + 4;
-            float va[4], vb[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                va[i] = recv[(fa + i) * my_rows + tl];
-                vb[i] = recv[(fb + i) * my_rows + tl];
-            }
-            for (int z = 1; z < split; ++z) {
-                const float* rz = recv + z * kBN * my_rows;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    va[i] += rz[(fa + i) * my_rows + tl];
-                    vb[i] += rz[(fb + i) * my_rows + tl];
-                }
-            }
-            const float4 sa = make_float4(va[0], va[1], va[2], va[3]);
-            const float4 sb = make_float4(vb[0], vb[1], vb[2], vb[3]);
+            const float* row = sums + tl * kBN;
+            const float4 sa = *reinterpret_cast<const float4*>(row + (p.fused ? 4 * g : 8 * g));
+            const float4 sb = *reinterpret_cast<const float4*>(row + (p.fused ? 64 + 4 * g : 8 * g + 4));
             if (p.fused) {
                 const int2 info = rowinfo[tl];
                 if (it >= 128) rope_pairs(p, head, g, info.y, pre01, pre23);
