@@ -82,11 +82,9 @@ PREFILL_TRAFFIC = {
 # captures of the two projection workloads, keyed by source hash and workload.
 QKV_TRAFFIC = {
     # the 3-stage instantiation (many tiles) for the prompt rows (dram bytes); the narrow form
-    # (token rows on the MMA's N, K split 8 ways) for a decode step (--set full); taken on the
-    # previous revision of the file, whose kernels are the same (only the host's occupancy cache
-    # changed since)
-    ("93e12ea1a3a2f8e396acdafb714c0c30ae41f6fcab554a095b69ebb6a3f9b06f", "qkv_prefill"): 36.07808e6 + 0.306176e6,
-    ("93e12ea1a3a2f8e396acdafb714c0c30ae41f6fcab554a095b69ebb6a3f9b06f", "qkv_decode"): 10.684672e6 + 0,
+    # (token rows on the MMA's N, K split 8 ways) for a decode step (--set full)
+    ("3c83e644a40657a6c7d50d11877dee6a84784bcc25e01e87b1ee6c3839d20621", "qkv_prefill"): 36.077824e6 + 0.34176e6,
+    ("3c83e644a40657a6c7d50d11877dee6a84784bcc25e01e87b1ee6c3839d20621", "qkv_decode"): 10.684672e6 + 0,
 }
 
 
