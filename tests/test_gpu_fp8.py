@@ -148,3 +148,44 @@ def test_decode_fp8_step_ragged_batch(oracle_lib):
                                            kv.numpy(), SCALE)
         check_o(f64(step.o[l]), o_ref, f"o layer {l}")
         check_lse(f64(step.lse[l]), lse_ref, f"lse layer {l}")
+
+
+@pytest.mark.parametrize("mode", [ops.ARK_LENGTH_AWARE, ops.ARK_MASKED_STATIC])
+def test_decode_fp8_one_kv_head_and_T_not_a_multiple_of_16(oracle_lib, mode):
+    """The head-major fp8 cache with a single KV head (8 query heads) and
+    T = 100: the last 16-position tile reaches past T, where the copy reads
+    zeros; lengths 1, 57 and T."""
+    B, T = 3, 100
+    kv = torch.tensor([1, 57, 100], dtype=torch.int32)
+    g = torch.Generator().manual_seed(340)
+    q = W.randn_bf16((B, 1, 8, 128), g)
+    fc = W.make_fp8_cache(341, B, T, kv, Hkv=1, garbage="big" if mode == ops.ARK_MASKED_STATIC else "nan")
+    o, lse = gpu_decode_fp8(q, fc, kv, mode)
+    o_ref, lse_ref = oracle.decode_fp8(bits(q), u8(fc.cache_k[0]), u8(fc.cache_v[0]), fc.k_scale[0].numpy(),
+                                       fc.v_scale[0].numpy(), kv.numpy(), SCALE,
+                                       static_mode=(mode == ops.ARK_MASKED_STATIC))
+    check_o(f64(o), o_ref, "o")
+    check_lse(f64(lse), lse_ref, "lse")
+
+
+def test_append_fp8_one_kv_head_bit_exact(oracle_lib):
+    """The append into a head-major fp8 cache with one KV head, T = 100,
+    rows landing in the last (partial) 16-position tile."""
+    B, S, T = 2, 3, 100
+    batch = W.make_batch(342, B=B, S=S, T=T, pos0=[0, 97], n_new=[3, 3], hq=8, hkv=1)
+    fc = W.make_fp8_cache(343, B, T, batch.pos0, garbage="none", Hkv=1)
+    dev = "cuda"
+    q = batch.q[0].to(dev).clone()
+    ck, cv = fc.cache_k[0].to(dev).clone(), fc.cache_v[0].to(dev).clone()
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ops.ark_attn_append_rope_fp8(q, batch.k_new[0].to(dev), batch.v_new[0].to(dev), ck, cv, fc.k_scale[0].to(dev),
+                                 fc.v_scale[0].to(dev), batch.pos0.to(dev), batch.n_new.to(dev), ops.rope_table(T),
+                                 status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    q_ref, ck_ref, cv_ref, skipped = oracle.append_rope_fp8(
+        bits(batch.q[0]), bits(batch.k_new[0]), bits(batch.v_new[0]), u8(fc.cache_k[0]), u8(fc.cache_v[0]),
+        fc.k_scale[0].numpy(), fc.v_scale[0].numpy(), batch.pos0.numpy(), batch.n_new.numpy())
+    assert skipped == 0
+    assert np.array_equal(bits(q), q_ref)
+    assert np.array_equal(u8(ck), ck_ref) and np.array_equal(u8(cv), cv_ref)
