@@ -560,11 +560,14 @@ __global__ void __launch_bounds__(qp::kThreads, NS <= 4 ? 2 : 1) qkv_proj_narrow
             bool ok = true;
             const int n_run = misaligned ? 0 : nk;
             // every weight tile that has a stage goes before the wait: they do not depend on the
-            // previous kernel
+            // previous kernel.  Each weight byte is read once per step: evict-first in L2, so that
+            // the step's small operands (x, the rows the epilogue writes) stay there
+            const uint64_t pol_w = l2_policy_evict_first();
             const int pre = min(n_run, kNStages);
             for (int c = 0; c < pre; ++c) {
                 mbar_arrive_expect_tx(&bars[Lay::kBarFull + c], stage_tx);
-                tma_load_2d(smem + c * kStage, &p.wmap, (c_begin + c) * kBK, head * kBN, &bars[Lay::kBarFull + c]);
+                tma_load_2d_hint(smem + c * kStage, &p.wmap, (c_begin + c) * kBK, head * kBN, &bars[Lay::kBarFull + c],
+                                 pol_w);
             }
             asm volatile("griddepcontrol.wait;" ::: "memory");    // x may be the previous kernel's output
             for (int c = 0; c < pre; ++c) {
@@ -576,7 +579,7 @@ __global__ void __launch_bounds__(qp::kThreads, NS <= 4 ? 2 : 1) qkv_proj_narrow
                 if (!(ok = mbar_wait(&bars[Lay::kBarEmpty + st], ((c / kNStages) - 1) & 1))) break;
                 mbar_arrive_expect_tx(&bars[Lay::kBarFull + st], stage_tx);
                 const int kc = (c_begin + c) * kBK;
-                tma_load_2d(smem + st * kStage, &p.wmap, kc, head * kBN, &bars[Lay::kBarFull + st]);
+                tma_load_2d_hint(smem + st * kStage, &p.wmap, kc, head * kBN, &bars[Lay::kBarFull + st], pol_w);
                 tma_load_2d(smem + st * kStage + kTileB, &p.xmap, kc, m0, &bars[Lay::kBarFull + st]);
                 last = c;
             }
