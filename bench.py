@@ -83,8 +83,8 @@ PREFILL_TRAFFIC = {
 QKV_TRAFFIC = {
     # the 3-stage instantiation (many tiles) for the prompt rows (dram bytes); the narrow form
     # (token rows on the MMA's N, K split 8 ways) for a decode step (--set full)
-    ("3c83e644a40657a6c7d50d11877dee6a84784bcc25e01e87b1ee6c3839d20621", "qkv_prefill"): 36.077824e6 + 0.34176e6,
-    ("3c83e644a40657a6c7d50d11877dee6a84784bcc25e01e87b1ee6c3839d20621", "qkv_decode"): 10.684672e6 + 0,
+    ("dbafa3a02e382f7a7a073b2e97a78056853bc297e8293e2f1726c646a5e573b9", "qkv_prefill"): 36.077824e6 + 0.27904e6,
+    ("dbafa3a02e382f7a7a073b2e97a78056853bc297e8293e2f1726c646a5e573b9", "qkv_decode"): 10.684928e6 + 0,
 }
 
 
